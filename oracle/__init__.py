@@ -1,0 +1,118 @@
+"""ctypes front of the fp64 CPU oracle (``oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` may import this module; the library package never does.
+
+``Oracle(path)`` wraps one build of the oracle (the tests also build deliberately
+broken copies of ``oracle.c`` and load them through the same class).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(HERE, "oracle.c")
+LIBRARY = os.path.join(HERE, "liboracle.so")
+
+
+def build(source: str = SOURCE, output: str = LIBRARY, force: bool = False) -> str:
+    """Compile ``source`` with gcc (fp64, OpenMP, no fast-math) into ``output``."""
+    if (not force and os.path.exists(output)
+            and os.path.getmtime(output) >= os.path.getmtime(source)):
+        return output
+    tmp = output + ".tmp%d" % os.getpid()
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+           "-o", tmp, source, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, output)
+    return output
+
+
+_dptr = ctypes.POINTER(ctypes.c_double)
+
+
+def _as_ptr(a: np.ndarray):
+    return a.ctypes.data_as(_dptr)
+
+
+class Oracle:
+    """fp64 reference for attention forward (O, LSE) and backward (dQ, dK, dV)."""
+
+    def __init__(self, path: str | None = None):
+        if path is None:
+            path = build()
+        self.lib = ctypes.CDLL(path)
+        L = ctypes.c_long
+        self.lib.oracle_attention_fwd.argtypes = [
+            _dptr, _dptr, _dptr, L, L, L, L, ctypes.c_double, ctypes.c_int, L, L, _dptr, _dptr]
+        self.lib.oracle_attention_fwd.restype = ctypes.c_int
+        self.lib.oracle_attention_bwd.argtypes = [
+            _dptr, _dptr, _dptr, _dptr, L, L, L, L, ctypes.c_double, ctypes.c_int, L, L,
+            _dptr, _dptr, _dptr]
+        self.lib.oracle_attention_bwd.restype = ctypes.c_int
+        self.lib.oracle_num_threads.restype = ctypes.c_int
+
+    @staticmethod
+    def _prep(*arrays):
+        out = []
+        shape = arrays[0].shape
+        for a in arrays:
+            a = np.ascontiguousarray(a, dtype=np.float64)
+            if a.shape != shape or a.ndim != 4:
+                raise ValueError("oracle inputs must share one (B, H, N, d) shape")
+            out.append(a)
+        return out
+
+    def fwd(self, q, k, v, scale, causal=False, window=(-1, -1)):
+        """Returns (O, LSE) in fp64 for (B, H, N, d) inputs."""
+        q, k, v = self._prep(q, k, v)
+        B, H, N, d = q.shape
+        o = np.empty_like(q)
+        lse = np.empty((B, H, N), dtype=np.float64)
+        rc = self.lib.oracle_attention_fwd(_as_ptr(q), _as_ptr(k), _as_ptr(v), B, H, N, d,
+                                           float(scale), int(bool(causal)), int(window[0]),
+                                           int(window[1]), _as_ptr(o), _as_ptr(lse))
+        if rc != 0:
+            raise RuntimeError("oracle_attention_fwd failed with %d" % rc)
+        return o, lse
+
+    def bwd(self, q, k, v, do, scale, causal=False, window=(-1, -1)):
+        """Returns (dQ, dK, dV) in fp64: the gradient of <O, dO> for (B, H, N, d) inputs."""
+        q, k, v, do = self._prep(q, k, v, do)
+        B, H, N, d = q.shape
+        dq = np.empty_like(q)
+        dk = np.empty_like(q)
+        dv = np.empty_like(q)
+        rc = self.lib.oracle_attention_bwd(_as_ptr(q), _as_ptr(k), _as_ptr(v), _as_ptr(do),
+                                           B, H, N, d, float(scale), int(bool(causal)),
+                                           int(window[0]), int(window[1]),
+                                           _as_ptr(dq), _as_ptr(dk), _as_ptr(dv))
+        if rc != 0:
+            raise RuntimeError("oracle_attention_bwd failed with %d" % rc)
+        return dq, dk, dv
+
+    def num_threads(self) -> int:
+        return int(self.lib.oracle_num_threads())
+
+
+_default = None
+
+
+def default() -> Oracle:
+    """The oracle built from ``oracle.c`` in this directory (built on first use)."""
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default
+
+
+def fwd(*args, **kw):
+    return default().fwd(*args, **kw)
+
+
+def bwd(*args, **kw):
+    return default().bwd(*args, **kw)

@@ -1,0 +1,210 @@
+/*
+ * Plain fp64 CPU oracle for exact softmax attention, forward and backward.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may call, link or load
+ * this file: only the tests, the smoke check and the benchmark's CPU-baseline
+ * leg use it. It shares no code, header or constant with the CUDA library.
+ *
+ * What it computes is the textbook definition, with every N x N matrix
+ * materialised in fp64, in the order the definition states it:
+ *
+ *   S = scale * Q K^T                         (page "PyTorch-CUDA-v2.9镜像中使用FlashAttention
+ *                                              提升训练速度", the Attention(Q,K,V) formula;
+ *                                              page "告别OOM和训练慢…(含A100环境配置)" §1, the
+ *                                              three-line PyTorch implementation)
+ *   S_ij = -inf where key j is not visible from query i (causal: "mask future
+ *          positions", page "Flash Attention 3.7 核心原理与实战" §3.2; sliding window
+ *          `window_size=(left,right)`, page "告别OOM和训练慢…" §4.2)
+ *   P = row-softmax(S), with the row maximum subtracted first (`safe_softmax`,
+ *       page "告别OOM和训练慢…" §2.2)
+ *   O = P V
+ *   LSE_i = m_i + ln sum_j exp(S_ij - m_i)    (the per-row normalisation factor the
+ *                                              forward keeps for the backward, same page §2.2)
+ *
+ * The pages print no backward; the backward here is the chain rule of the above
+ * for the scalar L = <O, dO> (the "recompute P" backward of page
+ * "告别OOM和训练慢…" §2.2 and the recomputation paragraph of page
+ * "PyTorch-CUDA-v2.9镜像…", restated from the definition):
+ *   dV = P^T dO;  dP = dO V^T;  D_i = sum_j P_ij dP_ij;  dS = P o (dP - D);
+ *   dQ = scale * dS K;  dK = scale * dS^T Q.
+ *
+ * Readings where the pages are silent:
+ *   - visible(i, j) <=> (left < 0 or j >= i - left) and (right < 0 or j <= i + right);
+ *     -1 means unbounded; causal forces right = min(right, 0) (right = 0 when unbounded).
+ *   - a row with no visible key has P_i = 0, O_i = 0, LSE_i = -inf, and adds nothing
+ *     to any gradient.
+ *
+ * Layout: every tensor is (B, H, N, d) row-major fp64; lse is (B, H, N).
+ * Loops over rows are shared out with OpenMP; each output element is still
+ * summed in plain index order.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static int resolve_right(int causal, long right)
+{
+    if (causal) {
+        if (right < 0 || right > 0) return 0;
+    }
+    return (int)right;
+}
+
+static int visible(long i, long j, long left, long right)
+{
+    if (left >= 0 && j < i - left) return 0;
+    if (right >= 0 && j > i + right) return 0;
+    return 1;
+}
+
+/* P (N x N) := softmax rows of the masked, scaled scores of one head; lse (N). */
+static void head_probabilities(const double *q, const double *k, long N, long d,
+                               double scale, long left, long right,
+                               double *P, double *lse)
+{
+    long i;
+#pragma omp parallel for schedule(static)
+    for (i = 0; i < N; ++i) {
+        double *Pi = P + i * N;
+        double m = -INFINITY;
+        long j, c;
+        for (j = 0; j < N; ++j) {
+            double s = 0.0;
+            for (c = 0; c < d; ++c) s += q[i * d + c] * k[j * d + c];
+            s *= scale;
+            if (!visible(i, j, left, right)) s = -INFINITY;
+            Pi[j] = s;
+            if (s > m) m = s;
+        }
+        if (m == -INFINITY) {
+            for (j = 0; j < N; ++j) Pi[j] = 0.0;
+            lse[i] = -INFINITY;
+            continue;
+        }
+        double sum = 0.0;
+        for (j = 0; j < N; ++j) {
+            Pi[j] = exp(Pi[j] - m);
+            sum += Pi[j];
+        }
+        for (j = 0; j < N; ++j) Pi[j] /= sum;
+        lse[i] = m + log(sum);
+    }
+}
+
+int oracle_attention_fwd(const double *q, const double *k, const double *v,
+                         long B, long H, long N, long d, double scale,
+                         int causal, long left, long right,
+                         double *o, double *lse)
+{
+    long bh;
+    if (B < 0 || H < 0 || N < 0 || d < 1) return 1;
+    right = resolve_right(causal, right);
+    double *P = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1) * (size_t)(N > 0 ? N : 1));
+    if (!P) return 2;
+    for (bh = 0; bh < B * H; ++bh) {
+        const double *qh = q + bh * N * d, *kh = k + bh * N * d, *vh = v + bh * N * d;
+        double *oh = o + bh * N * d;
+        long i;
+        head_probabilities(qh, kh, N, d, scale, left, right, P, lse + bh * N);
+        /* O = P V */
+#pragma omp parallel for schedule(static)
+        for (i = 0; i < N; ++i) {
+            long j, c;
+            for (c = 0; c < d; ++c) oh[i * d + c] = 0.0;
+            for (j = 0; j < N; ++j) {
+                double p = P[i * N + j];
+                for (c = 0; c < d; ++c) oh[i * d + c] += p * vh[j * d + c];
+            }
+        }
+    }
+    free(P);
+    return 0;
+}
+
+int oracle_attention_bwd(const double *q, const double *k, const double *v,
+                         const double *dout,
+                         long B, long H, long N, long d, double scale,
+                         int causal, long left, long right,
+                         double *dq, double *dk, double *dv)
+{
+    long bh;
+    if (B < 0 || H < 0 || N < 0 || d < 1) return 1;
+    right = resolve_right(causal, right);
+    size_t nn = (size_t)(N > 0 ? N : 1) * (size_t)(N > 0 ? N : 1);
+    double *P = (double *)malloc(sizeof(double) * nn);
+    double *dP = (double *)malloc(sizeof(double) * nn);
+    double *lse = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+    double *D = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+    if (!P || !dP || !lse || !D) {
+        free(P); free(dP); free(lse); free(D);
+        return 2;
+    }
+    for (bh = 0; bh < B * H; ++bh) {
+        const double *qh = q + bh * N * d, *kh = k + bh * N * d, *vh = v + bh * N * d;
+        const double *doh = dout + bh * N * d;
+        double *dqh = dq + bh * N * d, *dkh = dk + bh * N * d, *dvh = dv + bh * N * d;
+        long i, j;
+        head_probabilities(qh, kh, N, d, scale, left, right, P, lse);
+        /* dV = P^T dO */
+#pragma omp parallel for schedule(static)
+        for (j = 0; j < N; ++j) {
+            long ii, c;
+            for (c = 0; c < d; ++c) dvh[j * d + c] = 0.0;
+            for (ii = 0; ii < N; ++ii) {
+                double p = P[ii * N + j];
+                for (c = 0; c < d; ++c) dvh[j * d + c] += p * doh[ii * d + c];
+            }
+        }
+        /* dP = dO V^T ; D_i = sum_j P_ij dP_ij ; dS = P o (dP - D), stored over dP */
+#pragma omp parallel for schedule(static)
+        for (i = 0; i < N; ++i) {
+            long jj, c;
+            double acc = 0.0;
+            for (jj = 0; jj < N; ++jj) {
+                double s = 0.0;
+                for (c = 0; c < d; ++c) s += doh[i * d + c] * vh[jj * d + c];
+                dP[i * N + jj] = s;
+                acc += P[i * N + jj] * s;
+            }
+            D[i] = acc;
+            for (jj = 0; jj < N; ++jj) dP[i * N + jj] = P[i * N + jj] * (dP[i * N + jj] - D[i]);
+        }
+        /* dQ = scale * dS K */
+#pragma omp parallel for schedule(static)
+        for (i = 0; i < N; ++i) {
+            long jj, c;
+            for (c = 0; c < d; ++c) dqh[i * d + c] = 0.0;
+            for (jj = 0; jj < N; ++jj) {
+                double s = dP[i * N + jj];
+                for (c = 0; c < d; ++c) dqh[i * d + c] += s * kh[jj * d + c];
+            }
+            for (c = 0; c < d; ++c) dqh[i * d + c] *= scale;
+        }
+        /* dK = scale * dS^T Q */
+#pragma omp parallel for schedule(static)
+        for (j = 0; j < N; ++j) {
+            long ii, c;
+            for (c = 0; c < d; ++c) dkh[j * d + c] = 0.0;
+            for (ii = 0; ii < N; ++ii) {
+                double s = dP[ii * N + j];
+                for (c = 0; c < d; ++c) dkh[j * d + c] += s * qh[ii * d + c];
+            }
+            for (c = 0; c < d; ++c) dkh[j * d + c] *= scale;
+        }
+    }
+    free(P); free(dP); free(lse); free(D);
+    return 0;
+}
+
+/* Number of OpenMP threads the loops above use (for reporting the CPU baseline). */
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

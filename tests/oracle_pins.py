@@ -1,0 +1,285 @@
+"""Pins for the fp64 oracle: facts fixed by the mathematics of softmax attention,
+not by the oracle's own code.
+
+Each pin takes an ``oracle.Oracle`` and raises ``AssertionError`` when the oracle
+disagrees. ``test_oracle_pins.py`` runs them on the real oracle and
+``test_oracle_planted.py`` runs them on copies of the oracle with one planted
+mistake each, to show that every such mistake trips at least one pin.
+
+Sources of the facts:
+  * closed forms of the definition (page "PyTorch-CUDA-v2.9镜像中使用FlashAttention提升训练速度",
+    the Attention(Q,K,V) formula): Q = 0 gives the mean of the visible values; a row
+    that sees one key returns that key's value; one-hot keys with a large score select
+    one value row; constant value rows pass through unchanged;
+  * invariants of the softmax gradient: rows of dS sum to zero, so sum_j dK_j = 0 and
+    sum_j dV_j = sum_i dO_i; shifting K by u shifts LSE_i by scale * q_i . u; etc.;
+  * central finite differences of L = <O, dO> (the backward is the gradient of L);
+  * torch's fp64 CPU scaled_dot_product_attention and autograd, as an independent
+    library implementation of the same definition.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+# (causal, (left, right)) mask modes exercised by the pins
+MODES = [
+    (False, (-1, -1)),
+    (True, (-1, -1)),
+    (False, (2, 0)),
+    (False, (1, 1)),
+    (False, (0, 2)),
+    (True, (3, -1)),
+]
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _visible_count(i, N, causal, window):
+    """Number of keys row i sees: the width of the band [i-left, i+right] clipped to [0, N)."""
+    left, right = window
+    if causal:
+        right = 0 if (right < 0 or right > 0) else right
+    lo = 0 if left < 0 else max(0, i - left)
+    hi = N - 1 if right < 0 else min(N - 1, i + right)
+    return hi - lo + 1, lo, hi
+
+
+def pin_single_key(orc):
+    """N = 1: O = V, LSE = scale q.k, dQ = dK = 0, dV = dO (any mask mode)."""
+    r = _rng(1)
+    q, k, v, do = (r.standard_normal((2, 3, 1, 5)) for _ in range(4))
+    scale = 0.37
+    for causal, window in MODES:
+        o, lse = orc.fwd(q, k, v, scale, causal, window)
+        np.testing.assert_allclose(o, v, rtol=0, atol=1e-15)
+        np.testing.assert_allclose(lse, scale * np.sum(q * k, axis=-1), rtol=1e-14, atol=1e-14)
+        dq, dk, dv = orc.bwd(q, k, v, do, scale, causal, window)
+        np.testing.assert_allclose(dq, 0.0, atol=1e-15)
+        np.testing.assert_allclose(dk, 0.0, atol=1e-15)
+        np.testing.assert_allclose(dv, do, rtol=0, atol=1e-15)
+
+
+def pin_zero_queries(orc):
+    """Q = 0: every visible score is 0, so O_i is the plain mean of the visible V rows
+    and LSE_i = ln(number of visible keys), for every mask mode."""
+    r = _rng(2)
+    B, H, N, d = 1, 2, 9, 3
+    q = np.zeros((B, H, N, d))
+    k = r.standard_normal((B, H, N, d))
+    v = r.standard_normal((B, H, N, d))
+    for causal, window in MODES:
+        o, lse = orc.fwd(q, k, v, 0.5, causal, window)
+        for i in range(N):
+            cnt, lo, hi = _visible_count(i, N, causal, window)
+            np.testing.assert_allclose(o[:, :, i], v[:, :, lo:hi + 1].mean(axis=2),
+                                       rtol=1e-13, atol=1e-13)
+            np.testing.assert_allclose(lse[:, :, i], math.log(cnt), rtol=0, atol=1e-13)
+
+
+def pin_causal_first_row(orc):
+    """Causal row 0 sees only key 0: O_0 = V_0, LSE_0 = scale q_0.k_0 and dQ_0 = 0."""
+    r = _rng(3)
+    q, k, v, do = (r.standard_normal((2, 2, 6, 4)) for _ in range(4))
+    scale = 0.6
+    o, lse = orc.fwd(q, k, v, scale, True)
+    np.testing.assert_allclose(o[:, :, 0], v[:, :, 0], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse[:, :, 0], scale * np.sum(q[:, :, 0] * k[:, :, 0], axis=-1),
+                               rtol=1e-14, atol=1e-14)
+    dq, _, _ = orc.bwd(q, k, v, do, scale, True)
+    np.testing.assert_allclose(dq[:, :, 0], 0.0, atol=1e-15)
+
+
+def pin_one_hot_keys(orc):
+    """K_j = c e_j, Q_i = e_{pi(i)}, c * scale = 30: row i scores 30 on key pi(i) and 0
+    elsewhere, so LSE_i = ln(e^30 + N - 1) exactly and O_i = V_{pi(i)} up to N e^-30."""
+    N, d = 6, 8
+    c, scale = 256.0, 30.0 / 256.0
+    perm = np.array([3, 0, 5, 1, 4, 2])
+    k = np.zeros((1, 1, N, d))
+    q = np.zeros((1, 1, N, d))
+    for j in range(N):
+        k[0, 0, j, j] = c
+    for i in range(N):
+        q[0, 0, i, perm[i]] = 1.0
+    v = _rng(4).standard_normal((1, 1, N, d))
+    o, lse = orc.fwd(q, k, v, scale)
+    np.testing.assert_allclose(lse[0, 0], math.log(math.exp(30.0) + N - 1), rtol=0, atol=1e-13)
+    tol = 2 * N * math.exp(-30.0) * np.abs(v).max()
+    np.testing.assert_allclose(o[0, 0], v[0, 0, perm], rtol=0, atol=tol)
+
+
+def pin_constant_values(orc):
+    """All V rows equal w: O_i = w, and dP_ij = dO_i . w is constant along j, so dS = 0
+    and dQ = dK = 0, for every mask mode."""
+    r = _rng(5)
+    B, H, N, d = 1, 2, 7, 4
+    q = r.standard_normal((B, H, N, d))
+    k = r.standard_normal((B, H, N, d))
+    w = r.standard_normal((B, H, 1, d))
+    v = np.repeat(w, N, axis=2)
+    do = r.standard_normal((B, H, N, d))
+    for causal, window in MODES:
+        o, _ = orc.fwd(q, k, v, 0.8, causal, window)
+        np.testing.assert_allclose(o, v, rtol=1e-13, atol=1e-13)
+        dq, dk, _ = orc.bwd(q, k, v, do, 0.8, causal, window)
+        np.testing.assert_allclose(dq, 0.0, atol=1e-12)
+        np.testing.assert_allclose(dk, 0.0, atol=1e-12)
+
+
+def pin_two_keys_logistic(orc):
+    """Two keys, no mask, d = 1: P_i0 is the logistic function of s_i0 - s_i1, so
+    O_i = sigma(s_i0 - s_i1) v_0 + sigma(s_i1 - s_i0) v_1 and LSE_i = s_i1 + ln(1 + e^(s_i0 - s_i1))."""
+    q = np.array([0.3, -1.2]).reshape(1, 1, 2, 1)
+    k = np.array([1.5, -0.4]).reshape(1, 1, 2, 1)
+    v = np.array([2.0, -3.0]).reshape(1, 1, 2, 1)
+    scale = 0.9
+    o, lse = orc.fwd(q, k, v, scale)
+    for i in range(2):
+        s0 = scale * q[0, 0, i, 0] * k[0, 0, 0, 0]
+        s1 = scale * q[0, 0, i, 0] * k[0, 0, 1, 0]
+        p0 = 1.0 / (1.0 + math.exp(s1 - s0))
+        assert abs(o[0, 0, i, 0] - (p0 * 2.0 + (1 - p0) * -3.0)) < 1e-14
+        assert abs(lse[0, 0, i] - (s1 + math.log1p(math.exp(s0 - s1)))) < 1e-14
+
+
+def pin_finite_differences(orc):
+    """dQ, dK, dV equal central finite differences of L = <O, dO> on tiny inputs, for
+    every mask mode, to 1e-6 relative."""
+    h = 1e-6
+    for (N, d, seed) in [(1, 3, 11), (2, 1, 12), (5, 3, 13), (8, 4, 14)]:
+        r = _rng(seed)
+        q, k, v, do = (r.standard_normal((1, 1, N, d)) for _ in range(4))
+        scale = 0.7
+        for causal, window in MODES:
+            grads = orc.bwd(q, k, v, do, scale, causal, window)
+
+            def L(qq, kk, vv):
+                o, _ = orc.fwd(qq, kk, vv, scale, causal, window)
+                return float(np.sum(o * do))
+
+            for which, g in enumerate(grads):
+                fd = np.zeros_like(q)
+                for idx in np.ndindex(q.shape):
+                    args = [q.copy(), k.copy(), v.copy()]
+                    args[which][idx] += h
+                    lp = L(*args)
+                    args[which][idx] -= 2 * h
+                    lm = L(*args)
+                    fd[idx] = (lp - lm) / (2 * h)
+                err = np.abs(fd - g).max()
+                ref = max(1.0, np.abs(g).max())
+                assert err <= 1e-6 * ref, (N, d, causal, window, which, err)
+
+
+def pin_gradient_invariants(orc):
+    """Per head: sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i (every row sees a key);
+    <Q, dQ>_F = <K, dK>_F (scores are bilinear in Q and K)."""
+    r = _rng(6)
+    B, H, N, d = 2, 1, 33, 8
+    q, k, v, do = (r.standard_normal((B, H, N, d)) for _ in range(4))
+    for causal, window in MODES:
+        dq, dk, dv = orc.bwd(q, k, v, do, 0.35, causal, window)
+        np.testing.assert_allclose(dk.sum(axis=2), 0.0, atol=1e-11)
+        np.testing.assert_allclose(dv.sum(axis=2), do.sum(axis=2), rtol=1e-12, atol=1e-11)
+        lhs = np.sum(q * dq, axis=(2, 3))
+        rhs = np.sum(k * dk, axis=(2, 3))
+        np.testing.assert_allclose(lhs, rhs, rtol=1e-11, atol=1e-11)
+
+
+def pin_shift_invariants(orc):
+    """K_j -> K_j + u leaves O unchanged and shifts LSE_i by scale q_i . u;
+    V_j -> V_j + w shifts every O_i by w (rows of P sum to one)."""
+    r = _rng(7)
+    B, H, N, d = 1, 2, 17, 5
+    q, k, v = (r.standard_normal((B, H, N, d)) for _ in range(3))
+    u = r.standard_normal((B, H, 1, d))
+    w = r.standard_normal((B, H, 1, d))
+    scale = 0.45
+    for causal, window in MODES:
+        o, lse = orc.fwd(q, k, v, scale, causal, window)
+        o2, lse2 = orc.fwd(q, k + u, v, scale, causal, window)
+        np.testing.assert_allclose(o2, o, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(lse2 - lse, scale * np.sum(q * u, axis=-1), atol=1e-12)
+        o3, _ = orc.fwd(q, k, v + w, scale, causal, window)
+        np.testing.assert_allclose(o3 - o, np.broadcast_to(w, o.shape), atol=1e-12)
+
+
+def pin_key_permutation(orc):
+    """Without a mask, permuting the key/value rows together changes nothing."""
+    r = _rng(8)
+    q, k, v = (r.standard_normal((1, 2, 13, 6)) for _ in range(3))
+    perm = r.permutation(13)
+    o, lse = orc.fwd(q, k, v, 0.5)
+    o2, lse2 = orc.fwd(q, k[:, :, perm], v[:, :, perm], 0.5)
+    np.testing.assert_allclose(o2, o, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(lse2, lse, rtol=1e-13, atol=1e-13)
+
+
+def _band_mask(N, causal, window):
+    """Boolean (N, N) mask built from torch's tril/triu band routines."""
+    left, right = window
+    if causal:
+        right = 0 if (right < 0 or right > 0) else right
+    m = torch.ones(N, N, dtype=torch.bool)
+    if right >= 0:
+        m = torch.tril(m, diagonal=right)
+    if left >= 0:
+        m = torch.triu(m, diagonal=-left)
+    return m
+
+
+def pin_library_sdpa(orc):
+    """torch's fp64 CPU scaled_dot_product_attention (and autograd through it) gives the
+    same O and gradients; torch.logsumexp of the masked scores gives the same LSE."""
+    r = _rng(9)
+    B, H, N, d = 2, 2, 19, 7
+    q, k, v, do = (r.standard_normal((B, H, N, d)) for _ in range(4))
+    scale = 0.41
+    for causal, window in MODES:
+        mask = _band_mask(N, causal, window)
+        tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+        to = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask,
+                                                              scale=scale)
+        to.backward(torch.tensor(do))
+        scores = (torch.tensor(q) @ torch.tensor(k).transpose(-1, -2)) * scale
+        tlse = torch.logsumexp(scores.masked_fill(~mask, float("-inf")), dim=-1)
+        o, lse = orc.fwd(q, k, v, scale, causal, window)
+        dq, dk, dv = orc.bwd(q, k, v, do, scale, causal, window)
+        np.testing.assert_allclose(o, to.detach().numpy(), rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(lse, tlse.numpy(), rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=1e-11, atol=1e-11)
+        np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=1e-11, atol=1e-11)
+        np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=1e-11, atol=1e-11)
+
+
+def pin_self_similarity(orc):
+    """k = v = q (the page "显存神技：必学FlashAttention！" comparison input): each row's own
+    key has the largest score |q_i|^2 scale among keys of no larger norm, so O is finite,
+    LSE_i >= scale |q_i|^2 (the diagonal is one term of the sum) and the invariants hold."""
+    r = _rng(10)
+    q = r.standard_normal((1, 2, 11, 4))
+    for causal, window in MODES:
+        o, lse = orc.fwd(q, q, q, 0.5, causal, window)
+        assert np.all(np.isfinite(o))
+        assert np.all(lse >= 0.5 * np.sum(q * q, axis=-1) - 1e-12)
+
+
+ALL_PINS = [
+    pin_single_key,
+    pin_zero_queries,
+    pin_causal_first_row,
+    pin_one_hot_keys,
+    pin_constant_values,
+    pin_two_keys_logistic,
+    pin_finite_differences,
+    pin_gradient_invariants,
+    pin_shift_invariants,
+    pin_key_permutation,
+    pin_library_sdpa,
+    pin_self_similarity,
+]

@@ -1,0 +1,46 @@
+"""Plant one plausible mistake at a time in a copy of the oracle's C source and check
+that at least one pin catches it: the pins are not blind to dropped terms, wrong
+signs or indices, or transposed operands."""
+import os
+
+import pytest
+
+import oracle
+import oracle_pins
+
+# (name, exact text in oracle.c, replacement)
+PLANTS = [
+    ("scale dropped from the scores", "s *= scale;", "s *= 1.0;"),
+    ("window bound off by one", "if (left >= 0 && j < i - left) return 0;",
+     "if (left >= 0 && j <= i - left) return 0;"),
+    ("causal flag ignored", "if (right < 0 || right > 0) return 0;", "if (0) return 0;"),
+    ("row maximum left out of LSE", "lse[i] = m + log(sum);", "lse[i] = log(sum);"),
+    ("softmax not normalised", "for (j = 0; j < N; ++j) Pi[j] /= sum;",
+     "for (j = 0; j < N; ++j) Pi[j] /= 1.0;"),
+    ("O row index swapped", "oh[i * d + c] += p * vh[j * d + c];",
+     "oh[i * d + c] += p * vh[i * d + c];"),
+    ("dV uses P instead of P^T", "double p = P[ii * N + j];", "double p = P[j * N + ii];"),
+    ("dS sign of D flipped", "(dP[i * N + jj] - D[i])", "(dP[i * N + jj] + D[i])"),
+    ("dQ scale dropped", "dqh[i * d + c] *= scale;", "dqh[i * d + c] *= 1.0;"),
+    ("dK uses dS instead of dS^T", "double s = dP[ii * N + j];", "double s = dP[j * N + ii];"),
+    ("dK scale dropped", "dkh[j * d + c] *= scale;", "dkh[j * d + c] *= 1.0;"),
+    ("dP uses dO of the key row", "s += doh[i * d + c] * vh[jj * d + c];",
+     "s += doh[jj * d + c] * vh[jj * d + c];"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", PLANTS, ids=[p[0] for p in PLANTS])
+def test_plant_is_caught(tmp_path, name, old, new):
+    src = open(oracle.SOURCE).read()
+    assert src.count(old) == 1, "plant site must be unique: %r" % old
+    bad = tmp_path / "oracle_planted.c"
+    bad.write_text(src.replace(old, new))
+    lib = oracle.build(str(bad), str(tmp_path / "liboracle_planted.so"), force=True)
+    orc = oracle.Oracle(lib)
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(orc)
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, "no pin catches the planted mistake: %s" % name
