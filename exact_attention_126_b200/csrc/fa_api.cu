@@ -1,0 +1,302 @@
+// fa_api.cu - host side of the C ABI declared in include/fa.h.
+//
+// Validates every argument before touching the GPU, encodes one TMA tensor map per input
+// tensor ((B*H, N, d) viewed as a 3-D tensor so that the rows past N of a (batch, head)
+// read as zeros instead of the next head's rows), and launches the kernels of
+// fa_fwd.cuh / fa_bwd.cuh on the caller's stream.
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "fa.h"
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+
+namespace {
+
+using fa::kBlock;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// (B*H, N, d) bf16 tensor, box of 128 rows x 64 columns (128 bytes), 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)kBlock, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shared validation. Returns FA_OK and sets *empty when there is nothing to do.
+fa_status_t check_problem(int B, int H, int N, int d, bool* empty) {
+  *empty = false;
+  if (B < 0 || H < 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || N == 0) {
+    *empty = true;
+    return FA_OK;
+  }
+  const long long elems = (long long)B * H * N * d;
+  if (elems >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  if (fa::num_tiles(N) > 65535) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+fa_status_t check_mask(float scale, fa_window_t w) {
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (w.left < -1 || w.right < -1) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+fa_status_t check_ptrs(std::initializer_list<const void*> ptrs) {
+  for (const void* p : ptrs)
+    if (p == nullptr) return FA_ERR_INVALID_ARG;
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return FA_ERR_MISALIGNED;
+  return FA_OK;
+}
+
+template <typename Kernel>
+fa_status_t set_smem(Kernel k, int bytes) {
+  // Per device and kernel; cheap enough to repeat, but only needed once per device.
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
+             ? FA_OK
+             : FA_ERR_CUDA;
+}
+
+fa_status_t launched() {
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D>
+fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int BH,
+                       int N, float scale, int left, int right, cudaStream_t st) {
+  CUtensorMap mq, mkk, mv;
+  if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) || !make_map(&mv, v, BH, N, D))
+    return FA_ERR_CUDA;
+  using C = fa::FwdCfg<D>;
+  if (set_smem(fa::fa_fwd_kernel<D>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
+  fa::FwdArgs a;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.N = N;
+  a.n_qtiles = fa::num_tiles(N);
+  a.scale_log2 = scale * fa::kLog2e;
+  a.left = left;
+  a.right = right;
+  dim3 grid(BH, a.n_qtiles);
+  fa::fa_fwd_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, a);
+  return launched();
+}
+
+template <int D>
+fa_status_t launch_preprocess(const void* o, const void* dout, float* delta, long long rows,
+                              cudaStream_t st) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long rows_per_block = 8 * (32 / (D / 8));  // 8 warps
+  long long blocks = (rows + rows_per_block - 1) / rows_per_block;
+  const long long cap = (long long)sms * 8;
+  if (blocks > cap) blocks = cap;
+  fa::fa_bwd_preprocess_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), delta, rows);
+  return launched();
+}
+
+template <int D>
+fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void* dout,
+                        const float* lse, const float* delta, void* dk, void* dv, int BH, int N,
+                        float scale, int left, int right, cudaStream_t st) {
+  CUtensorMap mq, mkk, mv, mdo;
+  if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
+      !make_map(&mv, v, BH, N, D) || !make_map(&mdo, dout, BH, N, D))
+    return FA_ERR_CUDA;
+  using C = fa::BwdCfg<D>;
+  if (set_smem(fa::fa_bwd_dkdv_kernel<D>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
+  fa::BwdArgs a;
+  a.lse = lse;
+  a.delta = delta;
+  a.out0 = static_cast<__nv_bfloat16*>(dk);
+  a.out1 = static_cast<__nv_bfloat16*>(dv);
+  a.N = N;
+  a.n_tiles = fa::num_tiles(N);
+  a.scale = scale;
+  a.scale_log2 = scale * fa::kLog2e;
+  a.left = left;
+  a.right = right;
+  dim3 grid(BH, a.n_tiles);
+  fa::fa_bwd_dkdv_kernel<D><<<grid, 192, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, a);
+  return launched();
+}
+
+template <int D>
+fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* dout,
+                      const float* lse, const float* delta, void* dq, int BH, int N, float scale,
+                      int left, int right, cudaStream_t st) {
+  CUtensorMap mq, mkk, mv, mdo;
+  if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
+      !make_map(&mv, v, BH, N, D) || !make_map(&mdo, dout, BH, N, D))
+    return FA_ERR_CUDA;
+  using C = fa::BwdCfg<D>;
+  if (set_smem(fa::fa_bwd_dq_kernel<D>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
+  fa::BwdArgs a;
+  a.lse = lse;
+  a.delta = delta;
+  a.out0 = static_cast<__nv_bfloat16*>(dq);
+  a.out1 = nullptr;
+  a.N = N;
+  a.n_tiles = fa::num_tiles(N);
+  a.scale = scale;
+  a.scale_log2 = scale * fa::kLog2e;
+  a.left = left;
+  a.right = right;
+  dim3 grid(BH, a.n_tiles);
+  fa::fa_bwd_dq_kernel<D><<<grid, 192, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, a);
+  return launched();
+}
+
+size_t workspace_bytes(int B, int H, int N) {
+  const size_t raw = (size_t)B * H * N * sizeof(float);
+  return (raw + 255) & ~size_t(255);
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                   int N, int d, float scale, int causal, fa_window_t window, void* stream) {
+  bool empty;
+  fa_status_t s = check_problem(B, H, N, d, &empty);
+  if (s != FA_OK || empty) return s;
+  if ((s = check_mask(scale, window)) != FA_OK) return s;
+  if ((s = check_ptrs({q, k, v, o, lse})) != FA_OK) return s;
+  const int right = fa::resolve_right(causal, window.right);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_fwd<64>(q, k, v, o, lse, B * H, N, scale, window.left, right, st)
+                 : launch_fwd<128>(q, k, v, o, lse, B * H, N, scale, window.left, right, st);
+}
+
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
+  bool empty;
+  if (check_problem(B, H, N, d, &empty) != FA_OK || empty) return 0;
+  return workspace_bytes(B, H, N);
+}
+
+fa_status_t fa_bwd_preprocess(const void* o, const void* dout, float* delta, int B, int H, int N,
+                              int d, void* stream) {
+  bool empty;
+  fa_status_t s = check_problem(B, H, N, d, &empty);
+  if (s != FA_OK || empty) return s;
+  if ((s = check_ptrs({o, dout, delta})) != FA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long rows = (long long)B * H * N;
+  return d == 64 ? launch_preprocess<64>(o, dout, delta, rows, st)
+                 : launch_preprocess<128>(o, dout, delta, rows, st);
+}
+
+fa_status_t fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout,
+                        const float* lse, const float* delta, void* dk, void* dv, int B, int H,
+                        int N, int d, float scale, int causal, fa_window_t window, void* stream) {
+  bool empty;
+  fa_status_t s = check_problem(B, H, N, d, &empty);
+  if (s != FA_OK || empty) return s;
+  if ((s = check_mask(scale, window)) != FA_OK) return s;
+  if ((s = check_ptrs({q, k, v, dout, lse, delta, dk, dv})) != FA_OK) return s;
+  const int right = fa::resolve_right(causal, window.right);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_dkdv<64>(q, k, v, dout, lse, delta, dk, dv, B * H, N, scale,
+                                   window.left, right, st)
+                 : launch_dkdv<128>(q, k, v, dout, lse, delta, dk, dv, B * H, N, scale,
+                                    window.left, right, st);
+}
+
+fa_status_t fa_bwd_dq(const void* q, const void* k, const void* v, const void* dout,
+                      const float* lse, const float* delta, void* dq, int B, int H, int N, int d,
+                      float scale, int causal, fa_window_t window, void* stream) {
+  bool empty;
+  fa_status_t s = check_problem(B, H, N, d, &empty);
+  if (s != FA_OK || empty) return s;
+  if ((s = check_mask(scale, window)) != FA_OK) return s;
+  if ((s = check_ptrs({q, k, v, dout, lse, delta, dq})) != FA_OK) return s;
+  const int right = fa::resolve_right(causal, window.right);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_dq<64>(q, k, v, dout, lse, delta, dq, B * H, N, scale, window.left,
+                                 right, st)
+                 : launch_dq<128>(q, k, v, dout, lse, delta, dq, B * H, N, scale, window.left,
+                                  right, st);
+}
+
+fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                   const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                   float scale, int causal, fa_window_t window, void* workspace,
+                   size_t workspace_bytes_given, void* stream) {
+  bool empty;
+  fa_status_t s = check_problem(B, H, N, d, &empty);
+  if (s != FA_OK || empty) return s;
+  if ((s = check_mask(scale, window)) != FA_OK) return s;
+  if ((s = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv, workspace})) != FA_OK) return s;
+  if (workspace_bytes_given < workspace_bytes(B, H, N)) return FA_ERR_WORKSPACE;
+  float* delta = static_cast<float*>(workspace);
+  if ((s = fa_bwd_preprocess(o, dout, delta, B, H, N, d, stream)) != FA_OK) return s;
+  if ((s = fa_bwd_dkdv(q, k, v, dout, lse, delta, dk, dv, B, H, N, d, scale, causal, window,
+                       stream)) != FA_OK)
+    return s;
+  return fa_bwd_dq(q, k, v, dout, lse, delta, dq, B, H, N, d, scale, causal, window, stream);
+}
+
+const char* fa_status_string(fa_status_t status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: null pointer, negative size, bad scale or window";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: head_dim must be 64 or 128 and tensors < 2^31 elements";
+    case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED: pointers must be 16-byte aligned";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: workspace smaller than fa_bwd_workspace_bytes()";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA call failed";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a kernel abandoned a bounded wait";
+  }
+  return "FA_ERR_UNKNOWN";
+}
+
+fa_status_t fa_debug_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, fa::g_fa_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+    return FA_ERR_TIMEOUT;
+  }
+  return FA_OK;
+}
+
+int fa_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,575 @@
+// fa_bwd.cuh - attention backward for sm_100a: recompute P from the saved LSE.
+//
+// The pages give only the idea: keep the per-row normalisation factors and recompute
+// the attention matrix in the backward (page "告别OOM和训练慢…(含A100环境配置)" §2.2; page
+// "PyTorch-CUDA-v2.9镜像中使用FlashAttention提升训练速度", "3. 重计算策略"). The steps are the
+// chain rule of softmax attention for the loss L = <O, dO>:
+//
+//   delta_i = sum_c dO_ic O_ic                     fa_bwd_preprocess_kernel
+//   P_ij    = exp(scale q_i.k_j - LSE_i)           (recomputed, masked entries 0)
+//   dP_ij   = dO_i . v_j
+//   dS_ij   = P_ij (dP_ij - delta_i)
+//   dV_j    = sum_i P_ij dO_i ;  dK_j = scale sum_i dS_ij q_i      fa_bwd_dkdv_kernel
+//   dQ_i    = scale sum_j dS_ij k_j                                  fa_bwd_dq_kernel
+//
+// dK/dV are accumulated in TMEM by one CTA per 128-row key tile that walks the query
+// tiles it is visible from; it computes the transposed products S^T = K Q^T and
+// dP^T = V dO^T, so that each thread owns one key row and P^T, dS^T can go straight
+// back into TMEM as the A operand of dV += P^T dO and dK += dS^T Q. dQ is accumulated
+// the same way by one CTA per query tile walking its key tiles (S, dP, then
+// dQ += dS K). Nothing is reduced across CTAs, so the results are deterministic.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "sm100.cuh"
+#include "tiles.cuh"
+
+namespace fa {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ------------------------------------------------------------------------------------
+// delta = rowsum(dO * O) in fp32. G = D/8 lanes share a row, 16 bytes per lane.
+// ------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256)
+    fa_bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o,
+                             const __nv_bfloat16* __restrict__ dout, float* __restrict__ delta,
+                             long long rows) {
+  constexpr int G = D / 8;            // lanes per row
+  constexpr int kRowsPerWarp = 32 / G;
+  const int lane = threadIdx.x & 31;
+  const long long warp_global = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long n_warps = ((long long)gridDim.x * blockDim.x) >> 5;
+  const int sub = lane / G;           // row within the warp's group
+  const int part = lane % G;          // 16-byte slice of the row
+  for (long long base = warp_global * kRowsPerWarp; base < rows; base += n_warps * kRowsPerWarp) {
+    const long long r = base + sub;
+    float acc = 0.f;
+    if (r < rows) {
+      const uint4 a = *reinterpret_cast<const uint4*>(o + r * D + part * 8);
+      const uint4 b = *reinterpret_cast<const uint4*>(dout + r * D + part * 8);
+      const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+      const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        acc = fmaf(__uint_as_float(aw[w] << 16), __uint_as_float(bw[w] << 16), acc);
+        acc = fmaf(__uint_as_float(aw[w] & 0xFFFF0000u), __uint_as_float(bw[w] & 0xFFFF0000u), acc);
+      }
+    }
+#pragma unroll
+    for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (part == 0 && r < rows) delta[r] = acc;
+  }
+}
+
+struct BwdArgs {
+  const float* lse;
+  const float* delta;
+  __nv_bfloat16* out0;  // dkdv: dK ; dq: dQ
+  __nv_bfloat16* out1;  // dkdv: dV ; dq: unused
+  int N;
+  int n_tiles;
+  float scale;
+  float scale_log2;
+  int left;
+  int right;
+};
+
+// Shared layout of both backward kernels: two stationary tiles (X0, X1) loaded once, a
+// ring of stages holding two streamed tiles (Y0, Y1) each, plus per-stage row statistics.
+template <int D>
+struct BwdCfg {
+  static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  static constexpr int kTile = kBlock * D * 2;
+  static constexpr int kRegions = D / 64;
+  static constexpr int kRegionBytes = kBlock * 128;
+  static constexpr int kStages = (D == 64) ? 3 : 2;
+  static constexpr int kX0 = 0;
+  static constexpr int kX1 = kTile;
+  static constexpr int kY0 = 2 * kTile;                      // + s * kTile
+  static constexpr int kY1 = kY0 + kStages * kTile;          // + s * kTile
+  static constexpr int kLse = kY1 + kStages * kTile;         // + s * 512 (128 fp32)
+  static constexpr int kDelta = kLse + kStages * 512;        // + s * 512
+  static constexpr int kBar = kDelta + kStages * 512;
+  static constexpr int bXFull = 0;
+  static constexpr int bYFull = 1;
+  static constexpr int bYEmpty = bYFull + kStages;
+  static constexpr int bSFull = bYEmpty + kStages;
+  static constexpr int bDPFull = bSFull + 1;
+  static constexpr int bPFull = bDPFull + 1;
+  static constexpr int bDSFull = bPFull + 1;
+  static constexpr int bMmaDone = bDSFull + 1;
+  static constexpr int bMmaFin = bMmaDone + 1;
+  static constexpr int kNumBars = bMmaFin + 1;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kMisc + 16 + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t tS = 0;      // S or S^T (fp32), then P / dS in bf16 in place
+  static constexpr uint32_t tDP = 128;   // dP or dP^T (fp32), then dS^T in bf16 in place
+  static constexpr uint32_t tAcc0 = 256; // dK or dQ accumulator (D columns)
+  static constexpr uint32_t tAcc1 = 256 + D;  // dV accumulator (D columns)
+};
+
+// Loads row `t` (this thread's TMEM lane) of a 128-column fp32 block into x.
+__device__ __forceinline__ void load_row128(uint32_t taddr, float (&x)[128]) {
+  uint32_t u[4][32];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) tmem_ld32(taddr + 32 * q, u[q]);
+  tmem_wait_ld();
+#pragma unroll
+  for (int q = 0; q < 4; ++q) reg_fence(u[q]);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int c = 0; c < 32; ++c) x[32 * q + c] = __uint_as_float(u[q][c]);
+}
+
+// Writes this thread's D-column fp32 accumulator row, times `mul`, as bf16 to `dst`.
+template <int D>
+__device__ __forceinline__ void store_acc_row(uint32_t taddr, float mul, __nv_bfloat16* dst,
+                                              bool valid) {
+#pragma unroll
+  for (int q = 0; q < D / 32; ++q) {
+    uint32_t o[32];
+    tmem_ld32(taddr + 32 * q, o);
+    tmem_wait_ld();
+    reg_fence(o);
+    uint32_t w[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c)
+      w[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * mul, __uint_as_float(o[2 * c + 1]) * mul);
+    if (valid) {
+#pragma unroll
+      for (int v4 = 0; v4 < 4; ++v4)
+        st_global_v4(dst + 32 * q + 8 * v4, w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// dK, dV: one CTA per (batch*head, key tile j). X0 = K_j, X1 = V_j; per stage Y0 = Q_i,
+// Y1 = dO_i and the LSE (log2 units) and delta of the 128 rows of query tile i.
+// ------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ CUtensorMap tmdO, const BwdArgs a) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x;
+  const int j = blockIdx.y;  // causal: key tile 0 sees the most query tiles
+  const Mask mk{a.N, a.left, a.right};
+  int i_lo, i_hi;
+  q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
+  const int n_it = i_hi - i_lo + 1;
+
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
+  auto bar = [&](int i) -> uint32_t { return sb + C::kBar + 8u * i; };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::bXFull), 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar(C::bYFull + s), 32);
+      mbar_init(bar(C::bYEmpty + s), 1);
+    }
+    mbar_init(bar(C::bSFull), 1);
+    mbar_init(bar(C::bDPFull), 1);
+    mbar_init(bar(C::bPFull), 128);
+    mbar_init(bar(C::bDSFull), 128);
+    mbar_init(bar(C::bMmaDone), 1);
+    mbar_init(bar(C::bMmaFin), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 5) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_map(&tmQ);
+      tma_prefetch_map(&tmK);
+      tma_prefetch_map(&tmV);
+      tma_prefetch_map(&tmdO);
+      mbar_arrive_expect_tx(bar(C::bXFull), 2 * C::kTile);
+      for (int r = 0; r < C::kRegions; ++r) {
+        tma_load_3d(sb + C::kX0 + r * C::kRegionBytes, &tmK, bar(C::bXFull), r * 64, j * kBlock, bh);
+        tma_load_3d(sb + C::kX1 + r * C::kRegionBytes, &tmV, bar(C::bXFull), r * 64, j * kBlock, bh);
+      }
+    }
+    int ny = 0;
+    for (int it = 0; it < n_it; ++it) {
+      const int i = i_lo + it;
+      const int s = it % C::kStages;
+      if (!mbar_wait_warp(bar(C::bYEmpty + s), ((it / C::kStages) & 1) ^ 1, abort_flag)) break;
+      float* lse_s = reinterpret_cast<float*>(smem + C::kLse + s * 512);
+      float* del_s = reinterpret_cast<float*>(smem + C::kDelta + s * 512);
+      for (int e = lane; e < kBlock; e += 32) {
+        const int r = i * kBlock + e;
+        const bool v = r < a.N;
+        lse_s[e] = v ? a.lse[(size_t)bh * a.N + r] * kLog2e : INFINITY;
+        del_s[e] = v ? a.delta[(size_t)bh * a.N + r] : 0.f;
+      }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar(C::bYFull + s), 2 * C::kTile);
+        for (int r = 0; r < C::kRegions; ++r) {
+          tma_load_3d(sb + C::kY0 + s * C::kTile + r * C::kRegionBytes, &tmQ, bar(C::bYFull + s),
+                      r * 64, i * kBlock, bh);
+          tma_load_3d(sb + C::kY1 + s * C::kTile + r * C::kRegionBytes, &tmdO, bar(C::bYFull + s),
+                      r * 64, i * kBlock, bh);
+        }
+      } else {
+        mbar_arrive(bar(C::bYFull + s));
+      }
+      ++ny;
+    }
+    if (lane == 0) {
+      mbar_wait(bar(C::bXFull), 0, nullptr);
+      for (int s = 0; s < C::kStages; ++s) {
+        if (ny > s) {
+          const int last = s + C::kStages * ((ny - 1 - s) / C::kStages);
+          mbar_wait(bar(C::bYFull + s), (last / C::kStages) & 1, nullptr);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 4) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);
+      bool ok = mbar_wait(bar(C::bXFull), 0, abort_flag);
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int s = it % C::kStages;
+        if (!mbar_wait(bar(C::bYFull + s), (it / C::kStages) & 1, abort_flag)) break;
+        if (it > 0 && !mbar_wait(bar(C::bMmaDone), (it - 1) & 1, abort_flag)) break;
+        tc_fence_after();
+        // S^T = K_j Q_i^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
+          mma_ss(tmem + C::tS, sdesc_sw128(sb + C::kX0 + off, 16, 1024),
+                 sdesc_sw128(sb + C::kY0 + s * C::kTile + off, 16, 1024), idS, kk > 0);
+        }
+        tc_commit(bar(C::bSFull));
+        // dP^T = V_j dO_i^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
+          mma_ss(tmem + C::tDP, sdesc_sw128(sb + C::kX1 + off, 16, 1024),
+                 sdesc_sw128(sb + C::kY1 + s * C::kTile + off, 16, 1024), idS, kk > 0);
+        }
+        tc_commit(bar(C::bDPFull));
+        // dV += P^T dO_i
+        if (!mbar_wait(bar(C::bPFull), it & 1, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBlock / 16; ++kk)
+          mma_ts(tmem + C::tAcc1, tmem + C::tS + kk * 8,
+                 sdesc_sw128(sb + C::kY1 + s * C::kTile + kk * 2048, C::kRegionBytes, 1024), idA,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        // dK += dS^T Q_i
+        if (!mbar_wait(bar(C::bDSFull), it & 1, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBlock / 16; ++kk)
+          mma_ts(tmem + C::tAcc0, tmem + C::tDP + kk * 8,
+                 sdesc_sw128(sb + C::kY0 + s * C::kTile + kk * 2048, C::kRegionBytes, 1024), idA,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(C::bYEmpty + s));
+        tc_commit(bar(C::bMmaDone));
+      }
+      tc_commit(bar(C::bMmaFin));
+      mbar_wait(bar(C::bMmaFin), 0, nullptr);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ warps 0..3
+    const int t = threadIdx.x;
+    const int c = j * kBlock + t;  // this thread's key row
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const float sl2 = a.scale_log2;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int i = i_lo + it;
+      const int s = it % C::kStages;
+      if (!mbar_wait_warp(bar(C::bYFull + s), (it / C::kStages) & 1, abort_flag) ||
+          !mbar_wait_warp(bar(C::bSFull), it & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float* lse_s = reinterpret_cast<const float*>(smem + C::kLse + s * 512);
+      const float* del_s = reinterpret_cast<const float*>(smem + C::kDelta + s * 512);
+      float p[128];
+      load_row128(tmem + lane_base + C::tS, p);
+#pragma unroll
+      for (int r = 0; r < 128; ++r) p[r] = ex2(fmaf(p[r], sl2, -lse_s[r]));
+      if (!tile_all_visible(i, j, mk)) {
+#pragma unroll
+        for (int r = 0; r < 128; ++r)
+          if (!is_visible(i * kBlock + r, c, mk)) p[r] = 0.f;
+      }
+      {
+        uint32_t pk[64];
+#pragma unroll
+        for (int r = 0; r < 64; ++r) pk[r] = pack_bf16x2(p[2 * r], p[2 * r + 1]);
+        tmem_st32(tmem + lane_base + C::tS, pk);
+        tmem_st32(tmem + lane_base + C::tS + 32, pk + 32);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::bPFull));
+      if (!mbar_wait_warp(bar(C::bDPFull), it & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_base + C::tDP + 32 * q, u);
+        tmem_wait_ld();
+        reg_fence(u);
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int r0 = 32 * q + 2 * e;
+          const float ds0 = p[r0] * (__uint_as_float(u[2 * e]) - del_s[r0]);
+          const float ds1 = p[r0 + 1] * (__uint_as_float(u[2 * e + 1]) - del_s[r0 + 1]);
+          w[e] = pack_bf16x2(ds0, ds1);
+        }
+        // columns [16q, 16q+16) were already read (chunks <= q), so overwrite in place
+        tmem_st16(tmem + lane_base + C::tDP + 16 * q, w);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::bDSFull));
+    }
+    if (ok) ok = mbar_wait_warp(bar(C::bMmaDone), (n_it - 1) & 1, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      const bool valid = c < a.N;
+      const size_t off = ((size_t)bh * a.N + (valid ? c : 0)) * D;
+      store_acc_row<D>(tmem + lane_base + C::tAcc1, 1.f, a.out1 + off, valid);
+      store_acc_row<D>(tmem + lane_base + C::tAcc0, a.scale, a.out0 + off, valid);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// dQ: one CTA per (batch*head, query tile i). X0 = Q_i, X1 = dO_i; per stage Y0 = K_j,
+// Y1 = V_j.
+// ------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV,
+                     const __grid_constant__ CUtensorMap tmdO, const BwdArgs a) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x;
+  const int i = a.n_tiles - 1 - (int)blockIdx.y;  // longest causal rows first
+  const Mask mk{a.N, a.left, a.right};
+  int j_lo, j_hi;
+  kv_tiles_for_q_tile(i, mk, j_lo, j_hi);
+  const int n_it = j_hi - j_lo + 1;
+
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
+  auto bar = [&](int k) -> uint32_t { return sb + C::kBar + 8u * k; };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::bXFull), 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar(C::bYFull + s), 1);
+      mbar_init(bar(C::bYEmpty + s), 1);
+    }
+    mbar_init(bar(C::bSFull), 1);
+    mbar_init(bar(C::bDPFull), 1);
+    mbar_init(bar(C::bPFull), 128);  // unused here
+    mbar_init(bar(C::bDSFull), 128);
+    mbar_init(bar(C::bMmaDone), 1);
+    mbar_init(bar(C::bMmaFin), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 5) {
+    if (lane == 0) {
+      tma_prefetch_map(&tmQ);
+      tma_prefetch_map(&tmK);
+      tma_prefetch_map(&tmV);
+      tma_prefetch_map(&tmdO);
+      mbar_arrive_expect_tx(bar(C::bXFull), 2 * C::kTile);
+      for (int r = 0; r < C::kRegions; ++r) {
+        tma_load_3d(sb + C::kX0 + r * C::kRegionBytes, &tmQ, bar(C::bXFull), r * 64, i * kBlock, bh);
+        tma_load_3d(sb + C::kX1 + r * C::kRegionBytes, &tmdO, bar(C::bXFull), r * 64, i * kBlock, bh);
+      }
+      int ny = 0;
+      for (int it = 0; it < n_it; ++it) {
+        const int jj = j_lo + it;
+        const int s = it % C::kStages;
+        if (!mbar_wait(bar(C::bYEmpty + s), ((it / C::kStages) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::bYFull + s), 2 * C::kTile);
+        for (int r = 0; r < C::kRegions; ++r) {
+          tma_load_3d(sb + C::kY0 + s * C::kTile + r * C::kRegionBytes, &tmK, bar(C::bYFull + s),
+                      r * 64, jj * kBlock, bh);
+          tma_load_3d(sb + C::kY1 + s * C::kTile + r * C::kRegionBytes, &tmV, bar(C::bYFull + s),
+                      r * 64, jj * kBlock, bh);
+        }
+        ++ny;
+      }
+      mbar_wait(bar(C::bXFull), 0, nullptr);
+      for (int s = 0; s < C::kStages; ++s) {
+        if (ny > s) {
+          const int last = s + C::kStages * ((ny - 1 - s) / C::kStages);
+          mbar_wait(bar(C::bYFull + s), (last / C::kStages) & 1, nullptr);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 4) {
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);
+      bool ok = mbar_wait(bar(C::bXFull), 0, abort_flag);
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int s = it % C::kStages;
+        if (!mbar_wait(bar(C::bYFull + s), (it / C::kStages) & 1, abort_flag)) break;
+        if (it > 0 && !mbar_wait(bar(C::bMmaDone), (it - 1) & 1, abort_flag)) break;
+        tc_fence_after();
+        // S = Q_i K_j^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
+          mma_ss(tmem + C::tS, sdesc_sw128(sb + C::kX0 + off, 16, 1024),
+                 sdesc_sw128(sb + C::kY0 + s * C::kTile + off, 16, 1024), idS, kk > 0);
+        }
+        tc_commit(bar(C::bSFull));
+        // dP = dO_i V_j^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
+          mma_ss(tmem + C::tDP, sdesc_sw128(sb + C::kX1 + off, 16, 1024),
+                 sdesc_sw128(sb + C::kY1 + s * C::kTile + off, 16, 1024), idS, kk > 0);
+        }
+        tc_commit(bar(C::bDPFull));
+        // dQ += dS K_j
+        if (!mbar_wait(bar(C::bDSFull), it & 1, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBlock / 16; ++kk)
+          mma_ts(tmem + C::tAcc0, tmem + C::tS + kk * 8,
+                 sdesc_sw128(sb + C::kY0 + s * C::kTile + kk * 2048, C::kRegionBytes, 1024), idA,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(C::bYEmpty + s));
+        tc_commit(bar(C::bMmaDone));
+      }
+      tc_commit(bar(C::bMmaFin));
+      mbar_wait(bar(C::bMmaFin), 0, nullptr);
+    }
+    __syncwarp();
+  } else {
+    const int t = threadIdx.x;
+    const int r = i * kBlock + t;  // this thread's query row
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const float sl2 = a.scale_log2;
+    const bool valid = r < a.N;
+    const float lse2 = valid ? a.lse[(size_t)bh * a.N + r] * kLog2e : INFINITY;
+    const float dl = valid ? a.delta[(size_t)bh * a.N + r] : 0.f;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int jj = j_lo + it;
+      if (!mbar_wait_warp(bar(C::bSFull), it & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float p[128];
+      load_row128(tmem + lane_base + C::tS, p);
+#pragma unroll
+      for (int c = 0; c < 128; ++c) p[c] = ex2(fmaf(p[c], sl2, -lse2));
+      if (!tile_all_visible(i, jj, mk)) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (!is_visible(r, jj * kBlock + c, mk)) p[c] = 0.f;
+      }
+      if (!mbar_wait_warp(bar(C::bDPFull), it & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_base + C::tDP + 32 * q, u);
+        tmem_wait_ld();
+        reg_fence(u);
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c0 = 32 * q + 2 * e;
+          w[e] = pack_bf16x2(p[c0] * (__uint_as_float(u[2 * e]) - dl),
+                             p[c0 + 1] * (__uint_as_float(u[2 * e + 1]) - dl));
+        }
+        // dS goes over S, which is already in registers
+        tmem_st16(tmem + lane_base + C::tS + 16 * q, w);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::bDSFull));
+    }
+    if (ok) ok = mbar_wait_warp(bar(C::bMmaDone), (n_it - 1) & 1, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      const size_t off = ((size_t)bh * a.N + (valid ? r : 0)) * D;
+      store_acc_row<D>(tmem + lane_base + C::tAcc0, a.scale, a.out0 + off, valid);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,64 @@
+// tiles.cuh - which (query tile, key tile) pairs carry work, and which scores are masked.
+//
+// A tile is 128 consecutive rows of one (batch, head). Key j is visible from query i iff
+// i - left <= j <= i + right (-1 = unbounded), both < N; causal masking forces right = 0
+// (page "告别OOM和训练慢…(含A100环境配置)" §4.2, `causal`, `window_size=(-1,-1)`; page
+// "Flash Attention 3.7 核心原理与实战" §3.2, "mask future positions"). Tiles whose every
+// score is masked are never visited; tiles whose every score is visible skip the
+// element-wise test.
+#pragma once
+
+namespace fa {
+
+constexpr int kBlock = 128;  // rows of a tile; the M (and N) extent of every MMA
+
+struct Mask {
+  int N;      // sequence length
+  int left;   // -1 = unbounded
+  int right;  // -1 = unbounded, 0 when causal
+};
+
+__host__ __device__ inline int resolve_right(int causal, int right) {
+  return causal ? 0 : right;
+}
+
+__host__ __device__ inline int num_tiles(int N) { return (N + kBlock - 1) / kBlock; }
+
+// Key tiles [lo, hi] holding at least one key visible from some valid row of query tile m.
+__host__ __device__ inline void kv_tiles_for_q_tile(int m, const Mask& k, int& lo, int& hi) {
+  const long long r0 = (long long)m * kBlock;
+  const long long r1 = (r0 + kBlock < k.N ? r0 + kBlock : k.N) - 1;
+  long long c0 = 0, c1 = k.N - 1;
+  if (k.left >= 0 && r0 - k.left > c0) c0 = r0 - k.left;
+  if (k.right >= 0 && r1 + k.right < c1) c1 = r1 + k.right;
+  lo = (int)(c0 / kBlock);
+  hi = (int)(c1 / kBlock);
+}
+
+// Query tiles [lo, hi] holding at least one valid row that sees some key of key tile j.
+__host__ __device__ inline void q_tiles_for_kv_tile(int j, const Mask& k, int& lo, int& hi) {
+  const long long c0 = (long long)j * kBlock;
+  const long long c1 = (c0 + kBlock < k.N ? c0 + kBlock : k.N) - 1;
+  long long r0 = 0, r1 = k.N - 1;
+  if (k.right >= 0 && c0 - k.right > r0) r0 = c0 - k.right;
+  if (k.left >= 0 && c1 + k.left < r1) r1 = c1 + k.left;
+  lo = (int)(r0 / kBlock);
+  hi = (int)(r1 / kBlock);
+}
+
+// True when every (row, key) of the pair (query tile qt, key tile kt) is visible and valid.
+__host__ __device__ inline bool tile_all_visible(int qt, int kt, const Mask& k) {
+  const long long r0 = (long long)qt * kBlock, r1 = r0 + kBlock - 1;
+  const long long c0 = (long long)kt * kBlock, c1 = c0 + kBlock - 1;
+  if (r1 >= k.N || c1 >= k.N) return false;
+  if (k.right >= 0 && c1 - r0 > k.right) return false;
+  if (k.left >= 0 && r1 - c0 > k.left) return false;
+  return true;
+}
+
+__host__ __device__ inline bool is_visible(int r, int c, const Mask& k) {
+  return r < k.N && c < k.N && (k.left < 0 || r - c <= k.left) &&
+         (k.right < 0 || c - r <= k.right);
+}
+
+}  // namespace fa

@@ -1,0 +1,205 @@
+"""Python binding of libfa.so: the C entry points of include/fa.h under the same names.
+
+Only argument marshalling happens here: shapes, dtypes and devices are read off torch
+tensors, their data pointers and the current CUDA stream are passed to the C ABI, and a
+non-OK status is raised as ``FAError``. Every step of the computation runs in the
+library's kernels; if the library cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(_PKG, "libfa.so")
+
+FA_OK = 0
+STATUS_NAMES = {
+    0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_MISALIGNED",
+    4: "FA_ERR_WORKSPACE", 5: "FA_ERR_CUDA", 6: "FA_ERR_TIMEOUT",
+}
+
+#: every symbol include/fa.h declares
+EXPORTED = ("fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_dkdv",
+            "fa_bwd_dq", "fa_status_string", "fa_debug_status", "fa_version")
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib().fa_status_string(status).decode() if _LIB is not None else STATUS_NAMES.get(status)
+        super().__init__("%s returned %s" % (where, msg))
+
+
+class fa_window_t(ctypes.Structure):
+    _fields_ = [("left", ctypes.c_int), ("right", ctypes.c_int)]
+
+
+_LIB = None
+
+
+def _lib() -> ctypes.CDLL:
+    """The loaded library (built in-tree by ``build.build()``); raises if it is absent."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIBRARY):
+            raise RuntimeError("libfa.so is not built (run exact_attention_126_b200.build.build());"
+                               " there is no fallback path")
+        lib = ctypes.CDLL(LIBRARY)
+        vp, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        W = fa_window_t
+        lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp]
+        lib.fa_bwd_workspace_bytes.argtypes = [I, I, I, I]
+        lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
+        lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp,
+                               ctypes.c_size_t, vp]
+        lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, I, I, I, I, vp]
+        lib.fa_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp]
+        lib.fa_bwd_dq.argtypes = [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp]
+        lib.fa_status_string.argtypes = [I]
+        lib.fa_status_string.restype = ctypes.c_char_p
+        lib.fa_debug_status.argtypes = [vp]
+        lib.fa_version.argtypes = []
+        for name in ("fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_dkdv", "fa_bwd_dq",
+                     "fa_debug_status", "fa_version"):
+            getattr(lib, name).restype = I
+        _LIB = lib
+    return _LIB
+
+
+def library() -> ctypes.CDLL:
+    return _lib()
+
+
+def _check(status: int, where: str) -> None:
+    if status != FA_OK:
+        raise FAError(status, where)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _shape(q: torch.Tensor):
+    if q.dim() != 4:
+        raise ValueError("expected a (batch, heads, seq_len, head_dim) tensor")
+    return tuple(int(x) for x in q.shape)
+
+
+def _window(causal: bool, window) -> tuple[int, fa_window_t]:
+    left, right = (-1, -1) if window is None else window
+    return int(bool(causal)), fa_window_t(int(left), int(right))
+
+
+def default_scale(d: int) -> float:
+    """softmax_scale=None means 1/sqrt(head_dim)."""
+    return 1.0 / math.sqrt(d)
+
+
+# ------------------------------------------------------------------ raw entry points
+def fa_fwd(q, k, v, o, lse, scale=None, causal=False, window=(-1, -1), stream=None) -> None:
+    B, H, N, d = _shape(q)
+    c, w = _window(causal, window)
+    s = default_scale(d) if scale is None else float(scale)
+    _check(_lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, s, c, w,
+                         _stream(stream)), "fa_fwd")
+
+
+def fa_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(_lib().fa_bwd_workspace_bytes(B, H, N, d))
+
+
+def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale=None, causal=False,
+           window=(-1, -1), stream=None) -> None:
+    B, H, N, d = _shape(q)
+    c, w = _window(causal, window)
+    s = default_scale(d) if scale is None else float(scale)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                         _ptr(dk), _ptr(dv), B, H, N, d, s, c, w, _ptr(workspace), nbytes,
+                         _stream(stream)), "fa_bwd")
+
+
+def fa_bwd_preprocess(o, do, delta, stream=None) -> None:
+    B, H, N, d = _shape(o)
+    _check(_lib().fa_bwd_preprocess(_ptr(o), _ptr(do), _ptr(delta), B, H, N, d, _stream(stream)),
+           "fa_bwd_preprocess")
+
+
+def fa_bwd_dkdv(q, k, v, do, lse, delta, dk, dv, scale=None, causal=False, window=(-1, -1),
+                stream=None) -> None:
+    B, H, N, d = _shape(q)
+    c, w = _window(causal, window)
+    s = default_scale(d) if scale is None else float(scale)
+    _check(_lib().fa_bwd_dkdv(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(lse), _ptr(delta),
+                              _ptr(dk), _ptr(dv), B, H, N, d, s, c, w, _stream(stream)),
+           "fa_bwd_dkdv")
+
+
+def fa_bwd_dq(q, k, v, do, lse, delta, dq, scale=None, causal=False, window=(-1, -1),
+              stream=None) -> None:
+    B, H, N, d = _shape(q)
+    c, w = _window(causal, window)
+    s = default_scale(d) if scale is None else float(scale)
+    _check(_lib().fa_bwd_dq(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(lse), _ptr(delta),
+                            _ptr(dq), B, H, N, d, s, c, w, _stream(stream)), "fa_bwd_dq")
+
+
+def fa_status_string(status: int) -> str:
+    return _lib().fa_status_string(int(status)).decode()
+
+
+def fa_debug_status(stream=None) -> int:
+    return int(_lib().fa_debug_status(_stream(stream)))
+
+
+def fa_version() -> int:
+    return int(_lib().fa_version())
+
+
+# ------------------------------------------------------------------ allocating helpers
+def _check_inputs(*ts):
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must be on a CUDA device")
+        if t.dtype != torch.bfloat16:
+            raise ValueError("tensors must be bf16")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous (B, H, N, d)")
+        if t.shape != ts[0].shape:
+            raise ValueError("q, k, v (and dO) must share one shape")
+
+
+def attention_forward(q, k, v, scale=None, causal=False, window=(-1, -1), stream=None):
+    """Returns (O, LSE) for bf16 CUDA tensors q, k, v of shape (B, H, N, d)."""
+    _check_inputs(q, k, v)
+    B, H, N, d = _shape(q)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    fa_fwd(q, k, v, o, lse, scale, causal, window, stream)
+    return o, lse
+
+
+def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, window=(-1, -1),
+                       stream=None):
+    """Returns (dQ, dK, dV): the gradient of <O, dO>; lse comes from attention_forward."""
+    _check_inputs(q, k, v, o, do)
+    B, H, N, d = _shape(q)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(q)
+    dv = torch.empty_like(q)
+    ws = torch.empty(max(1, fa_bwd_workspace_bytes(B, H, N, d)), dtype=torch.uint8,
+                     device=q.device)
+    fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, scale, causal, window, stream)
+    return dq, dk, dv

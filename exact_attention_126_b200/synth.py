@@ -21,6 +21,9 @@ The pages' workloads use i.i.d. normal Q, K, V (and dO for the backward) in the
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import torch
 
@@ -64,16 +67,26 @@ def normal_f64(seed: int, count: int) -> np.ndarray:
     return _normal_range(seed, 0, count)
 
 
-def normal_bf16(seed: int, shape, chunk: int = 1 << 22) -> torch.Tensor:
-    """A host bf16 tensor of i.i.d. N(0,1) values with the given shape."""
+def normal_bf16(seed: int, shape, chunk: int = 1 << 21, pin: bool = False) -> torch.Tensor:
+    """A host bf16 tensor of i.i.d. N(0,1) values with the given shape (optionally in
+    pinned memory). Chunks are generated on a thread pool; the values do not depend on
+    the chunking."""
     count = int(np.prod(shape))
-    out = torch.empty(count, dtype=torch.bfloat16)
+    out = torch.empty(count, dtype=torch.bfloat16, pin_memory=pin)
     step = max(2, chunk - chunk % 2)
-    for lo in range(0, count, step):
-        hi = min(count, lo + step)
+
+    def fill(lo):
         # each chunk starts on an even element, so Box-Muller pairs never straddle chunks
+        hi = min(count, lo + step)
         vals = _normal_range(seed, lo, hi)
         out[lo:hi] = torch.from_numpy(vals.astype(np.float32)).to(torch.bfloat16)
+
+    starts = list(range(0, count, step))
+    if len(starts) > 1:
+        with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, starts))
+    elif starts:
+        fill(0)
     return out.view(*shape)
 
 
@@ -91,10 +104,10 @@ def _normal_range(seed: int, lo: int, hi: int) -> np.ndarray:
 
 
 def attention_inputs(B: int, H: int, N: int, d: int, cfg_index: int,
-                     with_grad: bool = True) -> dict:
+                     with_grad: bool = True, pin: bool = False) -> dict:
     """Host bf16 tensors q, k, v (and do) of shape (B, H, N, d), seeded per workload."""
     names = ["q", "k", "v"] + (["do"] if with_grad else [])
-    return {n: normal_bf16(config_seed(cfg_index, n), (B, H, N, d)) for n in names}
+    return {n: normal_bf16(config_seed(cfg_index, n), (B, H, N, d), pin=pin) for n in names}
 
 
 def to_f64(t: torch.Tensor) -> np.ndarray:

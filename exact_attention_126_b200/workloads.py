@@ -1,0 +1,81 @@
+"""The attention workloads the library is measured and checked on, and their work counts.
+
+Shapes follow the pages' own examples: B=2, H=8, N=1024, d=64 (page "Flash Attention 3.7
+核心原理与实战" §3.2); B=2, N=4096, model dim 512 in 8 heads (page "显存神技：必学FlashAttention！");
+B=32, H=16, N=2048, d=64 (page "告别OOM和训练慢…(含A100环境配置)" §1); 8192 tokens with
+head_dim 128 and a sliding window (page "PyTorch-CUDA-v2.9镜像…" on 8k sequences, page
+"Flash Attention 3.7 …" §5, page "告别OOM和训练慢…" §4.2 `window_size`).
+
+Work convention for throughput: forward 4*B*H*N^2*d flops, backward 2.5x the forward
+(fwd+bwd = 3.5x), halved for causal; a sliding window counts its visible (query, key)
+pairs, 4*B*H*d*pairs for the forward.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    window: tuple  # (left, right), -1 = unbounded
+    backward: bool
+    seed_index: int
+    scale: float | None = None  # None: 1/sqrt(d)
+
+    @property
+    def softmax_scale(self) -> float:
+        return self.scale if self.scale is not None else 1.0 / math.sqrt(self.d)
+
+    def visible_pairs(self) -> int:
+        """Exact number of visible (query, key) pairs of one (batch, head)."""
+        N = self.N
+        left, right = self.window
+        if self.causal:
+            right = 0
+        total = 0
+        # rows are grouped by which clip is active; closed form per row is
+        # hi - lo + 1 with lo = max(0, i-left) and hi = min(N-1, i+right)
+        for i in range(N):
+            lo = 0 if left < 0 else max(0, i - left)
+            hi = N - 1 if right < 0 else min(N - 1, i + right)
+            total += hi - lo + 1
+        return total
+
+    def fwd_flops(self) -> float:
+        """Forward flops by the metric's convention."""
+        base = 4.0 * self.B * self.H * self.N * self.N * self.d
+        if self.window != (-1, -1) and self.window[0] >= 0:
+            return 4.0 * self.B * self.H * self.d * self.visible_pairs()
+        return base / 2 if self.causal else base
+
+    def step_flops(self) -> float:
+        """Flops of one step: forward, plus backward (2.5x) when the workload has one."""
+        return self.fwd_flops() * (3.5 if self.backward else 1.0)
+
+    def tensor_bytes(self) -> int:
+        return self.B * self.H * self.N * self.d * 2
+
+    def fwd_bytes(self) -> int:
+        """Compulsory device-memory traffic of the forward: read Q, K, V; write O, LSE."""
+        return 4 * self.tensor_bytes() + 4 * self.B * self.H * self.N
+
+    def bwd_bytes(self) -> int:
+        """Compulsory traffic of the backward: read Q, K, V, O, dO, LSE; write dQ, dK, dV."""
+        return 8 * self.tensor_bytes() + 4 * self.B * self.H * self.N
+
+
+WORKLOADS = {
+    "c1": Workload("c1_tiny_b1h2n128d64", 1, 2, 128, 64, False, (-1, -1), True, 0, scale=0.125),
+    "c2": Workload("c2_fwd_b2h8n1024d64", 2, 8, 1024, 64, False, (-1, -1), False, 1),
+    "c3": Workload("c3_b2h8n4096d64", 2, 8, 4096, 64, False, (-1, -1), True, 2),
+    "c4": Workload("c4_causal_b32h16n2048d64", 32, 16, 2048, 64, True, (-1, -1), True, 3),
+    "c5c": Workload("c5_causal_b2h32n8192d128", 2, 32, 8192, 128, True, (-1, -1), True, 4),
+    "c5w": Workload("c5_window1024_b2h32n8192d128", 2, 32, 8192, 128, True, (1024, 0), True, 4),
+}

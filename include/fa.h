@@ -1,0 +1,151 @@
+/*
+ * fa.h - C ABI of the B200 (sm_100a) exact-attention library (libfa.so).
+ *
+ * The library computes exact softmax attention
+ *
+ *     O = softmax(scale * Q K^T + mask) V
+ *
+ * (page "PyTorch-CUDA-v2.9镜像中使用FlashAttention提升训练速度", the Attention(Q,K,V)
+ * formula) tile by tile with an online softmax, so that the N x N score matrix never
+ * reaches device memory (page "告别OOM和训练慢：用Flash Attention加速你的PyTorch大模型
+ * （含A100环境配置）" §2.1 tiling, §2.2 online softmax), and the training backward,
+ * which recomputes P from the per-row log-sum-exp saved by the forward (same page
+ * §2.2, "only the normalisation factors are stored").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Tensors.  q, k, v, o, dout, dq, dk, dv are bf16 tensors of shape
+ *   (B, H, N, d) = (batch, heads, seq_len, head_dim), fully contiguous, row-major
+ *   (page "Flash Attention 3.7 核心原理与实战" §3.2 states the problem in this shape).
+ *   lse is fp32 (B, H, N): the natural-log log-sum-exp of each row of the scaled,
+ *   masked scores. delta is fp32 (B, H, N): rowsum(dout * o).
+ *   Query and key sequences have the same length N.
+ * Sizes.  d must be 64 or 128 (else FA_ERR_UNSUPPORTED: the pages list 64 and 128
+ *   as the common head sizes and report "no available kernel" otherwise, page
+ *   "Flash Attention 3.7 …" §5). B, H, N >= 0; if any is 0 the call does nothing and
+ *   returns FA_OK. Each tensor must have fewer than 2^31 elements (else
+ *   FA_ERR_UNSUPPORTED).
+ * Scale.  scale multiplies Q K^T before the mask. It is used exactly as given and
+ *   must be finite and > 0 (else FA_ERR_INVALID_ARG); pass 1/sqrt(d) for the usual
+ *   default (`softmax_scale=None`, page "告别OOM和训练慢…" §4.2).
+ * Mask.  Key j is visible from query i iff
+ *     (window.left  < 0 or j >= i - window.left) and
+ *     (window.right < 0 or j <= i + window.right),
+ *   with -1 meaning unbounded (`window_size=(-1,-1)`, page "告别OOM和训练慢…" §4.2).
+ *   causal != 0 masks future positions, i.e. forces window.right = 0 when it is -1
+ *   or positive. Values below -1 give FA_ERR_INVALID_ARG. Every query sees at least
+ *   itself, so no row is fully masked.
+ * Memory.  Every pointer is caller-owned device memory that is only used during the
+ *   call's kernels; the library keeps nothing and allocates nothing. Pointers must be
+ *   non-null (FA_ERR_INVALID_ARG) and 16-byte aligned (FA_ERR_MISALIGNED: the
+ *   tensors are fetched by the Tensor Memory Accelerator, page "告别OOM和训练慢…" §4.3
+ *   "misaligned address").
+ * Streams.  stream is a cudaStream_t (NULL = the legacy default stream). All checks
+ *   run on the host before any launch and return synchronously; kernels are then
+ *   enqueued on the stream and the call returns without waiting. Launch failures
+ *   return FA_ERR_CUDA. Calls on distinct streams may run concurrently.
+ * Faults.  Every wait inside the kernels is bounded (about two seconds). A kernel
+ *   whose wait runs out abandons its work, records FA_ERR_TIMEOUT in a device
+ *   status word and exits; fa_debug_status() reports and clears it.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad scale or window  */
+    FA_ERR_UNSUPPORTED = 2,  /* head_dim not 64/128, or a tensor of >= 2^31 elements */
+    FA_ERR_MISALIGNED = 3,   /* a pointer that is not 16-byte aligned               */
+    FA_ERR_WORKSPACE = 4,    /* workspace smaller than fa_bwd_workspace_bytes()     */
+    FA_ERR_CUDA = 5,         /* a CUDA runtime or driver call failed                */
+    FA_ERR_TIMEOUT = 6       /* a kernel abandoned a bounded wait (fa_debug_status) */
+} fa_status_t;
+
+/* Sliding window (`window_size=(left,right)`): keys j with i-left <= j <= i+right. */
+typedef struct {
+    int left;
+    int right;
+} fa_window_t;
+
+/*
+ * Forward pass.
+ *   in : q, k, v  (B,H,N,d) bf16
+ *   out: o (B,H,N,d) bf16, rounded to nearest even from fp32;
+ *        lse (B,H,N) fp32, natural log.
+ * One fused kernel: S = scale Q K^T is formed tile by tile in tensor memory, the
+ * running max m and sum l are updated per row (page "告别OOM和训练慢…" §2.2), the output
+ * accumulates P V in tensor memory and is divided by l at the end; only O and LSE are
+ * written to device memory.
+ */
+fa_status_t fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                   int B, int H, int N, int d, float scale, int causal,
+                   fa_window_t window, void *stream);
+
+/*
+ * Bytes of device workspace fa_bwd() needs: room for delta, B*H*N fp32 values,
+ * rounded up to 256 bytes. Returns 0 for an empty problem or invalid sizes.
+ */
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * Backward pass: the gradient of the scalar <O, dO> with respect to q, k and v.
+ *   in : q, k, v, o, dout (B,H,N,d) bf16; lse (B,H,N) fp32 from fa_fwd with the
+ *        same q, k, v, scale and mask.
+ *   out: dq, dk, dv (B,H,N,d) bf16.
+ *   workspace: caller-owned device scratch of at least fa_bwd_workspace_bytes()
+ *        bytes (FA_ERR_WORKSPACE if workspace_bytes is smaller), 16-byte aligned.
+ * The pages state only that the backward recomputes the attention matrix from the
+ * stored normalisation factors (page "告别OOM和训练慢…" §2.2; page "PyTorch-CUDA-v2.9
+ * 镜像…", "3. 重计算策略"); the steps are the chain rule of softmax attention:
+ *   delta_i = sum_c dO_ic O_ic                 (fa_bwd_preprocess)
+ *   P = exp(scale Q K^T - LSE), dP = dO V^T, dS = P o (dP - delta),
+ *   dV = P^T dO, dK = scale dS^T Q             (fa_bwd_dkdv, one pass per key tile)
+ *   dQ = scale dS K                            (fa_bwd_dq, one pass per query tile)
+ * The three kernels run in that order on the stream; results are deterministic.
+ */
+fa_status_t fa_bwd(const void *q, const void *k, const void *v, const void *o,
+                   const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                   int B, int H, int N, int d, float scale, int causal,
+                   fa_window_t window, void *workspace, size_t workspace_bytes,
+                   void *stream);
+
+/* Step 1 of fa_bwd alone: delta (B,H,N) fp32 := rowsum(dout * o), summed in fp32. */
+fa_status_t fa_bwd_preprocess(const void *o, const void *dout, float *delta,
+                              int B, int H, int N, int d, void *stream);
+
+/* Step 2 of fa_bwd alone: dk, dv from q, k, v, dout, lse and delta (step 1's output). */
+fa_status_t fa_bwd_dkdv(const void *q, const void *k, const void *v, const void *dout,
+                        const float *lse, const float *delta, void *dk, void *dv,
+                        int B, int H, int N, int d, float scale, int causal,
+                        fa_window_t window, void *stream);
+
+/* Step 3 of fa_bwd alone: dq from q, k, v, dout, lse and delta (step 1's output). */
+fa_status_t fa_bwd_dq(const void *q, const void *k, const void *v, const void *dout,
+                      const float *lse, const float *delta, void *dq,
+                      int B, int H, int N, int d, float scale, int causal,
+                      fa_window_t window, void *stream);
+
+/* Static, human-readable name of a status code (never NULL). */
+const char *fa_status_string(fa_status_t status);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word the kernels of
+ * the current device write when a bounded wait runs out. Returns FA_ERR_TIMEOUT if it
+ * was set, FA_ERR_CUDA if the synchronisation failed, FA_OK otherwise.
+ */
+fa_status_t fa_debug_status(void *stream);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -1,0 +1,111 @@
+"""The C ABI without a GPU: the library loads, exports every entry point include/fa.h
+declares, and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_attention_126_b200 import build, fa
+
+HEADER = os.path.join(build.INCLUDE, "fa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return fa.library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    assert set(names) == set(fa.EXPORTED), names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_status_strings(lib):
+    for code, name in fa.STATUS_NAMES.items():
+        assert fa.fa_status_string(code).startswith(name)
+    assert fa.fa_status_string(99) == "FA_ERR_UNKNOWN"
+
+
+W = fa.fa_window_t
+A = 0x10000  # a fake, 16-byte aligned "device" address: never dereferenced on these paths
+
+
+def fwd(lib, q=A, k=A, v=A, o=A, lse=A, B=1, H=1, N=128, d=64, scale=0.125, causal=0,
+        window=(-1, -1)):
+    return lib.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, W(*window), None)
+
+
+def test_fwd_rejects_bad_arguments(lib):
+    assert fwd(lib, q=None) == 1
+    assert fwd(lib, lse=None) == 1
+    assert fwd(lib, q=A + 8) == 3
+    assert fwd(lib, o=A + 2) == 3
+    assert fwd(lib, d=96) == 2
+    assert fwd(lib, d=32) == 2
+    assert fwd(lib, B=-1) == 1
+    assert fwd(lib, N=-5) == 1
+    assert fwd(lib, scale=0.0) == 1
+    assert fwd(lib, scale=-0.1) == 1
+    assert fwd(lib, scale=float("nan")) == 1
+    assert fwd(lib, scale=float("inf")) == 1
+    assert fwd(lib, window=(-2, -1)) == 1
+    assert fwd(lib, window=(5, -3)) == 1
+    assert fwd(lib, B=1 << 12, H=1 << 12, N=256, d=64) == 2  # >= 2^31 elements
+
+
+def test_empty_problem_is_a_no_op(lib):
+    # nothing is launched, so even null pointers are accepted
+    assert fwd(lib, q=None, k=None, v=None, o=None, lse=None, N=0) == 0
+    assert fwd(lib, B=0) == 0
+    assert fwd(lib, H=0) == 0
+    assert lib.fa_bwd_workspace_bytes(1, 1, 0, 64) == 0
+
+
+def test_workspace_size(lib):
+    assert lib.fa_bwd_workspace_bytes(2, 8, 4096, 64) == 2 * 8 * 4096 * 4
+    assert lib.fa_bwd_workspace_bytes(1, 1, 3, 64) == 256
+    assert lib.fa_bwd_workspace_bytes(1, 1, 3, 80) == 0
+
+
+def bwd(lib, ws=A, ws_bytes=1 << 20, **kw):
+    args = dict(q=A, k=A, v=A, o=A, do=A, lse=A, dq=A, dk=A, dv=A, B=1, H=1, N=128, d=64,
+                scale=0.125, causal=0, window=(-1, -1))
+    args.update(kw)
+    a = args
+    return lib.fa_bwd(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"],
+                      a["dv"], a["B"], a["H"], a["N"], a["d"], a["scale"], a["causal"],
+                      W(*a["window"]), ws, ws_bytes, None)
+
+
+def test_bwd_rejects_bad_arguments(lib):
+    assert bwd(lib, dq=None) == 1
+    assert bwd(lib, ws=None) == 1
+    assert bwd(lib, dv=A + 4) == 3
+    assert bwd(lib, ws_bytes=128 * 4 - 1) == 4
+    assert bwd(lib, d=256) == 2
+    assert bwd(lib, window=(-7, 0)) == 1
+    assert lib.fa_bwd_preprocess(A, None, A, 1, 1, 128, 64, None) == 1
+    assert lib.fa_bwd_dkdv(A, A, A, A, A, A, A, A + 1, 1, 1, 128, 64, 0.1, 0, W(-1, -1),
+                           None) == 3
+    assert lib.fa_bwd_dq(A, A, A, A, A, A, A, 1, 1, 128, 128, -1.0, 0, W(-1, -1), None) == 1
+
+
+def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(fa, "_LIB", None)
+    monkeypatch.setattr(fa, "LIBRARY", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="no fallback"):
+        fa.library()
