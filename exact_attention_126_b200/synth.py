@@ -103,6 +103,22 @@ def _normal_range(seed: int, lo: int, hi: int) -> np.ndarray:
     return z[: hi - lo]
 
 
+def normal_bf16_range(seed: int, start: int, count: int) -> torch.Tensor:
+    """Elements ``start .. start+count-1`` of the tensor ``normal_bf16(seed, ...)`` would
+    produce (``start`` even), as a flat host bf16 tensor."""
+    vals = _normal_range(seed, start, start + count)
+    return torch.from_numpy(vals.astype(np.float32)).to(torch.bfloat16)
+
+
+def head_inputs(B: int, H: int, N: int, d: int, cfg_index: int, b: int, h: int,
+                names=("q", "k", "v", "do")) -> dict:
+    """The (N, d) slice of (batch b, head h) of each tensor of ``attention_inputs``,
+    without generating the other heads (N * d must be even)."""
+    start = (b * H + h) * N * d
+    return {n: normal_bf16_range(config_seed(cfg_index, n), start, N * d).view(1, 1, N, d)
+            for n in names}
+
+
 def attention_inputs(B: int, H: int, N: int, d: int, cfg_index: int,
                      with_grad: bool = True, pin: bool = False) -> dict:
     """Host bf16 tensors q, k, v (and do) of shape (B, H, N, d), seeded per workload."""

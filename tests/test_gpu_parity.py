@@ -60,21 +60,45 @@ def test_workload_full_size(name):
 
 
 def _rescale_inputs(N, d, alternate):
-    """Scores that grow by about 12 (base 2) per key tile along the sequence, so the running
-    maximum moves on every tile; with `alternate`, odd rows see falling scores instead, so
-    rows of one warp disagree on whether to rescale."""
+    """Inputs whose scores climb along the sequence, so that the running maximum of a row
+    keeps growing from key tile to key tile and the forward must rescale O and l.
+
+    q_i = 32 u (u a unit vector) and k_j = c j u + n_j with n_j ~ N(0, 1) and c chosen so
+    that the scores rise by about 6 nats per 128 keys, on top of noise of 4 nats (d = 64).
+    The large factor sits in Q, so K has no large common offset and dQ = scale dS K stays
+    well conditioned in bf16 (rounding dS to bf16 alone costs about 0.3%). With
+    `alternate`, odd rows get q_i = -32 u and see falling scores, so the rows of one warp
+    disagree on whether to rescale."""
     g = torch.Generator().manual_seed(7)
     u = torch.ones(d) / np.sqrt(d)
-    q = u.repeat(N, 1)
+    q = (32.0 * u).repeat(N, 1)
     if alternate:
         q[1::2] *= -1
-    step = 8.3 / (128 * (1.0 / np.sqrt(d)))  # ~8.3 nats per 128 keys
-    k = torch.arange(N, dtype=torch.float64)[:, None].float() * step * u[None] / (u @ u)
-    k = k + 0.05 * torch.randn(N, d, generator=g)
+    slope = 6.0 / (128 * (1.0 / np.sqrt(d)) * 32.0)
+    k = torch.arange(N, dtype=torch.float32)[:, None] * slope * u[None]
+    k = k + torch.randn(N, d, generator=g)
     v = torch.randn(N, d, generator=g)
     do = torch.randn(N, d, generator=g)
     cast = lambda t: t.to(torch.bfloat16).reshape(1, 1, N, d).contiguous()
     return {"q": cast(q), "k": cast(k), "v": cast(v), "do": cast(do)}
+
+
+def _rescale_events(inp, scale, causal):
+    """How many (row, key tile) steps raise a row's running maximum by more than 2^8
+    (8 in base-2 units), the threshold past which the forward rescales."""
+    q = synth.to_f64(inp["q"])[0, 0]
+    k = synth.to_f64(inp["k"])[0, 0]
+    s = (q @ k.T) * scale / np.log(2.0)
+    N = s.shape[0]
+    if causal:
+        s = np.where(np.tril(np.ones((N, N), dtype=bool)), s, -np.inf)
+    tiles = [s[:, t:t + 128].max(axis=1) for t in range(0, N, 128)]
+    run = tiles[0]
+    events = 0
+    for tmax in tiles[1:]:
+        events += int(np.sum(tmax > run + 8.0))
+        run = np.maximum(run, tmax)
+    return events
 
 
 @pytest.mark.parametrize("alternate", [False, True])
@@ -84,6 +108,7 @@ def test_running_max_rescale(d, alternate):
     inp = _rescale_inputs(N, d, alternate)
     scale = 1.0 / np.sqrt(d)
     for causal in (False, True):
+        assert _rescale_events(inp, scale, causal) >= 256  # the path is really taken
         out = G.run_library(inp, scale, causal, (-1, -1))
         errs = G.compare(inp, out, scale, causal, (-1, -1))
         G.assert_within_bounds(errs, (d, alternate, causal))
