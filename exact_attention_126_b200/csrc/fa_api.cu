@@ -64,7 +64,7 @@ fa_status_t check_problem(int B, int H, int N, int d, bool* empty) {
   }
   const long long elems = (long long)B * H * N * d;
   if (elems >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
-  if (fa::num_tiles(N) > 65535) return FA_ERR_UNSUPPORTED;
+  if ((long long)B * H > 65535) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 
@@ -110,7 +110,7 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   a.scale_log2 = scale * fa::kLog2e;
   a.left = left;
   a.right = right;
-  dim3 grid(BH, a.n_qtiles);
+  dim3 grid(a.n_qtiles, BH);
   fa::fa_fwd_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, a);
   return launched();
 }
@@ -151,7 +151,7 @@ fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void*
   a.scale_log2 = scale * fa::kLog2e;
   a.left = left;
   a.right = right;
-  dim3 grid(BH, a.n_tiles);
+  dim3 grid(a.n_tiles, BH);
   fa::fa_bwd_dkdv_kernel<D><<<grid, 192, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, a);
   return launched();
 }
@@ -177,7 +177,7 @@ fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* d
   a.scale_log2 = scale * fa::kLog2e;
   a.left = left;
   a.right = right;
-  dim3 grid(BH, a.n_tiles);
+  dim3 grid(a.n_tiles, BH);
   fa::fa_bwd_dq_kernel<D><<<grid, 192, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, a);
   return launched();
 }

@@ -165,8 +165,8 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
-  const int j = blockIdx.y;  // causal: key tile 0 sees the most query tiles
+  const int bh = blockIdx.y;
+  const int j = blockIdx.x;  // causal: key tile 0 sees the most query tiles
   const Mask mk{a.N, a.left, a.right};
   int i_lo, i_hi;
   q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
@@ -320,7 +320,13 @@ __global__ void __launch_bounds__(192, 1)
       float p[128];
       load_row128(tmem + lane_base + C::tS, p);
 #pragma unroll
-      for (int r = 0; r < 128; ++r) p[r] = ex2(fmaf(p[r], sl2, -lse_s[r]));
+      for (int r = 0; r < 128; r += 4) {
+        const float4 l4 = *reinterpret_cast<const float4*>(lse_s + r);
+        p[r] = ex2(fmaf(p[r], sl2, -l4.x));
+        p[r + 1] = ex2(fmaf(p[r + 1], sl2, -l4.y));
+        p[r + 2] = ex2(fmaf(p[r + 2], sl2, -l4.z));
+        p[r + 3] = ex2(fmaf(p[r + 3], sl2, -l4.w));
+      }
       if (!tile_all_visible(i, j, mk)) {
 #pragma unroll
         for (int r = 0; r < 128; ++r)
@@ -349,11 +355,13 @@ __global__ void __launch_bounds__(192, 1)
         reg_fence(u);
         uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
+        for (int e = 0; e < 16; e += 2) {
           const int r0 = 32 * q + 2 * e;
-          const float ds0 = p[r0] * (__uint_as_float(u[2 * e]) - del_s[r0]);
-          const float ds1 = p[r0 + 1] * (__uint_as_float(u[2 * e + 1]) - del_s[r0 + 1]);
-          w[e] = pack_bf16x2(ds0, ds1);
+          const float4 d4 = *reinterpret_cast<const float4*>(del_s + r0);
+          w[e] = pack_bf16x2(p[r0] * (__uint_as_float(u[2 * e]) - d4.x),
+                             p[r0 + 1] * (__uint_as_float(u[2 * e + 1]) - d4.y));
+          w[e + 1] = pack_bf16x2(p[r0 + 2] * (__uint_as_float(u[2 * e + 2]) - d4.z),
+                                 p[r0 + 3] * (__uint_as_float(u[2 * e + 3]) - d4.w));
         }
         // columns [16q, 16q+16) were already read (chunks <= q), so overwrite in place
         tmem_st16(tmem + lane_base + C::tDP + 16 * q, w);
@@ -396,8 +404,8 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
-  const int i = a.n_tiles - 1 - (int)blockIdx.y;  // longest causal rows first
+  const int bh = blockIdx.y;
+  const int i = a.n_tiles - 1 - (int)blockIdx.x;  // longest causal rows first
   const Mask mk{a.N, a.left, a.right};
   int j_lo, j_hi;
   kv_tiles_for_q_tile(i, mk, j_lo, j_hi);

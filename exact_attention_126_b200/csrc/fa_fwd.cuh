@@ -79,8 +79,8 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
-  const int m = a.n_qtiles - 1 - (int)blockIdx.y;  // longest causal rows first
+  const int bh = blockIdx.y;
+  const int m = a.n_qtiles - 1 - (int)blockIdx.x;  // within a head, longest causal rows first
   const Mask mk{a.N, a.left, a.right};
   int j_lo, j_hi;
   kv_tiles_for_q_tile(m, mk, j_lo, j_hi);
@@ -233,9 +233,16 @@ __global__ void __launch_bounds__(192, 1)
         for (int c = 0; c < 128; ++c)
           if (!is_visible(row, j * kBlock + c, mk)) x[c] = -INFINITY;
       }
-      float mx = x[0];
+      // row max as 8 independent chains folded by a tree (keeps the FMNMX pipe busy)
+      float mx8[8];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+      for (int c = 0; c < 8; ++c) mx8[c] = fmaxf(x[c], x[c + 8]);
+#pragma unroll
+      for (int c = 16; c < 128; c += 8)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], x[c + e]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_new = fmaxf(m_run, mx * sl2);
       const bool grow = m_new > m_run + 8.0f;
       float alpha = 1.f;
@@ -246,15 +253,15 @@ __global__ void __launch_bounds__(192, 1)
       }
       const float mb = (m_run == -INFINITY) ? 0.f : m_run;
       uint32_t pk[64];
-      float lsum = 0.f;
+      float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
         const float p0 = ex2(fmaf(x[2 * c], sl2, -mb));
         const float p1 = ex2(fmaf(x[2 * c + 1], sl2, -mb));
-        lsum += p0 + p1;
+        ls8[c & 7] += p0 + p1;
         pk[c] = pack_bf16x2(p0, p1);
       }
-      l_run += lsum;
+      l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       if (it > 0) {
         // O and the P buffer are busy until P_{j-1} V_{j-1} has finished.
         if (!mbar_wait_warp(bar(C::bODone), (it - 1) & 1, abort_flag)) {

@@ -23,8 +23,8 @@
  * Sizes.  d must be 64 or 128 (else FA_ERR_UNSUPPORTED: the pages list 64 and 128
  *   as the common head sizes and report "no available kernel" otherwise, page
  *   "Flash Attention 3.7 …" §5). B, H, N >= 0; if any is 0 the call does nothing and
- *   returns FA_OK. Each tensor must have fewer than 2^31 elements (else
- *   FA_ERR_UNSUPPORTED).
+ *   returns FA_OK. Each tensor must have fewer than 2^31 elements and B * H may be
+ *   at most 65535 (else FA_ERR_UNSUPPORTED).
  * Scale.  scale multiplies Q K^T before the mask. It is used exactly as given and
  *   must be finite and > 0 (else FA_ERR_INVALID_ARG); pass 1/sqrt(d) for the usual
  *   default (`softmax_scale=None`, page "告别OOM和训练慢…" §4.2).

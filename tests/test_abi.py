@@ -65,6 +65,7 @@ def test_fwd_rejects_bad_arguments(lib):
     assert fwd(lib, window=(-2, -1)) == 1
     assert fwd(lib, window=(5, -3)) == 1
     assert fwd(lib, B=1 << 12, H=1 << 12, N=256, d=64) == 2  # >= 2^31 elements
+    assert fwd(lib, B=65536, H=1, N=1, d=64) == 2  # more (batch, head) pairs than a grid holds
 
 
 def test_empty_problem_is_a_no_op(lib):
