@@ -90,8 +90,26 @@ fa_status_t set_smem(Kernel k, int bytes) {
              : FA_ERR_CUDA;
 }
 
+template <typename Kernel>
+int launch_regs(Kernel k) {
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, k) != cudaSuccess) return -1;
+  return attr.numRegs;
+}
+
 fa_status_t launched() {
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
 }
 
 template <int D>
@@ -102,15 +120,23 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     return FA_ERR_CUDA;
   using C = fa::FwdCfg<D>;
   if (set_smem(fa::fa_fwd_kernel<D>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
+  // The kernel moves registers between warpgroups (setmaxnreg); the split is sized for
+  // exactly kLaunchRegs per thread at launch. Any other build would leave a warpgroup
+  // waiting for registers that never come, so refuse to launch it.
+  if (launch_regs(fa::fa_fwd_kernel<D>) != C::kLaunchRegs) return FA_ERR_UNSUPPORTED;
   fa::FwdArgs a;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
   a.N = N;
+  a.BH = BH;
   a.n_qtiles = fa::num_tiles(N);
+  a.n_pairs = (a.n_qtiles + 1) / 2;
+  a.n_items = BH * a.n_pairs;
+  a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
   a.scale_log2 = scale * fa::kLog2e;
   a.left = left;
   a.right = right;
-  dim3 grid(a.n_qtiles, BH);
+  const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
   fa::fa_fwd_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, a);
   return launched();
 }

@@ -93,6 +93,27 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
+// A shared-memory lock taken by lane 0 of a warp: used to let the two warps that share
+// an SM sub-partition take turns on its special-function unit. Bounded like mbar_wait.
+__device__ __forceinline__ bool smem_lock_acquire(int* lock, volatile int* abort_flag) {
+  if (atomicCAS(lock, 0, 1) == 0) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t n = 1;; ++n) {
+    __nanosleep(20);
+    if (atomicCAS(lock, 0, 1) == 0) return true;
+    if ((n & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > kWaitLimitNs || n > kWaitLimitPolls) {
+        *abort_flag = 1;
+        atomicCAS(&g_fa_status, 0, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void smem_lock_release(int* lock) { atomicExch(lock, 0); }
+
 // ----------------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), no multicast
 // ----------------------------------------------------------------------------------
@@ -248,6 +269,20 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
 
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// ----------------------------------------------------------------------------------
+// Register reallocation between warpgroups (all four warps of a warpgroup execute it).
+// The sum over warpgroups must not exceed the registers the CTA was launched with.
+// ----------------------------------------------------------------------------------
+template <int N>
+__device__ __forceinline__ void regs_grow() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <int N>
+__device__ __forceinline__ void regs_shrink() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ----------------------------------------------------------------------------------
