@@ -120,18 +120,13 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     return FA_ERR_CUDA;
   using C = fa::FwdCfg<D>;
   if (set_smem(fa::fa_fwd_kernel<D>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
-  // The kernel moves registers between warpgroups (setmaxnreg); the split is sized for
-  // exactly kLaunchRegs per thread at launch. Any other build would leave a warpgroup
-  // waiting for registers that never come, so refuse to launch it.
-  if (launch_regs(fa::fa_fwd_kernel<D>) != C::kLaunchRegs) return FA_ERR_UNSUPPORTED;
   fa::FwdArgs a;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
   a.N = N;
   a.BH = BH;
   a.n_qtiles = fa::num_tiles(N);
-  a.n_pairs = (a.n_qtiles + 1) / 2;
-  a.n_items = BH * a.n_pairs;
+  a.n_items = BH * a.n_qtiles;
   a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
   a.scale_log2 = scale * fa::kLog2e;
   a.left = left;
@@ -178,7 +173,7 @@ fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void*
   a.left = left;
   a.right = right;
   dim3 grid(a.n_tiles, BH);
-  fa::fa_bwd_dkdv_kernel<D><<<grid, 192, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, a);
+  fa::fa_bwd_dkdv_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, a);
   return launched();
 }
 
@@ -204,7 +199,7 @@ fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* d
   a.left = left;
   a.right = right;
   dim3 grid(a.n_tiles, BH);
-  fa::fa_bwd_dq_kernel<D><<<grid, 192, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, a);
+  fa::fa_bwd_dq_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, a);
   return launched();
 }
 

@@ -18,6 +18,12 @@
 // back into TMEM as the A operand of dV += P^T dO and dK += dS^T Q. dQ is accumulated
 // the same way by one CTA per query tile walking its key tiles (S, dP, then
 // dQ += dS K). Nothing is reduced across CTAs, so the results are deterministic.
+//
+// In both kernels two warpgroups share every row: warpgroup h takes the 64 columns
+// 64h..64h+63 of it (query columns for dK/dV, key columns for dQ). P needs no row
+// maximum here (the LSE is known), so the two halves never wait for each other. The
+// MMA issuer orders the products so that the next tile's S and dP are computed while
+// the softmax warpgroups work on the current tile.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -93,45 +99,26 @@ struct BwdCfg {
   static constexpr int kLse = kY1 + kStages * kTile;         // + s * 512 (128 fp32)
   static constexpr int kDelta = kLse + kStages * 512;        // + s * 512
   static constexpr int kBar = kDelta + kStages * 512;
+  // barrier slots (meaning per kernel in the comments of each kernel)
   static constexpr int bXFull = 0;
   static constexpr int bYFull = 1;
   static constexpr int bYEmpty = bYFull + kStages;
-  static constexpr int bSFull = bYEmpty + kStages;
-  static constexpr int bDPFull = bSFull + 1;
-  static constexpr int bPFull = bDPFull + 1;
-  static constexpr int bDSFull = bPFull + 1;
-  static constexpr int bMmaDone = bDSFull + 1;
-  static constexpr int bMmaFin = bMmaDone + 1;
+  static constexpr int bA = bYEmpty + kStages;  // 8 kernel-specific barriers
+  static constexpr int bMmaFin = bA + 8;
   static constexpr int kNumBars = bMmaFin + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kSmemBytes = kMisc + 16 + 1024;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t tS = 0;      // S or S^T (fp32), then P / dS in bf16 in place
-  static constexpr uint32_t tDP = 128;   // dP or dP^T (fp32), then dS^T in bf16 in place
-  static constexpr uint32_t tAcc0 = 256; // dK or dQ accumulator (D columns)
-  static constexpr uint32_t tAcc1 = 256 + D;  // dV accumulator (D columns)
+  static constexpr int kThreads = 320;  // 8 softmax warps, MMA warp, producer warp
 };
 
-// Loads row `t` (this thread's TMEM lane) of a 128-column fp32 block into x.
-__device__ __forceinline__ void load_row128(uint32_t taddr, float (&x)[128]) {
-  uint32_t u[4][32];
+// Writes this thread's NC fp32 accumulator columns starting at `taddr`, times `mul`, as
+// bf16 to `dst`.
+template <int NC>
+__device__ __forceinline__ void store_acc_cols(uint32_t taddr, float mul, __nv_bfloat16* dst,
+                                               bool valid) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) tmem_ld32(taddr + 32 * q, u[q]);
-  tmem_wait_ld();
-#pragma unroll
-  for (int q = 0; q < 4; ++q) reg_fence(u[q]);
-#pragma unroll
-  for (int q = 0; q < 4; ++q)
-#pragma unroll
-    for (int c = 0; c < 32; ++c) x[32 * q + c] = __uint_as_float(u[q][c]);
-}
-
-// Writes this thread's D-column fp32 accumulator row, times `mul`, as bf16 to `dst`.
-template <int D>
-__device__ __forceinline__ void store_acc_row(uint32_t taddr, float mul, __nv_bfloat16* dst,
-                                              bool valid) {
-#pragma unroll
-  for (int q = 0; q < D / 32; ++q) {
+  for (int q = 0; q < NC / 32; ++q) {
     uint32_t o[32];
     tmem_ld32(taddr + 32 * q, o);
     tmem_wait_ld();
@@ -148,17 +135,49 @@ __device__ __forceinline__ void store_acc_row(uint32_t taddr, float mul, __nv_bf
   }
 }
 
+// Loads 64 consecutive fp32 TMEM columns of this thread's lane.
+__device__ __forceinline__ void load_cols64(uint32_t taddr, float (&x)[64]) {
+  uint32_t u[2][32];
+  tmem_ld32(taddr, u[0]);
+  tmem_ld32(taddr + 32, u[1]);
+  tmem_wait_ld();
+  reg_fence(u[0]);
+  reg_fence(u[1]);
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    x[c] = __uint_as_float(u[0][c]);
+    x[32 + c] = __uint_as_float(u[1][c]);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void bwd_init_common(uint8_t* smem, uint32_t sb, int warp) {
+  using C = BwdCfg<D>;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMisc);
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+}
+
 // ------------------------------------------------------------------------------------
 // dK, dV: one CTA per (batch*head, key tile j). X0 = K_j, X1 = V_j; per stage Y0 = Q_i,
 // Y1 = dO_i and the LSE (log2 units) and delta of the 128 rows of query tile i.
+// TMEM: S^T at 0, dP^T at 128, dK at 256, dV at 256 + D. Warpgroup h writes its bf16
+// half of P^T (dS^T) over the first 32 of its own 64 fp32 columns of S^T (dP^T), so the
+// A operand of dV (dK) takes K-steps 0..3 from columns 0..31 and 4..7 from 64..95.
+// MMA order per query tile i:  dV(i), S^T(i+1), dK(i), dP^T(i+1).
 // ------------------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmdO, const BwdArgs a) {
   using C = BwdCfg<D>;
+  constexpr uint32_t tS = 0, tDP = 128, tDK = 256, tDV = 256 + D;
+  constexpr int bSFull = C::bA + 0, bDPFull = C::bA + 1, bPFull = C::bA + 2,
+                bDSFull = C::bA + 3, bDVDone = C::bA + 4, bDKDone = C::bA + 5;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -182,25 +201,23 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(bar(C::bYFull + s), 32);
       mbar_init(bar(C::bYEmpty + s), 1);
     }
-    mbar_init(bar(C::bSFull), 1);
-    mbar_init(bar(C::bDPFull), 1);
-    mbar_init(bar(C::bPFull), 128);
-    mbar_init(bar(C::bDSFull), 128);
-    mbar_init(bar(C::bMmaDone), 1);
+    mbar_init(bar(bSFull), 1);
+    mbar_init(bar(bDPFull), 1);
+    mbar_init(bar(bPFull), 256);
+    mbar_init(bar(bDSFull), 256);
+    mbar_init(bar(bDVDone), 1);
+    mbar_init(bar(bDKDone), 1);
     mbar_init(bar(C::bMmaFin), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
-    tmem_relinquish();
-  }
+  bwd_init_common<D>(smem, sb, warp);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 5) {
+  if (warp == 9) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_map(&tmQ);
@@ -249,78 +266,102 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);
-      bool ok = mbar_wait(bar(C::bXFull), 0, abort_flag);
-      for (int it = 0; ok && it < n_it; ++it) {
-        const int s = it % C::kStages;
-        if (!mbar_wait(bar(C::bYFull + s), (it / C::kStages) & 1, abort_flag)) break;
-        if (it > 0 && !mbar_wait(bar(C::bMmaDone), (it - 1) & 1, abort_flag)) break;
-        tc_fence_after();
-        // S^T = K_j Q_i^T
+      // S^T = K_j Q_i^T and dP^T = V_j dO_i^T for the query tile in stage s
+      auto issue_s = [&](int s) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-          mma_ss(tmem + C::tS, sdesc_sw128(sb + C::kX0 + off, 16, 1024),
+          mma_ss(tmem + tS, sdesc_sw128(sb + C::kX0 + off, 16, 1024),
                  sdesc_sw128(sb + C::kY0 + s * C::kTile + off, 16, 1024), idS, kk > 0);
         }
-        tc_commit(bar(C::bSFull));
-        // dP^T = V_j dO_i^T
+        tc_commit(bar(bSFull));
+      };
+      auto issue_dp = [&](int s) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-          mma_ss(tmem + C::tDP, sdesc_sw128(sb + C::kX1 + off, 16, 1024),
+          mma_ss(tmem + tDP, sdesc_sw128(sb + C::kX1 + off, 16, 1024),
                  sdesc_sw128(sb + C::kY1 + s * C::kTile + off, 16, 1024), idS, kk > 0);
         }
-        tc_commit(bar(C::bDPFull));
+        tc_commit(bar(bDPFull));
+      };
+      bool ok = mbar_wait(bar(C::bXFull), 0, abort_flag) &&
+                mbar_wait(bar(C::bYFull + 0), 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        issue_dp(0);
+      }
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int s = it % C::kStages;
+        const bool more = it + 1 < n_it;
+        const int s1 = (it + 1) % C::kStages;
         // dV += P^T dO_i
-        if (!mbar_wait(bar(C::bPFull), it & 1, abort_flag)) break;
+        if (!mbar_wait(bar(bPFull), it & 1, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBlock / 16; ++kk)
-          mma_ts(tmem + C::tAcc1, tmem + C::tS + kk * 8,
+          mma_ts(tmem + tDV, tmem + tS + kk * 8 + (kk >> 2) * 32,
                  sdesc_sw128(sb + C::kY1 + s * C::kTile + kk * 2048, C::kRegionBytes, 1024), idA,
                  (it > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(bDVDone));
+        // S^T for the next query tile, once dV has read P^T out of the S^T columns
+        if (more) {
+          if (!mbar_wait(bar(C::bYFull + s1), ((it + 1) / C::kStages) & 1, abort_flag) ||
+              !mbar_wait(bar(bDVDone), it & 1, abort_flag))
+            break;
+          tc_fence_after();
+          issue_s(s1);
+        }
         // dK += dS^T Q_i
-        if (!mbar_wait(bar(C::bDSFull), it & 1, abort_flag)) break;
+        if (!mbar_wait(bar(bDSFull), it & 1, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBlock / 16; ++kk)
-          mma_ts(tmem + C::tAcc0, tmem + C::tDP + kk * 8,
+          mma_ts(tmem + tDK, tmem + tDP + kk * 8 + (kk >> 2) * 32,
                  sdesc_sw128(sb + C::kY0 + s * C::kTile + kk * 2048, C::kRegionBytes, 1024), idA,
                  (it > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar(C::bYEmpty + s));
-        tc_commit(bar(C::bMmaDone));
+        tc_commit(bar(bDKDone));
+        // dP^T for the next query tile, once dK has read dS^T out of the dP^T columns
+        if (more) {
+          if (!mbar_wait(bar(bDKDone), it & 1, abort_flag)) break;
+          tc_fence_after();
+          issue_dp(s1);
+        }
       }
       tc_commit(bar(C::bMmaFin));
       mbar_wait(bar(C::bMmaFin), 0, nullptr);
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------------ warps 0..3
-    const int t = threadIdx.x;
-    const int c = j * kBlock + t;  // this thread's key row
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    // ------------------------------------------------------------------ warps 0..7
+    const int h = warp >> 2;          // query columns 64h .. 64h+63 of the tile
+    const int t = threadIdx.x & 127;  // key row in the tile == TMEM lane
+    const int c = j * kBlock + t;     // this thread's key
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const float sl2 = a.scale_log2;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int i = i_lo + it;
       const int s = it % C::kStages;
       if (!mbar_wait_warp(bar(C::bYFull + s), (it / C::kStages) & 1, abort_flag) ||
-          !mbar_wait_warp(bar(C::bSFull), it & 1, abort_flag)) {
+          !mbar_wait_warp(bar(bSFull), it & 1, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float* lse_s = reinterpret_cast<const float*>(smem + C::kLse + s * 512);
-      const float* del_s = reinterpret_cast<const float*>(smem + C::kDelta + s * 512);
-      float p[128];
-      load_row128(tmem + lane_base + C::tS, p);
+      const float* lse_s = reinterpret_cast<const float*>(smem + C::kLse + s * 512) + 64 * h;
+      const float* del_s = reinterpret_cast<const float*>(smem + C::kDelta + s * 512) + 64 * h;
+      float p[64];
+      load_cols64(tmem + lane_base + tS + 64 * h, p);
 #pragma unroll
-      for (int r = 0; r < 128; r += 4) {
+      for (int r = 0; r < 64; r += 4) {
         const float4 l4 = *reinterpret_cast<const float4*>(lse_s + r);
         p[r] = ex2(fmaf(p[r], sl2, -l4.x));
         p[r + 1] = ex2(fmaf(p[r + 1], sl2, -l4.y));
@@ -329,54 +370,47 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (!tile_all_visible(i, j, mk)) {
 #pragma unroll
-        for (int r = 0; r < 128; ++r)
-          if (!is_visible(i * kBlock + r, c, mk)) p[r] = 0.f;
+        for (int r = 0; r < 64; ++r)
+          if (!is_visible(i * kBlock + 64 * h + r, c, mk)) p[r] = 0.f;
       }
       {
-        uint32_t pk[64];
+        uint32_t pk[32];
 #pragma unroll
-        for (int r = 0; r < 64; ++r) pk[r] = pack_bf16x2(p[2 * r], p[2 * r + 1]);
-        tmem_st32(tmem + lane_base + C::tS, pk);
-        tmem_st32(tmem + lane_base + C::tS + 32, pk + 32);
+        for (int r = 0; r < 32; ++r) pk[r] = pack_bf16x2(p[2 * r], p[2 * r + 1]);
+        tmem_st32(tmem + lane_base + tS + 64 * h, pk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(C::bPFull));
-      if (!mbar_wait_warp(bar(C::bDPFull), it & 1, abort_flag)) {
+      mbar_arrive(bar(bPFull));
+      if (!mbar_wait_warp(bar(bDPFull), it & 1, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      float dp[64];
+      load_cols64(tmem + lane_base + tDP + 64 * h, dp);
+      uint32_t w[32];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t u[32];
-        tmem_ld32(tmem + lane_base + C::tDP + 32 * q, u);
-        tmem_wait_ld();
-        reg_fence(u);
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          const int r0 = 32 * q + 2 * e;
-          const float4 d4 = *reinterpret_cast<const float4*>(del_s + r0);
-          w[e] = pack_bf16x2(p[r0] * (__uint_as_float(u[2 * e]) - d4.x),
-                             p[r0 + 1] * (__uint_as_float(u[2 * e + 1]) - d4.y));
-          w[e + 1] = pack_bf16x2(p[r0 + 2] * (__uint_as_float(u[2 * e + 2]) - d4.z),
-                                 p[r0 + 3] * (__uint_as_float(u[2 * e + 3]) - d4.w));
-        }
-        // columns [16q, 16q+16) were already read (chunks <= q), so overwrite in place
-        tmem_st16(tmem + lane_base + C::tDP + 16 * q, w);
+      for (int e = 0; e < 32; e += 2) {
+        const int r0 = 2 * e;
+        const float4 d4 = *reinterpret_cast<const float4*>(del_s + r0);
+        w[e] = pack_bf16x2(p[r0] * (dp[r0] - d4.x), p[r0 + 1] * (dp[r0 + 1] - d4.y));
+        w[e + 1] = pack_bf16x2(p[r0 + 2] * (dp[r0 + 2] - d4.z), p[r0 + 3] * (dp[r0 + 3] - d4.w));
       }
+      // bf16 dS^T goes over the first half of this warpgroup's own fp32 dP^T columns
+      tmem_st32(tmem + lane_base + tDP + 64 * h, w);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(C::bDSFull));
+      mbar_arrive(bar(bDSFull));
     }
-    if (ok) ok = mbar_wait_warp(bar(C::bMmaDone), (n_it - 1) & 1, abort_flag);
+    // dK(last) was committed after dV(last): its completion covers both accumulators
+    if (ok) ok = mbar_wait_warp(bar(bDKDone), (n_it - 1) & 1, abort_flag);
     if (ok) {
       tc_fence_after();
       const bool valid = c < a.N;
-      const size_t off = ((size_t)bh * a.N + (valid ? c : 0)) * D;
-      store_acc_row<D>(tmem + lane_base + C::tAcc1, 1.f, a.out1 + off, valid);
-      store_acc_row<D>(tmem + lane_base + C::tAcc0, a.scale, a.out0 + off, valid);
+      const size_t off = ((size_t)bh * a.N + (valid ? c : 0)) * D + (D / 2) * h;
+      store_acc_cols<D / 2>(tmem + lane_base + tDV + (D / 2) * h, 1.f, a.out1 + off, valid);
+      store_acc_cols<D / 2>(tmem + lane_base + tDK + (D / 2) * h, a.scale, a.out0 + off, valid);
     }
   }
 
@@ -390,14 +424,20 @@ __global__ void __launch_bounds__(192, 1)
 
 // ------------------------------------------------------------------------------------
 // dQ: one CTA per (batch*head, query tile i). X0 = Q_i, X1 = dO_i; per stage Y0 = K_j,
-// Y1 = V_j.
+// Y1 = V_j. TMEM: S in two buffers at 0 and 128 (bf16 dS goes over S, each warpgroup
+// over the first half of its own columns), dP at 256, dQ at 384. MMA order per key
+// tile j: S(j+1), dP(j+1), dQ(j).
 // ------------------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmdO, const BwdArgs a) {
   using C = BwdCfg<D>;
+  constexpr uint32_t tS0 = 0, tDP = 256, tDQ = 384;
+  // S full per buffer, dS full per buffer, dP full, dP free, dQ done
+  constexpr int bSFull = C::bA + 0, bDSFull = C::bA + 2, bDPFull = C::bA + 4,
+                bDPFree = C::bA + 5, bDQDone = C::bA + 6;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -421,25 +461,24 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(bar(C::bYFull + s), 1);
       mbar_init(bar(C::bYEmpty + s), 1);
     }
-    mbar_init(bar(C::bSFull), 1);
-    mbar_init(bar(C::bDPFull), 1);
-    mbar_init(bar(C::bPFull), 128);  // unused here
-    mbar_init(bar(C::bDSFull), 128);
-    mbar_init(bar(C::bMmaDone), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(bSFull + b), 1);
+      mbar_init(bar(bDSFull + b), 256);
+    }
+    mbar_init(bar(bDPFull), 1);
+    mbar_init(bar(bDPFree), 256);
+    mbar_init(bar(bDQDone), 1);
     mbar_init(bar(C::bMmaFin), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
-    tmem_relinquish();
-  }
+  bwd_init_common<D>(smem, sb, warp);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 5) {
+  if (warp == 9) {
     if (lane == 0) {
       tma_prefetch_map(&tmQ);
       tma_prefetch_map(&tmK);
@@ -473,51 +512,71 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);
-      bool ok = mbar_wait(bar(C::bXFull), 0, abort_flag);
-      for (int it = 0; ok && it < n_it; ++it) {
-        const int s = it % C::kStages;
-        if (!mbar_wait(bar(C::bYFull + s), (it / C::kStages) & 1, abort_flag)) break;
-        if (it > 0 && !mbar_wait(bar(C::bMmaDone), (it - 1) & 1, abort_flag)) break;
-        tc_fence_after();
-        // S = Q_i K_j^T
+      // S = Q_i K_j^T into buffer b, dP = dO_i V_j^T, for the key tile in stage s
+      auto issue_s = [&](int s, int b) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-          mma_ss(tmem + C::tS, sdesc_sw128(sb + C::kX0 + off, 16, 1024),
+          mma_ss(tmem + tS0 + 128u * b, sdesc_sw128(sb + C::kX0 + off, 16, 1024),
                  sdesc_sw128(sb + C::kY0 + s * C::kTile + off, 16, 1024), idS, kk > 0);
         }
-        tc_commit(bar(C::bSFull));
-        // dP = dO_i V_j^T
+        tc_commit(bar(bSFull + b));
+      };
+      auto issue_dp = [&](int s) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-          mma_ss(tmem + C::tDP, sdesc_sw128(sb + C::kX1 + off, 16, 1024),
+          mma_ss(tmem + tDP, sdesc_sw128(sb + C::kX1 + off, 16, 1024),
                  sdesc_sw128(sb + C::kY1 + s * C::kTile + off, 16, 1024), idS, kk > 0);
         }
-        tc_commit(bar(C::bDPFull));
+        tc_commit(bar(bDPFull));
+      };
+      bool ok = mbar_wait(bar(C::bXFull), 0, abort_flag) &&
+                mbar_wait(bar(C::bYFull + 0), 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_dp(0);
+      }
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int s = it % C::kStages;
+        const int b = it & 1;
+        if (it + 1 < n_it) {
+          const int s1 = (it + 1) % C::kStages;
+          // buffer 1-b held dS(it-1): dQ(it-1) must have read it
+          if (!mbar_wait(bar(C::bYFull + s1), ((it + 1) / C::kStages) & 1, abort_flag)) break;
+          if (it >= 1 && !mbar_wait(bar(bDQDone), (it - 1) & 1, abort_flag)) break;
+          tc_fence_after();
+          issue_s(s1, b ^ 1);
+          // dP has one buffer: the softmax must have read dP(it)
+          if (!mbar_wait(bar(bDPFree), it & 1, abort_flag)) break;
+          tc_fence_after();
+          issue_dp(s1);
+        }
         // dQ += dS K_j
-        if (!mbar_wait(bar(C::bDSFull), it & 1, abort_flag)) break;
+        if (!mbar_wait(bar(bDSFull + b), (it >> 1) & 1, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBlock / 16; ++kk)
-          mma_ts(tmem + C::tAcc0, tmem + C::tS + kk * 8,
+          mma_ts(tmem + tDQ, tmem + tS0 + 128u * b + kk * 8 + (kk >> 2) * 32,
                  sdesc_sw128(sb + C::kY0 + s * C::kTile + kk * 2048, C::kRegionBytes, 1024), idA,
                  (it > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar(C::bYEmpty + s));
-        tc_commit(bar(C::bMmaDone));
+        tc_commit(bar(bDQDone));
       }
       tc_commit(bar(C::bMmaFin));
       mbar_wait(bar(C::bMmaFin), 0, nullptr);
     }
     __syncwarp();
   } else {
-    const int t = threadIdx.x;
-    const int r = i * kBlock + t;  // this thread's query row
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int h = warp >> 2;          // key columns 64h .. 64h+63 of each key tile
+    const int t = threadIdx.x & 127;
+    const int r = i * kBlock + t;     // this thread's query row
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const float sl2 = a.scale_log2;
     const bool valid = r < a.N;
     const float lse2 = valid ? a.lse[(size_t)bh * a.N + r] * kLog2e : INFINITY;
@@ -525,50 +584,45 @@ __global__ void __launch_bounds__(192, 1)
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int jj = j_lo + it;
-      if (!mbar_wait_warp(bar(C::bSFull), it & 1, abort_flag)) {
+      const int b = it & 1;
+      if (!mbar_wait_warp(bar(bSFull + b), (it >> 1) & 1, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float p[128];
-      load_row128(tmem + lane_base + C::tS, p);
+      float p[64];
+      load_cols64(tmem + lane_base + tS0 + 128u * b + 64 * h, p);
 #pragma unroll
-      for (int c = 0; c < 128; ++c) p[c] = ex2(fmaf(p[c], sl2, -lse2));
+      for (int c = 0; c < 64; ++c) p[c] = ex2(fmaf(p[c], sl2, -lse2));
       if (!tile_all_visible(i, jj, mk)) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (!is_visible(r, jj * kBlock + c, mk)) p[c] = 0.f;
+        for (int c = 0; c < 64; ++c)
+          if (!is_visible(r, jj * kBlock + 64 * h + c, mk)) p[c] = 0.f;
       }
-      if (!mbar_wait_warp(bar(C::bDPFull), it & 1, abort_flag)) {
+      if (!mbar_wait_warp(bar(bDPFull), it & 1, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      float dp[64];
+      load_cols64(tmem + lane_base + tDP + 64 * h, dp);
+      tc_fence_before();
+      mbar_arrive(bar(bDPFree));
+      uint32_t w[32];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t u[32];
-        tmem_ld32(tmem + lane_base + C::tDP + 32 * q, u);
-        tmem_wait_ld();
-        reg_fence(u);
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c0 = 32 * q + 2 * e;
-          w[e] = pack_bf16x2(p[c0] * (__uint_as_float(u[2 * e]) - dl),
-                             p[c0 + 1] * (__uint_as_float(u[2 * e + 1]) - dl));
-        }
-        // dS goes over S, which is already in registers
-        tmem_st16(tmem + lane_base + C::tS + 16 * q, w);
-      }
+      for (int e = 0; e < 32; ++e)
+        w[e] = pack_bf16x2(p[2 * e] * (dp[2 * e] - dl), p[2 * e + 1] * (dp[2 * e + 1] - dl));
+      // bf16 dS goes over the first half of this warpgroup's own fp32 S columns
+      tmem_st32(tmem + lane_base + tS0 + 128u * b + 64 * h, w);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(C::bDSFull));
+      mbar_arrive(bar(bDSFull + b));
     }
-    if (ok) ok = mbar_wait_warp(bar(C::bMmaDone), (n_it - 1) & 1, abort_flag);
+    if (ok) ok = mbar_wait_warp(bar(bDQDone), (n_it - 1) & 1, abort_flag);
     if (ok) {
       tc_fence_after();
-      const size_t off = ((size_t)bh * a.N + (valid ? r : 0)) * D;
-      store_acc_row<D>(tmem + lane_base + C::tAcc0, a.scale, a.out0 + off, valid);
+      const size_t off = ((size_t)bh * a.N + (valid ? r : 0)) * D + (D / 2) * h;
+      store_acc_cols<D / 2>(tmem + lane_base + tDQ + (D / 2) * h, a.scale, a.out0 + off, valid);
     }
   }
 
