@@ -140,7 +140,6 @@ def run_ours(args, w, rank, world, local_rank):
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     ws = torch.empty(fa.fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
-    delta = ws.view(torch.float32)[: B * H * N]
     scale = w.softmax_scale
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
@@ -157,13 +156,13 @@ def run_ours(args, w, rank, world, local_rank):
         if evs is not None:
             evs[1].record(stream)
         if w.backward:
-            fa.fa_bwd_preprocess(o, do, delta, sp)
+            fa.fa_bwd_preprocess(o, do, lse, ws, sp)
             if evs is not None:
                 evs[2].record(stream)
-            fa.fa_bwd_dkdv(q, k, v, do, lse, delta, dk, dv, scale, w.causal, w.window, sp)
+            fa.fa_bwd_dkdv(q, k, v, do, ws, dk, dv, scale, w.causal, w.window, sp)
             if evs is not None:
                 evs[3].record(stream)
-            fa.fa_bwd_dq(q, k, v, do, lse, delta, dq, scale, w.causal, w.window, sp)
+            fa.fa_bwd_dq(q, k, v, do, ws, dq, scale, w.causal, w.window, sp)
             if evs is not None:
                 evs[4].record(stream)
 

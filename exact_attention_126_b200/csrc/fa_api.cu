@@ -136,24 +136,26 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   return launched();
 }
 
+int padded_rows(int N) { return fa::num_tiles(N) * kBlock; }
+
 template <int D>
-fa_status_t launch_preprocess(const void* o, const void* dout, float* delta, long long rows,
-                              cudaStream_t st) {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+fa_status_t launch_preprocess(const void* o, const void* dout, const float* lse, float* stats,
+                              int BH, int N, cudaStream_t st) {
+  const int Np = padded_rows(N);
+  const long long rows = (long long)BH * Np;
   const long long rows_per_block = 8 * (32 / (D / 8));  // 8 warps
   long long blocks = (rows + rows_per_block - 1) / rows_per_block;
-  const long long cap = (long long)sms * 8;
+  const long long cap = (long long)sm_count() * 8;
   if (blocks > cap) blocks = cap;
   fa::fa_bwd_preprocess_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), delta, rows);
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, stats,
+      BH, N, Np);
   return launched();
 }
 
 template <int D>
 fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void* dout,
-                        const float* lse, const float* delta, void* dk, void* dv, int BH, int N,
+                        const void* ws, void* dk, void* dv, int BH, int N,
                         float scale, int left, int right, cudaStream_t st) {
   CUtensorMap mq, mkk, mv, mdo;
   if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
@@ -162,8 +164,9 @@ fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void*
   using C = fa::BwdCfg<D>;
   if (set_smem(fa::fa_bwd_dkdv_kernel<D>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
   fa::BwdArgs a;
-  a.lse = lse;
-  a.delta = delta;
+  a.stats = static_cast<const float*>(ws);
+  a.stat_rows = (long long)BH * padded_rows(N);
+  a.Np = padded_rows(N);
   a.out0 = static_cast<__nv_bfloat16*>(dk);
   a.out1 = static_cast<__nv_bfloat16*>(dv);
   a.N = N;
@@ -179,7 +182,7 @@ fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void*
 
 template <int D>
 fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* dout,
-                      const float* lse, const float* delta, void* dq, int BH, int N, float scale,
+                      const void* ws, void* dq, int BH, int N, float scale,
                       int left, int right, cudaStream_t st) {
   CUtensorMap mq, mkk, mv, mdo;
   if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
@@ -188,8 +191,9 @@ fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* d
   using C = fa::BwdCfg<D>;
   if (set_smem(fa::fa_bwd_dq_kernel<D>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
   fa::BwdArgs a;
-  a.lse = lse;
-  a.delta = delta;
+  a.stats = static_cast<const float*>(ws);
+  a.stat_rows = (long long)BH * padded_rows(N);
+  a.Np = padded_rows(N);
   a.out0 = static_cast<__nv_bfloat16*>(dq);
   a.out1 = nullptr;
   a.N = N;
@@ -204,7 +208,7 @@ fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* d
 }
 
 size_t workspace_bytes(int B, int H, int N) {
-  const size_t raw = (size_t)B * H * N * sizeof(float);
+  const size_t raw = 2 * (size_t)B * H * padded_rows(N) * sizeof(float);
   return (raw + 255) & ~size_t(255);
 }
 
@@ -231,47 +235,47 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   return workspace_bytes(B, H, N);
 }
 
-fa_status_t fa_bwd_preprocess(const void* o, const void* dout, float* delta, int B, int H, int N,
-                              int d, void* stream) {
+fa_status_t fa_bwd_preprocess(const void* o, const void* dout, const float* lse,
+                              void* workspace, int B, int H, int N, int d, void* stream) {
   bool empty;
   fa_status_t s = check_problem(B, H, N, d, &empty);
   if (s != FA_OK || empty) return s;
-  if ((s = check_ptrs({o, dout, delta})) != FA_OK) return s;
+  if ((s = check_ptrs({o, dout, lse, workspace})) != FA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const long long rows = (long long)B * H * N;
-  return d == 64 ? launch_preprocess<64>(o, dout, delta, rows, st)
-                 : launch_preprocess<128>(o, dout, delta, rows, st);
+  float* stats = static_cast<float*>(workspace);
+  return d == 64 ? launch_preprocess<64>(o, dout, lse, stats, B * H, N, st)
+                 : launch_preprocess<128>(o, dout, lse, stats, B * H, N, st);
 }
 
 fa_status_t fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout,
-                        const float* lse, const float* delta, void* dk, void* dv, int B, int H,
-                        int N, int d, float scale, int causal, fa_window_t window, void* stream) {
+                        const void* workspace, void* dk, void* dv, int B, int H, int N, int d,
+                        float scale, int causal, fa_window_t window, void* stream) {
   bool empty;
   fa_status_t s = check_problem(B, H, N, d, &empty);
   if (s != FA_OK || empty) return s;
   if ((s = check_mask(scale, window)) != FA_OK) return s;
-  if ((s = check_ptrs({q, k, v, dout, lse, delta, dk, dv})) != FA_OK) return s;
+  if ((s = check_ptrs({q, k, v, dout, workspace, dk, dv})) != FA_OK) return s;
   const int right = fa::resolve_right(causal, window.right);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_dkdv<64>(q, k, v, dout, lse, delta, dk, dv, B * H, N, scale,
+  return d == 64 ? launch_dkdv<64>(q, k, v, dout, workspace, dk, dv, B * H, N, scale,
                                    window.left, right, st)
-                 : launch_dkdv<128>(q, k, v, dout, lse, delta, dk, dv, B * H, N, scale,
+                 : launch_dkdv<128>(q, k, v, dout, workspace, dk, dv, B * H, N, scale,
                                     window.left, right, st);
 }
 
 fa_status_t fa_bwd_dq(const void* q, const void* k, const void* v, const void* dout,
-                      const float* lse, const float* delta, void* dq, int B, int H, int N, int d,
-                      float scale, int causal, fa_window_t window, void* stream) {
+                      const void* workspace, void* dq, int B, int H, int N, int d, float scale,
+                      int causal, fa_window_t window, void* stream) {
   bool empty;
   fa_status_t s = check_problem(B, H, N, d, &empty);
   if (s != FA_OK || empty) return s;
   if ((s = check_mask(scale, window)) != FA_OK) return s;
-  if ((s = check_ptrs({q, k, v, dout, lse, delta, dq})) != FA_OK) return s;
+  if ((s = check_ptrs({q, k, v, dout, workspace, dq})) != FA_OK) return s;
   const int right = fa::resolve_right(causal, window.right);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_dq<64>(q, k, v, dout, lse, delta, dq, B * H, N, scale, window.left,
+  return d == 64 ? launch_dq<64>(q, k, v, dout, workspace, dq, B * H, N, scale, window.left,
                                  right, st)
-                 : launch_dq<128>(q, k, v, dout, lse, delta, dq, B * H, N, scale, window.left,
+                 : launch_dq<128>(q, k, v, dout, workspace, dq, B * H, N, scale, window.left,
                                   right, st);
 }
 
@@ -285,12 +289,11 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
   if ((s = check_mask(scale, window)) != FA_OK) return s;
   if ((s = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv, workspace})) != FA_OK) return s;
   if (workspace_bytes_given < workspace_bytes(B, H, N)) return FA_ERR_WORKSPACE;
-  float* delta = static_cast<float*>(workspace);
-  if ((s = fa_bwd_preprocess(o, dout, delta, B, H, N, d, stream)) != FA_OK) return s;
-  if ((s = fa_bwd_dkdv(q, k, v, dout, lse, delta, dk, dv, B, H, N, d, scale, causal, window,
+  if ((s = fa_bwd_preprocess(o, dout, lse, workspace, B, H, N, d, stream)) != FA_OK) return s;
+  if ((s = fa_bwd_dkdv(q, k, v, dout, workspace, dk, dv, B, H, N, d, scale, causal, window,
                        stream)) != FA_OK)
     return s;
-  return fa_bwd_dq(q, k, v, dout, lse, delta, dq, B, H, N, d, scale, causal, window, stream);
+  return fa_bwd_dq(q, k, v, dout, workspace, dq, B, H, N, d, scale, causal, window, stream);
 }
 
 const char* fa_status_string(fa_status_t status) {

@@ -5,7 +5,8 @@
 // "PyTorch-CUDA-v2.9镜像中使用FlashAttention提升训练速度", "3. 重计算策略"). The steps are the
 // chain rule of softmax attention for the loss L = <O, dO>:
 //
-//   delta_i = sum_c dO_ic O_ic                     fa_bwd_preprocess_kernel
+//   delta_i = sum_c dO_ic O_ic                     fa_bwd_preprocess_kernel (with LSE*log2e,
+//                                                  both padded to whole 128-row tiles)
 //   P_ij    = exp(scale q_i.k_j - LSE_i)           (recomputed, masked entries 0)
 //   dP_ij   = dO_i . v_j
 //   dS_ij   = P_ij (dP_ij - delta_i)
@@ -36,26 +37,34 @@ namespace fa {
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------------------------
-// delta = rowsum(dO * O) in fp32. G = D/8 lanes share a row, 16 bytes per lane.
+// Row statistics of the backward, over B*H rows of Np (N rounded up to 128) entries:
+//   stats[bh*Np + r]             = LSE_r * log2(e)        (+inf for r >= N)
+//   stats[BH*Np + bh*Np + r]     = rowsum(dO_r * O_r)     (0 for r >= N), summed in fp32
+// G = D/8 lanes share a row, 16 bytes of O and dO per lane.
 // ------------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256)
     fa_bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o,
-                             const __nv_bfloat16* __restrict__ dout, float* __restrict__ delta,
-                             long long rows) {
+                             const __nv_bfloat16* __restrict__ dout, const float* __restrict__ lse,
+                             float* __restrict__ stats, int BH, int N, int Np) {
   constexpr int G = D / 8;            // lanes per row
   constexpr int kRowsPerWarp = 32 / G;
+  const long long rows = (long long)BH * Np;
   const int lane = threadIdx.x & 31;
   const long long warp_global = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const long long n_warps = ((long long)gridDim.x * blockDim.x) >> 5;
   const int sub = lane / G;           // row within the warp's group
   const int part = lane % G;          // 16-byte slice of the row
   for (long long base = warp_global * kRowsPerWarp; base < rows; base += n_warps * kRowsPerWarp) {
-    const long long r = base + sub;
+    const long long rp = base + sub;  // padded row
+    const long long bh = rp / Np;
+    const int r = (int)(rp - bh * Np);
+    const bool real = rp < rows && r < N;
+    const long long src = bh * N + r;
     float acc = 0.f;
-    if (r < rows) {
-      const uint4 a = *reinterpret_cast<const uint4*>(o + r * D + part * 8);
-      const uint4 b = *reinterpret_cast<const uint4*>(dout + r * D + part * 8);
+    if (real) {
+      const uint4 a = *reinterpret_cast<const uint4*>(o + src * D + part * 8);
+      const uint4 b = *reinterpret_cast<const uint4*>(dout + src * D + part * 8);
       const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
       const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
@@ -66,16 +75,20 @@ __global__ void __launch_bounds__(256)
     }
 #pragma unroll
     for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (part == 0 && r < rows) delta[r] = acc;
+    if (part == 0 && rp < rows) {
+      stats[rp] = real ? lse[src] * 1.4426950408889634f : INFINITY;
+      stats[rows + rp] = acc;
+    }
   }
 }
 
 struct BwdArgs {
-  const float* lse;
-  const float* delta;
+  const float* stats;   // row statistics written by fa_bwd_preprocess_kernel
+  long long stat_rows;  // B*H*Np: offset of delta after LSE*log2e
   __nv_bfloat16* out0;  // dkdv: dK ; dq: dQ
   __nv_bfloat16* out1;  // dkdv: dV ; dq: unused
   int N;
+  int Np;               // N rounded up to a multiple of 128
   int n_tiles;
   float scale;
   float scale_log2;
@@ -198,7 +211,7 @@ __global__ void __launch_bounds__(320, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(C::bXFull), 1);
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(bar(C::bYFull + s), 32);
+      mbar_init(bar(C::bYFull + s), 1);
       mbar_init(bar(C::bYEmpty + s), 1);
     }
     mbar_init(bar(bSFull), 1);
@@ -229,34 +242,24 @@ __global__ void __launch_bounds__(320, 1)
         tma_load_3d(sb + C::kX0 + r * C::kRegionBytes, &tmK, bar(C::bXFull), r * 64, j * kBlock, bh);
         tma_load_3d(sb + C::kX1 + r * C::kRegionBytes, &tmV, bar(C::bXFull), r * 64, j * kBlock, bh);
       }
-    }
-    int ny = 0;
-    for (int it = 0; it < n_it; ++it) {
-      const int i = i_lo + it;
-      const int s = it % C::kStages;
-      if (!mbar_wait_warp(bar(C::bYEmpty + s), ((it / C::kStages) & 1) ^ 1, abort_flag)) break;
-      float* lse_s = reinterpret_cast<float*>(smem + C::kLse + s * 512);
-      float* del_s = reinterpret_cast<float*>(smem + C::kDelta + s * 512);
-      for (int e = lane; e < kBlock; e += 32) {
-        const int r = i * kBlock + e;
-        const bool v = r < a.N;
-        lse_s[e] = v ? a.lse[(size_t)bh * a.N + r] * kLog2e : INFINITY;
-        del_s[e] = v ? a.delta[(size_t)bh * a.N + r] : 0.f;
-      }
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bar(C::bYFull + s), 2 * C::kTile);
+      int ny = 0;
+      for (int it = 0; it < n_it; ++it) {
+        const int i = i_lo + it;
+        const int s = it % C::kStages;
+        if (!mbar_wait(bar(C::bYEmpty + s), ((it / C::kStages) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::bYFull + s), 2 * C::kTile + 2 * 512);
         for (int r = 0; r < C::kRegions; ++r) {
           tma_load_3d(sb + C::kY0 + s * C::kTile + r * C::kRegionBytes, &tmQ, bar(C::bYFull + s),
                       r * 64, i * kBlock, bh);
           tma_load_3d(sb + C::kY1 + s * C::kTile + r * C::kRegionBytes, &tmdO, bar(C::bYFull + s),
                       r * 64, i * kBlock, bh);
         }
-      } else {
-        mbar_arrive(bar(C::bYFull + s));
+        // LSE*log2e and delta of the 128 rows of query tile i (512 bytes each)
+        const float* st = a.stats + (size_t)bh * a.Np + (size_t)i * kBlock;
+        bulk_load(sb + C::kLse + s * 512, st, 512, bar(C::bYFull + s));
+        bulk_load(sb + C::kDelta + s * 512, st + a.stat_rows, 512, bar(C::bYFull + s));
+        ++ny;
       }
-      ++ny;
-    }
-    if (lane == 0) {
       mbar_wait(bar(C::bXFull), 0, nullptr);
       for (int s = 0; s < C::kStages; ++s) {
         if (ny > s) {
@@ -579,8 +582,9 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const float sl2 = a.scale_log2;
     const bool valid = r < a.N;
-    const float lse2 = valid ? a.lse[(size_t)bh * a.N + r] * kLog2e : INFINITY;
-    const float dl = valid ? a.delta[(size_t)bh * a.N + r] : 0.f;
+    // rows past N carry +inf and 0 in the padded statistics, which zero their P and dS
+    const float lse2 = a.stats[(size_t)bh * a.Np + r];
+    const float dl = a.stats[a.stat_rows + (size_t)bh * a.Np + r];
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int jj = j_lo + it;

@@ -56,9 +56,9 @@ def _lib() -> ctypes.CDLL:
         lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
         lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp,
                                ctypes.c_size_t, vp]
-        lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, I, I, I, I, vp]
-        lib.fa_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp]
-        lib.fa_bwd_dq.argtypes = [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp]
+        lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, vp, I, I, I, I, vp]
+        lib.fa_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp]
+        lib.fa_bwd_dq.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp]
         lib.fa_status_string.argtypes = [I]
         lib.fa_status_string.restype = ctypes.c_char_p
         lib.fa_debug_status.argtypes = [vp]
@@ -131,29 +131,28 @@ def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale=None, causal=False,
                          _stream(stream)), "fa_bwd")
 
 
-def fa_bwd_preprocess(o, do, delta, stream=None) -> None:
+def fa_bwd_preprocess(o, do, lse, workspace, stream=None) -> None:
     B, H, N, d = _shape(o)
-    _check(_lib().fa_bwd_preprocess(_ptr(o), _ptr(do), _ptr(delta), B, H, N, d, _stream(stream)),
-           "fa_bwd_preprocess")
+    _check(_lib().fa_bwd_preprocess(_ptr(o), _ptr(do), _ptr(lse), _ptr(workspace), B, H, N, d,
+                                    _stream(stream)), "fa_bwd_preprocess")
 
 
-def fa_bwd_dkdv(q, k, v, do, lse, delta, dk, dv, scale=None, causal=False, window=(-1, -1),
+def fa_bwd_dkdv(q, k, v, do, workspace, dk, dv, scale=None, causal=False, window=(-1, -1),
                 stream=None) -> None:
     B, H, N, d = _shape(q)
     c, w = _window(causal, window)
     s = default_scale(d) if scale is None else float(scale)
-    _check(_lib().fa_bwd_dkdv(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(lse), _ptr(delta),
-                              _ptr(dk), _ptr(dv), B, H, N, d, s, c, w, _stream(stream)),
-           "fa_bwd_dkdv")
+    _check(_lib().fa_bwd_dkdv(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(workspace), _ptr(dk),
+                              _ptr(dv), B, H, N, d, s, c, w, _stream(stream)), "fa_bwd_dkdv")
 
 
-def fa_bwd_dq(q, k, v, do, lse, delta, dq, scale=None, causal=False, window=(-1, -1),
+def fa_bwd_dq(q, k, v, do, workspace, dq, scale=None, causal=False, window=(-1, -1),
               stream=None) -> None:
     B, H, N, d = _shape(q)
     c, w = _window(causal, window)
     s = default_scale(d) if scale is None else float(scale)
-    _check(_lib().fa_bwd_dq(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(lse), _ptr(delta),
-                            _ptr(dq), B, H, N, d, s, c, w, _stream(stream)), "fa_bwd_dq")
+    _check(_lib().fa_bwd_dq(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(workspace), _ptr(dq),
+                            B, H, N, d, s, c, w, _stream(stream)), "fa_bwd_dq")
 
 
 def fa_status_string(status: int) -> str:

@@ -18,7 +18,7 @@
  *   (B, H, N, d) = (batch, heads, seq_len, head_dim), fully contiguous, row-major
  *   (page "Flash Attention 3.7 核心原理与实战" §3.2 states the problem in this shape).
  *   lse is fp32 (B, H, N): the natural-log log-sum-exp of each row of the scaled,
- *   masked scores. delta is fp32 (B, H, N): rowsum(dout * o).
+ *   masked scores.
  *   Query and key sequences have the same length N.
  * Sizes.  d must be 64 or 128 (else FA_ERR_UNSUPPORTED: the pages list 64 and 128
  *   as the common head sizes and report "no available kernel" otherwise, page
@@ -88,8 +88,10 @@ fa_status_t fa_fwd(const void *q, const void *k, const void *v, void *o, float *
                    fa_window_t window, void *stream);
 
 /*
- * Bytes of device workspace fa_bwd() needs: room for delta, B*H*N fp32 values,
- * rounded up to 256 bytes. Returns 0 for an empty problem or invalid sizes.
+ * Bytes of device workspace fa_bwd() needs: two fp32 arrays of B*H*Np values, where
+ * Np = N rounded up to a multiple of 128 (the row statistics of the backward, see
+ * fa_bwd_preprocess), rounded up to 256 bytes. Returns 0 for an empty problem or
+ * invalid sizes.
  */
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 
@@ -115,19 +117,26 @@ fa_status_t fa_bwd(const void *q, const void *k, const void *v, const void *o,
                    fa_window_t window, void *workspace, size_t workspace_bytes,
                    void *stream);
 
-/* Step 1 of fa_bwd alone: delta (B,H,N) fp32 := rowsum(dout * o), summed in fp32. */
-fa_status_t fa_bwd_preprocess(const void *o, const void *dout, float *delta,
-                              int B, int H, int N, int d, void *stream);
+/*
+ * Step 1 of fa_bwd alone: fills `workspace` (at least fa_bwd_workspace_bytes()) with
+ * the per-row statistics the two passes read, each as B*H rows of Np = N rounded up to
+ * 128 fp32 values (padding rows: +inf and 0):
+ *   workspace[0 .. B*H*Np)          LSE * log2(e)      (from `lse`)
+ *   workspace[B*H*Np .. 2*B*H*Np)   delta = rowsum(dout * o), summed in fp32
+ * The padding lets each 128-row tile of both arrays be fetched with one bulk copy.
+ */
+fa_status_t fa_bwd_preprocess(const void *o, const void *dout, const float *lse,
+                              void *workspace, int B, int H, int N, int d, void *stream);
 
-/* Step 2 of fa_bwd alone: dk, dv from q, k, v, dout, lse and delta (step 1's output). */
+/* Step 2 of fa_bwd alone: dk, dv from q, k, v, dout and the workspace of step 1. */
 fa_status_t fa_bwd_dkdv(const void *q, const void *k, const void *v, const void *dout,
-                        const float *lse, const float *delta, void *dk, void *dv,
+                        const void *workspace, void *dk, void *dv,
                         int B, int H, int N, int d, float scale, int causal,
                         fa_window_t window, void *stream);
 
-/* Step 3 of fa_bwd alone: dq from q, k, v, dout, lse and delta (step 1's output). */
+/* Step 3 of fa_bwd alone: dq from q, k, v, dout and the workspace of step 1. */
 fa_status_t fa_bwd_dq(const void *q, const void *k, const void *v, const void *dout,
-                      const float *lse, const float *delta, void *dq,
+                      const void *workspace, void *dq,
                       int B, int H, int N, int d, float scale, int causal,
                       fa_window_t window, void *stream);
 

@@ -77,8 +77,10 @@ def test_empty_problem_is_a_no_op(lib):
 
 
 def test_workspace_size(lib):
-    assert lib.fa_bwd_workspace_bytes(2, 8, 4096, 64) == 2 * 8 * 4096 * 4
-    assert lib.fa_bwd_workspace_bytes(1, 1, 3, 64) == 256
+    # two fp32 arrays (LSE*log2e and delta) of B*H rows padded to whole 128-row tiles
+    assert lib.fa_bwd_workspace_bytes(2, 8, 4096, 64) == 2 * 2 * 8 * 4096 * 4
+    assert lib.fa_bwd_workspace_bytes(1, 1, 3, 64) == 2 * 128 * 4
+    assert lib.fa_bwd_workspace_bytes(1, 2, 129, 128) == 2 * 2 * 256 * 4
     assert lib.fa_bwd_workspace_bytes(1, 1, 3, 80) == 0
 
 
@@ -96,13 +98,14 @@ def test_bwd_rejects_bad_arguments(lib):
     assert bwd(lib, dq=None) == 1
     assert bwd(lib, ws=None) == 1
     assert bwd(lib, dv=A + 4) == 3
-    assert bwd(lib, ws_bytes=128 * 4 - 1) == 4
+    assert bwd(lib, ws_bytes=2 * 128 * 4 - 1) == 4
     assert bwd(lib, d=256) == 2
     assert bwd(lib, window=(-7, 0)) == 1
-    assert lib.fa_bwd_preprocess(A, None, A, 1, 1, 128, 64, None) == 1
-    assert lib.fa_bwd_dkdv(A, A, A, A, A, A, A, A + 1, 1, 1, 128, 64, 0.1, 0, W(-1, -1),
+    assert lib.fa_bwd_preprocess(A, None, A, A, 1, 1, 128, 64, None) == 1
+    assert lib.fa_bwd_preprocess(A, A, A, A + 8, 1, 1, 128, 64, None) == 3
+    assert lib.fa_bwd_dkdv(A, A, A, A, A, A, A + 1, 1, 1, 128, 64, 0.1, 0, W(-1, -1),
                            None) == 3
-    assert lib.fa_bwd_dq(A, A, A, A, A, A, A, 1, 1, 128, 128, -1.0, 0, W(-1, -1), None) == 1
+    assert lib.fa_bwd_dq(A, A, A, A, A, A, 1, 1, 128, 128, -1.0, 0, W(-1, -1), None) == 1
 
 
 def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
