@@ -212,6 +212,36 @@ size_t workspace_bytes(int B, int H, int N) {
   return (raw + 255) & ~size_t(255);
 }
 
+// ------------------------------------------------------------------------------------
+// Backward without caller workspace (fa_bwd_noalloc): a fixed array in device memory
+// holds the row statistics instead. Every GPU that loads the library keeps this array
+// until the process exits.
+// ------------------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device. The symbol names a
+// host-side stand-in, not device memory, so the address is looked up once per device
+// (with that device current) and cached.
+fa_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return FA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -294,6 +324,26 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
                        stream)) != FA_OK)
     return s;
   return fa_bwd_dq(q, k, v, dout, workspace, dq, B, H, N, d, scale, causal, window, stream);
+}
+
+fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                           const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                           int B, int H, int N, int d, float scale, int causal,
+                           fa_window_t window, void* stream) {
+  bool empty;
+  fa_status_t s = check_problem(B, H, N, d, &empty);
+  if (s != FA_OK || empty) return s;
+  if ((s = check_mask(scale, window)) != FA_OK) return s;
+  if ((s = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv})) != FA_OK) return s;
+  if (workspace_bytes(B, H, N) > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != FA_OK) return s;
+  // The statistics are rewritten in full by the preprocess step, so nothing needs clearing.
+  if ((s = fa_bwd_preprocess(o, dout, lse, scratch, B, H, N, d, stream)) != FA_OK) return s;
+  if ((s = fa_bwd_dkdv(q, k, v, dout, scratch, dk, dv, B, H, N, d, scale, causal, window,
+                       stream)) != FA_OK)
+    return s;
+  return fa_bwd_dq(q, k, v, dout, scratch, dq, B, H, N, d, scale, causal, window, stream);
 }
 
 const char* fa_status_string(fa_status_t status) {

@@ -24,7 +24,7 @@ STATUS_NAMES = {
 
 #: every symbol include/fa.h declares
 EXPORTED = ("fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_dkdv",
-            "fa_bwd_dq", "fa_status_string", "fa_debug_status", "fa_version")
+            "fa_bwd_dq", "fa_bwd_noalloc", "fa_status_string", "fa_debug_status", "fa_version")
 
 
 class FAError(RuntimeError):
@@ -59,12 +59,14 @@ def _lib() -> ctypes.CDLL:
         lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, vp, I, I, I, I, vp]
         lib.fa_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp]
         lib.fa_bwd_dq.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp]
+        lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W,
+                                       vp]
         lib.fa_status_string.argtypes = [I]
         lib.fa_status_string.restype = ctypes.c_char_p
         lib.fa_debug_status.argtypes = [vp]
         lib.fa_version.argtypes = []
         for name in ("fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_dkdv", "fa_bwd_dq",
-                     "fa_debug_status", "fa_version"):
+                     "fa_bwd_noalloc", "fa_debug_status", "fa_version"):
             getattr(lib, name).restype = I
         _LIB = lib
     return _LIB
@@ -153,6 +155,19 @@ def fa_bwd_dq(q, k, v, do, workspace, dq, scale=None, causal=False, window=(-1, 
     s = default_scale(d) if scale is None else float(scale)
     _check(_lib().fa_bwd_dq(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(workspace), _ptr(dq),
                             B, H, N, d, s, c, w, _stream(stream)), "fa_bwd_dq")
+
+
+def fa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, scale=None, causal=False, window=(-1, -1),
+                   stream=None) -> None:
+    """fa_bwd without a workspace argument: for callers that cannot allocate device
+    memory; the library's own fixed device array holds the row statistics."""
+    B, H, N, d = _shape(q)
+    c, w = _window(causal, window)
+    s = default_scale(d) if scale is None else float(scale)
+    _check(_lib().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
+                                 _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, s, c, w,
+                                 _stream(stream)), "fa_bwd_noalloc")
+
 
 
 def fa_status_string(status: int) -> str:

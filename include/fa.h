@@ -140,6 +140,32 @@ fa_status_t fa_bwd_dq(const void *q, const void *k, const void *v, const void *d
                       int B, int H, int N, int d, float scale, int causal,
                       fa_window_t window, void *stream);
 
+/*
+ * Backward pass for callers that cannot allocate device memory. (The pages have no
+ * counterpart of this entry point; it is an interface addition of this library.)
+ *
+ * Some callers may not allocate: an engine that reserves all of its device memory up
+ * front and may not grow it while serving, or a framework plugin whose enqueue step
+ * is not allowed to call cudaMalloc. fa_bwd_noalloc computes exactly what fa_bwd
+ * computes, with the same arguments except the workspace: its row statistics go to a
+ * fixed 8 MiB array in device memory that the library holds on every GPU that loads
+ * it, until the process exits. It calls no cudaMalloc, cudaFree or other allocating
+ * routine.
+ *   Limit: 2 * B * H * Np * 4 bytes must fit in 8 MiB, i.e. B * H * Np <= 1,048,576
+ *   with Np = N rounded up to a multiple of 128; larger problems return
+ *   FA_ERR_WORKSPACE before anything is launched.
+ *   Set-up: the first call on a device (with that device current) looks up the
+ *   array's device address once; make that first call before any stream capture.
+ *   Sharing: every call on a device uses the same array. The statistics are fully
+ *   rewritten by each call, so nothing carries over, but calls whose kernels overlap
+ *   on the GPU (different streams, or several threads) race on the array: serialise
+ *   them.
+ */
+fa_status_t fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                           const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                           int B, int H, int N, int d, float scale, int causal,
+                           fa_window_t window, void *stream);
+
 /* Static, human-readable name of a status code (never NULL). */
 const char *fa_status_string(fa_status_t status);
 
