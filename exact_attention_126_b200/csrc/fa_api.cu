@@ -161,7 +161,7 @@ fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void*
   if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
       !make_map(&mv, v, BH, N, D) || !make_map(&mdo, dout, BH, N, D))
     return FA_ERR_CUDA;
-  using C = fa::BwdCfg<D>;
+  using C = fa::DkdvCfg<D>;
   if (set_smem(fa::fa_bwd_dkdv_kernel<D>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
   fa::BwdArgs a;
   a.stats = static_cast<const float*>(ws);
@@ -188,7 +188,7 @@ fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* d
   if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
       !make_map(&mv, v, BH, N, D) || !make_map(&mdo, dout, BH, N, D))
     return FA_ERR_CUDA;
-  using C = fa::BwdCfg<D>;
+  using C = fa::DqCfg<D>;
   if (set_smem(fa::fa_bwd_dq_kernel<D>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
   fa::BwdArgs a;
   a.stats = static_cast<const float*>(ws);

@@ -96,34 +96,54 @@ struct BwdArgs {
   int right;
 };
 
-// Shared layout of both backward kernels: two stationary tiles (X0, X1) loaded once, a
-// ring of stages holding two streamed tiles (Y0, Y1) each, plus per-stage row statistics.
-template <int D>
-struct BwdCfg {
+// Shared layout of both backward kernels: two stationary tiles (X0, X1) loaded once and
+// two rings of streamed tiles, Y0 (with per-stage row statistics when kStats) and Y1,
+// each with its own full/empty barriers so a tile is released right after its last
+// product. dK/dV: X = K, V; Y0 = Q (+ LSE, delta), Y1 = dO. dQ: X = Q, dO; Y0 = K, Y1 = V.
+template <int D, int S0, int S1, bool kStats>
+struct BwdCfgT {
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   static constexpr int kTile = kBlock * D * 2;
   static constexpr int kRegions = D / 64;
   static constexpr int kRegionBytes = kBlock * 128;
-  static constexpr int kStages = (D == 64) ? 3 : 2;
+  static constexpr int kStages0 = S0;
+  static constexpr int kStages1 = S1;
   static constexpr int kX0 = 0;
   static constexpr int kX1 = kTile;
   static constexpr int kY0 = 2 * kTile;                      // + s * kTile
-  static constexpr int kY1 = kY0 + kStages * kTile;          // + s * kTile
-  static constexpr int kLse = kY1 + kStages * kTile;         // + s * 512 (128 fp32)
-  static constexpr int kDelta = kLse + kStages * 512;        // + s * 512
-  static constexpr int kBar = kDelta + kStages * 512;
-  // barrier slots (meaning per kernel in the comments of each kernel)
+  static constexpr int kY1 = kY0 + S0 * kTile;               // + s * kTile
+  static constexpr int kLse = kY1 + S1 * kTile;              // + s * 512 (128 fp32), ring 0
+  static constexpr int kDelta = kLse + (kStats ? S0 * 512 : 0);
+  static constexpr int kBar = kDelta + (kStats ? S0 * 512 : 0);
   static constexpr int bXFull = 0;
-  static constexpr int bYFull = 1;
-  static constexpr int bYEmpty = bYFull + kStages;
-  static constexpr int bA = bYEmpty + kStages;  // 8 kernel-specific barriers
+  static constexpr int bY0Full = 1;
+  static constexpr int bY0Empty = bY0Full + S0;
+  static constexpr int bY1Full = bY0Empty + S0;
+  static constexpr int bY1Empty = bY1Full + S1;
+  static constexpr int bA = bY1Empty + S1;  // 8 kernel-specific barriers
   static constexpr int bMmaFin = bA + 8;
   static constexpr int kNumBars = bMmaFin + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kSmemBytes = kMisc + 16 + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kThreads = 320;  // 8 softmax warps, MMA warp, producer warp
 };
+
+template <int D>
+using DkdvCfg = BwdCfgT<D, (D == 64) ? 4 : 2, (D == 64) ? 4 : 2, true>;
+template <int D>
+using DqCfg = BwdCfgT<D, (D == 64) ? 5 : 3, (D == 64) ? 4 : 2, false>;
+
+// Waits until every copy a ring's producer issued (n uses of stages 0..S-1) has landed.
+__device__ __forceinline__ void drain_ring(uint32_t full_bar0, int S, int n) {
+  for (int s = 0; s < S; ++s) {
+    if (n > s) {
+      const int last = s + S * ((n - 1 - s) / S);
+      mbar_wait(full_bar0 + 8u * s, (last / S) & 1, nullptr);
+    }
+  }
+}
 
 // Writes this thread's NC fp32 accumulator columns starting at `taddr`, times `mul`, as
 // bf16 to `dst`.
@@ -163,9 +183,8 @@ __device__ __forceinline__ void load_cols64(uint32_t taddr, float (&x)[64]) {
   }
 }
 
-template <int D>
+template <typename C>
 __device__ __forceinline__ void bwd_init_common(uint8_t* smem, uint32_t sb, int warp) {
-  using C = BwdCfg<D>;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMisc);
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
@@ -187,7 +206,7 @@ __global__ void __launch_bounds__(320, 1)
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmdO, const BwdArgs a) {
-  using C = BwdCfg<D>;
+  using C = DkdvCfg<D>;
   constexpr uint32_t tS = 0, tDP = 128, tDK = 256, tDV = 256 + D;
   constexpr int bSFull = C::bA + 0, bDPFull = C::bA + 1, bPFull = C::bA + 2,
                 bDSFull = C::bA + 3, bDVDone = C::bA + 4, bDKDone = C::bA + 5;
@@ -210,9 +229,13 @@ __global__ void __launch_bounds__(320, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::bXFull), 1);
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(bar(C::bYFull + s), 1);
-      mbar_init(bar(C::bYEmpty + s), 1);
+    for (int s = 0; s < C::kStages0; ++s) {
+      mbar_init(bar(C::bY0Full + s), 1);
+      mbar_init(bar(C::bY0Empty + s), 1);
+    }
+    for (int s = 0; s < C::kStages1; ++s) {
+      mbar_init(bar(C::bY1Full + s), 1);
+      mbar_init(bar(C::bY1Empty + s), 1);
     }
     mbar_init(bar(bSFull), 1);
     mbar_init(bar(bDPFull), 1);
@@ -224,7 +247,7 @@ __global__ void __launch_bounds__(320, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  bwd_init_common<D>(smem, sb, warp);
+  bwd_init_common<C>(smem, sb, warp);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -242,31 +265,30 @@ __global__ void __launch_bounds__(320, 1)
         tma_load_3d(sb + C::kX0 + r * C::kRegionBytes, &tmK, bar(C::bXFull), r * 64, j * kBlock, bh);
         tma_load_3d(sb + C::kX1 + r * C::kRegionBytes, &tmV, bar(C::bXFull), r * 64, j * kBlock, bh);
       }
-      int ny = 0;
+      int n0 = 0, n1 = 0;  // loads issued into ring 0 (Q + statistics) and ring 1 (dO)
       for (int it = 0; it < n_it; ++it) {
         const int i = i_lo + it;
-        const int s = it % C::kStages;
-        if (!mbar_wait(bar(C::bYEmpty + s), ((it / C::kStages) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::bYFull + s), 2 * C::kTile + 2 * 512);
-        for (int r = 0; r < C::kRegions; ++r) {
-          tma_load_3d(sb + C::kY0 + s * C::kTile + r * C::kRegionBytes, &tmQ, bar(C::bYFull + s),
+        const int s0 = it % C::kStages0, s1 = it % C::kStages1;
+        if (!mbar_wait(bar(C::bY0Empty + s0), ((it / C::kStages0) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::bY0Full + s0), C::kTile + 2 * 512);
+        for (int r = 0; r < C::kRegions; ++r)
+          tma_load_3d(sb + C::kY0 + s0 * C::kTile + r * C::kRegionBytes, &tmQ, bar(C::bY0Full + s0),
                       r * 64, i * kBlock, bh);
-          tma_load_3d(sb + C::kY1 + s * C::kTile + r * C::kRegionBytes, &tmdO, bar(C::bYFull + s),
-                      r * 64, i * kBlock, bh);
-        }
         // LSE*log2e and delta of the 128 rows of query tile i (512 bytes each)
         const float* st = a.stats + (size_t)bh * a.Np + (size_t)i * kBlock;
-        bulk_load(sb + C::kLse + s * 512, st, 512, bar(C::bYFull + s));
-        bulk_load(sb + C::kDelta + s * 512, st + a.stat_rows, 512, bar(C::bYFull + s));
-        ++ny;
+        bulk_load(sb + C::kLse + s0 * 512, st, 512, bar(C::bY0Full + s0));
+        bulk_load(sb + C::kDelta + s0 * 512, st + a.stat_rows, 512, bar(C::bY0Full + s0));
+        ++n0;
+        if (!mbar_wait(bar(C::bY1Empty + s1), ((it / C::kStages1) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::bY1Full + s1), C::kTile);
+        for (int r = 0; r < C::kRegions; ++r)
+          tma_load_3d(sb + C::kY1 + s1 * C::kTile + r * C::kRegionBytes, &tmdO, bar(C::bY1Full + s1),
+                      r * 64, i * kBlock, bh);
+        ++n1;
       }
       mbar_wait(bar(C::bXFull), 0, nullptr);
-      for (int s = 0; s < C::kStages; ++s) {
-        if (ny > s) {
-          const int last = s + C::kStages * ((ny - 1 - s) / C::kStages);
-          mbar_wait(bar(C::bYFull + s), (last / C::kStages) & 1, nullptr);
-        }
-      }
+      drain_ring(bar(C::bY0Full), C::kStages0, n0);
+      drain_ring(bar(C::bY1Full), C::kStages1, n1);
     }
     __syncwarp();
   } else if (warp == 8) {
@@ -294,48 +316,53 @@ __global__ void __launch_bounds__(320, 1)
         tc_commit(bar(bDPFull));
       };
       bool ok = mbar_wait(bar(C::bXFull), 0, abort_flag) &&
-                mbar_wait(bar(C::bYFull + 0), 0, abort_flag);
+                mbar_wait(bar(C::bY0Full + 0), 0, abort_flag);
       if (ok) {
         tc_fence_after();
         issue_s(0);
-        issue_dp(0);
+        ok = mbar_wait(bar(C::bY1Full + 0), 0, abort_flag);
+        tc_fence_after();
+        if (ok) issue_dp(0);
       }
       for (int it = 0; ok && it < n_it; ++it) {
-        const int s = it % C::kStages;
+        const int s0 = it % C::kStages0, s1 = it % C::kStages1;
         const bool more = it + 1 < n_it;
-        const int s1 = (it + 1) % C::kStages;
-        // dV += P^T dO_i
+        const int t0 = (it + 1) % C::kStages0, t1 = (it + 1) % C::kStages1;
+        // dV += P^T dO_i; dO_i is then free
         if (!mbar_wait(bar(bPFull), it & 1, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBlock / 16; ++kk)
           mma_ts(tmem + tDV, tmem + tS + kk * 8 + (kk >> 2) * 32,
-                 sdesc_sw128(sb + C::kY1 + s * C::kTile + kk * 2048, C::kRegionBytes, 1024), idA,
+                 sdesc_sw128(sb + C::kY1 + s1 * C::kTile + kk * 2048, C::kRegionBytes, 1024), idA,
                  (it > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(C::bY1Empty + s1));
         tc_commit(bar(bDVDone));
         // S^T for the next query tile, once dV has read P^T out of the S^T columns
         if (more) {
-          if (!mbar_wait(bar(C::bYFull + s1), ((it + 1) / C::kStages) & 1, abort_flag) ||
+          if (!mbar_wait(bar(C::bY0Full + t0), ((it + 1) / C::kStages0) & 1, abort_flag) ||
               !mbar_wait(bar(bDVDone), it & 1, abort_flag))
             break;
           tc_fence_after();
-          issue_s(s1);
+          issue_s(t0);
         }
-        // dK += dS^T Q_i
+        // dK += dS^T Q_i; Q_i and its row statistics are then free
         if (!mbar_wait(bar(bDSFull), it & 1, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBlock / 16; ++kk)
           mma_ts(tmem + tDK, tmem + tDP + kk * 8 + (kk >> 2) * 32,
-                 sdesc_sw128(sb + C::kY0 + s * C::kTile + kk * 2048, C::kRegionBytes, 1024), idA,
+                 sdesc_sw128(sb + C::kY0 + s0 * C::kTile + kk * 2048, C::kRegionBytes, 1024), idA,
                  (it > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(C::bYEmpty + s));
+        tc_commit(bar(C::bY0Empty + s0));
         tc_commit(bar(bDKDone));
         // dP^T for the next query tile, once dK has read dS^T out of the dP^T columns
         if (more) {
-          if (!mbar_wait(bar(bDKDone), it & 1, abort_flag)) break;
+          if (!mbar_wait(bar(C::bY1Full + t1), ((it + 1) / C::kStages1) & 1, abort_flag) ||
+              !mbar_wait(bar(bDKDone), it & 1, abort_flag))
+            break;
           tc_fence_after();
-          issue_dp(s1);
+          issue_dp(t1);
         }
       }
       tc_commit(bar(C::bMmaFin));
@@ -352,8 +379,8 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int i = i_lo + it;
-      const int s = it % C::kStages;
-      if (!mbar_wait_warp(bar(C::bYFull + s), (it / C::kStages) & 1, abort_flag) ||
+      const int s = it % C::kStages0;
+      if (!mbar_wait_warp(bar(C::bY0Full + s), (it / C::kStages0) & 1, abort_flag) ||
           !mbar_wait_warp(bar(bSFull), it & 1, abort_flag)) {
         ok = false;
         break;
@@ -436,7 +463,7 @@ __global__ void __launch_bounds__(320, 1)
     fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmdO, const BwdArgs a) {
-  using C = BwdCfg<D>;
+  using C = DqCfg<D>;
   constexpr uint32_t tS0 = 0, tDP = 256, tDQ = 384;
   // S full per buffer, dS full per buffer, dP full, dP free, dQ done
   constexpr int bSFull = C::bA + 0, bDSFull = C::bA + 2, bDPFull = C::bA + 4,
@@ -460,9 +487,13 @@ __global__ void __launch_bounds__(320, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::bXFull), 1);
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(bar(C::bYFull + s), 1);
-      mbar_init(bar(C::bYEmpty + s), 1);
+    for (int s = 0; s < C::kStages0; ++s) {
+      mbar_init(bar(C::bY0Full + s), 1);
+      mbar_init(bar(C::bY0Empty + s), 1);
+    }
+    for (int s = 0; s < C::kStages1; ++s) {
+      mbar_init(bar(C::bY1Full + s), 1);
+      mbar_init(bar(C::bY1Empty + s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(bSFull + b), 1);
@@ -475,7 +506,7 @@ __global__ void __launch_bounds__(320, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  bwd_init_common<D>(smem, sb, warp);
+  bwd_init_common<C>(smem, sb, warp);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -492,27 +523,26 @@ __global__ void __launch_bounds__(320, 1)
         tma_load_3d(sb + C::kX0 + r * C::kRegionBytes, &tmQ, bar(C::bXFull), r * 64, i * kBlock, bh);
         tma_load_3d(sb + C::kX1 + r * C::kRegionBytes, &tmdO, bar(C::bXFull), r * 64, i * kBlock, bh);
       }
-      int ny = 0;
+      int n0 = 0, n1 = 0;  // loads issued into ring 0 (K) and ring 1 (V)
       for (int it = 0; it < n_it; ++it) {
         const int jj = j_lo + it;
-        const int s = it % C::kStages;
-        if (!mbar_wait(bar(C::bYEmpty + s), ((it / C::kStages) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::bYFull + s), 2 * C::kTile);
-        for (int r = 0; r < C::kRegions; ++r) {
-          tma_load_3d(sb + C::kY0 + s * C::kTile + r * C::kRegionBytes, &tmK, bar(C::bYFull + s),
+        const int s0 = it % C::kStages0, s1 = it % C::kStages1;
+        if (!mbar_wait(bar(C::bY0Empty + s0), ((it / C::kStages0) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::bY0Full + s0), C::kTile);
+        for (int r = 0; r < C::kRegions; ++r)
+          tma_load_3d(sb + C::kY0 + s0 * C::kTile + r * C::kRegionBytes, &tmK, bar(C::bY0Full + s0),
                       r * 64, jj * kBlock, bh);
-          tma_load_3d(sb + C::kY1 + s * C::kTile + r * C::kRegionBytes, &tmV, bar(C::bYFull + s),
+        ++n0;
+        if (!mbar_wait(bar(C::bY1Empty + s1), ((it / C::kStages1) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::bY1Full + s1), C::kTile);
+        for (int r = 0; r < C::kRegions; ++r)
+          tma_load_3d(sb + C::kY1 + s1 * C::kTile + r * C::kRegionBytes, &tmV, bar(C::bY1Full + s1),
                       r * 64, jj * kBlock, bh);
-        }
-        ++ny;
+        ++n1;
       }
       mbar_wait(bar(C::bXFull), 0, nullptr);
-      for (int s = 0; s < C::kStages; ++s) {
-        if (ny > s) {
-          const int last = s + C::kStages * ((ny - 1 - s) / C::kStages);
-          mbar_wait(bar(C::bYFull + s), (last / C::kStages) & 1, nullptr);
-        }
-      }
+      drain_ring(bar(C::bY0Full), C::kStages0, n0);
+      drain_ring(bar(C::bY1Full), C::kStages1, n1);
     }
     __syncwarp();
   } else if (warp == 8) {
@@ -529,6 +559,7 @@ __global__ void __launch_bounds__(320, 1)
         }
         tc_commit(bar(bSFull + b));
       };
+      // dP = dO_i V_j^T; V_j is then free
       auto issue_dp = [&](int s) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -537,38 +568,43 @@ __global__ void __launch_bounds__(320, 1)
                  sdesc_sw128(sb + C::kY1 + s * C::kTile + off, 16, 1024), idS, kk > 0);
         }
         tc_commit(bar(bDPFull));
+        tc_commit(bar(C::bY1Empty + s));
       };
       bool ok = mbar_wait(bar(C::bXFull), 0, abort_flag) &&
-                mbar_wait(bar(C::bYFull + 0), 0, abort_flag);
+                mbar_wait(bar(C::bY0Full + 0), 0, abort_flag);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
-        issue_dp(0);
+        ok = mbar_wait(bar(C::bY1Full + 0), 0, abort_flag);
+        tc_fence_after();
+        if (ok) issue_dp(0);
       }
       for (int it = 0; ok && it < n_it; ++it) {
-        const int s = it % C::kStages;
+        const int s0 = it % C::kStages0;
         const int b = it & 1;
         if (it + 1 < n_it) {
-          const int s1 = (it + 1) % C::kStages;
+          const int t0 = (it + 1) % C::kStages0, t1 = (it + 1) % C::kStages1;
           // buffer 1-b held dS(it-1): dQ(it-1) must have read it
-          if (!mbar_wait(bar(C::bYFull + s1), ((it + 1) / C::kStages) & 1, abort_flag)) break;
+          if (!mbar_wait(bar(C::bY0Full + t0), ((it + 1) / C::kStages0) & 1, abort_flag)) break;
           if (it >= 1 && !mbar_wait(bar(bDQDone), (it - 1) & 1, abort_flag)) break;
           tc_fence_after();
-          issue_s(s1, b ^ 1);
+          issue_s(t0, b ^ 1);
           // dP has one buffer: the softmax must have read dP(it)
-          if (!mbar_wait(bar(bDPFree), it & 1, abort_flag)) break;
+          if (!mbar_wait(bar(C::bY1Full + t1), ((it + 1) / C::kStages1) & 1, abort_flag) ||
+              !mbar_wait(bar(bDPFree), it & 1, abort_flag))
+            break;
           tc_fence_after();
-          issue_dp(s1);
+          issue_dp(t1);
         }
-        // dQ += dS K_j
+        // dQ += dS K_j; K_j is then free
         if (!mbar_wait(bar(bDSFull + b), (it >> 1) & 1, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBlock / 16; ++kk)
           mma_ts(tmem + tDQ, tmem + tS0 + 128u * b + kk * 8 + (kk >> 2) * 32,
-                 sdesc_sw128(sb + C::kY0 + s * C::kTile + kk * 2048, C::kRegionBytes, 1024), idA,
+                 sdesc_sw128(sb + C::kY0 + s0 * C::kTile + kk * 2048, C::kRegionBytes, 1024), idA,
                  (it > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(C::bYEmpty + s));
+        tc_commit(bar(C::bY0Empty + s0));
         tc_commit(bar(bDQDone));
       }
       tc_commit(bar(C::bMmaFin));
