@@ -4,6 +4,7 @@
 // tensor ((B*H, N, d) viewed as a 3-D tensor so that the rows past N of a (batch, head)
 // read as zeros instead of the next head's rows), and launches the kernels of
 // fa_fwd.cuh / fa_bwd.cuh on the caller's stream.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -18,6 +19,9 @@
 namespace {
 
 using fa::kBlock;
+
+// Test hook set by fa_debug_set_fault(); 0 in normal operation.
+std::atomic<int> g_fault{0};
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -131,6 +135,7 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   a.scale_log2 = scale * fa::kLog2e;
   a.left = left;
   a.right = right;
+  a.fault = g_fault.load(std::memory_order_relaxed);
   const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
   fa::fa_fwd_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, a);
   return launched();
@@ -368,6 +373,12 @@ fa_status_t fa_debug_status(void* stream) {
     if (cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
     return FA_ERR_TIMEOUT;
   }
+  return FA_OK;
+}
+
+fa_status_t fa_debug_set_fault(int fault) {
+  if (fault < 0 || fault > 1) return FA_ERR_INVALID_ARG;
+  g_fault.store(fault, std::memory_order_relaxed);
   return FA_OK;
 }
 

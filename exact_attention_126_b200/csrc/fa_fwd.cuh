@@ -39,6 +39,7 @@ struct FwdArgs {
   float scale_log2;   // scale * log2(e)
   int left;
   int right;
+  int fault;          // test hook: 1 = the producer never loads V (waits for it run out)
 };
 
 template <int D>
@@ -178,6 +179,7 @@ __global__ void __launch_bounds__(320, 1)
             tma_load_3d(sb + C::kK + s * C::kTile + r * C::kRegionBytes, &tmK, bar(C::bKFull + s),
                         r * 64, j * kBlock, it.bh);
           ++kc;
+          if (a.fault == 1) continue;
           if (!mbar_wait(bar(C::bVEmpty + s), ((vc / C::kStages) & 1) ^ 1, abort_flag)) {
             ok = false;
             break;

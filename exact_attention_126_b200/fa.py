@@ -24,7 +24,8 @@ STATUS_NAMES = {
 
 #: every symbol include/fa.h declares
 EXPORTED = ("fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_dkdv",
-            "fa_bwd_dq", "fa_bwd_noalloc", "fa_status_string", "fa_debug_status", "fa_version")
+            "fa_bwd_dq", "fa_bwd_noalloc", "fa_status_string", "fa_debug_status",
+            "fa_debug_set_fault", "fa_version")
 
 
 class FAError(RuntimeError):
@@ -64,9 +65,10 @@ def _lib() -> ctypes.CDLL:
         lib.fa_status_string.argtypes = [I]
         lib.fa_status_string.restype = ctypes.c_char_p
         lib.fa_debug_status.argtypes = [vp]
+        lib.fa_debug_set_fault.argtypes = [I]
         lib.fa_version.argtypes = []
         for name in ("fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_dkdv", "fa_bwd_dq",
-                     "fa_bwd_noalloc", "fa_debug_status", "fa_version"):
+                     "fa_bwd_noalloc", "fa_debug_status", "fa_debug_set_fault", "fa_version"):
             getattr(lib, name).restype = I
         _LIB = lib
     return _LIB
@@ -176,6 +178,11 @@ def fa_status_string(status: int) -> str:
 
 def fa_debug_status(stream=None) -> int:
     return int(_lib().fa_debug_status(_stream(stream)))
+
+
+def fa_debug_set_fault(fault: int) -> None:
+    """Test hook: 1 makes later fa_fwd launches time out on purpose (see include/fa.h)."""
+    _check(_lib().fa_debug_set_fault(int(fault)), "fa_debug_set_fault")
 
 
 def fa_version() -> int:
