@@ -180,7 +180,10 @@ fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void*
   a.scale_log2 = scale * fa::kLog2e;
   a.left = left;
   a.right = right;
-  dim3 grid(a.n_tiles, BH);
+  a.BH = BH;
+  a.n_items = BH * a.n_tiles;
+  a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
+  const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
   fa::fa_bwd_dkdv_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, a);
   return launched();
 }
@@ -207,7 +210,10 @@ fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* d
   a.scale_log2 = scale * fa::kLog2e;
   a.left = left;
   a.right = right;
-  dim3 grid(a.n_tiles, BH);
+  a.BH = BH;
+  a.n_items = BH * a.n_tiles;
+  a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
+  const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
   fa::fa_bwd_dq_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, a);
   return launched();
 }

@@ -89,39 +89,45 @@ struct BwdArgs {
   __nv_bfloat16* out1;  // dkdv: dV ; dq: unused
   int N;
   int Np;               // N rounded up to a multiple of 128
+  int BH;
   int n_tiles;
+  int n_items;          // BH * n_tiles: one item per (batch*head, stationary tile)
+  int longest_first;    // order items by decreasing length (masked problems)
   float scale;
   float scale_log2;
   int left;
   int right;
 };
 
-// Shared layout of both backward kernels: two stationary tiles (X0, X1) loaded once and
-// two rings of streamed tiles, Y0 (with per-stage row statistics when kStats) and Y1,
-// each with its own full/empty barriers so a tile is released right after its last
-// product. dK/dV: X = K, V; Y0 = Q (+ LSE, delta), Y1 = dO. dQ: X = Q, dO; Y0 = K, Y1 = V.
-template <int D, int S0, int S1, bool kStats>
+// Shared layout of both backward kernels: the stationary tiles X0, X1 of an item (in XB
+// buffers, so that the next item's can load while this one runs) and two rings of
+// streamed tiles, Y0 (with per-stage row statistics when kStats) and Y1, each with its own
+// full/empty barriers so a tile is released right after its last product.
+// dK/dV: X = K, V; Y0 = Q (+ LSE, delta), Y1 = dO. dQ: X = Q, dO; Y0 = K, Y1 = V.
+template <int D, int XB, int S0, int S1, bool kStats>
 struct BwdCfgT {
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   static constexpr int kTile = kBlock * D * 2;
   static constexpr int kRegions = D / 64;
   static constexpr int kRegionBytes = kBlock * 128;
+  static constexpr int kXBufs = XB;
   static constexpr int kStages0 = S0;
   static constexpr int kStages1 = S1;
-  static constexpr int kX0 = 0;
-  static constexpr int kX1 = kTile;
-  static constexpr int kY0 = 2 * kTile;                      // + s * kTile
+  static constexpr int kX0 = 0;                              // + xb * 2 * kTile
+  static constexpr int kX1 = kTile;                          // + xb * 2 * kTile
+  static constexpr int kY0 = XB * 2 * kTile;                 // + s * kTile
   static constexpr int kY1 = kY0 + S0 * kTile;               // + s * kTile
   static constexpr int kLse = kY1 + S1 * kTile;              // + s * 512 (128 fp32), ring 0
   static constexpr int kDelta = kLse + (kStats ? S0 * 512 : 0);
   static constexpr int kBar = kDelta + (kStats ? S0 * 512 : 0);
-  static constexpr int bXFull = 0;
-  static constexpr int bY0Full = 1;
+  static constexpr int bXFull = 0;                           // + xb
+  static constexpr int bXEmpty = 2;                          // + xb
+  static constexpr int bY0Full = 4;
   static constexpr int bY0Empty = bY0Full + S0;
   static constexpr int bY1Full = bY0Empty + S0;
   static constexpr int bY1Empty = bY1Full + S1;
-  static constexpr int bA = bY1Empty + S1;  // 8 kernel-specific barriers
-  static constexpr int bMmaFin = bA + 8;
+  static constexpr int bA = bY1Empty + S1;  // 9 kernel-specific barriers
+  static constexpr int bMmaFin = bA + 9;
   static constexpr int kNumBars = bMmaFin + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kSmemBytes = kMisc + 16 + 1024;
@@ -131,9 +137,9 @@ struct BwdCfgT {
 };
 
 template <int D>
-using DkdvCfg = BwdCfgT<D, (D == 64) ? 4 : 2, (D == 64) ? 4 : 2, true>;
+using DkdvCfg = BwdCfgT<D, (D == 64) ? 2 : 1, (D == 64) ? 4 : 2, (D == 64) ? 4 : 2, true>;
 template <int D>
-using DqCfg = BwdCfgT<D, (D == 64) ? 5 : 3, (D == 64) ? 4 : 2, false>;
+using DqCfg = BwdCfgT<D, (D == 64) ? 2 : 1, (D == 64) ? 5 : 3, (D == 64) ? 4 : 2, false>;
 
 // Waits until every copy a ring's producer issued (n uses of stages 0..S-1) has landed.
 __device__ __forceinline__ void drain_ring(uint32_t full_bar0, int S, int n) {
@@ -183,22 +189,52 @@ __device__ __forceinline__ void load_cols64(uint32_t taddr, float (&x)[64]) {
   }
 }
 
+// Item k of the persistent schedule: the (batch*head, stationary tile). Masked problems
+// go longest first across heads: key tiles in increasing order for dK/dV (key tile 0 is
+// seen by every query tile under a causal mask), query tiles in decreasing order for dQ.
+__device__ __forceinline__ void bwd_item(int k, const BwdArgs& a, bool rising, int& bh,
+                                         int& tile) {
+  if (a.longest_first) {
+    const int step = k / a.BH;
+    tile = rising ? step : a.n_tiles - 1 - step;
+    bh = k % a.BH;
+  } else {
+    bh = k / a.n_tiles;
+    tile = k % a.n_tiles;
+  }
+}
+
 template <typename C>
-__device__ __forceinline__ void bwd_init_common(uint8_t* smem, uint32_t sb, int warp) {
+__device__ __forceinline__ uint32_t bwd_setup(uint8_t* smem, int warp) {
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMisc);
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
     tmem_relinquish();
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  return *tmem_slot;
+}
+
+template <typename C>
+__device__ __forceinline__ void bwd_teardown(uint32_t tmem, int warp) {
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
 }
 
 // ------------------------------------------------------------------------------------
-// dK, dV: one CTA per (batch*head, key tile j). X0 = K_j, X1 = V_j; per stage Y0 = Q_i,
-// Y1 = dO_i and the LSE (log2 units) and delta of the 128 rows of query tile i.
+// dK, dV: persistent CTAs over items (batch*head, key tile j). X0 = K_j, X1 = V_j; per
+// stage Y0 = Q_i with the LSE (log2 units) and delta of its 128 rows, Y1 = dO_i.
 // TMEM: S^T at 0, dP^T at 128, dK at 256, dV at 256 + D. Warpgroup h writes its bf16
 // half of P^T (dS^T) over the first 32 of its own 64 fp32 columns of S^T (dP^T), so the
 // A operand of dV (dK) takes K-steps 0..3 from columns 0..31 and 4..7 from 64..95.
-// MMA order per query tile i:  dV(i), S^T(i+1), dK(i), dP^T(i+1).
+// MMA order per query tile i:  dV(i), S^T(i+1), dK(i), dP^T(i+1). Tile counters (for
+// barrier parities) run over all items of the CTA.
 // ------------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(320, 1)
@@ -209,26 +245,23 @@ __global__ void __launch_bounds__(320, 1)
   using C = DkdvCfg<D>;
   constexpr uint32_t tS = 0, tDP = 128, tDK = 256, tDV = 256 + D;
   constexpr int bSFull = C::bA + 0, bDPFull = C::bA + 1, bPFull = C::bA + 2,
-                bDSFull = C::bA + 3, bDVDone = C::bA + 4, bDKDone = C::bA + 5;
+                bDSFull = C::bA + 3, bDVDone = C::bA + 4, bDKDone = C::bA + 5,
+                bAccFree = C::bA + 6, bAccReady = C::bA + 7;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.y;
-  const int j = blockIdx.x;  // causal: key tile 0 sees the most query tiles
   const Mask mk{a.N, a.left, a.right};
-  int i_lo, i_hi;
-  q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
-  const int n_it = i_hi - i_lo + 1;
-
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
   auto bar = [&](int i) -> uint32_t { return sb + C::kBar + 8u * i; };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(C::bXFull), 1);
+    for (int b = 0; b < C::kXBufs; ++b) {
+      mbar_init(bar(C::bXFull + b), 1);
+      mbar_init(bar(C::bXEmpty + b), 1);
+    }
     for (int s = 0; s < C::kStages0; ++s) {
       mbar_init(bar(C::bY0Full + s), 1);
       mbar_init(bar(C::bY0Empty + s), 1);
@@ -243,15 +276,13 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(bar(bDSFull), 256);
     mbar_init(bar(bDVDone), 1);
     mbar_init(bar(bDKDone), 1);
+    mbar_init(bar(bAccFree), 256);
+    mbar_init(bar(bAccReady), 1);
     mbar_init(bar(C::bMmaFin), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  bwd_init_common<C>(smem, sb, warp);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = bwd_setup<C>(smem, warp);
 
   if (warp == 9) {
     // ------------------------------------------------------------------ producer
@@ -260,33 +291,52 @@ __global__ void __launch_bounds__(320, 1)
       tma_prefetch_map(&tmK);
       tma_prefetch_map(&tmV);
       tma_prefetch_map(&tmdO);
-      mbar_arrive_expect_tx(bar(C::bXFull), 2 * C::kTile);
-      for (int r = 0; r < C::kRegions; ++r) {
-        tma_load_3d(sb + C::kX0 + r * C::kRegionBytes, &tmK, bar(C::bXFull), r * 64, j * kBlock, bh);
-        tma_load_3d(sb + C::kX1 + r * C::kRegionBytes, &tmV, bar(C::bXFull), r * 64, j * kBlock, bh);
+      int items = 0, n0 = 0, n1 = 0;  // items started; loads into ring 0 and ring 1
+      bool ok = true;
+      for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
+        int bh, j;
+        bwd_item(k, a, true, bh, j);
+        int i_lo, i_hi;
+        q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
+        const int xb = items % C::kXBufs, xu = items / C::kXBufs;
+        if (!mbar_wait(bar(C::bXEmpty + xb), (xu & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::bXFull + xb), 2 * C::kTile);
+        for (int r = 0; r < C::kRegions; ++r) {
+          tma_load_3d(sb + C::kX0 + xb * 2 * C::kTile + r * C::kRegionBytes, &tmK,
+                      bar(C::bXFull + xb), r * 64, j * kBlock, bh);
+          tma_load_3d(sb + C::kX1 + xb * 2 * C::kTile + r * C::kRegionBytes, &tmV,
+                      bar(C::bXFull + xb), r * 64, j * kBlock, bh);
+        }
+        ++items;
+        for (int i = i_lo; i <= i_hi; ++i) {
+          const int s0 = n0 % C::kStages0, s1 = n1 % C::kStages1;
+          if (!mbar_wait(bar(C::bY0Empty + s0), ((n0 / C::kStages0) & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(C::bY0Full + s0), C::kTile + 2 * 512);
+          for (int r = 0; r < C::kRegions; ++r)
+            tma_load_3d(sb + C::kY0 + s0 * C::kTile + r * C::kRegionBytes, &tmQ,
+                        bar(C::bY0Full + s0), r * 64, i * kBlock, bh);
+          // LSE*log2e and delta of the 128 rows of query tile i (512 bytes each)
+          const float* st = a.stats + (size_t)bh * a.Np + (size_t)i * kBlock;
+          bulk_load(sb + C::kLse + s0 * 512, st, 512, bar(C::bY0Full + s0));
+          bulk_load(sb + C::kDelta + s0 * 512, st + a.stat_rows, 512, bar(C::bY0Full + s0));
+          ++n0;
+          if (!mbar_wait(bar(C::bY1Empty + s1), ((n1 / C::kStages1) & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(C::bY1Full + s1), C::kTile);
+          for (int r = 0; r < C::kRegions; ++r)
+            tma_load_3d(sb + C::kY1 + s1 * C::kTile + r * C::kRegionBytes, &tmdO,
+                        bar(C::bY1Full + s1), r * 64, i * kBlock, bh);
+          ++n1;
+        }
       }
-      int n0 = 0, n1 = 0;  // loads issued into ring 0 (Q + statistics) and ring 1 (dO)
-      for (int it = 0; it < n_it; ++it) {
-        const int i = i_lo + it;
-        const int s0 = it % C::kStages0, s1 = it % C::kStages1;
-        if (!mbar_wait(bar(C::bY0Empty + s0), ((it / C::kStages0) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::bY0Full + s0), C::kTile + 2 * 512);
-        for (int r = 0; r < C::kRegions; ++r)
-          tma_load_3d(sb + C::kY0 + s0 * C::kTile + r * C::kRegionBytes, &tmQ, bar(C::bY0Full + s0),
-                      r * 64, i * kBlock, bh);
-        // LSE*log2e and delta of the 128 rows of query tile i (512 bytes each)
-        const float* st = a.stats + (size_t)bh * a.Np + (size_t)i * kBlock;
-        bulk_load(sb + C::kLse + s0 * 512, st, 512, bar(C::bY0Full + s0));
-        bulk_load(sb + C::kDelta + s0 * 512, st + a.stat_rows, 512, bar(C::bY0Full + s0));
-        ++n0;
-        if (!mbar_wait(bar(C::bY1Empty + s1), ((it / C::kStages1) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::bY1Full + s1), C::kTile);
-        for (int r = 0; r < C::kRegions; ++r)
-          tma_load_3d(sb + C::kY1 + s1 * C::kTile + r * C::kRegionBytes, &tmdO, bar(C::bY1Full + s1),
-                      r * 64, i * kBlock, bh);
-        ++n1;
-      }
-      mbar_wait(bar(C::bXFull), 0, nullptr);
+      // Drain: every copy issued must have landed before the CTA may exit.
+      for (int n = (items > C::kXBufs ? items - C::kXBufs : 0); n < items; ++n)
+        mbar_wait(bar(C::bXFull + n % C::kXBufs), (n / C::kXBufs) & 1, nullptr);
       drain_ring(bar(C::bY0Full), C::kStages0, n0);
       drain_ring(bar(C::bY1Full), C::kStages1, n1);
     }
@@ -296,74 +346,109 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);
-      // S^T = K_j Q_i^T and dP^T = V_j dO_i^T for the query tile in stage s
-      auto issue_s = [&](int s) {
+      int items = 0, g = 0;  // items and query tiles done (all items)
+      bool ok = true;
+      // S^T = K_j Q_i^T (Q in ring-0 stage s) and dP^T = V_j dO_i^T (dO in ring-1 stage s)
+      auto issue_s = [&](int xb, int s) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-          mma_ss(tmem + tS, sdesc_sw128(sb + C::kX0 + off, 16, 1024),
+          mma_ss(tmem + tS, sdesc_sw128(sb + C::kX0 + xb * 2 * C::kTile + off, 16, 1024),
                  sdesc_sw128(sb + C::kY0 + s * C::kTile + off, 16, 1024), idS, kk > 0);
         }
         tc_commit(bar(bSFull));
       };
-      auto issue_dp = [&](int s) {
+      auto issue_dp = [&](int xb, int s) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-          mma_ss(tmem + tDP, sdesc_sw128(sb + C::kX1 + off, 16, 1024),
+          mma_ss(tmem + tDP, sdesc_sw128(sb + C::kX1 + xb * 2 * C::kTile + off, 16, 1024),
                  sdesc_sw128(sb + C::kY1 + s * C::kTile + off, 16, 1024), idS, kk > 0);
         }
         tc_commit(bar(bDPFull));
       };
-      bool ok = mbar_wait(bar(C::bXFull), 0, abort_flag) &&
-                mbar_wait(bar(C::bY0Full + 0), 0, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0);
-        ok = mbar_wait(bar(C::bY1Full + 0), 0, abort_flag);
-        tc_fence_after();
-        if (ok) issue_dp(0);
-      }
-      for (int it = 0; ok && it < n_it; ++it) {
-        const int s0 = it % C::kStages0, s1 = it % C::kStages1;
-        const bool more = it + 1 < n_it;
-        const int t0 = (it + 1) % C::kStages0, t1 = (it + 1) % C::kStages1;
-        // dV += P^T dO_i; dO_i is then free
-        if (!mbar_wait(bar(bPFull), it & 1, abort_flag)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kBlock / 16; ++kk)
-          mma_ts(tmem + tDV, tmem + tS + kk * 8 + (kk >> 2) * 32,
-                 sdesc_sw128(sb + C::kY1 + s1 * C::kTile + kk * 2048, C::kRegionBytes, 1024), idA,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(C::bY1Empty + s1));
-        tc_commit(bar(bDVDone));
-        // S^T for the next query tile, once dV has read P^T out of the S^T columns
-        if (more) {
-          if (!mbar_wait(bar(C::bY0Full + t0), ((it + 1) / C::kStages0) & 1, abort_flag) ||
-              !mbar_wait(bar(bDVDone), it & 1, abort_flag))
-            break;
-          tc_fence_after();
-          issue_s(t0);
+      for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
+        int bh, j;
+        bwd_item(k, a, true, bh, j);
+        int i_lo, i_hi;
+        q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
+        const int n_it = i_hi - i_lo + 1;
+        const int xb = items % C::kXBufs, xu = items / C::kXBufs;
+        if (!mbar_wait(bar(C::bXFull + xb), xu & 1, abort_flag)) break;
+        // first tile of the item: S^T once dV of the previous tile has read P^T out of the
+        // S^T columns, dP^T once dK has read dS^T out of the dP^T columns
+        if (!mbar_wait(bar(C::bY0Full + g % C::kStages0), (g / C::kStages0) & 1, abort_flag) ||
+            (g > 0 && !mbar_wait(bar(bDVDone), (g - 1) & 1, abort_flag))) {
+          ok = false;
+          break;
         }
-        // dK += dS^T Q_i; Q_i and its row statistics are then free
-        if (!mbar_wait(bar(bDSFull), it & 1, abort_flag)) break;
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kBlock / 16; ++kk)
-          mma_ts(tmem + tDK, tmem + tDP + kk * 8 + (kk >> 2) * 32,
-                 sdesc_sw128(sb + C::kY0 + s0 * C::kTile + kk * 2048, C::kRegionBytes, 1024), idA,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(C::bY0Empty + s0));
-        tc_commit(bar(bDKDone));
-        // dP^T for the next query tile, once dK has read dS^T out of the dP^T columns
-        if (more) {
-          if (!mbar_wait(bar(C::bY1Full + t1), ((it + 1) / C::kStages1) & 1, abort_flag) ||
-              !mbar_wait(bar(bDKDone), it & 1, abort_flag))
-            break;
-          tc_fence_after();
-          issue_dp(t1);
+        issue_s(xb, g % C::kStages0);
+        if (!mbar_wait(bar(C::bY1Full + g % C::kStages1), (g / C::kStages1) & 1, abort_flag) ||
+            (g > 0 && !mbar_wait(bar(bDKDone), (g - 1) & 1, abort_flag))) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        issue_dp(xb, g % C::kStages1);
+        if (n_it == 1) tc_commit(bar(C::bXEmpty + xb));  // K_j, V_j read for the last time
+        for (int it = 0; it < n_it; ++it) {
+          const int t = g + it;
+          const int s0 = t % C::kStages0, s1 = t % C::kStages1;
+          const bool more = it + 1 < n_it;
+          // dV += P^T dO_i; dO_i is then free. The item's first product overwrites dV,
+          // which the previous item's epilogue must have read.
+          if (!mbar_wait(bar(bPFull), t & 1, abort_flag) ||
+              (it == 0 && items > 0 && !mbar_wait(bar(bAccFree), (items - 1) & 1, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kBlock / 16; ++kk)
+            mma_ts(tmem + tDV, tmem + tS + kk * 8 + (kk >> 2) * 32,
+                   sdesc_sw128(sb + C::kY1 + s1 * C::kTile + kk * 2048, C::kRegionBytes, 1024),
+                   idA, (it > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bar(C::bY1Empty + s1));
+          tc_commit(bar(bDVDone));
+          if (more) {
+            const int u0 = (t + 1) % C::kStages0;
+            if (!mbar_wait(bar(C::bY0Full + u0), ((t + 1) / C::kStages0) & 1, abort_flag) ||
+                !mbar_wait(bar(bDVDone), t & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(xb, u0);
+          }
+          // dK += dS^T Q_i; Q_i and its row statistics are then free
+          if (!mbar_wait(bar(bDSFull), t & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kBlock / 16; ++kk)
+            mma_ts(tmem + tDK, tmem + tDP + kk * 8 + (kk >> 2) * 32,
+                   sdesc_sw128(sb + C::kY0 + s0 * C::kTile + kk * 2048, C::kRegionBytes, 1024),
+                   idA, (it > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bar(C::bY0Empty + s0));
+          tc_commit(bar(bDKDone));
+          if (!more) tc_commit(bar(bAccReady));  // dK, dV of the item are complete
+          if (more) {
+            const int u1 = (t + 1) % C::kStages1;
+            if (!mbar_wait(bar(C::bY1Full + u1), ((t + 1) / C::kStages1) & 1, abort_flag) ||
+                !mbar_wait(bar(bDKDone), t & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_dp(xb, u1);
+            if (it + 2 == n_it) tc_commit(bar(C::bXEmpty + xb));  // last read of K_j, V_j
+          }
+        }
+        g += n_it;
+        ++items;
       }
       tc_commit(bar(C::bMmaFin));
       mbar_wait(bar(C::bMmaFin), 0, nullptr);
@@ -371,92 +456,102 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ warps 0..7
-    const int h = warp >> 2;          // query columns 64h .. 64h+63 of the tile
-    const int t = threadIdx.x & 127;  // key row in the tile == TMEM lane
-    const int c = j * kBlock + t;     // this thread's key
+    const int h = warp >> 2;          // query columns 64h .. 64h+63 of each query tile
+    const int t_row = threadIdx.x & 127;  // key row in the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const float sl2 = a.scale_log2;
+    int g = 0, items = 0;
     bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      const int i = i_lo + it;
-      const int s = it % C::kStages0;
-      if (!mbar_wait_warp(bar(C::bY0Full + s), (it / C::kStages0) & 1, abort_flag) ||
-          !mbar_wait_warp(bar(bSFull), it & 1, abort_flag)) {
+    for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
+      int bh, j;
+      bwd_item(k, a, true, bh, j);
+      int i_lo, i_hi;
+      q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
+      const int n_it = i_hi - i_lo + 1;
+      const int c = j * kBlock + t_row;  // this thread's key
+      for (int it = 0; it < n_it; ++it) {
+        const int i = i_lo + it;
+        const int t = g + it;
+        const int s = t % C::kStages0;
+        if (!mbar_wait_warp(bar(C::bY0Full + s), (t / C::kStages0) & 1, abort_flag) ||
+            !mbar_wait_warp(bar(bSFull), t & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float* lse_s = reinterpret_cast<const float*>(smem + C::kLse + s * 512) + 64 * h;
+        const float* del_s = reinterpret_cast<const float*>(smem + C::kDelta + s * 512) + 64 * h;
+        float p[64];
+        load_cols64(tmem + lane_base + tS + 64 * h, p);
+#pragma unroll
+        for (int r = 0; r < 64; r += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse_s + r);
+          p[r] = ex2(fmaf(p[r], sl2, -l4.x));
+          p[r + 1] = ex2(fmaf(p[r + 1], sl2, -l4.y));
+          p[r + 2] = ex2(fmaf(p[r + 2], sl2, -l4.z));
+          p[r + 3] = ex2(fmaf(p[r + 3], sl2, -l4.w));
+        }
+        if (!tile_all_visible(i, j, mk)) {
+#pragma unroll
+          for (int r = 0; r < 64; ++r)
+            if (!is_visible(i * kBlock + 64 * h + r, c, mk)) p[r] = 0.f;
+        }
+        {
+          uint32_t pk[32];
+#pragma unroll
+          for (int r = 0; r < 32; ++r) pk[r] = pack_bf16x2(p[2 * r], p[2 * r + 1]);
+          tmem_st32(tmem + lane_base + tS + 64 * h, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(bPFull));
+        if (!mbar_wait_warp(bar(bDPFull), t & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float dp[64];
+        load_cols64(tmem + lane_base + tDP + 64 * h, dp);
+        uint32_t w[32];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int r0 = 2 * e;
+          const float4 d4 = *reinterpret_cast<const float4*>(del_s + r0);
+          w[e] = pack_bf16x2(p[r0] * (dp[r0] - d4.x), p[r0 + 1] * (dp[r0 + 1] - d4.y));
+          w[e + 1] = pack_bf16x2(p[r0 + 2] * (dp[r0 + 2] - d4.z), p[r0 + 3] * (dp[r0 + 3] - d4.w));
+        }
+        // bf16 dS^T goes over the first half of this warpgroup's own fp32 dP^T columns
+        tmem_st32(tmem + lane_base + tDP + 64 * h, w);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(bDSFull));
+      }
+      if (!ok) break;
+      g += n_it;
+      // once per item, after its last dK (which follows its last dV)
+      if (!mbar_wait_warp(bar(bAccReady), items & 1, abort_flag)) {
         ok = false;
         break;
       }
-      tc_fence_after();
-      const float* lse_s = reinterpret_cast<const float*>(smem + C::kLse + s * 512) + 64 * h;
-      const float* del_s = reinterpret_cast<const float*>(smem + C::kDelta + s * 512) + 64 * h;
-      float p[64];
-      load_cols64(tmem + lane_base + tS + 64 * h, p);
-#pragma unroll
-      for (int r = 0; r < 64; r += 4) {
-        const float4 l4 = *reinterpret_cast<const float4*>(lse_s + r);
-        p[r] = ex2(fmaf(p[r], sl2, -l4.x));
-        p[r + 1] = ex2(fmaf(p[r + 1], sl2, -l4.y));
-        p[r + 2] = ex2(fmaf(p[r + 2], sl2, -l4.z));
-        p[r + 3] = ex2(fmaf(p[r + 3], sl2, -l4.w));
-      }
-      if (!tile_all_visible(i, j, mk)) {
-#pragma unroll
-        for (int r = 0; r < 64; ++r)
-          if (!is_visible(i * kBlock + 64 * h + r, c, mk)) p[r] = 0.f;
-      }
-      {
-        uint32_t pk[32];
-#pragma unroll
-        for (int r = 0; r < 32; ++r) pk[r] = pack_bf16x2(p[2 * r], p[2 * r + 1]);
-        tmem_st32(tmem + lane_base + tS + 64 * h, pk);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(bPFull));
-      if (!mbar_wait_warp(bar(bDPFull), it & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float dp[64];
-      load_cols64(tmem + lane_base + tDP + 64 * h, dp);
-      uint32_t w[32];
-#pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        const int r0 = 2 * e;
-        const float4 d4 = *reinterpret_cast<const float4*>(del_s + r0);
-        w[e] = pack_bf16x2(p[r0] * (dp[r0] - d4.x), p[r0 + 1] * (dp[r0 + 1] - d4.y));
-        w[e + 1] = pack_bf16x2(p[r0 + 2] * (dp[r0 + 2] - d4.z), p[r0 + 3] * (dp[r0 + 3] - d4.w));
-      }
-      // bf16 dS^T goes over the first half of this warpgroup's own fp32 dP^T columns
-      tmem_st32(tmem + lane_base + tDP + 64 * h, w);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(bDSFull));
-    }
-    // dK(last) was committed after dV(last): its completion covers both accumulators
-    if (ok) ok = mbar_wait_warp(bar(bDKDone), (n_it - 1) & 1, abort_flag);
-    if (ok) {
+      ++items;
       tc_fence_after();
       const bool valid = c < a.N;
       const size_t off = ((size_t)bh * a.N + (valid ? c : 0)) * D + (D / 2) * h;
       store_acc_cols<D / 2>(tmem + lane_base + tDV + (D / 2) * h, 1.f, a.out1 + off, valid);
       store_acc_cols<D / 2>(tmem + lane_base + tDK + (D / 2) * h, a.scale, a.out0 + off, valid);
+      // dK, dV have been read: the next item's first products may overwrite them
+      tc_fence_before();
+      mbar_arrive(bar(bAccFree));
     }
   }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
-  }
+  bwd_teardown<C>(tmem, warp);
 }
 
 // ------------------------------------------------------------------------------------
-// dQ: one CTA per (batch*head, query tile i). X0 = Q_i, X1 = dO_i; per stage Y0 = K_j,
-// Y1 = V_j. TMEM: S in two buffers at 0 and 128 (bf16 dS goes over S, each warpgroup
-// over the first half of its own columns), dP at 256, dQ at 384. MMA order per key
-// tile j: S(j+1), dP(j+1), dQ(j).
+// dQ: persistent CTAs over items (batch*head, query tile i). X0 = Q_i, X1 = dO_i; per
+// stage Y0 = K_j, Y1 = V_j. TMEM: S in two buffers at 0 and 128 (bf16 dS goes over S,
+// each warpgroup over the first half of its own columns), dP at 256, dQ at 384. MMA
+// order per key tile j: S(j+1), dP(j+1), dQ(j). Tile counters run over all items.
 // ------------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(320, 1)
@@ -465,28 +560,25 @@ __global__ void __launch_bounds__(320, 1)
                      const __grid_constant__ CUtensorMap tmdO, const BwdArgs a) {
   using C = DqCfg<D>;
   constexpr uint32_t tS0 = 0, tDP = 256, tDQ = 384;
-  // S full per buffer, dS full per buffer, dP full, dP free, dQ done
+  // S full per buffer, dS full per buffer, dP full, dP free, dQ done, dQ read
   constexpr int bSFull = C::bA + 0, bDSFull = C::bA + 2, bDPFull = C::bA + 4,
-                bDPFree = C::bA + 5, bDQDone = C::bA + 6;
+                bDPFree = C::bA + 5, bDQDone = C::bA + 6, bAccFree = C::bA + 7,
+                bAccReady = C::bA + 8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.y;
-  const int i = a.n_tiles - 1 - (int)blockIdx.x;  // longest causal rows first
   const Mask mk{a.N, a.left, a.right};
-  int j_lo, j_hi;
-  kv_tiles_for_q_tile(i, mk, j_lo, j_hi);
-  const int n_it = j_hi - j_lo + 1;
-
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
   auto bar = [&](int k) -> uint32_t { return sb + C::kBar + 8u * k; };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(C::bXFull), 1);
+    for (int b = 0; b < C::kXBufs; ++b) {
+      mbar_init(bar(C::bXFull + b), 1);
+      mbar_init(bar(C::bXEmpty + b), 1);
+    }
     for (int s = 0; s < C::kStages0; ++s) {
       mbar_init(bar(C::bY0Full + s), 1);
       mbar_init(bar(C::bY0Empty + s), 1);
@@ -502,15 +594,13 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(bar(bDPFull), 1);
     mbar_init(bar(bDPFree), 256);
     mbar_init(bar(bDQDone), 1);
+    mbar_init(bar(bAccFree), 256);
+    mbar_init(bar(bAccReady), 1);
     mbar_init(bar(C::bMmaFin), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  bwd_init_common<C>(smem, sb, warp);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = bwd_setup<C>(smem, warp);
 
   if (warp == 9) {
     if (lane == 0) {
@@ -518,29 +608,47 @@ __global__ void __launch_bounds__(320, 1)
       tma_prefetch_map(&tmK);
       tma_prefetch_map(&tmV);
       tma_prefetch_map(&tmdO);
-      mbar_arrive_expect_tx(bar(C::bXFull), 2 * C::kTile);
-      for (int r = 0; r < C::kRegions; ++r) {
-        tma_load_3d(sb + C::kX0 + r * C::kRegionBytes, &tmQ, bar(C::bXFull), r * 64, i * kBlock, bh);
-        tma_load_3d(sb + C::kX1 + r * C::kRegionBytes, &tmdO, bar(C::bXFull), r * 64, i * kBlock, bh);
+      int items = 0, n0 = 0, n1 = 0;
+      bool ok = true;
+      for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
+        int bh, i;
+        bwd_item(k, a, false, bh, i);
+        int j_lo, j_hi;
+        kv_tiles_for_q_tile(i, mk, j_lo, j_hi);
+        const int xb = items % C::kXBufs, xu = items / C::kXBufs;
+        if (!mbar_wait(bar(C::bXEmpty + xb), (xu & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::bXFull + xb), 2 * C::kTile);
+        for (int r = 0; r < C::kRegions; ++r) {
+          tma_load_3d(sb + C::kX0 + xb * 2 * C::kTile + r * C::kRegionBytes, &tmQ,
+                      bar(C::bXFull + xb), r * 64, i * kBlock, bh);
+          tma_load_3d(sb + C::kX1 + xb * 2 * C::kTile + r * C::kRegionBytes, &tmdO,
+                      bar(C::bXFull + xb), r * 64, i * kBlock, bh);
+        }
+        ++items;
+        for (int jj = j_lo; jj <= j_hi; ++jj) {
+          const int s0 = n0 % C::kStages0, s1 = n1 % C::kStages1;
+          if (!mbar_wait(bar(C::bY0Empty + s0), ((n0 / C::kStages0) & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(C::bY0Full + s0), C::kTile);
+          for (int r = 0; r < C::kRegions; ++r)
+            tma_load_3d(sb + C::kY0 + s0 * C::kTile + r * C::kRegionBytes, &tmK,
+                        bar(C::bY0Full + s0), r * 64, jj * kBlock, bh);
+          ++n0;
+          if (!mbar_wait(bar(C::bY1Empty + s1), ((n1 / C::kStages1) & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(C::bY1Full + s1), C::kTile);
+          for (int r = 0; r < C::kRegions; ++r)
+            tma_load_3d(sb + C::kY1 + s1 * C::kTile + r * C::kRegionBytes, &tmV,
+                        bar(C::bY1Full + s1), r * 64, jj * kBlock, bh);
+          ++n1;
+        }
       }
-      int n0 = 0, n1 = 0;  // loads issued into ring 0 (K) and ring 1 (V)
-      for (int it = 0; it < n_it; ++it) {
-        const int jj = j_lo + it;
-        const int s0 = it % C::kStages0, s1 = it % C::kStages1;
-        if (!mbar_wait(bar(C::bY0Empty + s0), ((it / C::kStages0) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::bY0Full + s0), C::kTile);
-        for (int r = 0; r < C::kRegions; ++r)
-          tma_load_3d(sb + C::kY0 + s0 * C::kTile + r * C::kRegionBytes, &tmK, bar(C::bY0Full + s0),
-                      r * 64, jj * kBlock, bh);
-        ++n0;
-        if (!mbar_wait(bar(C::bY1Empty + s1), ((it / C::kStages1) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::bY1Full + s1), C::kTile);
-        for (int r = 0; r < C::kRegions; ++r)
-          tma_load_3d(sb + C::kY1 + s1 * C::kTile + r * C::kRegionBytes, &tmV, bar(C::bY1Full + s1),
-                      r * 64, jj * kBlock, bh);
-        ++n1;
-      }
-      mbar_wait(bar(C::bXFull), 0, nullptr);
+      for (int n = (items > C::kXBufs ? items - C::kXBufs : 0); n < items; ++n)
+        mbar_wait(bar(C::bXFull + n % C::kXBufs), (n / C::kXBufs) & 1, nullptr);
       drain_ring(bar(C::bY0Full), C::kStages0, n0);
       drain_ring(bar(C::bY1Full), C::kStages1, n1);
     }
@@ -549,63 +657,84 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);
-      // S = Q_i K_j^T into buffer b, dP = dO_i V_j^T, for the key tile in stage s
-      auto issue_s = [&](int s, int b) {
+      int items = 0, g = 0;
+      bool ok = true;
+      // S(t) = Q_i K_j^T into buffer t & 1 (K in ring-0 stage t % S0); its buffer held
+      // dS(t-2), which dQ(t-2) must have read
+      auto issue_s = [&](int xb, int t) -> bool {
+        const int s = t % C::kStages0;
+        if (!mbar_wait(bar(C::bY0Full + s), (t / C::kStages0) & 1, abort_flag)) return false;
+        if (t >= 2 && !mbar_wait(bar(bDQDone), (t - 2) & 1, abort_flag)) return false;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-          mma_ss(tmem + tS0 + 128u * b, sdesc_sw128(sb + C::kX0 + off, 16, 1024),
+          mma_ss(tmem + tS0 + 128u * (t & 1),
+                 sdesc_sw128(sb + C::kX0 + xb * 2 * C::kTile + off, 16, 1024),
                  sdesc_sw128(sb + C::kY0 + s * C::kTile + off, 16, 1024), idS, kk > 0);
         }
-        tc_commit(bar(bSFull + b));
+        tc_commit(bar(bSFull + (t & 1)));
+        return true;
       };
-      // dP = dO_i V_j^T; V_j is then free
-      auto issue_dp = [&](int s) {
+      // dP(t) = dO_i V_j^T (V in ring-1 stage t % S1), once the softmax read dP(t-1); V_j
+      // is then free
+      auto issue_dp = [&](int xb, int t) -> bool {
+        const int s = t % C::kStages1;
+        if (!mbar_wait(bar(C::bY1Full + s), (t / C::kStages1) & 1, abort_flag)) return false;
+        if (t >= 1 && !mbar_wait(bar(bDPFree), (t - 1) & 1, abort_flag)) return false;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-          mma_ss(tmem + tDP, sdesc_sw128(sb + C::kX1 + off, 16, 1024),
+          mma_ss(tmem + tDP, sdesc_sw128(sb + C::kX1 + xb * 2 * C::kTile + off, 16, 1024),
                  sdesc_sw128(sb + C::kY1 + s * C::kTile + off, 16, 1024), idS, kk > 0);
         }
         tc_commit(bar(bDPFull));
         tc_commit(bar(C::bY1Empty + s));
+        return true;
       };
-      bool ok = mbar_wait(bar(C::bXFull), 0, abort_flag) &&
-                mbar_wait(bar(C::bY0Full + 0), 0, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        ok = mbar_wait(bar(C::bY1Full + 0), 0, abort_flag);
-        tc_fence_after();
-        if (ok) issue_dp(0);
-      }
-      for (int it = 0; ok && it < n_it; ++it) {
-        const int s0 = it % C::kStages0;
-        const int b = it & 1;
-        if (it + 1 < n_it) {
-          const int t0 = (it + 1) % C::kStages0, t1 = (it + 1) % C::kStages1;
-          // buffer 1-b held dS(it-1): dQ(it-1) must have read it
-          if (!mbar_wait(bar(C::bY0Full + t0), ((it + 1) / C::kStages0) & 1, abort_flag)) break;
-          if (it >= 1 && !mbar_wait(bar(bDQDone), (it - 1) & 1, abort_flag)) break;
-          tc_fence_after();
-          issue_s(t0, b ^ 1);
-          // dP has one buffer: the softmax must have read dP(it)
-          if (!mbar_wait(bar(C::bY1Full + t1), ((it + 1) / C::kStages1) & 1, abort_flag) ||
-              !mbar_wait(bar(bDPFree), it & 1, abort_flag))
-            break;
-          tc_fence_after();
-          issue_dp(t1);
+      for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
+        int bh, i;
+        bwd_item(k, a, false, bh, i);
+        int j_lo, j_hi;
+        kv_tiles_for_q_tile(i, mk, j_lo, j_hi);
+        const int n_it = j_hi - j_lo + 1;
+        const int xb = items % C::kXBufs, xu = items / C::kXBufs;
+        if (!mbar_wait(bar(C::bXFull + xb), xu & 1, abort_flag)) break;
+        if (!issue_s(xb, g) || !issue_dp(xb, g)) {
+          ok = false;
+          break;
         }
-        // dQ += dS K_j; K_j is then free
-        if (!mbar_wait(bar(bDSFull + b), (it >> 1) & 1, abort_flag)) break;
-        tc_fence_after();
+        if (n_it == 1) tc_commit(bar(C::bXEmpty + xb));  // Q_i, dO_i read for the last time
+        for (int it = 0; it < n_it; ++it) {
+          const int t = g + it;
+          if (it + 1 < n_it) {
+            if (!issue_s(xb, t + 1) || !issue_dp(xb, t + 1)) {
+              ok = false;
+              break;
+            }
+            if (it + 2 == n_it) tc_commit(bar(C::bXEmpty + xb));
+          }
+          // dQ += dS K_j; K_j is then free. The item's first product overwrites dQ, which
+          // the previous item's epilogue must have read.
+          if (!mbar_wait(bar(bDSFull + (t & 1)), (t >> 1) & 1, abort_flag) ||
+              (it == 0 && items > 0 && !mbar_wait(bar(bAccFree), (items - 1) & 1, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kBlock / 16; ++kk)
-          mma_ts(tmem + tDQ, tmem + tS0 + 128u * b + kk * 8 + (kk >> 2) * 32,
-                 sdesc_sw128(sb + C::kY0 + s0 * C::kTile + kk * 2048, C::kRegionBytes, 1024), idA,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(C::bY0Empty + s0));
-        tc_commit(bar(bDQDone));
+          for (int kk = 0; kk < kBlock / 16; ++kk)
+            mma_ts(tmem + tDQ, tmem + tS0 + 128u * (t & 1) + kk * 8 + (kk >> 2) * 32,
+                   sdesc_sw128(sb + C::kY0 + (t % C::kStages0) * C::kTile + kk * 2048,
+                               C::kRegionBytes, 1024),
+                   idA, (it > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bar(C::bY0Empty + t % C::kStages0));
+          tc_commit(bar(bDQDone));
+          if (it + 1 == n_it) tc_commit(bar(bAccReady));  // dQ of the item is complete
+        }
+        g += n_it;
+        ++items;
       }
       tc_commit(bar(C::bMmaFin));
       mbar_wait(bar(C::bMmaFin), 0, nullptr);
@@ -613,65 +742,76 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else {
     const int h = warp >> 2;          // key columns 64h .. 64h+63 of each key tile
-    const int t = threadIdx.x & 127;
-    const int r = i * kBlock + t;     // this thread's query row
+    const int t_row = threadIdx.x & 127;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const float sl2 = a.scale_log2;
-    const bool valid = r < a.N;
-    // rows past N carry +inf and 0 in the padded statistics, which zero their P and dS
-    const float lse2 = a.stats[(size_t)bh * a.Np + r];
-    const float dl = a.stats[a.stat_rows + (size_t)bh * a.Np + r];
+    int g = 0, items = 0;
     bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      const int jj = j_lo + it;
-      const int b = it & 1;
-      if (!mbar_wait_warp(bar(bSFull + b), (it >> 1) & 1, abort_flag)) {
+    for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
+      int bh, i;
+      bwd_item(k, a, false, bh, i);
+      int j_lo, j_hi;
+      kv_tiles_for_q_tile(i, mk, j_lo, j_hi);
+      const int n_it = j_hi - j_lo + 1;
+      const int r = i * kBlock + t_row;  // this thread's query row
+      const bool valid = r < a.N;
+      // rows past N carry +inf and 0 in the padded statistics, which zero their P and dS
+      const float lse2 = a.stats[(size_t)bh * a.Np + r];
+      const float dl = a.stats[a.stat_rows + (size_t)bh * a.Np + r];
+      for (int it = 0; it < n_it; ++it) {
+        const int jj = j_lo + it;
+        const int t = g + it;
+        const int b = t & 1;
+        if (!mbar_wait_warp(bar(bSFull + b), (t >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float p[64];
+        load_cols64(tmem + lane_base + tS0 + 128u * b + 64 * h, p);
+#pragma unroll
+        for (int c = 0; c < 64; ++c) p[c] = ex2(fmaf(p[c], sl2, -lse2));
+        if (!tile_all_visible(i, jj, mk)) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (!is_visible(r, jj * kBlock + 64 * h + c, mk)) p[c] = 0.f;
+        }
+        if (!mbar_wait_warp(bar(bDPFull), t & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float dp[64];
+        load_cols64(tmem + lane_base + tDP + 64 * h, dp);
+        tc_fence_before();
+        mbar_arrive(bar(bDPFree));
+        uint32_t w[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          w[e] = pack_bf16x2(p[2 * e] * (dp[2 * e] - dl), p[2 * e + 1] * (dp[2 * e + 1] - dl));
+        // bf16 dS goes over the first half of this warpgroup's own fp32 S columns
+        tmem_st32(tmem + lane_base + tS0 + 128u * b + 64 * h, w);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(bDSFull + b));
+      }
+      if (!ok) break;
+      g += n_it;
+      // once per item, after its last dQ product
+      if (!mbar_wait_warp(bar(bAccReady), items & 1, abort_flag)) {
         ok = false;
         break;
       }
-      tc_fence_after();
-      float p[64];
-      load_cols64(tmem + lane_base + tS0 + 128u * b + 64 * h, p);
-#pragma unroll
-      for (int c = 0; c < 64; ++c) p[c] = ex2(fmaf(p[c], sl2, -lse2));
-      if (!tile_all_visible(i, jj, mk)) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (!is_visible(r, jj * kBlock + 64 * h + c, mk)) p[c] = 0.f;
-      }
-      if (!mbar_wait_warp(bar(bDPFull), it & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float dp[64];
-      load_cols64(tmem + lane_base + tDP + 64 * h, dp);
-      tc_fence_before();
-      mbar_arrive(bar(bDPFree));
-      uint32_t w[32];
-#pragma unroll
-      for (int e = 0; e < 32; ++e)
-        w[e] = pack_bf16x2(p[2 * e] * (dp[2 * e] - dl), p[2 * e + 1] * (dp[2 * e + 1] - dl));
-      // bf16 dS goes over the first half of this warpgroup's own fp32 S columns
-      tmem_st32(tmem + lane_base + tS0 + 128u * b + 64 * h, w);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(bDSFull + b));
-    }
-    if (ok) ok = mbar_wait_warp(bar(bDQDone), (n_it - 1) & 1, abort_flag);
-    if (ok) {
+      ++items;
       tc_fence_after();
       const size_t off = ((size_t)bh * a.N + (valid ? r : 0)) * D + (D / 2) * h;
       store_acc_cols<D / 2>(tmem + lane_base + tDQ + (D / 2) * h, a.scale, a.out0 + off, valid);
+      // dQ has been read: the next item's first product may overwrite it
+      tc_fence_before();
+      mbar_arrive(bar(bAccFree));
     }
   }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
-  }
+  bwd_teardown<C>(tmem, warp);
 }
 
 }  // namespace fa

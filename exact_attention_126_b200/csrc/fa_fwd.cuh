@@ -50,15 +50,15 @@ struct FwdCfg {
   static constexpr int kRegionBytes = kBlock * 128;
   static constexpr int kStages = (D == 64) ? 4 : 2;
   // shared memory map (offsets from a 1024-aligned base)
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTile;               // + s * kTile
+  static constexpr int kQ = 0;                        // + (item & 1) * kTile
+  static constexpr int kK = kQ + 2 * kTile;           // + s * kTile
   static constexpr int kV = kK + kStages * kTile;     // + s * kTile
   static constexpr int kRed = kV + kStages * kTile;   // [2 slots][2 halves][128 rows] fp32
   static constexpr int kBar = kRed + 2 * 2 * kBlock * 4;
   // barrier slots
-  static constexpr int bQFull = 0;
-  static constexpr int bQEmpty = 1;
-  static constexpr int bKFull = 2;
+  static constexpr int bQFull = 0;                  // + (item & 1)
+  static constexpr int bQEmpty = 2;                 // + (item & 1)
+  static constexpr int bKFull = 4;
   static constexpr int bKEmpty = bKFull + kStages;
   static constexpr int bVFull = bKEmpty + kStages;
   static constexpr int bVEmpty = bVFull + kStages;
@@ -122,8 +122,10 @@ __global__ void __launch_bounds__(320, 1)
   auto bar = [&](int i) -> uint32_t { return sb + C::kBar + 8u * i; };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(C::bQFull), 1);
-    mbar_init(bar(C::bQEmpty), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(C::bQFull + b), 1);
+      mbar_init(bar(C::bQEmpty + b), 1);
+    }
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(bar(C::bKFull + s), 1);
       mbar_init(bar(C::bKEmpty + s), 1);
@@ -162,11 +164,13 @@ __global__ void __launch_bounds__(320, 1)
       bool ok = true;
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         const FwdItem it = fwd_item(k, a);
-        if (!mbar_wait(bar(C::bQEmpty), (n_items_done & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::bQFull), C::kTile);
+        // two Q buffers: the next item's Q streams in while this one is being processed
+        const int qb = n_items_done & 1;
+        if (!mbar_wait(bar(C::bQEmpty + qb), ((n_items_done >> 1) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::bQFull + qb), C::kTile);
         for (int r = 0; r < C::kRegions; ++r)
-          tma_load_3d(sb + C::kQ + r * C::kRegionBytes, &tmQ, bar(C::bQFull), r * 64,
-                      it.m * kBlock, it.bh);
+          tma_load_3d(sb + C::kQ + qb * C::kTile + r * C::kRegionBytes, &tmQ, bar(C::bQFull + qb),
+                      r * 64, it.m * kBlock, it.bh);
         ++n_items_done;
         for (int j = it.lo; j <= it.hi; ++j) {
           const int s = kc % C::kStages;
@@ -192,7 +196,8 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       // Drain: every copy issued must have landed before the CTA may exit.
-      if (n_items_done > 0) mbar_wait(bar(C::bQFull), (n_items_done - 1) & 1, nullptr);
+      for (int n = (n_items_done > 2 ? n_items_done - 2 : 0); n < n_items_done; ++n)
+        mbar_wait(bar(C::bQFull + (n & 1)), (n >> 1) & 1, nullptr);
       for (int s = 0; s < C::kStages; ++s) {
         if (kc > s) {
           const int last = s + C::kStages * ((kc - 1 - s) / C::kStages);
@@ -215,8 +220,8 @@ __global__ void __launch_bounds__(320, 1)
       int ns = 0, npv = 0; // S and P V products issued (all items)
       bool ok = true;
 
-      // S_j = Q K_j^T into buffer ns & 1; after the item's last S, Q may be replaced.
-      auto issue_s = [&](int j, int hi) -> bool {
+      // S_j = Q K_j^T into buffer ns & 1; after the item's last S, its Q may be replaced.
+      auto issue_s = [&](int j, int hi, int qb) -> bool {
         const int s = kc % C::kStages;
         const int b = ns & 1;
         if (!mbar_wait(bar(C::bKFull + s), (kc / C::kStages) & 1, abort_flag)) return false;
@@ -228,12 +233,12 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-          mma_ss(tmem + C::tS0 + 128u * b, sdesc_sw128(sb + C::kQ + off, 16, 1024),
+          mma_ss(tmem + C::tS0 + 128u * b, sdesc_sw128(sb + C::kQ + qb * C::kTile + off, 16, 1024),
                  sdesc_sw128(sb + C::kK + s * C::kTile + off, 16, 1024), idS, kk > 0);
         }
         tc_commit(bar(C::bKEmpty + s));
         tc_commit(bar(C::bSFull + b));
-        if (j == hi) tc_commit(bar(C::bQEmpty));
+        if (j == hi) tc_commit(bar(C::bQEmpty + qb));
         ++ns;
         return true;
       };
@@ -260,11 +265,12 @@ __global__ void __launch_bounds__(320, 1)
 
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         const FwdItem it = fwd_item(k, a);
-        if (!mbar_wait(bar(C::bQFull), n_items_done & 1, abort_flag)) break;
+        const int qb = n_items_done & 1;
+        if (!mbar_wait(bar(C::bQFull + qb), (n_items_done >> 1) & 1, abort_flag)) break;
         ++n_items_done;
-        ok = issue_s(it.lo, it.hi);
+        ok = issue_s(it.lo, it.hi, qb);
         for (int j = it.lo; ok && j <= it.hi; ++j) {
-          if (j + 1 <= it.hi) ok = issue_s(j + 1, it.hi);
+          if (j + 1 <= it.hi) ok = issue_s(j + 1, it.hi, qb);
           if (ok) ok = issue_pv(j == it.lo, j == it.lo && n_items_done > 1);
         }
       }
