@@ -126,8 +126,8 @@ struct BwdCfgT {
   static constexpr int bY0Empty = bY0Full + S0;
   static constexpr int bY1Full = bY0Empty + S0;
   static constexpr int bY1Empty = bY1Full + S1;
-  static constexpr int bA = bY1Empty + S1;  // 9 kernel-specific barriers
-  static constexpr int bMmaFin = bA + 9;
+  static constexpr int bA = bY1Empty + S1;  // 10 kernel-specific barriers
+  static constexpr int bMmaFin = bA + 10;
   static constexpr int kNumBars = bMmaFin + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kSmemBytes = kMisc + 16 + 1024;
@@ -560,10 +560,11 @@ __global__ void __launch_bounds__(320, 1)
                      const __grid_constant__ CUtensorMap tmdO, const BwdArgs a) {
   using C = DqCfg<D>;
   constexpr uint32_t tS0 = 0, tDP = 256, tDQ = 384;
-  // S full per buffer, dS full per buffer, dP full, dP free, dQ done, dQ read
-  constexpr int bSFull = C::bA + 0, bDSFull = C::bA + 2, bDPFull = C::bA + 4,
-                bDPFree = C::bA + 5, bDQDone = C::bA + 6, bAccFree = C::bA + 7,
-                bAccReady = C::bA + 8;
+  // per S buffer: S full, dS full, dQ done (dQ read that buffer's dS); dP full, dP free;
+  // dQ read by the epilogue, dQ of the item complete
+  constexpr int bSFull = C::bA + 0, bDSFull = C::bA + 2, bDQDone = C::bA + 4,
+                bDPFull = C::bA + 6, bDPFree = C::bA + 7, bAccFree = C::bA + 8,
+                bAccReady = C::bA + 9;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -590,10 +591,10 @@ __global__ void __launch_bounds__(320, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(bSFull + b), 1);
       mbar_init(bar(bDSFull + b), 256);
+      mbar_init(bar(bDQDone + b), 1);
     }
     mbar_init(bar(bDPFull), 1);
     mbar_init(bar(bDPFree), 256);
-    mbar_init(bar(bDQDone), 1);
     mbar_init(bar(bAccFree), 256);
     mbar_init(bar(bAccReady), 1);
     mbar_init(bar(C::bMmaFin), 1);
@@ -660,11 +661,13 @@ __global__ void __launch_bounds__(320, 1)
       int items = 0, g = 0;
       bool ok = true;
       // S(t) = Q_i K_j^T into buffer t & 1 (K in ring-0 stage t % S0); its buffer held
-      // dS(t-2), which dQ(t-2) must have read
+      // dS(t-2), which dQ(t-2) must have read. dQ completions are counted per buffer, so
+      // the next completion of that barrier (dQ(t)) cannot come before this S(t).
       auto issue_s = [&](int xb, int t) -> bool {
         const int s = t % C::kStages0;
         if (!mbar_wait(bar(C::bY0Full + s), (t / C::kStages0) & 1, abort_flag)) return false;
-        if (t >= 2 && !mbar_wait(bar(bDQDone), (t - 2) & 1, abort_flag)) return false;
+        if (t >= 2 && !mbar_wait(bar(bDQDone + (t & 1)), ((t >> 1) - 1) & 1, abort_flag))
+          return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -730,7 +733,7 @@ __global__ void __launch_bounds__(320, 1)
                                C::kRegionBytes, 1024),
                    idA, (it > 0 || kk > 0) ? 1u : 0u);
           tc_commit(bar(C::bY0Empty + t % C::kStages0));
-          tc_commit(bar(bDQDone));
+          tc_commit(bar(bDQDone + (t & 1)));
           if (it + 1 == n_it) tc_commit(bar(bAccReady));  // dQ of the item is complete
         }
         g += n_it;
