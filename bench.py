@@ -117,6 +117,20 @@ class ClockSampler:
                 "samples": len(self.samples), "reasons": sorted(self.reasons)}
 
 
+# ------------------------------------------------------------------------- ranks
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest of `value` over all ranks (every rank gets it)."""
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the flops of every rank over the slowest rank's step time."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------------- our arm
 def run_ours(args, w, rank, world, local_rank):
     import torch
@@ -211,9 +225,7 @@ def run_ours(args, w, rank, world, local_rank):
         ms_per_step = bracket_ms / args.steps  # nothing but the steps in the bracket
 
     if dist is not None:
-        t = torch.tensor([ms_per_step], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_per_step = float(t.item())
+        ms_per_step = max_over_ranks(ms_per_step, dist, dev)
 
     # ---------------------------------------------------------------- end to end
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
@@ -253,9 +265,7 @@ def run_ours(args, w, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
     if dist is not None:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e2e_ms, dist, dev)
         dist.barrier()
         dist.destroy_process_group()
 
@@ -264,7 +274,7 @@ def run_ours(args, w, rank, world, local_rank):
 
     peaks, peak_src = load_peaks()
     flops = w.step_flops()
-    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    value = job_tflops(flops, world, ms_per_step)
     kernel_flops = {"fwd": w.fwd_flops(), "bwd_preprocess": 0.0,
                     "bwd_dkdv": 2.0 * w.fwd_flops(), "bwd_dq": 0.5 * w.fwd_flops()}
     kernels = {}
@@ -316,7 +326,7 @@ def run_ours(args, w, rank, world, local_rank):
         "pct_of_dense_peak": round(100 * value / world / DATASHEET_BF16_TFLOPS, 2),
         "pct_of_measured_peak": round(100 * value / world / burst, 2),
         "clocks": clocks.summary(),
-        "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+        "e2e": {"value": round(job_tflops(flops, world, e2e_ms), 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "steps": e2e_steps,
                 "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes},
         "gpu_launches": launches_per_step * args.steps,

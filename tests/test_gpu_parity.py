@@ -37,6 +37,23 @@ def test_small_and_ragged(N, d, mode):
     G.assert_within_bounds(errs, (N, d, mode))
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("mode", ["none", "causal", "win100_30"])
+def test_many_items_per_cta(d, mode):
+    """More (head, tile) work items than SMs, so every persistent CTA runs several items
+    back to back (the stationary tiles, accumulators and barrier phases carry over)."""
+    causal, window = MODES[mode]
+    B, H, N = 4, 64, 384  # 256 heads x 3 tiles = 768 items per kernel
+    inp = inputs(B, H, N, d, 800 + d)
+    scale = 1.0 / np.sqrt(d)
+    out = G.run_library(inp, scale, causal, window)
+    heads = [(0, 0), (1, 17), (2, 40), (3, 63)]
+    errs = G.compare(inp, out, scale, causal, window, heads)
+    G.assert_within_bounds(errs, (d, mode))
+    for n in ("o", "dq", "dk", "dv"):
+        assert torch.isfinite(out[n].float()).all(), n
+
+
 def _sampled_heads(w, count=4):
     rng = np.random.default_rng(w.seed_index)
     BH = w.B * w.H
