@@ -101,10 +101,6 @@ int launch_regs(Kernel k) {
   return attr.numRegs;
 }
 
-fa_status_t launched() {
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-}
-
 int sm_count() {
   static int cache[64] = {0};
   int dev = 0;
@@ -115,6 +111,19 @@ int sm_count() {
   if (dev >= 0 && dev < 64) cache[dev] = n;
   return n;
 }
+
+// Heads per chunk of the masked schedules: enough for about one item per SM.
+int head_group(int BH, int tiles) {
+  int g = (sm_count() + tiles - 1) / tiles;
+  if (g < 1) g = 1;
+  if (g > BH) g = BH;
+  return g;
+}
+
+fa_status_t launched() {
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 
 template <int D>
 fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int BH,
@@ -132,6 +141,7 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   a.n_qtiles = fa::num_tiles(N);
   a.n_items = BH * a.n_qtiles;
   a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
+  a.group = head_group(BH, a.n_qtiles);
   a.scale_log2 = scale * fa::kLog2e;
   a.left = left;
   a.right = right;
@@ -183,6 +193,7 @@ fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void*
   a.BH = BH;
   a.n_items = BH * a.n_tiles;
   a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
+  a.group = head_group(BH, a.n_tiles);
   const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
   fa::fa_bwd_dkdv_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, a);
   return launched();
@@ -213,6 +224,7 @@ fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* d
   a.BH = BH;
   a.n_items = BH * a.n_tiles;
   a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
+  a.group = head_group(BH, a.n_tiles);
   const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
   fa::fa_bwd_dq_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, a);
   return launched();

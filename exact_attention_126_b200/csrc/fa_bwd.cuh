@@ -92,7 +92,8 @@ struct BwdArgs {
   int BH;
   int n_tiles;
   int n_items;          // BH * n_tiles: one item per (batch*head, stationary tile)
-  int longest_first;    // order items by decreasing length (masked problems)
+  int longest_first;    // masked problems: chunks of `group` heads, longest items first
+  int group;
   float scale;
   float scale_log2;
   int left;
@@ -190,14 +191,12 @@ __device__ __forceinline__ void load_cols64(uint32_t taddr, float (&x)[64]) {
 }
 
 // Item k of the persistent schedule: the (batch*head, stationary tile). Masked problems
-// go longest first across heads: key tiles in increasing order for dK/dV (key tile 0 is
-// seen by every query tile under a causal mask), query tiles in decreasing order for dQ.
+// use chunks of heads with the longest items first (see chunked_item): key tiles in
+// increasing order for dK/dV, query tiles in decreasing order for dQ.
 __device__ __forceinline__ void bwd_item(int k, const BwdArgs& a, bool rising, int& bh,
                                          int& tile) {
   if (a.longest_first) {
-    const int step = k / a.BH;
-    tile = rising ? step : a.n_tiles - 1 - step;
-    bh = k % a.BH;
+    chunked_item(k, a.BH, a.n_tiles, a.group, rising, bh, tile);
   } else {
     bh = k / a.n_tiles;
     tile = k % a.n_tiles;

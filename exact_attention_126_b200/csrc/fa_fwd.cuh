@@ -35,7 +35,8 @@ struct FwdArgs {
   int BH;
   int n_qtiles;
   int n_items;        // BH * n_qtiles
-  int longest_first;  // order items by decreasing length (masked problems)
+  int longest_first;  // masked problems: chunks of `group` heads, longest items first
+  int group;
   float scale_log2;   // scale * log2(e)
   int left;
   int right;
@@ -92,8 +93,7 @@ struct FwdItem {
 __device__ __forceinline__ FwdItem fwd_item(int k, const FwdArgs& a) {
   FwdItem it;
   if (a.longest_first) {
-    it.m = a.n_qtiles - 1 - k / a.BH;
-    it.bh = k % a.BH;
+    chunked_item(k, a.BH, a.n_qtiles, a.group, false, it.bh, it.m);
   } else {
     it.bh = k / a.n_qtiles;
     it.m = k % a.n_qtiles;

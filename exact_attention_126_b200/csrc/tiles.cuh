@@ -61,4 +61,21 @@ __host__ __device__ inline bool is_visible(int r, int c, const Mask& k) {
          (k.right < 0 || c - r <= k.right);
 }
 
+// Work item k of a persistent schedule over BH heads of T tiles each, for masked problems
+// (tiles of different lengths). Heads go in chunks of `group` (chosen so that a chunk has
+// about one item per SM): every CTA works on a few heads at a time, whose K/V (or Q/dO)
+// tiles then stay in L2 while all of them are read. Inside a chunk, items go longest
+// first: tile index increasing when `rising` (dK/dV: key tile 0 is seen by the most query
+// tiles), decreasing otherwise (forward, dQ: the last query tile sees the most keys).
+__host__ __device__ inline void chunked_item(int k, int BH, int T, int group, bool rising,
+                                             int& bh, int& tile) {
+  const int per_chunk = group * T;
+  const int chunk = k / per_chunk;
+  const int r = k - chunk * per_chunk;
+  const int heads = (BH - chunk * group) < group ? (BH - chunk * group) : group;
+  const int step = r / heads;
+  bh = chunk * group + (r - step * heads);
+  tile = rising ? step : T - 1 - step;
+}
+
 }  // namespace fa
