@@ -20,11 +20,12 @@
 // the same way by one CTA per query tile walking its key tiles (S, dP, then
 // dQ += dS K). Nothing is reduced across CTAs, so the results are deterministic.
 //
-// In both kernels two warpgroups share every row: warpgroup h takes the 64 columns
-// 64h..64h+63 of it (query columns for dK/dV, key columns for dQ). P needs no row
-// maximum here (the LSE is known), so the two halves never wait for each other. The
-// MMA issuer orders the products so that the next tile's S and dP are computed while
-// the softmax warpgroups work on the current tile.
+// In both kernels four warpgroups share every row: warpgroup h takes the 32 columns
+// 32h..32h+31 of it (query columns for dK/dV, key columns for dQ), so that four warps
+// per SM sub-partition hide each other's latencies. P needs no row maximum here (the
+// LSE is known), so the groups never wait for each other. The MMA issuer (warp 16;
+// warp 17 issues the TMA copies) orders the products so that the next tile's S and dP
+// are computed while the softmax warpgroups work on the current tile.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -134,7 +135,12 @@ struct BwdCfgT {
   static constexpr int kSmemBytes = kMisc + 16 + 1024;
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr int kThreads = 320;  // 8 softmax warps, MMA warp, producer warp
+  static constexpr int kGroups = 4;               // softmax warpgroups per row
+  static constexpr int kCols = kBlock / kGroups;  // columns of a row per thread
+  static constexpr int kSoftmax = 128 * kGroups;  // softmax threads
+  static constexpr int kThreads = kSoftmax + 64;  // softmax warps, MMA warp, producer warp
+  static constexpr int kWarpMma = 4 * kGroups;
+  static constexpr int kWarpProducer = 4 * kGroups + 1;
 };
 
 template <int D>
@@ -153,41 +159,43 @@ __device__ __forceinline__ void drain_ring(uint32_t full_bar0, int S, int n) {
 }
 
 // Writes this thread's NC fp32 accumulator columns starting at `taddr`, times `mul`, as
-// bf16 to `dst`.
+// bf16 to `dst` (16 columns, 32 bytes, per step).
 template <int NC>
 __device__ __forceinline__ void store_acc_cols(uint32_t taddr, float mul, __nv_bfloat16* dst,
                                                bool valid) {
+  static_assert(NC % 16 == 0, "whole 16-column steps");
 #pragma unroll
-  for (int q = 0; q < NC / 32; ++q) {
-    uint32_t o[32];
-    tmem_ld32(taddr + 32 * q, o);
+  for (int q = 0; q < NC / 16; ++q) {
+    uint32_t o[16];
+    tmem_ld16(taddr + 16 * q, o);
     tmem_wait_ld();
     reg_fence(o);
-    uint32_t w[16];
+    uint32_t w[8];
 #pragma unroll
-    for (int c = 0; c < 16; ++c)
+    for (int c = 0; c < 8; ++c)
       w[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * mul, __uint_as_float(o[2 * c + 1]) * mul);
     if (valid) {
-#pragma unroll
-      for (int v4 = 0; v4 < 4; ++v4)
-        st_global_v4(dst + 32 * q + 8 * v4, w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+      st_global_v4(dst + 16 * q, w[0], w[1], w[2], w[3]);
+      st_global_v4(dst + 16 * q + 8, w[4], w[5], w[6], w[7]);
     }
   }
 }
 
-// Loads 64 consecutive fp32 TMEM columns of this thread's lane.
-__device__ __forceinline__ void load_cols64(uint32_t taddr, float (&x)[64]) {
-  uint32_t u[2][32];
-  tmem_ld32(taddr, u[0]);
-  tmem_ld32(taddr + 32, u[1]);
+// Loads 32 consecutive fp32 TMEM columns of this thread's lane.
+__device__ __forceinline__ void load_cols32(uint32_t taddr, float (&x)[32]) {
+  uint32_t u[32];
+  tmem_ld32(taddr, u);
   tmem_wait_ld();
-  reg_fence(u[0]);
-  reg_fence(u[1]);
+  reg_fence(u);
 #pragma unroll
-  for (int c = 0; c < 32; ++c) {
-    x[c] = __uint_as_float(u[0][c]);
-    x[32 + c] = __uint_as_float(u[1][c]);
-  }
+  for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(u[c]);
+}
+
+// TMEM column (from the buffer base) of K-step kk of a bf16 A operand that the softmax
+// warpgroups packed: group h holds its 32 bf16 entries (16 columns) over the first half
+// of its own 32 fp32 columns, so K-steps 2h and 2h+1 sit at columns 32h and 32h+8.
+__device__ __forceinline__ constexpr uint32_t packed_col(int kk) {
+  return 8u * kk + 16u * (kk >> 1);
 }
 
 // Item k of the persistent schedule: the (batch*head, stationary tile). Masked problems
@@ -230,13 +238,13 @@ __device__ __forceinline__ void bwd_teardown(uint32_t tmem, int warp) {
 // dK, dV: persistent CTAs over items (batch*head, key tile j). X0 = K_j, X1 = V_j; per
 // stage Y0 = Q_i with the LSE (log2 units) and delta of its 128 rows, Y1 = dO_i.
 // TMEM: S^T at 0, dP^T at 128, dK at 256, dV at 256 + D. Warpgroup h writes its bf16
-// half of P^T (dS^T) over the first 32 of its own 64 fp32 columns of S^T (dP^T), so the
-// A operand of dV (dK) takes K-steps 0..3 from columns 0..31 and 4..7 from 64..95.
+// part of P^T (dS^T) over the first 16 of its own 32 fp32 columns of S^T (dP^T), so the
+// A operand of dV (dK) takes K-step kk from column packed_col(kk).
 // MMA order per query tile i:  dV(i), S^T(i+1), dK(i), dP^T(i+1). Tile counters (for
 // barrier parities) run over all items of the CTA.
 // ------------------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
     fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
@@ -271,11 +279,11 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(bar(bSFull), 1);
     mbar_init(bar(bDPFull), 1);
-    mbar_init(bar(bPFull), 256);
-    mbar_init(bar(bDSFull), 256);
+    mbar_init(bar(bPFull), C::kSoftmax / 32);
+    mbar_init(bar(bDSFull), C::kSoftmax / 32);
     mbar_init(bar(bDVDone), 1);
     mbar_init(bar(bDKDone), 1);
-    mbar_init(bar(bAccFree), 256);
+    mbar_init(bar(bAccFree), C::kSoftmax / 32);
     mbar_init(bar(bAccReady), 1);
     mbar_init(bar(C::bMmaFin), 1);
     *abort_flag = 0;
@@ -283,7 +291,7 @@ __global__ void __launch_bounds__(320, 1)
   }
   const uint32_t tmem = bwd_setup<C>(smem, warp);
 
-  if (warp == 9) {
+  if (warp == C::kWarpProducer) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_map(&tmQ);
@@ -340,7 +348,7 @@ __global__ void __launch_bounds__(320, 1)
       drain_ring(bar(C::bY1Full), C::kStages1, n1);
     }
     __syncwarp();
-  } else if (warp == 8) {
+  } else if (warp == C::kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
@@ -405,7 +413,7 @@ __global__ void __launch_bounds__(320, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kBlock / 16; ++kk)
-            mma_ts(tmem + tDV, tmem + tS + kk * 8 + (kk >> 2) * 32,
+            mma_ts(tmem + tDV, tmem + tS + packed_col(kk),
                    sdesc_sw128(sb + C::kY1 + s1 * C::kTile + kk * 2048, C::kRegionBytes, 1024),
                    idA, (it > 0 || kk > 0) ? 1u : 0u);
           tc_commit(bar(C::bY1Empty + s1));
@@ -428,7 +436,7 @@ __global__ void __launch_bounds__(320, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kBlock / 16; ++kk)
-            mma_ts(tmem + tDK, tmem + tDP + kk * 8 + (kk >> 2) * 32,
+            mma_ts(tmem + tDK, tmem + tDP + packed_col(kk),
                    sdesc_sw128(sb + C::kY0 + s0 * C::kTile + kk * 2048, C::kRegionBytes, 1024),
                    idA, (it > 0 || kk > 0) ? 1u : 0u);
           tc_commit(bar(C::bY0Empty + s0));
@@ -454,8 +462,9 @@ __global__ void __launch_bounds__(320, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------------ warps 0..7
-    const int h = warp >> 2;          // query columns 64h .. 64h+63 of each query tile
+    // ------------------------------------------------------------------ softmax warps
+    constexpr int NC = C::kCols;
+    const int h = warp >> 2;              // query columns NC*h .. NC*h+NC-1 of each tile
     const int t_row = threadIdx.x & 127;  // key row in the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const float sl2 = a.scale_log2;
@@ -478,12 +487,12 @@ __global__ void __launch_bounds__(320, 1)
           break;
         }
         tc_fence_after();
-        const float* lse_s = reinterpret_cast<const float*>(smem + C::kLse + s * 512) + 64 * h;
-        const float* del_s = reinterpret_cast<const float*>(smem + C::kDelta + s * 512) + 64 * h;
-        float p[64];
-        load_cols64(tmem + lane_base + tS + 64 * h, p);
+        const float* lse_s = reinterpret_cast<const float*>(smem + C::kLse + s * 512) + NC * h;
+        const float* del_s = reinterpret_cast<const float*>(smem + C::kDelta + s * 512) + NC * h;
+        float p[NC];
+        load_cols32(tmem + lane_base + tS + NC * h, p);
 #pragma unroll
-        for (int r = 0; r < 64; r += 4) {
+        for (int r = 0; r < NC; r += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse_s + r);
           p[r] = ex2(fmaf(p[r], sl2, -l4.x));
           p[r + 1] = ex2(fmaf(p[r + 1], sl2, -l4.y));
@@ -492,38 +501,38 @@ __global__ void __launch_bounds__(320, 1)
         }
         if (!tile_all_visible(i, j, mk)) {
 #pragma unroll
-          for (int r = 0; r < 64; ++r)
-            if (!is_visible(i * kBlock + 64 * h + r, c, mk)) p[r] = 0.f;
+          for (int r = 0; r < NC; ++r)
+            if (!is_visible(i * kBlock + NC * h + r, c, mk)) p[r] = 0.f;
         }
         {
-          uint32_t pk[32];
+          uint32_t pk[NC / 2];
 #pragma unroll
-          for (int r = 0; r < 32; ++r) pk[r] = pack_bf16x2(p[2 * r], p[2 * r + 1]);
-          tmem_st32(tmem + lane_base + tS + 64 * h, pk);
+          for (int r = 0; r < NC / 2; ++r) pk[r] = pack_bf16x2(p[2 * r], p[2 * r + 1]);
+          tmem_st16(tmem + lane_base + tS + NC * h, pk);
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(bPFull));
+        mbar_arrive_warp(bar(bPFull));
         if (!mbar_wait_warp(bar(bDPFull), t & 1, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        float dp[64];
-        load_cols64(tmem + lane_base + tDP + 64 * h, dp);
-        uint32_t w[32];
+        float dp[NC];
+        load_cols32(tmem + lane_base + tDP + NC * h, dp);
+        uint32_t w[NC / 2];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
+        for (int e = 0; e < NC / 2; e += 2) {
           const int r0 = 2 * e;
           const float4 d4 = *reinterpret_cast<const float4*>(del_s + r0);
           w[e] = pack_bf16x2(p[r0] * (dp[r0] - d4.x), p[r0 + 1] * (dp[r0 + 1] - d4.y));
           w[e + 1] = pack_bf16x2(p[r0 + 2] * (dp[r0 + 2] - d4.z), p[r0 + 3] * (dp[r0 + 3] - d4.w));
         }
         // bf16 dS^T goes over the first half of this warpgroup's own fp32 dP^T columns
-        tmem_st32(tmem + lane_base + tDP + 64 * h, w);
+        tmem_st16(tmem + lane_base + tDP + NC * h, w);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(bDSFull));
+        mbar_arrive_warp(bar(bDSFull));
       }
       if (!ok) break;
       g += n_it;
@@ -534,13 +543,14 @@ __global__ void __launch_bounds__(320, 1)
       }
       ++items;
       tc_fence_after();
+      constexpr int NO = D / C::kGroups;
       const bool valid = c < a.N;
-      const size_t off = ((size_t)bh * a.N + (valid ? c : 0)) * D + (D / 2) * h;
-      store_acc_cols<D / 2>(tmem + lane_base + tDV + (D / 2) * h, 1.f, a.out1 + off, valid);
-      store_acc_cols<D / 2>(tmem + lane_base + tDK + (D / 2) * h, a.scale, a.out0 + off, valid);
+      const size_t off = ((size_t)bh * a.N + (valid ? c : 0)) * D + NO * h;
+      store_acc_cols<NO>(tmem + lane_base + tDV + NO * h, 1.f, a.out1 + off, valid);
+      store_acc_cols<NO>(tmem + lane_base + tDK + NO * h, a.scale, a.out0 + off, valid);
       // dK, dV have been read: the next item's first products may overwrite them
       tc_fence_before();
-      mbar_arrive(bar(bAccFree));
+      mbar_arrive_warp(bar(bAccFree));
     }
   }
   bwd_teardown<C>(tmem, warp);
@@ -549,11 +559,11 @@ __global__ void __launch_bounds__(320, 1)
 // ------------------------------------------------------------------------------------
 // dQ: persistent CTAs over items (batch*head, query tile i). X0 = Q_i, X1 = dO_i; per
 // stage Y0 = K_j, Y1 = V_j. TMEM: S in two buffers at 0 and 128 (bf16 dS goes over S,
-// each warpgroup over the first half of its own columns), dP at 256, dQ at 384. MMA
+// each warpgroup over the first half of its own 32 columns), dP at 256, dQ at 384. MMA
 // order per key tile j: S(j+1), dP(j+1), dQ(j). Tile counters run over all items.
 // ------------------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
     fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmdO, const BwdArgs a) {
@@ -589,12 +599,12 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(bSFull + b), 1);
-      mbar_init(bar(bDSFull + b), 256);
+      mbar_init(bar(bDSFull + b), C::kSoftmax / 32);
       mbar_init(bar(bDQDone + b), 1);
     }
     mbar_init(bar(bDPFull), 1);
-    mbar_init(bar(bDPFree), 256);
-    mbar_init(bar(bAccFree), 256);
+    mbar_init(bar(bDPFree), C::kSoftmax / 32);
+    mbar_init(bar(bAccFree), C::kSoftmax / 32);
     mbar_init(bar(bAccReady), 1);
     mbar_init(bar(C::bMmaFin), 1);
     *abort_flag = 0;
@@ -602,7 +612,7 @@ __global__ void __launch_bounds__(320, 1)
   }
   const uint32_t tmem = bwd_setup<C>(smem, warp);
 
-  if (warp == 9) {
+  if (warp == C::kWarpProducer) {
     if (lane == 0) {
       tma_prefetch_map(&tmQ);
       tma_prefetch_map(&tmK);
@@ -653,7 +663,7 @@ __global__ void __launch_bounds__(320, 1)
       drain_ring(bar(C::bY1Full), C::kStages1, n1);
     }
     __syncwarp();
-  } else if (warp == 8) {
+  } else if (warp == C::kWarpMma) {
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);
@@ -727,7 +737,7 @@ __global__ void __launch_bounds__(320, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kBlock / 16; ++kk)
-            mma_ts(tmem + tDQ, tmem + tS0 + 128u * (t & 1) + kk * 8 + (kk >> 2) * 32,
+            mma_ts(tmem + tDQ, tmem + tS0 + 128u * (t & 1) + packed_col(kk),
                    sdesc_sw128(sb + C::kY0 + (t % C::kStages0) * C::kTile + kk * 2048,
                                C::kRegionBytes, 1024),
                    idA, (it > 0 || kk > 0) ? 1u : 0u);
@@ -743,7 +753,8 @@ __global__ void __launch_bounds__(320, 1)
     }
     __syncwarp();
   } else {
-    const int h = warp >> 2;          // key columns 64h .. 64h+63 of each key tile
+    constexpr int NC = C::kCols;
+    const int h = warp >> 2;          // key columns NC*h .. NC*h+NC-1 of each key tile
     const int t_row = threadIdx.x & 127;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const float sl2 = a.scale_log2;
@@ -769,33 +780,33 @@ __global__ void __launch_bounds__(320, 1)
           break;
         }
         tc_fence_after();
-        float p[64];
-        load_cols64(tmem + lane_base + tS0 + 128u * b + 64 * h, p);
+        float p[NC];
+        load_cols32(tmem + lane_base + tS0 + 128u * b + NC * h, p);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) p[c] = ex2(fmaf(p[c], sl2, -lse2));
+        for (int c = 0; c < NC; ++c) p[c] = ex2(fmaf(p[c], sl2, -lse2));
         if (!tile_all_visible(i, jj, mk)) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (!is_visible(r, jj * kBlock + 64 * h + c, mk)) p[c] = 0.f;
+          for (int c = 0; c < NC; ++c)
+            if (!is_visible(r, jj * kBlock + NC * h + c, mk)) p[c] = 0.f;
         }
         if (!mbar_wait_warp(bar(bDPFull), t & 1, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        float dp[64];
-        load_cols64(tmem + lane_base + tDP + 64 * h, dp);
+        float dp[NC];
+        load_cols32(tmem + lane_base + tDP + NC * h, dp);
         tc_fence_before();
-        mbar_arrive(bar(bDPFree));
-        uint32_t w[32];
+        mbar_arrive_warp(bar(bDPFree));
+        uint32_t w[NC / 2];
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
+        for (int e = 0; e < NC / 2; ++e)
           w[e] = pack_bf16x2(p[2 * e] * (dp[2 * e] - dl), p[2 * e + 1] * (dp[2 * e + 1] - dl));
         // bf16 dS goes over the first half of this warpgroup's own fp32 S columns
-        tmem_st32(tmem + lane_base + tS0 + 128u * b + 64 * h, w);
+        tmem_st16(tmem + lane_base + tS0 + 128u * b + NC * h, w);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(bDSFull + b));
+        mbar_arrive_warp(bar(bDSFull + b));
       }
       if (!ok) break;
       g += n_it;
@@ -806,11 +817,12 @@ __global__ void __launch_bounds__(320, 1)
       }
       ++items;
       tc_fence_after();
-      const size_t off = ((size_t)bh * a.N + (valid ? r : 0)) * D + (D / 2) * h;
-      store_acc_cols<D / 2>(tmem + lane_base + tDQ + (D / 2) * h, a.scale, a.out0 + off, valid);
+      constexpr int NO = D / C::kGroups;
+      const size_t off = ((size_t)bh * a.N + (valid ? r : 0)) * D + NO * h;
+      store_acc_cols<NO>(tmem + lane_base + tDQ + NO * h, a.scale, a.out0 + off, valid);
       // dQ has been read: the next item's first product may overwrite it
       tc_fence_before();
-      mbar_arrive(bar(bAccFree));
+      mbar_arrive_warp(bar(bAccFree));
     }
   }
   bwd_teardown<C>(tmem, warp);

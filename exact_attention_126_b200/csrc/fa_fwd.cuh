@@ -5,18 +5,19 @@
 // load a Q block, iterate over the K, V blocks; page "告别OOM和训练慢…(含A100环境配置)" §2.1
 // tiling). Roles:
 //
-//   warp 9       TMA producer: Q per item, then K_j and V_j through a ring of shared-memory
+//   warp 17      TMA producer: Q per item, then K_j and V_j through a ring of shared-memory
 //                stages (128-byte swizzle), guarded by full/empty mbarriers.
-//   warp 8       MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM buffers, so that
+//   warp 16      MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM buffers, so that
 //                S_{j+1} is computed while the softmax works on S_j; then, once P_j is
 //                published, O += P_j V_j with P_j read from TMEM.
-//   warps 0..7   softmax, two warpgroups that split every score row by columns: thread
-//                (h, r) owns keys 64h..64h+63 of query row r. They exchange their partial
+//   warps 0..15  softmax, four warpgroups that split every score row by columns: thread
+//                (h, r) owns keys 32h..32h+31 of query row r (four warps per SM
+//                sub-partition hide each other's latencies). They exchange their partial
 //                row maxima through shared memory, update the running max m and sum l
-//                (page "告别OOM和训练慢…" §2.2), write their half of P_j =
-//                exp2(s*scale*log2e - m) in bf16 to TMEM, rescale their half of O when m
+//                (page "告别OOM和训练慢…" §2.2), write their part of P_j =
+//                exp2(s*scale*log2e - m) in bf16 to TMEM, rescale their quarter of O when m
 //                grew by more than 2^8 (exact: O and l carry the same stale m), and at the
-//                end of the item write their half of O / l (and LSE = ln2 * (m + log2 l)).
+//                end of the item write their quarter of O / l (and LSE = ln2 * (m + log2 l)).
 //
 // TMEM: S0, S1 (128 columns each), O (head_dim columns), P (64 columns).
 #pragma once
@@ -54,8 +55,12 @@ struct FwdCfg {
   static constexpr int kQ = 0;                        // + (item & 1) * kTile
   static constexpr int kK = kQ + 2 * kTile;           // + s * kTile
   static constexpr int kV = kK + kStages * kTile;     // + s * kTile
-  static constexpr int kRed = kV + kStages * kTile;   // [2 slots][2 halves][128 rows] fp32
-  static constexpr int kBar = kRed + 2 * 2 * kBlock * 4;
+  static constexpr int kGroups = 4;                   // softmax warpgroups per row
+  static constexpr int kCols = kBlock / kGroups;      // score columns per thread
+  static constexpr int kOCols = D / kGroups;          // output columns per thread
+  static constexpr int kSoftmax = 128 * kGroups;      // softmax threads
+  static constexpr int kRed = kV + kStages * kTile;   // [2 slots][kGroups][128 rows] fp32
+  static constexpr int kBar = kRed + 2 * kGroups * kBlock * 4;
   // barrier slots
   static constexpr int bQFull = 0;                  // + (item & 1)
   static constexpr int bQEmpty = 2;                 // + (item & 1)
@@ -78,9 +83,9 @@ struct FwdCfg {
   static constexpr uint32_t tS0 = 0;
   static constexpr uint32_t tO = 256;
   static constexpr uint32_t tP = 256 + D;
-  static constexpr int kThreads = 320;  // 8 softmax warps, MMA warp, producer warp
-  static constexpr int kWarpMma = 8;
-  static constexpr int kWarpProducer = 9;
+  static constexpr int kThreads = kSoftmax + 64;  // softmax warps, MMA warp, producer warp
+  static constexpr int kWarpMma = 4 * kGroups;
+  static constexpr int kWarpProducer = 4 * kGroups + 1;
 };
 
 struct FwdItem {
@@ -104,7 +109,7 @@ __device__ __forceinline__ FwdItem fwd_item(int k, const FwdArgs& a) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
   using C = FwdCfg<D>;
@@ -134,12 +139,12 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(C::bSFull + b), 1);
-      mbar_init(bar(C::bSFree + b), 256);
-      mbar_init(bar(C::bRed + b), 256);
+      mbar_init(bar(C::bSFree + b), C::kSoftmax / 32);
+      mbar_init(bar(C::bRed + b), C::kSoftmax / 32);
     }
-    mbar_init(bar(C::bPFull), 256);
+    mbar_init(bar(C::bPFull), C::kSoftmax / 32);
     mbar_init(bar(C::bODone), 1);
-    mbar_init(bar(C::bOFree), 256);
+    mbar_init(bar(C::bOFree), C::kSoftmax / 32);
     mbar_init(bar(C::bMmaFin), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -226,7 +231,7 @@ __global__ void __launch_bounds__(320, 1)
         const int b = ns & 1;
         if (!mbar_wait(bar(C::bKFull + s), (kc / C::kStages) & 1, abort_flag)) return false;
         ++kc;
-        // buffer b is free once both softmax warpgroups have read the S it held before
+        // buffer b is free once every softmax warpgroup has read the S it held before
         if (ns >= 2 && !mbar_wait(bar(C::bSFree + b), ((ns >> 1) - 1) & 1, abort_flag))
           return false;
         tc_fence_after();
@@ -280,33 +285,48 @@ __global__ void __launch_bounds__(320, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------------ softmax, warps 0..7
-    const int h = warp >> 2;                     // column half: keys 64h .. 64h+63
+    // ------------------------------------------------------------------ softmax warps
+    constexpr int G = C::kGroups, NC = C::kCols, NO = C::kOCols;
+    const int h = warp >> 2;                     // column group: keys NC*h .. NC*h+NC-1
     const int r = threadIdx.x & 127;             // query row in the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tO = tmem + lane_base + C::tO + (D / 2) * h;
-    const uint32_t tP = tmem + lane_base + C::tP + 32 * h;
+    const uint32_t tO = tmem + lane_base + C::tO + NO * h;
+    const uint32_t tP = tmem + lane_base + C::tP + (NC / 2) * h;
     const float sl2 = a.scale_log2;
     int ns = 0;  // S tiles consumed (all items)
-    int nx = 0;  // row-statistic exchanges between the two warpgroups
+    int nx = 0;  // row-statistic exchanges between the warpgroups
     bool ok = true;
 
-    // Exchanges a per-row value with the other warpgroup; `other` gets that half's value.
-    auto exchange = [&](float v, float& other) -> bool {
-      float* slot = red + (nx & 1) * 256;
+    // Shares a per-row value with the other warpgroups; `all` gets the G values of the row.
+    auto exchange = [&](float v, float (&all)[G]) -> bool {
+      float* slot = red + (nx & 1) * (G * 128);
       slot[h * 128 + r] = v;
-      mbar_arrive(bar(C::bRed + (nx & 1)));
+      mbar_arrive_warp(bar(C::bRed + (nx & 1)));
       if (!mbar_wait_warp(bar(C::bRed + (nx & 1)), (nx >> 1) & 1, abort_flag)) return false;
-      other = slot[(1 - h) * 128 + r];
+#pragma unroll
+      for (int g = 0; g < G; ++g) all[g] = slot[g * 128 + r];
       ++nx;
       return true;
+    };
+    // NO accumulator columns of O: fp32 in, scaled by `mul`, back to TMEM (rescale)
+    auto scale_o = [&](float mul) {
+#pragma unroll
+      for (int q = 0; q < NO / 16; ++q) {
+        uint32_t o[16];
+        tmem_ld16(tO + 16 * q, o);
+        tmem_wait_ld();
+        reg_fence(o);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * mul);
+        tmem_st16(tO + 16 * q, o);
+      }
     };
 
     for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
       const FwdItem it = fwd_item(k, a);
       const int row = it.m * kBlock + r;
       float m_run = -INFINITY;  // running max of scale*log2e*s (the m that P and O carry)
-      float l_run = 0.f;        // this half's running sum of P
+      float l_run = 0.f;        // this group's running sum of P
       for (int j = it.lo; j <= it.hi; ++j) {
         const int b = ns & 1;
         if (!mbar_wait_warp(bar(C::bSFull + b), (ns >> 1) & 1, abort_flag)) {
@@ -314,42 +334,37 @@ __global__ void __launch_bounds__(320, 1)
           break;
         }
         tc_fence_after();
-        uint32_t u[2][32];
-        const uint32_t tS = tmem + lane_base + C::tS0 + 128u * b + 64 * h;
-        tmem_ld32(tS, u[0]);
-        tmem_ld32(tS + 32, u[1]);
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_base + C::tS0 + 128u * b + NC * h, u);
         tmem_wait_ld();
-        reg_fence(u[0]);
-        reg_fence(u[1]);
-        // this half of S_j is in registers: the tensor core may reuse the buffer
+        reg_fence(u);
+        // this group's part of S_j is in registers: the tensor core may reuse the buffer
         tc_fence_before();
-        mbar_arrive(bar(C::bSFree + b));
-        float x[64];
+        mbar_arrive_warp(bar(C::bSFree + b));
+        float x[NC];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          x[c] = __uint_as_float(u[0][c]);
-          x[32 + c] = __uint_as_float(u[1][c]);
-        }
+        for (int c = 0; c < NC; ++c) x[c] = __uint_as_float(u[c]);
         if (!tile_all_visible(it.m, j, mk)) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (!is_visible(row, j * kBlock + 64 * h + c, mk)) x[c] = -INFINITY;
+          for (int c = 0; c < NC; ++c)
+            if (!is_visible(row, j * kBlock + NC * h + c, mk)) x[c] = -INFINITY;
         }
         float mx8[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) mx8[c] = fmaxf(x[c], x[c + 8]);
 #pragma unroll
-        for (int c = 16; c < 64; c += 8)
+        for (int c = 16; c < NC; c += 8)
 #pragma unroll
           for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], x[c + e]);
         float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                          fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        float mx_other;
-        if (!exchange(mx, mx_other)) {
+        float mx_all[G];
+        if (!exchange(mx, mx_all)) {
           ok = false;
           break;
         }
-        mx = fmaxf(mx, mx_other);
+#pragma unroll
+        for (int g = 0; g < G; ++g) mx = fmaxf(mx, mx_all[g]);
         const float m_new = fmaxf(m_run, mx * sl2);
         const bool grow = m_new > m_run + 8.0f;
         float alpha = 1.f;
@@ -359,17 +374,17 @@ __global__ void __launch_bounds__(320, 1)
           l_run *= alpha;
         }
         const float mb = (m_run == -INFINITY) ? 0.f : m_run;
-        // this half of P = exp2(s*scale*log2e - m), packed to bf16 pairs
-        float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        uint32_t pk[32];
+        // this group's part of P = exp2(s*scale*log2e - m), packed to bf16 pairs
+        float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pk[NC / 2];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < NC / 2; ++c) {
           const float p0 = ex2(fmaf(x[2 * c], sl2, -mb));
           const float p1 = ex2(fmaf(x[2 * c + 1], sl2, -mb));
-          ls8[c & 7] += p0 + p1;
+          ls4[c & 3] += p0 + p1;
           pk[c] = pack_bf16x2(p0, p1);
         }
-        l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
+        l_run += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
         if (j > it.lo) {
           // O and the P buffer are busy until P_{j-1} V_{j-1} has finished
           if (!mbar_wait_warp(bar(C::bODone), (ns - 1) & 1, abort_flag)) {
@@ -378,60 +393,50 @@ __global__ void __launch_bounds__(320, 1)
           }
           tc_fence_after();
         }
-        tmem_st32(tP, pk);
-        // rescale this half of O before P_j V_j accumulates into it (that waits for p_full)
-        if (j > it.lo && __any_sync(0xffffffffu, grow)) {
-#pragma unroll
-          for (int q = 0; q < D / 64; ++q) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32 * q, o);
-            tmem_wait_ld();
-            reg_fence(o);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(tO + 32 * q, o);
-          }
-        }
+        tmem_st16(tP, pk);
+        // rescale this group's part of O before P_j V_j accumulates into it (that waits
+        // for p_full)
+        if (j > it.lo && __any_sync(0xffffffffu, grow)) scale_o(alpha);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(C::bPFull));
+        mbar_arrive_warp(bar(C::bPFull));
         ++ns;
       }
       if (!ok) break;
-      // epilogue of the item: l of the whole row, then this half of O / l, and LSE
-      float l_other;
-      if (!exchange(l_run, l_other)) {
+      // epilogue of the item: l of the whole row, then this group's part of O / l, and LSE
+      float l_all[G];
+      if (!exchange(l_run, l_all)) {
         ok = false;
         break;
       }
-      const float l_row = l_run + l_other;
+      float l_row = 0.f;
+#pragma unroll
+      for (int g = 0; g < G; ++g) l_row += l_all[g];
       if (!mbar_wait_warp(bar(C::bODone), (ns - 1) & 1, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const float inv_l = (l_row > 0.f) ? 1.f / l_row : 0.f;
-      __nv_bfloat16* orow = a.o + ((size_t)it.bh * a.N + row) * D + (D / 2) * h;
+      __nv_bfloat16* orow = a.o + ((size_t)it.bh * a.N + row) * D + NO * h;
 #pragma unroll
-      for (int q = 0; q < D / 64; ++q) {
-        uint32_t o[32];
-        tmem_ld32(tO + 32 * q, o);
+      for (int q = 0; q < NO / 16; ++q) {
+        uint32_t o[16];
+        tmem_ld16(tO + 16 * q, o);
         tmem_wait_ld();
         reg_fence(o);
-        uint32_t w[16];
+        uint32_t w[8];
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
+        for (int c = 0; c < 8; ++c)
           w[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
         if (row < a.N) {
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            st_global_v4(orow + 32 * q + 8 * v4, w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2],
-                         w[4 * v4 + 3]);
+          st_global_v4(orow + 16 * q, w[0], w[1], w[2], w[3]);
+          st_global_v4(orow + 16 * q + 8, w[4], w[5], w[6], w[7]);
         }
       }
       // O has been read: the next item's first P V may overwrite it
       tc_fence_before();
-      mbar_arrive(bar(C::bOFree));
+      mbar_arrive_warp(bar(C::bOFree));
       if (h == 0 && row < a.N)
         a.lse[(size_t)it.bh * a.N + row] =
             (l_row > 0.f) ? (m_run + log2f(l_row)) * 0.69314718055994531f : -INFINITY;
