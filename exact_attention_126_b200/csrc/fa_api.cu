@@ -139,9 +139,10 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   a.N = N;
   a.BH = BH;
   a.n_qtiles = fa::num_tiles(N);
-  a.n_items = BH * a.n_qtiles;
+  a.n_pairs = (a.n_qtiles + 1) / 2;
+  a.n_items = BH * a.n_pairs;
   a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
-  a.group = head_group(BH, a.n_qtiles);
+  a.group = head_group(BH, a.n_pairs);
   a.scale_log2 = scale * fa::kLog2e;
   a.left = left;
   a.right = right;

@@ -1,25 +1,29 @@
 // fa_fwd.cuh - fused attention forward for sm_100a.
 //
-// Each persistent CTA takes work items of one 128-row query tile of one (batch, head) and
-// walks the key/value tiles the tile can see (page "Flash Attention 3.7 核心原理与实战" §3.1:
-// load a Q block, iterate over the K, V blocks; page "告别OOM和训练慢…(含A100环境配置)" §2.1
-// tiling). Roles:
+// Each persistent CTA takes work items of two consecutive 128-row query tiles (A and B)
+// of one (batch, head) and walks the key/value tiles they can see (page "Flash Attention
+// 3.7 核心原理与实战" §3.1: load a Q block, iterate over the K, V blocks; page
+// "告别OOM和训练慢…(含A100环境配置)" §2.1 tiling). The two query tiles are independent
+// streams that share every K/V tile: while the softmax of one works on its scores, the
+// tensor core computes the other's products, so neither the special-function unit nor
+// the tensor core waits for the other. Roles:
 //
-//   warp 17      TMA producer: Q per item, then K_j and V_j through a ring of shared-memory
-//                stages (128-byte swizzle), guarded by full/empty mbarriers.
-//   warp 16      MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM buffers, so that
-//                S_{j+1} is computed while the softmax works on S_j; then, once P_j is
-//                published, O += P_j V_j with P_j read from TMEM.
-//   warps 0..15  softmax, four warpgroups that split every score row by columns: thread
-//                (h, r) owns keys 32h..32h+31 of query row r (four warps per SM
-//                sub-partition hide each other's latencies). They exchange their partial
-//                row maxima through shared memory, update the running max m and sum l
-//                (page "告别OOM和训练慢…" §2.2), write their part of P_j =
-//                exp2(s*scale*log2e - m) in bf16 to TMEM, rescale their quarter of O when m
-//                grew by more than 2^8 (exact: O and l carry the same stale m), and at the
-//                end of the item write their quarter of O / l (and LSE = ln2 * (m + log2 l)).
+//   warp 10      TMA producer: Q_A, Q_B per item, then K_j and V_j through two rings of
+//                shared-memory stages (128-byte swizzle), guarded by full/empty mbarriers.
+//   warps 8, 9   MMA issuers (one thread each), for stream A and B: per key tile j,
+//                S_s = Q_s K_j^T, and O_s += P_s V_j once P_s is published; S_s of the
+//                next tile reuses the same TMEM columns once that product has completed.
+//   warps 0..3   softmax of stream A, warps 4..7 of stream B: thread r owns query row r
+//                of its tile (TMEM lane r) and all 128 scores of it. Per key tile it
+//                updates the running max m and sum l (page "告别OOM和训练慢…" §2.2),
+//                rescales its row of O when m grew by more than 2^8 (exact: O and l carry
+//                the same stale m), and writes P = exp2(s*scale*log2e - m) in bf16 to
+//                TMEM, where the P V product reads it. The two streams take turns on the
+//                exponentials. At the end of an item it writes O / l and
+//                LSE = ln2 * (m + log2 l).
 //
-// TMEM: S0, S1 (128 columns each), O (head_dim columns), P (64 columns).
+// TMEM: S_A (128 columns), S_B (128), O_A (head_dim), O_B (head_dim), and for head_dim 64
+// P_A, P_B (64 each); for head_dim 128 P_s goes over the first half of S_s.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -35,7 +39,8 @@ struct FwdArgs {
   int N;
   int BH;
   int n_qtiles;
-  int n_items;        // BH * n_qtiles
+  int n_pairs;        // items per (batch, head): query tiles taken two at a time
+  int n_items;        // BH * n_pairs
   int longest_first;  // masked problems: chunks of `group` heads, longest items first
   int group;
   float scale_log2;   // scale * log2(e)
@@ -50,62 +55,115 @@ struct FwdCfg {
   static constexpr int kTile = kBlock * D * 2;  // bytes of a 128 x D bf16 tile
   static constexpr int kRegions = D / 64;       // 128-byte-wide column regions per tile
   static constexpr int kRegionBytes = kBlock * 128;
-  static constexpr int kStages = (D == 64) ? 4 : 2;
+  static constexpr int kStagesK = (D == 64) ? 4 : 2;
+  static constexpr int kStagesV = (D == 64) ? 4 : 2;
   // shared memory map (offsets from a 1024-aligned base)
-  static constexpr int kQ = 0;                        // + (item & 1) * kTile
-  static constexpr int kK = kQ + 2 * kTile;           // + s * kTile
-  static constexpr int kV = kK + kStages * kTile;     // + s * kTile
-  static constexpr int kGroups = 4;                   // softmax warpgroups per row
-  static constexpr int kCols = kBlock / kGroups;      // score columns per thread
-  static constexpr int kOCols = D / kGroups;          // output columns per thread
-  static constexpr int kSoftmax = 128 * kGroups;      // softmax threads
-  static constexpr int kRed = kV + kStages * kTile;   // [2 slots][kGroups][128 rows] fp32
-  static constexpr int kBar = kRed + 2 * kGroups * kBlock * 4;
+  static constexpr int kQ = 0;                        // + stream * kTile
+  static constexpr int kK = kQ + 2 * kTile;           // + stage * kTile
+  static constexpr int kV = kK + kStagesK * kTile;    // + stage * kTile
+  static constexpr int kBar = kV + kStagesV * kTile;
   // barrier slots
-  static constexpr int bQFull = 0;                  // + (item & 1)
-  static constexpr int bQEmpty = 2;                 // + (item & 1)
-  static constexpr int bKFull = 4;
-  static constexpr int bKEmpty = bKFull + kStages;
-  static constexpr int bVFull = bKEmpty + kStages;
-  static constexpr int bVEmpty = bVFull + kStages;
-  static constexpr int bSFull = bVEmpty + kStages;  // + buffer
-  static constexpr int bSFree = bSFull + 2;         // + buffer
-  static constexpr int bRed = bSFree + 2;           // + slot
-  static constexpr int bPFull = bRed + 2;
-  static constexpr int bODone = bPFull + 1;
-  static constexpr int bOFree = bODone + 1;
-  static constexpr int bMmaFin = bOFree + 1;
-  static constexpr int kNumBars = bMmaFin + 1;
+  static constexpr int bQFull = 0;                  // + stream
+  static constexpr int bQEmpty = 2;                 // + stream
+  static constexpr int bKFull = 4;                  // + stage
+  static constexpr int bKEmpty = bKFull + kStagesK;
+  static constexpr int bVFull = bKEmpty + kStagesK;
+  static constexpr int bVEmpty = bVFull + kStagesV;
+  static constexpr int bSFull = bVEmpty + kStagesV;  // + stream: S_s computed
+  static constexpr int bPFull = bSFull + 2;          // + stream: P_s published (4 warps)
+  static constexpr int bODone = bPFull + 2;          // + stream: a P_s V product completed
+  static constexpr int bOFree = bODone + 2;          // + stream: O_s read by the epilogue
+  static constexpr int bSFree = bOFree + 2;          // + stream: S_s loaded (separate P)
+  static constexpr int bTurn = bSFree + 2;           // + stream: its turn on the exps
+  static constexpr int bMmaFin = bTurn + 2;          // + stream
+  static constexpr int kNumBars = bMmaFin + 2;
   static constexpr int kMisc = kBar + kNumBars * 8;  // TMEM base address (+0), abort flag (+4)
   static constexpr int kSmemBytes = kMisc + 16 + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
   // tensor memory columns (128 lanes each)
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t tS0 = 0;
-  static constexpr uint32_t tO = 256;
-  static constexpr uint32_t tP = 256 + D;
-  static constexpr int kThreads = kSoftmax + 64;  // softmax warps, MMA warp, producer warp
-  static constexpr int kWarpMma = 4 * kGroups;
-  static constexpr int kWarpProducer = 4 * kGroups + 1;
+  static constexpr uint32_t tS = 0;    // + 128 * stream
+  static constexpr uint32_t tO = 256;  // + D * stream
+  // With head_dim 64 there is room for P in its own columns: S_s of the next key tile may
+  // then be computed as soon as the softmax has loaded S_s, instead of waiting for the
+  // P V product that reads P from the columns of S_s.
+  static constexpr bool kSepP = (D == 64);
+  static constexpr uint32_t tP = 256 + 2 * D;  // + 64 * stream, when kSepP
+  static constexpr int kThreads = 352;  // 8 softmax warps, 2 MMA warps, producer warp
+  static constexpr int kWarpMma = 8;     // + stream
+  static constexpr int kWarpProducer = 10;
 };
 
+// One work item: query tiles m[0] = 2p and m[1] = 2p + 1 (absent past the last tile) of
+// one (batch, head), and the key tiles [lo[s], hi[s]] each of them sees. The producer
+// walks [first, last], the union (the ranges of consecutive query tiles overlap or touch).
 struct FwdItem {
   int bh;
-  int m;   // query tile
-  int lo;  // key tiles [lo, hi] it sees
-  int hi;
+  int m[2];
+  bool has_b;
+  int lo[2];
+  int hi[2];
+  int first;
+  int last;
 };
 
 __device__ __forceinline__ FwdItem fwd_item(int k, const FwdArgs& a) {
   FwdItem it;
+  int pair;
   if (a.longest_first) {
-    chunked_item(k, a.BH, a.n_qtiles, a.group, false, it.bh, it.m);
+    chunked_item(k, a.BH, a.n_pairs, a.group, false, it.bh, pair);
   } else {
-    it.bh = k / a.n_qtiles;
-    it.m = k % a.n_qtiles;
+    it.bh = k / a.n_pairs;
+    pair = k % a.n_pairs;
   }
   const Mask mk{a.N, a.left, a.right};
-  kv_tiles_for_q_tile(it.m, mk, it.lo, it.hi);
+  it.m[0] = 2 * pair;
+  it.m[1] = 2 * pair + 1;
+  it.has_b = it.m[1] < a.n_qtiles;
+  kv_tiles_for_q_tile(it.m[0], mk, it.lo[0], it.hi[0]);
+  if (it.has_b) {
+    kv_tiles_for_q_tile(it.m[1], mk, it.lo[1], it.hi[1]);
+  } else {
+    it.lo[1] = 1;
+    it.hi[1] = 0;
+  }
+  it.first = it.lo[0];
+  it.last = it.hi[0];
+  if (it.has_b) {
+    if (it.lo[1] < it.first) it.first = it.lo[1];
+    if (it.hi[1] > it.last) it.last = it.hi[1];
+  }
   return it;
+}
+
+// Stream s's query tile and key range of item `it`, as scalars (s need not be a constant).
+struct FwdRange {
+  bool has;  // stream s has a query tile in this item
+  int m;
+  int lo;
+  int hi;
+};
+
+__device__ __forceinline__ FwdRange fwd_range(const FwdItem& it, int s) {
+  FwdRange r;
+  r.has = s == 0 || it.has_b;
+  r.m = s ? it.m[1] : it.m[0];
+  r.lo = s ? it.lo[1] : it.lo[0];
+  r.hi = s ? it.hi[1] : it.hi[0];
+  return r;
+}
+
+// Local columns [c_lo, c_hi] of key tile j visible from query `row` (empty for rows past N).
+__device__ __forceinline__ void visible_cols(int row, int j, const Mask& mk, int& c_lo,
+                                             int& c_hi) {
+  const long long kb = (long long)j * kBlock;
+  long long lo = 0, hi = kBlock - 1;
+  if (mk.left >= 0 && row - mk.left - kb > lo) lo = row - mk.left - kb;
+  if (mk.right >= 0 && row + (long long)mk.right - kb < hi) hi = row + (long long)mk.right - kb;
+  if (mk.N - 1 - kb < hi) hi = mk.N - 1 - kb;
+  if (row >= mk.N) hi = -1;
+  c_lo = (int)(lo > kBlock ? kBlock : lo);
+  c_hi = (int)(hi < -1 ? -1 : hi);
 }
 
 template <int D>
@@ -123,29 +181,29 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
 
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
-  float* red = reinterpret_cast<float*>(smem + C::kRed);
   auto bar = [&](int i) -> uint32_t { return sb + C::kBar + 8u * i; };
 
   if (threadIdx.x == 0) {
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(C::bQFull + b), 1);
-      mbar_init(bar(C::bQEmpty + b), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(C::bQFull + s), 1);
+      mbar_init(bar(C::bQEmpty + s), 1);
+      mbar_init(bar(C::bSFull + s), 1);
+      mbar_init(bar(C::bPFull + s), 4);
+      mbar_init(bar(C::bODone + s), 1);
+      mbar_init(bar(C::bOFree + s), 4);
+      mbar_init(bar(C::bTurn + s), 4);
+      mbar_init(bar(C::bSFree + s), 4);
     }
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < C::kStagesK; ++s) {
       mbar_init(bar(C::bKFull + s), 1);
-      mbar_init(bar(C::bKEmpty + s), 1);
+      mbar_init(bar(C::bKEmpty + s), 2);  // one release per stream
+    }
+    for (int s = 0; s < C::kStagesV; ++s) {
       mbar_init(bar(C::bVFull + s), 1);
-      mbar_init(bar(C::bVEmpty + s), 1);
+      mbar_init(bar(C::bVEmpty + s), 2);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(C::bSFull + b), 1);
-      mbar_init(bar(C::bSFree + b), C::kSoftmax / 32);
-      mbar_init(bar(C::bRed + b), C::kSoftmax / 32);
-    }
-    mbar_init(bar(C::bPFull), C::kSoftmax / 32);
-    mbar_init(bar(C::bODone), 1);
-    mbar_init(bar(C::bOFree), C::kSoftmax / 32);
     mbar_init(bar(C::bMmaFin), 1);
+    mbar_init(bar(C::bMmaFin + 1), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -164,207 +222,248 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
       tma_prefetch_map(&tmQ);
       tma_prefetch_map(&tmK);
       tma_prefetch_map(&tmV);
-      int n_items_done = 0;
+      int nq[2] = {0, 0};  // Q loads per stream
       int kc = 0, vc = 0;  // K and V loads issued (ring positions)
       bool ok = true;
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         const FwdItem it = fwd_item(k, a);
-        // two Q buffers: the next item's Q streams in while this one is being processed
-        const int qb = n_items_done & 1;
-        if (!mbar_wait(bar(C::bQEmpty + qb), ((n_items_done >> 1) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::bQFull + qb), C::kTile);
-        for (int r = 0; r < C::kRegions; ++r)
-          tma_load_3d(sb + C::kQ + qb * C::kTile + r * C::kRegionBytes, &tmQ, bar(C::bQFull + qb),
-                      r * 64, it.m * kBlock, it.bh);
-        ++n_items_done;
-        for (int j = it.lo; j <= it.hi; ++j) {
-          const int s = kc % C::kStages;
-          if (!mbar_wait(bar(C::bKEmpty + s), ((kc / C::kStages) & 1) ^ 1, abort_flag)) {
+        for (int s = 0; s < 2; ++s) {
+          if (s == 1 && !it.has_b) break;
+          // Q_s of this item replaces the previous item's once its last S_s has been read
+          if (!mbar_wait(bar(C::bQEmpty + s), (nq[s] & 1) ^ 1, abort_flag)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(bar(C::bKFull + s), C::kTile);
+          mbar_arrive_expect_tx(bar(C::bQFull + s), C::kTile);
           for (int r = 0; r < C::kRegions; ++r)
-            tma_load_3d(sb + C::kK + s * C::kTile + r * C::kRegionBytes, &tmK, bar(C::bKFull + s),
-                        r * 64, j * kBlock, it.bh);
+            tma_load_3d(sb + C::kQ + s * C::kTile + r * C::kRegionBytes, &tmQ, bar(C::bQFull + s),
+                        r * 64, it.m[s] * kBlock, it.bh);
+          ++nq[s];
+        }
+        for (int j = it.first; ok && j <= it.last; ++j) {
+          const int sk = kc % C::kStagesK;
+          if (!mbar_wait(bar(C::bKEmpty + sk), ((kc / C::kStagesK) & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(C::bKFull + sk), C::kTile);
+          for (int r = 0; r < C::kRegions; ++r)
+            tma_load_3d(sb + C::kK + sk * C::kTile + r * C::kRegionBytes, &tmK,
+                        bar(C::bKFull + sk), r * 64, j * kBlock, it.bh);
           ++kc;
           if (a.fault == 1) continue;
-          if (!mbar_wait(bar(C::bVEmpty + s), ((vc / C::kStages) & 1) ^ 1, abort_flag)) {
+          const int sv = vc % C::kStagesV;
+          if (!mbar_wait(bar(C::bVEmpty + sv), ((vc / C::kStagesV) & 1) ^ 1, abort_flag)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(bar(C::bVFull + s), C::kTile);
+          mbar_arrive_expect_tx(bar(C::bVFull + sv), C::kTile);
           for (int r = 0; r < C::kRegions; ++r)
-            tma_load_3d(sb + C::kV + s * C::kTile + r * C::kRegionBytes, &tmV, bar(C::bVFull + s),
-                        r * 64, j * kBlock, it.bh);
+            tma_load_3d(sb + C::kV + sv * C::kTile + r * C::kRegionBytes, &tmV,
+                        bar(C::bVFull + sv), r * 64, j * kBlock, it.bh);
           ++vc;
         }
       }
       // Drain: every copy issued must have landed before the CTA may exit.
-      for (int n = (n_items_done > 2 ? n_items_done - 2 : 0); n < n_items_done; ++n)
-        mbar_wait(bar(C::bQFull + (n & 1)), (n >> 1) & 1, nullptr);
-      for (int s = 0; s < C::kStages; ++s) {
+      for (int s = 0; s < 2; ++s)
+        if (nq[s] > 0) mbar_wait(bar(C::bQFull + s), (nq[s] - 1) & 1, nullptr);
+      for (int s = 0; s < C::kStagesK; ++s) {
         if (kc > s) {
-          const int last = s + C::kStages * ((kc - 1 - s) / C::kStages);
-          mbar_wait(bar(C::bKFull + s), (last / C::kStages) & 1, nullptr);
+          const int last = s + C::kStagesK * ((kc - 1 - s) / C::kStagesK);
+          mbar_wait(bar(C::bKFull + s), (last / C::kStagesK) & 1, nullptr);
         }
+      }
+      for (int s = 0; s < C::kStagesV; ++s) {
         if (vc > s) {
-          const int last = s + C::kStages * ((vc - 1 - s) / C::kStages);
-          mbar_wait(bar(C::bVFull + s), (last / C::kStages) & 1, nullptr);
+          const int last = s + C::kStagesV * ((vc - 1 - s) / C::kStagesV);
+          mbar_wait(bar(C::bVFull + s), (last / C::kStagesV) & 1, nullptr);
         }
       }
     }
     __syncwarp();
-  } else if (warp == C::kWarpMma) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == C::kWarpMma || warp == C::kWarpMma + 1) {
+    // ------------------------------------------------------------------ MMA issuers
+    // One issuing thread per stream, so that a stream whose softmax is late never holds
+    // up the other's products (issuing a product group occupies its thread for about as
+    // long as the tensor core takes to run it). Each steps through every K/V ring position
+    // of every item in order, issuing S or P V where its query tile sees the key tile and
+    // only passing where it does not; a ring slot is released by one arrival per stream.
     if (lane == 0) {
+      const int s = warp - C::kWarpMma;
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);
-      int n_items_done = 0;
-      int kc = 0, vc = 0;  // ring positions consumed
-      int ns = 0, npv = 0; // S and P V products issued (all items)
+      int nq = 0;     // Q tiles consumed
+      int nsi = 0;    // S products issued (all items)
+      int npv = 0;    // P V products issued (all items)
+      int nitem = 0;  // items whose last P V has been issued
+      int pos = 0;    // K/V ring position
       bool ok = true;
-
-      // S_j = Q K_j^T into buffer ns & 1; after the item's last S, its Q may be replaced.
-      auto issue_s = [&](int j, int hi, int qb) -> bool {
-        const int s = kc % C::kStages;
-        const int b = ns & 1;
-        if (!mbar_wait(bar(C::bKFull + s), (kc / C::kStages) & 1, abort_flag)) return false;
-        ++kc;
-        // buffer b is free once every softmax warpgroup has read the S it held before
-        if (ns >= 2 && !mbar_wait(bar(C::bSFree + b), ((ns >> 1) - 1) & 1, abort_flag))
-          return false;
-        tc_fence_after();
+      // K step of key tile j (ring position p): S_s = Q_s K_j^T if the stream sees j
+      auto k_step = [&](const FwdItem& it, const FwdRange& rg, int j, int p) -> bool {
+        const bool sees = rg.has && rg.lo <= j && j <= rg.hi;
+        const bool first = j == rg.lo;
+        const int sk = p % C::kStagesK;
+        if (!mbar_wait(bar(C::bKFull + sk), (p / C::kStagesK) & 1, abort_flag)) return false;
+        if (sees) {
+          // S_s overwrites the stream's previous scores, which the softmax must have
+          // loaded, and (without separate P) P_s, whose P V must be complete
+          const bool free_s =
+              C::kSepP ? (nsi == 0 || mbar_wait(bar(C::bSFree + s), (nsi - 1) & 1, abort_flag))
+                       : (npv == 0 || mbar_wait(bar(C::bODone + s), (npv - 1) & 1, abort_flag));
+          if ((first && !mbar_wait(bar(C::bQFull + s), nq & 1, abort_flag)) || !free_s)
+            return false;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-          mma_ss(tmem + C::tS0 + 128u * b, sdesc_sw128(sb + C::kQ + qb * C::kTile + off, 16, 1024),
-                 sdesc_sw128(sb + C::kK + s * C::kTile + off, 16, 1024), idS, kk > 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
+            mma_ss(tmem + C::tS + 128u * s, sdesc_sw128(sb + C::kQ + s * C::kTile + off, 16, 1024),
+                   sdesc_sw128(sb + C::kK + sk * C::kTile + off, 16, 1024), idS, kk > 0);
+          }
+          tc_commit(bar(C::bSFull + s));
+          ++nsi;
+          if (first) ++nq;
+          if (j == rg.hi) tc_commit(bar(C::bQEmpty + s));  // last read of Q_s
         }
-        tc_commit(bar(C::bKEmpty + s));
-        tc_commit(bar(C::bSFull + b));
-        if (j == hi) tc_commit(bar(C::bQEmpty + qb));
-        ++ns;
+        tc_commit(bar(C::bKEmpty + sk));
         return true;
       };
-      // O += P_j V_j
-      auto issue_pv = [&](bool first, bool wait_o_free) -> bool {
-        const int s = vc % C::kStages;
-        if (!mbar_wait(bar(C::bVFull + s), (vc / C::kStages) & 1, abort_flag)) return false;
-        ++vc;
-        if (!mbar_wait(bar(C::bPFull), npv & 1, abort_flag)) return false;
-        // the first product of an item overwrites O: the previous epilogue must have read it
-        if (wait_o_free && !mbar_wait(bar(C::bOFree), (n_items_done - 2) & 1, abort_flag))
-          return false;
-        tc_fence_after();
+      // V step of key tile j (ring position p): O_s += P_s V_j if the stream sees j
+      auto v_step = [&](const FwdItem& it, const FwdRange& rg, int j, int p) -> bool {
+        const bool sees = rg.has && rg.lo <= j && j <= rg.hi;
+        const bool first = j == rg.lo;
+        const int sv = p % C::kStagesV;
+        if (!mbar_wait(bar(C::bVFull + sv), (p / C::kStagesV) & 1, abort_flag)) return false;
+        if (sees) {
+          // the first product of an item overwrites O_s: the previous epilogue must have
+          // read it
+          if (!mbar_wait(bar(C::bPFull + s), npv & 1, abort_flag) ||
+              (first && nitem > 0 && !mbar_wait(bar(C::bOFree + s), (nitem - 1) & 1, abort_flag)))
+            return false;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kBlock / 16; ++kk)
-          mma_ts(tmem + C::tO, tmem + C::tP + kk * 8,
-                 sdesc_sw128(sb + C::kV + s * C::kTile + kk * 2048, C::kRegionBytes, 1024), idO,
-                 (!first || kk > 0) ? 1u : 0u);
-        tc_commit(bar(C::bVEmpty + s));
-        tc_commit(bar(C::bODone));
-        ++npv;
+          for (int kk = 0; kk < kBlock / 16; ++kk)
+            mma_ts(tmem + C::tO + D * s,
+                   tmem + (C::kSepP ? C::tP + 64u * s : C::tS + 128u * s) + kk * 8,
+                   sdesc_sw128(sb + C::kV + sv * C::kTile + kk * 2048, C::kRegionBytes, 1024),
+                   idO, (!first || kk > 0) ? 1u : 0u);
+          tc_commit(bar(C::bODone + s));
+          ++npv;
+          if (j == rg.hi) ++nitem;
+        }
+        tc_commit(bar(C::bVEmpty + sv));
         return true;
       };
 
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         const FwdItem it = fwd_item(k, a);
-        const int qb = n_items_done & 1;
-        if (!mbar_wait(bar(C::bQFull + qb), (n_items_done >> 1) & 1, abort_flag)) break;
-        ++n_items_done;
-        ok = issue_s(it.lo, it.hi, qb);
-        for (int j = it.lo; ok && j <= it.hi; ++j) {
-          if (j + 1 <= it.hi) ok = issue_s(j + 1, it.hi, qb);
-          if (ok) ok = issue_pv(j == it.lo, j == it.lo && n_items_done > 1);
+        const FwdRange rg = fwd_range(it, s);
+        const int n = it.last - it.first + 1;
+        if (C::kSepP) {
+          // S one key tile ahead of P V: S_s(j+1) is computed while the softmax works on j
+          ok = k_step(it, rg, it.first, pos);
+          for (int t = 0; ok && t < n; ++t) {
+            if (t + 1 < n) ok = k_step(it, rg, it.first + t + 1, pos + t + 1);
+            if (ok) ok = v_step(it, rg, it.first + t, pos + t);
+          }
+        } else {
+          for (int t = 0; ok && t < n; ++t) {
+            ok = k_step(it, rg, it.first + t, pos + t);
+            if (ok) ok = v_step(it, rg, it.first + t, pos + t);
+          }
         }
+        pos += n;
       }
-      // Wait for every MMA issued so far before the CTA may release tensor memory.
-      tc_commit(bar(C::bMmaFin));
-      mbar_wait(bar(C::bMmaFin), 0, nullptr);
+      // Wait for every MMA this thread issued before the CTA may release tensor memory.
+      tc_commit(bar(C::bMmaFin + s));
+      mbar_wait(bar(C::bMmaFin + s), 0, nullptr);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ softmax warps
-    constexpr int G = C::kGroups, NC = C::kCols, NO = C::kOCols;
-    const int h = warp >> 2;                     // column group: keys NC*h .. NC*h+NC-1
+    const int s = warp >> 2;                     // stream: query tile A or B of the item
     const int r = threadIdx.x & 127;             // query row in the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tO = tmem + lane_base + C::tO + NO * h;
-    const uint32_t tP = tmem + lane_base + C::tP + (NC / 2) * h;
+    const uint32_t tS = tmem + lane_base + C::tS + 128u * s;
+    const uint32_t tP = C::kSepP ? tmem + lane_base + C::tP + 64u * s : tS;
+    const uint32_t tO = tmem + lane_base + C::tO + D * s;
     const float sl2 = a.scale_log2;
-    int ns = 0;  // S tiles consumed (all items)
-    int nx = 0;  // row-statistic exchanges between the warpgroups
+    int ns = 0;  // S tiles of this stream consumed (all items)
     bool ok = true;
 
-    // Shares a per-row value with the other warpgroups; `all` gets the G values of the row.
-    auto exchange = [&](float v, float (&all)[G]) -> bool {
-      float* slot = red + (nx & 1) * (G * 128);
-      slot[h * 128 + r] = v;
-      mbar_arrive_warp(bar(C::bRed + (nx & 1)));
-      if (!mbar_wait_warp(bar(C::bRed + (nx & 1)), (nx >> 1) & 1, abort_flag)) return false;
-#pragma unroll
-      for (int g = 0; g < G; ++g) all[g] = slot[g * 128 + r];
-      ++nx;
-      return true;
+    // When an item has both query tiles, the streams take turns on the exponentials of
+    // each key tile of the item (A first), so that one stream's exponentials run while the
+    // other loads and reduces its scores and the tensor core serves it. A stream that does
+    // not see a key tile only passes the turn on.
+    int nturn = 0;  // turns taken
+    if (s == 1) mbar_arrive_warp(bar(C::bTurn + 0));  // stream A starts
+    auto take_turn = [&]() -> bool {
+      const bool got = mbar_wait_warp(bar(C::bTurn + s), nturn & 1, abort_flag);
+      ++nturn;
+      return got;
     };
-    // NO accumulator columns of O: fp32 in, scaled by `mul`, back to TMEM (rescale)
-    auto scale_o = [&](float mul) {
-#pragma unroll
-      for (int q = 0; q < NO / 16; ++q) {
-        uint32_t o[16];
-        tmem_ld16(tO + 16 * q, o);
-        tmem_wait_ld();
-        reg_fence(o);
-#pragma unroll
-        for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * mul);
-        tmem_st16(tO + 16 * q, o);
-      }
-    };
+    auto pass_turn = [&]() { mbar_arrive_warp(bar(C::bTurn + (s ^ 1))); };
 
     for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
       const FwdItem it = fwd_item(k, a);
-      const int row = it.m * kBlock + r;
+      const FwdRange rg = fwd_range(it, s);
+      if (!rg.has) continue;
+      const bool turns = it.has_b;
+      const int row = rg.m * kBlock + r;
       float m_run = -INFINITY;  // running max of scale*log2e*s (the m that P and O carry)
-      float l_run = 0.f;        // this group's running sum of P
-      for (int j = it.lo; j <= it.hi; ++j) {
-        const int b = ns & 1;
-        if (!mbar_wait_warp(bar(C::bSFull + b), (ns >> 1) & 1, abort_flag)) {
+      float l_run = 0.f;        // running sum of P
+      for (int j = turns ? it.first : rg.lo; j <= (turns ? it.last : rg.hi); ++j) {
+        if (j < rg.lo || j > rg.hi) {
+          if (!take_turn()) {
+            ok = false;
+            break;
+          }
+          pass_turn();
+          continue;
+        }
+        if (!mbar_wait_warp(bar(C::bSFull + s), ns & 1, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        uint32_t u[32];
-        tmem_ld32(tmem + lane_base + C::tS0 + 128u * b + NC * h, u);
-        tmem_wait_ld();
-        reg_fence(u);
-        // this group's part of S_j is in registers: the tensor core may reuse the buffer
-        tc_fence_before();
-        mbar_arrive_warp(bar(C::bSFree + b));
-        float x[NC];
+        float x[kBlock];
+        {
+          uint32_t u[32];
 #pragma unroll
-        for (int c = 0; c < NC; ++c) x[c] = __uint_as_float(u[c]);
-        if (!tile_all_visible(it.m, j, mk)) {
+          for (int q = 0; q < 4; ++q) {
+            tmem_ld32(tS + 32 * q, u);
+            tmem_wait_ld();
+            reg_fence(u);
 #pragma unroll
-          for (int c = 0; c < NC; ++c)
-            if (!is_visible(row, j * kBlock + NC * h + c, mk)) x[c] = -INFINITY;
+            for (int c = 0; c < 32; ++c) x[32 * q + c] = __uint_as_float(u[c]);
+          }
         }
-        float mx8[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) mx8[c] = fmaxf(x[c], x[c + 8]);
-#pragma unroll
-        for (int c = 16; c < NC; c += 8)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], x[c + e]);
-        float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        float mx_all[G];
-        if (!exchange(mx, mx_all)) {
-          ok = false;
-          break;
+        if (C::kSepP) {
+          // S_s is in registers: the next key tile's S_s may overwrite it
+          tc_fence_before();
+          mbar_arrive_warp(bar(C::bSFree + s));
         }
+        if (!tile_all_visible(rg.m, j, mk)) {
+          int c_lo, c_hi;
+          visible_cols(row, j, mk, c_lo, c_hi);
 #pragma unroll
-        for (int g = 0; g < G; ++g) mx = fmaxf(mx, mx_all[g]);
+          for (int c = 0; c < kBlock; ++c) x[c] = (c >= c_lo && c <= c_hi) ? x[c] : -INFINITY;
+        }
+        float mx;
+        {
+          float t[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) t[e] = fmax3(x[e], x[e + 16], x[e + 32]);
+#pragma unroll
+          for (int c = 48; c < kBlock; c += 32)
+#pragma unroll
+            for (int e = 0; e < 16; ++e) t[e] = fmax3(t[e], x[c + e], x[c + 16 + e]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) t[e] = fmax3(t[e], t[e + 4], t[e + 8]);
+          // t[0..3] and t[12..15] remain
+          mx = fmax3(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[12], t[13]), fmaxf(t[14], t[15]));
+        }
+        // O_s is stable once the stream's previous P V product has completed: implied by
+        // S_full when P shares the columns of S_s, waited for below otherwise.
         const float m_new = fmaxf(m_run, mx * sl2);
         const bool grow = m_new > m_run + 8.0f;
         float alpha = 1.f;
@@ -374,72 +473,85 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
           l_run *= alpha;
         }
         const float mb = (m_run == -INFINITY) ? 0.f : m_run;
-        // this group's part of P = exp2(s*scale*log2e - m), packed to bf16 pairs
-        float ls4[4] = {0.f, 0.f, 0.f, 0.f};
-        uint32_t pk[NC / 2];
-#pragma unroll
-        for (int c = 0; c < NC / 2; ++c) {
-          const float p0 = ex2(fmaf(x[2 * c], sl2, -mb));
-          const float p1 = ex2(fmaf(x[2 * c + 1], sl2, -mb));
-          ls4[c & 3] += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
+        if (turns && !take_turn()) {
+          ok = false;
+          break;
         }
-        l_run += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
-        if (j > it.lo) {
-          // O and the P buffer are busy until P_{j-1} V_{j-1} has finished
-          if (!mbar_wait_warp(bar(C::bODone), (ns - 1) & 1, abort_flag)) {
+        // with separate P, P_s and O_s are free once the previous P V has completed
+        if (C::kSepP && ns > 0) {
+          if (!mbar_wait_warp(bar(C::bODone + s), (ns - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
         }
-        tmem_st16(tP, pk);
-        // rescale this group's part of O before P_j V_j accumulates into it (that waits
-        // for p_full)
-        if (j > it.lo && __any_sync(0xffffffffu, grow)) scale_o(alpha);
+        // P = exp2(s*scale*log2e - m) in bf16 pairs (over columns 0..63 of S_s without
+        // separate P)
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float p0 = ex2(fmaf(x[32 * h + 2 * c], sl2, -mb));
+            const float p1 = ex2(fmaf(x[32 * h + 2 * c + 1], sl2, -mb));
+            ls[c & 3] += p0 + p1;
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tP + 16 * h, pk);
+        }
+        if (turns) pass_turn();
+        l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        // rescale this row of O before P_s V_j accumulates into it (that waits for p_full)
+        if (j > rg.lo && __any_sync(0xffffffffu, grow)) {
+#pragma unroll
+          for (int q = 0; q < D / 32; ++q) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * q, o);
+            tmem_wait_ld();
+            reg_fence(o);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st32(tO + 32 * q, o);
+          }
+        }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive_warp(bar(C::bPFull));
+        mbar_arrive_warp(bar(C::bPFull + s));
         ++ns;
       }
       if (!ok) break;
-      // epilogue of the item: l of the whole row, then this group's part of O / l, and LSE
-      float l_all[G];
-      if (!exchange(l_run, l_all)) {
-        ok = false;
-        break;
-      }
-      float l_row = 0.f;
-#pragma unroll
-      for (int g = 0; g < G; ++g) l_row += l_all[g];
-      if (!mbar_wait_warp(bar(C::bODone), (ns - 1) & 1, abort_flag)) {
+      // epilogue of the item: O / l and LSE, once the last P V product has completed
+      if (!mbar_wait_warp(bar(C::bODone + s), (ns - 1) & 1, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float inv_l = (l_row > 0.f) ? 1.f / l_row : 0.f;
-      __nv_bfloat16* orow = a.o + ((size_t)it.bh * a.N + row) * D + NO * h;
+      const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+      __nv_bfloat16* orow = a.o + ((size_t)it.bh * a.N + (row < a.N ? row : 0)) * D;
 #pragma unroll
-      for (int q = 0; q < NO / 16; ++q) {
-        uint32_t o[16];
-        tmem_ld16(tO + 16 * q, o);
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * q, o);
         tmem_wait_ld();
         reg_fence(o);
-        uint32_t w[8];
+        uint32_t w[16];
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
+        for (int c = 0; c < 16; ++c)
           w[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
         if (row < a.N) {
-          st_global_v4(orow + 16 * q, w[0], w[1], w[2], w[3]);
-          st_global_v4(orow + 16 * q + 8, w[4], w[5], w[6], w[7]);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            st_global_v4(orow + 32 * q + 8 * v4, w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2],
+                         w[4 * v4 + 3]);
         }
       }
-      // O has been read: the next item's first P V may overwrite it
+      // O_s has been read: the next item's first P V may overwrite it
       tc_fence_before();
-      mbar_arrive_warp(bar(C::bOFree));
-      if (h == 0 && row < a.N)
+      mbar_arrive_warp(bar(C::bOFree + s));
+      if (row < a.N)
         a.lse[(size_t)it.bh * a.N + row] =
-            (l_row > 0.f) ? (m_run + log2f(l_row)) * 0.69314718055994531f : -INFINITY;
+            (l_run > 0.f) ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
     }
   }
 

@@ -71,6 +71,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
+// Non-blocking test: true if the phase of parity `parity` of barrier `bar` has completed.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Gives up a wait that ran out of time: raises the CTA's abort flag (so that its other
+// roles stop too) and records FA_ERR_TIMEOUT in the device status word.
+__device__ __forceinline__ void wait_timed_out(volatile int* abort_flag) {
+  if (abort_flag != nullptr) *abort_flag = 1;
+  atomicCAS(&g_fa_status, 0, kStatusTimeout);
+}
+
 // Waits until the phase of parity `parity` of barrier `bar` has completed.
 // Returns false, without waiting further, once `abort_flag` (shared memory) is set, or
 // after the time limit; in the latter case it sets the flag and the device status word
@@ -85,8 +105,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
     if ((n & 31u) == 0) {
       if (abort_flag != nullptr && *abort_flag) return false;
       if (global_ns() - t0 > kWaitLimitNs || n > kWaitLimitPolls) {
-        if (abort_flag != nullptr) *abort_flag = 1;
-        atomicCAS(&g_fa_status, 0, kStatusTimeout);
+        wait_timed_out(abort_flag);
         return false;
       }
     }
@@ -323,6 +342,13 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// max(a, b, c) in one instruction (three-input form of max.f32).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 // Two fp32 values rounded to nearest even into one bf16x2 word, `lo` in the low half.
