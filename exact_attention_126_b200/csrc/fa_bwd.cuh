@@ -23,9 +23,11 @@
 // In both kernels four warpgroups share every row: warpgroup h takes the 32 columns
 // 32h..32h+31 of it (query columns for dK/dV, key columns for dQ), so that four warps
 // per SM sub-partition hide each other's latencies. P needs no row maximum here (the
-// LSE is known), so the groups never wait for each other. The MMA issuer (warp 16;
-// warp 17 issues the TMA copies) orders the products so that the next tile's S and dP
-// are computed while the softmax warpgroups work on the current tile.
+// LSE is known), so the groups never wait for each other. Two MMA issuers (warps 16 and
+// 17; warp 18 issues the TMA copies) work side by side: one computes the score products
+// S and dP tile after tile, the other the gradient products as soon as the softmax
+// publishes P and dS. Issuing a product group occupies its thread for about as long as
+// the tensor core takes to run it, so one issuer for both would serialise them.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -128,9 +130,9 @@ struct BwdCfgT {
   static constexpr int bY0Empty = bY0Full + S0;
   static constexpr int bY1Full = bY0Empty + S0;
   static constexpr int bY1Empty = bY1Full + S1;
-  static constexpr int bA = bY1Empty + S1;  // 10 kernel-specific barriers
-  static constexpr int bMmaFin = bA + 10;
-  static constexpr int kNumBars = bMmaFin + 1;
+  static constexpr int bA = bY1Empty + S1;  // 12 kernel-specific barriers
+  static constexpr int bMmaFin = bA + 12;   // + issuer
+  static constexpr int kNumBars = bMmaFin + 2;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kSmemBytes = kMisc + 16 + 1024;
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
@@ -138,9 +140,9 @@ struct BwdCfgT {
   static constexpr int kGroups = 4;               // softmax warpgroups per row
   static constexpr int kCols = kBlock / kGroups;  // columns of a row per thread
   static constexpr int kSoftmax = 128 * kGroups;  // softmax threads
-  static constexpr int kThreads = kSoftmax + 64;  // softmax warps, MMA warp, producer warp
-  static constexpr int kWarpMma = 4 * kGroups;
-  static constexpr int kWarpProducer = 4 * kGroups + 1;
+  static constexpr int kThreads = kSoftmax + 96;  // softmax warps, 2 MMA warps, producer
+  static constexpr int kWarpMma = 4 * kGroups;    // + issuer: 0 = score products, 1 = gradients
+  static constexpr int kWarpProducer = 4 * kGroups + 2;
 };
 
 template <int D>
@@ -237,11 +239,13 @@ __device__ __forceinline__ void bwd_teardown(uint32_t tmem, int warp) {
 // ------------------------------------------------------------------------------------
 // dK, dV: persistent CTAs over items (batch*head, key tile j). X0 = K_j, X1 = V_j; per
 // stage Y0 = Q_i with the LSE (log2 units) and delta of its 128 rows, Y1 = dO_i.
-// TMEM: S^T at 0, dP^T at 128, dK at 256, dV at 256 + D. Warpgroup h writes its bf16
-// part of P^T (dS^T) over the first 16 of its own 32 fp32 columns of S^T (dP^T), so the
-// A operand of dV (dK) takes K-step kk from column packed_col(kk).
-// MMA order per query tile i:  dV(i), S^T(i+1), dK(i), dP^T(i+1). Tile counters (for
-// barrier parities) run over all items of the CTA.
+// TMEM: S^T in kSBufs buffers (two for head_dim 64, so that S^T of the next query tile
+// is computed while the softmax works on this one), dP^T, dK, dV. Warpgroup h writes its
+// bf16 part of P^T (dS^T) over the first 16 of its own 32 fp32 columns of S^T (dP^T), so
+// the A operand of dV (dK) takes K-step kk from column packed_col(kk).
+// Two MMA issuers: one computes S^T and dP^T of each query tile in order, the other
+// dV += P^T dO and dK += dS^T Q as soon as the softmax publishes P^T and dS^T. Tile
+// counters (for barrier parities) run over all items of the CTA.
 // ------------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
@@ -250,10 +254,15 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
                        const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmdO, const BwdArgs a) {
   using C = DkdvCfg<D>;
-  constexpr uint32_t tS = 0, tDP = 128, tDK = 256, tDV = 256 + D;
-  constexpr int bSFull = C::bA + 0, bDPFull = C::bA + 1, bPFull = C::bA + 2,
-                bDSFull = C::bA + 3, bDVDone = C::bA + 4, bDKDone = C::bA + 5,
-                bAccFree = C::bA + 6, bAccReady = C::bA + 7;
+  constexpr int kSBufs = (D == 64) ? 2 : 1;
+  constexpr uint32_t tS = 0;                         // + 128 * buffer
+  constexpr uint32_t tDP = 128 * kSBufs, tDK = tDP + 128, tDV = tDK + D;
+  static_assert(tDV + D <= C::kTmemCols, "tensor memory columns");
+  // per S^T buffer: S^T full, dV done (dV read that buffer's P^T); dP^T full, P^T full,
+  // dS^T full, dK done, dK/dV read by the epilogue, dK/dV of the item complete
+  constexpr int bSFull = C::bA + 0, bDVDone = C::bA + 2, bDPFull = C::bA + 4,
+                bPFull = C::bA + 5, bDSFull = C::bA + 6, bDKDone = C::bA + 7,
+                bAccFree = C::bA + 8, bAccReady = C::bA + 9;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -269,23 +278,27 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
       mbar_init(bar(C::bXFull + b), 1);
       mbar_init(bar(C::bXEmpty + b), 1);
     }
+    // Q_i (with its statistics) is read by S^T and dK, dO_i by dP^T and dV: one release
+    // from each issuer
     for (int s = 0; s < C::kStages0; ++s) {
       mbar_init(bar(C::bY0Full + s), 1);
-      mbar_init(bar(C::bY0Empty + s), 1);
+      mbar_init(bar(C::bY0Empty + s), 2);
     }
     for (int s = 0; s < C::kStages1; ++s) {
       mbar_init(bar(C::bY1Full + s), 1);
-      mbar_init(bar(C::bY1Empty + s), 1);
+      mbar_init(bar(C::bY1Empty + s), 2);
     }
-    mbar_init(bar(bSFull), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(bSFull + b), 1);
+      mbar_init(bar(bDVDone + b), 1);
+      mbar_init(bar(C::bMmaFin + b), 1);
+    }
     mbar_init(bar(bDPFull), 1);
     mbar_init(bar(bPFull), C::kSoftmax / 32);
     mbar_init(bar(bDSFull), C::kSoftmax / 32);
-    mbar_init(bar(bDVDone), 1);
     mbar_init(bar(bDKDone), 1);
     mbar_init(bar(bAccFree), C::kSoftmax / 32);
     mbar_init(bar(bAccReady), 1);
-    mbar_init(bar(C::bMmaFin), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -349,87 +362,93 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
     }
     __syncwarp();
   } else if (warp == C::kWarpMma) {
-    // ------------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------------ score products
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);
-      int items = 0, g = 0;  // items and query tiles done (all items)
+      int items = 0, t = 0;  // items and query tiles started (all items)
       bool ok = true;
-      // S^T = K_j Q_i^T (Q in ring-0 stage s) and dP^T = V_j dO_i^T (dO in ring-1 stage s)
-      auto issue_s = [&](int xb, int s) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-          mma_ss(tmem + tS, sdesc_sw128(sb + C::kX0 + xb * 2 * C::kTile + off, 16, 1024),
-                 sdesc_sw128(sb + C::kY0 + s * C::kTile + off, 16, 1024), idS, kk > 0);
-        }
-        tc_commit(bar(bSFull));
-      };
-      auto issue_dp = [&](int xb, int s) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-          mma_ss(tmem + tDP, sdesc_sw128(sb + C::kX1 + xb * 2 * C::kTile + off, 16, 1024),
-                 sdesc_sw128(sb + C::kY1 + s * C::kTile + off, 16, 1024), idS, kk > 0);
-        }
-        tc_commit(bar(bDPFull));
-      };
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, j;
         bwd_item(k, a, true, bh, j);
         int i_lo, i_hi;
         q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
-        const int n_it = i_hi - i_lo + 1;
         const int xb = items % C::kXBufs, xu = items / C::kXBufs;
         if (!mbar_wait(bar(C::bXFull + xb), xu & 1, abort_flag)) break;
-        // first tile of the item: S^T once dV of the previous tile has read P^T out of the
-        // S^T columns, dP^T once dK has read dS^T out of the dP^T columns
-        if (!mbar_wait(bar(C::bY0Full + g % C::kStages0), (g / C::kStages0) & 1, abort_flag) ||
-            (g > 0 && !mbar_wait(bar(bDVDone), (g - 1) & 1, abort_flag))) {
-          ok = false;
-          break;
+        for (int i = i_lo; i <= i_hi; ++i, ++t) {
+          const int b = t % kSBufs, s0 = t % C::kStages0, s1 = t % C::kStages1;
+          // S^T = K_j Q_i^T, once dV has read the P^T its buffer held
+          if (!mbar_wait(bar(C::bY0Full + s0), (t / C::kStages0) & 1, abort_flag) ||
+              (t >= kSBufs &&
+               !mbar_wait(bar(bDVDone + b), ((t / kSBufs) - 1) & 1, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
+            mma_ss(tmem + tS + 128u * b,
+                   sdesc_sw128(sb + C::kX0 + xb * 2 * C::kTile + off, 16, 1024),
+                   sdesc_sw128(sb + C::kY0 + s0 * C::kTile + off, 16, 1024), idS, kk > 0);
+          }
+          tc_commit(bar(bSFull + b));
+          tc_commit(bar(C::bY0Empty + s0));
+          // dP^T = V_j dO_i^T, once dK has read the dS^T of the previous tile
+          if (!mbar_wait(bar(C::bY1Full + s1), (t / C::kStages1) & 1, abort_flag) ||
+              (t >= 1 && !mbar_wait(bar(bDKDone), (t - 1) & 1, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
+            mma_ss(tmem + tDP, sdesc_sw128(sb + C::kX1 + xb * 2 * C::kTile + off, 16, 1024),
+                   sdesc_sw128(sb + C::kY1 + s1 * C::kTile + off, 16, 1024), idS, kk > 0);
+          }
+          tc_commit(bar(bDPFull));
+          tc_commit(bar(C::bY1Empty + s1));
+          if (i == i_hi) tc_commit(bar(C::bXEmpty + xb));  // last read of K_j, V_j
         }
-        tc_fence_after();
-        issue_s(xb, g % C::kStages0);
-        if (!mbar_wait(bar(C::bY1Full + g % C::kStages1), (g / C::kStages1) & 1, abort_flag) ||
-            (g > 0 && !mbar_wait(bar(bDKDone), (g - 1) & 1, abort_flag))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        issue_dp(xb, g % C::kStages1);
-        if (n_it == 1) tc_commit(bar(C::bXEmpty + xb));  // K_j, V_j read for the last time
-        for (int it = 0; it < n_it; ++it) {
-          const int t = g + it;
-          const int s0 = t % C::kStages0, s1 = t % C::kStages1;
-          const bool more = it + 1 < n_it;
-          // dV += P^T dO_i; dO_i is then free. The item's first product overwrites dV,
-          // which the previous item's epilogue must have read.
-          if (!mbar_wait(bar(bPFull), t & 1, abort_flag) ||
-              (it == 0 && items > 0 && !mbar_wait(bar(bAccFree), (items - 1) & 1, abort_flag))) {
+        ++items;
+      }
+      tc_commit(bar(C::bMmaFin));
+      mbar_wait(bar(C::bMmaFin), 0, nullptr);
+    }
+    __syncwarp();
+  } else if (warp == C::kWarpMma + 1) {
+    // ------------------------------------------------------------------ dV, dK products
+    if (lane == 0) {
+      constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);
+      int items = 0, t = 0;
+      bool ok = true;
+      for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
+        int bh, j;
+        bwd_item(k, a, true, bh, j);
+        int i_lo, i_hi;
+        q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
+        for (int i = i_lo; i <= i_hi; ++i, ++t) {
+          const int b = t % kSBufs, s0 = t % C::kStages0, s1 = t % C::kStages1;
+          const bool first = i == i_lo;
+          // dV += P^T dO_i; the item's first product overwrites dV, which the previous
+          // item's epilogue must have read
+          if (!mbar_wait(bar(C::bY1Full + s1), (t / C::kStages1) & 1, abort_flag) ||
+              !mbar_wait(bar(bPFull), t & 1, abort_flag) ||
+              (first && items > 0 && !mbar_wait(bar(bAccFree), (items - 1) & 1, abort_flag))) {
             ok = false;
             break;
           }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kBlock / 16; ++kk)
-            mma_ts(tmem + tDV, tmem + tS + packed_col(kk),
+            mma_ts(tmem + tDV, tmem + tS + 128u * b + packed_col(kk),
                    sdesc_sw128(sb + C::kY1 + s1 * C::kTile + kk * 2048, C::kRegionBytes, 1024),
-                   idA, (it > 0 || kk > 0) ? 1u : 0u);
+                   idA, (!first || kk > 0) ? 1u : 0u);
           tc_commit(bar(C::bY1Empty + s1));
-          tc_commit(bar(bDVDone));
-          if (more) {
-            const int u0 = (t + 1) % C::kStages0;
-            if (!mbar_wait(bar(C::bY0Full + u0), ((t + 1) / C::kStages0) & 1, abort_flag) ||
-                !mbar_wait(bar(bDVDone), t & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            issue_s(xb, u0);
-          }
-          // dK += dS^T Q_i; Q_i and its row statistics are then free
-          if (!mbar_wait(bar(bDSFull), t & 1, abort_flag)) {
+          tc_commit(bar(bDVDone + b));
+          // dK += dS^T Q_i
+          if (!mbar_wait(bar(C::bY0Full + s0), (t / C::kStages0) & 1, abort_flag) ||
+              !mbar_wait(bar(bDSFull), t & 1, abort_flag)) {
             ok = false;
             break;
           }
@@ -438,27 +457,15 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
           for (int kk = 0; kk < kBlock / 16; ++kk)
             mma_ts(tmem + tDK, tmem + tDP + packed_col(kk),
                    sdesc_sw128(sb + C::kY0 + s0 * C::kTile + kk * 2048, C::kRegionBytes, 1024),
-                   idA, (it > 0 || kk > 0) ? 1u : 0u);
+                   idA, (!first || kk > 0) ? 1u : 0u);
           tc_commit(bar(C::bY0Empty + s0));
           tc_commit(bar(bDKDone));
-          if (!more) tc_commit(bar(bAccReady));  // dK, dV of the item are complete
-          if (more) {
-            const int u1 = (t + 1) % C::kStages1;
-            if (!mbar_wait(bar(C::bY1Full + u1), ((t + 1) / C::kStages1) & 1, abort_flag) ||
-                !mbar_wait(bar(bDKDone), t & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            issue_dp(xb, u1);
-            if (it + 2 == n_it) tc_commit(bar(C::bXEmpty + xb));  // last read of K_j, V_j
-          }
+          if (i == i_hi) tc_commit(bar(bAccReady));  // dK, dV of the item are complete
         }
-        g += n_it;
         ++items;
       }
-      tc_commit(bar(C::bMmaFin));
-      mbar_wait(bar(C::bMmaFin), 0, nullptr);
+      tc_commit(bar(C::bMmaFin + 1));
+      mbar_wait(bar(C::bMmaFin + 1), 0, nullptr);
     }
     __syncwarp();
   } else {
@@ -482,7 +489,7 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
         const int t = g + it;
         const int s = t % C::kStages0;
         if (!mbar_wait_warp(bar(C::bY0Full + s), (t / C::kStages0) & 1, abort_flag) ||
-            !mbar_wait_warp(bar(bSFull), t & 1, abort_flag)) {
+            !mbar_wait_warp(bar(bSFull + t % kSBufs), (t / kSBufs) & 1, abort_flag)) {
           ok = false;
           break;
         }
@@ -490,7 +497,8 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
         const float* lse_s = reinterpret_cast<const float*>(smem + C::kLse + s * 512) + NC * h;
         const float* del_s = reinterpret_cast<const float*>(smem + C::kDelta + s * 512) + NC * h;
         float p[NC];
-        load_cols32(tmem + lane_base + tS + NC * h, p);
+        const uint32_t tSb = tmem + lane_base + tS + 128u * (t % kSBufs) + NC * h;
+        load_cols32(tSb, p);
 #pragma unroll
         for (int r = 0; r < NC; r += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse_s + r);
@@ -500,15 +508,16 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
           p[r + 3] = ex2(fmaf(p[r + 3], sl2, -l4.w));
         }
         if (!tile_all_visible(i, j, mk)) {
+          int r_lo, r_hi;
+          visible_queries(c, (long long)i * kBlock + NC * h, NC, mk, r_lo, r_hi);
 #pragma unroll
-          for (int r = 0; r < NC; ++r)
-            if (!is_visible(i * kBlock + NC * h + r, c, mk)) p[r] = 0.f;
+          for (int r = 0; r < NC; ++r) p[r] = (r >= r_lo && r <= r_hi) ? p[r] : 0.f;
         }
         {
           uint32_t pk[NC / 2];
 #pragma unroll
           for (int r = 0; r < NC / 2; ++r) pk[r] = pack_bf16x2(p[2 * r], p[2 * r + 1]);
-          tmem_st16(tmem + lane_base + tS + NC * h, pk);
+          tmem_st16(tSb, pk);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -559,8 +568,9 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
 // ------------------------------------------------------------------------------------
 // dQ: persistent CTAs over items (batch*head, query tile i). X0 = Q_i, X1 = dO_i; per
 // stage Y0 = K_j, Y1 = V_j. TMEM: S in two buffers at 0 and 128 (bf16 dS goes over S,
-// each warpgroup over the first half of its own 32 columns), dP at 256, dQ at 384. MMA
-// order per key tile j: S(j+1), dP(j+1), dQ(j). Tile counters run over all items.
+// each warpgroup over the first half of its own 32 columns), dP at 256, dQ at 384. Two
+// MMA issuers: one computes S and dP of each key tile in order, the other dQ += dS K_j
+// as soon as the softmax publishes dS. Tile counters run over all items.
 // ------------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
@@ -589,9 +599,10 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
       mbar_init(bar(C::bXFull + b), 1);
       mbar_init(bar(C::bXEmpty + b), 1);
     }
+    // K_j is read by S and dQ: one release from each issuer
     for (int s = 0; s < C::kStages0; ++s) {
       mbar_init(bar(C::bY0Full + s), 1);
-      mbar_init(bar(C::bY0Empty + s), 1);
+      mbar_init(bar(C::bY0Empty + s), 2);
     }
     for (int s = 0; s < C::kStages1; ++s) {
       mbar_init(bar(C::bY1Full + s), 1);
@@ -601,12 +612,12 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
       mbar_init(bar(bSFull + b), 1);
       mbar_init(bar(bDSFull + b), C::kSoftmax / 32);
       mbar_init(bar(bDQDone + b), 1);
+      mbar_init(bar(C::bMmaFin + b), 1);
     }
     mbar_init(bar(bDPFull), 1);
     mbar_init(bar(bDPFree), C::kSoftmax / 32);
     mbar_init(bar(bAccFree), C::kSoftmax / 32);
     mbar_init(bar(bAccReady), 1);
-    mbar_init(bar(C::bMmaFin), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -664,73 +675,78 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
     }
     __syncwarp();
   } else if (warp == C::kWarpMma) {
+    // ------------------------------------------------------------------ S, dP products
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);
-      int items = 0, g = 0;
+      int items = 0, t = 0;
       bool ok = true;
-      // S(t) = Q_i K_j^T into buffer t & 1 (K in ring-0 stage t % S0); its buffer held
-      // dS(t-2), which dQ(t-2) must have read. dQ completions are counted per buffer, so
-      // the next completion of that barrier (dQ(t)) cannot come before this S(t).
-      auto issue_s = [&](int xb, int t) -> bool {
-        const int s = t % C::kStages0;
-        if (!mbar_wait(bar(C::bY0Full + s), (t / C::kStages0) & 1, abort_flag)) return false;
-        if (t >= 2 && !mbar_wait(bar(bDQDone + (t & 1)), ((t >> 1) - 1) & 1, abort_flag))
-          return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-          mma_ss(tmem + tS0 + 128u * (t & 1),
-                 sdesc_sw128(sb + C::kX0 + xb * 2 * C::kTile + off, 16, 1024),
-                 sdesc_sw128(sb + C::kY0 + s * C::kTile + off, 16, 1024), idS, kk > 0);
-        }
-        tc_commit(bar(bSFull + (t & 1)));
-        return true;
-      };
-      // dP(t) = dO_i V_j^T (V in ring-1 stage t % S1), once the softmax read dP(t-1); V_j
-      // is then free
-      auto issue_dp = [&](int xb, int t) -> bool {
-        const int s = t % C::kStages1;
-        if (!mbar_wait(bar(C::bY1Full + s), (t / C::kStages1) & 1, abort_flag)) return false;
-        if (t >= 1 && !mbar_wait(bar(bDPFree), (t - 1) & 1, abort_flag)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-          mma_ss(tmem + tDP, sdesc_sw128(sb + C::kX1 + xb * 2 * C::kTile + off, 16, 1024),
-                 sdesc_sw128(sb + C::kY1 + s * C::kTile + off, 16, 1024), idS, kk > 0);
-        }
-        tc_commit(bar(bDPFull));
-        tc_commit(bar(C::bY1Empty + s));
-        return true;
-      };
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, i;
         bwd_item(k, a, false, bh, i);
         int j_lo, j_hi;
         kv_tiles_for_q_tile(i, mk, j_lo, j_hi);
-        const int n_it = j_hi - j_lo + 1;
         const int xb = items % C::kXBufs, xu = items / C::kXBufs;
         if (!mbar_wait(bar(C::bXFull + xb), xu & 1, abort_flag)) break;
-        if (!issue_s(xb, g) || !issue_dp(xb, g)) {
-          ok = false;
-          break;
-        }
-        if (n_it == 1) tc_commit(bar(C::bXEmpty + xb));  // Q_i, dO_i read for the last time
-        for (int it = 0; it < n_it; ++it) {
-          const int t = g + it;
-          if (it + 1 < n_it) {
-            if (!issue_s(xb, t + 1) || !issue_dp(xb, t + 1)) {
-              ok = false;
-              break;
-            }
-            if (it + 2 == n_it) tc_commit(bar(C::bXEmpty + xb));
+        for (int jj = j_lo; jj <= j_hi; ++jj, ++t) {
+          const int s0 = t % C::kStages0, s1 = t % C::kStages1;
+          // S(t) = Q_i K_j^T into buffer t & 1, which held dS(t-2): dQ(t-2) must have read it
+          if (!mbar_wait(bar(C::bY0Full + s0), (t / C::kStages0) & 1, abort_flag) ||
+              (t >= 2 && !mbar_wait(bar(bDQDone + (t & 1)), ((t >> 1) - 1) & 1, abort_flag))) {
+            ok = false;
+            break;
           }
-          // dQ += dS K_j; K_j is then free. The item's first product overwrites dQ, which
-          // the previous item's epilogue must have read.
-          if (!mbar_wait(bar(bDSFull + (t & 1)), (t >> 1) & 1, abort_flag) ||
-              (it == 0 && items > 0 && !mbar_wait(bar(bAccFree), (items - 1) & 1, abort_flag))) {
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
+            mma_ss(tmem + tS0 + 128u * (t & 1),
+                   sdesc_sw128(sb + C::kX0 + xb * 2 * C::kTile + off, 16, 1024),
+                   sdesc_sw128(sb + C::kY0 + s0 * C::kTile + off, 16, 1024), idS, kk > 0);
+          }
+          tc_commit(bar(bSFull + (t & 1)));
+          tc_commit(bar(C::bY0Empty + s0));
+          // dP(t) = dO_i V_j^T, once the softmax has loaded dP(t-1); V_j is then free
+          if (!mbar_wait(bar(C::bY1Full + s1), (t / C::kStages1) & 1, abort_flag) ||
+              (t >= 1 && !mbar_wait(bar(bDPFree), (t - 1) & 1, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
+            mma_ss(tmem + tDP, sdesc_sw128(sb + C::kX1 + xb * 2 * C::kTile + off, 16, 1024),
+                   sdesc_sw128(sb + C::kY1 + s1 * C::kTile + off, 16, 1024), idS, kk > 0);
+          }
+          tc_commit(bar(bDPFull));
+          tc_commit(bar(C::bY1Empty + s1));
+          if (jj == j_hi) tc_commit(bar(C::bXEmpty + xb));  // last read of Q_i, dO_i
+        }
+        ++items;
+      }
+      tc_commit(bar(C::bMmaFin));
+      mbar_wait(bar(C::bMmaFin), 0, nullptr);
+    }
+    __syncwarp();
+  } else if (warp == C::kWarpMma + 1) {
+    // ------------------------------------------------------------------ dQ products
+    if (lane == 0) {
+      constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);
+      int items = 0, t = 0;
+      bool ok = true;
+      for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
+        int bh, i;
+        bwd_item(k, a, false, bh, i);
+        int j_lo, j_hi;
+        kv_tiles_for_q_tile(i, mk, j_lo, j_hi);
+        for (int jj = j_lo; jj <= j_hi; ++jj, ++t) {
+          const int s0 = t % C::kStages0;
+          const bool first = jj == j_lo;
+          // dQ += dS K_j; the item's first product overwrites dQ, which the previous
+          // item's epilogue must have read
+          if (!mbar_wait(bar(C::bY0Full + s0), (t / C::kStages0) & 1, abort_flag) ||
+              !mbar_wait(bar(bDSFull + (t & 1)), (t >> 1) & 1, abort_flag) ||
+              (first && items > 0 && !mbar_wait(bar(bAccFree), (items - 1) & 1, abort_flag))) {
             ok = false;
             break;
           }
@@ -738,18 +754,16 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kBlock / 16; ++kk)
             mma_ts(tmem + tDQ, tmem + tS0 + 128u * (t & 1) + packed_col(kk),
-                   sdesc_sw128(sb + C::kY0 + (t % C::kStages0) * C::kTile + kk * 2048,
-                               C::kRegionBytes, 1024),
-                   idA, (it > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(bar(C::bY0Empty + t % C::kStages0));
+                   sdesc_sw128(sb + C::kY0 + s0 * C::kTile + kk * 2048, C::kRegionBytes, 1024),
+                   idA, (!first || kk > 0) ? 1u : 0u);
+          tc_commit(bar(C::bY0Empty + s0));
           tc_commit(bar(bDQDone + (t & 1)));
-          if (it + 1 == n_it) tc_commit(bar(bAccReady));  // dQ of the item is complete
+          if (jj == j_hi) tc_commit(bar(bAccReady));  // dQ of the item is complete
         }
-        g += n_it;
         ++items;
       }
-      tc_commit(bar(C::bMmaFin));
-      mbar_wait(bar(C::bMmaFin), 0, nullptr);
+      tc_commit(bar(C::bMmaFin + 1));
+      mbar_wait(bar(C::bMmaFin + 1), 0, nullptr);
     }
     __syncwarp();
   } else {
@@ -785,9 +799,10 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < NC; ++c) p[c] = ex2(fmaf(p[c], sl2, -lse2));
         if (!tile_all_visible(i, jj, mk)) {
+          int c_lo, c_hi;
+          visible_keys(r, (long long)jj * kBlock + NC * h, NC, mk, c_lo, c_hi);
 #pragma unroll
-          for (int c = 0; c < NC; ++c)
-            if (!is_visible(r, jj * kBlock + NC * h + c, mk)) p[c] = 0.f;
+          for (int c = 0; c < NC; ++c) p[c] = (c >= c_lo && c <= c_hi) ? p[c] : 0.f;
         }
         if (!mbar_wait_warp(bar(bDPFull), t & 1, abort_flag)) {
           ok = false;

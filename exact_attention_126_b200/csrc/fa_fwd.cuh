@@ -58,14 +58,17 @@ struct FwdCfg {
   static constexpr int kStagesK = (D == 64) ? 4 : 2;
   static constexpr int kStagesV = (D == 64) ? 4 : 2;
   // shared memory map (offsets from a 1024-aligned base)
-  static constexpr int kQ = 0;                        // + stream * kTile
-  static constexpr int kK = kQ + 2 * kTile;           // + stage * kTile
+  // Q buffers per stream: with head_dim 64 two, so that the next item's Q_s loads while
+  // the current one is in use
+  static constexpr int kQBufs = (D == 64) ? 2 : 1;
+  static constexpr int kQ = 0;                        // + (stream * kQBufs + buffer) * kTile
+  static constexpr int kK = kQ + 2 * kQBufs * kTile;  // + stage * kTile
   static constexpr int kV = kK + kStagesK * kTile;    // + stage * kTile
   static constexpr int kBar = kV + kStagesV * kTile;
   // barrier slots
-  static constexpr int bQFull = 0;                  // + stream
-  static constexpr int bQEmpty = 2;                 // + stream
-  static constexpr int bKFull = 4;                  // + stage
+  static constexpr int bQFull = 0;                  // + stream * 2 + buffer
+  static constexpr int bQEmpty = 4;                 // + stream * 2 + buffer
+  static constexpr int bKFull = 8;                  // + stage
   static constexpr int bKEmpty = bKFull + kStagesK;
   static constexpr int bVFull = bKEmpty + kStagesK;
   static constexpr int bVEmpty = bVFull + kStagesV;
@@ -153,19 +156,6 @@ __device__ __forceinline__ FwdRange fwd_range(const FwdItem& it, int s) {
   return r;
 }
 
-// Local columns [c_lo, c_hi] of key tile j visible from query `row` (empty for rows past N).
-__device__ __forceinline__ void visible_cols(int row, int j, const Mask& mk, int& c_lo,
-                                             int& c_hi) {
-  const long long kb = (long long)j * kBlock;
-  long long lo = 0, hi = kBlock - 1;
-  if (mk.left >= 0 && row - mk.left - kb > lo) lo = row - mk.left - kb;
-  if (mk.right >= 0 && row + (long long)mk.right - kb < hi) hi = row + (long long)mk.right - kb;
-  if (mk.N - 1 - kb < hi) hi = mk.N - 1 - kb;
-  if (row >= mk.N) hi = -1;
-  c_lo = (int)(lo > kBlock ? kBlock : lo);
-  c_hi = (int)(hi < -1 ? -1 : hi);
-}
-
 template <int D>
 __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -185,8 +175,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(C::bQFull + s), 1);
-      mbar_init(bar(C::bQEmpty + s), 1);
+      mbar_init(bar(C::bQFull + 2 * s), 1);
+      mbar_init(bar(C::bQEmpty + 2 * s), 1);
+      mbar_init(bar(C::bQFull + 2 * s + 1), 1);
+      mbar_init(bar(C::bQEmpty + 2 * s + 1), 1);
       mbar_init(bar(C::bSFull + s), 1);
       mbar_init(bar(C::bPFull + s), 4);
       mbar_init(bar(C::bODone + s), 1);
@@ -230,13 +222,15 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         for (int s = 0; s < 2; ++s) {
           if (s == 1 && !it.has_b) break;
           // Q_s of this item replaces the previous item's once its last S_s has been read
-          if (!mbar_wait(bar(C::bQEmpty + s), (nq[s] & 1) ^ 1, abort_flag)) {
+          const int qb = 2 * s + nq[s] % C::kQBufs, qu = nq[s] / C::kQBufs;
+          if (!mbar_wait(bar(C::bQEmpty + qb), (qu & 1) ^ 1, abort_flag)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(bar(C::bQFull + s), C::kTile);
+          mbar_arrive_expect_tx(bar(C::bQFull + qb), C::kTile);
+          const int qslot = s * C::kQBufs + nq[s] % C::kQBufs;
           for (int r = 0; r < C::kRegions; ++r)
-            tma_load_3d(sb + C::kQ + s * C::kTile + r * C::kRegionBytes, &tmQ, bar(C::bQFull + s),
+            tma_load_3d(sb + C::kQ + qslot * C::kTile + r * C::kRegionBytes, &tmQ, bar(C::bQFull + qb),
                         r * 64, it.m[s] * kBlock, it.bh);
           ++nq[s];
         }
@@ -266,7 +260,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
       }
       // Drain: every copy issued must have landed before the CTA may exit.
       for (int s = 0; s < 2; ++s)
-        if (nq[s] > 0) mbar_wait(bar(C::bQFull + s), (nq[s] - 1) & 1, nullptr);
+        for (int n = (nq[s] > C::kQBufs ? nq[s] - C::kQBufs : 0); n < nq[s]; ++n)
+          mbar_wait(bar(C::bQFull + 2 * s + n % C::kQBufs), (n / C::kQBufs) & 1, nullptr);
       for (int s = 0; s < C::kStagesK; ++s) {
         if (kc > s) {
           const int last = s + C::kStagesK * ((kc - 1 - s) / C::kStagesK);
@@ -310,19 +305,25 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
           const bool free_s =
               C::kSepP ? (nsi == 0 || mbar_wait(bar(C::bSFree + s), (nsi - 1) & 1, abort_flag))
                        : (npv == 0 || mbar_wait(bar(C::bODone + s), (npv - 1) & 1, abort_flag));
-          if ((first && !mbar_wait(bar(C::bQFull + s), nq & 1, abort_flag)) || !free_s)
+          const int qb = 2 * s + nq % C::kQBufs;
+          if ((first && !mbar_wait(bar(C::bQFull + qb), (nq / C::kQBufs) & 1, abort_flag)) ||
+              !free_s)
             return false;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-            mma_ss(tmem + C::tS + 128u * s, sdesc_sw128(sb + C::kQ + s * C::kTile + off, 16, 1024),
+            mma_ss(tmem + C::tS + 128u * s,
+                   sdesc_sw128(sb + C::kQ + (s * C::kQBufs + nq % C::kQBufs) * C::kTile + off, 16,
+                               1024),
                    sdesc_sw128(sb + C::kK + sk * C::kTile + off, 16, 1024), idS, kk > 0);
           }
           tc_commit(bar(C::bSFull + s));
           ++nsi;
-          if (first) ++nq;
-          if (j == rg.hi) tc_commit(bar(C::bQEmpty + s));  // last read of Q_s
+          if (j == rg.hi) {
+            tc_commit(bar(C::bQEmpty + qb));  // last read of this Q_s buffer
+            ++nq;
+          }
         }
         tc_commit(bar(C::bKEmpty + sk));
         return true;
@@ -444,7 +445,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         }
         if (!tile_all_visible(rg.m, j, mk)) {
           int c_lo, c_hi;
-          visible_cols(row, j, mk, c_lo, c_hi);
+          visible_keys(row, (long long)j * kBlock, kBlock, mk, c_lo, c_hi);
 #pragma unroll
           for (int c = 0; c < kBlock; ++c) x[c] = (c >= c_lo && c <= c_hi) ? x[c] : -INFINITY;
         }

@@ -61,6 +61,33 @@ __host__ __device__ inline bool is_visible(int r, int c, const Mask& k) {
          (k.right < 0 || c - r <= k.right);
 }
 
+// Keys col_base + [c_lo, c_hi] of the `width` keys from col_base that query `row` sees
+// (c_lo > c_hi when none): the per-row form of is_visible, for masking a row of scores
+// with two compares per element.
+__host__ __device__ inline void visible_keys(int row, long long col_base, int width,
+                                             const Mask& k, int& c_lo, int& c_hi) {
+  long long lo = 0, hi = width - 1;
+  if (k.left >= 0 && row - k.left - col_base > lo) lo = row - k.left - col_base;
+  if (k.right >= 0 && row + (long long)k.right - col_base < hi) hi = row + (long long)k.right - col_base;
+  if (k.N - 1 - col_base < hi) hi = k.N - 1 - col_base;
+  if (row >= k.N) hi = -1;
+  c_lo = (int)(lo > width ? width : lo);
+  c_hi = (int)(hi < -1 ? -1 : hi);
+}
+
+// Queries row_base + [r_lo, r_hi] of the `width` queries from row_base that see key `col`
+// (r_lo > r_hi when none): the per-key form of is_visible.
+__host__ __device__ inline void visible_queries(int col, long long row_base, int width,
+                                                const Mask& k, int& r_lo, int& r_hi) {
+  long long lo = 0, hi = width - 1;
+  if (k.right >= 0 && col - k.right - row_base > lo) lo = col - k.right - row_base;
+  if (k.left >= 0 && col + (long long)k.left - row_base < hi) hi = col + (long long)k.left - row_base;
+  if (k.N - 1 - row_base < hi) hi = k.N - 1 - row_base;
+  if (col >= k.N) hi = -1;
+  r_lo = (int)(lo > width ? width : lo);
+  r_hi = (int)(hi < -1 ? -1 : hi);
+}
+
 // Work item k of a persistent schedule over BH heads of T tiles each, for masked problems
 // (tiles of different lengths). Heads go in chunks of `group` (chosen so that a chunk has
 // about one item per SM): every CTA works on a few heads at a time, whose K/V (or Q/dO)
