@@ -1,0 +1,88 @@
+// Host-side check of the tile and mask logic the kernels share (tiles.cuh), against
+// brute force over every (query, key) pair: the key-tile ranges of a query tile and the
+// query-tile ranges of a key tile hold exactly the tiles with a visible pair, the
+// per-row and per-key column ranges equal the element-wise visibility test, and the
+// chunked schedule visits every (head, tile) item exactly once. Prints "OK" or the first
+// mismatch and exits non-zero.
+#define __host__
+#define __device__
+#include <cstdio>
+#include <vector>
+#include "tiles.cuh"
+
+using namespace fa;
+
+static int fail(const char* what, int a, int b, int c, int d) {
+  std::printf("FAIL %s (%d %d %d %d)\n", what, a, b, c, d);
+  return 1;
+}
+
+static int check_mask(const Mask& mk) {
+  const int N = mk.N, T = num_tiles(N);
+  for (int m = 0; m < T; ++m) {
+    int lo, hi;
+    kv_tiles_for_q_tile(m, mk, lo, hi);
+    for (int j = 0; j < T; ++j) {
+      bool any = false, all = true;
+      for (int r = m * kBlock; r < m * kBlock + kBlock; ++r)
+        for (int c = j * kBlock; c < j * kBlock + kBlock; ++c) {
+          const bool v = is_visible(r, c, mk);
+          any = any || v;
+          all = all && v;
+        }
+      if (any != (lo <= j && j <= hi)) return fail("kv_tiles_for_q_tile", N, mk.left, m, j);
+      if (all != tile_all_visible(m, j, mk)) return fail("tile_all_visible", N, mk.left, m, j);
+    }
+  }
+  for (int j = 0; j < T; ++j) {
+    int lo, hi;
+    q_tiles_for_kv_tile(j, mk, lo, hi);
+    for (int m = 0; m < T; ++m) {
+      bool any = false;
+      for (int r = m * kBlock; r < m * kBlock + kBlock && !any; ++r)
+        for (int c = j * kBlock; c < j * kBlock + kBlock && !any; ++c) any = is_visible(r, c, mk);
+      if (any != (lo <= m && m <= hi)) return fail("q_tiles_for_kv_tile", N, mk.left, j, m);
+    }
+  }
+  const int widths[3] = {32, 64, 128};
+  for (int w : widths)
+    for (int base = 0; base < T * kBlock; base += w)
+      for (int x = 0; x < T * kBlock; ++x) {
+        int lo, hi;
+        visible_keys(x, base, w, mk, lo, hi);
+        for (int c = 0; c < w; ++c)
+          if ((lo <= c && c <= hi) != is_visible(x, base + c, mk))
+            return fail("visible_keys", N, x, base, c);
+        visible_queries(x, base, w, mk, lo, hi);
+        for (int r = 0; r < w; ++r)
+          if ((lo <= r && r <= hi) != is_visible(base + r, x, mk))
+            return fail("visible_queries", N, x, base, r);
+      }
+  return 0;
+}
+
+int main() {
+  const int Ns[5] = {1, 127, 128, 300, 640};
+  const int windows[7][2] = {{-1, -1}, {-1, 0}, {0, 0}, {100, 0}, {0, 37}, {200, 129}, {5, -1}};
+  for (int N : Ns)
+    for (auto& w : windows) {
+      const Mask mk{N, w[0], w[1]};
+      if (check_mask(mk)) return 1;
+    }
+  for (int BH = 1; BH <= 7; ++BH)
+    for (int T = 1; T <= 9; ++T)
+      for (int group = 1; group <= BH; ++group)
+        for (int rising = 0; rising < 2; ++rising) {
+          std::vector<int> seen(BH * T, 0);
+          for (int k = 0; k < BH * T; ++k) {
+            int bh, tile;
+            chunked_item(k, BH, T, group, rising != 0, bh, tile);
+            if (bh < 0 || bh >= BH || tile < 0 || tile >= T) return fail("chunked_item range", BH, T, group, k);
+            ++seen[bh * T + tile];
+          }
+          for (int v : seen)
+            if (v != 1) return fail("chunked_item cover", BH, T, group, rising);
+        }
+  std::printf("OK\n");
+  return 0;
+}
