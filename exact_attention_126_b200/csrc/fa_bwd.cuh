@@ -258,11 +258,13 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
   constexpr uint32_t tS = 0;                         // + 128 * buffer
   constexpr uint32_t tDP = 128 * kSBufs, tDK = tDP + 128, tDV = tDK + D;
   static_assert(tDV + D <= C::kTmemCols, "tensor memory columns");
-  // per S^T buffer: S^T full, dV done (dV read that buffer's P^T); dP^T full, P^T full,
-  // dS^T full, dK done, dK/dV read by the epilogue, dK/dV of the item complete
-  constexpr int bSFull = C::bA + 0, bDVDone = C::bA + 2, bDPFull = C::bA + 4,
-                bPFull = C::bA + 5, bDSFull = C::bA + 6, bDKDone = C::bA + 7,
-                bAccFree = C::bA + 8, bAccReady = C::bA + 9;
+  // per S^T buffer: S^T full, P^T full, dV done (dV read that buffer's P^T); dP^T full,
+  // dS^T full, dK done, dK/dV read by the epilogue, dK/dV of the item complete. Every
+  // barrier that one side may complete twice before the other has waited once is kept
+  // per buffer, so that no parity wait can mistake a later phase for the one it wants.
+  constexpr int bSFull = C::bA + 0, bPFull = C::bA + 2, bDVDone = C::bA + 4,
+                bDPFull = C::bA + 6, bDSFull = C::bA + 7, bDKDone = C::bA + 8,
+                bAccFree = C::bA + 9, bAccReady = C::bA + 10;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -290,11 +292,11 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(bSFull + b), 1);
+      mbar_init(bar(bPFull + b), C::kSoftmax / 32);
       mbar_init(bar(bDVDone + b), 1);
       mbar_init(bar(C::bMmaFin + b), 1);
     }
     mbar_init(bar(bDPFull), 1);
-    mbar_init(bar(bPFull), C::kSoftmax / 32);
     mbar_init(bar(bDSFull), C::kSoftmax / 32);
     mbar_init(bar(bDKDone), 1);
     mbar_init(bar(bAccFree), C::kSoftmax / 32);
@@ -433,7 +435,7 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
           // dV += P^T dO_i; the item's first product overwrites dV, which the previous
           // item's epilogue must have read
           if (!mbar_wait(bar(C::bY1Full + s1), (t / C::kStages1) & 1, abort_flag) ||
-              !mbar_wait(bar(bPFull), t & 1, abort_flag) ||
+              !mbar_wait(bar(bPFull + b), (t / kSBufs) & 1, abort_flag) ||
               (first && items > 0 && !mbar_wait(bar(bAccFree), (items - 1) & 1, abort_flag))) {
             ok = false;
             break;
@@ -521,7 +523,7 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive_warp(bar(bPFull));
+        mbar_arrive_warp(bar(bPFull + t % kSBufs));
         if (!mbar_wait_warp(bar(bDPFull), t & 1, abort_flag)) {
           ok = false;
           break;
