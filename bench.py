@@ -34,6 +34,15 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 L2_BYTES = 126 * 1024 * 1024
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a kernel on a
+# workload, from one ncu capture of the kernels as they are now; an entry must be removed
+# when its kernel changes. Compulsory traffic of the dK/dV pass on c4 is 537 MB read
+# (Q, K, V, dO and the row statistics) and 268 MB written (dK, dV).
+MEASURED_TRAFFIC = {
+    ("c4_causal_b32h16n2048d64", "bwd_dkdv"): 787141120,
+}
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -294,7 +303,7 @@ def run_ours(args, w, rank, world, local_rank):
                     "peak_kind": "bf16 sustained (%s)" % peak_src,
                     "frac_of_burst": round(achieved / burst, 4),
                     "frac_of_datasheet": round(achieved / DATASHEET_BF16_TFLOPS, 4),
-                    "traffic": None}
+                    "traffic": MEASURED_TRAFFIC.get((w.name, dominant))}
     else:
         nbytes = w.bwd_bytes() if dominant.startswith("bwd") else w.fwd_bytes()
         achieved = 2 * w.tensor_bytes() / (dom_ms * 1e-3) / 1e9

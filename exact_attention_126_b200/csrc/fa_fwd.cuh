@@ -451,13 +451,17 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         }
         float mx;
         {
+          // 16 partial maxima: x[0..47], then two columns at a time up to x[111], then x[112..127]
           float t[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) t[e] = fmax3(x[e], x[e + 16], x[e + 32]);
 #pragma unroll
-          for (int c = 48; c < kBlock; c += 32)
+          for (int c = 48; c + 32 <= kBlock; c += 32)
 #pragma unroll
             for (int e = 0; e < 16; ++e) t[e] = fmax3(t[e], x[c + e], x[c + 16 + e]);
+          static_assert(kBlock == 128, "the tail below covers columns 112..127");
+#pragma unroll
+          for (int e = 0; e < 16; ++e) t[e] = fmaxf(t[e], x[112 + e]);
 #pragma unroll
           for (int e = 0; e < 4; ++e) t[e] = fmax3(t[e], t[e + 4], t[e + 8]);
           // t[0..3] and t[12..15] remain

@@ -71,19 +71,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
-// Non-blocking test: true if the phase of parity `parity` of barrier `bar` has completed.
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-
 // Gives up a wait that ran out of time: raises the CTA's abort flag (so that its other
 // roles stop too) and records FA_ERR_TIMEOUT in the device status word.
 __device__ __forceinline__ void wait_timed_out(volatile int* abort_flag) {
@@ -119,27 +106,6 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
   const bool ok = mbar_wait(bar, parity, abort_flag);
   return __all_sync(0xffffffffu, ok);
 }
-
-// A shared-memory lock taken by lane 0 of a warp: used to let the two warps that share
-// an SM sub-partition take turns on its special-function unit. Bounded like mbar_wait.
-__device__ __forceinline__ bool smem_lock_acquire(int* lock, volatile int* abort_flag) {
-  if (atomicCAS(lock, 0, 1) == 0) return true;
-  const unsigned long long t0 = global_ns();
-  for (uint32_t n = 1;; ++n) {
-    __nanosleep(20);
-    if (atomicCAS(lock, 0, 1) == 0) return true;
-    if ((n & 15u) == 0) {
-      if (*abort_flag) return false;
-      if (global_ns() - t0 > kWaitLimitNs || n > kWaitLimitPolls) {
-        *abort_flag = 1;
-        atomicCAS(&g_fa_status, 0, kStatusTimeout);
-        return false;
-      }
-    }
-  }
-}
-
-__device__ __forceinline__ void smem_lock_release(int* lock) { atomicExch(lock, 0); }
 
 // ----------------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), no multicast
@@ -318,20 +284,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
 
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-// ----------------------------------------------------------------------------------
-// Register reallocation between warpgroups (all four warps of a warpgroup execute it).
-// The sum over warpgroups must not exceed the registers the CTA was launched with.
-// ----------------------------------------------------------------------------------
-template <int N>
-__device__ __forceinline__ void regs_grow() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-
-template <int N>
-__device__ __forceinline__ void regs_shrink() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ----------------------------------------------------------------------------------
