@@ -173,9 +173,10 @@ template <int D>
 fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void* dout,
                         const void* ws, void* dk, void* dv, int BH, int N,
                         float scale, int left, int right, cudaStream_t st) {
-  CUtensorMap mq, mkk, mv, mdo;
+  CUtensorMap mq, mkk, mv, mdo, mdk, mdv;
   if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
-      !make_map(&mv, v, BH, N, D) || !make_map(&mdo, dout, BH, N, D))
+      !make_map(&mv, v, BH, N, D) || !make_map(&mdo, dout, BH, N, D) ||
+      !make_map(&mdk, dk, BH, N, D) || !make_map(&mdv, dv, BH, N, D))
     return FA_ERR_CUDA;
   using C = fa::DkdvCfg<D>;
   if (set_smem(fa::fa_bwd_dkdv_kernel<D>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
@@ -183,8 +184,6 @@ fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void*
   a.stats = static_cast<const float*>(ws);
   a.stat_rows = (long long)BH * padded_rows(N);
   a.Np = padded_rows(N);
-  a.out0 = static_cast<__nv_bfloat16*>(dk);
-  a.out1 = static_cast<__nv_bfloat16*>(dv);
   a.N = N;
   a.n_tiles = fa::num_tiles(N);
   a.scale = scale;
@@ -196,7 +195,8 @@ fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void*
   a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
   a.group = head_group(BH, a.n_tiles);
   const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
-  fa::fa_bwd_dkdv_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, a);
+  fa::fa_bwd_dkdv_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, mdk, mdv,
+                                                                       a);
   return launched();
 }
 
@@ -204,9 +204,10 @@ template <int D>
 fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* dout,
                       const void* ws, void* dq, int BH, int N, float scale,
                       int left, int right, cudaStream_t st) {
-  CUtensorMap mq, mkk, mv, mdo;
+  CUtensorMap mq, mkk, mv, mdo, mdq;
   if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
-      !make_map(&mv, v, BH, N, D) || !make_map(&mdo, dout, BH, N, D))
+      !make_map(&mv, v, BH, N, D) || !make_map(&mdo, dout, BH, N, D) ||
+      !make_map(&mdq, dq, BH, N, D))
     return FA_ERR_CUDA;
   using C = fa::DqCfg<D>;
   if (set_smem(fa::fa_bwd_dq_kernel<D>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
@@ -214,8 +215,6 @@ fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* d
   a.stats = static_cast<const float*>(ws);
   a.stat_rows = (long long)BH * padded_rows(N);
   a.Np = padded_rows(N);
-  a.out0 = static_cast<__nv_bfloat16*>(dq);
-  a.out1 = nullptr;
   a.N = N;
   a.n_tiles = fa::num_tiles(N);
   a.scale = scale;
@@ -227,7 +226,7 @@ fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* d
   a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
   a.group = head_group(BH, a.n_tiles);
   const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
-  fa::fa_bwd_dq_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, a);
+  fa::fa_bwd_dq_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, mdq, a);
   return launched();
 }
 

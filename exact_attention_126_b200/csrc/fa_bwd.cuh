@@ -88,8 +88,6 @@ __global__ void __launch_bounds__(256)
 struct BwdArgs {
   const float* stats;   // row statistics written by fa_bwd_preprocess_kernel
   long long stat_rows;  // B*H*Np: offset of delta after LSE*log2e
-  __nv_bfloat16* out0;  // dkdv: dK ; dq: dQ
-  __nv_bfloat16* out1;  // dkdv: dV ; dq: unused
   int N;
   int Np;               // N rounded up to a multiple of 128
   int BH;
@@ -160,11 +158,14 @@ __device__ __forceinline__ void drain_ring(uint32_t full_bar0, int S, int n) {
   }
 }
 
-// Writes this thread's NC fp32 accumulator columns starting at `taddr`, times `mul`, as
-// bf16 to `dst` (16 columns, 32 bytes, per step).
+// Writes this thread's NC fp32 accumulator columns (columns col0 .. col0+NC-1 of row `row`
+// of a 128-row output tile), times `mul`, in bf16 to the shared-memory tile at `tile`, in
+// the layout a TMA load of the tile's 64-column boxes leaves (128-byte rows; 16-byte chunks
+// swizzled by the row's low three bits), ready for tma_store_3d. Writing the tile through
+// one bulk store keeps each warp's stores from touching 32 separate rows of global memory.
 template <int NC>
-__device__ __forceinline__ void store_acc_cols(uint32_t taddr, float mul, __nv_bfloat16* dst,
-                                               bool valid) {
+__device__ __forceinline__ void stage_acc_cols(uint32_t taddr, float mul, uint32_t tile, int row,
+                                               int col0) {
   static_assert(NC % 16 == 0, "whole 16-column steps");
 #pragma unroll
   for (int q = 0; q < NC / 16; ++q) {
@@ -176,9 +177,12 @@ __device__ __forceinline__ void store_acc_cols(uint32_t taddr, float mul, __nv_b
 #pragma unroll
     for (int c = 0; c < 8; ++c)
       w[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * mul, __uint_as_float(o[2 * c + 1]) * mul);
-    if (valid) {
-      st_global_v4(dst + 16 * q, w[0], w[1], w[2], w[3]);
-      st_global_v4(dst + 16 * q + 8, w[4], w[5], w[6], w[7]);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int col = col0 + 16 * q + 8 * k;
+      const uint32_t addr = tile + (uint32_t)(col >> 6) * (kBlock * 128) + (uint32_t)row * 128 +
+                            ((uint32_t)(((col & 63) >> 3) ^ (row & 7)) << 4);
+      st_shared_v4(addr, w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
     }
   }
 }
@@ -252,7 +256,9 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
     fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
-                       const __grid_constant__ CUtensorMap tmdO, const BwdArgs a) {
+                       const __grid_constant__ CUtensorMap tmdO,
+                       const __grid_constant__ CUtensorMap tmdK,
+                       const __grid_constant__ CUtensorMap tmdV, const BwdArgs a) {
   using C = DkdvCfg<D>;
   constexpr int kSBufs = (D == 64) ? 2 : 1;
   constexpr uint32_t tS = 0;                         // + 128 * buffer
@@ -264,7 +270,7 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
   // per buffer, so that no parity wait can mistake a later phase for the one it wants.
   constexpr int bSFull = C::bA + 0, bPFull = C::bA + 2, bDVDone = C::bA + 4,
                 bDPFull = C::bA + 6, bDSFull = C::bA + 7, bDKDone = C::bA + 8,
-                bAccFree = C::bA + 9, bAccReady = C::bA + 10;
+                bAccFree = C::bA + 9, bAccReady = C::bA + 10, bStaged = C::bA + 11;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -301,6 +307,7 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
     mbar_init(bar(bDKDone), 1);
     mbar_init(bar(bAccFree), C::kSoftmax / 32);
     mbar_init(bar(bAccReady), 1);
+    mbar_init(bar(bStaged), C::kSoftmax / 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -410,7 +417,6 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
           }
           tc_commit(bar(bDPFull));
           tc_commit(bar(C::bY1Empty + s1));
-          if (i == i_hi) tc_commit(bar(C::bXEmpty + xb));  // last read of K_j, V_j
         }
         ++items;
       }
@@ -552,17 +558,32 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
         ok = false;
         break;
       }
+      // dK and dV go through the item's K_j, V_j buffer, which no product reads any more,
+      // and leave in two bulk stores; the producer reuses the buffer once they have read it
+      const int xb = items % C::kXBufs;
+      const uint32_t tK = sb + C::kX0 + xb * 2 * C::kTile, tV = sb + C::kX1 + xb * 2 * C::kTile;
       ++items;
       tc_fence_after();
       constexpr int NO = D / C::kGroups;
-      const bool valid = c < a.N;
-      const size_t off = ((size_t)bh * a.N + (valid ? c : 0)) * D + NO * h;
-      store_acc_cols<NO>(tmem + lane_base + tDV + NO * h, 1.f, a.out1 + off, valid);
-      store_acc_cols<NO>(tmem + lane_base + tDK + NO * h, a.scale, a.out0 + off, valid);
+      stage_acc_cols<NO>(tmem + lane_base + tDV + NO * h, 1.f, tV, t_row, NO * h);
+      stage_acc_cols<NO>(tmem + lane_base + tDK + NO * h, a.scale, tK, t_row, NO * h);
+      fence_async_smem();
       // dK, dV have been read: the next item's first products may overwrite them
       tc_fence_before();
       mbar_arrive_warp(bar(bAccFree));
+      mbar_arrive_warp(bar(bStaged));
+      // (a failed wait has raised the abort flag: the whole warp then stops at its next wait)
+      if (threadIdx.x == 0 && mbar_wait(bar(bStaged), (items - 1) & 1, abort_flag)) {
+        for (int r = 0; r < C::kRegions; ++r) {
+          tma_store_3d(&tmdK, tK + r * C::kRegionBytes, r * 64, j * kBlock, bh);
+          tma_store_3d(&tmdV, tV + r * C::kRegionBytes, r * 64, j * kBlock, bh);
+        }
+        bulk_commit();
+        bulk_wait_read();
+        mbar_arrive(bar(C::bXEmpty + xb));
+      }
     }
+    if (threadIdx.x == 0) bulk_wait_all();
   }
   bwd_teardown<C>(tmem, warp);
 }
@@ -578,14 +599,15 @@ template <int D>
 __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
     fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV,
-                     const __grid_constant__ CUtensorMap tmdO, const BwdArgs a) {
+                     const __grid_constant__ CUtensorMap tmdO,
+                     const __grid_constant__ CUtensorMap tmdQ, const BwdArgs a) {
   using C = DqCfg<D>;
   constexpr uint32_t tS0 = 0, tDP = 256, tDQ = 384;
   // per S buffer: S full, dS full, dQ done (dQ read that buffer's dS); dP full, dP free;
   // dQ read by the epilogue, dQ of the item complete
   constexpr int bSFull = C::bA + 0, bDSFull = C::bA + 2, bDQDone = C::bA + 4,
                 bDPFull = C::bA + 6, bDPFree = C::bA + 7, bAccFree = C::bA + 8,
-                bAccReady = C::bA + 9;
+                bAccReady = C::bA + 9, bStaged = C::bA + 10;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -620,6 +642,7 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
     mbar_init(bar(bDPFree), C::kSoftmax / 32);
     mbar_init(bar(bAccFree), C::kSoftmax / 32);
     mbar_init(bar(bAccReady), 1);
+    mbar_init(bar(bStaged), C::kSoftmax / 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -722,7 +745,6 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
           }
           tc_commit(bar(bDPFull));
           tc_commit(bar(C::bY1Empty + s1));
-          if (jj == j_hi) tc_commit(bar(C::bXEmpty + xb));  // last read of Q_i, dO_i
         }
         ++items;
       }
@@ -783,7 +805,6 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
       kv_tiles_for_q_tile(i, mk, j_lo, j_hi);
       const int n_it = j_hi - j_lo + 1;
       const int r = i * kBlock + t_row;  // this thread's query row
-      const bool valid = r < a.N;
       // rows past N carry +inf and 0 in the padded statistics, which zero their P and dS
       const float lse2 = a.stats[(size_t)bh * a.Np + r];
       const float dl = a.stats[a.stat_rows + (size_t)bh * a.Np + r];
@@ -832,15 +853,29 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
         ok = false;
         break;
       }
+      // dQ goes through the item's Q_i buffer, which no product reads any more, and leaves
+      // in one bulk store; the producer reuses the buffer once it has been read
+      const int xb = items % C::kXBufs;
+      const uint32_t tQ = sb + C::kX0 + xb * 2 * C::kTile;
       ++items;
       tc_fence_after();
       constexpr int NO = D / C::kGroups;
-      const size_t off = ((size_t)bh * a.N + (valid ? r : 0)) * D + NO * h;
-      store_acc_cols<NO>(tmem + lane_base + tDQ + NO * h, a.scale, a.out0 + off, valid);
+      stage_acc_cols<NO>(tmem + lane_base + tDQ + NO * h, a.scale, tQ, t_row, NO * h);
+      fence_async_smem();
       // dQ has been read: the next item's first product may overwrite it
       tc_fence_before();
       mbar_arrive_warp(bar(bAccFree));
+      mbar_arrive_warp(bar(bStaged));
+      // (a failed wait has raised the abort flag: the whole warp then stops at its next wait)
+      if (threadIdx.x == 0 && mbar_wait(bar(bStaged), (items - 1) & 1, abort_flag)) {
+        for (int rg = 0; rg < C::kRegions; ++rg)
+          tma_store_3d(&tmdQ, tQ + rg * C::kRegionBytes, rg * 64, i * kBlock, bh);
+        bulk_commit();
+        bulk_wait_read();
+        mbar_arrive(bar(C::bXEmpty + xb));
+      }
     }
+    if (threadIdx.x == 0) bulk_wait_all();
   }
   bwd_teardown<C>(tmem, warp);
 }
