@@ -182,6 +182,8 @@ fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void*
   if (set_smem(fa::fa_bwd_dkdv_kernel<D>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
   fa::BwdArgs a;
   a.stats = static_cast<const float*>(ws);
+  a.out0 = static_cast<__nv_bfloat16*>(dk);
+  a.out1 = static_cast<__nv_bfloat16*>(dv);
   a.stat_rows = (long long)BH * padded_rows(N);
   a.Np = padded_rows(N);
   a.N = N;
@@ -213,6 +215,8 @@ fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* d
   if (set_smem(fa::fa_bwd_dq_kernel<D>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
   fa::BwdArgs a;
   a.stats = static_cast<const float*>(ws);
+  a.out0 = static_cast<__nv_bfloat16*>(dq);
+  a.out1 = nullptr;
   a.stat_rows = (long long)BH * padded_rows(N);
   a.Np = padded_rows(N);
   a.N = N;

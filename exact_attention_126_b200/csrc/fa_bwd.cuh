@@ -24,7 +24,7 @@
 // 32h..32h+31 of it (query columns for dK/dV, key columns for dQ), so that four warps
 // per SM sub-partition hide each other's latencies. P needs no row maximum here (the
 // LSE is known), so the groups never wait for each other. Two MMA issuers (warps 16 and
-// 17; warp 18 issues the TMA copies) work side by side: one computes the score products
+// 17; warp 18 issues the TMA loads, warp 19 the output stores) work side by side: one computes the score products
 // S and dP tile after tile, the other the gradient products as soon as the softmax
 // publishes P and dS. Issuing a product group occupies its thread for about as long as
 // the tensor core takes to run it, so one issuer for both would serialise them.
@@ -87,6 +87,8 @@ __global__ void __launch_bounds__(256)
 
 struct BwdArgs {
   const float* stats;   // row statistics written by fa_bwd_preprocess_kernel
+  __nv_bfloat16* out0;  // dkdv: dK ; dq: dQ (written directly when outputs are not staged)
+  __nv_bfloat16* out1;  // dkdv: dV
   long long stat_rows;  // B*H*Np: offset of delta after LSE*log2e
   int N;
   int Np;               // N rounded up to a multiple of 128
@@ -138,9 +140,14 @@ struct BwdCfgT {
   static constexpr int kGroups = 4;               // softmax warpgroups per row
   static constexpr int kCols = kBlock / kGroups;  // columns of a row per thread
   static constexpr int kSoftmax = 128 * kGroups;  // softmax threads
-  static constexpr int kThreads = kSoftmax + 96;  // softmax warps, 2 MMA warps, producer
-  static constexpr int kWarpMma = 4 * kGroups;    // + issuer: 0 = score products, 1 = gradients
+  static constexpr int kThreads = kSoftmax + 128;  // softmax, 2 MMA, producer, store warps
+  static constexpr int kWarpMma = 4 * kGroups;     // + issuer: 0 = score products, 1 = gradients
   static constexpr int kWarpProducer = 4 * kGroups + 2;
+  static constexpr int kWarpStore = 4 * kGroups + 3;  // bulk stores of the staged outputs
+  // Outputs are staged in the finished item's stationary buffer and leave by bulk stores
+  // when there are two such buffers; with one, waiting for the stores would hold up the
+  // next item's loads, so the softmax warps write their rows directly instead.
+  static constexpr bool kStageOut = XB >= 2;
 };
 
 template <int D>
@@ -183,6 +190,30 @@ __device__ __forceinline__ void stage_acc_cols(uint32_t taddr, float mul, uint32
       const uint32_t addr = tile + (uint32_t)(col >> 6) * (kBlock * 128) + (uint32_t)row * 128 +
                             ((uint32_t)(((col & 63) >> 3) ^ (row & 7)) << 4);
       st_shared_v4(addr, w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+    }
+  }
+}
+
+// Writes this thread's NC fp32 accumulator columns starting at `taddr`, times `mul`, as
+// bf16 straight to global memory at `dst` (16 columns, 32 bytes, per step); used where no
+// shared-memory buffer is free to stage the tile in.
+template <int NC>
+__device__ __forceinline__ void store_acc_cols(uint32_t taddr, float mul, __nv_bfloat16* dst,
+                                               bool valid) {
+  static_assert(NC % 16 == 0, "whole 16-column steps");
+#pragma unroll
+  for (int q = 0; q < NC / 16; ++q) {
+    uint32_t o[16];
+    tmem_ld16(taddr + 16 * q, o);
+    tmem_wait_ld();
+    reg_fence(o);
+    uint32_t w[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      w[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * mul, __uint_as_float(o[2 * c + 1]) * mul);
+    if (valid) {
+      st_global_v4(dst + 16 * q, w[0], w[1], w[2], w[3]);
+      st_global_v4(dst + 16 * q + 8, w[4], w[5], w[6], w[7]);
     }
   }
 }
@@ -417,6 +448,8 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
           }
           tc_commit(bar(bDPFull));
           tc_commit(bar(C::bY1Empty + s1));
+          // without staged outputs, K_j and V_j are free after their last product
+          if (!C::kStageOut && i == i_hi) tc_commit(bar(C::bXEmpty + xb));
         }
         ++items;
       }
@@ -474,6 +507,30 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
       }
       tc_commit(bar(C::bMmaFin + 1));
       mbar_wait(bar(C::bMmaFin + 1), 0, nullptr);
+    }
+    __syncwarp();
+  } else if (warp == C::kWarpStore) {
+    // ------------------------------------------------------------------ output stores
+    // dK, dV of each item leave through two bulk stores from the buffer the softmax warps
+    // staged them in; the buffer goes back to the producer once the stores have read it.
+    if (lane == 0 && C::kStageOut) {
+      int items = 0;
+      for (int k = blockIdx.x; k < a.n_items; k += gridDim.x, ++items) {
+        int bh, j;
+        bwd_item(k, a, true, bh, j);
+        const int xb = items % C::kXBufs;
+        if (!mbar_wait(bar(bStaged), items & 1, abort_flag)) break;
+        for (int r = 0; r < C::kRegions; ++r) {
+          tma_store_3d(&tmdK, sb + C::kX0 + xb * 2 * C::kTile + r * C::kRegionBytes, r * 64,
+                       j * kBlock, bh);
+          tma_store_3d(&tmdV, sb + C::kX1 + xb * 2 * C::kTile + r * C::kRegionBytes, r * 64,
+                       j * kBlock, bh);
+        }
+        bulk_commit();
+        bulk_wait_read();
+        mbar_arrive(bar(C::bXEmpty + xb));
+      }
+      bulk_wait_all();
     }
     __syncwarp();
   } else {
@@ -558,32 +615,29 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
         ok = false;
         break;
       }
-      // dK and dV go through the item's K_j, V_j buffer, which no product reads any more,
-      // and leave in two bulk stores; the producer reuses the buffer once they have read it
+      // With staged outputs, dK and dV go through the item's K_j, V_j buffer, which no
+      // product reads any more; the store warp writes them out and hands the buffer back to
+      // the producer. Otherwise each thread writes its part of its row directly.
       const int xb = items % C::kXBufs;
       const uint32_t tK = sb + C::kX0 + xb * 2 * C::kTile, tV = sb + C::kX1 + xb * 2 * C::kTile;
       ++items;
       tc_fence_after();
       constexpr int NO = D / C::kGroups;
-      stage_acc_cols<NO>(tmem + lane_base + tDV + NO * h, 1.f, tV, t_row, NO * h);
-      stage_acc_cols<NO>(tmem + lane_base + tDK + NO * h, a.scale, tK, t_row, NO * h);
-      fence_async_smem();
+      if (C::kStageOut) {
+        stage_acc_cols<NO>(tmem + lane_base + tDV + NO * h, 1.f, tV, t_row, NO * h);
+        stage_acc_cols<NO>(tmem + lane_base + tDK + NO * h, a.scale, tK, t_row, NO * h);
+        fence_async_smem();
+      } else {
+        const bool valid = c < a.N;
+        const size_t off = ((size_t)bh * a.N + (valid ? c : 0)) * D + NO * h;
+        store_acc_cols<NO>(tmem + lane_base + tDV + NO * h, 1.f, a.out1 + off, valid);
+        store_acc_cols<NO>(tmem + lane_base + tDK + NO * h, a.scale, a.out0 + off, valid);
+      }
       // dK, dV have been read: the next item's first products may overwrite them
       tc_fence_before();
       mbar_arrive_warp(bar(bAccFree));
-      mbar_arrive_warp(bar(bStaged));
-      // (a failed wait has raised the abort flag: the whole warp then stops at its next wait)
-      if (threadIdx.x == 0 && mbar_wait(bar(bStaged), (items - 1) & 1, abort_flag)) {
-        for (int r = 0; r < C::kRegions; ++r) {
-          tma_store_3d(&tmdK, tK + r * C::kRegionBytes, r * 64, j * kBlock, bh);
-          tma_store_3d(&tmdV, tV + r * C::kRegionBytes, r * 64, j * kBlock, bh);
-        }
-        bulk_commit();
-        bulk_wait_read();
-        mbar_arrive(bar(C::bXEmpty + xb));
-      }
+      if (C::kStageOut) mbar_arrive_warp(bar(bStaged));
     }
-    if (threadIdx.x == 0) bulk_wait_all();
   }
   bwd_teardown<C>(tmem, warp);
 }
@@ -745,6 +799,8 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
           }
           tc_commit(bar(bDPFull));
           tc_commit(bar(C::bY1Empty + s1));
+          // without a staged output, Q_i and dO_i are free after their last product
+          if (!C::kStageOut && jj == j_hi) tc_commit(bar(C::bXEmpty + xb));
         }
         ++items;
       }
@@ -788,6 +844,25 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
       }
       tc_commit(bar(C::bMmaFin + 1));
       mbar_wait(bar(C::bMmaFin + 1), 0, nullptr);
+    }
+    __syncwarp();
+  } else if (warp == C::kWarpStore) {
+    // ------------------------------------------------------------------ output stores
+    if (lane == 0 && C::kStageOut) {
+      int items = 0;
+      for (int k = blockIdx.x; k < a.n_items; k += gridDim.x, ++items) {
+        int bh, i;
+        bwd_item(k, a, false, bh, i);
+        const int xb = items % C::kXBufs;
+        if (!mbar_wait(bar(bStaged), items & 1, abort_flag)) break;
+        for (int rg = 0; rg < C::kRegions; ++rg)
+          tma_store_3d(&tmdQ, sb + C::kX0 + xb * 2 * C::kTile + rg * C::kRegionBytes, rg * 64,
+                       i * kBlock, bh);
+        bulk_commit();
+        bulk_wait_read();
+        mbar_arrive(bar(C::bXEmpty + xb));
+      }
+      bulk_wait_all();
     }
     __syncwarp();
   } else {
@@ -853,29 +928,27 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
         ok = false;
         break;
       }
-      // dQ goes through the item's Q_i buffer, which no product reads any more, and leaves
-      // in one bulk store; the producer reuses the buffer once it has been read
+      // With a staged output, dQ goes through the item's Q_i buffer, which no product reads
+      // any more; the store warp writes it out and hands the buffer back to the producer.
+      // Otherwise each thread writes its part of its row directly.
       const int xb = items % C::kXBufs;
       const uint32_t tQ = sb + C::kX0 + xb * 2 * C::kTile;
       ++items;
       tc_fence_after();
       constexpr int NO = D / C::kGroups;
-      stage_acc_cols<NO>(tmem + lane_base + tDQ + NO * h, a.scale, tQ, t_row, NO * h);
-      fence_async_smem();
+      if (C::kStageOut) {
+        stage_acc_cols<NO>(tmem + lane_base + tDQ + NO * h, a.scale, tQ, t_row, NO * h);
+        fence_async_smem();
+      } else {
+        const bool valid = r < a.N;
+        const size_t off = ((size_t)bh * a.N + (valid ? r : 0)) * D + NO * h;
+        store_acc_cols<NO>(tmem + lane_base + tDQ + NO * h, a.scale, a.out0 + off, valid);
+      }
       // dQ has been read: the next item's first product may overwrite it
       tc_fence_before();
       mbar_arrive_warp(bar(bAccFree));
-      mbar_arrive_warp(bar(bStaged));
-      // (a failed wait has raised the abort flag: the whole warp then stops at its next wait)
-      if (threadIdx.x == 0 && mbar_wait(bar(bStaged), (items - 1) & 1, abort_flag)) {
-        for (int rg = 0; rg < C::kRegions; ++rg)
-          tma_store_3d(&tmdQ, tQ + rg * C::kRegionBytes, rg * 64, i * kBlock, bh);
-        bulk_commit();
-        bulk_wait_read();
-        mbar_arrive(bar(C::bXEmpty + xb));
-      }
+      if (C::kStageOut) mbar_arrive_warp(bar(bStaged));
     }
-    if (threadIdx.x == 0) bulk_wait_all();
   }
   bwd_teardown<C>(tmem, warp);
 }
