@@ -24,10 +24,11 @@
 // 32h..32h+31 of it (query columns for dK/dV, key columns for dQ), so that four warps
 // per SM sub-partition hide each other's latencies. P needs no row maximum here (the
 // LSE is known), so the groups never wait for each other. Two MMA issuers (warps 16 and
-// 17; warp 18 issues the TMA loads, warp 19 the output stores) work side by side: one computes the score products
-// S and dP tile after tile, the other the gradient products as soon as the softmax
-// publishes P and dS. Issuing a product group occupies its thread for about as long as
-// the tensor core takes to run it, so one issuer for both would serialise them.
+// 17) work side by side: one computes the score products S and dP tile after tile, the
+// other the gradient products as soon as the softmax publishes P and dS. Issuing a
+// product group occupies its thread for about as long as the tensor core takes to run
+// it, so one issuer for both would serialise them. Warp 18 issues the TMA loads and
+// warp 19 the bulk stores of staged outputs.
 #pragma once
 
 #include <cuda_bf16.h>

@@ -179,7 +179,7 @@ fa_status_t fa_debug_status(void *stream);
 /*
  * Test hook for the timeout path (no GPU fault is involved). fault = 1: fa_fwd calls
  * made afterwards in this process launch with their copy warp skipping every V tile, so
- * the MMA warp's bounded wait for V runs out after about two seconds; the kernel then
+ * the MMA warps' bounded waits for V run out after about two seconds; the kernel then
  * abandons its work, drains the copies and products already in flight, frees its tensor
  * memory and exits, and fa_debug_status() returns FA_ERR_TIMEOUT. fault = 0 restores
  * normal operation. Other values return FA_ERR_INVALID_ARG.
