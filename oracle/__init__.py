@@ -48,10 +48,11 @@ class Oracle:
         self.lib = ctypes.CDLL(path)
         L = ctypes.c_long
         self.lib.oracle_attention_fwd.argtypes = [
-            _dptr, _dptr, _dptr, L, L, L, L, ctypes.c_double, ctypes.c_int, L, L, _dptr, _dptr]
+            _dptr, _dptr, _dptr, L, L, L, L, ctypes.c_double, ctypes.c_int, L, L, _dptr, _dptr,
+            _dptr]
         self.lib.oracle_attention_fwd.restype = ctypes.c_int
         self.lib.oracle_attention_bwd.argtypes = [
-            _dptr, _dptr, _dptr, _dptr, L, L, L, L, ctypes.c_double, ctypes.c_int, L, L,
+            _dptr, _dptr, _dptr, _dptr, L, L, L, L, ctypes.c_double, ctypes.c_int, L, L, _dptr,
             _dptr, _dptr, _dptr]
         self.lib.oracle_attention_bwd.restype = ctypes.c_int
         self.lib.oracle_num_threads.restype = ctypes.c_int
@@ -67,29 +68,40 @@ class Oracle:
             out.append(a)
         return out
 
-    def fwd(self, q, k, v, scale, causal=False, window=(-1, -1)):
-        """Returns (O, LSE) in fp64 for (B, H, N, d) inputs."""
+    @staticmethod
+    def _slopes(alibi, H):
+        if alibi is None:
+            return None, None
+        a = np.ascontiguousarray(alibi, dtype=np.float64).reshape(-1)
+        if a.shape != (H,):
+            raise ValueError("alibi_slopes must hold one slope per head")
+        return a, _as_ptr(a)
+
+    def fwd(self, q, k, v, scale, causal=False, window=(-1, -1), alibi=None):
+        """Returns (O, LSE) in fp64 for (B, H, N, d) inputs; `alibi`: H slopes or None."""
         q, k, v = self._prep(q, k, v)
         B, H, N, d = q.shape
         o = np.empty_like(q)
         lse = np.empty((B, H, N), dtype=np.float64)
+        keep, slopes = self._slopes(alibi, H)
         rc = self.lib.oracle_attention_fwd(_as_ptr(q), _as_ptr(k), _as_ptr(v), B, H, N, d,
                                            float(scale), int(bool(causal)), int(window[0]),
-                                           int(window[1]), _as_ptr(o), _as_ptr(lse))
+                                           int(window[1]), slopes, _as_ptr(o), _as_ptr(lse))
         if rc != 0:
             raise RuntimeError("oracle_attention_fwd failed with %d" % rc)
         return o, lse
 
-    def bwd(self, q, k, v, do, scale, causal=False, window=(-1, -1)):
+    def bwd(self, q, k, v, do, scale, causal=False, window=(-1, -1), alibi=None):
         """Returns (dQ, dK, dV) in fp64: the gradient of <O, dO> for (B, H, N, d) inputs."""
         q, k, v, do = self._prep(q, k, v, do)
         B, H, N, d = q.shape
         dq = np.empty_like(q)
         dk = np.empty_like(q)
         dv = np.empty_like(q)
+        keep, slopes = self._slopes(alibi, H)
         rc = self.lib.oracle_attention_bwd(_as_ptr(q), _as_ptr(k), _as_ptr(v), _as_ptr(do),
                                            B, H, N, d, float(scale), int(bool(causal)),
-                                           int(window[0]), int(window[1]),
+                                           int(window[0]), int(window[1]), slopes,
                                            _as_ptr(dq), _as_ptr(dk), _as_ptr(dv))
         if rc != 0:
             raise RuntimeError("oracle_attention_bwd failed with %d" % rc)

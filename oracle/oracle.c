@@ -12,6 +12,8 @@
  *                                              提升训练速度", the Attention(Q,K,V) formula;
  *                                              page "告别OOM和训练慢…(含A100环境配置)" §1, the
  *                                              three-line PyTorch implementation)
+ *   S_ij += -m_h |i - j|  when per-head ALiBi slopes m_h are given (the linear bias
+ *          `alibi_slopes` of `flash_attn_fn`, page "告别OOM和训练慢…" §4.2)
  *   S_ij = -inf where key j is not visible from query i (causal: "mask future
  *          positions", page "Flash Attention 3.7 核心原理与实战" §3.2; sliding window
  *          `window_size=(left,right)`, page "告别OOM和训练慢…" §4.2)
@@ -33,6 +35,9 @@
  *     -1 means unbounded; causal forces right = min(right, 0) (right = 0 when unbounded).
  *   - a row with no visible key has P_i = 0, O_i = 0, LSE_i = -inf, and adds nothing
  *     to any gradient.
+ *   - ALiBi (the page names the parameter and calls it a linear bias, nothing more): a
+ *     slope m_h per head, the bias -m_h |i - j| added to the scaled score; it is a
+ *     constant of the scores, so the backward formulas are unchanged.
  *
  * Layout: every tensor is (B, H, N, d) row-major fp64; lse is (B, H, N).
  * Loops over rows are shared out with OpenMP; each output element is still
@@ -60,9 +65,16 @@ static int visible(long i, long j, long left, long right)
     return 1;
 }
 
-/* P (N x N) := softmax rows of the masked, scaled scores of one head; lse (N). */
+/* The ALiBi slope of head bh (of B*H, heads fastest): 0 without slopes. */
+static double head_slope(const double *alibi_slopes, long bh, long H)
+{
+    return alibi_slopes ? alibi_slopes[bh % H] : 0.0;
+}
+
+/* P (N x N) := softmax rows of the masked, scaled (and biased, when slope != 0) scores of
+ * one head; lse (N). */
 static void head_probabilities(const double *q, const double *k, long N, long d,
-                               double scale, long left, long right,
+                               double scale, double slope, long left, long right,
                                double *P, double *lse)
 {
     long i;
@@ -75,6 +87,7 @@ static void head_probabilities(const double *q, const double *k, long N, long d,
             double s = 0.0;
             for (c = 0; c < d; ++c) s += q[i * d + c] * k[j * d + c];
             s *= scale;
+            s += -slope * fabs((double)(i - j));
             if (!visible(i, j, left, right)) s = -INFINITY;
             Pi[j] = s;
             if (s > m) m = s;
@@ -94,9 +107,10 @@ static void head_probabilities(const double *q, const double *k, long N, long d,
     }
 }
 
+/* alibi_slopes: H slopes, or NULL for no bias. */
 int oracle_attention_fwd(const double *q, const double *k, const double *v,
                          long B, long H, long N, long d, double scale,
-                         int causal, long left, long right,
+                         int causal, long left, long right, const double *alibi_slopes,
                          double *o, double *lse)
 {
     long bh;
@@ -108,7 +122,8 @@ int oracle_attention_fwd(const double *q, const double *k, const double *v,
         const double *qh = q + bh * N * d, *kh = k + bh * N * d, *vh = v + bh * N * d;
         double *oh = o + bh * N * d;
         long i;
-        head_probabilities(qh, kh, N, d, scale, left, right, P, lse + bh * N);
+        head_probabilities(qh, kh, N, d, scale, head_slope(alibi_slopes, bh, H), left, right, P,
+                           lse + bh * N);
         /* O = P V */
 #pragma omp parallel for schedule(static)
         for (i = 0; i < N; ++i) {
@@ -127,7 +142,7 @@ int oracle_attention_fwd(const double *q, const double *k, const double *v,
 int oracle_attention_bwd(const double *q, const double *k, const double *v,
                          const double *dout,
                          long B, long H, long N, long d, double scale,
-                         int causal, long left, long right,
+                         int causal, long left, long right, const double *alibi_slopes,
                          double *dq, double *dk, double *dv)
 {
     long bh;
@@ -147,7 +162,8 @@ int oracle_attention_bwd(const double *q, const double *k, const double *v,
         const double *doh = dout + bh * N * d;
         double *dqh = dq + bh * N * d, *dkh = dk + bh * N * d, *dvh = dv + bh * N * d;
         long i, j;
-        head_probabilities(qh, kh, N, d, scale, left, right, P, lse);
+        head_probabilities(qh, kh, N, d, scale, head_slope(alibi_slopes, bh, H), left, right, P,
+                           lse);
         /* dV = P^T dO */
 #pragma omp parallel for schedule(static)
         for (j = 0; j < N; ++j) {

@@ -16,6 +16,11 @@ Sources of the facts:
   * central finite differences of L = <O, dO> (the backward is the gradient of L);
   * torch's fp64 CPU scaled_dot_product_attention and autograd, as an independent
     library implementation of the same definition.
+
+The ALiBi pins (linear bias -m_h |i - j| on the scaled scores, the `alibi_slopes` parameter
+of page "告别OOM和训练慢…(含A100环境配置)" §4.2) use the same kinds of facts: closed forms
+where the scores are the bias alone, the limit of a bias so steep that each row sees only
+itself, finite differences, zero slopes, and torch's SDPA with the bias as a float mask.
 """
 from __future__ import annotations
 
@@ -257,6 +262,105 @@ def pin_library_sdpa(orc):
         np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=1e-11, atol=1e-11)
 
 
+def _alibi_slopes(H):
+    """The geometric slopes of the ALiBi paper: 2^(-8 h / H) for h = 1..H."""
+    return np.array([2.0 ** (-8.0 * (h + 1) / H) for h in range(H)])
+
+
+def pin_alibi_two_keys(orc):
+    """Q = 0 and N = 2: the scores are the bias alone, so row 0 weighs key 1 by e^-m
+    against 1: O_0 = (v_0 + e^-m v_1) / (1 + e^-m), LSE_0 = ln(1 + e^-m); row 1 the same
+    with the keys swapped."""
+    r = _rng(11)
+    H = 3
+    slopes = np.array([0.3, 1.7, 4.0])
+    q = np.zeros((1, H, 2, 4))
+    k, v = (r.standard_normal((1, H, 2, 4)) for _ in range(2))
+    o, lse = orc.fwd(q, k, v, 0.5, False, (-1, -1), slopes)
+    for h, m in enumerate(slopes):
+        w = math.exp(-m)
+        np.testing.assert_allclose(o[0, h, 0], (v[0, h, 0] + w * v[0, h, 1]) / (1 + w), rtol=1e-13)
+        np.testing.assert_allclose(o[0, h, 1], (v[0, h, 1] + w * v[0, h, 0]) / (1 + w), rtol=1e-13)
+        np.testing.assert_allclose(lse[0, h], [math.log1p(w)] * 2, rtol=1e-13)
+
+
+def pin_alibi_steep_bias(orc):
+    """A slope of 60 with scores of order one: every other key is damped by e^-60 or more,
+    so each row returns its own value, O_i = v_i, and LSE_i = scale q_i . k_i, in every mask
+    mode (the diagonal is always visible)."""
+    r = _rng(12)
+    q, k, v = (0.3 * r.standard_normal((1, 2, 9, 4)) for _ in range(3))
+    slopes = np.array([60.0, 80.0])
+    for causal, window in MODES:
+        o, lse = orc.fwd(q, k, v, 0.5, causal, window, slopes)
+        np.testing.assert_allclose(o, v, rtol=0, atol=1e-20)
+        np.testing.assert_allclose(lse, 0.5 * np.sum(q * k, axis=-1), rtol=1e-14, atol=1e-14)
+
+
+def pin_alibi_zero_slopes(orc):
+    """Zero slopes are no bias at all: bit-identical results."""
+    r = _rng(13)
+    q, k, v, do = (r.standard_normal((1, 2, 7, 3)) for _ in range(4))
+    for causal, window in MODES:
+        a = orc.fwd(q, k, v, 0.6, causal, window)
+        b = orc.fwd(q, k, v, 0.6, causal, window, np.zeros(2))
+        ga = orc.bwd(q, k, v, do, 0.6, causal, window)
+        gb = orc.bwd(q, k, v, do, 0.6, causal, window, np.zeros(2))
+        for x, y in zip(a + ga, b + gb):
+            assert np.array_equal(x, y)
+
+
+def pin_alibi_finite_differences(orc):
+    """With a bias, the backward is still the gradient of L = <O, dO>: central
+    differences in every entry of Q, K, V (the bias does not depend on them)."""
+    r = _rng(14)
+    B, H, N, d = 1, 2, 5, 3
+    q, k, v, do = (r.standard_normal((B, H, N, d)) for _ in range(4))
+    slopes = np.array([0.7, 2.5])
+    scale, eps = 0.45, 1e-6
+    for causal, window in MODES[:3]:
+        grads = orc.bwd(q, k, v, do, scale, causal, window, slopes)
+        for which in range(3):
+            num = np.zeros_like(q)
+            for idx in np.ndindex(q.shape):
+                args = [q.copy(), k.copy(), v.copy()]
+                args[which][idx] += eps
+                lp = np.sum(orc.fwd(*args, scale, causal, window, slopes)[0] * do)
+                args[which][idx] -= 2 * eps
+                lm = np.sum(orc.fwd(*args, scale, causal, window, slopes)[0] * do)
+                num[idx] = (lp - lm) / (2 * eps)
+            np.testing.assert_allclose(grads[which], num, rtol=1e-6, atol=1e-7)
+
+
+def pin_alibi_library_sdpa(orc):
+    """torch's fp64 SDPA with the bias -m_h |i - j| (and -inf where masked) as a float
+    mask, and autograd through it, give the same O, LSE and gradients."""
+    r = _rng(15)
+    B, H, N, d = 2, 3, 17, 6
+    q, k, v, do = (r.standard_normal((B, H, N, d)) for _ in range(4))
+    slopes = _alibi_slopes(H)
+    scale = 0.35
+    idx = torch.arange(N, dtype=torch.float64)
+    dist = (idx[:, None] - idx[None, :]).abs()
+    bias = -torch.tensor(slopes)[:, None, None] * dist[None]
+    for causal, window in MODES:
+        band = _band_mask(N, causal, window)
+        fmask = bias.masked_fill(~band, float("-inf"))
+        tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+        to = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=fmask,
+                                                              scale=scale)
+        to.backward(torch.tensor(do))
+        scores = (torch.tensor(q) @ torch.tensor(k).transpose(-1, -2)) * scale + fmask
+        tlse = torch.logsumexp(scores, dim=-1)
+        o, lse = orc.fwd(q, k, v, scale, causal, window, slopes)
+        dq, dk, dv = orc.bwd(q, k, v, do, scale, causal, window, slopes)
+        np.testing.assert_allclose(o, to.detach().numpy(), rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(lse, tlse.numpy(), rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=1e-11, atol=1e-11)
+        np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=1e-11, atol=1e-11)
+        np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=1e-11, atol=1e-11)
+
+
 def pin_self_similarity(orc):
     """k = v = q (the page "显存神技：必学FlashAttention！" comparison input): each row's own
     key has the largest score |q_i|^2 scale among keys of no larger norm, so O is finite,
@@ -282,4 +386,9 @@ ALL_PINS = [
     pin_key_permutation,
     pin_library_sdpa,
     pin_self_similarity,
+    pin_alibi_two_keys,
+    pin_alibi_steep_bias,
+    pin_alibi_zero_slopes,
+    pin_alibi_finite_differences,
+    pin_alibi_library_sdpa,
 ]

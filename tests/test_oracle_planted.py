@@ -26,6 +26,14 @@ PLANTS = [
     ("dK scale dropped", "dkh[j * d + c] *= scale;", "dkh[j * d + c] *= 1.0;"),
     ("dP uses dO of the key row", "s += doh[i * d + c] * vh[jj * d + c];",
      "s += doh[jj * d + c] * vh[jj * d + c];"),
+    ("ALiBi bias sign flipped", "s += -slope * fabs((double)(i - j));",
+     "s += slope * fabs((double)(i - j));"),
+    ("ALiBi distance without the absolute value", "s += -slope * fabs((double)(i - j));",
+     "s += -slope * (double)(i - j);"),
+    ("ALiBi bias scaled with the scores", "s += -slope * fabs((double)(i - j));",
+     "s += -slope * scale * fabs((double)(i - j));"),
+    ("ALiBi slope of the wrong head", "return alibi_slopes ? alibi_slopes[bh % H] : 0.0;",
+     "return alibi_slopes ? alibi_slopes[0] : 0.0;"),
 ]
 
 
