@@ -144,7 +144,7 @@ def job_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
 def run_ours(args, w, rank, world, local_rank):
     import torch
 
-    from exact_attention_126_b200 import build, fa, synth
+    from exact_attention_126_b200 import build, fa, synth, workloads
 
     build.build()
     torch.cuda.set_device(local_rank)
@@ -164,6 +164,9 @@ def run_ours(args, w, rank, world, local_rank):
     dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     ws = torch.empty(fa.fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
     scale = w.softmax_scale
+    slopes = None
+    if w.alibi:
+        slopes = torch.tensor(workloads.alibi_slopes(H), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
     inputs_bytes = 4 * w.tensor_bytes()
@@ -172,9 +175,20 @@ def run_ours(args, w, rank, world, local_rank):
         flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
 
     def step(evs=None):
-        # fa_fwd, then the three phases of fa_bwd, with optional events between kernels
+        # fa_fwd, then the three phases of fa_bwd, with optional events between kernels;
+        # with ALiBi, fa_fwd_alibi and fa_bwd_alibi (the backward timed as one)
         if evs is not None:
             evs[0].record(stream)
+        if w.alibi:
+            fa.fa_fwd_alibi(q, k, v, o, lse, slopes, scale, w.causal, w.window, sp)
+            if evs is not None:
+                evs[1].record(stream)
+            if w.backward:
+                fa.fa_bwd_alibi(q, k, v, o, do, lse, dq, dk, dv, ws, slopes, scale, w.causal,
+                                w.window, sp)
+                if evs is not None:
+                    evs[2].record(stream)
+            return
         fa.fa_fwd(q, k, v, o, lse, scale, w.causal, w.window, sp)
         if evs is not None:
             evs[1].record(stream)
@@ -189,7 +203,7 @@ def run_ours(args, w, rank, world, local_rank):
             if evs is not None:
                 evs[4].record(stream)
 
-    n_ev = 5 if w.backward else 2
+    n_ev = (3 if w.alibi else 5) if w.backward else 2
     launches_per_step = 4 if w.backward else 1
 
     for _ in range(args.warmup):
@@ -221,7 +235,8 @@ def run_ours(args, w, rank, world, local_rank):
         raise RuntimeError("a kernel abandoned a bounded wait in the timed region")
 
     # device time of the K steps (flushes excluded), and per kernel
-    names = ["fwd", "bwd_preprocess", "bwd_dkdv", "bwd_dq"][: n_ev - 1]
+    names = (["fwd", "bwd"] if w.alibi else ["fwd", "bwd_preprocess", "bwd_dkdv", "bwd_dq"])[
+        : n_ev - 1]
     per_kernel = {n: 0.0 for n in names}
     step_ms = 0.0
     for evs in events:
@@ -252,11 +267,15 @@ def run_ours(args, w, rank, world, local_rank):
         v.copy_(inp_host["v"], non_blocking=True)
         if w.backward:
             do.copy_(inp_host["do"], non_blocking=True)
-        fa.fa_fwd(q, k, v, o, lse, scale, w.causal, w.window, sp)
+        if w.alibi:
+            fa.fa_fwd_alibi(q, k, v, o, lse, slopes, scale, w.causal, w.window, sp)
+        else:
+            fa.fa_fwd(q, k, v, o, lse, scale, w.causal, w.window, sp)
         host_out["o"].copy_(o, non_blocking=True)
         host_out["lse"].copy_(lse, non_blocking=True)
         if w.backward:
-            dqq, dkk, dvv = fa.attention_backward(q, k, v, o, lse, do, scale, w.causal, w.window, sp)
+            dqq, dkk, dvv = fa.attention_backward(q, k, v, o, lse, do, scale, w.causal, w.window, sp,
+                                                  alibi_slopes=slopes)
             host_out["dq"].copy_(dqq, non_blocking=True)
             host_out["dk"].copy_(dkk, non_blocking=True)
             host_out["dv"].copy_(dvv, non_blocking=True)
@@ -285,7 +304,8 @@ def run_ours(args, w, rank, world, local_rank):
     flops = w.step_flops()
     value = job_tflops(flops, world, ms_per_step)
     kernel_flops = {"fwd": w.fwd_flops(), "bwd_preprocess": 0.0,
-                    "bwd_dkdv": 2.0 * w.fwd_flops(), "bwd_dq": 0.5 * w.fwd_flops()}
+                    "bwd_dkdv": 2.0 * w.fwd_flops(), "bwd_dq": 0.5 * w.fwd_flops(),
+                    "bwd": 2.5 * w.fwd_flops()}
     kernels = {}
     for n in names:
         avg = per_kernel[n] / args.steps
@@ -356,6 +376,14 @@ def _oracle_sample(w, b, h):
     return {n: synth.to_f64(t) for n, t in x.items()}
 
 
+def _head_slope(w, h):
+    """The ALiBi slope of head h as a one-head slope list for the oracle (None without)."""
+    if not w.alibi:
+        return None
+    from exact_attention_126_b200 import workloads
+    return [workloads.alibi_slopes(w.H)[h]]
+
+
 def cpu_baseline(w, seconds: float):
     """Times the fp64 oracle, as it stands, on whole (batch, head) problems of the workload
     until `seconds` have passed (at least one head)."""
@@ -367,10 +395,11 @@ def cpu_baseline(w, seconds: float):
     while elapsed < seconds and done < BH:
         b, h = divmod(done, w.H)
         x = _oracle_sample(w, b, h)
+        slope = _head_slope(w, h)
         t0 = time.perf_counter()
-        orc.fwd(x["q"], x["k"], x["v"], w.softmax_scale, w.causal, w.window)
+        orc.fwd(x["q"], x["k"], x["v"], w.softmax_scale, w.causal, w.window, slope)
         if w.backward:
-            orc.bwd(x["q"], x["k"], x["v"], x["do"], w.softmax_scale, w.causal, w.window)
+            orc.bwd(x["q"], x["k"], x["v"], x["do"], w.softmax_scale, w.causal, w.window, slope)
         elapsed += time.perf_counter() - t0
         done += 1
     return {"value": round(flops_per_head * done / elapsed / 1e12, 6), "unit": "TFLOP/s",
@@ -392,10 +421,11 @@ def run_reference(args, w, rank):
     def one(idx):
         b, h = divmod(idx % BH, w.H)
         x = _oracle_sample(w, b, h)
+        slope = _head_slope(w, h)
         t0 = time.perf_counter()
-        orc.fwd(x["q"], x["k"], x["v"], w.softmax_scale, w.causal, w.window)
+        orc.fwd(x["q"], x["k"], x["v"], w.softmax_scale, w.causal, w.window, slope)
         if w.backward:
-            orc.bwd(x["q"], x["k"], x["v"], x["do"], w.softmax_scale, w.causal, w.window)
+            orc.bwd(x["q"], x["k"], x["v"], x["do"], w.softmax_scale, w.causal, w.window, slope)
         return time.perf_counter() - t0
 
     for i in range(args.warmup):

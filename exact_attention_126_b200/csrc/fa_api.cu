@@ -125,14 +125,16 @@ fa_status_t launched() {
 }
 
 
-template <int D>
+// alibi: H slopes for the ALiBi kernels (kAlibi), unused otherwise.
+template <int D, bool kAlibi>
 fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int BH,
-                       int N, float scale, int left, int right, cudaStream_t st) {
+                       int H, int N, float scale, int left, int right, const float* alibi,
+                       cudaStream_t st) {
   CUtensorMap mq, mkk, mv;
   if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) || !make_map(&mv, v, BH, N, D))
     return FA_ERR_CUDA;
   using C = fa::FwdCfg<D>;
-  if (set_smem(fa::fa_fwd_kernel<D>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
+  if (set_smem(fa::fa_fwd_kernel<D, kAlibi>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
   fa::FwdArgs a;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
@@ -147,8 +149,10 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   a.left = left;
   a.right = right;
   a.fault = g_fault.load(std::memory_order_relaxed);
+  a.alibi = alibi;
+  a.H = H;
   const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
-  fa::fa_fwd_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, a);
+  fa::fa_fwd_kernel<D, kAlibi><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, a);
   return launched();
 }
 
@@ -169,17 +173,17 @@ fa_status_t launch_preprocess(const void* o, const void* dout, const float* lse,
   return launched();
 }
 
-template <int D>
+template <int D, bool kAlibi>
 fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void* dout,
-                        const void* ws, void* dk, void* dv, int BH, int N,
-                        float scale, int left, int right, cudaStream_t st) {
+                        const void* ws, void* dk, void* dv, int BH, int H, int N,
+                        float scale, int left, int right, const float* alibi, cudaStream_t st) {
   CUtensorMap mq, mkk, mv, mdo, mdk, mdv;
   if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
       !make_map(&mv, v, BH, N, D) || !make_map(&mdo, dout, BH, N, D) ||
       !make_map(&mdk, dk, BH, N, D) || !make_map(&mdv, dv, BH, N, D))
     return FA_ERR_CUDA;
   using C = fa::DkdvCfg<D>;
-  if (set_smem(fa::fa_bwd_dkdv_kernel<D>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
+  if (set_smem(fa::fa_bwd_dkdv_kernel<D, kAlibi>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
   fa::BwdArgs a;
   a.stats = static_cast<const float*>(ws);
   a.out0 = static_cast<__nv_bfloat16*>(dk);
@@ -197,22 +201,24 @@ fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void*
   a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
   a.group = head_group(BH, a.n_tiles);
   const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
-  fa::fa_bwd_dkdv_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, mdk, mdv,
-                                                                       a);
+  a.alibi = alibi;
+  a.H = H;
+  fa::fa_bwd_dkdv_kernel<D, kAlibi><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo,
+                                                                               mdk, mdv, a);
   return launched();
 }
 
-template <int D>
+template <int D, bool kAlibi>
 fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* dout,
-                      const void* ws, void* dq, int BH, int N, float scale,
-                      int left, int right, cudaStream_t st) {
+                      const void* ws, void* dq, int BH, int H, int N, float scale,
+                      int left, int right, const float* alibi, cudaStream_t st) {
   CUtensorMap mq, mkk, mv, mdo, mdq;
   if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
       !make_map(&mv, v, BH, N, D) || !make_map(&mdo, dout, BH, N, D) ||
       !make_map(&mdq, dq, BH, N, D))
     return FA_ERR_CUDA;
   using C = fa::DqCfg<D>;
-  if (set_smem(fa::fa_bwd_dq_kernel<D>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
+  if (set_smem(fa::fa_bwd_dq_kernel<D, kAlibi>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
   fa::BwdArgs a;
   a.stats = static_cast<const float*>(ws);
   a.out0 = static_cast<__nv_bfloat16*>(dq);
@@ -230,7 +236,10 @@ fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* d
   a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
   a.group = head_group(BH, a.n_tiles);
   const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
-  fa::fa_bwd_dq_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, mdq, a);
+  a.alibi = alibi;
+  a.H = H;
+  fa::fa_bwd_dq_kernel<D, kAlibi><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, mdq,
+                                                                             a);
   return launched();
 }
 
@@ -271,10 +280,16 @@ fa_status_t noalloc_scratch(void** out) {
 
 }  // namespace
 
-extern "C" {
+fa_status_t check_slopes(const float* alibi) {
+  if (alibi == nullptr) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(alibi) & 3u) != 0) return FA_ERR_MISALIGNED;
+  return FA_OK;
+}
 
-fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                   int N, int d, float scale, int causal, fa_window_t window, void* stream) {
+// fa_fwd and fa_fwd_alibi (alibi != nullptr)
+fa_status_t forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                    int N, int d, float scale, int causal, fa_window_t window, const float* alibi,
+                    void* stream) {
   bool empty;
   fa_status_t s = check_problem(B, H, N, d, &empty);
   if (s != FA_OK || empty) return s;
@@ -282,8 +297,60 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
   if ((s = check_ptrs({q, k, v, o, lse})) != FA_OK) return s;
   const int right = fa::resolve_right(causal, window.right);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_fwd<64>(q, k, v, o, lse, B * H, N, scale, window.left, right, st)
-                 : launch_fwd<128>(q, k, v, o, lse, B * H, N, scale, window.left, right, st);
+  const int l = window.left, BH = B * H;
+  if (alibi != nullptr)
+    return d == 64 ? launch_fwd<64, true>(q, k, v, o, lse, BH, H, N, scale, l, right, alibi, st)
+                   : launch_fwd<128, true>(q, k, v, o, lse, BH, H, N, scale, l, right, alibi, st);
+  return d == 64 ? launch_fwd<64, false>(q, k, v, o, lse, BH, H, N, scale, l, right, nullptr, st)
+                 : launch_fwd<128, false>(q, k, v, o, lse, BH, H, N, scale, l, right, nullptr, st);
+}
+
+// The two passes of the backward after the preprocess step, with or without ALiBi.
+fa_status_t backward_passes(const void* q, const void* k, const void* v, const void* dout,
+                            const void* ws, void* dq, void* dk, void* dv, int B, int H, int N,
+                            int d, float scale, int causal, fa_window_t window,
+                            const float* alibi, void* stream) {
+  const int right = fa::resolve_right(causal, window.right);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int l = window.left, BH = B * H;
+  fa_status_t s;
+  if (alibi != nullptr) {
+    s = d == 64 ? launch_dkdv<64, true>(q, k, v, dout, ws, dk, dv, BH, H, N, scale, l, right,
+                                        alibi, st)
+                : launch_dkdv<128, true>(q, k, v, dout, ws, dk, dv, BH, H, N, scale, l, right,
+                                         alibi, st);
+    if (s != FA_OK) return s;
+    return d == 64 ? launch_dq<64, true>(q, k, v, dout, ws, dq, BH, H, N, scale, l, right,
+                                         alibi, st)
+                   : launch_dq<128, true>(q, k, v, dout, ws, dq, BH, H, N, scale, l, right,
+                                          alibi, st);
+  }
+  s = d == 64 ? launch_dkdv<64, false>(q, k, v, dout, ws, dk, dv, BH, H, N, scale, l, right,
+                                       nullptr, st)
+              : launch_dkdv<128, false>(q, k, v, dout, ws, dk, dv, BH, H, N, scale, l, right,
+                                        nullptr, st);
+  if (s != FA_OK) return s;
+  return d == 64 ? launch_dq<64, false>(q, k, v, dout, ws, dq, BH, H, N, scale, l, right,
+                                        nullptr, st)
+                 : launch_dq<128, false>(q, k, v, dout, ws, dq, BH, H, N, scale, l, right,
+                                         nullptr, st);
+}
+
+extern "C" {
+
+fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                   int N, int d, float scale, int causal, fa_window_t window, void* stream) {
+  return forward(q, k, v, o, lse, B, H, N, d, scale, causal, window, nullptr, stream);
+}
+
+fa_status_t fa_fwd_alibi(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int H, int N, int d, float scale, int causal, fa_window_t window,
+                         const float* alibi_slopes, void* stream) {
+  bool empty;
+  fa_status_t s = check_problem(B, H, N, d, &empty);
+  if (s != FA_OK || empty) return s;
+  if ((s = check_slopes(alibi_slopes)) != FA_OK) return s;
+  return forward(q, k, v, o, lse, B, H, N, d, scale, causal, window, alibi_slopes, stream);
 }
 
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
@@ -314,10 +381,10 @@ fa_status_t fa_bwd_dkdv(const void* q, const void* k, const void* v, const void*
   if ((s = check_ptrs({q, k, v, dout, workspace, dk, dv})) != FA_OK) return s;
   const int right = fa::resolve_right(causal, window.right);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_dkdv<64>(q, k, v, dout, workspace, dk, dv, B * H, N, scale,
-                                   window.left, right, st)
-                 : launch_dkdv<128>(q, k, v, dout, workspace, dk, dv, B * H, N, scale,
-                                    window.left, right, st);
+  return d == 64 ? launch_dkdv<64, false>(q, k, v, dout, workspace, dk, dv, B * H, H, N, scale,
+                                          window.left, right, nullptr, st)
+                 : launch_dkdv<128, false>(q, k, v, dout, workspace, dk, dv, B * H, H, N, scale,
+                                           window.left, right, nullptr, st);
 }
 
 fa_status_t fa_bwd_dq(const void* q, const void* k, const void* v, const void* dout,
@@ -330,10 +397,10 @@ fa_status_t fa_bwd_dq(const void* q, const void* k, const void* v, const void* d
   if ((s = check_ptrs({q, k, v, dout, workspace, dq})) != FA_OK) return s;
   const int right = fa::resolve_right(causal, window.right);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_dq<64>(q, k, v, dout, workspace, dq, B * H, N, scale, window.left,
-                                 right, st)
-                 : launch_dq<128>(q, k, v, dout, workspace, dq, B * H, N, scale, window.left,
-                                  right, st);
+  return d == 64 ? launch_dq<64, false>(q, k, v, dout, workspace, dq, B * H, H, N, scale,
+                                        window.left, right, nullptr, st)
+                 : launch_dq<128, false>(q, k, v, dout, workspace, dq, B * H, H, N, scale,
+                                         window.left, right, nullptr, st);
 }
 
 fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -351,6 +418,23 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
                        stream)) != FA_OK)
     return s;
   return fa_bwd_dq(q, k, v, dout, workspace, dq, B, H, N, d, scale, causal, window, stream);
+}
+
+fa_status_t fa_bwd_alibi(const void* q, const void* k, const void* v, const void* o,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                         int H, int N, int d, float scale, int causal, fa_window_t window,
+                         const float* alibi_slopes, void* workspace,
+                         size_t workspace_bytes_given, void* stream) {
+  bool empty;
+  fa_status_t s = check_problem(B, H, N, d, &empty);
+  if (s != FA_OK || empty) return s;
+  if ((s = check_mask(scale, window)) != FA_OK) return s;
+  if ((s = check_slopes(alibi_slopes)) != FA_OK) return s;
+  if ((s = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv, workspace})) != FA_OK) return s;
+  if (workspace_bytes_given < workspace_bytes(B, H, N)) return FA_ERR_WORKSPACE;
+  if ((s = fa_bwd_preprocess(o, dout, lse, workspace, B, H, N, d, stream)) != FA_OK) return s;
+  return backward_passes(q, k, v, dout, workspace, dq, dk, dv, B, H, N, d, scale, causal, window,
+                         alibi_slopes, stream);
 }
 
 fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,

@@ -38,7 +38,6 @@
 
 namespace fa {
 
-constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------------------------
 // Row statistics of the backward, over B*H rows of Np (N rounded up to 128) entries:
@@ -102,6 +101,8 @@ struct BwdArgs {
   float scale_log2;
   int left;
   int right;
+  const float* alibi;   // ALiBi kernels: one slope per head (heads = H)
+  int H;
 };
 
 // Shared layout of both backward kernels: the stationary tiles X0, X1 of an item (in XB
@@ -283,7 +284,8 @@ __device__ __forceinline__ void bwd_teardown(uint32_t tmem, int warp) {
 // dV += P^T dO and dK += dS^T Q as soon as the softmax publishes P^T and dS^T. Tile
 // counters (for barrier parities) run over all items of the CTA.
 // ------------------------------------------------------------------------------------
-template <int D>
+// kAlibi: the scores carry the linear bias -m_h |i - j| (m_h = alibi[bh % H]).
+template <int D, bool kAlibi = false>
 __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
     fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -550,6 +552,7 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
       q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
       const int n_it = i_hi - i_lo + 1;
       const int c = j * kBlock + t_row;  // this thread's key
+      const float slope2 = kAlibi ? a.alibi[bh % a.H] * kLog2e : 0.f;
       for (int it = 0; it < n_it; ++it) {
         const int i = i_lo + it;
         const int t = g + it;
@@ -568,10 +571,17 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
 #pragma unroll
         for (int r = 0; r < NC; r += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse_s + r);
-          p[r] = ex2(fmaf(p[r], sl2, -l4.x));
-          p[r + 1] = ex2(fmaf(p[r + 1], sl2, -l4.y));
-          p[r + 2] = ex2(fmaf(p[r + 2], sl2, -l4.z));
-          p[r + 3] = ex2(fmaf(p[r + 3], sl2, -l4.w));
+          float b4[4] = {0.f, 0.f, 0.f, 0.f};
+          if (kAlibi) {
+            // -m |query - key| in log2 units for the queries of these four columns
+            const float base = (float)((long long)i * kBlock + NC * h + r - c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) b4[e] = -slope2 * fabsf(base + (float)e);
+          }
+          p[r] = ex2(fmaf(p[r], sl2, b4[0] - l4.x));
+          p[r + 1] = ex2(fmaf(p[r + 1], sl2, b4[1] - l4.y));
+          p[r + 2] = ex2(fmaf(p[r + 2], sl2, b4[2] - l4.z));
+          p[r + 3] = ex2(fmaf(p[r + 3], sl2, b4[3] - l4.w));
         }
         if (!tile_all_visible(i, j, mk)) {
           int r_lo, r_hi;
@@ -650,7 +660,8 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
 // MMA issuers: one computes S and dP of each key tile in order, the other dQ += dS K_j
 // as soon as the softmax publishes dS. Tile counters run over all items.
 // ------------------------------------------------------------------------------------
-template <int D>
+// kAlibi: the scores carry the linear bias -m_h |i - j| (m_h = alibi[bh % H]).
+template <int D, bool kAlibi = false>
 __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
     fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV,
@@ -884,6 +895,7 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
       // rows past N carry +inf and 0 in the padded statistics, which zero their P and dS
       const float lse2 = a.stats[(size_t)bh * a.Np + r];
       const float dl = a.stats[a.stat_rows + (size_t)bh * a.Np + r];
+      const float slope2 = kAlibi ? a.alibi[bh % a.H] * kLog2e : 0.f;
       for (int it = 0; it < n_it; ++it) {
         const int jj = j_lo + it;
         const int t = g + it;
@@ -895,8 +907,15 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
         tc_fence_after();
         float p[NC];
         load_cols32(tmem + lane_base + tS0 + 128u * b + NC * h, p);
+        {
+          // with ALiBi, -m |key - query| in log2 units joins the exponent
+          const float base = (float)((long long)jj * kBlock + NC * h - r);
 #pragma unroll
-        for (int c = 0; c < NC; ++c) p[c] = ex2(fmaf(p[c], sl2, -lse2));
+          for (int c = 0; c < NC; ++c) {
+            const float bias = kAlibi ? -slope2 * fabsf(base + (float)c) : 0.f;
+            p[c] = ex2(fmaf(p[c], sl2, bias - lse2));
+          }
+        }
         if (!tile_all_visible(i, jj, mk)) {
           int c_lo, c_hi;
           visible_keys(r, (long long)jj * kBlock + NC * h, NC, mk, c_lo, c_hi);

@@ -47,6 +47,8 @@ struct FwdArgs {
   int left;
   int right;
   int fault;          // test hook: 1 = the producer never loads V (waits for it run out)
+  const float* alibi; // ALiBi kernels: one slope per head (heads = H)
+  int H;
 };
 
 template <int D>
@@ -156,7 +158,8 @@ __device__ __forceinline__ FwdRange fwd_range(const FwdItem& it, int s) {
   return r;
 }
 
-template <int D>
+// kAlibi: add the linear bias -m_h |i - j| (m_h = alibi[bh % H]) to every scaled score.
+template <int D, bool kAlibi = false>
 __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
@@ -410,6 +413,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
       if (!rg.has) continue;
       const bool turns = it.has_b;
       const int row = rg.m * kBlock + r;
+      // with ALiBi the scores are scaled and biased as they are loaded (in log2 units), so
+      // the later steps take them as they are
+      const float slope2 = kAlibi ? a.alibi[it.bh % a.H] * kLog2e : 0.f;
+      const float xs = kAlibi ? 1.f : sl2;
       float m_run = -INFINITY;  // running max of scale*log2e*s (the m that P and O carry)
       float l_run = 0.f;        // running sum of P
       for (int j = turns ? it.first : rg.lo; j <= (turns ? it.last : rg.hi); ++j) {
@@ -443,6 +450,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
           tc_fence_before();
           mbar_arrive_warp(bar(C::bSFree + s));
         }
+        if (kAlibi) {
+          // key minus query index at column 0 of the tile
+          const float base = (float)((long long)j * kBlock - row);
+#pragma unroll
+          for (int c = 0; c < kBlock; ++c)
+            x[c] = fmaf(x[c], sl2, -slope2 * fabsf(base + (float)c));
+        }
         if (!tile_all_visible(rg.m, j, mk)) {
           int c_lo, c_hi;
           visible_keys(row, (long long)j * kBlock, kBlock, mk, c_lo, c_hi);
@@ -469,7 +483,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         }
         // O_s is stable once the stream's previous P V product has completed: implied by
         // S_full when P shares the columns of S_s, waited for below otherwise.
-        const float m_new = fmaxf(m_run, mx * sl2);
+        const float m_new = fmaxf(m_run, mx * xs);
         const bool grow = m_new > m_run + 8.0f;
         float alpha = 1.f;
         if (grow) {
@@ -498,8 +512,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const float p0 = ex2(fmaf(x[32 * h + 2 * c], sl2, -mb));
-            const float p1 = ex2(fmaf(x[32 * h + 2 * c + 1], sl2, -mb));
+            const float p0 = ex2(fmaf(x[32 * h + 2 * c], xs, -mb));
+            const float p1 = ex2(fmaf(x[32 * h + 2 * c + 1], xs, -mb));
             ls[c & 3] += p0 + p1;
             pk[c] = pack_bf16x2(p0, p1);
           }

@@ -11,6 +11,7 @@
 namespace fa {
 
 constexpr int kBlock = 128;  // rows of a tile; the M (and N) extent of every MMA
+constexpr float kLog2e = 1.4426950408889634f;
 
 struct Mask {
   int N;      // sequence length

@@ -23,9 +23,9 @@ STATUS_NAMES = {
 }
 
 #: every symbol include/fa.h declares
-EXPORTED = ("fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_dkdv",
-            "fa_bwd_dq", "fa_bwd_noalloc", "fa_status_string", "fa_debug_status",
-            "fa_debug_set_fault", "fa_version")
+EXPORTED = ("fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_fwd_alibi", "fa_bwd_alibi",
+            "fa_bwd_preprocess", "fa_bwd_dkdv", "fa_bwd_dq", "fa_bwd_noalloc",
+            "fa_status_string", "fa_debug_status", "fa_debug_set_fault", "fa_version")
 
 
 class FAError(RuntimeError):
@@ -57,6 +57,9 @@ def _lib() -> ctypes.CDLL:
         lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
         lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp,
                                ctypes.c_size_t, vp]
+        lib.fa_fwd_alibi.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp, vp]
+        lib.fa_bwd_alibi.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp,
+                                     vp, ctypes.c_size_t, vp]
         lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, vp, I, I, I, I, vp]
         lib.fa_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp]
         lib.fa_bwd_dq.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp]
@@ -67,8 +70,9 @@ def _lib() -> ctypes.CDLL:
         lib.fa_debug_status.argtypes = [vp]
         lib.fa_debug_set_fault.argtypes = [I]
         lib.fa_version.argtypes = []
-        for name in ("fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_dkdv", "fa_bwd_dq",
-                     "fa_bwd_noalloc", "fa_debug_status", "fa_debug_set_fault", "fa_version"):
+        for name in ("fa_fwd", "fa_bwd", "fa_fwd_alibi", "fa_bwd_alibi", "fa_bwd_preprocess",
+                     "fa_bwd_dkdv", "fa_bwd_dq", "fa_bwd_noalloc", "fa_debug_status",
+                     "fa_debug_set_fault", "fa_version"):
             getattr(lib, name).restype = I
         _LIB = lib
     return _LIB
@@ -133,6 +137,29 @@ def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale=None, causal=False,
     _check(_lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
                          _ptr(dk), _ptr(dv), B, H, N, d, s, c, w, _ptr(workspace), nbytes,
                          _stream(stream)), "fa_bwd")
+
+
+def fa_fwd_alibi(q, k, v, o, lse, alibi_slopes, scale=None, causal=False, window=(-1, -1),
+                 stream=None) -> None:
+    """fa_fwd with the linear bias -alibi_slopes[h] * |i - j| (alibi_slopes: H fp32 values
+    on the device)."""
+    B, H, N, d = _shape(q)
+    c, w = _window(causal, window)
+    s = default_scale(d) if scale is None else float(scale)
+    _check(_lib().fa_fwd_alibi(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, s, c,
+                               w, _ptr(alibi_slopes), _stream(stream)), "fa_fwd_alibi")
+
+
+def fa_bwd_alibi(q, k, v, o, do, lse, dq, dk, dv, workspace, alibi_slopes, scale=None,
+                 causal=False, window=(-1, -1), stream=None) -> None:
+    B, H, N, d = _shape(q)
+    c, w = _window(causal, window)
+    s = default_scale(d) if scale is None else float(scale)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib().fa_bwd_alibi(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
+                               _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, s, c, w,
+                               _ptr(alibi_slopes), _ptr(workspace), nbytes, _stream(stream)),
+           "fa_bwd_alibi")
 
 
 def fa_bwd_preprocess(o, do, lse, workspace, stream=None) -> None:
@@ -202,19 +229,33 @@ def _check_inputs(*ts):
             raise ValueError("q, k, v (and dO) must share one shape")
 
 
-def attention_forward(q, k, v, scale=None, causal=False, window=(-1, -1), stream=None):
-    """Returns (O, LSE) for bf16 CUDA tensors q, k, v of shape (B, H, N, d)."""
+def _check_slopes(alibi_slopes, q):
+    if not alibi_slopes.is_cuda or alibi_slopes.dtype != torch.float32:
+        raise ValueError("alibi_slopes must be an fp32 CUDA tensor")
+    if alibi_slopes.numel() != q.shape[1] or not alibi_slopes.is_contiguous():
+        raise ValueError("alibi_slopes must hold one slope per head, contiguous")
+
+
+def attention_forward(q, k, v, scale=None, causal=False, window=(-1, -1), stream=None,
+                      alibi_slopes=None):
+    """Returns (O, LSE) for bf16 CUDA tensors q, k, v of shape (B, H, N, d); with
+    alibi_slopes (H fp32 values), the scores carry the bias -alibi_slopes[h] * |i - j|."""
     _check_inputs(q, k, v)
     B, H, N, d = _shape(q)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    fa_fwd(q, k, v, o, lse, scale, causal, window, stream)
+    if alibi_slopes is None:
+        fa_fwd(q, k, v, o, lse, scale, causal, window, stream)
+    else:
+        _check_slopes(alibi_slopes, q)
+        fa_fwd_alibi(q, k, v, o, lse, alibi_slopes, scale, causal, window, stream)
     return o, lse
 
 
 def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, window=(-1, -1),
-                       stream=None):
-    """Returns (dQ, dK, dV): the gradient of <O, dO>; lse comes from attention_forward."""
+                       stream=None, alibi_slopes=None):
+    """Returns (dQ, dK, dV): the gradient of <O, dO>; lse comes from attention_forward
+    (with the same alibi_slopes)."""
     _check_inputs(q, k, v, o, do)
     B, H, N, d = _shape(q)
     dq = torch.empty_like(q)
@@ -222,5 +263,10 @@ def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, window=(-1
     dv = torch.empty_like(q)
     ws = torch.empty(max(1, fa_bwd_workspace_bytes(B, H, N, d)), dtype=torch.uint8,
                      device=q.device)
-    fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, scale, causal, window, stream)
+    if alibi_slopes is None:
+        fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, scale, causal, window, stream)
+    else:
+        _check_slopes(alibi_slopes, q)
+        fa_bwd_alibi(q, k, v, o, do, lse, dq, dk, dv, ws, alibi_slopes, scale, causal, window,
+                     stream)
     return dq, dk, dv

@@ -28,6 +28,7 @@ class Workload:
     backward: bool
     seed_index: int
     scale: float | None = None  # None: 1/sqrt(d)
+    alibi: bool = False         # linear bias -m_h |i - j| with the slopes of alibi_slopes()
 
     @property
     def softmax_scale(self) -> float:
@@ -78,4 +79,12 @@ WORKLOADS = {
     "c4": Workload("c4_causal_b32h16n2048d64", 32, 16, 2048, 64, True, (-1, -1), True, 3),
     "c5c": Workload("c5_causal_b2h32n8192d128", 2, 32, 8192, 128, True, (-1, -1), True, 4),
     "c5w": Workload("c5_window1024_b2h32n8192d128", 2, 32, 8192, 128, True, (1024, 0), True, 4),
+    # C4 with the ALiBi bias of the `alibi_slopes` parameter (page "告别OOM和训练慢…" §4.2)
+    "c4a": Workload("c4_causal_alibi_b32h16n2048d64", 32, 16, 2048, 64, True, (-1, -1), True, 3,
+                    alibi=True),
 }
+
+
+def alibi_slopes(H: int) -> list:
+    """The geometric ALiBi slopes 2^(-8 h / H), h = 1..H (one per head)."""
+    return [2.0 ** (-8.0 * (h + 1) / H) for h in range(H)]

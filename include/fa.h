@@ -118,6 +118,26 @@ fa_status_t fa_bwd(const void *q, const void *k, const void *v, const void *o,
                    void *stream);
 
 /*
+ * ALiBi: fa_fwd and fa_bwd with a linear bias. Page "告别OOM和训练慢…(含A100环境配置)" §4.2
+ * lists `alibi_slopes` among the parameters of flash_attn_fn and calls it a linear bias;
+ * the reading taken is that of ALiBi: head h has a slope m_h, and -m_h * |i - j| is added
+ * to the scaled score of query i and key j before masking and softmax (LSE includes it).
+ *   alibi_slopes: device pointer to H fp32 slopes, shared by all batch entries; 4-byte
+ *        aligned; not null (FA_ERR_INVALID_ARG). The slopes must be finite.
+ * All other arguments, layouts, errors and guarantees are those of fa_fwd / fa_bwd;
+ * fa_bwd_alibi needs the lse of fa_fwd_alibi with the same slopes.
+ */
+fa_status_t fa_fwd_alibi(const void *q, const void *k, const void *v, void *o, float *lse,
+                         int B, int H, int N, int d, float scale, int causal,
+                         fa_window_t window, const float *alibi_slopes, void *stream);
+
+fa_status_t fa_bwd_alibi(const void *q, const void *k, const void *v, const void *o,
+                         const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                         int B, int H, int N, int d, float scale, int causal,
+                         fa_window_t window, const float *alibi_slopes, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/*
  * Step 1 of fa_bwd alone: fills `workspace` (at least fa_bwd_workspace_bytes()) with
  * the per-row statistics the two passes read, each as B*H rows of Np = N rounded up to
  * 128 fp32 values (padding rows: +inf and 0):

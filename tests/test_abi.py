@@ -113,3 +113,25 @@ def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(fa, "LIBRARY", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="no fallback"):
         fa.library()
+
+
+def test_alibi_rejects_bad_arguments(lib):
+    def fwd_alibi(slopes=A, q=A, d=64, scale=0.125):
+        return lib.fa_fwd_alibi(q, A, A, A, A, 1, 2, 128, d, scale, 0, W(-1, -1), slopes, None)
+
+    def bwd_alibi(slopes=A, ws_bytes=1 << 20, dk=A):
+        return lib.fa_bwd_alibi(A, A, A, A, A, A, A, dk, A, 1, 2, 128, 64, 0.125, 0, W(-1, -1),
+                                slopes, A, ws_bytes, None)
+
+    assert fwd_alibi(slopes=None) == 1
+    assert fwd_alibi(slopes=A + 2) == 3
+    assert fwd_alibi(q=None) == 1
+    assert fwd_alibi(d=80) == 2
+    assert fwd_alibi(scale=0.0) == 1
+    assert bwd_alibi(slopes=None) == 1
+    assert bwd_alibi(slopes=A + 1) == 3
+    assert bwd_alibi(dk=None) == 1
+    assert bwd_alibi(ws_bytes=16) == 4
+    # an empty problem launches nothing, with or without slopes
+    assert lib.fa_fwd_alibi(None, None, None, None, None, 1, 2, 0, 64, 0.125, 0, W(-1, -1), None,
+                            None) == 0

@@ -8,7 +8,7 @@ import torch
 
 import gpu_helpers as G
 from exact_attention_126_b200 import fa, synth
-from exact_attention_126_b200.workloads import WORKLOADS
+from exact_attention_126_b200.workloads import WORKLOADS, alibi_slopes
 
 pytestmark = pytest.mark.gpu
 
@@ -69,9 +69,10 @@ def test_workload_full_size(name):
     the first, the last and two seeded random (batch, head) pairs (c4, c5)."""
     w = WORKLOADS[name]
     inp = inputs(w.B, w.H, w.N, w.d, w.seed_index)
-    out = G.run_library(inp, w.softmax_scale, w.causal, w.window, w.backward)
+    slopes = alibi_slopes(w.H) if w.alibi else None
+    out = G.run_library(inp, w.softmax_scale, w.causal, w.window, w.backward, slopes)
     heads = None if w.B * w.H * w.N <= 2 * 8 * 4096 else _sampled_heads(w)
-    errs = G.compare(inp, out, w.softmax_scale, w.causal, w.window, heads, w.backward)
+    errs = G.compare(inp, out, w.softmax_scale, w.causal, w.window, heads, w.backward, slopes)
     print(name, errs)
     G.assert_within_bounds(errs, name)
 
