@@ -39,7 +39,7 @@ L2_BYTES = 126 * 1024 * 1024
 # when its kernel changes. Compulsory traffic of the dK/dV pass on c4 is 537 MB read
 # (Q, K, V, dO and the row statistics) and 268 MB written (dK, dV).
 MEASURED_TRAFFIC = {
-    ("c4_causal_b32h16n2048d64", "bwd_dkdv"): 791226880,
+    ("c4_causal_b32h16n2048d64", "bwd_dkdv"): 792387840,
 }
 
 

@@ -578,10 +578,10 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) b4[e] = -slope2 * fabsf(base + (float)e);
           }
-          p[r] = ex2(fmaf(p[r], sl2, b4[0] - l4.x));
-          p[r + 1] = ex2(fmaf(p[r + 1], sl2, b4[1] - l4.y));
-          p[r + 2] = ex2(fmaf(p[r + 2], sl2, b4[2] - l4.z));
-          p[r + 3] = ex2(fmaf(p[r + 3], sl2, b4[3] - l4.w));
+          p[r] = ex2(fmaf(p[r], sl2, kAlibi ? b4[0] - l4.x : -l4.x));
+          p[r + 1] = ex2(fmaf(p[r + 1], sl2, kAlibi ? b4[1] - l4.y : -l4.y));
+          p[r + 2] = ex2(fmaf(p[r + 2], sl2, kAlibi ? b4[2] - l4.z : -l4.z));
+          p[r + 3] = ex2(fmaf(p[r + 3], sl2, kAlibi ? b4[3] - l4.w : -l4.w));
         }
         if (!tile_all_visible(i, j, mk)) {
           int r_lo, r_hi;
@@ -912,8 +912,8 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
           const float base = (float)((long long)jj * kBlock + NC * h - r);
 #pragma unroll
           for (int c = 0; c < NC; ++c) {
-            const float bias = kAlibi ? -slope2 * fabsf(base + (float)c) : 0.f;
-            p[c] = ex2(fmaf(p[c], sl2, bias - lse2));
+            const float arg = kAlibi ? -slope2 * fabsf(base + (float)c) - lse2 : -lse2;
+            p[c] = ex2(fmaf(p[c], sl2, arg));
           }
         }
         if (!tile_all_visible(i, jj, mk)) {

@@ -452,10 +452,22 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         }
         if (kAlibi) {
           // key minus query index at column 0 of the tile
-          const float base = (float)((long long)j * kBlock - row);
+          const long long kq = (long long)j * kBlock - row;
+          const float base = (float)kq;
+          // off the diagonal the distance is linear in the column: -m|k - q| is
+          // s2 * (base + c) with s2 = +m below it (keys before the query) and -m above
+          const bool below = __all_sync(0xffffffffu, kq + kBlock - 1 <= 0);
+          const bool above = __all_sync(0xffffffffu, kq >= 0);
+          if (below || above) {
+            const float s2 = below ? slope2 : -slope2;
+            const float c0 = s2 * base;
 #pragma unroll
-          for (int c = 0; c < kBlock; ++c)
-            x[c] = fmaf(x[c], sl2, -slope2 * fabsf(base + (float)c));
+            for (int c = 0; c < kBlock; ++c) x[c] = fmaf(x[c], sl2, fmaf(s2, (float)c, c0));
+          } else {
+#pragma unroll
+            for (int c = 0; c < kBlock; ++c)
+              x[c] = fmaf(x[c], sl2, -slope2 * fabsf(base + (float)c));
+          }
         }
         if (!tile_all_visible(rg.m, j, mk)) {
           int c_lo, c_hi;
