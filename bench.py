@@ -346,7 +346,8 @@ def run_ours(args, w, rank, world, local_rank):
         "data": "synthetic (seeded i.i.d. N(0,1) bf16, SplitMix64 + Box-Muller)",
         "config": {
             "workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
-            "window": list(w.window), "pass": "fwd+bwd" if w.backward else "fwd",
+            "window": list(w.window), "alibi": w.alibi,
+            "pass": "fwd+bwd" if w.backward else "fwd",
             "step_gflop": round(flops / 1e9, 3),
             "parallelism": "replicas" if world > 1 else "single",
             "l2": ("inputs larger than L2 (%d MB of inputs)" % (inputs_bytes >> 20))
@@ -442,7 +443,7 @@ def run_reference(args, w, rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded i.i.d. N(0,1) bf16 widened to fp64)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                   "causal": w.causal, "window": list(w.window),
+                   "causal": w.causal, "window": list(w.window), "alibi": w.alibi,
                    "pass": "fwd+bwd" if w.backward else "fwd"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": orc.num_threads(),
                          "kind": "oracle", "sample": sample},
