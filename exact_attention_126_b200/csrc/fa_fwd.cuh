@@ -11,15 +11,18 @@
 //   warp 10      TMA producer: Q_A, Q_B per item, then K_j and V_j through two rings of
 //                shared-memory stages (128-byte swizzle), guarded by full/empty mbarriers.
 //   warps 8, 9   MMA issuers (one thread each), for stream A and B: per key tile j,
-//                S_s = Q_s K_j^T, and O_s += P_s V_j once P_s is published; S_s of the
-//                next tile reuses the same TMEM columns once that product has completed.
+//                S_s = Q_s K_j^T, and O_s += P_s V_j once P_s is published. At head_dim 128
+//                P_s lies over S_s, so the next tile's S_s waits for that product; at
+//                head_dim 64 P_s has its own columns and the next S_s is issued one key tile
+//                ahead, as soon as the softmax has loaded S_s.
 //   warps 0..3   softmax of stream A, warps 4..7 of stream B: thread r owns query row r
 //                of its tile (TMEM lane r) and all 128 scores of it. Per key tile it
 //                updates the running max m and sum l (page "告别OOM和训练慢…" §2.2),
 //                rescales its row of O when m grew by more than 2^8 (exact: O and l carry
 //                the same stale m), and writes P = exp2(s*scale*log2e - m) in bf16 to
-//                TMEM, where the P V product reads it. The two streams take turns on the
-//                exponentials. At the end of an item it writes O / l and
+//                TMEM, where the P V product reads it (with ALiBi, the linear bias
+//                -m_h |i - j| joins every scaled score first). The two streams take turns
+//                on the exponentials. At the end of an item it writes O / l and
 //                LSE = ln2 * (m + log2 l).
 //
 // TMEM: S_A (128 columns), S_B (128), O_A (head_dim), O_B (head_dim), and for head_dim 64
