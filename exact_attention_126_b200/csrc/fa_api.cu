@@ -162,12 +162,8 @@ template <int D>
 fa_status_t launch_preprocess(const void* o, const void* dout, const float* lse, float* stats,
                               int BH, int N, cudaStream_t st) {
   const int Np = padded_rows(N);
-  const long long rows = (long long)BH * Np;
-  const long long rows_per_block = 8 * (32 / (D / 8));  // 8 warps
-  long long blocks = (rows + rows_per_block - 1) / rows_per_block;
-  const long long cap = (long long)sm_count() * 8;
-  if (blocks > cap) blocks = cap;
-  fa::fa_bwd_preprocess_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
+  const dim3 grid(Np / 64, BH);  // 64 rows per block; Np is a multiple of 128, BH <= 65535
+  fa::fa_bwd_preprocess_kernel<D><<<grid, 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, stats,
       BH, N, Np);
   return launched();

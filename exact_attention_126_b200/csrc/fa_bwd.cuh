@@ -43,43 +43,53 @@ namespace fa {
 // Row statistics of the backward, over B*H rows of Np (N rounded up to 128) entries:
 //   stats[bh*Np + r]             = LSE_r * log2(e)        (+inf for r >= N)
 //   stats[BH*Np + bh*Np + r]     = rowsum(dO_r * O_r)     (0 for r >= N), summed in fp32
-// G = D/8 lanes share a row, 16 bytes of O and dO per lane.
+// Block (x, bh) covers rows 64x .. 64x+63 of head bh, 8 rows per warp; G = D/8 lanes share
+// a row, 16 bytes of O and dO per lane, and a warp's loads for its 8 rows are all issued
+// before any is used.
 // ------------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256)
     fa_bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o,
                              const __nv_bfloat16* __restrict__ dout, const float* __restrict__ lse,
                              float* __restrict__ stats, int BH, int N, int Np) {
-  constexpr int G = D / 8;            // lanes per row
-  constexpr int kRowsPerWarp = 32 / G;
-  const long long rows = (long long)BH * Np;
+  constexpr int G = D / 8;                      // lanes per row
+  constexpr int kRowsPerPass = 32 / G;          // rows a warp covers per load
+  constexpr int kPasses = 8 / kRowsPerPass;     // 8 rows per warp
+  const int bh = blockIdx.y;
   const int lane = threadIdx.x & 31;
-  const long long warp_global = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const long long n_warps = ((long long)gridDim.x * blockDim.x) >> 5;
-  const int sub = lane / G;           // row within the warp's group
-  const int part = lane % G;          // 16-byte slice of the row
-  for (long long base = warp_global * kRowsPerWarp; base < rows; base += n_warps * kRowsPerWarp) {
-    const long long rp = base + sub;  // padded row
-    const long long bh = rp / Np;
-    const int r = (int)(rp - bh * Np);
-    const bool real = rp < rows && r < N;
-    const long long src = bh * N + r;
-    float acc = 0.f;
-    if (real) {
-      const uint4 a = *reinterpret_cast<const uint4*>(o + src * D + part * 8);
-      const uint4 b = *reinterpret_cast<const uint4*>(dout + src * D + part * 8);
-      const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
-      const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+  const int sub = lane / G;                     // row within the pass
+  const int part = lane % G;                    // 16-byte slice of the row
+  const int row0 = blockIdx.x * 64 + (threadIdx.x >> 5) * 8;
+  uint4 a[kPasses], b[kPasses];
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        acc = fmaf(__uint_as_float(aw[w] << 16), __uint_as_float(bw[w] << 16), acc);
-        acc = fmaf(__uint_as_float(aw[w] & 0xFFFF0000u), __uint_as_float(bw[w] & 0xFFFF0000u), acc);
-      }
+  for (int p = 0; p < kPasses; ++p) {
+    const int r = row0 + p * kRowsPerPass + sub;
+    if (r < N) {
+      const size_t src = ((size_t)bh * N + r) * D + part * 8;
+      a[p] = *reinterpret_cast<const uint4*>(o + src);
+      b[p] = *reinterpret_cast<const uint4*>(dout + src);
+    } else {
+      a[p] = make_uint4(0, 0, 0, 0);
+      b[p] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  const size_t rows = (size_t)BH * Np;
+#pragma unroll
+  for (int p = 0; p < kPasses; ++p) {
+    const uint32_t aw[4] = {a[p].x, a[p].y, a[p].z, a[p].w};
+    const uint32_t bw[4] = {b[p].x, b[p].y, b[p].z, b[p].w};
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      acc = fmaf(__uint_as_float(aw[w] << 16), __uint_as_float(bw[w] << 16), acc);
+      acc = fmaf(__uint_as_float(aw[w] & 0xFFFF0000u), __uint_as_float(bw[w] & 0xFFFF0000u), acc);
     }
 #pragma unroll
     for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (part == 0 && rp < rows) {
-      stats[rp] = real ? lse[src] * 1.4426950408889634f : INFINITY;
+    const int r = row0 + p * kRowsPerPass + sub;
+    if (part == 0 && r < Np) {
+      const size_t rp = (size_t)bh * Np + r;
+      stats[rp] = r < N ? lse[(size_t)bh * N + r] * kLog2e : INFINITY;
       stats[rows + rp] = acc;
     }
   }
