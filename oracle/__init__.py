@@ -33,6 +33,7 @@ def build(source: str = SOURCE, output: str = LIBRARY, force: bool = False) -> s
 
 
 _dptr = ctypes.POINTER(ctypes.c_double)
+_bptr = ctypes.POINTER(ctypes.c_ubyte)
 
 
 def _as_ptr(a: np.ndarray):
@@ -48,12 +49,12 @@ class Oracle:
         self.lib = ctypes.CDLL(path)
         L = ctypes.c_long
         self.lib.oracle_attention_fwd.argtypes = [
-            _dptr, _dptr, _dptr, L, L, L, L, ctypes.c_double, ctypes.c_int, L, L, _dptr, _dptr,
-            _dptr]
+            _dptr, _dptr, _dptr, L, L, L, L, ctypes.c_double, ctypes.c_int, L, L, _dptr, _bptr,
+            _dptr, _dptr]
         self.lib.oracle_attention_fwd.restype = ctypes.c_int
         self.lib.oracle_attention_bwd.argtypes = [
             _dptr, _dptr, _dptr, _dptr, L, L, L, L, ctypes.c_double, ctypes.c_int, L, L, _dptr,
-            _dptr, _dptr, _dptr]
+            _bptr, _dptr, _dptr, _dptr]
         self.lib.oracle_attention_bwd.restype = ctypes.c_int
         self.lib.oracle_num_threads.restype = ctypes.c_int
 
@@ -77,21 +78,34 @@ class Oracle:
             raise ValueError("alibi_slopes must hold one slope per head")
         return a, _as_ptr(a)
 
-    def fwd(self, q, k, v, scale, causal=False, window=(-1, -1), alibi=None):
-        """Returns (O, LSE) in fp64 for (B, H, N, d) inputs; `alibi`: H slopes or None."""
+    @staticmethod
+    def _padding(key_padding, B, N):
+        if key_padding is None:
+            return None, None
+        a = np.ascontiguousarray(key_padding, dtype=np.uint8)
+        if a.shape != (B, N):
+            raise ValueError("key_padding must be a (B, N) array of flags")
+        return a, a.ctypes.data_as(_bptr)
+
+    def fwd(self, q, k, v, scale, causal=False, window=(-1, -1), alibi=None, key_padding=None):
+        """Returns (O, LSE) in fp64 for (B, H, N, d) inputs; `alibi`: H slopes or None;
+        `key_padding`: (B, N) flags, True for a padded key, or None."""
         q, k, v = self._prep(q, k, v)
         B, H, N, d = q.shape
         o = np.empty_like(q)
         lse = np.empty((B, H, N), dtype=np.float64)
         keep, slopes = self._slopes(alibi, H)
+        keep_pad, pad = self._padding(key_padding, B, N)
         rc = self.lib.oracle_attention_fwd(_as_ptr(q), _as_ptr(k), _as_ptr(v), B, H, N, d,
                                            float(scale), int(bool(causal)), int(window[0]),
-                                           int(window[1]), slopes, _as_ptr(o), _as_ptr(lse))
+                                           int(window[1]), slopes, pad, _as_ptr(o),
+                                           _as_ptr(lse))
         if rc != 0:
             raise RuntimeError("oracle_attention_fwd failed with %d" % rc)
         return o, lse
 
-    def bwd(self, q, k, v, do, scale, causal=False, window=(-1, -1), alibi=None):
+    def bwd(self, q, k, v, do, scale, causal=False, window=(-1, -1), alibi=None,
+            key_padding=None):
         """Returns (dQ, dK, dV) in fp64: the gradient of <O, dO> for (B, H, N, d) inputs."""
         q, k, v, do = self._prep(q, k, v, do)
         B, H, N, d = q.shape
@@ -99,9 +113,10 @@ class Oracle:
         dk = np.empty_like(q)
         dv = np.empty_like(q)
         keep, slopes = self._slopes(alibi, H)
+        keep_pad, pad = self._padding(key_padding, B, N)
         rc = self.lib.oracle_attention_bwd(_as_ptr(q), _as_ptr(k), _as_ptr(v), _as_ptr(do),
                                            B, H, N, d, float(scale), int(bool(causal)),
-                                           int(window[0]), int(window[1]), slopes,
+                                           int(window[0]), int(window[1]), slopes, pad,
                                            _as_ptr(dq), _as_ptr(dk), _as_ptr(dv))
         if rc != 0:
             raise RuntimeError("oracle_attention_bwd failed with %d" % rc)

@@ -16,7 +16,10 @@
  *          `alibi_slopes` of `flash_attn_fn`, page "告别OOM和训练慢…" §4.2)
  *   S_ij = -inf where key j is not visible from query i (causal: "mask future
  *          positions", page "Flash Attention 3.7 核心原理与实战" §3.2; sliding window
- *          `window_size=(left,right)`, page "告别OOM和训练慢…" §4.2)
+ *          `window_size=(left,right)`, page "告别OOM和训练慢…" §4.2), and where key j of
+ *          the batch entry is padding (`key_padding_mask`, True = padded, applied with
+ *          masked_fill(-inf) to every head and query: page "PyTorch-CUDA-v2.9镜像…", the
+ *          MultiheadAttention replacement)
  *   P = row-softmax(S), with the row maximum subtracted first (`safe_softmax`,
  *       page "告别OOM和训练慢…" §2.2)
  *   O = P V
@@ -72,10 +75,11 @@ static double head_slope(const double *alibi_slopes, long bh, long H)
 }
 
 /* P (N x N) := softmax rows of the masked, scaled (and biased, when slope != 0) scores of
- * one head; lse (N). */
+ * one head; lse (N). kpad: N flags of the head's batch entry (nonzero = padded key), or
+ * NULL. */
 static void head_probabilities(const double *q, const double *k, long N, long d,
                                double scale, double slope, long left, long right,
-                               double *P, double *lse)
+                               const unsigned char *kpad, double *P, double *lse)
 {
     long i;
 #pragma omp parallel for schedule(static)
@@ -89,6 +93,7 @@ static void head_probabilities(const double *q, const double *k, long N, long d,
             s *= scale;
             s += -slope * fabs((double)(i - j));
             if (!visible(i, j, left, right)) s = -INFINITY;
+            if (kpad && kpad[j]) s = -INFINITY;
             Pi[j] = s;
             if (s > m) m = s;
         }
@@ -107,11 +112,19 @@ static void head_probabilities(const double *q, const double *k, long N, long d,
     }
 }
 
-/* alibi_slopes: H slopes, or NULL for no bias. */
+/* The key-padding flags of head bh's batch entry (B*H heads, heads fastest), or NULL. */
+static const unsigned char *head_padding(const unsigned char *key_padding, long bh, long H,
+                                         long N)
+{
+    return key_padding ? key_padding + (bh / H) * N : NULL;
+}
+
+/* alibi_slopes: H slopes, or NULL for no bias; key_padding: B x N flags (nonzero = padded
+ * key), or NULL for none. */
 int oracle_attention_fwd(const double *q, const double *k, const double *v,
                          long B, long H, long N, long d, double scale,
                          int causal, long left, long right, const double *alibi_slopes,
-                         double *o, double *lse)
+                         const unsigned char *key_padding, double *o, double *lse)
 {
     long bh;
     if (B < 0 || H < 0 || N < 0 || d < 1) return 1;
@@ -122,8 +135,8 @@ int oracle_attention_fwd(const double *q, const double *k, const double *v,
         const double *qh = q + bh * N * d, *kh = k + bh * N * d, *vh = v + bh * N * d;
         double *oh = o + bh * N * d;
         long i;
-        head_probabilities(qh, kh, N, d, scale, head_slope(alibi_slopes, bh, H), left, right, P,
-                           lse + bh * N);
+        head_probabilities(qh, kh, N, d, scale, head_slope(alibi_slopes, bh, H), left, right,
+                           head_padding(key_padding, bh, H, N), P, lse + bh * N);
         /* O = P V */
 #pragma omp parallel for schedule(static)
         for (i = 0; i < N; ++i) {
@@ -143,6 +156,7 @@ int oracle_attention_bwd(const double *q, const double *k, const double *v,
                          const double *dout,
                          long B, long H, long N, long d, double scale,
                          int causal, long left, long right, const double *alibi_slopes,
+                         const unsigned char *key_padding,
                          double *dq, double *dk, double *dv)
 {
     long bh;
@@ -162,8 +176,8 @@ int oracle_attention_bwd(const double *q, const double *k, const double *v,
         const double *doh = dout + bh * N * d;
         double *dqh = dq + bh * N * d, *dkh = dk + bh * N * d, *dvh = dv + bh * N * d;
         long i, j;
-        head_probabilities(qh, kh, N, d, scale, head_slope(alibi_slopes, bh, H), left, right, P,
-                           lse);
+        head_probabilities(qh, kh, N, d, scale, head_slope(alibi_slopes, bh, H), left, right,
+                           head_padding(key_padding, bh, H, N), P, lse);
         /* dV = P^T dO */
 #pragma omp parallel for schedule(static)
         for (j = 0; j < N; ++j) {

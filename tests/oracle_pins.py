@@ -17,6 +17,13 @@ Sources of the facts:
   * torch's fp64 CPU scaled_dot_product_attention and autograd, as an independent
     library implementation of the same definition.
 
+The key-padding pins (`key_padding_mask`, True = padded key, masked_fill(-inf) on every head
+and query: page "PyTorch-CUDA-v2.9镜像中使用FlashAttention提升训练速度", the MultiheadAttention
+replacement) use: no flags set is no mask at all; padded keys' K and V rows do not matter and
+get zero gradients; a single unpadded key is returned exactly; a fully padded batch entry
+gives O = 0, LSE = -inf and zero gradients; finite differences; torch's SDPA with the combined
+boolean mask.
+
 The ALiBi pins (linear bias -m_h |i - j| on the scaled scores, the `alibi_slopes` parameter
 of page "告别OOM和训练慢…(含A100环境配置)" §4.2) use the same kinds of facts: closed forms
 where the scores are the bias alone, the limit of a bias so steep that each row sees only
@@ -361,6 +368,133 @@ def pin_alibi_library_sdpa(orc):
         np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=1e-11, atol=1e-11)
 
 
+def _padding(B, N, seed):
+    """Seeded key-padding flags with key 0 of every batch entry unpadded (so that every row,
+    causal ones included, sees at least one key), about a third of the rest padded."""
+    r = _rng(seed)
+    pad = r.random((B, N)) < 0.35
+    pad[:, 0] = False
+    return pad
+
+
+def pin_padding_none_set(orc):
+    """All flags False is no padding at all: bit-identical results in every mode."""
+    r = _rng(21)
+    q, k, v, do = (r.standard_normal((2, 2, 9, 3)) for _ in range(4))
+    none = np.zeros((2, 9), dtype=bool)
+    for causal, window in MODES:
+        a = orc.fwd(q, k, v, 0.7, causal, window)
+        b = orc.fwd(q, k, v, 0.7, causal, window, key_padding=none)
+        ga = orc.bwd(q, k, v, do, 0.7, causal, window)
+        gb = orc.bwd(q, k, v, do, 0.7, causal, window, key_padding=none)
+        for x, y in zip(a + ga, b + gb):
+            assert np.array_equal(x, y)
+
+
+def pin_padding_keys_do_not_matter(orc):
+    """Changing the K and V rows of padded keys changes nothing; their dK and dV are 0."""
+    r = _rng(22)
+    B, H, N, d = 2, 2, 11, 4
+    q, k, v, do = (r.standard_normal((B, H, N, d)) for _ in range(4))
+    pad = _padding(B, N, 23)
+    k2, v2 = k.copy(), v.copy()
+    k2[pad[:, None, :, None].repeat(H, 1).repeat(d, 3)] += 5.0
+    v2[pad[:, None, :, None].repeat(H, 1).repeat(d, 3)] -= 3.0
+    for causal, window in MODES:
+        o, lse = orc.fwd(q, k, v, 0.5, causal, window, key_padding=pad)
+        o2, lse2 = orc.fwd(q, k2, v2, 0.5, causal, window, key_padding=pad)
+        np.testing.assert_allclose(o2, o, rtol=1e-13, atol=1e-13)
+        np.testing.assert_allclose(lse2, lse, rtol=1e-13, atol=1e-13)
+        dq, dk, dv = orc.bwd(q, k, v, do, 0.5, causal, window, key_padding=pad)
+        dq2, _, _ = orc.bwd(q, k2, v2, do, 0.5, causal, window, key_padding=pad)
+        np.testing.assert_allclose(dq2, dq, rtol=1e-12, atol=1e-12)
+        for b in range(B):
+            assert np.all(dk[b][:, pad[b]] == 0.0) and np.all(dv[b][:, pad[b]] == 0.0)
+
+
+def pin_padding_single_key(orc):
+    """Only key 0 unpadded: a row that sees key 0 returns v_0 with LSE = scale q_i . k_0;
+    a row that does not (a window that ends before it) has O = 0 and LSE = -inf."""
+    r = _rng(24)
+    B, H, N, d = 1, 2, 7, 3
+    q, k, v = (r.standard_normal((B, H, N, d)) for _ in range(3))
+    pad = np.ones((B, N), dtype=bool)
+    pad[:, 0] = False
+    for causal, window in MODES:
+        o, lse = orc.fwd(q, k, v, 0.9, causal, window, key_padding=pad)
+        for i in range(N):
+            _, lo, hi = _visible_count(i, N, causal, window)
+            if lo <= 0 <= hi:
+                np.testing.assert_allclose(o[0, :, i], v[0, :, 0], rtol=1e-14, atol=1e-15)
+                np.testing.assert_allclose(lse[0, :, i], 0.9 * np.sum(q[0, :, i] * k[0, :, 0], -1),
+                                           rtol=1e-14, atol=1e-14)
+            else:
+                assert np.all(o[0, :, i] == 0.0) and np.all(lse[0, :, i] == -np.inf)
+
+
+def pin_padding_whole_entry(orc):
+    """A batch entry whose every key is padded: O = 0, LSE = -inf and zero gradients for it,
+    while the other entry is untouched by the flags of this one."""
+    r = _rng(25)
+    q, k, v, do = (r.standard_normal((2, 2, 6, 3)) for _ in range(4))
+    pad = np.zeros((2, 6), dtype=bool)
+    pad[1] = True
+    o, lse = orc.fwd(q, k, v, 0.5, False, (-1, -1), key_padding=pad)
+    dq, dk, dv = orc.bwd(q, k, v, do, 0.5, False, (-1, -1), key_padding=pad)
+    assert np.all(o[1] == 0.0) and np.all(lse[1] == -np.inf)
+    assert np.all(dq[1] == 0.0) and np.all(dk[1] == 0.0) and np.all(dv[1] == 0.0)
+    o0, lse0 = orc.fwd(q[:1], k[:1], v[:1], 0.5)
+    np.testing.assert_array_equal(o[0], o0[0])
+    np.testing.assert_array_equal(lse[0], lse0[0])
+
+
+def pin_padding_finite_differences(orc):
+    """With padded keys, the backward is still the gradient of L = <O, dO>."""
+    r = _rng(26)
+    B, H, N, d = 2, 1, 5, 2
+    q, k, v, do = (r.standard_normal((B, H, N, d)) for _ in range(4))
+    pad = np.array([[False, True, False, False, True], [False, False, True, True, False]])
+    scale, eps = 0.6, 1e-6
+    for causal, window in MODES[:3]:
+        grads = orc.bwd(q, k, v, do, scale, causal, window, key_padding=pad)
+        for which in range(3):
+            num = np.zeros_like(q)
+            for idx in np.ndindex(q.shape):
+                args = [q.copy(), k.copy(), v.copy()]
+                args[which][idx] += eps
+                lp = np.sum(orc.fwd(*args, scale, causal, window, key_padding=pad)[0] * do)
+                args[which][idx] -= 2 * eps
+                lm = np.sum(orc.fwd(*args, scale, causal, window, key_padding=pad)[0] * do)
+                num[idx] = (lp - lm) / (2 * eps)
+            np.testing.assert_allclose(grads[which], num, rtol=1e-6, atol=1e-7)
+
+
+def pin_padding_library_sdpa(orc):
+    """torch's fp64 SDPA with the band mask and the padding combined into one boolean mask
+    (and autograd through it) gives the same O, LSE and gradients."""
+    r = _rng(27)
+    B, H, N, d = 2, 2, 15, 5
+    q, k, v, do = (r.standard_normal((B, H, N, d)) for _ in range(4))
+    pad = _padding(B, N, 28)
+    scale = 0.4
+    keep = torch.tensor(~pad)[:, None, None, :]
+    for causal, window in MODES:
+        mask = _band_mask(N, causal, window)[None, None] & keep
+        tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+        to = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask,
+                                                              scale=scale)
+        to.backward(torch.tensor(do))
+        scores = (torch.tensor(q) @ torch.tensor(k).transpose(-1, -2)) * scale
+        tlse = torch.logsumexp(scores.masked_fill(~mask, float("-inf")), dim=-1)
+        o, lse = orc.fwd(q, k, v, scale, causal, window, key_padding=pad)
+        dq, dk, dv = orc.bwd(q, k, v, do, scale, causal, window, key_padding=pad)
+        np.testing.assert_allclose(o, to.detach().numpy(), rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(lse, tlse.numpy(), rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=1e-11, atol=1e-11)
+        np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=1e-11, atol=1e-11)
+        np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=1e-11, atol=1e-11)
+
+
 def pin_self_similarity(orc):
     """k = v = q (the page "显存神技：必学FlashAttention！" comparison input): each row's own
     key has the largest score |q_i|^2 scale among keys of no larger norm, so O is finite,
@@ -391,4 +525,10 @@ ALL_PINS = [
     pin_alibi_zero_slopes,
     pin_alibi_finite_differences,
     pin_alibi_library_sdpa,
+    pin_padding_none_set,
+    pin_padding_keys_do_not_matter,
+    pin_padding_single_key,
+    pin_padding_whole_entry,
+    pin_padding_finite_differences,
+    pin_padding_library_sdpa,
 ]

@@ -34,6 +34,12 @@ PLANTS = [
      "s += -slope * scale * fabs((double)(i - j));"),
     ("ALiBi slope of the wrong head", "return alibi_slopes ? alibi_slopes[bh % H] : 0.0;",
      "return alibi_slopes ? alibi_slopes[0] : 0.0;"),
+    ("key padding ignored", "if (kpad && kpad[j]) s = -INFINITY;", "if (0) s = -INFINITY;"),
+    ("key padding applied by query", "if (kpad && kpad[j]) s = -INFINITY;",
+     "if (kpad && kpad[i]) s = -INFINITY;"),
+    ("key padding of the first batch entry for all",
+     "return key_padding ? key_padding + (bh / H) * N : NULL;",
+     "return key_padding ? key_padding : NULL;"),
 ]
 
 
