@@ -35,12 +35,40 @@ L2_BYTES = 126 * 1024 * 1024
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a kernel on a
-# workload, from one ncu capture of the kernels as they are now; an entry must be removed
-# when its kernel changes. Compulsory traffic of the dK/dV pass on c4 is 537 MB read
-# (Q, K, V, dO and the row statistics) and 268 MB written (dK, dV).
-MEASURED_TRAFFIC = {
-    ("c4_causal_b32h16n2048d64", "bwd_dkdv"): 792387840,
-}
+# workload, from one ncu capture, keyed by the SHA-256 of the kernel sources the capture
+# ran (kernel_source_hash()); an entry whose hash no longer matches is reported as null.
+MEASURED_TRAFFIC = {}
+
+
+def kernel_source_hash() -> str:
+    """SHA-256 (first 12 hex digits) of the CUDA sources of the library."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_attention_126_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:12]
+
+
+def measured_traffic(workload: str, kernel: str):
+    """(bytes per launch, source) from MEASURED_TRAFFIC if it was taken on these sources."""
+    entry = MEASURED_TRAFFIC.get((workload, kernel))
+    if entry is None or entry[1] != kernel_source_hash():
+        return None, None
+    return entry[0], entry[2]
+
+
+def roofline_peak(peaks, region_ms: float):
+    """The bf16 peak a kernel timed inside a region of `region_ms` is held to: the burst
+    figure (cuBLAS timed alone, full boost clock) for regions under a second, the sustained
+    figure (a seconds-long loop under the power cap) for longer ones."""
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    if region_ms < 1000.0:
+        return burst, "burst", sustained
+    return sustained, "sustained", sustained
 
 
 def load_peaks():
@@ -141,10 +169,144 @@ def job_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
 
 
 # ------------------------------------------------------------------------- our arm
+KERNEL_NAMES = ["fwd", "bwd_preprocess", "bwd_dkdv", "bwd_dq"]
+
+
+class Problem:
+    """Device buffers of one workload and the library calls of one step.
+
+    A step is the training path: the forward keeps O - bf16(O) (fa_options_t.o_low) and
+    the backward's three phases form delta from it; with ALiBi the slopes ride in the same
+    options. Each phase is its own C-ABI call, so CUDA events can sit between kernels."""
+
+    def __init__(self, w, dev, host=None, seed=0):
+        import torch
+        from exact_attention_126_b200 import fa, workloads
+        self.w, self.dev, self.fa = w, dev, fa
+        B, H, N, d = w.B, w.H, w.N, w.d
+        shape = (B, H, N, d)
+        if host is not None:
+            self.q, self.k, self.v, self.do = (host[n].to(dev, non_blocking=True)
+                                               for n in ("q", "k", "v", "do"))
+        else:
+            # i.i.d. N(0, 1) drawn on the device from a seeded generator (timing only: the
+            # values' distribution is the workload's, their bits are not the oracle's)
+            g = torch.Generator(device=dev)
+            g.manual_seed(seed)
+            self.q, self.k, self.v, self.do = (
+                torch.randn(shape, generator=g, device=dev, dtype=torch.float32)
+                .to(torch.bfloat16) for _ in range(4))
+        self.o = torch.empty_like(self.q)
+        self.o_low = torch.empty_like(self.q)
+        self.lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        self.dq, self.dk, self.dv = (torch.empty_like(self.q) for _ in range(3))
+        self.ws = torch.empty(max(1, fa.fa_bwd_workspace_bytes(B, H, N, d)), dtype=torch.uint8,
+                              device=dev)
+        self.slopes = None
+        if w.alibi:
+            self.slopes = torch.tensor(workloads.alibi_slopes(H), dtype=torch.float32,
+                                       device=dev)
+        self.opt = fa.options(alibi_slopes=self.slopes, o_low=self.o_low)
+        self.launches = 4 if w.backward else 1
+
+    def step(self, sp, evs=None):
+        """One pass of the path on stream handle `sp`; evs: len(KERNEL_NAMES) + 1 events
+        (only the first two with a forward-only workload), recorded between kernels."""
+        fa, w = self.fa, self.w
+        stream = self.stream
+        if evs is not None:
+            evs[0].record(stream)
+        fa.fa_fwd_ex(self.q, self.k, self.v, self.o, self.lse, self.opt, w.softmax_scale,
+                     w.causal, w.window, sp)
+        if evs is not None:
+            evs[1].record(stream)
+        if not w.backward:
+            return
+        fa.fa_bwd_preprocess(self.o, self.do, self.lse, self.ws, self.opt, sp)
+        if evs is not None:
+            evs[2].record(stream)
+        fa.fa_bwd_dkdv(self.q, self.k, self.v, self.do, self.ws, self.dk, self.dv,
+                       w.softmax_scale, w.causal, w.window, sp, self.opt)
+        if evs is not None:
+            evs[3].record(stream)
+        fa.fa_bwd_dq(self.q, self.k, self.v, self.do, self.ws, self.dq, w.softmax_scale,
+                     w.causal, w.window, sp, self.opt)
+        if evs is not None:
+            evs[4].record(stream)
+
+    def time(self, steps, warmup, stream, clocks=None):
+        """Device time of `steps` steps after `warmup` untimed ones: (ms per step, per-kernel
+        ms per step, bracket ms). L2 is flushed before every step when the inputs fit in it."""
+        import torch
+        self.stream = stream
+        sp = stream.cuda_stream
+        w = self.w
+        flush = None
+        if 4 * w.tensor_bytes() <= L2_BYTES:
+            flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=self.dev)
+        self.flushed = flush is not None
+        for _ in range(warmup):
+            if flush is not None:
+                flush.zero_()
+            self.step(sp)
+        torch.cuda.synchronize(self.dev)
+        if self.fa.fa_debug_status(sp) != 0:
+            raise RuntimeError("a kernel abandoned a bounded wait during warm-up")
+        n_ev = len(KERNEL_NAMES) + 1 if w.backward else 2
+        events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+                  for _ in range(steps)]
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(self.dev)
+        t0.record(stream)
+        for s in range(steps):
+            if flush is not None:
+                flush.zero_()
+            self.step(sp, events[s])
+        t1.record(stream)
+        torch.cuda.synchronize(self.dev)
+        if self.fa.fa_debug_status(sp) != 0:
+            raise RuntimeError("a kernel abandoned a bounded wait in the timed region")
+        names = KERNEL_NAMES[: n_ev - 1]
+        per_kernel = {n: 0.0 for n in names}
+        step_ms = 0.0
+        for evs in events:
+            step_ms += evs[0].elapsed_time(evs[-1])
+            for i, n in enumerate(names):
+                per_kernel[n] += evs[i].elapsed_time(evs[i + 1])
+        bracket = t0.elapsed_time(t1)
+        ms = step_ms / steps if flush is not None else bracket / steps
+        return ms, {n: t / steps for n, t in per_kernel.items()}, bracket
+
+
+def kernel_flops(w):
+    """Algorithmic flops credited to each kernel (the metric's convention): forward = the
+    forward count; dK/dV = 2x (S^T, dP^T, dV, dK products); dQ = 0.5x (its dQ product;
+    the recomputation of S and dP is not credited)."""
+    f = w.fwd_flops()
+    return {"fwd": f, "bwd_preprocess": 0.0, "bwd_dkdv": 2.0 * f, "bwd_dq": 0.5 * f}
+
+
+def workload_line(w, ms, per_kernel, flushed):
+    """The summary of one workload's timing: ms, TFLOP/s, and the shares of its kernels."""
+    value = w.step_flops() / (ms * 1e-3) / 1e12
+    kf = kernel_flops(w)
+    kernels = {}
+    for n, t in per_kernel.items():
+        kernels[n] = {"ms": round(t, 5), "share": round(t / sum(per_kernel.values()), 4),
+                      "algorithmic_tflops": round(kf[n] / (t * 1e-3) / 1e12, 2) if kf[n] else None}
+    return {"workload": w.name, "pass": "fwd+bwd" if w.backward else "fwd",
+            "ms_per_step": round(ms, 5), "tflops": round(value, 2),
+            "pct_of_dense_peak": round(100 * value / DATASHEET_BF16_TFLOPS, 2),
+            "step_gflop": round(w.step_flops() / 1e9, 3), "kernels": kernels,
+            "l2": "L2 flushed before every timed step" if flushed else "inputs larger than L2"}
+
+
 def run_ours(args, w, rank, world, local_rank):
     import torch
 
-    from exact_attention_126_b200 import build, fa, synth, workloads
+    from exact_attention_126_b200 import build, fa, synth
+    from exact_attention_126_b200.workloads import WORKLOADS
 
     build.build()
     torch.cuda.set_device(local_rank)
@@ -157,128 +319,46 @@ def run_ours(args, w, rank, world, local_rank):
                                 device_id=dev)
 
     inp_host = synth.attention_inputs(w.B, w.H, w.N, w.d, w.seed_index, with_grad=True, pin=True)
-    q, k, v, do = (inp_host[n].to(dev, non_blocking=True) for n in ("q", "k", "v", "do"))
-    B, H, N, d = w.B, w.H, w.N, w.d
-    o = torch.empty_like(q)
-    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
-    ws = torch.empty(fa.fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
-    scale = w.softmax_scale
-    slopes = None
-    if w.alibi:
-        slopes = torch.tensor(workloads.alibi_slopes(H), dtype=torch.float32, device=dev)
+    prob = Problem(w, dev, host=inp_host)
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
-    inputs_bytes = 4 * w.tensor_bytes()
-    flush = None
-    if inputs_bytes <= L2_BYTES:
-        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
 
-    def step(evs=None):
-        # fa_fwd, then the three phases of fa_bwd, with optional events between kernels;
-        # with ALiBi, fa_fwd_alibi and fa_bwd_alibi (the backward timed as one)
-        if evs is not None:
-            evs[0].record(stream)
-        if w.alibi:
-            fa.fa_fwd_alibi(q, k, v, o, lse, slopes, scale, w.causal, w.window, sp)
-            if evs is not None:
-                evs[1].record(stream)
-            if w.backward:
-                fa.fa_bwd_alibi(q, k, v, o, do, lse, dq, dk, dv, ws, slopes, scale, w.causal,
-                                w.window, sp)
-                if evs is not None:
-                    evs[2].record(stream)
-            return
-        fa.fa_fwd(q, k, v, o, lse, scale, w.causal, w.window, sp)
-        if evs is not None:
-            evs[1].record(stream)
-        if w.backward:
-            fa.fa_bwd_preprocess(o, do, lse, ws, sp)
-            if evs is not None:
-                evs[2].record(stream)
-            fa.fa_bwd_dkdv(q, k, v, do, ws, dk, dv, scale, w.causal, w.window, sp)
-            if evs is not None:
-                evs[3].record(stream)
-            fa.fa_bwd_dq(q, k, v, do, ws, dq, scale, w.causal, w.window, sp)
-            if evs is not None:
-                evs[4].record(stream)
-
-    n_ev = (3 if w.alibi else 5) if w.backward else 2
-    launches_per_step = 4 if w.backward else 1
-
-    for _ in range(args.warmup):
-        if flush is not None:
-            flush.zero_()
-        step()
-    torch.cuda.synchronize(dev)
-    if fa.fa_debug_status(sp) != 0:
-        raise RuntimeError("a kernel abandoned a bounded wait during warm-up")
-
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
-              for _ in range(args.steps)]
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local_rank) as clocks:
-        t_start = torch.cuda.Event(enable_timing=True)
-        t_end = torch.cuda.Event(enable_timing=True)
-        t_start.record(stream)
-        for s in range(args.steps):
-            if flush is not None:
-                flush.zero_()
-            step(events[s])
-        t_end.record(stream)
-        torch.cuda.synchronize(dev)
+        ms_per_step, per_kernel, bracket_ms = prob.time(args.steps, args.warmup, stream)
     if dist is not None:
         dist.barrier()
-    if fa.fa_debug_status(sp) != 0:
-        raise RuntimeError("a kernel abandoned a bounded wait in the timed region")
-
-    # device time of the K steps (flushes excluded), and per kernel
-    names = (["fwd", "bwd"] if w.alibi else ["fwd", "bwd_preprocess", "bwd_dkdv", "bwd_dq"])[
-        : n_ev - 1]
-    per_kernel = {n: 0.0 for n in names}
-    step_ms = 0.0
-    for evs in events:
-        step_ms += evs[0].elapsed_time(evs[-1])
-        for i, n in enumerate(names):
-            per_kernel[n] += evs[i].elapsed_time(evs[i + 1])
-    bracket_ms = t_start.elapsed_time(t_end)
-    ms_per_step = step_ms / args.steps
-    if flush is None:
-        ms_per_step = bracket_ms / args.steps  # nothing but the steps in the bracket
-
-    if dist is not None:
         ms_per_step = max_over_ranks(ms_per_step, dist, dev)
 
     # ---------------------------------------------------------------- end to end
+    # The public call a user makes (attention_forward / attention_backward: the same
+    # training path, with their own output allocations), inputs copied from pinned host
+    # memory and every output read back, each step.
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    q, k, v, do = prob.q, prob.k, prob.v, prob.do
     host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-                for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
-    h2d_bytes = sum(inp_host[n].numel() * inp_host[n].element_size() for n in ("q", "k", "v", "do"))
-    d2h_bytes = sum(t.numel() * t.element_size() for t in host_out.values())
-    if not w.backward:
-        h2d_bytes = sum(inp_host[n].numel() * inp_host[n].element_size() for n in ("q", "k", "v"))
-        d2h_bytes = sum(host_out[n].numel() * host_out[n].element_size() for n in ("o", "lse"))
+                for n, t in (("o", prob.o), ("lse", prob.lse), ("dq", prob.dq),
+                             ("dk", prob.dk), ("dv", prob.dv))}
+    in_names = ("q", "k", "v", "do") if w.backward else ("q", "k", "v")
+    out_names = ("o", "lse", "dq", "dk", "dv") if w.backward else ("o", "lse")
+    h2d_bytes = sum(inp_host[n].numel() * inp_host[n].element_size() for n in in_names)
+    d2h_bytes = sum(host_out[n].numel() * host_out[n].element_size() for n in out_names)
 
     def e2e_step():
-        q.copy_(inp_host["q"], non_blocking=True)
-        k.copy_(inp_host["k"], non_blocking=True)
-        v.copy_(inp_host["v"], non_blocking=True)
+        for n, t in zip(("q", "k", "v", "do"), (q, k, v, do)):
+            if n in in_names:
+                t.copy_(inp_host[n], non_blocking=True)
+        res = fa.attention_forward(q, k, v, w.softmax_scale, w.causal, w.window, sp,
+                                   alibi_slopes=prob.slopes, keep_residual=w.backward)
+        host_out["o"].copy_(res[0], non_blocking=True)
+        host_out["lse"].copy_(res[1], non_blocking=True)
         if w.backward:
-            do.copy_(inp_host["do"], non_blocking=True)
-        if w.alibi:
-            fa.fa_fwd_alibi(q, k, v, o, lse, slopes, scale, w.causal, w.window, sp)
-        else:
-            fa.fa_fwd(q, k, v, o, lse, scale, w.causal, w.window, sp)
-        host_out["o"].copy_(o, non_blocking=True)
-        host_out["lse"].copy_(lse, non_blocking=True)
-        if w.backward:
-            dqq, dkk, dvv = fa.attention_backward(q, k, v, o, lse, do, scale, w.causal, w.window, sp,
-                                                  alibi_slopes=slopes)
-            host_out["dq"].copy_(dqq, non_blocking=True)
-            host_out["dk"].copy_(dkk, non_blocking=True)
-            host_out["dv"].copy_(dvv, non_blocking=True)
+            grads = fa.attention_backward(q, k, v, res[0], res[1], do, w.softmax_scale, w.causal,
+                                          w.window, sp, alibi_slopes=prob.slopes, o_low=res[2])
+            for n, t in zip(("dq", "dk", "dv"), grads):
+                host_out[n].copy_(t, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize(dev)
@@ -294,6 +374,27 @@ def run_ours(args, w, rank, world, local_rank):
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
     if dist is not None:
         e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+    del prob
+
+    # ---------------------------------------------------------------- other workloads
+    # The other configurations at full size (rank 0 only, after the headline and its
+    # end-to-end run; each its own warm-up and timed steps).
+    others = {}
+    if rank == 0 and not args.no_workloads:
+        for name in args.also:
+            if WORKLOADS[name].name == w.name:
+                continue
+            ow = WORKLOADS[name]
+            op = Problem(ow, dev, seed=1000 + ow.seed_index)
+            with ClockSampler(local_rank) as oc:
+                oms, oker, _ = op.time(max(20, args.steps), args.warmup, stream)
+            line = workload_line(ow, oms, oker, op.flushed)
+            line["clocks"] = oc.summary()
+            line["data"] = "synthetic (seeded torch.randn on the device, bf16)"
+            others[name] = line
+            del op
+            torch.cuda.empty_cache()
+    if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
 
@@ -303,34 +404,31 @@ def run_ours(args, w, rank, world, local_rank):
     peaks, peak_src = load_peaks()
     flops = w.step_flops()
     value = job_tflops(flops, world, ms_per_step)
-    kernel_flops = {"fwd": w.fwd_flops(), "bwd_preprocess": 0.0,
-                    "bwd_dkdv": 2.0 * w.fwd_flops(), "bwd_dq": 0.5 * w.fwd_flops(),
-                    "bwd": 2.5 * w.fwd_flops()}
-    kernels = {}
-    for n in names:
-        avg = per_kernel[n] / args.steps
-        kernels[n] = {"ms": round(avg, 5), "share": round(per_kernel[n] / step_ms, 4),
-                      "algorithmic_tflops": round(kernel_flops[n] / (avg * 1e-3) / 1e12, 2)
-                      if kernel_flops[n] else None}
+    summary = workload_line(w, ms_per_step, per_kernel, prob_flushed(w))
+    kernels = summary["kernels"]
+    names = list(per_kernel)
     dominant = max(names, key=lambda n: per_kernel[n])
-    dom_ms = per_kernel[dominant] / args.steps
-    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    if kernel_flops[dominant] > 0:
-        achieved = kernel_flops[dominant] / (dom_ms * 1e-3) / 1e12
+    dom_ms = per_kernel[dominant]
+    kf = kernel_flops(w)
+    peak, peak_kind, sustained = roofline_peak(peaks, bracket_ms)
+    traffic, traffic_src = measured_traffic(w.name, dominant)
+    if kf[dominant] > 0:
+        achieved = kf[dominant] / (dom_ms * 1e-3) / 1e12
         roofline = {"kernel": dominant, "bound": "tensor", "achieved": round(achieved, 2),
-                    "peak": sustained, "unit": "TFLOP/s", "frac": round(achieved / sustained, 4),
-                    "peak_kind": "bf16 sustained (%s)" % peak_src,
-                    "frac_of_burst": round(achieved / burst, 4),
+                    "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                    "peak_kind": "bf16 %s (%s): timed region %.0f ms" % (peak_kind, peak_src,
+                                                                          bracket_ms),
+                    "frac_of_sustained": round(achieved / sustained, 4),
                     "frac_of_datasheet": round(achieved / DATASHEET_BF16_TFLOPS, 4),
-                    "traffic": MEASURED_TRAFFIC.get((w.name, dominant))}
+                    "traffic": traffic, "traffic_source": traffic_src}
     else:
         nbytes = w.bwd_bytes() if dominant.startswith("bwd") else w.fwd_bytes()
-        achieved = 2 * w.tensor_bytes() / (dom_ms * 1e-3) / 1e9
+        achieved = nbytes / (dom_ms * 1e-3) / 1e9
         hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         roofline = {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1),
                     "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
-                    "traffic": None, "compulsory_bytes": nbytes}
+                    "traffic": traffic, "traffic_source": traffic_src}
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -345,13 +443,13 @@ def run_ours(args, w, rank, world, local_rank):
         "dtype": "bf16",
         "data": "synthetic (seeded i.i.d. N(0,1) bf16, SplitMix64 + Box-Muller)",
         "config": {
-            "workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
+            "workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
             "window": list(w.window), "alibi": w.alibi,
             "pass": "fwd+bwd" if w.backward else "fwd",
+            "path": "training path: forward keeps O - bf16(O) for the backward's delta",
             "step_gflop": round(flops / 1e9, 3),
             "parallelism": "replicas" if world > 1 else "single",
-            "l2": ("inputs larger than L2 (%d MB of inputs)" % (inputs_bytes >> 20))
-            if flush is None else "L2 flushed before every timed step",
+            "l2": summary["l2"],
         },
         "pct_of_dense_peak": round(100 * value / world / DATASHEET_BF16_TFLOPS, 2),
         "pct_of_measured_peak": round(100 * value / world / burst, 2),
@@ -359,13 +457,20 @@ def run_ours(args, w, rank, world, local_rank):
         "e2e": {"value": round(job_tflops(flops, world, e2e_ms), 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "steps": e2e_steps,
                 "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes},
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": (4 if w.backward else 1) * args.steps,
         "kernels": kernels,
         "roofline": roofline,
+        "kernel_source_hash": kernel_source_hash(),
     }
+    if others:
+        line["workloads"] = others
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     return line
+
+
+def prob_flushed(w) -> bool:
+    return 4 * w.tensor_bytes() <= L2_BYTES
 
 
 # ------------------------------------------------------------------------- CPU oracle
@@ -462,9 +567,14 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--also", default="c2,c3,c4,c5c,c5w",
+                    help="other workloads timed at full size in the same run (comma list)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="time the headline workload only")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    args.also = [x for x in args.also.split(",") if x]
 
     from exact_attention_126_b200.workloads import WORKLOADS
     w = WORKLOADS[args.workload]

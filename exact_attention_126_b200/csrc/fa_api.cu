@@ -68,7 +68,6 @@ fa_status_t check_problem(int B, int H, int N, int d, bool* empty) {
   }
   const long long elems = (long long)B * H * N * d;
   if (elems >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
-  if ((long long)B * H > 65535) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 
@@ -125,10 +124,16 @@ fa_status_t launched() {
 }
 
 
-// alibi: H slopes for the ALiBi kernels (kAlibi), unused otherwise.
+// Optional inputs and outputs of one call (fa_options_t, checked and resolved).
+struct Extras {
+  const float* alibi = nullptr;    // H slopes: the kAlibi kernels
+  const uint8_t* kpad = nullptr;   // (B, N) key-padding flags
+  void* o_low = nullptr;           // bf16 residual of O: written by the forward, read by delta
+};
+
 template <int D, bool kAlibi>
 fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int BH,
-                       int H, int N, float scale, int left, int right, const float* alibi,
+                       int H, int N, float scale, int left, int right, const Extras& x,
                        cudaStream_t st) {
   CUtensorMap mq, mkk, mv;
   if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) || !make_map(&mv, v, BH, N, D))
@@ -149,8 +154,10 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   a.left = left;
   a.right = right;
   a.fault = g_fault.load(std::memory_order_relaxed);
-  a.alibi = alibi;
+  a.alibi = x.alibi;
   a.H = H;
+  a.kpad = x.kpad;
+  a.o_low = static_cast<__nv_bfloat16*>(x.o_low);
   const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
   fa::fa_fwd_kernel<D, kAlibi><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, a);
   return launched();
@@ -159,65 +166,24 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
 int padded_rows(int N) { return fa::num_tiles(N) * kBlock; }
 
 template <int D>
-fa_status_t launch_preprocess(const void* o, const void* dout, const float* lse, float* stats,
-                              int BH, int N, cudaStream_t st) {
+fa_status_t launch_preprocess(const void* o, const void* o_low, const void* dout,
+                              const float* lse, float* stats, int BH, int N, cudaStream_t st) {
   const int Np = padded_rows(N);
-  const dim3 grid(Np / 64, BH);  // 64 rows per block; Np is a multiple of 128, BH <= 65535
-  fa::fa_bwd_preprocess_kernel<D><<<grid, 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, stats,
-      BH, N, Np);
+  // 64 rows per block, blocks of one head consecutive; BH * Np / 64 < 2^31 because every
+  // tensor has fewer than 2^31 elements (d >= 64)
+  const long long blocks = (long long)BH * (Np / 64);
+  fa::fa_bwd_preprocess_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(o_low),
+      static_cast<const __nv_bfloat16*>(dout), lse, stats, BH, N, Np);
   return launched();
 }
 
-template <int D, bool kAlibi>
-fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void* dout,
-                        const void* ws, void* dk, void* dv, int BH, int H, int N,
-                        float scale, int left, int right, const float* alibi, cudaStream_t st) {
-  CUtensorMap mq, mkk, mv, mdo, mdk, mdv;
-  if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
-      !make_map(&mv, v, BH, N, D) || !make_map(&mdo, dout, BH, N, D) ||
-      !make_map(&mdk, dk, BH, N, D) || !make_map(&mdv, dv, BH, N, D))
-    return FA_ERR_CUDA;
-  using C = fa::DkdvCfg<D>;
-  if (set_smem(fa::fa_bwd_dkdv_kernel<D, kAlibi>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
+// Arguments both backward passes share.
+fa::BwdArgs bwd_args(const void* ws, int BH, int H, int N, float scale, int left, int right,
+                     const Extras& x) {
   fa::BwdArgs a;
   a.stats = static_cast<const float*>(ws);
-  a.out0 = static_cast<__nv_bfloat16*>(dk);
-  a.out1 = static_cast<__nv_bfloat16*>(dv);
-  a.stat_rows = (long long)BH * padded_rows(N);
-  a.Np = padded_rows(N);
-  a.N = N;
-  a.n_tiles = fa::num_tiles(N);
-  a.scale = scale;
-  a.scale_log2 = scale * fa::kLog2e;
-  a.left = left;
-  a.right = right;
-  a.BH = BH;
-  a.n_items = BH * a.n_tiles;
-  a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
-  a.group = head_group(BH, a.n_tiles);
-  const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
-  a.alibi = alibi;
-  a.H = H;
-  fa::fa_bwd_dkdv_kernel<D, kAlibi><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo,
-                                                                               mdk, mdv, a);
-  return launched();
-}
-
-template <int D, bool kAlibi>
-fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* dout,
-                      const void* ws, void* dq, int BH, int H, int N, float scale,
-                      int left, int right, const float* alibi, cudaStream_t st) {
-  CUtensorMap mq, mkk, mv, mdo, mdq;
-  if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
-      !make_map(&mv, v, BH, N, D) || !make_map(&mdo, dout, BH, N, D) ||
-      !make_map(&mdq, dq, BH, N, D))
-    return FA_ERR_CUDA;
-  using C = fa::DqCfg<D>;
-  if (set_smem(fa::fa_bwd_dq_kernel<D, kAlibi>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
-  fa::BwdArgs a;
-  a.stats = static_cast<const float*>(ws);
-  a.out0 = static_cast<__nv_bfloat16*>(dq);
+  a.out0 = nullptr;
   a.out1 = nullptr;
   a.stat_rows = (long long)BH * padded_rows(N);
   a.Np = padded_rows(N);
@@ -231,9 +197,46 @@ fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* d
   a.n_items = BH * a.n_tiles;
   a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
   a.group = head_group(BH, a.n_tiles);
-  const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
-  a.alibi = alibi;
+  a.alibi = x.alibi;
   a.H = H;
+  a.kpad = x.kpad;
+  return a;
+}
+
+template <int D, bool kAlibi>
+fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void* dout,
+                        const void* ws, void* dk, void* dv, int BH, int H, int N, float scale,
+                        int left, int right, const Extras& x, cudaStream_t st) {
+  CUtensorMap mq, mkk, mv, mdo, mdk, mdv;
+  if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
+      !make_map(&mv, v, BH, N, D) || !make_map(&mdo, dout, BH, N, D) ||
+      !make_map(&mdk, dk, BH, N, D) || !make_map(&mdv, dv, BH, N, D))
+    return FA_ERR_CUDA;
+  using C = fa::DkdvCfg<D>;
+  if (set_smem(fa::fa_bwd_dkdv_kernel<D, kAlibi>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
+  fa::BwdArgs a = bwd_args(ws, BH, H, N, scale, left, right, x);
+  a.out0 = static_cast<__nv_bfloat16*>(dk);
+  a.out1 = static_cast<__nv_bfloat16*>(dv);
+  const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
+  fa::fa_bwd_dkdv_kernel<D, kAlibi><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo,
+                                                                               mdk, mdv, a);
+  return launched();
+}
+
+template <int D, bool kAlibi>
+fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* dout,
+                      const void* ws, void* dq, int BH, int H, int N, float scale, int left,
+                      int right, const Extras& x, cudaStream_t st) {
+  CUtensorMap mq, mkk, mv, mdo, mdq;
+  if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
+      !make_map(&mv, v, BH, N, D) || !make_map(&mdo, dout, BH, N, D) ||
+      !make_map(&mdq, dq, BH, N, D))
+    return FA_ERR_CUDA;
+  using C = fa::DqCfg<D>;
+  if (set_smem(fa::fa_bwd_dq_kernel<D, kAlibi>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
+  fa::BwdArgs a = bwd_args(ws, BH, H, N, scale, left, right, x);
+  a.out0 = static_cast<__nv_bfloat16*>(dq);
+  const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
   fa::fa_bwd_dq_kernel<D, kAlibi><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, mdq,
                                                                              a);
   return launched();
@@ -244,37 +247,19 @@ size_t workspace_bytes(int B, int H, int N) {
   return (raw + 255) & ~size_t(255);
 }
 
-// ------------------------------------------------------------------------------------
-// Backward without caller workspace (fa_bwd_noalloc): a fixed array in device memory
-// holds the row statistics instead. Every GPU that loads the library keeps this array
-// until the process exits.
-// ------------------------------------------------------------------------------------
-constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
-static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
-
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {nullptr};
-
-// Device address of g_noalloc_scratch on the current device. The symbol names a
-// host-side stand-in, not device memory, so the address is looked up once per device
-// (with that device current) and cached.
-fa_status_t noalloc_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-      return FA_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
+// Checks the optional arguments of an _ex call and resolves them; a null `opt` means none.
+fa_status_t resolve_options(const fa_options_t* opt, Extras* x) {
+  *x = Extras();
+  if (opt == nullptr) return FA_OK;
+  if (opt->alibi_slopes != nullptr && (reinterpret_cast<uintptr_t>(opt->alibi_slopes) & 3u) != 0)
+    return FA_ERR_MISALIGNED;
+  if (opt->o_low != nullptr && !aligned16(opt->o_low)) return FA_ERR_MISALIGNED;
+  if (!(opt->dropout_p == 0.f)) return FA_ERR_UNSUPPORTED;
+  x->alibi = opt->alibi_slopes;
+  x->kpad = opt->key_padding;
+  x->o_low = opt->o_low;
   return FA_OK;
 }
-
-}  // namespace
 
 fa_status_t check_slopes(const float* alibi) {
   if (alibi == nullptr) return FA_ERR_INVALID_ARG;
@@ -282,9 +267,9 @@ fa_status_t check_slopes(const float* alibi) {
   return FA_OK;
 }
 
-// fa_fwd and fa_fwd_alibi (alibi != nullptr)
+// The forward for every entry point: checks, then the kernel for (d, ALiBi or not).
 fa_status_t forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                    int N, int d, float scale, int causal, fa_window_t window, const float* alibi,
+                    int N, int d, float scale, int causal, fa_window_t window, const Extras& x,
                     void* stream) {
   bool empty;
   fa_status_t s = check_problem(B, H, N, d, &empty);
@@ -294,49 +279,188 @@ fa_status_t forward(const void* q, const void* k, const void* v, void* o, float*
   const int right = fa::resolve_right(causal, window.right);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int l = window.left, BH = B * H;
-  if (alibi != nullptr)
-    return d == 64 ? launch_fwd<64, true>(q, k, v, o, lse, BH, H, N, scale, l, right, alibi, st)
-                   : launch_fwd<128, true>(q, k, v, o, lse, BH, H, N, scale, l, right, alibi, st);
-  return d == 64 ? launch_fwd<64, false>(q, k, v, o, lse, BH, H, N, scale, l, right, nullptr, st)
-                 : launch_fwd<128, false>(q, k, v, o, lse, BH, H, N, scale, l, right, nullptr, st);
+  if (x.alibi != nullptr)
+    return d == 64 ? launch_fwd<64, true>(q, k, v, o, lse, BH, H, N, scale, l, right, x, st)
+                   : launch_fwd<128, true>(q, k, v, o, lse, BH, H, N, scale, l, right, x, st);
+  return d == 64 ? launch_fwd<64, false>(q, k, v, o, lse, BH, H, N, scale, l, right, x, st)
+                 : launch_fwd<128, false>(q, k, v, o, lse, BH, H, N, scale, l, right, x, st);
 }
 
-// The two passes of the backward after the preprocess step, with or without ALiBi.
-fa_status_t backward_passes(const void* q, const void* k, const void* v, const void* dout,
-                            const void* ws, void* dq, void* dk, void* dv, int B, int H, int N,
-                            int d, float scale, int causal, fa_window_t window,
-                            const float* alibi, void* stream) {
+// Step 1 of the backward: the row statistics in `workspace`.
+fa_status_t preprocess(const void* o, const void* dout, const float* lse, void* workspace, int B,
+                       int H, int N, int d, const Extras& x, void* stream) {
+  bool empty;
+  fa_status_t s = check_problem(B, H, N, d, &empty);
+  if (s != FA_OK || empty) return s;
+  if ((s = check_ptrs({o, dout, lse, workspace})) != FA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* stats = static_cast<float*>(workspace);
+  return d == 64 ? launch_preprocess<64>(o, x.o_low, dout, lse, stats, B * H, N, st)
+                 : launch_preprocess<128>(o, x.o_low, dout, lse, stats, B * H, N, st);
+}
+
+// Step 2: dK, dV.
+fa_status_t dkdv_pass(const void* q, const void* k, const void* v, const void* dout,
+                      const void* workspace, void* dk, void* dv, int B, int H, int N, int d,
+                      float scale, int causal, fa_window_t window, const Extras& x,
+                      void* stream) {
+  bool empty;
+  fa_status_t s = check_problem(B, H, N, d, &empty);
+  if (s != FA_OK || empty) return s;
+  if ((s = check_mask(scale, window)) != FA_OK) return s;
+  if ((s = check_ptrs({q, k, v, dout, workspace, dk, dv})) != FA_OK) return s;
   const int right = fa::resolve_right(causal, window.right);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int l = window.left, BH = B * H;
-  fa_status_t s;
-  if (alibi != nullptr) {
-    s = d == 64 ? launch_dkdv<64, true>(q, k, v, dout, ws, dk, dv, BH, H, N, scale, l, right,
-                                        alibi, st)
-                : launch_dkdv<128, true>(q, k, v, dout, ws, dk, dv, BH, H, N, scale, l, right,
-                                         alibi, st);
-    if (s != FA_OK) return s;
-    return d == 64 ? launch_dq<64, true>(q, k, v, dout, ws, dq, BH, H, N, scale, l, right,
-                                         alibi, st)
-                   : launch_dq<128, true>(q, k, v, dout, ws, dq, BH, H, N, scale, l, right,
-                                          alibi, st);
-  }
-  s = d == 64 ? launch_dkdv<64, false>(q, k, v, dout, ws, dk, dv, BH, H, N, scale, l, right,
-                                       nullptr, st)
-              : launch_dkdv<128, false>(q, k, v, dout, ws, dk, dv, BH, H, N, scale, l, right,
-                                        nullptr, st);
-  if (s != FA_OK) return s;
-  return d == 64 ? launch_dq<64, false>(q, k, v, dout, ws, dq, BH, H, N, scale, l, right,
-                                        nullptr, st)
-                 : launch_dq<128, false>(q, k, v, dout, ws, dq, BH, H, N, scale, l, right,
-                                         nullptr, st);
+  if (x.alibi != nullptr)
+    return d == 64 ? launch_dkdv<64, true>(q, k, v, dout, workspace, dk, dv, BH, H, N, scale, l,
+                                           right, x, st)
+                   : launch_dkdv<128, true>(q, k, v, dout, workspace, dk, dv, BH, H, N, scale, l,
+                                            right, x, st);
+  return d == 64 ? launch_dkdv<64, false>(q, k, v, dout, workspace, dk, dv, BH, H, N, scale, l,
+                                          right, x, st)
+                 : launch_dkdv<128, false>(q, k, v, dout, workspace, dk, dv, BH, H, N, scale, l,
+                                           right, x, st);
 }
+
+// Step 3: dQ.
+fa_status_t dq_pass(const void* q, const void* k, const void* v, const void* dout,
+                    const void* workspace, void* dq, int B, int H, int N, int d, float scale,
+                    int causal, fa_window_t window, const Extras& x, void* stream) {
+  bool empty;
+  fa_status_t s = check_problem(B, H, N, d, &empty);
+  if (s != FA_OK || empty) return s;
+  if ((s = check_mask(scale, window)) != FA_OK) return s;
+  if ((s = check_ptrs({q, k, v, dout, workspace, dq})) != FA_OK) return s;
+  const int right = fa::resolve_right(causal, window.right);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int l = window.left, BH = B * H;
+  if (x.alibi != nullptr)
+    return d == 64 ? launch_dq<64, true>(q, k, v, dout, workspace, dq, BH, H, N, scale, l, right,
+                                         x, st)
+                   : launch_dq<128, true>(q, k, v, dout, workspace, dq, BH, H, N, scale, l,
+                                          right, x, st);
+  return d == 64 ? launch_dq<64, false>(q, k, v, dout, workspace, dq, BH, H, N, scale, l, right,
+                                        x, st)
+                 : launch_dq<128, false>(q, k, v, dout, workspace, dq, BH, H, N, scale, l, right,
+                                         x, st);
+}
+
+// The three steps of the backward, with the statistics in `stats` (caller workspace or the
+// fixed array of fa_bwd_noalloc).
+fa_status_t backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                     const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                     float scale, int causal, fa_window_t window, const Extras& x, void* stats,
+                     void* stream) {
+  fa_status_t s;
+  if ((s = preprocess(o, dout, lse, stats, B, H, N, d, x, stream)) != FA_OK) return s;
+  if ((s = dkdv_pass(q, k, v, dout, stats, dk, dv, B, H, N, d, scale, causal, window, x,
+                     stream)) != FA_OK)
+    return s;
+  return dq_pass(q, k, v, dout, stats, dq, B, H, N, d, scale, causal, window, x, stream);
+}
+
+// Checks shared by every full backward before anything is launched.
+fa_status_t check_backward(const void* q, const void* k, const void* v, const void* o,
+                           const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                           int B, int H, int N, int d, float scale, fa_window_t window,
+                           bool* empty) {
+  fa_status_t s = check_problem(B, H, N, d, empty);
+  if (s != FA_OK || *empty) return s;
+  if ((s = check_mask(scale, window)) != FA_OK) return s;
+  return check_ptrs({q, k, v, o, dout, lse, dq, dk, dv});
+}
+
+// ------------------------------------------------------------------------------------
+// Backward without caller workspace (fa_bwd_noalloc): a fixed array in device memory
+// holds the row statistics instead. Every GPU that loads the library keeps this array
+// until the process exits.
+// ------------------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// The driver's identifier of the calling thread's current context: unique for the life of
+// the process, so that a context created after a cudaDeviceReset never matches an earlier
+// one. Returns false if the driver cannot tell.
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+constexpr int kMaxContexts = 64;
+std::mutex g_noalloc_mu;
+unsigned long long g_noalloc_ctx[kMaxContexts] = {0};
+void* g_noalloc_ptr[kMaxContexts] = {nullptr};
+int g_noalloc_used = 0;
+
+// Device address of g_noalloc_scratch in the calling thread's current context. In host
+// code the symbol names a host-side stand-in, not device memory, so the address is looked
+// up with cudaGetSymbolAddress, once per context (a module is loaded per context, so the
+// address belongs to the context: a cache by device number alone would go stale after a
+// cudaDeviceReset or in a second context on the same device), and cached by context id.
+// If no context is current yet (the runtime creates it lazily), the lookup below creates
+// it and the address is cached from the next call on.
+fa_status_t noalloc_scratch(void** out) {
+  unsigned long long id = 0;
+  const bool have_id = current_context_id(&id);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (have_id) {
+    for (int i = 0; i < g_noalloc_used; ++i) {
+      if (g_noalloc_ctx[i] == id) {
+        *out = g_noalloc_ptr[i];
+        return FA_OK;
+      }
+    }
+  }
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+    return FA_ERR_CUDA;
+  if (have_id && g_noalloc_used < kMaxContexts) {
+    g_noalloc_ctx[g_noalloc_used] = id;
+    g_noalloc_ptr[g_noalloc_used] = p;
+    ++g_noalloc_used;
+  }
+  *out = p;
+  return FA_OK;
+}
+
+}  // namespace
 
 extern "C" {
 
 fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                    int N, int d, float scale, int causal, fa_window_t window, void* stream) {
-  return forward(q, k, v, o, lse, B, H, N, d, scale, causal, window, nullptr, stream);
+  return forward(q, k, v, o, lse, B, H, N, d, scale, causal, window, Extras(), stream);
+}
+
+fa_status_t fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                      int H, int N, int d, float scale, int causal, fa_window_t window,
+                      const fa_options_t* options, void* stream) {
+  bool empty;
+  fa_status_t s = check_problem(B, H, N, d, &empty);
+  if (s != FA_OK || empty) return s;
+  Extras x;
+  if ((s = resolve_options(options, &x)) != FA_OK) return s;
+  return forward(q, k, v, o, lse, B, H, N, d, scale, causal, window, x, stream);
 }
 
 fa_status_t fa_fwd_alibi(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -346,7 +470,9 @@ fa_status_t fa_fwd_alibi(const void* q, const void* k, const void* v, void* o, f
   fa_status_t s = check_problem(B, H, N, d, &empty);
   if (s != FA_OK || empty) return s;
   if ((s = check_slopes(alibi_slopes)) != FA_OK) return s;
-  return forward(q, k, v, o, lse, B, H, N, d, scale, causal, window, alibi_slopes, stream);
+  Extras x;
+  x.alibi = alibi_slopes;
+  return forward(q, k, v, o, lse, B, H, N, d, scale, causal, window, x, stream);
 }
 
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
@@ -356,64 +482,58 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
 }
 
 fa_status_t fa_bwd_preprocess(const void* o, const void* dout, const float* lse,
-                              void* workspace, int B, int H, int N, int d, void* stream) {
-  bool empty;
-  fa_status_t s = check_problem(B, H, N, d, &empty);
-  if (s != FA_OK || empty) return s;
-  if ((s = check_ptrs({o, dout, lse, workspace})) != FA_OK) return s;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* stats = static_cast<float*>(workspace);
-  return d == 64 ? launch_preprocess<64>(o, dout, lse, stats, B * H, N, st)
-                 : launch_preprocess<128>(o, dout, lse, stats, B * H, N, st);
+                              void* workspace, int B, int H, int N, int d,
+                              const fa_options_t* options, void* stream) {
+  Extras x;
+  fa_status_t s = resolve_options(options, &x);
+  if (s != FA_OK) return s;
+  return preprocess(o, dout, lse, workspace, B, H, N, d, x, stream);
 }
 
 fa_status_t fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout,
                         const void* workspace, void* dk, void* dv, int B, int H, int N, int d,
-                        float scale, int causal, fa_window_t window, void* stream) {
-  bool empty;
-  fa_status_t s = check_problem(B, H, N, d, &empty);
-  if (s != FA_OK || empty) return s;
-  if ((s = check_mask(scale, window)) != FA_OK) return s;
-  if ((s = check_ptrs({q, k, v, dout, workspace, dk, dv})) != FA_OK) return s;
-  const int right = fa::resolve_right(causal, window.right);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_dkdv<64, false>(q, k, v, dout, workspace, dk, dv, B * H, H, N, scale,
-                                          window.left, right, nullptr, st)
-                 : launch_dkdv<128, false>(q, k, v, dout, workspace, dk, dv, B * H, H, N, scale,
-                                           window.left, right, nullptr, st);
+                        float scale, int causal, fa_window_t window,
+                        const fa_options_t* options, void* stream) {
+  Extras x;
+  fa_status_t s = resolve_options(options, &x);
+  if (s != FA_OK) return s;
+  return dkdv_pass(q, k, v, dout, workspace, dk, dv, B, H, N, d, scale, causal, window, x,
+                   stream);
 }
 
 fa_status_t fa_bwd_dq(const void* q, const void* k, const void* v, const void* dout,
                       const void* workspace, void* dq, int B, int H, int N, int d, float scale,
-                      int causal, fa_window_t window, void* stream) {
-  bool empty;
-  fa_status_t s = check_problem(B, H, N, d, &empty);
-  if (s != FA_OK || empty) return s;
-  if ((s = check_mask(scale, window)) != FA_OK) return s;
-  if ((s = check_ptrs({q, k, v, dout, workspace, dq})) != FA_OK) return s;
-  const int right = fa::resolve_right(causal, window.right);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_dq<64, false>(q, k, v, dout, workspace, dq, B * H, H, N, scale,
-                                        window.left, right, nullptr, st)
-                 : launch_dq<128, false>(q, k, v, dout, workspace, dq, B * H, H, N, scale,
-                                         window.left, right, nullptr, st);
+                      int causal, fa_window_t window, const fa_options_t* options,
+                      void* stream) {
+  Extras x;
+  fa_status_t s = resolve_options(options, &x);
+  if (s != FA_OK) return s;
+  return dq_pass(q, k, v, dout, workspace, dq, B, H, N, d, scale, causal, window, x, stream);
 }
 
 fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                    float scale, int causal, fa_window_t window, void* workspace,
                    size_t workspace_bytes_given, void* stream) {
+  return fa_bwd_ex(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, window, nullptr,
+                   workspace, workspace_bytes_given, stream);
+}
+
+fa_status_t fa_bwd_ex(const void* q, const void* k, const void* v, const void* o,
+                      const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                      int H, int N, int d, float scale, int causal, fa_window_t window,
+                      const fa_options_t* options, void* workspace,
+                      size_t workspace_bytes_given, void* stream) {
   bool empty;
-  fa_status_t s = check_problem(B, H, N, d, &empty);
+  fa_status_t s =
+      check_backward(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, window, &empty);
   if (s != FA_OK || empty) return s;
-  if ((s = check_mask(scale, window)) != FA_OK) return s;
-  if ((s = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv, workspace})) != FA_OK) return s;
+  Extras x;
+  if ((s = resolve_options(options, &x)) != FA_OK) return s;
+  if ((s = check_ptrs({workspace})) != FA_OK) return s;
   if (workspace_bytes_given < workspace_bytes(B, H, N)) return FA_ERR_WORKSPACE;
-  if ((s = fa_bwd_preprocess(o, dout, lse, workspace, B, H, N, d, stream)) != FA_OK) return s;
-  if ((s = fa_bwd_dkdv(q, k, v, dout, workspace, dk, dv, B, H, N, d, scale, causal, window,
-                       stream)) != FA_OK)
-    return s;
-  return fa_bwd_dq(q, k, v, dout, workspace, dq, B, H, N, d, scale, causal, window, stream);
+  return backward(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, window, x,
+                  workspace, stream);
 }
 
 fa_status_t fa_bwd_alibi(const void* q, const void* k, const void* v, const void* o,
@@ -422,15 +542,16 @@ fa_status_t fa_bwd_alibi(const void* q, const void* k, const void* v, const void
                          const float* alibi_slopes, void* workspace,
                          size_t workspace_bytes_given, void* stream) {
   bool empty;
-  fa_status_t s = check_problem(B, H, N, d, &empty);
+  fa_status_t s =
+      check_backward(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, window, &empty);
   if (s != FA_OK || empty) return s;
-  if ((s = check_mask(scale, window)) != FA_OK) return s;
   if ((s = check_slopes(alibi_slopes)) != FA_OK) return s;
-  if ((s = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv, workspace})) != FA_OK) return s;
+  if ((s = check_ptrs({workspace})) != FA_OK) return s;
   if (workspace_bytes_given < workspace_bytes(B, H, N)) return FA_ERR_WORKSPACE;
-  if ((s = fa_bwd_preprocess(o, dout, lse, workspace, B, H, N, d, stream)) != FA_OK) return s;
-  return backward_passes(q, k, v, dout, workspace, dq, dk, dv, B, H, N, d, scale, causal, window,
-                         alibi_slopes, stream);
+  Extras x;
+  x.alibi = alibi_slopes;
+  return backward(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, window, x,
+                  workspace, stream);
 }
 
 fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
@@ -438,28 +559,24 @@ fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const vo
                            int B, int H, int N, int d, float scale, int causal,
                            fa_window_t window, void* stream) {
   bool empty;
-  fa_status_t s = check_problem(B, H, N, d, &empty);
+  fa_status_t s =
+      check_backward(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, window, &empty);
   if (s != FA_OK || empty) return s;
-  if ((s = check_mask(scale, window)) != FA_OK) return s;
-  if ((s = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv})) != FA_OK) return s;
   if (workspace_bytes(B, H, N) > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
   void* scratch = nullptr;
   if ((s = noalloc_scratch(&scratch)) != FA_OK) return s;
   // The statistics are rewritten in full by the preprocess step, so nothing needs clearing.
-  if ((s = fa_bwd_preprocess(o, dout, lse, scratch, B, H, N, d, stream)) != FA_OK) return s;
-  if ((s = fa_bwd_dkdv(q, k, v, dout, scratch, dk, dv, B, H, N, d, scale, causal, window,
-                       stream)) != FA_OK)
-    return s;
-  return fa_bwd_dq(q, k, v, dout, scratch, dq, B, H, N, d, scale, causal, window, stream);
+  return backward(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, window, Extras(),
+                  scratch, stream);
 }
 
 const char* fa_status_string(fa_status_t status) {
   switch (status) {
     case FA_OK: return "FA_OK";
     case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: null pointer, negative size, bad scale or window";
-    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: head_dim must be 64 or 128 and tensors < 2^31 elements";
-    case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED: pointers must be 16-byte aligned";
-    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: workspace smaller than fa_bwd_workspace_bytes()";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: head_dim must be 64 or 128, tensors < 2^31 elements, options as documented";
+    case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED: tensor pointers must be 16-byte aligned, slopes 4-byte aligned";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: the workspace (or fa_bwd_noalloc's fixed 8 MiB array) is too small for this problem";
     case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA call failed";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a kernel abandoned a bounded wait";
   }
@@ -484,6 +601,6 @@ fa_status_t fa_debug_set_fault(int fault) {
   return FA_OK;
 }
 
-int fa_version(void) { return 100; }
+int fa_version(void) { return 200; }
 
 }  // extern "C"

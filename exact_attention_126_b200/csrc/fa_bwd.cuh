@@ -43,34 +43,42 @@ namespace fa {
 // Row statistics of the backward, over B*H rows of Np (N rounded up to 128) entries:
 //   stats[bh*Np + r]             = LSE_r * log2(e)        (+inf for r >= N)
 //   stats[BH*Np + bh*Np + r]     = rowsum(dO_r * O_r)     (0 for r >= N), summed in fp32
-// Block (x, bh) covers rows 64x .. 64x+63 of head bh, 8 rows per warp; G = D/8 lanes share
-// a row, 16 bytes of O and dO per lane, and a warp's loads for its 8 rows are all issued
-// before any is used.
+// With o_low (the residual O - bf16(O) the forward can write), O_r is taken as
+// o_r + o_low_r, which carries about 16 significant bits instead of 8: for rows whose
+// softmax is nearly one-hot, dS = P (dP - delta) cancels almost completely and the
+// rounding of a bf16 O would dominate dQ and dK.
+// Block b covers rows 64x .. 64x+63 of head bh, with (bh, x) = divmod(b, Np/64), 8 rows
+// per warp; G = D/8 lanes share a row, 16 bytes of O and dO per lane, and a warp's loads
+// for its 8 rows are all issued before any is used.
 // ------------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256)
     fa_bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o,
+                             const __nv_bfloat16* __restrict__ o_low,
                              const __nv_bfloat16* __restrict__ dout, const float* __restrict__ lse,
                              float* __restrict__ stats, int BH, int N, int Np) {
   constexpr int G = D / 8;                      // lanes per row
   constexpr int kRowsPerPass = 32 / G;          // rows a warp covers per load
   constexpr int kPasses = 8 / kRowsPerPass;     // 8 rows per warp
-  const int bh = blockIdx.y;
+  const int blocks_per_head = Np / 64;
+  const int bh = blockIdx.x / blocks_per_head;
+  const int xb = blockIdx.x - bh * blocks_per_head;
   const int lane = threadIdx.x & 31;
   const int sub = lane / G;                     // row within the pass
   const int part = lane % G;                    // 16-byte slice of the row
-  const int row0 = blockIdx.x * 64 + (threadIdx.x >> 5) * 8;
-  uint4 a[kPasses], b[kPasses];
+  const int row0 = xb * 64 + (threadIdx.x >> 5) * 8;
+  uint4 a[kPasses], b[kPasses], c[kPasses];
 #pragma unroll
   for (int p = 0; p < kPasses; ++p) {
     const int r = row0 + p * kRowsPerPass + sub;
+    a[p] = make_uint4(0, 0, 0, 0);
+    b[p] = make_uint4(0, 0, 0, 0);
+    c[p] = make_uint4(0, 0, 0, 0);
     if (r < N) {
       const size_t src = ((size_t)bh * N + r) * D + part * 8;
       a[p] = *reinterpret_cast<const uint4*>(o + src);
       b[p] = *reinterpret_cast<const uint4*>(dout + src);
-    } else {
-      a[p] = make_uint4(0, 0, 0, 0);
-      b[p] = make_uint4(0, 0, 0, 0);
+      if (o_low != nullptr) c[p] = *reinterpret_cast<const uint4*>(o_low + src);
     }
   }
   const size_t rows = (size_t)BH * Np;
@@ -78,11 +86,16 @@ __global__ void __launch_bounds__(256)
   for (int p = 0; p < kPasses; ++p) {
     const uint32_t aw[4] = {a[p].x, a[p].y, a[p].z, a[p].w};
     const uint32_t bw[4] = {b[p].x, b[p].y, b[p].z, b[p].w};
+    const uint32_t cw[4] = {c[p].x, c[p].y, c[p].z, c[p].w};
     float acc = 0.f;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
-      acc = fmaf(__uint_as_float(aw[w] << 16), __uint_as_float(bw[w] << 16), acc);
-      acc = fmaf(__uint_as_float(aw[w] & 0xFFFF0000u), __uint_as_float(bw[w] & 0xFFFF0000u), acc);
+      const float d0 = __uint_as_float(bw[w] << 16), d1 = __uint_as_float(bw[w] & 0xFFFF0000u);
+      acc = fmaf(__uint_as_float(aw[w] << 16), d0, acc);
+      acc = fmaf(__uint_as_float(aw[w] & 0xFFFF0000u), d1, acc);
+      // the residual is zero without o_low
+      acc = fmaf(__uint_as_float(cw[w] << 16), d0, acc);
+      acc = fmaf(__uint_as_float(cw[w] & 0xFFFF0000u), d1, acc);
     }
 #pragma unroll
     for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -112,7 +125,8 @@ struct BwdArgs {
   int left;
   int right;
   const float* alibi;   // ALiBi kernels: one slope per head (heads = H)
-  int H;
+  int H;                // heads per batch entry (batch entry of bh = bh / H)
+  const uint8_t* kpad;  // (B, N) key-padding flags (nonzero = padded key), or null
 };
 
 // Shared layout of both backward kernels: the stationary tiles X0, X1 of an item (in XB
@@ -563,6 +577,9 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
       const int n_it = i_hi - i_lo + 1;
       const int c = j * kBlock + t_row;  // this thread's key
       const float slope2 = kAlibi ? a.alibi[bh % a.H] * kLog2e : 0.f;
+      // a padded key gets no attention from any query: its rows of P^T and dS^T are zero
+      const bool key_padded =
+          a.kpad != nullptr && c < a.N && a.kpad[(size_t)(bh / a.H) * a.N + c] != 0;
       for (int it = 0; it < n_it; ++it) {
         const int i = i_lo + it;
         const int t = g + it;
@@ -598,6 +615,10 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
           visible_queries(c, (long long)i * kBlock + NC * h, NC, mk, r_lo, r_hi);
 #pragma unroll
           for (int r = 0; r < NC; ++r) p[r] = (r >= r_lo && r <= r_hi) ? p[r] : 0.f;
+        }
+        if (a.kpad != nullptr) {
+#pragma unroll
+          for (int r = 0; r < NC; ++r) p[r] = key_padded ? 0.f : p[r];
         }
         {
           uint32_t pk[NC / 2];
@@ -931,6 +952,17 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
           visible_keys(r, (long long)jj * kBlock + NC * h, NC, mk, c_lo, c_hi);
 #pragma unroll
           for (int c = 0; c < NC; ++c) p[c] = (c >= c_lo && c <= c_hi) ? p[c] : 0.f;
+        }
+        if (a.kpad != nullptr) {
+          // lane l reads the flag of key NC*h + l of the tile; the ballot gives all 32
+          static_assert(NC == 32, "one ballot covers a warpgroup's columns");
+          const int col = jj * kBlock + NC * h + lane;
+          const uint32_t pm = __ballot_sync(
+              0xffffffffu, col < a.N && a.kpad[(size_t)(bh / a.H) * a.N + col] != 0);
+          if (pm != 0u) {
+#pragma unroll
+            for (int c = 0; c < NC; ++c) p[c] = ((pm >> c) & 1u) ? 0.f : p[c];
+          }
         }
         if (!mbar_wait_warp(bar(bDPFull), t & 1, abort_flag)) {
           ok = false;

@@ -51,7 +51,9 @@ struct FwdArgs {
   int right;
   int fault;          // test hook: 1 = the producer never loads V (waits for it run out)
   const float* alibi; // ALiBi kernels: one slope per head (heads = H)
-  int H;
+  int H;              // heads per batch entry (batch entry of bh = bh / H)
+  const uint8_t* kpad;       // (B, N) key-padding flags (nonzero = padded key), or null
+  __nv_bfloat16* o_low;      // (B, H, N, d) bf16 residual O - bf16(O), or null
 };
 
 template <int D>
@@ -478,6 +480,22 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
 #pragma unroll
           for (int c = 0; c < kBlock; ++c) x[c] = (c >= c_lo && c <= c_hi) ? x[c] : -INFINITY;
         }
+        if (a.kpad != nullptr) {
+          // padded keys of this tile: lane l reads the flag of key 32g + l, one ballot per
+          // 32 keys; the same 128 bits for every row
+          uint32_t pm[4];
+          const uint8_t* fl = a.kpad + (size_t)(it.bh / a.H) * a.N;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int col = j * kBlock + 32 * g + lane;
+            pm[g] = __ballot_sync(0xffffffffu, col < a.N && fl[col] != 0);
+          }
+          if ((pm[0] | pm[1] | pm[2] | pm[3]) != 0u) {
+#pragma unroll
+            for (int c = 0; c < kBlock; ++c)
+              x[c] = ((pm[c >> 5] >> (c & 31)) & 1u) ? -INFINITY : x[c];
+          }
+        }
         float mx;
         {
           // 16 partial maxima: x[0..47], then two columns at a time up to x[111], then x[112..127]
@@ -578,6 +596,24 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
           for (int v4 = 0; v4 < 4; ++v4)
             st_global_v4(orow + 32 * q + 8 * v4, w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2],
                          w[4 * v4 + 3]);
+        }
+        if (a.o_low != nullptr) {
+          // what rounding to bf16 left out: O - bf16(O), itself rounded to bf16, so that
+          // the backward can form rowsum(dO o O) from O to about 16 significant bits
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float r0 = __uint_as_float(o[2 * c]) * inv_l - __uint_as_float(w[c] << 16);
+            const float r1 =
+                __uint_as_float(o[2 * c + 1]) * inv_l - __uint_as_float(w[c] & 0xFFFF0000u);
+            w[c] = pack_bf16x2(r0, r1);
+          }
+          if (row < a.N) {
+            __nv_bfloat16* lrow = a.o_low + ((size_t)it.bh * a.N + row) * D;
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              st_global_v4(lrow + 32 * q + 8 * v4, w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2],
+                           w[4 * v4 + 3]);
+          }
         }
       }
       // O_s has been read: the next item's first P V may overwrite it

@@ -23,9 +23,10 @@ STATUS_NAMES = {
 }
 
 #: every symbol include/fa.h declares
-EXPORTED = ("fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_fwd_alibi", "fa_bwd_alibi",
-            "fa_bwd_preprocess", "fa_bwd_dkdv", "fa_bwd_dq", "fa_bwd_noalloc",
-            "fa_status_string", "fa_debug_status", "fa_debug_set_fault", "fa_version")
+EXPORTED = ("fa_fwd", "fa_fwd_ex", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_ex",
+            "fa_fwd_alibi", "fa_bwd_alibi", "fa_bwd_preprocess", "fa_bwd_dkdv", "fa_bwd_dq",
+            "fa_bwd_noalloc", "fa_status_string", "fa_debug_status", "fa_debug_set_fault",
+            "fa_version")
 
 
 class FAError(RuntimeError):
@@ -37,6 +38,18 @@ class FAError(RuntimeError):
 
 class fa_window_t(ctypes.Structure):
     _fields_ = [("left", ctypes.c_int), ("right", ctypes.c_int)]
+
+
+class fa_options_t(ctypes.Structure):
+    """Optional inputs and outputs of the _ex entry points (include/fa.h)."""
+    _fields_ = [("alibi_slopes", ctypes.c_void_p), ("key_padding", ctypes.c_void_p),
+                ("o_low", ctypes.c_void_p), ("dropout_p", ctypes.c_float),
+                ("dropout_seed", ctypes.c_ulonglong), ("dropout_offset", ctypes.c_ulonglong)]
+
+
+def options(alibi_slopes=None, key_padding=None, o_low=None):
+    """An fa_options_t holding the device pointers of the given tensors (None = absent)."""
+    return fa_options_t(_ptr(alibi_slopes), _ptr(key_padding), _ptr(o_low), 0.0, 0, 0)
 
 
 _LIB = None
@@ -52,7 +65,11 @@ def _lib() -> ctypes.CDLL:
         lib = ctypes.CDLL(LIBRARY)
         vp, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         W = fa_window_t
+        OP = ctypes.POINTER(fa_options_t)
         lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp]
+        lib.fa_fwd_ex.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, W, OP, vp]
+        lib.fa_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, OP,
+                                  vp, ctypes.c_size_t, vp]
         lib.fa_bwd_workspace_bytes.argtypes = [I, I, I, I]
         lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
         lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp,
@@ -60,9 +77,9 @@ def _lib() -> ctypes.CDLL:
         lib.fa_fwd_alibi.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp, vp]
         lib.fa_bwd_alibi.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp,
                                      vp, ctypes.c_size_t, vp]
-        lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, vp, I, I, I, I, vp]
-        lib.fa_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp]
-        lib.fa_bwd_dq.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp]
+        lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, vp, I, I, I, I, OP, vp]
+        lib.fa_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, OP, vp]
+        lib.fa_bwd_dq.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, OP, vp]
         lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W,
                                        vp]
         lib.fa_status_string.argtypes = [I]
@@ -70,7 +87,8 @@ def _lib() -> ctypes.CDLL:
         lib.fa_debug_status.argtypes = [vp]
         lib.fa_debug_set_fault.argtypes = [I]
         lib.fa_version.argtypes = []
-        for name in ("fa_fwd", "fa_bwd", "fa_fwd_alibi", "fa_bwd_alibi", "fa_bwd_preprocess",
+        for name in ("fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_ex", "fa_fwd_alibi",
+                     "fa_bwd_alibi", "fa_bwd_preprocess",
                      "fa_bwd_dkdv", "fa_bwd_dq", "fa_bwd_noalloc", "fa_debug_status",
                      "fa_debug_set_fault", "fa_version"):
             getattr(lib, name).restype = I
@@ -162,28 +180,55 @@ def fa_bwd_alibi(q, k, v, o, do, lse, dq, dk, dv, workspace, alibi_slopes, scale
            "fa_bwd_alibi")
 
 
-def fa_bwd_preprocess(o, do, lse, workspace, stream=None) -> None:
+def _opt_ref(opt):
+    return None if opt is None else ctypes.byref(opt)
+
+
+def fa_fwd_ex(q, k, v, o, lse, opt=None, scale=None, causal=False, window=(-1, -1),
+              stream=None) -> None:
+    """fa_fwd with an fa_options_t (see options())."""
+    B, H, N, d = _shape(q)
+    c, w = _window(causal, window)
+    s = default_scale(d) if scale is None else float(scale)
+    _check(_lib().fa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, s, c, w,
+                            _opt_ref(opt), _stream(stream)), "fa_fwd_ex")
+
+
+def fa_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, workspace, opt=None, scale=None, causal=False,
+              window=(-1, -1), stream=None) -> None:
+    """fa_bwd with an fa_options_t (see options())."""
+    B, H, N, d = _shape(q)
+    c, w = _window(causal, window)
+    s = default_scale(d) if scale is None else float(scale)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib().fa_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                            _ptr(dk), _ptr(dv), B, H, N, d, s, c, w, _opt_ref(opt),
+                            _ptr(workspace), nbytes, _stream(stream)), "fa_bwd_ex")
+
+
+def fa_bwd_preprocess(o, do, lse, workspace, opt=None, stream=None) -> None:
     B, H, N, d = _shape(o)
     _check(_lib().fa_bwd_preprocess(_ptr(o), _ptr(do), _ptr(lse), _ptr(workspace), B, H, N, d,
-                                    _stream(stream)), "fa_bwd_preprocess")
+                                    _opt_ref(opt), _stream(stream)), "fa_bwd_preprocess")
 
 
 def fa_bwd_dkdv(q, k, v, do, workspace, dk, dv, scale=None, causal=False, window=(-1, -1),
-                stream=None) -> None:
+                stream=None, opt=None) -> None:
     B, H, N, d = _shape(q)
     c, w = _window(causal, window)
     s = default_scale(d) if scale is None else float(scale)
     _check(_lib().fa_bwd_dkdv(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(workspace), _ptr(dk),
-                              _ptr(dv), B, H, N, d, s, c, w, _stream(stream)), "fa_bwd_dkdv")
+                              _ptr(dv), B, H, N, d, s, c, w, _opt_ref(opt), _stream(stream)),
+           "fa_bwd_dkdv")
 
 
 def fa_bwd_dq(q, k, v, do, workspace, dq, scale=None, causal=False, window=(-1, -1),
-              stream=None) -> None:
+              stream=None, opt=None) -> None:
     B, H, N, d = _shape(q)
     c, w = _window(causal, window)
     s = default_scale(d) if scale is None else float(scale)
     _check(_lib().fa_bwd_dq(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(workspace), _ptr(dq),
-                            B, H, N, d, s, c, w, _stream(stream)), "fa_bwd_dq")
+                            B, H, N, d, s, c, w, _opt_ref(opt), _stream(stream)), "fa_bwd_dq")
 
 
 def fa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, scale=None, causal=False, window=(-1, -1),
@@ -236,26 +281,42 @@ def _check_slopes(alibi_slopes, q):
         raise ValueError("alibi_slopes must hold one slope per head, contiguous")
 
 
+def _check_padding(key_padding, q):
+    if not key_padding.is_cuda or key_padding.dtype not in (torch.bool, torch.uint8):
+        raise ValueError("key_padding must be a bool or uint8 CUDA tensor")
+    if tuple(key_padding.shape) != (q.shape[0], q.shape[2]) or not key_padding.is_contiguous():
+        raise ValueError("key_padding must be a contiguous (batch, seq_len) tensor")
+
+
 def attention_forward(q, k, v, scale=None, causal=False, window=(-1, -1), stream=None,
-                      alibi_slopes=None):
-    """Returns (O, LSE) for bf16 CUDA tensors q, k, v of shape (B, H, N, d); with
-    alibi_slopes (H fp32 values), the scores carry the bias -alibi_slopes[h] * |i - j|."""
+                      alibi_slopes=None, key_padding=None, keep_residual=False):
+    """Returns (O, LSE) for bf16 CUDA tensors q, k, v of shape (B, H, N, d), or
+    (O, LSE, O_low) with keep_residual: O_low = O_fp32 - bf16(O) in bf16, which
+    attention_backward uses to form rowsum(dO o O) from O to about 16 bits.
+    alibi_slopes (H fp32 values): the scores carry the bias -alibi_slopes[h] * |i - j|.
+    key_padding ((B, N) bool or uint8, True = padded key): padded keys are masked out
+    for every head and query."""
     _check_inputs(q, k, v)
     B, H, N, d = _shape(q)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    if alibi_slopes is None:
+    o_low = torch.empty_like(q) if keep_residual else None
+    if alibi_slopes is not None:
+        _check_slopes(alibi_slopes, q)
+    if key_padding is not None:
+        _check_padding(key_padding, q)
+    if alibi_slopes is None and key_padding is None and o_low is None:
         fa_fwd(q, k, v, o, lse, scale, causal, window, stream)
     else:
-        _check_slopes(alibi_slopes, q)
-        fa_fwd_alibi(q, k, v, o, lse, alibi_slopes, scale, causal, window, stream)
-    return o, lse
+        opt = options(alibi_slopes, key_padding, o_low)
+        fa_fwd_ex(q, k, v, o, lse, opt, scale, causal, window, stream)
+    return (o, lse, o_low) if keep_residual else (o, lse)
 
 
 def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, window=(-1, -1),
-                       stream=None, alibi_slopes=None):
-    """Returns (dQ, dK, dV): the gradient of <O, dO>; lse comes from attention_forward
-    (with the same alibi_slopes)."""
+                       stream=None, alibi_slopes=None, key_padding=None, o_low=None):
+    """Returns (dQ, dK, dV): the gradient of <O, dO>; lse (and o_low, if kept) come from
+    attention_forward with the same alibi_slopes and key_padding."""
     _check_inputs(q, k, v, o, do)
     B, H, N, d = _shape(q)
     dq = torch.empty_like(q)
@@ -263,10 +324,15 @@ def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, window=(-1
     dv = torch.empty_like(q)
     ws = torch.empty(max(1, fa_bwd_workspace_bytes(B, H, N, d)), dtype=torch.uint8,
                      device=q.device)
-    if alibi_slopes is None:
+    if alibi_slopes is not None:
+        _check_slopes(alibi_slopes, q)
+    if key_padding is not None:
+        _check_padding(key_padding, q)
+    if o_low is not None:
+        _check_inputs(q, o_low)
+    if alibi_slopes is None and key_padding is None and o_low is None:
         fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, scale, causal, window, stream)
     else:
-        _check_slopes(alibi_slopes, q)
-        fa_bwd_alibi(q, k, v, o, do, lse, dq, dk, dv, ws, alibi_slopes, scale, causal, window,
-                     stream)
+        opt = options(alibi_slopes, key_padding, o_low)
+        fa_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, ws, opt, scale, causal, window, stream)
     return dq, dk, dv

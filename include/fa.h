@@ -23,8 +23,8 @@
  * Sizes.  d must be 64 or 128 (else FA_ERR_UNSUPPORTED: the pages list 64 and 128
  *   as the common head sizes and report "no available kernel" otherwise, page
  *   "Flash Attention 3.7 …" §5). B, H, N >= 0; if any is 0 the call does nothing and
- *   returns FA_OK. Each tensor must have fewer than 2^31 elements and B * H may be
- *   at most 65535 (else FA_ERR_UNSUPPORTED).
+ *   returns FA_OK. Each tensor must have fewer than 2^31 elements (else
+ *   FA_ERR_UNSUPPORTED).
  * Scale.  scale multiplies Q K^T before the mask. It is used exactly as given and
  *   must be finite and > 0 (else FA_ERR_INVALID_ARG); pass 1/sqrt(d) for the usual
  *   default (`softmax_scale=None`, page "告别OOM和训练慢…" §4.2).
@@ -34,7 +34,8 @@
  *   with -1 meaning unbounded (`window_size=(-1,-1)`, page "告别OOM和训练慢…" §4.2).
  *   causal != 0 masks future positions, i.e. forces window.right = 0 when it is -1
  *   or positive. Values below -1 give FA_ERR_INVALID_ARG. Every query sees at least
- *   itself, so no row is fully masked.
+ *   itself, so no row is fully masked unless key padding (fa_options_t) removes all of
+ *   its keys.
  * Memory.  Every pointer is caller-owned device memory that is only used during the
  *   call's kernels; the library keeps nothing and allocates nothing. Pointers must be
  *   non-null (FA_ERR_INVALID_ARG) and 16-byte aligned (FA_ERR_MISALIGNED: the
@@ -62,7 +63,7 @@ typedef enum {
     FA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad scale or window  */
     FA_ERR_UNSUPPORTED = 2,  /* head_dim not 64/128, or a tensor of >= 2^31 elements */
     FA_ERR_MISALIGNED = 3,   /* a pointer that is not 16-byte aligned               */
-    FA_ERR_WORKSPACE = 4,    /* workspace smaller than fa_bwd_workspace_bytes()     */
+    FA_ERR_WORKSPACE = 4,    /* workspace (or the no-alloc array) too small         */
     FA_ERR_CUDA = 5,         /* a CUDA runtime or driver call failed                */
     FA_ERR_TIMEOUT = 6       /* a kernel abandoned a bounded wait (fa_debug_status) */
 } fa_status_t;
@@ -72,6 +73,41 @@ typedef struct {
     int left;
     int right;
 } fa_window_t;
+
+/*
+ * Optional inputs and outputs of the _ex entry points (and of the backward's phase entry
+ * points). A null fa_options_t pointer, or a zero-initialised struct, means none of them.
+ *
+ *   alibi_slopes  H fp32 slopes, device memory, 4-byte aligned, or NULL: the ALiBi bias
+ *                 (see fa_fwd_alibi).
+ *   key_padding   (B, N) bytes, device memory, any alignment, or NULL: nonzero marks key
+ *                 n of batch entry b as padding. Page "PyTorch-CUDA-v2.9镜像中使用
+ *                 FlashAttention提升训练速度" passes such a `key_padding_mask` (True = padded)
+ *                 and applies it with masked_fill(-inf) to every head and query: a padded
+ *                 key's score is -inf before the softmax. A query left with no visible,
+ *                 unpadded key gets O = 0, LSE = -inf and no gradient (the backward must
+ *                 get the same flags as the forward).
+ *   o_low         bf16 (B, H, N, d), device memory, 16-byte aligned, or NULL. The forward
+ *                 writes there what rounding O to bf16 left out, O_fp32 - bf16(O), itself
+ *                 rounded to bf16; the backward then forms delta = rowsum(dO o O) from
+ *                 o + o_low, about 16 significant bits instead of 8. This matters for rows
+ *                 whose softmax is nearly one-hot: there dS = P o (dP - delta) cancels
+ *                 almost completely and the bf16 rounding of O alone would move dQ and dK
+ *                 by several percent. Costs one more bf16 tensor written by the forward and
+ *                 read by the backward.
+ *   dropout_p, dropout_seed, dropout_offset
+ *                 reserved: dropout_p must be 0 (else FA_ERR_UNSUPPORTED); the seed and
+ *                 offset are ignored.
+ * The layout is that of a C struct with natural alignment (48 bytes on LP64).
+ */
+typedef struct {
+    const float *alibi_slopes;
+    const unsigned char *key_padding;
+    void *o_low;
+    float dropout_p;
+    unsigned long long dropout_seed;
+    unsigned long long dropout_offset;
+} fa_options_t;
 
 /*
  * Forward pass.
@@ -86,6 +122,14 @@ typedef struct {
 fa_status_t fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
                    int B, int H, int N, int d, float scale, int causal,
                    fa_window_t window, void *stream);
+
+/*
+ * fa_fwd with the optional inputs and outputs of `options` (may be NULL). Misaligned
+ * slopes or o_low give FA_ERR_MISALIGNED; a nonzero dropout_p gives FA_ERR_UNSUPPORTED.
+ */
+fa_status_t fa_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse,
+                      int B, int H, int N, int d, float scale, int causal,
+                      fa_window_t window, const fa_options_t *options, void *stream);
 
 /*
  * Bytes of device workspace fa_bwd() needs: two fp32 arrays of B*H*Np values, where
@@ -118,6 +162,16 @@ fa_status_t fa_bwd(const void *q, const void *k, const void *v, const void *o,
                    void *stream);
 
 /*
+ * fa_bwd with the optional inputs of `options` (may be NULL): the same alibi_slopes and
+ * key_padding as the forward had, and o_low if the forward wrote it.
+ */
+fa_status_t fa_bwd_ex(const void *q, const void *k, const void *v, const void *o,
+                      const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                      int B, int H, int N, int d, float scale, int causal,
+                      fa_window_t window, const fa_options_t *options, void *workspace,
+                      size_t workspace_bytes, void *stream);
+
+/*
  * ALiBi: fa_fwd and fa_bwd with a linear bias. Page "告别OOM和训练慢…(含A100环境配置)" §4.2
  * lists `alibi_slopes` among the parameters of flash_attn_fn and calls it a linear bias;
  * the reading taken is that of ALiBi: head h has a slope m_h, and -m_h * |i - j| is added
@@ -143,22 +197,27 @@ fa_status_t fa_bwd_alibi(const void *q, const void *k, const void *v, const void
  * 128 fp32 values (padding rows: +inf and 0):
  *   workspace[0 .. B*H*Np)          LSE * log2(e)      (from `lse`)
  *   workspace[B*H*Np .. 2*B*H*Np)   delta = rowsum(dout * o), summed in fp32
+ *                                   (o + options->o_low when o_low is given)
  * The padding lets each 128-row tile of both arrays be fetched with one bulk copy.
+ * `options` may be NULL; only its o_low is used here.
  */
 fa_status_t fa_bwd_preprocess(const void *o, const void *dout, const float *lse,
-                              void *workspace, int B, int H, int N, int d, void *stream);
+                              void *workspace, int B, int H, int N, int d,
+                              const fa_options_t *options, void *stream);
 
-/* Step 2 of fa_bwd alone: dk, dv from q, k, v, dout and the workspace of step 1. */
+/* Step 2 of fa_bwd alone: dk, dv from q, k, v, dout and the workspace of step 1
+ * (`options`: alibi_slopes and key_padding, or NULL). */
 fa_status_t fa_bwd_dkdv(const void *q, const void *k, const void *v, const void *dout,
                         const void *workspace, void *dk, void *dv,
                         int B, int H, int N, int d, float scale, int causal,
-                        fa_window_t window, void *stream);
+                        fa_window_t window, const fa_options_t *options, void *stream);
 
-/* Step 3 of fa_bwd alone: dq from q, k, v, dout and the workspace of step 1. */
+/* Step 3 of fa_bwd alone: dq from q, k, v, dout and the workspace of step 1
+ * (`options`: alibi_slopes and key_padding, or NULL). */
 fa_status_t fa_bwd_dq(const void *q, const void *k, const void *v, const void *dout,
                       const void *workspace, void *dq,
                       int B, int H, int N, int d, float scale, int causal,
-                      fa_window_t window, void *stream);
+                      fa_window_t window, const fa_options_t *options, void *stream);
 
 /*
  * Backward pass for callers that cannot allocate device memory. (The pages have no
@@ -174,8 +233,12 @@ fa_status_t fa_bwd_dq(const void *q, const void *k, const void *v, const void *d
  *   Limit: 2 * B * H * Np * 4 bytes must fit in 8 MiB, i.e. B * H * Np <= 1,048,576
  *   with Np = N rounded up to a multiple of 128; larger problems return
  *   FA_ERR_WORKSPACE before anything is launched.
- *   Set-up: the first call on a device (with that device current) looks up the
- *   array's device address once; make that first call before any stream capture.
+ *   Set-up: in host code the array's name is only a host-side stand-in, so the first
+ *   call in each CUDA context (with that context current) looks up the array's device
+ *   address with cudaGetSymbolAddress. The address belongs to that context, so it is
+ *   cached by the driver's context id: a second context on the same device, or the new
+ *   primary context after a cudaDeviceReset, gets its own lookup. Make the first call in a
+ *   context before any stream capture.
  *   Sharing: every call on a device uses the same array. The statistics are fully
  *   rewritten by each call, so nothing carries over, but calls whose kernels overlap
  *   on the GPU (different streams, or several threads) race on the array: serialise

@@ -31,19 +31,25 @@ def rel_frob(x: np.ndarray, ref: np.ndarray) -> float:
 
 
 def run_library(inp: dict, scale: float, causal: bool, window, backward: bool = True,
-                alibi=None) -> dict:
-    """Runs fa_fwd (and fa_bwd) on cuda:0, or their ALiBi forms when `alibi` (H slopes) is
-    given; returns host tensors."""
+                alibi=None, key_padding=None, residual: bool = True) -> dict:
+    """Runs the forward (and backward) on cuda:0 through the C ABI and returns host tensors.
+    `alibi`: H slopes; `key_padding`: a (B, N) bool host tensor (True = padded key);
+    `residual`: the forward keeps O - bf16(O) for the backward's delta (the training path
+    the benchmark times); False runs plain fa_fwd / fa_bwd."""
     ensure_built()
     dev = torch.device("cuda:0")
     q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
     slopes = None if alibi is None else torch.tensor(alibi, dtype=torch.float32, device=dev)
-    o, lse = fa.attention_forward(q, k, v, scale, causal, window, alibi_slopes=slopes)
+    kpad = None if key_padding is None else key_padding.to(dev)
+    res = fa.attention_forward(q, k, v, scale, causal, window, alibi_slopes=slopes,
+                               key_padding=kpad, keep_residual=residual and backward)
+    o, lse = res[0], res[1]
+    o_low = res[2] if len(res) > 2 else None
     out = {"o": o, "lse": lse}
     if backward:
         do = inp["do"].to(dev)
         dq, dk, dv = fa.attention_backward(q, k, v, o, lse, do, scale, causal, window,
-                                           alibi_slopes=slopes)
+                                           alibi_slopes=slopes, key_padding=kpad, o_low=o_low)
         out.update(dq=dq, dk=dk, dv=dv)
     torch.cuda.synchronize()
     assert fa.fa_debug_status() == 0
@@ -51,10 +57,12 @@ def run_library(inp: dict, scale: float, causal: bool, window, backward: bool = 
 
 
 def compare(inp: dict, out: dict, scale: float, causal: bool, window, heads=None,
-            backward: bool = True, alibi=None) -> dict:
+            backward: bool = True, alibi=None, key_padding=None) -> dict:
     """Errors of the library's outputs against the oracle, on all heads or on the listed
     (b, h) pairs (each head is an independent problem, so a subset is exact); `alibi`: the
-    H slopes the library ran with, if any."""
+    H slopes the library ran with, if any; `key_padding`: its (B, N) flags, if any.
+    Rows the oracle leaves with no visible key (LSE = -inf) must have LSE = -inf exactly;
+    the LSE error is taken over the other rows."""
     def pick(t):
         a = synth.to_f64(t) if t.dtype == torch.bfloat16 else t.double().numpy()
         if heads is None:
@@ -65,14 +73,24 @@ def compare(inp: dict, out: dict, scale: float, causal: bool, window, heads=None
     slopes = None
     if alibi is not None:
         slopes = list(alibi) if heads is None else [alibi[h] for _, h in heads]
-    o_ref, lse_ref = oracle.fwd(q, k, v, scale, causal, window, slopes)
+    kp = None
+    if key_padding is not None:
+        kp = key_padding.numpy().astype(np.uint8)
+        if heads is not None:
+            # one batch entry per sampled head, in the layout pick() gives: (1, n, N, d)
+            # tensors need (1, N) flags per head, so compare head by head instead
+            raise ValueError("sampled heads with key padding are not supported")
+    o_ref, lse_ref = oracle.fwd(q, k, v, scale, causal, window, slopes, kp)
+    lse = pick(out["lse"])
+    dead = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(lse), dead), "rows with no visible key differ"
     errs = {
         "o": rel_frob(pick(out["o"]), o_ref),
-        "lse": float(np.abs(pick(out["lse"]) - lse_ref).max()),
+        "lse": float(np.abs(lse[~dead] - lse_ref[~dead]).max()) if (~dead).any() else 0.0,
     }
     if backward:
         do = pick(inp["do"])
-        dq_ref, dk_ref, dv_ref = oracle.bwd(q, k, v, do, scale, causal, window, slopes)
+        dq_ref, dk_ref, dv_ref = oracle.bwd(q, k, v, do, scale, causal, window, slopes, kp)
         errs["dq"] = rel_frob(pick(out["dq"]), dq_ref)
         errs["dk"] = rel_frob(pick(out["dk"]), dk_ref)
         errs["dv"] = rel_frob(pick(out["dv"]), dv_ref)

@@ -65,7 +65,8 @@ def test_fwd_rejects_bad_arguments(lib):
     assert fwd(lib, window=(-2, -1)) == 1
     assert fwd(lib, window=(5, -3)) == 1
     assert fwd(lib, B=1 << 12, H=1 << 12, N=256, d=64) == 2  # >= 2^31 elements
-    assert fwd(lib, B=65536, H=1, N=1, d=64) == 2  # more (batch, head) pairs than a grid holds
+    # more than 65535 (batch, head) pairs is accepted (no grid dimension is limited by it)
+    assert lib.fa_bwd_workspace_bytes(1 << 17, 1, 128, 64) == 2 * (1 << 17) * 128 * 4
 
 
 def test_empty_problem_is_a_no_op(lib):
@@ -101,11 +102,42 @@ def test_bwd_rejects_bad_arguments(lib):
     assert bwd(lib, ws_bytes=2 * 128 * 4 - 1) == 4
     assert bwd(lib, d=256) == 2
     assert bwd(lib, window=(-7, 0)) == 1
-    assert lib.fa_bwd_preprocess(A, None, A, A, 1, 1, 128, 64, None) == 1
-    assert lib.fa_bwd_preprocess(A, A, A, A + 8, 1, 1, 128, 64, None) == 3
+    assert lib.fa_bwd_preprocess(A, None, A, A, 1, 1, 128, 64, None, None) == 1
+    assert lib.fa_bwd_preprocess(A, A, A, A + 8, 1, 1, 128, 64, None, None) == 3
     assert lib.fa_bwd_dkdv(A, A, A, A, A, A, A + 1, 1, 1, 128, 64, 0.1, 0, W(-1, -1),
-                           None) == 3
-    assert lib.fa_bwd_dq(A, A, A, A, A, A, 1, 1, 128, 128, -1.0, 0, W(-1, -1), None) == 1
+                           None, None) == 3
+    assert lib.fa_bwd_dq(A, A, A, A, A, A, 1, 1, 128, 128, -1.0, 0, W(-1, -1), None,
+                         None) == 1
+
+
+def test_options_are_checked(lib):
+    def fwd_ex(opt, q=A, d=64):
+        return lib.fa_fwd_ex(q, A, A, A, A, 1, 2, 128, d, 0.125, 0, W(-1, -1), opt, None)
+
+    def bwd_ex(opt, ws_bytes=1 << 20):
+        return lib.fa_bwd_ex(A, A, A, A, A, A, A, A, A, 1, 2, 128, 64, 0.125, 0, W(-1, -1), opt,
+                             A, ws_bytes, None)
+
+    O = fa.fa_options_t
+    assert fwd_ex(O(A + 2, None, None, 0.0, 0, 0)) == 3   # slopes not 4-byte aligned
+    assert fwd_ex(O(None, None, A + 8, 0.0, 0, 0)) == 3   # o_low not 16-byte aligned
+    assert fwd_ex(O(None, None, None, 0.1, 0, 0)) == 2    # dropout is not offered
+    assert fwd_ex(O(None, A + 1, None, 0.0, 0, 0), q=None) == 1
+    assert fwd_ex(None, d=96) == 2
+    assert bwd_ex(O(None, None, A + 4, 0.0, 0, 0)) == 3
+    assert bwd_ex(O(None, None, None, 0.5, 0, 0)) == 2
+    assert bwd_ex(None, ws_bytes=8) == 4
+    # empty problems launch nothing, whatever the options
+    assert lib.fa_fwd_ex(None, None, None, None, None, 1, 2, 0, 64, 0.125, 0, W(-1, -1),
+                         O(A + 2, None, None, 0.5, 0, 0), None) == 0
+
+
+def test_options_struct_layout():
+    import ctypes
+    O = fa.fa_options_t
+    assert ctypes.sizeof(O) == 48
+    assert [O.alibi_slopes.offset, O.key_padding.offset, O.o_low.offset, O.dropout_p.offset,
+            O.dropout_seed.offset, O.dropout_offset.offset] == [0, 8, 16, 24, 32, 40]
 
 
 def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -71,3 +71,24 @@ def test_reference_arm_other_ranks_do_nothing():
            "--workload", "c1", "--steps", "1", "--warmup", "3"]
     res = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
     assert res.returncode == 0 and res.stdout.strip() == ""
+
+
+def test_roofline_peak_follows_the_timed_region():
+    """Regions under a second are held to the burst peak, longer ones to the sustained."""
+    sys.path.insert(0, ROOT)
+    import bench
+    peaks = {"bf16_tflops": 1679.8, "bf16_tflops_sustained": 1394.0}
+    assert bench.roofline_peak(peaks, 47.0)[:2] == (1679.8, "burst")
+    assert bench.roofline_peak(peaks, 2500.0)[:2] == (1394.0, "sustained")
+    assert bench.roofline_peak({}, 10.0)[0] == bench.FALLBACK_PEAKS["bf16_tflops"]
+
+
+def test_traffic_is_null_once_the_kernels_change(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    h = bench.kernel_source_hash()
+    monkeypatch.setattr(bench, "MEASURED_TRAFFIC", {
+        ("w", "k"): (123, h, "ncu capture"), ("w", "old"): (456, "0" * 12, "old capture")})
+    assert bench.measured_traffic("w", "k") == (123, "ncu capture")
+    assert bench.measured_traffic("w", "old") == (None, None)
+    assert bench.measured_traffic("w", "none") == (None, None)

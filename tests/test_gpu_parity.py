@@ -146,38 +146,47 @@ def test_self_similar_inputs(d):
     """k = v = q (the comparison input of page "显存神技：必学FlashAttention！").
 
     Each row's own key dominates its softmax here (P_ii ~ 0.77 at d = 64, 0.98 at d = 128),
-    so dS = P o (dP - delta) cancels almost to zero on the diagonal, and the rounding of the
-    stored bf16 O, from which delta = rowsum(dO o O) is formed, dominates dQ and dK.
-    Round-to-nearest-even perturbs each O_ic by a relative error of RMS 2^-9/sqrt(3), so
-        sigma_i = 2^-9/sqrt(3) * sqrt(sum_c (dO_ic O_ic)^2)
-    is the RMS shift of delta_i. It moves dQ_i by scale * shift_i * (P K)_i = scale * shift_i
-    * O_i (K = V here), and dK by scale * P^T (shift * q), whose norm is at most
-    scale * sqrt(max column sum of P) * |shift * |q||. dQ and dK are held to 1e-2 relative
-    plus four times that RMS model (computed from the oracle's fp64 O; the column sums of P
-    are the oracle's dV for dO = 1). O, LSE and dV are held to the plain bounds."""
+    so dS = P o (dP - delta) cancels almost to zero on the diagonal and delta must be
+    formed from O to better than bf16: the training path keeps O - bf16(O) from the
+    forward for that. Every output is held to the plain bounds."""
     base = inputs(1, 2, 384, d, 400 + d)
     inp = {"q": base["q"], "k": base["q"].clone(), "v": base["q"].clone(), "do": base["do"]}
     scale = 1.0 / np.sqrt(d)
-    q = synth.to_f64(inp["q"])
-    do = synth.to_f64(inp["do"])
     for causal in (False, True):
         out = G.run_library(inp, scale, causal, (-1, -1))
-        o_ref, lse_ref = G.oracle.fwd(q, q, q, scale, causal)
-        dq_ref, dk_ref, dv_ref = G.oracle.bwd(q, q, q, do, scale, causal)
-        col_sum = G.oracle.bwd(q, q, q, np.ones_like(q), scale, causal)[2][..., 0]
-        assert G.rel_frob(synth.to_f64(out["o"]), o_ref) <= G.TOL_O
-        assert np.abs(out["lse"].double().numpy() - lse_ref).max() <= G.TOL_LSE
-        assert G.rel_frob(synth.to_f64(out["dv"]), dv_ref) <= G.TOL_GRAD
-        sigma = 2.0 ** -9 / np.sqrt(3.0) * np.sqrt(np.sum((do * o_ref) ** 2, axis=-1))
-        dq_model = scale * np.sqrt(np.sum((sigma * np.linalg.norm(o_ref, axis=-1)) ** 2))
-        dk_model = scale * np.sqrt(col_sum.max()) * np.sqrt(
-            np.sum((sigma * np.linalg.norm(q, axis=-1)) ** 2))
-        dq_err = np.linalg.norm((synth.to_f64(out["dq"]) - dq_ref).ravel())
-        dk_err = np.linalg.norm((synth.to_f64(out["dk"]) - dk_ref).ravel())
-        print(d, causal, "dq err %.3g model %.3g, dk err %.3g model %.3g" % (
-            dq_err, dq_model, dk_err, dk_model))
-        assert dq_err <= G.TOL_GRAD * np.linalg.norm(dq_ref.ravel()) + 4 * dq_model, (d, causal)
-        assert dk_err <= G.TOL_GRAD * np.linalg.norm(dk_ref.ravel()) + 4 * dk_model, (d, causal)
+        errs = G.compare(inp, out, scale, causal, (-1, -1))
+        print(d, causal, errs)
+        G.assert_within_bounds(errs, (d, causal))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_self_similar_inputs_without_residual(d):
+    """The same input through plain fa_fwd / fa_bwd, whose delta is formed from the bf16 O:
+    O, LSE and dV keep the plain bounds, while dQ and dK carry the rounding of O amplified
+    by the cancellation in dS (measured here, not bounded by the target's 1e-2: fp64
+    emulation puts it near 1.2% at d = 64 and 11% at d = 128). The test pins that the
+    residual is what removes it: with it, the same run is within 1e-2 (test above)."""
+    base = inputs(1, 2, 384, d, 400 + d)
+    inp = {"q": base["q"], "k": base["q"].clone(), "v": base["q"].clone(), "do": base["do"]}
+    scale = 1.0 / np.sqrt(d)
+    out = G.run_library(inp, scale, False, (-1, -1), residual=False)
+    errs = G.compare(inp, out, scale, False, (-1, -1))
+    print(d, errs)
+    assert errs["o"] <= G.TOL_O and errs["lse"] <= G.TOL_LSE and errs["dv"] <= G.TOL_GRAD
+    assert errs["dq"] > G.TOL_GRAD / 4 and errs["dk"] > G.TOL_GRAD / 4, errs
+
+
+@pytest.mark.parametrize("name", ["c1", "c3", "c4", "c5w"])
+def test_plain_path_without_residual(name):
+    """fa_fwd / fa_bwd as the target names them (delta from the bf16 O) on i.i.d. inputs:
+    within the plain bounds on the full-size workloads."""
+    w = WORKLOADS[name]
+    inp = inputs(w.B, w.H, w.N, w.d, w.seed_index)
+    out = G.run_library(inp, w.softmax_scale, w.causal, w.window, w.backward, residual=False)
+    heads = None if w.B * w.H * w.N <= 2 * 8 * 4096 else _sampled_heads(w)
+    errs = G.compare(inp, out, w.softmax_scale, w.causal, w.window, heads, w.backward)
+    print(name, errs)
+    G.assert_within_bounds(errs, name)
 
 
 def test_zero_queries_closed_form():
