@@ -48,14 +48,20 @@ class Oracle:
             path = build()
         self.lib = ctypes.CDLL(path)
         L = ctypes.c_long
+        D, U64 = ctypes.c_double, ctypes.c_ulonglong
         self.lib.oracle_attention_fwd.argtypes = [
-            _dptr, _dptr, _dptr, L, L, L, L, ctypes.c_double, ctypes.c_int, L, L, _dptr, _bptr,
+            _dptr, _dptr, _dptr, L, L, L, L, D, ctypes.c_int, L, L, _dptr, _bptr, D, U64, U64,
             _dptr, _dptr]
         self.lib.oracle_attention_fwd.restype = ctypes.c_int
         self.lib.oracle_attention_bwd.argtypes = [
-            _dptr, _dptr, _dptr, _dptr, L, L, L, L, ctypes.c_double, ctypes.c_int, L, L, _dptr,
-            _bptr, _dptr, _dptr, _dptr]
+            _dptr, _dptr, _dptr, _dptr, L, L, L, L, D, ctypes.c_int, L, L, _dptr, _bptr, D, U64,
+            U64, _dptr, _dptr, _dptr]
         self.lib.oracle_attention_bwd.restype = ctypes.c_int
+        u32p = ctypes.POINTER(ctypes.c_uint32)
+        self.lib.oracle_philox4x32_10.argtypes = [u32p, u32p, u32p]
+        self.lib.oracle_philox4x32_10.restype = None
+        self.lib.oracle_dropout_mask.argtypes = [U64, U64, L, L, D, _bptr]
+        self.lib.oracle_dropout_mask.restype = ctypes.c_int
         self.lib.oracle_num_threads.restype = ctypes.c_int
 
     @staticmethod
@@ -87,25 +93,52 @@ class Oracle:
             raise ValueError("key_padding must be a (B, N) array of flags")
         return a, a.ctypes.data_as(_bptr)
 
-    def fwd(self, q, k, v, scale, causal=False, window=(-1, -1), alibi=None, key_padding=None):
+    @staticmethod
+    def _dropout(dropout):
+        if dropout is None:
+            return 0.0, 0, 0
+        p, seed, offset = dropout
+        return float(p), int(seed), int(offset)
+
+    def philox4x32_10(self, counter, key):
+        """The four output words of Philox4x32-10 for a 4-word counter and 2-word key."""
+        c = (ctypes.c_uint32 * 4)(*counter)
+        k = (ctypes.c_uint32 * 2)(*key)
+        out = (ctypes.c_uint32 * 4)()
+        self.lib.oracle_philox4x32_10(c, k, out)
+        return [int(x) for x in out]
+
+    def dropout_mask(self, seed, offset, bh, N, p):
+        """The (N, N) keep flags (query, key) of head bh (= b * H + h)."""
+        m = np.empty((N, N), dtype=np.uint8)
+        rc = self.lib.oracle_dropout_mask(int(seed), int(offset), int(bh), int(N), float(p),
+                                          m.ctypes.data_as(_bptr))
+        if rc != 0:
+            raise ValueError("dropout probability out of range")
+        return m
+
+    def fwd(self, q, k, v, scale, causal=False, window=(-1, -1), alibi=None, key_padding=None,
+            dropout=None):
         """Returns (O, LSE) in fp64 for (B, H, N, d) inputs; `alibi`: H slopes or None;
-        `key_padding`: (B, N) flags, True for a padded key, or None."""
+        `key_padding`: (B, N) flags, True for a padded key, or None; `dropout`:
+        (p, seed, offset) or None."""
         q, k, v = self._prep(q, k, v)
         B, H, N, d = q.shape
         o = np.empty_like(q)
         lse = np.empty((B, H, N), dtype=np.float64)
         keep, slopes = self._slopes(alibi, H)
         keep_pad, pad = self._padding(key_padding, B, N)
+        dp, seed, offset = self._dropout(dropout)
         rc = self.lib.oracle_attention_fwd(_as_ptr(q), _as_ptr(k), _as_ptr(v), B, H, N, d,
                                            float(scale), int(bool(causal)), int(window[0]),
-                                           int(window[1]), slopes, pad, _as_ptr(o),
-                                           _as_ptr(lse))
+                                           int(window[1]), slopes, pad, dp, seed, offset,
+                                           _as_ptr(o), _as_ptr(lse))
         if rc != 0:
             raise RuntimeError("oracle_attention_fwd failed with %d" % rc)
         return o, lse
 
     def bwd(self, q, k, v, do, scale, causal=False, window=(-1, -1), alibi=None,
-            key_padding=None):
+            key_padding=None, dropout=None):
         """Returns (dQ, dK, dV) in fp64: the gradient of <O, dO> for (B, H, N, d) inputs."""
         q, k, v, do = self._prep(q, k, v, do)
         B, H, N, d = q.shape
@@ -114,10 +147,11 @@ class Oracle:
         dv = np.empty_like(q)
         keep, slopes = self._slopes(alibi, H)
         keep_pad, pad = self._padding(key_padding, B, N)
+        dp, seed, offset = self._dropout(dropout)
         rc = self.lib.oracle_attention_bwd(_as_ptr(q), _as_ptr(k), _as_ptr(v), _as_ptr(do),
                                            B, H, N, d, float(scale), int(bool(causal)),
-                                           int(window[0]), int(window[1]), slopes, pad,
-                                           _as_ptr(dq), _as_ptr(dk), _as_ptr(dv))
+                                           int(window[0]), int(window[1]), slopes, pad, dp,
+                                           seed, offset, _as_ptr(dq), _as_ptr(dk), _as_ptr(dv))
         if rc != 0:
             raise RuntimeError("oracle_attention_bwd failed with %d" % rc)
         return dq, dk, dv

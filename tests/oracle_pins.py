@@ -24,6 +24,14 @@ get zero gradients; a single unpadded key is returned exactly; a fully padded ba
 gives O = 0, LSE = -inf and zero gradients; finite differences; torch's SDPA with the combined
 boolean mask.
 
+The dropout pins (`dropout_p` of page "告别OOM和训练慢…" §4.2; F.dropout on the softmax
+weights before the product with V in the reference layer of page "Flash Attention 3.7 核心原理
+与实战" §4.2) pin the generator by the known-answer vectors of Philox4x32-10 (Salmon, Moraes,
+Dror and Shaw, SC 2011, as published with the authors' Random123 library), the keep flags by
+their documented counter/byte layout computed from those pinned outputs, p = 0 as no dropout
+at all, the dropped fraction by a binomial bound, and the arithmetic by torch autograd in
+fp64 with the same flags as an explicit multiplicative mask and by finite differences.
+
 The ALiBi pins (linear bias -m_h |i - j| on the scaled scores, the `alibi_slopes` parameter
 of page "告别OOM和训练慢…(含A100环境配置)" §4.2) use the same kinds of facts: closed forms
 where the scores are the bias alone, the limit of a bias so steep that each row sees only
@@ -507,6 +515,134 @@ def pin_self_similarity(orc):
         assert np.all(lse >= 0.5 * np.sum(q * q, axis=-1) - 1e-12)
 
 
+# Philox4x32-10 known-answer vectors: (counter, key) -> output, the three published with
+# the generator (all-zero, all-one and pi-digit inputs).
+PHILOX_KAT = [
+    ((0x00000000, 0x00000000, 0x00000000, 0x00000000), (0x00000000, 0x00000000),
+     (0x6627e8d5, 0xe169c58d, 0xbc57ac4c, 0x9b00dbd8)),
+    ((0xffffffff, 0xffffffff, 0xffffffff, 0xffffffff), (0xffffffff, 0xffffffff),
+     (0x408f276d, 0x41c83b0e, 0xa20bc7c6, 0x6d5451fd)),
+    ((0x243f6a88, 0x85a308d3, 0x13198a2e, 0x03707344), (0xa4093822, 0x299f31d0),
+     (0xd16cfe09, 0x94fdcceb, 0x5001e420, 0x24126ea1)),
+]
+
+
+def pin_philox_known_answers(orc):
+    """The generator reproduces the published known-answer vectors of Philox4x32-10."""
+    for ctr, key, want in PHILOX_KAT:
+        assert tuple(orc.philox4x32_10(ctr, key)) == want, (ctr, key)
+
+
+def pin_dropout_mask_layout(orc):
+    """The keep flag of (query i, key j) of head bh is byte j mod 4 of output word
+    (j mod 16) / 4 of Philox4x32-10 at counter (j / 16, i, bh, offset) and key (seed low,
+    seed high), compared with t = floor(256 p + 1/2): kept iff byte >= t."""
+    seed, offset, N = 0x0123456789ABCDEF, 77, 40
+    for p, bh in [(0.1, 0), (0.5, 5), (0.97, 3)]:
+        t = math.floor(256 * p + 0.5)
+        m = orc.dropout_mask(seed, offset, bh, N, p)
+        for i in range(N):
+            for j in range(N):
+                words = orc.philox4x32_10((j // 16, i, bh, offset),
+                                          (seed & 0xFFFFFFFF, seed >> 32))
+                byte = (words[(j % 16) // 4] >> (8 * (j % 4))) & 0xFF
+                assert m[i, j] == (1 if byte >= t else 0), (p, bh, i, j)
+
+
+def pin_dropout_zero_is_identity(orc):
+    """p = 0 (and any p < 1/512, which rounds to no threshold) is no dropout at all:
+    bit-identical outputs and gradients."""
+    r = _rng(21)
+    q, k, v, do = (r.standard_normal((1, 2, 21, 5)) for _ in range(4))
+    for causal, window in MODES[:3]:
+        o, lse = orc.fwd(q, k, v, 0.4, causal, window)
+        g = orc.bwd(q, k, v, do, 0.4, causal, window)
+        for p in (0.0, 0.0019):
+            o2, lse2 = orc.fwd(q, k, v, 0.4, causal, window, dropout=(p, 5, 6))
+            g2 = orc.bwd(q, k, v, do, 0.4, causal, window, dropout=(p, 5, 6))
+            assert np.array_equal(o, o2) and np.array_equal(lse, lse2)
+            for a, b in zip(g, g2):
+                assert np.array_equal(a, b)
+
+
+def pin_dropout_keep_fraction(orc):
+    """Over 256 x 256 flags the dropped fraction is t / 256 within five binomial standard
+    deviations; flags differ between heads, offsets and seeds."""
+    n = 256 * 256
+    for p in (0.1, 0.3, 0.5):
+        t = math.floor(256 * p + 0.5)
+        m = orc.dropout_mask(99, 0, 1, 256, p)
+        dropped = n - int(m.sum())
+        sigma = math.sqrt(n * (t / 256) * (1 - t / 256))
+        assert abs(dropped - n * t / 256) <= 5 * sigma, (p, dropped)
+    a = orc.dropout_mask(99, 0, 1, 64, 0.5)
+    for other in (orc.dropout_mask(99, 0, 2, 64, 0.5), orc.dropout_mask(99, 1, 1, 64, 0.5),
+                  orc.dropout_mask(98, 0, 1, 64, 0.5)):
+        assert not np.array_equal(a, other)
+
+
+def _dropout_factor(orc, B, H, N, p, seed, offset):
+    """Z / (1 - p') per head as a (B, H, N, N) array, from the oracle's keep flags."""
+    t = math.floor(256 * p + 0.5)
+    z = np.stack([orc.dropout_mask(seed, offset, bh, N, p) for bh in range(B * H)])
+    return (z.astype(np.float64) * (256.0 / (256.0 - t))).reshape(B, H, N, N)
+
+
+def pin_dropout_library(orc):
+    """torch in fp64: O = (softmax(masked scores) o Z / (1 - p')) V with the oracle's keep
+    flags as an explicit factor, LSE unchanged by dropout, and autograd through that
+    expression for dQ, dK, dV."""
+    r = _rng(22)
+    B, H, N, d = 2, 2, 37, 6
+    q, k, v, do = (r.standard_normal((B, H, N, d)) for _ in range(4))
+    scale, p, seed, offset = 0.37, 0.2, 1234, 9
+    zf = torch.tensor(_dropout_factor(orc, B, H, N, p, seed, offset))
+    for causal, window in MODES:
+        mask = _band_mask(N, causal, window)
+        tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+        s = (tq @ tk.transpose(-1, -2)) * scale
+        s = s.masked_fill(~mask, float("-inf"))
+        to = (torch.softmax(s, dim=-1) * zf) @ tv
+        to.backward(torch.tensor(do))
+        tlse = torch.logsumexp(s.detach(), dim=-1)
+        o, lse = orc.fwd(q, k, v, scale, causal, window, dropout=(p, seed, offset))
+        dq, dk, dv = orc.bwd(q, k, v, do, scale, causal, window, dropout=(p, seed, offset))
+        np.testing.assert_allclose(o, to.detach().numpy(), rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(lse, tlse.numpy(), rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=1e-11, atol=1e-11)
+        np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=1e-11, atol=1e-11)
+        np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=1e-11, atol=1e-11)
+
+
+def pin_dropout_finite_differences(orc):
+    """With dropout (fixed seed, so fixed flags), the backward is the gradient of
+    L = <O, dO>: central finite differences, every mask mode."""
+    h = 1e-6
+    for (N, d, seed) in [(5, 3, 31), (18, 2, 32)]:
+        r = _rng(seed)
+        q, k, v, do = (r.standard_normal((1, 1, N, d)) for _ in range(4))
+        scale, drop = 0.6, (0.4, 555, 3)
+        for causal, window in MODES:
+            grads = orc.bwd(q, k, v, do, scale, causal, window, dropout=drop)
+
+            def L(qq, kk, vv):
+                o, _ = orc.fwd(qq, kk, vv, scale, causal, window, dropout=drop)
+                return float(np.sum(o * do))
+
+            for which, g in enumerate(grads):
+                fd = np.zeros_like(q)
+                for idx in np.ndindex(q.shape):
+                    args = [q.copy(), k.copy(), v.copy()]
+                    args[which][idx] += h
+                    lp = L(*args)
+                    args[which][idx] -= 2 * h
+                    lm = L(*args)
+                    fd[idx] = (lp - lm) / (2 * h)
+                err = np.abs(fd - g).max()
+                ref = max(1.0, np.abs(g).max())
+                assert err <= 1e-6 * ref, (N, d, causal, window, which, err)
+
+
 ALL_PINS = [
     pin_single_key,
     pin_zero_queries,
@@ -531,4 +667,10 @@ ALL_PINS = [
     pin_padding_whole_entry,
     pin_padding_finite_differences,
     pin_padding_library_sdpa,
+    pin_philox_known_answers,
+    pin_dropout_mask_layout,
+    pin_dropout_zero_is_identity,
+    pin_dropout_keep_fraction,
+    pin_dropout_library,
+    pin_dropout_finite_differences,
 ]

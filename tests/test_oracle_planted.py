@@ -19,7 +19,7 @@ PLANTS = [
      "for (j = 0; j < N; ++j) Pi[j] /= 1.0;"),
     ("O row index swapped", "oh[i * d + c] += p * vh[j * d + c];",
      "oh[i * d + c] += p * vh[i * d + c];"),
-    ("dV uses P instead of P^T", "double p = P[ii * N + j];", "double p = P[j * N + ii];"),
+    ("dV uses P instead of P^T", "double p = Pd[ii * N + j];", "double p = Pd[j * N + ii];"),
     ("dS sign of D flipped", "(dP[i * N + jj] - D[i])", "(dP[i * N + jj] + D[i])"),
     ("dQ scale dropped", "dqh[i * d + c] *= scale;", "dqh[i * d + c] *= 1.0;"),
     ("dK uses dS instead of dS^T", "double s = dP[ii * N + j];", "double s = dP[j * N + ii];"),
@@ -40,6 +40,15 @@ PLANTS = [
     ("key padding of the first batch entry for all",
      "return key_padding ? key_padding + (bh / H) * N : NULL;",
      "return key_padding ? key_padding : NULL;"),
+    ("Philox multiplier typo", "M0 = 0xD2511F53u", "M0 = 0xD2511F55u"),
+    ("Philox key not bumped", "k1 += W1;", "k1 += 0;"),
+    ("dropout counter takes the key as row", "ctr[1] = (uint32_t)i;", "ctr[1] = (uint32_t)j;"),
+    ("dropout threshold off by one", "return (int)byte >= t ? 1 : 0;",
+     "return (int)byte > t ? 1 : 0;"),
+    ("dropout kept weights not rescaled",
+     "P[i * N + j] = dropout_keep(seed, offset, bh, i, j, t) ? P[i * N + j] * keep_scale : 0.0;",
+     "P[i * N + j] = dropout_keep(seed, offset, bh, i, j, t) ? P[i * N + j] : 0.0;"),
+    ("dropout flags left out of dP", "dP[i * N + jj] = s * zs;", "dP[i * N + jj] = s;"),
 ]
 
 
