@@ -169,7 +169,15 @@ def job_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
 
 
 # ------------------------------------------------------------------------- our arm
-KERNEL_NAMES = ["fwd", "bwd_preprocess", "bwd_dkdv", "bwd_dq"]
+def kernel_names(w, deterministic=False):
+    """The kernels of one step, in launch order: the forward, then the backward's delta
+    preprocess and either the fused pass and the dQ conversion (head_dim 64) or the dK/dV
+    and dQ passes."""
+    if not w.backward:
+        return ["fwd"]
+    if w.d == 64 and not deterministic:
+        return ["fwd", "bwd_preprocess", "bwd_fused", "bwd_dq_convert"]
+    return ["fwd", "bwd_preprocess", "bwd_dkdv", "bwd_dq"]
 
 
 class Problem:
@@ -179,7 +187,7 @@ class Problem:
     the backward's three phases form delta from it; with ALiBi the slopes ride in the same
     options. Each phase is its own C-ABI call, so CUDA events can sit between kernels."""
 
-    def __init__(self, w, dev, host=None, seed=0):
+    def __init__(self, w, dev, host=None, seed=0, plain=False, deterministic=False):
         import torch
         from exact_attention_126_b200 import fa, workloads
         self.w, self.dev, self.fa = w, dev, fa
@@ -206,12 +214,16 @@ class Problem:
         if w.alibi:
             self.slopes = torch.tensor(workloads.alibi_slopes(H), dtype=torch.float32,
                                        device=dev)
-        self.opt = fa.options(alibi_slopes=self.slopes, o_low=self.o_low)
-        self.launches = 4 if w.backward else 1
+        # plain: the forward keeps no residual and delta is formed from the bf16 O
+        self.opt = fa.options(alibi_slopes=self.slopes, o_low=None if plain else self.o_low,
+                              deterministic=deterministic)
+        self.names = kernel_names(w, deterministic)
+        self.fused = "bwd_fused" in self.names
+        self.launches = len(self.names)
 
     def step(self, sp, evs=None):
-        """One pass of the path on stream handle `sp`; evs: len(KERNEL_NAMES) + 1 events
-        (only the first two with a forward-only workload), recorded between kernels."""
+        """One pass of the path on stream handle `sp`; evs: len(self.names) + 1 events,
+        recorded between kernels."""
         fa, w = self.fa, self.w
         stream = self.stream
         if evs is not None:
@@ -225,12 +237,19 @@ class Problem:
         fa.fa_bwd_preprocess(self.o, self.do, self.lse, self.ws, self.opt, sp)
         if evs is not None:
             evs[2].record(stream)
-        fa.fa_bwd_dkdv(self.q, self.k, self.v, self.do, self.ws, self.dk, self.dv,
-                       w.softmax_scale, w.causal, w.window, sp, self.opt)
-        if evs is not None:
-            evs[3].record(stream)
-        fa.fa_bwd_dq(self.q, self.k, self.v, self.do, self.ws, self.dq, w.softmax_scale,
-                     w.causal, w.window, sp, self.opt)
+        if self.fused:
+            fa.fa_bwd_fused(self.q, self.k, self.v, self.do, self.ws, self.dk, self.dv,
+                            w.softmax_scale, w.causal, w.window, sp, self.opt)
+            if evs is not None:
+                evs[3].record(stream)
+            fa.fa_bwd_dq_convert(self.ws, self.dq, w.softmax_scale, sp)
+        else:
+            fa.fa_bwd_dkdv(self.q, self.k, self.v, self.do, self.ws, self.dk, self.dv,
+                           w.softmax_scale, w.causal, w.window, sp, self.opt)
+            if evs is not None:
+                evs[3].record(stream)
+            fa.fa_bwd_dq(self.q, self.k, self.v, self.do, self.ws, self.dq, w.softmax_scale,
+                         w.causal, w.window, sp, self.opt)
         if evs is not None:
             evs[4].record(stream)
 
@@ -252,7 +271,7 @@ class Problem:
         torch.cuda.synchronize(self.dev)
         if self.fa.fa_debug_status(sp) != 0:
             raise RuntimeError("a kernel abandoned a bounded wait during warm-up")
-        n_ev = len(KERNEL_NAMES) + 1 if w.backward else 2
+        n_ev = len(self.names) + 1
         events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
                   for _ in range(steps)]
         t0 = torch.cuda.Event(enable_timing=True)
@@ -267,7 +286,7 @@ class Problem:
         torch.cuda.synchronize(self.dev)
         if self.fa.fa_debug_status(sp) != 0:
             raise RuntimeError("a kernel abandoned a bounded wait in the timed region")
-        names = KERNEL_NAMES[: n_ev - 1]
+        names = self.names
         per_kernel = {n: 0.0 for n in names}
         step_ms = 0.0
         for evs in events:
@@ -282,9 +301,11 @@ class Problem:
 def kernel_flops(w):
     """Algorithmic flops credited to each kernel (the metric's convention): forward = the
     forward count; dK/dV = 2x (S^T, dP^T, dV, dK products); dQ = 0.5x (its dQ product;
-    the recomputation of S and dP is not credited)."""
+    the recomputation of S and dP is not credited); the fused pass = 2.5x (all five
+    products); preprocess and dQ conversion move bytes only."""
     f = w.fwd_flops()
-    return {"fwd": f, "bwd_preprocess": 0.0, "bwd_dkdv": 2.0 * f, "bwd_dq": 0.5 * f}
+    return {"fwd": f, "bwd_preprocess": 0.0, "bwd_dkdv": 2.0 * f, "bwd_dq": 0.5 * f,
+            "bwd_fused": 2.5 * f, "bwd_dq_convert": 0.0}
 
 
 def workload_line(w, ms, per_kernel, flushed):
@@ -319,7 +340,7 @@ def run_ours(args, w, rank, world, local_rank):
                                 device_id=dev)
 
     inp_host = synth.attention_inputs(w.B, w.H, w.N, w.d, w.seed_index, with_grad=True, pin=True)
-    prob = Problem(w, dev, host=inp_host)
+    prob = Problem(w, dev, host=inp_host, plain=args.plain, deterministic=args.deterministic)
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
 
@@ -356,7 +377,8 @@ def run_ours(args, w, rank, world, local_rank):
         host_out["lse"].copy_(res[1], non_blocking=True)
         if w.backward:
             grads = fa.attention_backward(q, k, v, res[0], res[1], do, w.softmax_scale, w.causal,
-                                          w.window, sp, alibi_slopes=prob.slopes, o_low=res[2])
+                                          w.window, sp, alibi_slopes=prob.slopes, o_low=res[2],
+                                          deterministic=args.deterministic)
             for n, t in zip(("dq", "dk", "dv"), grads):
                 host_out[n].copy_(t, non_blocking=True)
 
@@ -385,7 +407,8 @@ def run_ours(args, w, rank, world, local_rank):
             if WORKLOADS[name].name == w.name:
                 continue
             ow = WORKLOADS[name]
-            op = Problem(ow, dev, seed=1000 + ow.seed_index)
+            op = Problem(ow, dev, seed=1000 + ow.seed_index, plain=args.plain,
+                         deterministic=args.deterministic)
             with ClockSampler(local_rank) as oc:
                 oms, oker, _ = op.time(max(20, args.steps), args.warmup, stream)
             line = workload_line(ow, oms, oker, op.flushed)
@@ -446,7 +469,11 @@ def run_ours(args, w, rank, world, local_rank):
             "workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
             "window": list(w.window), "alibi": w.alibi,
             "pass": "fwd+bwd" if w.backward else "fwd",
-            "path": "training path: forward keeps O - bf16(O) for the backward's delta",
+            "path": ("plain: delta from the bf16 O" if args.plain else
+                     "training path: forward keeps O - bf16(O) for the backward's delta")
+                    + ("; deterministic backward (separate dQ pass)" if args.deterministic else
+                       ""),
+            "kernels": list(per_kernel),
             "step_gflop": round(flops / 1e9, 3),
             "parallelism": "replicas" if world > 1 else "single",
             "l2": summary["l2"],
@@ -457,7 +484,7 @@ def run_ours(args, w, rank, world, local_rank):
         "e2e": {"value": round(job_tflops(flops, world, e2e_ms), 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "steps": e2e_steps,
                 "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes},
-        "gpu_launches": (4 if w.backward else 1) * args.steps,
+        "gpu_launches": len(per_kernel) * args.steps,
         "kernels": kernels,
         "roofline": roofline,
         "kernel_source_hash": kernel_source_hash(),
@@ -569,6 +596,10 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--also", default="c2,c3,c4,c5c,c5w",
                     help="other workloads timed at full size in the same run (comma list)")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="time the backward with the separate dQ pass at head_dim 64 too")
+    ap.add_argument("--plain", action="store_true",
+                    help="time the path without the O residual (delta from the bf16 O)")
     ap.add_argument("--no-workloads", action="store_true",
                     help="time the headline workload only")
     args = ap.parse_args(argv)

@@ -11,15 +11,14 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "libfa.so")
-MAIN = os.path.join(CSRC, "fa_api.cu")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo", "-O3", "-std=c++17",
     "--expt-relaxed-constexpr",
-    "-Xcompiler", "-fPIC,-O2",
-    "-shared",
+    "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden",
 ]
+BUILD_DIR = os.path.join(PKG, "_build")
 
 
 def _nvcc() -> str:
@@ -29,9 +28,14 @@ def _nvcc() -> str:
     return "nvcc"
 
 
+def units() -> list[str]:
+    """The compilation units: the host side of the C ABI and one unit per kernel family."""
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+
+
 def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
-                  + glob.glob(os.path.join(INCLUDE, "*.h")))
+                  + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
 def up_to_date() -> bool:
@@ -42,13 +46,24 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    """Compiles the library unless it is newer than every source; returns its path."""
+    """Compiles the library unless it is newer than every source; returns its path. The
+    units compile in parallel (one nvcc each), then nvcc links them into libfa.so."""
     if not force and up_to_date():
         return LIBRARY
+    os.makedirs(BUILD_DIR, exist_ok=True)
+    flags = NVCC_FLAGS + (["-Xptxas", "-v"] if verbose else []) + (extra or [])
+    procs, objs = [], []
+    for src in units():
+        obj = os.path.join(BUILD_DIR, os.path.basename(src)[:-3] + ".o")
+        objs.append(obj)
+        cmd = [_nvcc()] + flags + ["-I", INCLUDE, "-I", CSRC, "-c", "-o", obj, src]
+        procs.append((src, subprocess.Popen(cmd)))
+    failed = [src for src, p in procs if p.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, "nvcc " + " ".join(failed))
     tmp = LIBRARY + ".tmp%d" % os.getpid()
-    cmd = [_nvcc()] + NVCC_FLAGS + (["-Xptxas", "-v"] if verbose else []) + (extra or []) + [
-        "-I", INCLUDE, "-I", CSRC, "-o", tmp, MAIN]
-    subprocess.run(cmd, check=True)
+    subprocess.run([_nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp]
+                   + objs, check=True)
     os.replace(tmp, LIBRARY)
     return LIBRARY
 

@@ -1,59 +1,27 @@
 // fa_api.cu - host side of the C ABI declared in include/fa.h.
 //
-// Validates every argument before touching the GPU, encodes one TMA tensor map per input
-// tensor ((B*H, N, d) viewed as a 3-D tensor so that the rows past N of a (batch, head)
-// read as zeros instead of the next head's rows), and launches the kernels of
-// fa_fwd.cuh / fa_bwd.cuh on the caller's stream.
+// Validates every argument before touching the GPU, resolves the options into a kernel
+// variant and calls the launchers of the kernel units (fa_kern_*.cu) on the caller's
+// stream. Holds the fixed device array of fa_bwd_noalloc.
 #include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <utility>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "fa.h"
-#include "fa_bwd.cuh"
-#include "fa_fwd.cuh"
+#include "launch.h"
 
 namespace {
 
-using fa::kBlock;
+using fa_host::Extras;
+using fa_host::Problem;
 
 // Test hook set by fa_debug_set_fault(); 0 in normal operation.
 std::atomic<int> g_fault{0};
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
-// (B*H, N, d) bf16 tensor, box of 128 rows x 64 columns (128 bytes), 128-byte swizzle.
-bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
-  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
-  const cuuint32_t box[3] = {64, (cuuint32_t)kBlock, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -85,166 +53,73 @@ fa_status_t check_ptrs(std::initializer_list<const void*> ptrs) {
   return FA_OK;
 }
 
-template <typename Kernel>
-fa_status_t set_smem(Kernel k, int bytes) {
-  // Per device and kernel; cheap enough to repeat, but only needed once per device.
-  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
-             ? FA_OK
-             : FA_ERR_CUDA;
+// Calls L::template run<F>(args...) for the compile-time F in Fs... equal to `feat`; the
+// lists below are the feature sets each kernel family is instantiated for.
+template <typename L, int... Fs, typename... Args>
+fa_status_t dispatch_features(std::integer_sequence<int, Fs...>, int feat, Args&&... args) {
+  fa_status_t s = FA_ERR_UNSUPPORTED;
+  const bool found = ((feat == Fs ? (s = L::template run<Fs>(std::forward<Args>(args)...), true)
+                                  : false) || ...);
+  return found ? s : FA_ERR_UNSUPPORTED;
 }
 
-template <typename Kernel>
-int launch_regs(Kernel k) {
-  cudaFuncAttributes attr;
-  if (cudaFuncGetAttributes(&attr, k) != cudaSuccess) return -1;
-  return attr.numRegs;
-}
+// forward: every combination of ALiBi, key padding, residual and dropout
+using FwdFeatures = std::integer_sequence<int, 0, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14, 15>;
+// backward passes: ALiBi, key padding and dropout (the residual only changes delta)
+using BwdFeatures = std::integer_sequence<int, 0, 1, 2, 3, 8, 9, 10, 11>;
 
-int sm_count() {
-  static int cache[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
-  int n = 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
-  if (dev >= 0 && dev < 64) cache[dev] = n;
-  return n;
-}
-
-// Heads per chunk of the masked schedules: enough for about one item per SM.
-int head_group(int BH, int tiles) {
-  int g = (sm_count() + tiles - 1) / tiles;
-  if (g < 1) g = 1;
-  if (g > BH) g = BH;
-  return g;
-}
-
-fa_status_t launched() {
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-}
-
-
-// Optional inputs and outputs of one call (fa_options_t, checked and resolved).
-struct Extras {
-  const float* alibi = nullptr;    // H slopes: the kAlibi kernels
-  const uint8_t* kpad = nullptr;   // (B, N) key-padding flags
-  void* o_low = nullptr;           // bf16 residual of O: written by the forward, read by delta
+// The launchers as class templates over the feature flags, for dispatch_features.
+template <int D>
+struct FwdLaunch {
+  template <int F, typename... Args>
+  static fa_status_t run(Args&&... args) {
+    return fa_host::launch_fwd<D, F>(std::forward<Args>(args)...);
+  }
+};
+template <int D>
+struct DkdvLaunch {
+  template <int F, typename... Args>
+  static fa_status_t run(Args&&... args) {
+    return fa_host::launch_dkdv<D, F>(std::forward<Args>(args)...);
+  }
+};
+template <int D>
+struct DqLaunch {
+  template <int F, typename... Args>
+  static fa_status_t run(Args&&... args) {
+    return fa_host::launch_dq<D, F>(std::forward<Args>(args)...);
+  }
 };
 
-template <int D, bool kAlibi>
-fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int BH,
-                       int H, int N, float scale, int left, int right, const Extras& x,
-                       cudaStream_t st) {
-  CUtensorMap mq, mkk, mv;
-  if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) || !make_map(&mv, v, BH, N, D))
-    return FA_ERR_CUDA;
-  using C = fa::FwdCfg<D>;
-  if (set_smem(fa::fa_fwd_kernel<D, kAlibi>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
-  fa::FwdArgs a;
-  a.o = static_cast<__nv_bfloat16*>(o);
-  a.lse = lse;
-  a.N = N;
-  a.BH = BH;
-  a.n_qtiles = fa::num_tiles(N);
-  a.n_pairs = (a.n_qtiles + 1) / 2;
-  a.n_items = BH * a.n_pairs;
-  a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
-  a.group = head_group(BH, a.n_pairs);
-  a.scale_log2 = scale * fa::kLog2e;
-  a.left = left;
-  a.right = right;
-  a.fault = g_fault.load(std::memory_order_relaxed);
-  a.alibi = x.alibi;
-  a.H = H;
-  a.kpad = x.kpad;
-  a.o_low = static_cast<__nv_bfloat16*>(x.o_low);
-  const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
-  fa::fa_fwd_kernel<D, kAlibi><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, a);
-  return launched();
-}
+struct FusedLaunch {
+  template <int F, typename... Args>
+  static fa_status_t run(Args&&... args) {
+    return fa_host::launch_fused<F>(std::forward<Args>(args)...);
+  }
+};
 
-int padded_rows(int N) { return fa::num_tiles(N) * kBlock; }
+int padded_rows(int N) { return fa::num_tiles(N) * fa::kBlock; }
 
-template <int D>
-fa_status_t launch_preprocess(const void* o, const void* o_low, const void* dout,
-                              const float* lse, float* stats, int BH, int N, cudaStream_t st) {
-  const int Np = padded_rows(N);
-  // 64 rows per block, blocks of one head consecutive; BH * Np / 64 < 2^31 because every
-  // tensor has fewer than 2^31 elements (d >= 64)
-  const long long blocks = (long long)BH * (Np / 64);
-  fa::fa_bwd_preprocess_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(o_low),
-      static_cast<const __nv_bfloat16*>(dout), lse, stats, BH, N, Np);
-  return launched();
-}
-
-// Arguments both backward passes share.
-fa::BwdArgs bwd_args(const void* ws, int BH, int H, int N, float scale, int left, int right,
-                     const Extras& x) {
-  fa::BwdArgs a;
-  a.stats = static_cast<const float*>(ws);
-  a.out0 = nullptr;
-  a.out1 = nullptr;
-  a.stat_rows = (long long)BH * padded_rows(N);
-  a.Np = padded_rows(N);
-  a.N = N;
-  a.n_tiles = fa::num_tiles(N);
-  a.scale = scale;
-  a.scale_log2 = scale * fa::kLog2e;
-  a.left = left;
-  a.right = right;
-  a.BH = BH;
-  a.n_items = BH * a.n_tiles;
-  a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
-  a.group = head_group(BH, a.n_tiles);
-  a.alibi = x.alibi;
-  a.H = H;
-  a.kpad = x.kpad;
-  return a;
-}
-
-template <int D, bool kAlibi>
-fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void* dout,
-                        const void* ws, void* dk, void* dv, int BH, int H, int N, float scale,
-                        int left, int right, const Extras& x, cudaStream_t st) {
-  CUtensorMap mq, mkk, mv, mdo, mdk, mdv;
-  if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
-      !make_map(&mv, v, BH, N, D) || !make_map(&mdo, dout, BH, N, D) ||
-      !make_map(&mdk, dk, BH, N, D) || !make_map(&mdv, dv, BH, N, D))
-    return FA_ERR_CUDA;
-  using C = fa::DkdvCfg<D>;
-  if (set_smem(fa::fa_bwd_dkdv_kernel<D, kAlibi>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
-  fa::BwdArgs a = bwd_args(ws, BH, H, N, scale, left, right, x);
-  a.out0 = static_cast<__nv_bfloat16*>(dk);
-  a.out1 = static_cast<__nv_bfloat16*>(dv);
-  const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
-  fa::fa_bwd_dkdv_kernel<D, kAlibi><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo,
-                                                                               mdk, mdv, a);
-  return launched();
-}
-
-template <int D, bool kAlibi>
-fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* dout,
-                      const void* ws, void* dq, int BH, int H, int N, float scale, int left,
-                      int right, const Extras& x, cudaStream_t st) {
-  CUtensorMap mq, mkk, mv, mdo, mdq;
-  if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
-      !make_map(&mv, v, BH, N, D) || !make_map(&mdo, dout, BH, N, D) ||
-      !make_map(&mdq, dq, BH, N, D))
-    return FA_ERR_CUDA;
-  using C = fa::DqCfg<D>;
-  if (set_smem(fa::fa_bwd_dq_kernel<D, kAlibi>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
-  fa::BwdArgs a = bwd_args(ws, BH, H, N, scale, left, right, x);
-  a.out0 = static_cast<__nv_bfloat16*>(dq);
-  const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
-  fa::fa_bwd_dq_kernel<D, kAlibi><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, mdq,
-                                                                             a);
-  return launched();
-}
-
-size_t workspace_bytes(int B, int H, int N) {
+// Workspace of the backward: the row statistics (two fp32 arrays of B*H*Np), then, for the
+// fused pass (head_dim 64), the fp32 dQ accumulator (B*H*Np rows of 64), each part rounded
+// up to 256 bytes.
+size_t stats_bytes(int B, int H, int N) {
   const size_t raw = 2 * (size_t)B * H * padded_rows(N) * sizeof(float);
   return (raw + 255) & ~size_t(255);
+}
+
+bool uses_fused(int d, const Extras& x) { return d == 64 && !x.deterministic; }
+
+size_t dq_acc_bytes(int B, int H, int N, int d) {
+  return (size_t)B * H * padded_rows(N) * (size_t)d * sizeof(float);
+}
+
+size_t workspace_bytes(int B, int H, int N, int d, const Extras& x) {
+  return stats_bytes(B, H, N) + (uses_fused(d, x) ? dq_acc_bytes(B, H, N, d) : 0);
+}
+
+float* dq_acc_of(void* workspace, int B, int H, int N) {
+  return reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + stats_bytes(B, H, N));
 }
 
 // Checks the optional arguments of an _ex call and resolves them; a null `opt` means none.
@@ -254,10 +129,25 @@ fa_status_t resolve_options(const fa_options_t* opt, Extras* x) {
   if (opt->alibi_slopes != nullptr && (reinterpret_cast<uintptr_t>(opt->alibi_slopes) & 3u) != 0)
     return FA_ERR_MISALIGNED;
   if (opt->o_low != nullptr && !aligned16(opt->o_low)) return FA_ERR_MISALIGNED;
-  if (!(opt->dropout_p == 0.f)) return FA_ERR_UNSUPPORTED;
+  // dropout: t = floor(256 p + 1/2) must leave some weights (t <= 255); the offset is the
+  // fourth 32-bit counter word
+  const float p = opt->dropout_p;
+  if (!(p >= 0.f && p < 1.f) || opt->dropout_offset > 0xFFFFFFFFull) return FA_ERR_INVALID_ARG;
+  const int t = (int)std::floor(256.0 * (double)p + 0.5);
+  if (t > 255) return FA_ERR_INVALID_ARG;
+  if ((opt->flags & ~(unsigned)FA_BWD_DETERMINISTIC) != 0) return FA_ERR_INVALID_ARG;
   x->alibi = opt->alibi_slopes;
   x->kpad = opt->key_padding;
   x->o_low = opt->o_low;
+  x->deterministic = (opt->flags & FA_BWD_DETERMINISTIC) != 0;
+  if (t > 0) {
+    x->dropout = true;
+    x->drop.seed_lo = (uint32_t)(opt->dropout_seed & 0xFFFFFFFFull);
+    x->drop.seed_hi = (uint32_t)(opt->dropout_seed >> 32);
+    x->drop.offset = (uint32_t)opt->dropout_offset;
+    x->drop.threshold = (uint32_t)t;
+    x->drop.keep_scale = (float)(256.0 / (256.0 - t));
+  }
   return FA_OK;
 }
 
@@ -279,11 +169,12 @@ fa_status_t forward(const void* q, const void* k, const void* v, void* o, float*
   const int right = fa::resolve_right(causal, window.right);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int l = window.left, BH = B * H;
-  if (x.alibi != nullptr)
-    return d == 64 ? launch_fwd<64, true>(q, k, v, o, lse, BH, H, N, scale, l, right, x, st)
-                   : launch_fwd<128, true>(q, k, v, o, lse, BH, H, N, scale, l, right, x, st);
-  return d == 64 ? launch_fwd<64, false>(q, k, v, o, lse, BH, H, N, scale, l, right, x, st)
-                 : launch_fwd<128, false>(q, k, v, o, lse, BH, H, N, scale, l, right, x, st);
+  const Problem pb{BH, H, N, scale, l, right};
+  const int fault = g_fault.load(std::memory_order_relaxed);
+  return d == 64 ? dispatch_features<FwdLaunch<64>>(FwdFeatures(), x.features(), q, k, v, o, lse, pb, x,
+                                                        fault, st)
+                 : dispatch_features<FwdLaunch<128>>(FwdFeatures(), x.features(), q, k, v, o, lse, pb, x,
+                                                         fault, st);
 }
 
 // Step 1 of the backward: the row statistics in `workspace`.
@@ -295,8 +186,43 @@ fa_status_t preprocess(const void* o, const void* dout, const float* lse, void* 
   if ((s = check_ptrs({o, dout, lse, workspace})) != FA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* stats = static_cast<float*>(workspace);
-  return d == 64 ? launch_preprocess<64>(o, x.o_low, dout, lse, stats, B * H, N, st)
-                 : launch_preprocess<128>(o, x.o_low, dout, lse, stats, B * H, N, st);
+  // the fused pass accumulates dQ: its accumulator starts at zero
+  float* acc = uses_fused(d, x) ? dq_acc_of(workspace, B, H, N) : nullptr;
+  return d == 64 ? fa_host::launch_preprocess<64>(o, x.o_low, dout, lse, stats, acc, B * H, N, st)
+                 : fa_host::launch_preprocess<128>(o, x.o_low, dout, lse, stats, acc, B * H, N,
+                                                   st);
+}
+
+// The fused pass (head_dim 64): dK, dV, and dQ added into the workspace's accumulator.
+fa_status_t fused_pass(const void* q, const void* k, const void* v, const void* dout,
+                       void* workspace, void* dk, void* dv, int B, int H, int N, int d,
+                       float scale, int causal, fa_window_t window, const Extras& x,
+                       void* stream) {
+  bool empty;
+  fa_status_t s = check_problem(B, H, N, d, &empty);
+  if (s != FA_OK || empty) return s;
+  if (d != 64) return FA_ERR_UNSUPPORTED;
+  if ((s = check_mask(scale, window)) != FA_OK) return s;
+  if ((s = check_ptrs({q, k, v, dout, workspace, dk, dv})) != FA_OK) return s;
+  const int right = fa::resolve_right(causal, window.right);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Problem pb{B * H, H, N, scale, window.left, right};
+  const int feat = x.features() & ~fa::kFeatResidual;
+  return dispatch_features<FusedLaunch>(BwdFeatures(), feat, q, k, v, dout, workspace,
+                                        dq_acc_of(workspace, B, H, N), dk, dv, pb, x, st);
+}
+
+// dQ from the fused pass's accumulator.
+fa_status_t dq_convert(void* workspace, void* dq, int B, int H, int N, int d, float scale,
+                       void* stream) {
+  bool empty;
+  fa_status_t s = check_problem(B, H, N, d, &empty);
+  if (s != FA_OK || empty) return s;
+  if (d != 64) return FA_ERR_UNSUPPORTED;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if ((s = check_ptrs({workspace, dq})) != FA_OK) return s;
+  return fa_host::launch_dq_convert<64>(dq_acc_of(workspace, B, H, N), dq, B * H, N, scale,
+                                        static_cast<cudaStream_t>(stream));
 }
 
 // Step 2: dK, dV.
@@ -312,15 +238,12 @@ fa_status_t dkdv_pass(const void* q, const void* k, const void* v, const void* d
   const int right = fa::resolve_right(causal, window.right);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int l = window.left, BH = B * H;
-  if (x.alibi != nullptr)
-    return d == 64 ? launch_dkdv<64, true>(q, k, v, dout, workspace, dk, dv, BH, H, N, scale, l,
-                                           right, x, st)
-                   : launch_dkdv<128, true>(q, k, v, dout, workspace, dk, dv, BH, H, N, scale, l,
-                                            right, x, st);
-  return d == 64 ? launch_dkdv<64, false>(q, k, v, dout, workspace, dk, dv, BH, H, N, scale, l,
-                                          right, x, st)
-                 : launch_dkdv<128, false>(q, k, v, dout, workspace, dk, dv, BH, H, N, scale, l,
-                                           right, x, st);
+  const int feat = x.features() & ~fa::kFeatResidual;
+  const Problem pb{BH, H, N, scale, l, right};
+  return d == 64 ? dispatch_features<DkdvLaunch<64>>(BwdFeatures(), feat, q, k, v, dout, workspace, dk, dv,
+                                                        pb, x, st)
+                 : dispatch_features<DkdvLaunch<128>>(BwdFeatures(), feat, q, k, v, dout, workspace, dk, dv,
+                                                         pb, x, st);
 }
 
 // Step 3: dQ.
@@ -335,15 +258,12 @@ fa_status_t dq_pass(const void* q, const void* k, const void* v, const void* dou
   const int right = fa::resolve_right(causal, window.right);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int l = window.left, BH = B * H;
-  if (x.alibi != nullptr)
-    return d == 64 ? launch_dq<64, true>(q, k, v, dout, workspace, dq, BH, H, N, scale, l, right,
-                                         x, st)
-                   : launch_dq<128, true>(q, k, v, dout, workspace, dq, BH, H, N, scale, l,
-                                          right, x, st);
-  return d == 64 ? launch_dq<64, false>(q, k, v, dout, workspace, dq, BH, H, N, scale, l, right,
-                                        x, st)
-                 : launch_dq<128, false>(q, k, v, dout, workspace, dq, BH, H, N, scale, l, right,
-                                         x, st);
+  const int feat = x.features() & ~fa::kFeatResidual;
+  const Problem pb{BH, H, N, scale, l, right};
+  return d == 64 ? dispatch_features<DqLaunch<64>>(BwdFeatures(), feat, q, k, v, dout, workspace, dq, pb, x,
+                                                      st)
+                 : dispatch_features<DqLaunch<128>>(BwdFeatures(), feat, q, k, v, dout, workspace, dq, pb, x,
+                                                       st);
 }
 
 // The three steps of the backward, with the statistics in `stats` (caller workspace or the
@@ -354,6 +274,12 @@ fa_status_t backward(const void* q, const void* k, const void* v, const void* o,
                      void* stream) {
   fa_status_t s;
   if ((s = preprocess(o, dout, lse, stats, B, H, N, d, x, stream)) != FA_OK) return s;
+  if (uses_fused(d, x)) {
+    if ((s = fused_pass(q, k, v, dout, stats, dk, dv, B, H, N, d, scale, causal, window, x,
+                        stream)) != FA_OK)
+      return s;
+    return dq_convert(stats, dq, B, H, N, d, scale, stream);
+  }
   if ((s = dkdv_pass(q, k, v, dout, stats, dk, dv, B, H, N, d, scale, causal, window, x,
                      stream)) != FA_OK)
     return s;
@@ -445,6 +371,9 @@ fa_status_t noalloc_scratch(void** out) {
 
 }  // namespace
 
+// The library is compiled with hidden visibility: only the entry points of include/fa.h
+// are exported.
+#pragma GCC visibility push(default)
 extern "C" {
 
 fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
@@ -478,7 +407,7 @@ fa_status_t fa_fwd_alibi(const void* q, const void* k, const void* v, void* o, f
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   bool empty;
   if (check_problem(B, H, N, d, &empty) != FA_OK || empty) return 0;
-  return workspace_bytes(B, H, N);
+  return workspace_bytes(B, H, N, d, Extras());
 }
 
 fa_status_t fa_bwd_preprocess(const void* o, const void* dout, const float* lse,
@@ -511,6 +440,22 @@ fa_status_t fa_bwd_dq(const void* q, const void* k, const void* v, const void* d
   return dq_pass(q, k, v, dout, workspace, dq, B, H, N, d, scale, causal, window, x, stream);
 }
 
+fa_status_t fa_bwd_fused(const void* q, const void* k, const void* v, const void* dout,
+                         void* workspace, void* dk, void* dv, int B, int H, int N, int d,
+                         float scale, int causal, fa_window_t window, const fa_options_t* options,
+                         void* stream) {
+  Extras x;
+  fa_status_t s = resolve_options(options, &x);
+  if (s != FA_OK) return s;
+  return fused_pass(q, k, v, dout, workspace, dk, dv, B, H, N, d, scale, causal, window, x,
+                    stream);
+}
+
+fa_status_t fa_bwd_dq_convert(void* workspace, void* dq, int B, int H, int N, int d, float scale,
+                              void* stream) {
+  return dq_convert(workspace, dq, B, H, N, d, scale, stream);
+}
+
 fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                    float scale, int causal, fa_window_t window, void* workspace,
@@ -531,7 +476,7 @@ fa_status_t fa_bwd_ex(const void* q, const void* k, const void* v, const void* o
   Extras x;
   if ((s = resolve_options(options, &x)) != FA_OK) return s;
   if ((s = check_ptrs({workspace})) != FA_OK) return s;
-  if (workspace_bytes_given < workspace_bytes(B, H, N)) return FA_ERR_WORKSPACE;
+  if (workspace_bytes_given < workspace_bytes(B, H, N, d, x)) return FA_ERR_WORKSPACE;
   return backward(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, window, x,
                   workspace, stream);
 }
@@ -547,9 +492,9 @@ fa_status_t fa_bwd_alibi(const void* q, const void* k, const void* v, const void
   if (s != FA_OK || empty) return s;
   if ((s = check_slopes(alibi_slopes)) != FA_OK) return s;
   if ((s = check_ptrs({workspace})) != FA_OK) return s;
-  if (workspace_bytes_given < workspace_bytes(B, H, N)) return FA_ERR_WORKSPACE;
   Extras x;
   x.alibi = alibi_slopes;
+  if (workspace_bytes_given < workspace_bytes(B, H, N, d, x)) return FA_ERR_WORKSPACE;
   return backward(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, window, x,
                   workspace, stream);
 }
@@ -562,11 +507,14 @@ fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const vo
   fa_status_t s =
       check_backward(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, window, &empty);
   if (s != FA_OK || empty) return s;
-  if (workspace_bytes(B, H, N) > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
+  // the three-kernel backward, whose only scratch is the row statistics
+  Extras x;
+  x.deterministic = true;
+  if (workspace_bytes(B, H, N, d, x) > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
   void* scratch = nullptr;
   if ((s = noalloc_scratch(&scratch)) != FA_OK) return s;
   // The statistics are rewritten in full by the preprocess step, so nothing needs clearing.
-  return backward(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, window, Extras(),
+  return backward(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, window, x,
                   scratch, stream);
 }
 
@@ -585,14 +533,16 @@ const char* fa_status_string(fa_status_t status) {
 
 fa_status_t fa_debug_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
-  int v = 0;
-  if (cudaMemcpyFromSymbol(&v, fa::g_fa_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
-  if (v != 0) {
-    const int zero = 0;
-    if (cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
-    return FA_ERR_TIMEOUT;
+  // every kernel unit has its own copy of the status word: read and clear them all
+  const int words[5] = {fa_host::take_status_fwd64(), fa_host::take_status_fwd128(),
+                        fa_host::take_status_bwd64(), fa_host::take_status_bwd128(),
+                        fa_host::take_status_fused64()};
+  bool timeout = false;
+  for (int w : words) {
+    if (w < 0) return FA_ERR_CUDA;
+    if (w != 0) timeout = true;
   }
-  return FA_OK;
+  return timeout ? FA_ERR_TIMEOUT : FA_OK;
 }
 
 fa_status_t fa_debug_set_fault(int fault) {
@@ -604,3 +554,4 @@ fa_status_t fa_debug_set_fault(int fault) {
 int fa_version(void) { return 200; }
 
 }  // extern "C"
+#pragma GCC visibility pop

@@ -33,6 +33,7 @@
 
 #include <cuda_bf16.h>
 
+#include "rng.cuh"
 #include "sm100.cuh"
 #include "tiles.cuh"
 
@@ -47,6 +48,8 @@ namespace fa {
 // o_r + o_low_r, which carries about 16 significant bits instead of 8: for rows whose
 // softmax is nearly one-hot, dS = P (dP - delta) cancels almost completely and the
 // rounding of a bf16 O would dominate dQ and dK.
+// With dq_acc (the fused backward's fp32 dQ accumulator, (B*H, Np, D)), each block also
+// zeroes the accumulator rows it covers.
 // Block b covers rows 64x .. 64x+63 of head bh, with (bh, x) = divmod(b, Np/64), 8 rows
 // per warp; G = D/8 lanes share a row, 16 bytes of O and dO per lane, and a warp's loads
 // for its 8 rows are all issued before any is used.
@@ -56,7 +59,8 @@ __global__ void __launch_bounds__(256)
     fa_bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o,
                              const __nv_bfloat16* __restrict__ o_low,
                              const __nv_bfloat16* __restrict__ dout, const float* __restrict__ lse,
-                             float* __restrict__ stats, int BH, int N, int Np) {
+                             float* __restrict__ stats, float* __restrict__ dq_acc, int BH, int N,
+                             int Np) {
   constexpr int G = D / 8;                      // lanes per row
   constexpr int kRowsPerPass = 32 / G;          // rows a warp covers per load
   constexpr int kPasses = 8 / kRowsPerPass;     // 8 rows per warp
@@ -67,6 +71,13 @@ __global__ void __launch_bounds__(256)
   const int sub = lane / G;                     // row within the pass
   const int part = lane % G;                    // 16-byte slice of the row
   const int row0 = xb * 64 + (threadIdx.x >> 5) * 8;
+  if (dq_acc != nullptr) {
+    // the fused backward's dQ accumulator: this block's 64 rows (D fp32 each) start at zero
+    float4* z = reinterpret_cast<float4*>(dq_acc + ((size_t)bh * Np + (size_t)xb * 64) * D);
+    constexpr int kVec = 64 * D / 4;
+#pragma unroll
+    for (int e = threadIdx.x; e < kVec; e += 256) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   uint4 a[kPasses], b[kPasses], c[kPasses];
 #pragma unroll
   for (int p = 0; p < kPasses; ++p) {
@@ -127,6 +138,7 @@ struct BwdArgs {
   const float* alibi;   // ALiBi kernels: one slope per head (heads = H)
   int H;                // heads per batch entry (batch entry of bh = bh / H)
   const uint8_t* kpad;  // (B, N) key-padding flags (nonzero = padded key), or null
+  DropoutArgs drop;     // kFeatDropout kernels
 };
 
 // Shared layout of both backward kernels: the stationary tiles X0, X1 of an item (in XB
@@ -308,8 +320,12 @@ __device__ __forceinline__ void bwd_teardown(uint32_t tmem, int warp) {
 // dV += P^T dO and dK += dS^T Q as soon as the softmax publishes P^T and dS^T. Tile
 // counters (for barrier parities) run over all items of the CTA.
 // ------------------------------------------------------------------------------------
-// kAlibi: the scores carry the linear bias -m_h |i - j| (m_h = alibi[bh % H]).
-template <int D, bool kAlibi = false>
+// kFeat: kFeatAlibi, the scores carry the linear bias -m_h |i - j| (m_h = alibi[bh % H]);
+// kFeatKpad, keys flagged in a.kpad get no attention; kFeatDropout, the forward's keep
+// flags Z are regenerated: dV += (P o Z / (1-p'))^T dO and dS = P o (dP o Z / (1-p') - delta).
+// A warp owns 32 keys and 32 queries of each tile; lane l draws the flags of query l for
+// all 32 keys (two Philox calls), and 32 ballots hand each lane the flags of its own key.
+template <int D, int kFeat = 0>
 __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
     fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -318,6 +334,9 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
                        const __grid_constant__ CUtensorMap tmdK,
                        const __grid_constant__ CUtensorMap tmdV, const BwdArgs a) {
   using C = DkdvCfg<D>;
+  constexpr bool kAlibi = (kFeat & kFeatAlibi) != 0;
+  constexpr bool kKpad = (kFeat & kFeatKpad) != 0;
+  constexpr bool kDropout = (kFeat & kFeatDropout) != 0;
   constexpr int kSBufs = (D == 64) ? 2 : 1;
   constexpr uint32_t tS = 0;                         // + 128 * buffer
   constexpr uint32_t tDP = 128 * kSBufs, tDK = tDP + 128, tDV = tDK + D;
@@ -578,12 +597,25 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
       const int c = j * kBlock + t_row;  // this thread's key
       const float slope2 = kAlibi ? a.alibi[bh % a.H] * kLog2e : 0.f;
       // a padded key gets no attention from any query: its rows of P^T and dS^T are zero
-      const bool key_padded =
-          a.kpad != nullptr && c < a.N && a.kpad[(size_t)(bh / a.H) * a.N + c] != 0;
+      const bool key_padded = kKpad && c < a.N && a.kpad[(size_t)(bh / a.H) * a.N + c] != 0;
       for (int it = 0; it < n_it; ++it) {
         const int i = i_lo + it;
         const int t = g + it;
         const int s = t % C::kStages0;
+        // keep flags of this thread's key for the queries NC*h + r of tile i (bit r)
+        uint32_t keep = ~0u;
+        if (kDropout) {
+          const uint32_t blk = (uint32_t)(8 * j + 2 * (warp & 3));
+          const uint32_t qrow = (uint32_t)(i * kBlock + NC * h + lane);
+          const uint32_t mine = keep_bits16(a.drop, blk, qrow, (uint32_t)bh) |
+                                (keep_bits16(a.drop, blk + 1, qrow, (uint32_t)bh) << 16);
+          static_assert(NC == 32, "one lane per query of the warp's 32");
+#pragma unroll
+          for (int b = 0; b < 32; ++b) {
+            const uint32_t col = __ballot_sync(0xffffffffu, (mine >> b) & 1u);
+            keep = (lane == b) ? col : keep;
+          }
+        }
         if (!mbar_wait_warp(bar(C::bY0Full + s), (t / C::kStages0) & 1, abort_flag) ||
             !mbar_wait_warp(bar(bSFull + t % kSBufs), (t / kSBufs) & 1, abort_flag)) {
           ok = false;
@@ -616,14 +648,23 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
 #pragma unroll
           for (int r = 0; r < NC; ++r) p[r] = (r >= r_lo && r <= r_hi) ? p[r] : 0.f;
         }
-        if (a.kpad != nullptr) {
+        if (kKpad) {
 #pragma unroll
           for (int r = 0; r < NC; ++r) p[r] = key_padded ? 0.f : p[r];
         }
         {
           uint32_t pk[NC / 2];
+          if (kDropout) {
+            // the weights that multiplied V: P o Z / (1 - p')
+            const float ks = a.drop.keep_scale;
 #pragma unroll
-          for (int r = 0; r < NC / 2; ++r) pk[r] = pack_bf16x2(p[2 * r], p[2 * r + 1]);
+            for (int r = 0; r < NC / 2; ++r)
+              pk[r] = pack_bf16x2(((keep >> (2 * r)) & 1u) ? p[2 * r] * ks : 0.f,
+                                  ((keep >> (2 * r + 1)) & 1u) ? p[2 * r + 1] * ks : 0.f);
+          } else {
+#pragma unroll
+            for (int r = 0; r < NC / 2; ++r) pk[r] = pack_bf16x2(p[2 * r], p[2 * r + 1]);
+          }
           tmem_st16(tSb, pk);
         }
         tmem_wait_st();
@@ -636,6 +677,12 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
         tc_fence_after();
         float dp[NC];
         load_cols32(tmem + lane_base + tDP + NC * h, dp);
+        if (kDropout) {
+          // dP o Z / (1 - p'): the gradient reaching the weights before dropout
+          const float ks = a.drop.keep_scale;
+#pragma unroll
+          for (int r = 0; r < NC; ++r) dp[r] = ((keep >> r) & 1u) ? dp[r] * ks : 0.f;
+        }
         uint32_t w[NC / 2];
 #pragma unroll
         for (int e = 0; e < NC / 2; e += 2) {
@@ -691,14 +738,19 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
 // MMA issuers: one computes S and dP of each key tile in order, the other dQ += dS K_j
 // as soon as the softmax publishes dS. Tile counters run over all items.
 // ------------------------------------------------------------------------------------
-// kAlibi: the scores carry the linear bias -m_h |i - j| (m_h = alibi[bh % H]).
-template <int D, bool kAlibi = false>
+// kFeat: kFeatAlibi, the scores carry the linear bias -m_h |i - j| (m_h = alibi[bh % H]);
+// kFeatKpad, keys flagged in a.kpad get no attention; kFeatDropout, the forward's keep
+// flags Z are regenerated and dS = P o (dP o Z / (1-p') - delta).
+template <int D, int kFeat = 0>
 __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
     fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmdO,
                      const __grid_constant__ CUtensorMap tmdQ, const BwdArgs a) {
   using C = DqCfg<D>;
+  constexpr bool kAlibi = (kFeat & kFeatAlibi) != 0;
+  constexpr bool kKpad = (kFeat & kFeatKpad) != 0;
+  constexpr bool kDropout = (kFeat & kFeatDropout) != 0;
   constexpr uint32_t tS0 = 0, tDP = 256, tDQ = 384;
   // per S buffer: S full, dS full, dQ done (dQ read that buffer's dS); dP full, dP free;
   // dQ read by the epilogue, dQ of the item complete
@@ -931,6 +983,13 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
         const int jj = j_lo + it;
         const int t = g + it;
         const int b = t & 1;
+        // keep flags of this row for keys NC*h + c of tile jj (bit c)
+        uint32_t keep = ~0u;
+        if (kDropout) {
+          const uint32_t blk = (uint32_t)(8 * jj + 2 * h);
+          keep = keep_bits16(a.drop, blk, (uint32_t)r, (uint32_t)bh) |
+                 (keep_bits16(a.drop, blk + 1, (uint32_t)r, (uint32_t)bh) << 16);
+        }
         if (!mbar_wait_warp(bar(bSFull + b), (t >> 1) & 1, abort_flag)) {
           ok = false;
           break;
@@ -953,7 +1012,7 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
 #pragma unroll
           for (int c = 0; c < NC; ++c) p[c] = (c >= c_lo && c <= c_hi) ? p[c] : 0.f;
         }
-        if (a.kpad != nullptr) {
+        if (kKpad) {
           // lane l reads the flag of key NC*h + l of the tile; the ballot gives all 32
           static_assert(NC == 32, "one ballot covers a warpgroup's columns");
           const int col = jj * kBlock + NC * h + lane;
@@ -973,6 +1032,11 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
         load_cols32(tmem + lane_base + tDP + NC * h, dp);
         tc_fence_before();
         mbar_arrive_warp(bar(bDPFree));
+        if (kDropout) {
+          const float ks = a.drop.keep_scale;
+#pragma unroll
+          for (int c = 0; c < NC; ++c) dp[c] = ((keep >> c) & 1u) ? dp[c] * ks : 0.f;
+        }
         uint32_t w[NC / 2];
 #pragma unroll
         for (int e = 0; e < NC / 2; ++e)

@@ -31,6 +31,7 @@
 
 #include <cuda_bf16.h>
 
+#include "rng.cuh"
 #include "sm100.cuh"
 #include "tiles.cuh"
 
@@ -54,6 +55,7 @@ struct FwdArgs {
   int H;              // heads per batch entry (batch entry of bh = bh / H)
   const uint8_t* kpad;       // (B, N) key-padding flags (nonzero = padded key), or null
   __nv_bfloat16* o_low;      // (B, H, N, d) bf16 residual O - bf16(O), or null
+  DropoutArgs drop;          // kFeatDropout kernels
 };
 
 template <int D>
@@ -163,12 +165,20 @@ __device__ __forceinline__ FwdRange fwd_range(const FwdItem& it, int s) {
   return r;
 }
 
-// kAlibi: add the linear bias -m_h |i - j| (m_h = alibi[bh % H]) to every scaled score.
-template <int D, bool kAlibi = false>
+// kFeat: kFeatAlibi adds the linear bias -m_h |i - j| (m_h = alibi[bh % H]) to every
+// scaled score; kFeatKpad masks the keys a.kpad flags; kFeatResidual also writes
+// O - bf16(O) to a.o_low; kFeatDropout zeroes the weights whose Philox keep flag is
+// clear before the P V product (the row sum l keeps them: dropout follows the softmax)
+// and scales O by 1 / (1 - p').
+template <int D, int kFeat = 0>
 __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
   using C = FwdCfg<D>;
+  constexpr bool kAlibi = (kFeat & kFeatAlibi) != 0;
+  constexpr bool kKpad = (kFeat & kFeatKpad) != 0;
+  constexpr bool kResidual = (kFeat & kFeatResidual) != 0;
+  constexpr bool kDropout = (kFeat & kFeatDropout) != 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -433,6 +443,17 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
           pass_turn();
           continue;
         }
+        // keep flags of this row's 128 weights (they depend on no score, so they are drawn
+        // before S is ready): bit c of keep[g] for key 32g + c of the tile
+        uint32_t keep[4] = {~0u, ~0u, ~0u, ~0u};
+        if (kDropout) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const uint32_t blk = (uint32_t)(8 * j + 2 * g);
+            keep[g] = keep_bits16(a.drop, blk, (uint32_t)row, (uint32_t)it.bh) |
+                      (keep_bits16(a.drop, blk + 1, (uint32_t)row, (uint32_t)it.bh) << 16);
+          }
+        }
         if (!mbar_wait_warp(bar(C::bSFull + s), ns & 1, abort_flag)) {
           ok = false;
           break;
@@ -480,7 +501,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
 #pragma unroll
           for (int c = 0; c < kBlock; ++c) x[c] = (c >= c_lo && c <= c_hi) ? x[c] : -INFINITY;
         }
-        if (a.kpad != nullptr) {
+        if (kKpad) {
           // padded keys of this tile: lane l reads the flag of key 32g + l, one ballot per
           // 32 keys; the same 128 bits for every row
           uint32_t pm[4];
@@ -545,9 +566,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const float p0 = ex2(fmaf(x[32 * h + 2 * c], xs, -mb));
-            const float p1 = ex2(fmaf(x[32 * h + 2 * c + 1], xs, -mb));
+            float p0 = ex2(fmaf(x[32 * h + 2 * c], xs, -mb));
+            float p1 = ex2(fmaf(x[32 * h + 2 * c + 1], xs, -mb));
             ls[c & 3] += p0 + p1;
+            if (kDropout) {
+              p0 = ((keep[h] >> (2 * c)) & 1u) ? p0 : 0.f;
+              p1 = ((keep[h] >> (2 * c + 1)) & 1u) ? p1 : 0.f;
+            }
             pk[c] = pack_bf16x2(p0, p1);
           }
           tmem_st16(tP + 16 * h, pk);
@@ -579,7 +604,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         break;
       }
       tc_fence_after();
-      const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+      float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+      if (kDropout) inv_l *= a.drop.keep_scale;
       __nv_bfloat16* orow = a.o + ((size_t)it.bh * a.N + (row < a.N ? row : 0)) * D;
 #pragma unroll
       for (int q = 0; q < D / 32; ++q) {
@@ -597,7 +623,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
             st_global_v4(orow + 32 * q + 8 * v4, w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2],
                          w[4 * v4 + 3]);
         }
-        if (a.o_low != nullptr) {
+        if (kResidual) {
           // what rounding to bf16 left out: O - bf16(O), itself rounded to bf16, so that
           // the backward can form rowsum(dO o O) from O to about 16 significant bits
 #pragma unroll

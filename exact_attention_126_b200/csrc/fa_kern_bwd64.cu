@@ -1,0 +1,17 @@
+// fa_kern_bwd64.cu - the backward kernels for head_dim 64 (delta preprocess, dK/dV pass,
+// dQ pass) in every feature combination.
+#include "launch_impl.cuh"
+
+namespace fa_host {
+
+// the 8 combinations of kFeatAlibi, kFeatKpad, kFeatDropout (bit kFeatResidual unset)
+FA_INSTANTIATE_BWD(64, 0) FA_INSTANTIATE_BWD(64, 1) FA_INSTANTIATE_BWD(64, 2)
+FA_INSTANTIATE_BWD(64, 3) FA_INSTANTIATE_BWD(64, 8) FA_INSTANTIATE_BWD(64, 9)
+FA_INSTANTIATE_BWD(64, 10) FA_INSTANTIATE_BWD(64, 11)
+template fa_status_t launch_preprocess<64>(const void*, const void*, const void*, const float*,
+                                           float*, float*, int, int, cudaStream_t);
+template fa_status_t launch_dq_convert<64>(const float*, void*, int, int, float, cudaStream_t);
+
+int take_status_bwd64() { return take_unit_status(); }
+
+}  // namespace fa_host

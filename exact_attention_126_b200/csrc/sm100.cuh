@@ -13,9 +13,11 @@
 namespace fa {
 
 // ----------------------------------------------------------------------------------
-// Status word written by a kernel that abandons a bounded wait (read by fa_debug_status)
+// Status word written by a kernel that abandons a bounded wait (read by fa_debug_status).
+// Internal linkage: every compilation unit that holds kernels has its own copy, which that
+// unit's host code reads and clears.
 // ----------------------------------------------------------------------------------
-__device__ int g_fa_status;
+static __device__ int g_fa_status;
 
 constexpr int kStatusTimeout = 6;                         // FA_ERR_TIMEOUT
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
@@ -144,6 +146,18 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t sr
   asm volatile(
       "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
           reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// Adds the 3-D box at coordinates (c0, c1, c2) from shared memory `src` (laid out as a
+// load of the same box would leave it) into the tensor in global memory, element by
+// element (fp32 add, performed at L2). Tracked by the issuing thread's bulk async-groups.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, uint32_t src, int c0,
+                                                  int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
       "r"(src), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }

@@ -11,6 +11,13 @@
 namespace fa {
 
 constexpr int kBlock = 128;  // rows of a tile; the M (and N) extent of every MMA
+
+// Optional parts of the computation, compiled in as template flags so that a kernel
+// without them carries no trace of them (one bit each, combined into `kFeat`).
+constexpr int kFeatAlibi = 1;     // linear bias -m_h |i - j| on the scaled scores
+constexpr int kFeatKpad = 2;      // (B, N) key-padding flags
+constexpr int kFeatResidual = 4;  // forward also writes O - bf16(O)
+constexpr int kFeatDropout = 8;   // attention weights dropped with Philox keep flags
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Mask {

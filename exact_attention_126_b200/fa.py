@@ -25,8 +25,11 @@ STATUS_NAMES = {
 #: every symbol include/fa.h declares
 EXPORTED = ("fa_fwd", "fa_fwd_ex", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_ex",
             "fa_fwd_alibi", "fa_bwd_alibi", "fa_bwd_preprocess", "fa_bwd_dkdv", "fa_bwd_dq",
-            "fa_bwd_noalloc", "fa_status_string", "fa_debug_status", "fa_debug_set_fault",
-            "fa_version")
+            "fa_bwd_fused", "fa_bwd_dq_convert", "fa_bwd_noalloc", "fa_status_string",
+            "fa_debug_status", "fa_debug_set_fault", "fa_version")
+
+#: fa_options_t.flags: the backward with a separate, deterministic dQ pass
+FA_BWD_DETERMINISTIC = 1
 
 
 class FAError(RuntimeError):
@@ -44,12 +47,17 @@ class fa_options_t(ctypes.Structure):
     """Optional inputs and outputs of the _ex entry points (include/fa.h)."""
     _fields_ = [("alibi_slopes", ctypes.c_void_p), ("key_padding", ctypes.c_void_p),
                 ("o_low", ctypes.c_void_p), ("dropout_p", ctypes.c_float),
-                ("dropout_seed", ctypes.c_ulonglong), ("dropout_offset", ctypes.c_ulonglong)]
+                ("flags", ctypes.c_uint), ("dropout_seed", ctypes.c_ulonglong),
+                ("dropout_offset", ctypes.c_ulonglong)]
 
 
-def options(alibi_slopes=None, key_padding=None, o_low=None):
-    """An fa_options_t holding the device pointers of the given tensors (None = absent)."""
-    return fa_options_t(_ptr(alibi_slopes), _ptr(key_padding), _ptr(o_low), 0.0, 0, 0)
+def options(alibi_slopes=None, key_padding=None, o_low=None, dropout_p=0.0, dropout_seed=0,
+            dropout_offset=0, deterministic=False):
+    """An fa_options_t holding the device pointers of the given tensors (None = absent), the
+    dropout parameters (probability, 64-bit seed, 32-bit offset) and the backward's flags."""
+    return fa_options_t(_ptr(alibi_slopes), _ptr(key_padding), _ptr(o_low), float(dropout_p),
+                        FA_BWD_DETERMINISTIC if deterministic else 0,
+                        int(dropout_seed) & 0xFFFFFFFFFFFFFFFF, int(dropout_offset))
 
 
 _LIB = None
@@ -80,6 +88,8 @@ def _lib() -> ctypes.CDLL:
         lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, vp, I, I, I, I, OP, vp]
         lib.fa_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, OP, vp]
         lib.fa_bwd_dq.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, OP, vp]
+        lib.fa_bwd_fused.argtypes = [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, OP, vp]
+        lib.fa_bwd_dq_convert.argtypes = [vp, vp, I, I, I, I, F, vp]
         lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W,
                                        vp]
         lib.fa_status_string.argtypes = [I]
@@ -88,7 +98,7 @@ def _lib() -> ctypes.CDLL:
         lib.fa_debug_set_fault.argtypes = [I]
         lib.fa_version.argtypes = []
         for name in ("fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_ex", "fa_fwd_alibi",
-                     "fa_bwd_alibi", "fa_bwd_preprocess",
+                     "fa_bwd_alibi", "fa_bwd_preprocess", "fa_bwd_fused", "fa_bwd_dq_convert",
                      "fa_bwd_dkdv", "fa_bwd_dq", "fa_bwd_noalloc", "fa_debug_status",
                      "fa_debug_set_fault", "fa_version"):
             getattr(lib, name).restype = I
@@ -222,6 +232,23 @@ def fa_bwd_dkdv(q, k, v, do, workspace, dk, dv, scale=None, causal=False, window
            "fa_bwd_dkdv")
 
 
+def fa_bwd_fused(q, k, v, do, workspace, dk, dv, scale=None, causal=False, window=(-1, -1),
+                 stream=None, opt=None) -> None:
+    B, H, N, d = _shape(q)
+    c, w = _window(causal, window)
+    s = default_scale(d) if scale is None else float(scale)
+    _check(_lib().fa_bwd_fused(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(workspace), _ptr(dk),
+                               _ptr(dv), B, H, N, d, s, c, w, _opt_ref(opt), _stream(stream)),
+           "fa_bwd_fused")
+
+
+def fa_bwd_dq_convert(workspace, dq, scale=None, stream=None) -> None:
+    B, H, N, d = _shape(dq)
+    s = default_scale(d) if scale is None else float(scale)
+    _check(_lib().fa_bwd_dq_convert(_ptr(workspace), _ptr(dq), B, H, N, d, s, _stream(stream)),
+           "fa_bwd_dq_convert")
+
+
 def fa_bwd_dq(q, k, v, do, workspace, dq, scale=None, causal=False, window=(-1, -1),
               stream=None, opt=None) -> None:
     B, H, N, d = _shape(q)
@@ -289,13 +316,15 @@ def _check_padding(key_padding, q):
 
 
 def attention_forward(q, k, v, scale=None, causal=False, window=(-1, -1), stream=None,
-                      alibi_slopes=None, key_padding=None, keep_residual=False):
+                      alibi_slopes=None, key_padding=None, keep_residual=False, dropout=None):
     """Returns (O, LSE) for bf16 CUDA tensors q, k, v of shape (B, H, N, d), or
     (O, LSE, O_low) with keep_residual: O_low = O_fp32 - bf16(O) in bf16, which
     attention_backward uses to form rowsum(dO o O) from O to about 16 bits.
     alibi_slopes (H fp32 values): the scores carry the bias -alibi_slopes[h] * |i - j|.
     key_padding ((B, N) bool or uint8, True = padded key): padded keys are masked out
-    for every head and query."""
+    for every head and query. dropout: (p, seed, offset) drops each attention weight with
+    probability p (rounded to a multiple of 1/256) after the softmax and scales the kept
+    ones by 1 / (1 - p); the backward needs the same triple."""
     _check_inputs(q, k, v)
     B, H, N, d = _shape(q)
     o = torch.empty_like(q)
@@ -305,18 +334,21 @@ def attention_forward(q, k, v, scale=None, causal=False, window=(-1, -1), stream
         _check_slopes(alibi_slopes, q)
     if key_padding is not None:
         _check_padding(key_padding, q)
-    if alibi_slopes is None and key_padding is None and o_low is None:
+    if alibi_slopes is None and key_padding is None and o_low is None and dropout is None:
         fa_fwd(q, k, v, o, lse, scale, causal, window, stream)
     else:
-        opt = options(alibi_slopes, key_padding, o_low)
+        opt = options(alibi_slopes, key_padding, o_low, *(dropout or ()))
         fa_fwd_ex(q, k, v, o, lse, opt, scale, causal, window, stream)
     return (o, lse, o_low) if keep_residual else (o, lse)
 
 
 def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, window=(-1, -1),
-                       stream=None, alibi_slopes=None, key_padding=None, o_low=None):
+                       stream=None, alibi_slopes=None, key_padding=None, o_low=None,
+                       dropout=None, deterministic=False):
     """Returns (dQ, dK, dV): the gradient of <O, dO>; lse (and o_low, if kept) come from
-    attention_forward with the same alibi_slopes and key_padding."""
+    attention_forward with the same alibi_slopes, key_padding and dropout. deterministic:
+    the backward with a separate dQ pass (bit-identical results run to run); otherwise
+    head_dim 64 adds dQ up in fp32 in no fixed order."""
     _check_inputs(q, k, v, o, do)
     B, H, N, d = _shape(q)
     dq = torch.empty_like(q)
@@ -330,9 +362,11 @@ def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, window=(-1
         _check_padding(key_padding, q)
     if o_low is not None:
         _check_inputs(q, o_low)
-    if alibi_slopes is None and key_padding is None and o_low is None:
+    if (alibi_slopes is None and key_padding is None and o_low is None and dropout is None
+            and not deterministic):
         fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, scale, causal, window, stream)
     else:
-        opt = options(alibi_slopes, key_padding, o_low)
+        opt = options(alibi_slopes, key_padding, o_low, *(dropout or ()),
+                      **({"deterministic": True} if deterministic else {}))
         fa_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, ws, opt, scale, causal, window, stream)
     return dq, dk, dv

@@ -81,10 +81,11 @@ typedef struct {
  *   alibi_slopes  H fp32 slopes, device memory, 4-byte aligned, or NULL: the ALiBi bias
  *                 (see fa_fwd_alibi).
  *   key_padding   (B, N) bytes, device memory, any alignment, or NULL: nonzero marks key
- *                 n of batch entry b as padding. Page "PyTorch-CUDA-v2.9镜像中使用
- *                 FlashAttention提升训练速度" passes such a `key_padding_mask` (True = padded)
- *                 and applies it with masked_fill(-inf) to every head and query: a padded
- *                 key's score is -inf before the softmax. A query left with no visible,
+ *                 n of batch entry b as padding. The attention layer of page "PyTorch-
+ *                 CUDA-v2.9镜像中使用FlashAttention提升训练速度" takes such a `key_padding_mask`
+ *                 (True = padded), and the reference layer of page "Flash Attention 3.7 核心
+ *                 原理与实战" §4.2 applies it with masked_fill(-inf) to every head and query:
+ *                 a padded key's score is -inf before the softmax. A query left with no visible,
  *                 unpadded key gets O = 0, LSE = -inf and no gradient (the backward must
  *                 get the same flags as the forward).
  *   o_low         bf16 (B, H, N, d), device memory, 16-byte aligned, or NULL. The forward
@@ -96,8 +97,19 @@ typedef struct {
  *                 by several percent. Costs one more bf16 tensor written by the forward and
  *                 read by the backward.
  *   dropout_p, dropout_seed, dropout_offset
- *                 reserved: dropout_p must be 0 (else FA_ERR_UNSUPPORTED); the seed and
- *                 offset are ignored.
+ *                 dropout on the attention weights (`dropout_p` of flash_attn_fn, page
+ *                 "告别OOM和训练慢…" §4.2; the reference layer of page "Flash Attention 3.7
+ *                 核心原理与实战" §4.2 applies it to the softmax weights before the product with
+ *                 V): O = (P o Z / (1 - p')) V, LSE unchanged. The keep flags Z are drawn from
+ *                 Philox4x32-10 (Salmon et al., SC 2011) under key dropout_seed (low, high
+ *                 32 bits) at counter (key / 16, query, b*H + h, dropout_offset): key j uses
+ *                 byte j mod 4 of output word (j mod 16) / 4 and is dropped iff that byte is
+ *                 below t = floor(256 p + 1/2); p' = t / 256 (p rounded to a multiple of
+ *                 1/256). dropout_p must be in [0, 1) with t <= 255, and dropout_offset below
+ *                 2^32 (else FA_ERR_INVALID_ARG); t = 0 is no dropout. The backward must get
+ *                 the same three values; it regenerates the flags instead of storing them.
+ *                 Use a new offset (or seed) per call to draw new flags.
+ *   flags         FA_BWD_DETERMINISTIC or 0 (see below).
  * The layout is that of a C struct with natural alignment (48 bytes on LP64).
  */
 typedef struct {
@@ -105,9 +117,21 @@ typedef struct {
     const unsigned char *key_padding;
     void *o_low;
     float dropout_p;
+    unsigned int flags;                 /* FA_BWD_* bits below; 0 = none */
     unsigned long long dropout_seed;
     unsigned long long dropout_offset;
 } fa_options_t;
+
+/*
+ * flags: FA_BWD_DETERMINISTIC selects the backward whose dQ comes from a separate pass per
+ * query tile (fa_bwd_dkdv, then fa_bwd_dq): bit-identical results from run to run. Without
+ * it, head_dim 64 uses the fused pass (fa_bwd_fused), which adds each (query tile, key
+ * tile) share of dQ into an fp32 accumulator with L2 reductions in no fixed order, so dQ is
+ * reproducible to fp32 rounding only (dK and dV are still bit-identical); it does about 2/7
+ * less tensor work. head_dim 128 always uses the separate pass. Other bits give
+ * FA_ERR_INVALID_ARG.
+ */
+#define FA_BWD_DETERMINISTIC 1u
 
 /*
  * Forward pass.
@@ -125,7 +149,7 @@ fa_status_t fa_fwd(const void *q, const void *k, const void *v, void *o, float *
 
 /*
  * fa_fwd with the optional inputs and outputs of `options` (may be NULL). Misaligned
- * slopes or o_low give FA_ERR_MISALIGNED; a nonzero dropout_p gives FA_ERR_UNSUPPORTED.
+ * slopes or o_low give FA_ERR_MISALIGNED; dropout values out of range FA_ERR_INVALID_ARG.
  */
 fa_status_t fa_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse,
                       int B, int H, int N, int d, float scale, int causal,
@@ -134,8 +158,9 @@ fa_status_t fa_fwd_ex(const void *q, const void *k, const void *v, void *o, floa
 /*
  * Bytes of device workspace fa_bwd() needs: two fp32 arrays of B*H*Np values, where
  * Np = N rounded up to a multiple of 128 (the row statistics of the backward, see
- * fa_bwd_preprocess), rounded up to 256 bytes. Returns 0 for an empty problem or
- * invalid sizes.
+ * fa_bwd_preprocess), rounded up to 256 bytes; for head_dim 64, followed by the fused
+ * pass's fp32 dQ accumulator of B*H*Np*64 values. (With FA_BWD_DETERMINISTIC the first
+ * part alone is enough.) Returns 0 for an empty problem or invalid sizes.
  */
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 
@@ -153,7 +178,9 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
  *   P = exp(scale Q K^T - LSE), dP = dO V^T, dS = P o (dP - delta),
  *   dV = P^T dO, dK = scale dS^T Q             (fa_bwd_dkdv, one pass per key tile)
  *   dQ = scale dS K                            (fa_bwd_dq, one pass per query tile)
- * The three kernels run in that order on the stream; results are deterministic.
+ * The kernels run in that order on the stream. At head_dim 64 the two passes are fused
+ * into one over key tiles that also adds dQ into an fp32 accumulator, converted to bf16 by
+ * a last kernel (see FA_BWD_DETERMINISTIC for what that changes).
  */
 fa_status_t fa_bwd(const void *q, const void *k, const void *v, const void *o,
                    const void *dout, const float *lse, void *dq, void *dk, void *dv,
@@ -162,8 +189,8 @@ fa_status_t fa_bwd(const void *q, const void *k, const void *v, const void *o,
                    void *stream);
 
 /*
- * fa_bwd with the optional inputs of `options` (may be NULL): the same alibi_slopes and
- * key_padding as the forward had, and o_low if the forward wrote it.
+ * fa_bwd with the optional inputs of `options` (may be NULL): the same alibi_slopes,
+ * key_padding and dropout values as the forward had, and o_low if the forward wrote it.
  */
 fa_status_t fa_bwd_ex(const void *q, const void *k, const void *v, const void *o,
                       const void *dout, const float *lse, void *dq, void *dk, void *dv,
@@ -199,25 +226,42 @@ fa_status_t fa_bwd_alibi(const void *q, const void *k, const void *v, const void
  *   workspace[B*H*Np .. 2*B*H*Np)   delta = rowsum(dout * o), summed in fp32
  *                                   (o + options->o_low when o_low is given)
  * The padding lets each 128-row tile of both arrays be fetched with one bulk copy.
- * `options` may be NULL; only its o_low is used here.
+ * At head_dim 64 without FA_BWD_DETERMINISTIC it also zeroes the fused pass's dQ
+ * accumulator (the workspace must then hold fa_bwd_workspace_bytes()).
+ * `options` may be NULL; its o_low and flags are used here.
  */
 fa_status_t fa_bwd_preprocess(const void *o, const void *dout, const float *lse,
                               void *workspace, int B, int H, int N, int d,
                               const fa_options_t *options, void *stream);
 
 /* Step 2 of fa_bwd alone: dk, dv from q, k, v, dout and the workspace of step 1
- * (`options`: alibi_slopes and key_padding, or NULL). */
+ * (`options`: alibi_slopes, key_padding and dropout, or NULL). */
 fa_status_t fa_bwd_dkdv(const void *q, const void *k, const void *v, const void *dout,
                         const void *workspace, void *dk, void *dv,
                         int B, int H, int N, int d, float scale, int causal,
                         fa_window_t window, const fa_options_t *options, void *stream);
 
 /* Step 3 of fa_bwd alone: dq from q, k, v, dout and the workspace of step 1
- * (`options`: alibi_slopes and key_padding, or NULL). */
+ * (`options`: alibi_slopes, key_padding and dropout, or NULL). */
 fa_status_t fa_bwd_dq(const void *q, const void *k, const void *v, const void *dout,
                       const void *workspace, void *dq,
                       int B, int H, int N, int d, float scale, int causal,
                       fa_window_t window, const fa_options_t *options, void *stream);
+
+/*
+ * Step 2 of the fused backward alone (head_dim 64, else FA_ERR_UNSUPPORTED): dk, dv, and
+ * dQ / scale added into the accumulator part of `workspace` (which fa_bwd_preprocess,
+ * called without FA_BWD_DETERMINISTIC, zeroed). `options`: alibi_slopes, key_padding and
+ * dropout, or NULL.
+ */
+fa_status_t fa_bwd_fused(const void *q, const void *k, const void *v, const void *dout,
+                         void *workspace, void *dk, void *dv,
+                         int B, int H, int N, int d, float scale, int causal,
+                         fa_window_t window, const fa_options_t *options, void *stream);
+
+/* Step 3 of the fused backward alone: dq = bf16(scale * accumulator). */
+fa_status_t fa_bwd_dq_convert(void *workspace, void *dq, int B, int H, int N, int d,
+                              float scale, void *stream);
 
 /*
  * Backward pass for callers that cannot allocate device memory. (The pages have no
@@ -225,11 +269,11 @@ fa_status_t fa_bwd_dq(const void *q, const void *k, const void *v, const void *d
  *
  * Some callers may not allocate: an engine that reserves all of its device memory up
  * front and may not grow it while serving, or a framework plugin whose enqueue step
- * is not allowed to call cudaMalloc. fa_bwd_noalloc computes exactly what fa_bwd
- * computes, with the same arguments except the workspace: its row statistics go to a
- * fixed 8 MiB array in device memory that the library holds on every GPU that loads
- * it, until the process exits. It calls no cudaMalloc, cudaFree or other allocating
- * routine.
+ * is not allowed to call cudaMalloc. fa_bwd_noalloc computes exactly what fa_bwd with
+ * FA_BWD_DETERMINISTIC computes, with the same arguments except the workspace: its row
+ * statistics go to a fixed 8 MiB array in device memory that the library holds on every
+ * GPU that loads it, until the process exits. It calls no cudaMalloc, cudaFree or other
+ * allocating routine.
  *   Limit: 2 * B * H * Np * 4 bytes must fit in 8 MiB, i.e. B * H * Np <= 1,048,576
  *   with Np = N rounded up to a multiple of 128; larger problems return
  *   FA_ERR_WORKSPACE before anything is launched.

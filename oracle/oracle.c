@@ -17,9 +17,10 @@
  *   S_ij = -inf where key j is not visible from query i (causal: "mask future
  *          positions", page "Flash Attention 3.7 核心原理与实战" §3.2; sliding window
  *          `window_size=(left,right)`, page "告别OOM和训练慢…" §4.2), and where key j of
- *          the batch entry is padding (`key_padding_mask`, True = padded, applied with
- *          masked_fill(-inf) to every head and query: page "PyTorch-CUDA-v2.9镜像…", the
- *          MultiheadAttention replacement)
+ *          the batch entry is padding (`key_padding_mask`, True = padded: the attention
+ *          layer of page "PyTorch-CUDA-v2.9镜像…" accepts it, and the reference layer of page
+ *          "Flash Attention 3.7 核心原理与实战" §4.2 applies it with masked_fill(-inf),
+ *          broadcast over every head and query)
  *   P = row-softmax(S), with the row maximum subtracted first (`safe_softmax`,
  *       page "告别OOM和训练慢…" §2.2)
  *   O = P V

@@ -17,9 +17,10 @@ Sources of the facts:
   * torch's fp64 CPU scaled_dot_product_attention and autograd, as an independent
     library implementation of the same definition.
 
-The key-padding pins (`key_padding_mask`, True = padded key, masked_fill(-inf) on every head
-and query: page "PyTorch-CUDA-v2.9镜像中使用FlashAttention提升训练速度", the MultiheadAttention
-replacement) use: no flags set is no mask at all; padded keys' K and V rows do not matter and
+The key-padding pins (`key_padding_mask`, True = padded key: accepted by the attention layer
+of page "PyTorch-CUDA-v2.9镜像中使用FlashAttention提升训练速度", applied with masked_fill(-inf) on
+every head and query by the reference layer of page "Flash Attention 3.7 核心原理与实战" §4.2)
+use: no flags set is no mask at all; padded keys' K and V rows do not matter and
 get zero gradients; a single unpadded key is returned exactly; a fully padded batch entry
 gives O = 0, LSE = -inf and zero gradients; finite differences; torch's SDPA with the combined
 boolean mask.

@@ -34,6 +34,19 @@ def test_every_declared_symbol_is_exported(lib):
         assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
 
 
+def test_only_the_declared_entry_points_are_exported(lib):
+    import shutil
+    import subprocess
+    nm = shutil.which("nm")
+    if nm is None:
+        pytest.skip("nm is not available")
+    out = subprocess.run([nm, "-D", "--defined-only", fa.LIBRARY], capture_output=True,
+                         text=True, check=True).stdout
+    names = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    names = {n for n in names if not n.startswith(("_init", "_fini"))}
+    assert names == set(declared_functions()), sorted(names ^ set(declared_functions()))
+
+
 def test_status_strings(lib):
     for code, name in fa.STATUS_NAMES.items():
         assert fa.fa_status_string(code).startswith(name)
@@ -66,7 +79,7 @@ def test_fwd_rejects_bad_arguments(lib):
     assert fwd(lib, window=(5, -3)) == 1
     assert fwd(lib, B=1 << 12, H=1 << 12, N=256, d=64) == 2  # >= 2^31 elements
     # more than 65535 (batch, head) pairs is accepted (no grid dimension is limited by it)
-    assert lib.fa_bwd_workspace_bytes(1 << 17, 1, 128, 64) == 2 * (1 << 17) * 128 * 4
+    assert lib.fa_bwd_workspace_bytes(1 << 17, 1, 64, 128) == 2 * (1 << 17) * 128 * 4
 
 
 def test_empty_problem_is_a_no_op(lib):
@@ -78,9 +91,10 @@ def test_empty_problem_is_a_no_op(lib):
 
 
 def test_workspace_size(lib):
-    # two fp32 arrays (LSE*log2e and delta) of B*H rows padded to whole 128-row tiles
-    assert lib.fa_bwd_workspace_bytes(2, 8, 4096, 64) == 2 * 2 * 8 * 4096 * 4
-    assert lib.fa_bwd_workspace_bytes(1, 1, 3, 64) == 2 * 128 * 4
+    # two fp32 arrays (LSE*log2e and delta) of B*H rows padded to whole 128-row tiles; at
+    # head_dim 64 followed by the fused pass's fp32 dQ accumulator (64 values per row)
+    assert lib.fa_bwd_workspace_bytes(2, 8, 4096, 64) == 2 * 2 * 8 * 4096 * 4 * (1 + 32)
+    assert lib.fa_bwd_workspace_bytes(1, 1, 3, 64) == 2 * 128 * 4 + 128 * 64 * 4
     assert lib.fa_bwd_workspace_bytes(1, 2, 129, 128) == 2 * 2 * 256 * 4
     assert lib.fa_bwd_workspace_bytes(1, 1, 3, 80) == 0
 
@@ -118,18 +132,32 @@ def test_options_are_checked(lib):
         return lib.fa_bwd_ex(A, A, A, A, A, A, A, A, A, 1, 2, 128, 64, 0.125, 0, W(-1, -1), opt,
                              A, ws_bytes, None)
 
-    O = fa.fa_options_t
-    assert fwd_ex(O(A + 2, None, None, 0.0, 0, 0)) == 3   # slopes not 4-byte aligned
-    assert fwd_ex(O(None, None, A + 8, 0.0, 0, 0)) == 3   # o_low not 16-byte aligned
-    assert fwd_ex(O(None, None, None, 0.1, 0, 0)) == 2    # dropout is not offered
-    assert fwd_ex(O(None, A + 1, None, 0.0, 0, 0), q=None) == 1
+    def O(**kw):
+        return fa.fa_options_t(**kw)
+
+    assert fwd_ex(O(alibi_slopes=A + 2)) == 3       # slopes not 4-byte aligned
+    assert fwd_ex(O(o_low=A + 8)) == 3              # o_low not 16-byte aligned
+    assert fwd_ex(O(dropout_p=1.0)) == 1            # dropout probability >= 1
+    assert fwd_ex(O(dropout_p=-0.1)) == 1           # negative probability
+    assert fwd_ex(O(dropout_p=0.999)) == 1          # rounds to 256/256: nothing kept
+    assert fwd_ex(O(dropout_p=float("nan"))) == 1
+    assert fwd_ex(O(dropout_p=0.1, dropout_offset=1 << 32)) == 1  # offset wider than 32 bits
+    assert fwd_ex(O(flags=2)) == 1                  # unknown flag
+    assert fwd_ex(O(key_padding=A + 1), q=None) == 1
     assert fwd_ex(None, d=96) == 2
-    assert bwd_ex(O(None, None, A + 4, 0.0, 0, 0)) == 3
-    assert bwd_ex(O(None, None, None, 0.5, 0, 0)) == 2
+    assert bwd_ex(O(o_low=A + 4)) == 3
+    assert bwd_ex(O(dropout_p=1.5)) == 1
     assert bwd_ex(None, ws_bytes=8) == 4
+    # the fused backward (head_dim 64) needs the dQ accumulator; the deterministic one not
+    stats = 2 * 2 * 128 * 4
+    assert bwd_ex(None, ws_bytes=stats) == 4
+    assert lib.fa_bwd_fused(A, A, A, A, A, A, A, 1, 1, 128, 128, 0.1, 0, W(-1, -1), None,
+                            None) == 2   # the fused pass is for head_dim 64
+    assert lib.fa_bwd_dq_convert(A, None, 1, 1, 128, 64, 0.1, None) == 1
+    assert lib.fa_bwd_dq_convert(A, A, 1, 1, 128, 128, 0.1, None) == 2
     # empty problems launch nothing, whatever the options
     assert lib.fa_fwd_ex(None, None, None, None, None, 1, 2, 0, 64, 0.125, 0, W(-1, -1),
-                         O(A + 2, None, None, 0.5, 0, 0), None) == 0
+                         O(alibi_slopes=A + 2, dropout_p=0.5), None) == 0
 
 
 def test_options_struct_layout():
@@ -137,7 +165,8 @@ def test_options_struct_layout():
     O = fa.fa_options_t
     assert ctypes.sizeof(O) == 48
     assert [O.alibi_slopes.offset, O.key_padding.offset, O.o_low.offset, O.dropout_p.offset,
-            O.dropout_seed.offset, O.dropout_offset.offset] == [0, 8, 16, 24, 32, 40]
+            O.flags.offset, O.dropout_seed.offset, O.dropout_offset.offset] == [
+                0, 8, 16, 24, 28, 32, 40]
 
 
 def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -1,6 +1,7 @@
 """Key padding (fa_options_t.key_padding) against the fp64 oracle with the same flags: the
-`key_padding_mask` of page "PyTorch-CUDA-v2.9镜像中使用FlashAttention提升训练速度" (True = padded
-key, masked_fill(-inf) on every head and query), forward and backward, on suffix padding
+`key_padding_mask` (True = padded key) of page "PyTorch-CUDA-v2.9镜像中使用FlashAttention提升训练
+速度", applied with masked_fill(-inf) on every head and query as in the reference layer of page
+"Flash Attention 3.7 核心原理与实战" §4.2, forward and backward, on suffix padding
 of different lengths per batch entry (one entry fully padded), random flags, whole padded
 key tiles in the middle of a sequence, every mask mode, both head sizes, with ALiBi, and
 with many work items per persistent CTA."""

@@ -204,13 +204,47 @@ def test_zero_queries_closed_form():
 
 
 def test_deterministic():
-    """Two runs give bit-identical O, LSE, dQ, dK and dV (no atomics anywhere)."""
+    """With FA_BWD_DETERMINISTIC, two runs give bit-identical O, LSE, dQ, dK and dV (no
+    atomics anywhere on that path)."""
+    w = WORKLOADS["c3"]
+    inp = inputs(w.B, w.H, w.N, w.d, w.seed_index)
+    a = G.run_library(inp, w.softmax_scale, True, (-1, -1), deterministic=True)
+    b = G.run_library(inp, w.softmax_scale, True, (-1, -1), deterministic=True)
+    for n in a:
+        assert torch.equal(a[n], b[n]), n
+
+
+def test_fused_backward_run_to_run():
+    """The fused backward (head_dim 64): O, LSE, dK and dV are bit-identical from run to run;
+    dQ, added up in fp32 in no fixed order, differs by fp32 rounding only (far below bf16's
+    resolution), and both runs agree with the deterministic backward within the bounds."""
     w = WORKLOADS["c3"]
     inp = inputs(w.B, w.H, w.N, w.d, w.seed_index)
     a = G.run_library(inp, w.softmax_scale, True, (-1, -1))
     b = G.run_library(inp, w.softmax_scale, True, (-1, -1))
-    for n in a:
+    c = G.run_library(inp, w.softmax_scale, True, (-1, -1), deterministic=True)
+    for n in ("o", "lse", "dk", "dv"):
         assert torch.equal(a[n], b[n]), n
+    spread = G.rel_frob(synth.to_f64(a["dq"]), synth.to_f64(b["dq"]))
+    to_det = G.rel_frob(synth.to_f64(a["dq"]), synth.to_f64(c["dq"]))
+    print("fused dQ run-to-run relative spread %.3g, vs deterministic %.3g" % (spread, to_det))
+    assert spread <= 1e-3 and to_det <= 2e-3
+    errs = G.compare(inp, a, w.softmax_scale, True, (-1, -1))
+    G.assert_within_bounds(errs, "fused")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("mode", ["none", "causal", "win100_30"])
+def test_deterministic_path_small_and_ragged(d, mode):
+    """The three-kernel backward (separate dQ pass) against the oracle at head_dim 64, where
+    the default is the fused pass (and at 128, where both are the same path)."""
+    causal, window = MODES[mode]
+    for N in (17, 300):
+        inp = inputs(2, 2, N, d, 150 + N + d)
+        scale = 1.0 / np.sqrt(d)
+        out = G.run_library(inp, scale, causal, window, deterministic=True)
+        errs = G.compare(inp, out, scale, causal, window)
+        G.assert_within_bounds(errs, (N, d, mode))
 
 
 @pytest.mark.parametrize("d", [64, 128])
