@@ -49,13 +49,14 @@ class Oracle:
         self.lib = ctypes.CDLL(path)
         L = ctypes.c_long
         D, U64 = ctypes.c_double, ctypes.c_ulonglong
+        lp = ctypes.POINTER(ctypes.c_long)
         self.lib.oracle_attention_fwd.argtypes = [
-            _dptr, _dptr, _dptr, L, L, L, L, D, ctypes.c_int, L, L, _dptr, _bptr, D, U64, U64,
-            _dptr, _dptr]
+            _dptr, _dptr, _dptr, L, L, L, L, D, ctypes.c_int, L, L, _dptr, _bptr, lp, D, U64,
+            U64, _dptr, _dptr]
         self.lib.oracle_attention_fwd.restype = ctypes.c_int
         self.lib.oracle_attention_bwd.argtypes = [
-            _dptr, _dptr, _dptr, _dptr, L, L, L, L, D, ctypes.c_int, L, L, _dptr, _bptr, D, U64,
-            U64, _dptr, _dptr, _dptr]
+            _dptr, _dptr, _dptr, _dptr, L, L, L, L, D, ctypes.c_int, L, L, _dptr, _bptr, lp, D,
+            U64, U64, _dptr, _dptr, _dptr]
         self.lib.oracle_attention_bwd.restype = ctypes.c_int
         u32p = ctypes.POINTER(ctypes.c_uint32)
         self.lib.oracle_philox4x32_10.argtypes = [u32p, u32p, u32p]
@@ -94,6 +95,15 @@ class Oracle:
         return a, a.ctypes.data_as(_bptr)
 
     @staticmethod
+    def _lengths(lengths, B, N):
+        if lengths is None:
+            return None, None
+        a = np.ascontiguousarray(lengths, dtype=np.int64).reshape(-1)
+        if a.shape != (B,) or np.any(a < 0) or np.any(a > N):
+            raise ValueError("lengths must hold one length in [0, N] per batch entry")
+        return a, a.ctypes.data_as(ctypes.POINTER(ctypes.c_long))
+
+    @staticmethod
     def _dropout(dropout):
         if dropout is None:
             return 0.0, 0, 0
@@ -118,10 +128,10 @@ class Oracle:
         return m
 
     def fwd(self, q, k, v, scale, causal=False, window=(-1, -1), alibi=None, key_padding=None,
-            dropout=None):
+            dropout=None, lengths=None):
         """Returns (O, LSE) in fp64 for (B, H, N, d) inputs; `alibi`: H slopes or None;
         `key_padding`: (B, N) flags, True for a padded key, or None; `dropout`:
-        (p, seed, offset) or None."""
+        (p, seed, offset) or None; `lengths`: B real lengths or None."""
         q, k, v = self._prep(q, k, v)
         B, H, N, d = q.shape
         o = np.empty_like(q)
@@ -129,16 +139,17 @@ class Oracle:
         keep, slopes = self._slopes(alibi, H)
         keep_pad, pad = self._padding(key_padding, B, N)
         dp, seed, offset = self._dropout(dropout)
+        keep_len, lens = self._lengths(lengths, B, N)
         rc = self.lib.oracle_attention_fwd(_as_ptr(q), _as_ptr(k), _as_ptr(v), B, H, N, d,
                                            float(scale), int(bool(causal)), int(window[0]),
-                                           int(window[1]), slopes, pad, dp, seed, offset,
+                                           int(window[1]), slopes, pad, lens, dp, seed, offset,
                                            _as_ptr(o), _as_ptr(lse))
         if rc != 0:
             raise RuntimeError("oracle_attention_fwd failed with %d" % rc)
         return o, lse
 
     def bwd(self, q, k, v, do, scale, causal=False, window=(-1, -1), alibi=None,
-            key_padding=None, dropout=None):
+            key_padding=None, dropout=None, lengths=None):
         """Returns (dQ, dK, dV) in fp64: the gradient of <O, dO> for (B, H, N, d) inputs."""
         q, k, v, do = self._prep(q, k, v, do)
         B, H, N, d = q.shape
@@ -148,10 +159,12 @@ class Oracle:
         keep, slopes = self._slopes(alibi, H)
         keep_pad, pad = self._padding(key_padding, B, N)
         dp, seed, offset = self._dropout(dropout)
+        keep_len, lens = self._lengths(lengths, B, N)
         rc = self.lib.oracle_attention_bwd(_as_ptr(q), _as_ptr(k), _as_ptr(v), _as_ptr(do),
                                            B, H, N, d, float(scale), int(bool(causal)),
-                                           int(window[0]), int(window[1]), slopes, pad, dp,
-                                           seed, offset, _as_ptr(dq), _as_ptr(dk), _as_ptr(dv))
+                                           int(window[0]), int(window[1]), slopes, pad, lens,
+                                           dp, seed, offset, _as_ptr(dq), _as_ptr(dk),
+                                           _as_ptr(dv))
         if rc != 0:
             raise RuntimeError("oracle_attention_bwd failed with %d" % rc)
         return dq, dk, dv

@@ -34,6 +34,12 @@
  *   dV = P^T dO;  dP = dO V^T;  D_i = sum_j P_ij dP_ij;  dS = P o (dP - D);
  *   dQ = scale * dS K;  dK = scale * dS^T Q.
  *
+ * Variable-length batches (`lengths`: each sample's real length, the dynamic batching of
+ * page "告别OOM和训练慢…" §6, which groups sequences by length to avoid computing on
+ * padding): batch entry b holds L_b real tokens; query i and key j of that entry interact
+ * only if i < L_b and j < L_b (on top of the mask). Rows i >= L_b see no key (O = 0,
+ * LSE = -inf, no gradient) and keys j >= L_b get none.
+ *
  * Dropout on the attention weights (`dropout_p` of `flash_attn_fn`, page "告别OOM和训练慢…"
  * §4.2; the reference layer of page "Flash Attention 3.7 核心原理与实战" §4.2 applies
  * F.dropout to the softmax weights and then multiplies by V): with keep flags Z_ij,
@@ -95,10 +101,10 @@ static double head_slope(const double *alibi_slopes, long bh, long H)
 
 /* P (N x N) := softmax rows of the masked, scaled (and biased, when slope != 0) scores of
  * one head; lse (N). kpad: N flags of the head's batch entry (nonzero = padded key), or
- * NULL. */
+ * NULL; len: the entry's real length (N when the batch is not variable-length). */
 static void head_probabilities(const double *q, const double *k, long N, long d,
                                double scale, double slope, long left, long right,
-                               const unsigned char *kpad, double *P, double *lse)
+                               const unsigned char *kpad, long len, double *P, double *lse)
 {
     long i;
 #pragma omp parallel for schedule(static)
@@ -113,6 +119,7 @@ static void head_probabilities(const double *q, const double *k, long N, long d,
             s += -slope * fabs((double)(i - j));
             if (!visible(i, j, left, right)) s = -INFINITY;
             if (kpad && kpad[j]) s = -INFINITY;
+            if (i >= len || j >= len) s = -INFINITY;
             Pi[j] = s;
             if (s > m) m = s;
         }
@@ -211,6 +218,12 @@ static void apply_dropout(double *P, long N, long bh, double dropout_p, unsigned
     }
 }
 
+/* The real length of head bh's batch entry: lengths[b], or N without lengths. */
+static long head_length(const long *lengths, long bh, long H, long N)
+{
+    return lengths ? lengths[bh / H] : N;
+}
+
 /* The key-padding flags of head bh's batch entry (B*H heads, heads fastest), or NULL. */
 static const unsigned char *head_padding(const unsigned char *key_padding, long bh, long H,
                                          long N)
@@ -219,12 +232,13 @@ static const unsigned char *head_padding(const unsigned char *key_padding, long 
 }
 
 /* alibi_slopes: H slopes, or NULL for no bias; key_padding: B x N flags (nonzero = padded
- * key), or NULL for none; dropout_p in [0, 1), 0 for none, with its seed and offset. */
+ * key), or NULL for none; lengths: B real lengths in [0, N], or NULL; dropout_p in [0, 1),
+ * 0 for none, with its seed and offset. */
 int oracle_attention_fwd(const double *q, const double *k, const double *v,
                          long B, long H, long N, long d, double scale,
                          int causal, long left, long right, const double *alibi_slopes,
-                         const unsigned char *key_padding, double dropout_p,
-                         unsigned long long seed, unsigned long long offset,
+                         const unsigned char *key_padding, const long *lengths,
+                         double dropout_p, unsigned long long seed, unsigned long long offset,
                          double *o, double *lse)
 {
     long bh;
@@ -238,7 +252,8 @@ int oracle_attention_fwd(const double *q, const double *k, const double *v,
         double *oh = o + bh * N * d;
         long i;
         head_probabilities(qh, kh, N, d, scale, head_slope(alibi_slopes, bh, H), left, right,
-                           head_padding(key_padding, bh, H, N), P, lse + bh * N);
+                           head_padding(key_padding, bh, H, N),
+                           head_length(lengths, bh, H, N), P, lse + bh * N);
         apply_dropout(P, N, bh, dropout_p, seed, offset);
         /* O = P V (P with dropout applied) */
 #pragma omp parallel for schedule(static)
@@ -259,8 +274,8 @@ int oracle_attention_bwd(const double *q, const double *k, const double *v,
                          const double *dout,
                          long B, long H, long N, long d, double scale,
                          int causal, long left, long right, const double *alibi_slopes,
-                         const unsigned char *key_padding, double dropout_p,
-                         unsigned long long seed, unsigned long long offset,
+                         const unsigned char *key_padding, const long *lengths,
+                         double dropout_p, unsigned long long seed, unsigned long long offset,
                          double *dq, double *dk, double *dv)
 {
     long bh;
@@ -285,7 +300,8 @@ int oracle_attention_bwd(const double *q, const double *k, const double *v,
         double *dqh = dq + bh * N * d, *dkh = dk + bh * N * d, *dvh = dv + bh * N * d;
         long i, j;
         head_probabilities(qh, kh, N, d, scale, head_slope(alibi_slopes, bh, H), left, right,
-                           head_padding(key_padding, bh, H, N), P, lse);
+                           head_padding(key_padding, bh, H, N),
+                           head_length(lengths, bh, H, N), P, lse);
         /* Pd = P o Z / (1 - p'): the weights that multiplied V (Pd = P without dropout) */
         memcpy(Pd, P, sizeof(double) * (size_t)N * (size_t)N);
         apply_dropout(Pd, N, bh, dropout_p, seed, offset);

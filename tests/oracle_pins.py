@@ -25,6 +25,11 @@ get zero gradients; a single unpadded key is returned exactly; a fully padded ba
 gives O = 0, LSE = -inf and zero gradients; finite differences; torch's SDPA with the combined
 boolean mask.
 
+The variable-length pins (`lengths`, each sample's real length: the dynamic batching of page
+"告别OOM和训练慢…" §6) use: full lengths are no restriction at all; an entry of length L is the
+problem truncated to its first L tokens, with zero outputs, -inf LSE and zero gradients past
+it; a zero-length entry is all zeros; finite differences.
+
 The dropout pins (`dropout_p` of page "告别OOM和训练慢…" §4.2; F.dropout on the softmax
 weights before the product with V in the reference layer of page "Flash Attention 3.7 核心原理
 与实战" §4.2) pin the generator by the known-answer vectors of Philox4x32-10 (Salmon, Moraes,
@@ -516,6 +521,82 @@ def pin_self_similarity(orc):
         assert np.all(lse >= 0.5 * np.sum(q * q, axis=-1) - 1e-12)
 
 
+def pin_lengths_full_is_identity(orc):
+    """lengths = N for every entry is no restriction: bit-identical results."""
+    r = _rng(41)
+    q, k, v, do = (r.standard_normal((2, 2, 13, 4)) for _ in range(4))
+    for causal, window in MODES[:4]:
+        a = orc.fwd(q, k, v, 0.5, causal, window)
+        b = orc.fwd(q, k, v, 0.5, causal, window, lengths=[13, 13])
+        ga = orc.bwd(q, k, v, do, 0.5, causal, window)
+        gb = orc.bwd(q, k, v, do, 0.5, causal, window, lengths=[13, 13])
+        for x, y in zip(a + ga, b + gb):
+            assert np.array_equal(x, y)
+
+
+def pin_lengths_truncated_problem(orc):
+    """An entry of real length L is the same problem truncated to its first L tokens: its
+    outputs and gradients there equal those of the truncated inputs; past L, O = 0,
+    LSE = -inf and every gradient row is zero."""
+    r = _rng(42)
+    B, H, N, d = 3, 2, 17, 5
+    q, k, v, do = (r.standard_normal((B, H, N, d)) for _ in range(4))
+    lens = [17, 9, 1]
+    for causal, window in MODES:
+        o, lse = orc.fwd(q, k, v, 0.45, causal, window, lengths=lens)
+        dq, dk, dv = orc.bwd(q, k, v, do, 0.45, causal, window, lengths=lens)
+        for b, L in enumerate(lens):
+            sl = (slice(b, b + 1), slice(None), slice(0, L))
+            ot, lt = orc.fwd(q[sl], k[sl], v[sl], 0.45, causal, window)
+            gt = orc.bwd(q[sl], k[sl], v[sl], do[sl], 0.45, causal, window)
+            np.testing.assert_allclose(o[sl], ot, rtol=1e-13, atol=1e-13)
+            np.testing.assert_allclose(lse[b:b + 1, :, :L], lt, rtol=1e-13, atol=1e-13)
+            for g, t in zip((dq, dk, dv), gt):
+                np.testing.assert_allclose(g[sl], t, rtol=1e-12, atol=1e-12)
+            assert np.all(o[b, :, L:] == 0.0) and np.all(np.isneginf(lse[b, :, L:]))
+            for g in (dq, dk, dv):
+                assert np.all(g[b, :, L:] == 0.0)
+
+
+def pin_lengths_zero_entry(orc):
+    """A zero-length entry: O = 0, LSE = -inf, zero gradients; the others are unaffected."""
+    r = _rng(43)
+    q, k, v, do = (r.standard_normal((2, 1, 7, 3)) for _ in range(4))
+    o, lse = orc.fwd(q, k, v, 0.7, True, lengths=[7, 0])
+    g = orc.bwd(q, k, v, do, 0.7, True, lengths=[7, 0])
+    o1, lse1 = orc.fwd(q[:1], k[:1], v[:1], 0.7, True)
+    assert np.all(o[1] == 0.0) and np.all(np.isneginf(lse[1]))
+    np.testing.assert_allclose(o[:1], o1, rtol=1e-14, atol=1e-14)
+    for x in g:
+        assert np.all(x[1] == 0.0)
+
+
+def pin_lengths_finite_differences(orc):
+    """With variable lengths, the backward is still the gradient of L = <O, dO>."""
+    h = 1e-6
+    r = _rng(44)
+    q, k, v, do = (r.standard_normal((2, 1, 6, 2)) for _ in range(4))
+    lens = [6, 4]
+    for causal, window in MODES[:3]:
+        grads = orc.bwd(q, k, v, do, 0.6, causal, window, lengths=lens)
+
+        def L(qq, kk, vv):
+            o, _ = orc.fwd(qq, kk, vv, 0.6, causal, window, lengths=lens)
+            return float(np.sum(o * do))
+
+        for which, g in enumerate(grads):
+            fd = np.zeros_like(q)
+            for idx in np.ndindex(q.shape):
+                args = [q.copy(), k.copy(), v.copy()]
+                args[which][idx] += h
+                lp = L(*args)
+                args[which][idx] -= 2 * h
+                lm = L(*args)
+                fd[idx] = (lp - lm) / (2 * h)
+            err = np.abs(fd - g).max()
+            assert err <= 1e-6 * max(1.0, np.abs(g).max()), (causal, window, which, err)
+
+
 # Philox4x32-10 known-answer vectors: (counter, key) -> output, the three published with
 # the generator (all-zero, all-one and pi-digit inputs).
 PHILOX_KAT = [
@@ -668,6 +749,10 @@ ALL_PINS = [
     pin_padding_whole_entry,
     pin_padding_finite_differences,
     pin_padding_library_sdpa,
+    pin_lengths_full_is_identity,
+    pin_lengths_truncated_problem,
+    pin_lengths_zero_entry,
+    pin_lengths_finite_differences,
     pin_philox_known_answers,
     pin_dropout_mask_layout,
     pin_dropout_zero_is_identity,

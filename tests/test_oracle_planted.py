@@ -40,6 +40,10 @@ PLANTS = [
     ("key padding of the first batch entry for all",
      "return key_padding ? key_padding + (bh / H) * N : NULL;",
      "return key_padding ? key_padding : NULL;"),
+    ("lengths applied to keys only", "if (i >= len || j >= len) s = -INFINITY;",
+     "if (j >= len) s = -INFINITY;"),
+    ("lengths of the first entry for all", "return lengths ? lengths[bh / H] : N;",
+     "return lengths ? lengths[0] : N;"),
     ("Philox multiplier typo", "M0 = 0xD2511F53u", "M0 = 0xD2511F55u"),
     ("Philox key not bumped", "k1 += W1;", "k1 += 0;"),
     ("dropout counter takes the key as row", "ctr[1] = (uint32_t)i;", "ctr[1] = (uint32_t)j;"),
