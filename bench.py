@@ -169,13 +169,13 @@ def job_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
 
 
 # ------------------------------------------------------------------------- our arm
-def kernel_names(w, deterministic=False):
+def kernel_names(w, fused=False):
     """The kernels of one step, in launch order: the forward, then the backward's delta
-    preprocess and either the fused pass and the dQ conversion (head_dim 64) or the dK/dV
-    and dQ passes."""
+    preprocess and either the dK/dV and dQ passes or (fused, head_dim 64) the fused pass and
+    the dQ conversion."""
     if not w.backward:
         return ["fwd"]
-    if w.d == 64 and not deterministic:
+    if w.d == 64 and fused:
         return ["fwd", "bwd_preprocess", "bwd_fused", "bwd_dq_convert"]
     return ["fwd", "bwd_preprocess", "bwd_dkdv", "bwd_dq"]
 
@@ -187,7 +187,7 @@ class Problem:
     the backward's three phases form delta from it; with ALiBi the slopes ride in the same
     options. Each phase is its own C-ABI call, so CUDA events can sit between kernels."""
 
-    def __init__(self, w, dev, host=None, seed=0, plain=False, deterministic=False):
+    def __init__(self, w, dev, host=None, seed=0, plain=False, fused=False):
         import torch
         from exact_attention_126_b200 import fa, workloads
         self.w, self.dev, self.fa = w, dev, fa
@@ -208,16 +208,20 @@ class Problem:
         self.o_low = torch.empty_like(self.q)
         self.lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
         self.dq, self.dk, self.dv = (torch.empty_like(self.q) for _ in range(3))
-        self.ws = torch.empty(max(1, fa.fa_bwd_workspace_bytes(B, H, N, d)), dtype=torch.uint8,
-                              device=dev)
+        self.ws = torch.empty(max(1, fa.fa_bwd_workspace_bytes_ex(B, H, N, d,
+                                                                  fa.options(fused=fused))),
+                              dtype=torch.uint8, device=dev)
         self.slopes = None
         if w.alibi:
             self.slopes = torch.tensor(workloads.alibi_slopes(H), dtype=torch.float32,
                                        device=dev)
         # plain: the forward keeps no residual and delta is formed from the bf16 O
+        self.lengths = None
+        if w.varlen:
+            self.lengths = torch.tensor(w.seq_lengths(), dtype=torch.int32, device=dev)
         self.opt = fa.options(alibi_slopes=self.slopes, o_low=None if plain else self.o_low,
-                              deterministic=deterministic)
-        self.names = kernel_names(w, deterministic)
+                              fused=fused, seq_lengths=self.lengths)
+        self.names = kernel_names(w, fused)
         self.fused = "bwd_fused" in self.names
         self.launches = len(self.names)
 
@@ -340,7 +344,7 @@ def run_ours(args, w, rank, world, local_rank):
                                 device_id=dev)
 
     inp_host = synth.attention_inputs(w.B, w.H, w.N, w.d, w.seed_index, with_grad=True, pin=True)
-    prob = Problem(w, dev, host=inp_host, plain=args.plain, deterministic=args.deterministic)
+    prob = Problem(w, dev, host=inp_host, plain=args.plain, fused=args.fused)
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
 
@@ -372,13 +376,15 @@ def run_ours(args, w, rank, world, local_rank):
             if n in in_names:
                 t.copy_(inp_host[n], non_blocking=True)
         res = fa.attention_forward(q, k, v, w.softmax_scale, w.causal, w.window, sp,
-                                   alibi_slopes=prob.slopes, keep_residual=w.backward)
+                                   alibi_slopes=prob.slopes, keep_residual=w.backward,
+                                   seq_lengths=prob.lengths)
         host_out["o"].copy_(res[0], non_blocking=True)
         host_out["lse"].copy_(res[1], non_blocking=True)
         if w.backward:
             grads = fa.attention_backward(q, k, v, res[0], res[1], do, w.softmax_scale, w.causal,
                                           w.window, sp, alibi_slopes=prob.slopes, o_low=res[2],
-                                          deterministic=args.deterministic)
+                                          fused=args.fused,
+                                          seq_lengths=prob.lengths)
             for n, t in zip(("dq", "dk", "dv"), grads):
                 host_out[n].copy_(t, non_blocking=True)
 
@@ -408,7 +414,7 @@ def run_ours(args, w, rank, world, local_rank):
                 continue
             ow = WORKLOADS[name]
             op = Problem(ow, dev, seed=1000 + ow.seed_index, plain=args.plain,
-                         deterministic=args.deterministic)
+                         fused=args.fused)
             with ClockSampler(local_rank) as oc:
                 oms, oker, _ = op.time(max(20, args.steps), args.warmup, stream)
             line = workload_line(ow, oms, oker, op.flushed)
@@ -467,12 +473,11 @@ def run_ours(args, w, rank, world, local_rank):
         "data": "synthetic (seeded i.i.d. N(0,1) bf16, SplitMix64 + Box-Muller)",
         "config": {
             "workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
-            "window": list(w.window), "alibi": w.alibi,
+            "window": list(w.window), "alibi": w.alibi, "varlen": w.varlen,
             "pass": "fwd+bwd" if w.backward else "fwd",
             "path": ("plain: delta from the bf16 O" if args.plain else
                      "training path: forward keeps O - bf16(O) for the backward's delta")
-                    + ("; deterministic backward (separate dQ pass)" if args.deterministic else
-                       ""),
+                    + ("; fused backward (dQ by fp32 bulk reductions)" if args.fused else ""),
             "kernels": list(per_kernel),
             "step_gflop": round(flops / 1e9, 3),
             "parallelism": "replicas" if world > 1 else "single",
@@ -517,25 +522,38 @@ def _head_slope(w, h):
     return [workloads.alibi_slopes(w.H)[h]]
 
 
+def _oracle_head(orc, w, b, h):
+    """Runs the oracle, as it stands, on the (batch b, head h) problem of the workload;
+    returns (seconds, the problem's flops by the metric's convention)."""
+    x = _oracle_sample(w, b, h)
+    slope = _head_slope(w, h)
+    lengths = [w.seq_lengths()[b]] if w.varlen else None
+    pairs = w.visible_pairs(lengths[0]) if w.varlen else None
+    flops = (4.0 * w.d * pairs * (3.5 if w.backward else 1.0) if w.varlen
+             else w.step_flops() / (w.B * w.H))
+    t0 = time.perf_counter()
+    orc.fwd(x["q"], x["k"], x["v"], w.softmax_scale, w.causal, w.window, slope,
+            lengths=lengths)
+    if w.backward:
+        orc.bwd(x["q"], x["k"], x["v"], x["do"], w.softmax_scale, w.causal, w.window, slope,
+                lengths=lengths)
+    return time.perf_counter() - t0, flops
+
+
 def cpu_baseline(w, seconds: float):
     """Times the fp64 oracle, as it stands, on whole (batch, head) problems of the workload
     until `seconds` have passed (at least one head)."""
     import oracle
     orc = oracle.default()
-    flops_per_head = w.step_flops() / (w.B * w.H)
-    done, elapsed = 0, 0.0
+    done, elapsed, flops = 0, 0.0, 0.0
     BH = w.B * w.H
     while elapsed < seconds and done < BH:
         b, h = divmod(done, w.H)
-        x = _oracle_sample(w, b, h)
-        slope = _head_slope(w, h)
-        t0 = time.perf_counter()
-        orc.fwd(x["q"], x["k"], x["v"], w.softmax_scale, w.causal, w.window, slope)
-        if w.backward:
-            orc.bwd(x["q"], x["k"], x["v"], x["do"], w.softmax_scale, w.causal, w.window, slope)
-        elapsed += time.perf_counter() - t0
+        dt, f = _oracle_head(orc, w, b, h)
+        elapsed += dt
+        flops += f
         done += 1
-    return {"value": round(flops_per_head * done / elapsed / 1e12, 6), "unit": "TFLOP/s",
+    return {"value": round(flops / elapsed / 1e12, 6), "unit": "TFLOP/s",
             "cores": orc.num_threads(), "kind": "oracle",
             "sample": "%d of %d (batch, head) problems of %s, fwd%s, %.1f s" % (
                 done, BH, w.name, "+bwd" if w.backward else "", elapsed)}
@@ -548,24 +566,18 @@ def run_reference(args, w, rank):
     import oracle
     orc = oracle.default()
     BH = w.B * w.H
-    flops_per_head = w.step_flops() / BH
     heads_per_step = 1
 
     def one(idx):
         b, h = divmod(idx % BH, w.H)
-        x = _oracle_sample(w, b, h)
-        slope = _head_slope(w, h)
-        t0 = time.perf_counter()
-        orc.fwd(x["q"], x["k"], x["v"], w.softmax_scale, w.causal, w.window, slope)
-        if w.backward:
-            orc.bwd(x["q"], x["k"], x["v"], x["do"], w.softmax_scale, w.causal, w.window, slope)
-        return time.perf_counter() - t0
+        return _oracle_head(orc, w, b, h)
 
     for i in range(args.warmup):
         one(i)
-    total = sum(one(args.warmup + s) for s in range(args.steps))
+    runs = [one(args.warmup + s) for s in range(args.steps)]
+    total = sum(t for t, _ in runs)
     ms_per_step = total * 1e3 / args.steps
-    value = flops_per_head * heads_per_step / (ms_per_step * 1e-3) / 1e12
+    value = sum(f for _, f in runs) / total / 1e12
     sample = "%d (batch, head) problem(s) of %s per step, fwd%s" % (
         heads_per_step, w.name, "+bwd" if w.backward else "")
     return {
@@ -589,15 +601,15 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="c4", help="c1, c2, c3, c4, c5c or c5w")
+    ap.add_argument("--workload", default="c4", help="c1, c2, c3, c4, c5c, c5w, c4a or c4v")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--also", default="c2,c3,c4,c5c,c5w",
+    ap.add_argument("--also", default="c2,c3,c4,c5c,c5w,c4v",
                     help="other workloads timed at full size in the same run (comma list)")
-    ap.add_argument("--deterministic", action="store_true",
-                    help="time the backward with the separate dQ pass at head_dim 64 too")
+    ap.add_argument("--fused", action="store_true",
+                    help="time the fused backward (dQ by fp32 bulk reductions) at head_dim 64")
     ap.add_argument("--plain", action="store_true",
                     help="time the path without the O residual (delta from the bf16 O)")
     ap.add_argument("--no-workloads", action="store_true",

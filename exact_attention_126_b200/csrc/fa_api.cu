@@ -63,8 +63,12 @@ fa_status_t dispatch_features(std::integer_sequence<int, Fs...>, int feat, Args&
   return found ? s : FA_ERR_UNSUPPORTED;
 }
 
-// forward: every combination of ALiBi, key padding, residual and dropout
-using FwdFeatures = std::integer_sequence<int, 0, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14, 15>;
+// forward: every combination of ALiBi, key padding, residual and dropout; at head_dim 128
+// also the e4m3 forward
+using FwdFeatures64 = std::integer_sequence<int, 0, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14,
+                                            15>;
+using FwdFeatures128 = std::integer_sequence<int, 0, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13,
+                                             14, 15, 16>;
 // backward passes: ALiBi, key padding and dropout (the residual only changes delta)
 using BwdFeatures = std::integer_sequence<int, 0, 1, 2, 3, 8, 9, 10, 11>;
 
@@ -108,7 +112,7 @@ size_t stats_bytes(int B, int H, int N) {
   return (raw + 255) & ~size_t(255);
 }
 
-bool uses_fused(int d, const Extras& x) { return d == 64 && !x.deterministic; }
+bool uses_fused(int d, const Extras& x) { return d == 64 && x.fused; }
 
 size_t dq_acc_bytes(int B, int H, int N, int d) {
   return (size_t)B * H * padded_rows(N) * (size_t)d * sizeof(float);
@@ -135,11 +139,14 @@ fa_status_t resolve_options(const fa_options_t* opt, Extras* x) {
   if (!(p >= 0.f && p < 1.f) || opt->dropout_offset > 0xFFFFFFFFull) return FA_ERR_INVALID_ARG;
   const int t = (int)std::floor(256.0 * (double)p + 0.5);
   if (t > 255) return FA_ERR_INVALID_ARG;
-  if ((opt->flags & ~(unsigned)FA_BWD_DETERMINISTIC) != 0) return FA_ERR_INVALID_ARG;
+  if ((opt->flags & ~(unsigned)FA_BWD_FUSED) != 0) return FA_ERR_INVALID_ARG;
   x->alibi = opt->alibi_slopes;
   x->kpad = opt->key_padding;
   x->o_low = opt->o_low;
-  x->deterministic = (opt->flags & FA_BWD_DETERMINISTIC) != 0;
+  x->fused = (opt->flags & FA_BWD_FUSED) != 0;
+  if (opt->seq_lengths != nullptr && (reinterpret_cast<uintptr_t>(opt->seq_lengths) & 3u) != 0)
+    return FA_ERR_MISALIGNED;
+  x->seq_len = opt->seq_lengths;
   if (t > 0) {
     x->dropout = true;
     x->drop.seed_lo = (uint32_t)(opt->dropout_seed & 0xFFFFFFFFull);
@@ -157,6 +164,13 @@ fa_status_t check_slopes(const float* alibi) {
   return FA_OK;
 }
 
+// Variable-length batches: what the kernels leave past each entry's real length.
+fa_status_t fill(void* t0, void* t1, void* t2, float* lse, int d, int BH, int H, int N,
+                 const Extras& x, cudaStream_t st) {
+  return d == 64 ? fa_host::launch_fill_past_length<64>(t0, t1, t2, lse, x.seq_len, BH, H, N, st)
+                 : fa_host::launch_fill_past_length<128>(t0, t1, t2, lse, x.seq_len, BH, H, N, st);
+}
+
 // The forward for every entry point: checks, then the kernel for (d, ALiBi or not).
 fa_status_t forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                     int N, int d, float scale, int causal, fa_window_t window, const Extras& x,
@@ -171,10 +185,12 @@ fa_status_t forward(const void* q, const void* k, const void* v, void* o, float*
   const int l = window.left, BH = B * H;
   const Problem pb{BH, H, N, scale, l, right};
   const int fault = g_fault.load(std::memory_order_relaxed);
-  return d == 64 ? dispatch_features<FwdLaunch<64>>(FwdFeatures(), x.features(), q, k, v, o, lse, pb, x,
-                                                        fault, st)
-                 : dispatch_features<FwdLaunch<128>>(FwdFeatures(), x.features(), q, k, v, o, lse, pb, x,
-                                                         fault, st);
+  s = d == 64 ? dispatch_features<FwdLaunch<64>>(FwdFeatures64(), x.features(), q, k, v, o, lse,
+                                                 pb, x, fault, st)
+              : dispatch_features<FwdLaunch<128>>(FwdFeatures128(), x.features(), q, k, v, o,
+                                                  lse, pb, x, fault, st);
+  if (s != FA_OK || x.seq_len == nullptr) return s;
+  return fill(o, x.o_low, nullptr, lse, d, BH, H, N, x, st);
 }
 
 // Step 1 of the backward: the row statistics in `workspace`.
@@ -208,8 +224,11 @@ fa_status_t fused_pass(const void* q, const void* k, const void* v, const void* 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Problem pb{B * H, H, N, scale, window.left, right};
   const int feat = x.features() & ~fa::kFeatResidual;
-  return dispatch_features<FusedLaunch>(BwdFeatures(), feat, q, k, v, dout, workspace,
-                                        dq_acc_of(workspace, B, H, N), dk, dv, pb, x, st);
+  s = dispatch_features<FusedLaunch>(BwdFeatures(), feat, q, k, v, dout, workspace,
+                                     dq_acc_of(workspace, B, H, N), dk, dv, pb, x, st);
+  // rows of dQ past the real length stay zero in the accumulator
+  if (s != FA_OK || x.seq_len == nullptr) return s;
+  return fill(dk, dv, nullptr, nullptr, d, B * H, H, N, x, st);
 }
 
 // dQ from the fused pass's accumulator.
@@ -240,10 +259,12 @@ fa_status_t dkdv_pass(const void* q, const void* k, const void* v, const void* d
   const int l = window.left, BH = B * H;
   const int feat = x.features() & ~fa::kFeatResidual;
   const Problem pb{BH, H, N, scale, l, right};
-  return d == 64 ? dispatch_features<DkdvLaunch<64>>(BwdFeatures(), feat, q, k, v, dout, workspace, dk, dv,
-                                                        pb, x, st)
-                 : dispatch_features<DkdvLaunch<128>>(BwdFeatures(), feat, q, k, v, dout, workspace, dk, dv,
-                                                         pb, x, st);
+  s = d == 64 ? dispatch_features<DkdvLaunch<64>>(BwdFeatures(), feat, q, k, v, dout, workspace,
+                                                  dk, dv, pb, x, st)
+              : dispatch_features<DkdvLaunch<128>>(BwdFeatures(), feat, q, k, v, dout, workspace,
+                                                   dk, dv, pb, x, st);
+  if (s != FA_OK || x.seq_len == nullptr) return s;
+  return fill(dk, dv, nullptr, nullptr, d, BH, H, N, x, st);
 }
 
 // Step 3: dQ.
@@ -260,10 +281,12 @@ fa_status_t dq_pass(const void* q, const void* k, const void* v, const void* dou
   const int l = window.left, BH = B * H;
   const int feat = x.features() & ~fa::kFeatResidual;
   const Problem pb{BH, H, N, scale, l, right};
-  return d == 64 ? dispatch_features<DqLaunch<64>>(BwdFeatures(), feat, q, k, v, dout, workspace, dq, pb, x,
-                                                      st)
-                 : dispatch_features<DqLaunch<128>>(BwdFeatures(), feat, q, k, v, dout, workspace, dq, pb, x,
-                                                       st);
+  s = d == 64 ? dispatch_features<DqLaunch<64>>(BwdFeatures(), feat, q, k, v, dout, workspace,
+                                                dq, pb, x, st)
+              : dispatch_features<DqLaunch<128>>(BwdFeatures(), feat, q, k, v, dout, workspace,
+                                                 dq, pb, x, st);
+  if (s != FA_OK || x.seq_len == nullptr) return s;
+  return fill(dq, nullptr, nullptr, nullptr, d, BH, H, N, x, st);
 }
 
 // The three steps of the backward, with the statistics in `stats` (caller workspace or the
@@ -392,6 +415,24 @@ fa_status_t fa_fwd_ex(const void* q, const void* k, const void* v, void* o, floa
   return forward(q, k, v, o, lse, B, H, N, d, scale, causal, window, x, stream);
 }
 
+fa_status_t fa_fwd_fp8(const void* q, const void* k, const void* v, float q_scale, float k_scale,
+                       float v_scale, void* o, float* lse, int B, int H, int N, int d,
+                       float scale, int causal, fa_window_t window, void* stream) {
+  bool empty;
+  fa_status_t s = check_problem(B, H, N, d, &empty);
+  if (s != FA_OK || empty) return s;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  for (float f : {q_scale, k_scale, v_scale})
+    if (!std::isfinite(f) || !(f > 0.f)) return FA_ERR_INVALID_ARG;
+  if ((s = check_mask(scale, window)) != FA_OK) return s;
+  const float s_all = scale * q_scale * k_scale;  // the descales of Q and K join the scale
+  if (!std::isfinite(s_all) || !(s_all > 0.f)) return FA_ERR_INVALID_ARG;
+  Extras x;
+  x.fp8 = true;
+  x.o_scale = v_scale;
+  return forward(q, k, v, o, lse, B, H, N, d, s_all, causal, window, x, stream);
+}
+
 fa_status_t fa_fwd_alibi(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                          int H, int N, int d, float scale, int causal, fa_window_t window,
                          const float* alibi_slopes, void* stream) {
@@ -408,6 +449,14 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   bool empty;
   if (check_problem(B, H, N, d, &empty) != FA_OK || empty) return 0;
   return workspace_bytes(B, H, N, d, Extras());
+}
+
+size_t fa_bwd_workspace_bytes_ex(int B, int H, int N, int d, const fa_options_t* options) {
+  bool empty;
+  if (check_problem(B, H, N, d, &empty) != FA_OK || empty) return 0;
+  Extras x;
+  if (resolve_options(options, &x) != FA_OK) return 0;
+  return workspace_bytes(B, H, N, d, x);
 }
 
 fa_status_t fa_bwd_preprocess(const void* o, const void* dout, const float* lse,
@@ -509,7 +558,6 @@ fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const vo
   if (s != FA_OK || empty) return s;
   // the three-kernel backward, whose only scratch is the row statistics
   Extras x;
-  x.deterministic = true;
   if (workspace_bytes(B, H, N, d, x) > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
   void* scratch = nullptr;
   if ((s = noalloc_scratch(&scratch)) != FA_OK) return s;

@@ -119,6 +119,32 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// ------------------------------------------------------------------------------------
+// Variable-length batches: rows r >= L_b (the real length of the row's batch entry) of up to
+// three bf16 (B*H, N, D) tensors become zero and, with `lse`, their LSE becomes -inf. The
+// attention kernels skip every tile that lies wholly past the real length; this fills what
+// they leave. 8 values (16 bytes) per thread; threads of rows below L_b do nothing.
+// ------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256)
+    fa_fill_past_length_kernel(__nv_bfloat16* __restrict__ t0, __nv_bfloat16* __restrict__ t1,
+                               __nv_bfloat16* __restrict__ t2, float* __restrict__ lse,
+                               const int* __restrict__ seq_len, long long rows, int N, int H) {
+  constexpr int kPerRow = D / 8;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long row = idx / kPerRow;  // over the B*H*N rows
+  if (row >= rows) return;
+  const int part = (int)(idx - row * kPerRow);
+  const long long bh = row / N;
+  const int r = (int)(row - bh * N);
+  if (r < real_length(seq_len, (int)bh, H, N)) return;
+  const size_t off = (size_t)row * D + part * 8;
+  if (t0 != nullptr) st_global_v4(t0 + off, 0u, 0u, 0u, 0u);
+  if (t1 != nullptr) st_global_v4(t1 + off, 0u, 0u, 0u, 0u);
+  if (t2 != nullptr) st_global_v4(t2 + off, 0u, 0u, 0u, 0u);
+  if (lse != nullptr && part == 0) lse[row] = -INFINITY;
+}
+
 struct BwdArgs {
   const float* stats;   // row statistics written by fa_bwd_preprocess_kernel
   __nv_bfloat16* out0;  // dkdv: dK ; dq: dQ (written directly when outputs are not staged)
@@ -139,6 +165,7 @@ struct BwdArgs {
   int H;                // heads per batch entry (batch entry of bh = bh / H)
   const uint8_t* kpad;  // (B, N) key-padding flags (nonzero = padded key), or null
   DropoutArgs drop;     // kFeatDropout kernels
+  const int* seq_len;   // variable-length batch: B real lengths, or null
 };
 
 // Shared layout of both backward kernels: the stationary tiles X0, X1 of an item (in XB
@@ -276,14 +303,20 @@ __device__ __forceinline__ constexpr uint32_t packed_col(int kk) {
 // Item k of the persistent schedule: the (batch*head, stationary tile). Masked problems
 // use chunks of heads with the longest items first (see chunked_item): key tiles in
 // increasing order for dK/dV, query tiles in decreasing order for dQ.
-__device__ __forceinline__ void bwd_item(int k, const BwdArgs& a, bool rising, int& bh,
-                                         int& tile) {
+// Returns false when the stationary tile lies past the sequence's real length (a
+// variable-length batch): such an item has no work, and every role skips it without
+// advancing its counters. `mk` is the item's mask, over the real length.
+__device__ __forceinline__ bool bwd_item(int k, const BwdArgs& a, bool rising, int& bh,
+                                         int& tile, Mask& mk) {
   if (a.longest_first) {
     chunked_item(k, a.BH, a.n_tiles, a.group, rising, bh, tile);
   } else {
     bh = k / a.n_tiles;
     tile = k % a.n_tiles;
   }
+  const int n = real_length(a.seq_len, bh, a.H, a.N);
+  mk = Mask{n, a.left, a.right};
+  return tile < num_tiles(n);
 }
 
 template <typename C>
@@ -354,7 +387,6 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const Mask mk{a.N, a.left, a.right};
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
   auto bar = [&](int i) -> uint32_t { return sb + C::kBar + 8u * i; };
 
@@ -401,7 +433,8 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
       bool ok = true;
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, j;
-        bwd_item(k, a, true, bh, j);
+        Mask mk;
+        if (!bwd_item(k, a, true, bh, j, mk)) continue;
         int i_lo, i_hi;
         q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
         const int xb = items % C::kXBufs, xu = items / C::kXBufs;
@@ -455,7 +488,8 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
       bool ok = true;
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, j;
-        bwd_item(k, a, true, bh, j);
+        Mask mk;
+        if (!bwd_item(k, a, true, bh, j, mk)) continue;
         int i_lo, i_hi;
         q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
         const int xb = items % C::kXBufs, xu = items / C::kXBufs;
@@ -511,7 +545,8 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
       bool ok = true;
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, j;
-        bwd_item(k, a, true, bh, j);
+        Mask mk;
+        if (!bwd_item(k, a, true, bh, j, mk)) continue;
         int i_lo, i_hi;
         q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
         for (int i = i_lo; i <= i_hi; ++i, ++t) {
@@ -561,11 +596,13 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
     // staged them in; the buffer goes back to the producer once the stores have read it.
     if (lane == 0 && C::kStageOut) {
       int items = 0;
-      for (int k = blockIdx.x; k < a.n_items; k += gridDim.x, ++items) {
+      for (int k = blockIdx.x; k < a.n_items; k += gridDim.x) {
         int bh, j;
-        bwd_item(k, a, true, bh, j);
+        Mask mk;
+        if (!bwd_item(k, a, true, bh, j, mk)) continue;
         const int xb = items % C::kXBufs;
         if (!mbar_wait(bar(bStaged), items & 1, abort_flag)) break;
+        ++items;
         for (int r = 0; r < C::kRegions; ++r) {
           tma_store_3d(&tmdK, sb + C::kX0 + xb * 2 * C::kTile + r * C::kRegionBytes, r * 64,
                        j * kBlock, bh);
@@ -590,7 +627,8 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
     bool ok = true;
     for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
       int bh, j;
-      bwd_item(k, a, true, bh, j);
+      Mask mk;
+      if (!bwd_item(k, a, true, bh, j, mk)) continue;
       int i_lo, i_hi;
       q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
       const int n_it = i_hi - i_lo + 1;
@@ -763,7 +801,6 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const Mask mk{a.N, a.left, a.right};
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
   auto bar = [&](int k) -> uint32_t { return sb + C::kBar + 8u * k; };
 
@@ -807,7 +844,8 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
       bool ok = true;
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, i;
-        bwd_item(k, a, false, bh, i);
+        Mask mk;
+        if (!bwd_item(k, a, false, bh, i, mk)) continue;
         int j_lo, j_hi;
         kv_tiles_for_q_tile(i, mk, j_lo, j_hi);
         const int xb = items % C::kXBufs, xu = items / C::kXBufs;
@@ -856,7 +894,8 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
       bool ok = true;
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, i;
-        bwd_item(k, a, false, bh, i);
+        Mask mk;
+        if (!bwd_item(k, a, false, bh, i, mk)) continue;
         int j_lo, j_hi;
         kv_tiles_for_q_tile(i, mk, j_lo, j_hi);
         const int xb = items % C::kXBufs, xu = items / C::kXBufs;
@@ -911,7 +950,8 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
       bool ok = true;
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, i;
-        bwd_item(k, a, false, bh, i);
+        Mask mk;
+        if (!bwd_item(k, a, false, bh, i, mk)) continue;
         int j_lo, j_hi;
         kv_tiles_for_q_tile(i, mk, j_lo, j_hi);
         for (int jj = j_lo; jj <= j_hi; ++jj, ++t) {
@@ -945,11 +985,13 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
     // ------------------------------------------------------------------ output stores
     if (lane == 0 && C::kStageOut) {
       int items = 0;
-      for (int k = blockIdx.x; k < a.n_items; k += gridDim.x, ++items) {
+      for (int k = blockIdx.x; k < a.n_items; k += gridDim.x) {
         int bh, i;
-        bwd_item(k, a, false, bh, i);
+        Mask mk;
+        if (!bwd_item(k, a, false, bh, i, mk)) continue;
         const int xb = items % C::kXBufs;
         if (!mbar_wait(bar(bStaged), items & 1, abort_flag)) break;
+        ++items;
         for (int rg = 0; rg < C::kRegions; ++rg)
           tma_store_3d(&tmdQ, sb + C::kX0 + xb * 2 * C::kTile + rg * C::kRegionBytes, rg * 64,
                        i * kBlock, bh);
@@ -970,7 +1012,8 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
     bool ok = true;
     for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
       int bh, i;
-      bwd_item(k, a, false, bh, i);
+      Mask mk;
+      if (!bwd_item(k, a, false, bh, i, mk)) continue;
       int j_lo, j_hi;
       kv_tiles_for_q_tile(i, mk, j_lo, j_hi);
       const int n_it = j_hi - j_lo + 1;

@@ -133,7 +133,6 @@ __global__ void __launch_bounds__(FusedCfg::kThreads, 1)
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const Mask mk{a.N, a.left, a.right};
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
   auto bar = [&](int i) -> uint32_t { return sb + C::kBar + 8u * i; };
   constexpr uint32_t kSoftWarps = C::kSoftmax / 32;
@@ -183,7 +182,8 @@ __global__ void __launch_bounds__(FusedCfg::kThreads, 1)
       bool ok = true;
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, j;
-        bwd_item(k, a, true, bh, j);
+        Mask mk;
+        if (!bwd_item(k, a, true, bh, j, mk)) continue;
         int i_lo, i_hi;
         q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
         const int xb = items & 1, xu = items >> 1;
@@ -229,7 +229,8 @@ __global__ void __launch_bounds__(FusedCfg::kThreads, 1)
       bool ok = true;
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, j;
-        bwd_item(k, a, true, bh, j);
+        Mask mk;
+        if (!bwd_item(k, a, true, bh, j, mk)) continue;
         int i_lo, i_hi;
         q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
         const int xb = items & 1, xu = items >> 1;
@@ -281,7 +282,8 @@ __global__ void __launch_bounds__(FusedCfg::kThreads, 1)
       bool ok = true;
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, j;
-        bwd_item(k, a, true, bh, j);
+        Mask mk;
+        if (!bwd_item(k, a, true, bh, j, mk)) continue;
         int i_lo, i_hi;
         q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
         const uint32_t xK = sb + C::kX + (items & 1) * 2 * C::kTile;
@@ -346,9 +348,10 @@ __global__ void __launch_bounds__(FusedCfg::kThreads, 1)
       tma_prefetch_map(&tmDQ);
       int items = 0, t = 0;
       bool ok = true;
-      for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x, ++items) {
+      for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, j;
-        bwd_item(k, a, true, bh, j);
+        Mask mk;
+        if (!bwd_item(k, a, true, bh, j, mk)) continue;
         int i_lo, i_hi;
         q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
         for (int i = i_lo; i <= i_hi; ++i, ++t) {
@@ -365,6 +368,7 @@ __global__ void __launch_bounds__(FusedCfg::kThreads, 1)
         if (!ok) break;
         const int xb = items & 1;
         if (!mbar_wait(bar(C::bStaged), items & 1, abort_flag)) break;
+        ++items;
         tma_store_3d(&tmdK, sb + C::kX + xb * 2 * C::kTile, 0, j * kBlock, bh);
         tma_store_3d(&tmdV, sb + C::kX + xb * 2 * C::kTile + C::kTile, 0, j * kBlock, bh);
         bulk_commit();
@@ -405,7 +409,8 @@ __global__ void __launch_bounds__(FusedCfg::kThreads, 1)
     };
     for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
       int bh, j;
-      bwd_item(k, a, true, bh, j);
+      Mask mk;
+      if (!bwd_item(k, a, true, bh, j, mk)) continue;
       int i_lo, i_hi;
       q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
       const int n_it = i_hi - i_lo + 1;

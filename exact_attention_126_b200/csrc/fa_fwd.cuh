@@ -56,13 +56,18 @@ struct FwdArgs {
   const uint8_t* kpad;       // (B, N) key-padding flags (nonzero = padded key), or null
   __nv_bfloat16* o_low;      // (B, H, N, d) bf16 residual O - bf16(O), or null
   DropoutArgs drop;          // kFeatDropout kernels
+  const int* seq_len;        // variable-length batch: B real lengths, or null
+  float o_scale;             // kFeatFp8: the V descale, applied to O in the epilogue
 };
 
-template <int D>
+// kFp8: 8-bit (e4m3) Q, K, V tiles (head_dim 128 only: one 128-byte row per token).
+template <int D, bool kFp8 = false>
 struct FwdCfg {
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
-  static constexpr int kTile = kBlock * D * 2;  // bytes of a 128 x D bf16 tile
-  static constexpr int kRegions = D / 64;       // 128-byte-wide column regions per tile
+  static_assert(!kFp8 || D == 128, "the e4m3 forward is for head_dim 128");
+  static constexpr int kElemBytes = kFp8 ? 1 : 2;
+  static constexpr int kTile = kBlock * D * kElemBytes;  // bytes of a 128 x D tile
+  static constexpr int kRegions = D * kElemBytes / 128;  // 128-byte-wide column regions per tile
   static constexpr int kRegionBytes = kBlock * 128;
   static constexpr int kStagesK = (D == 64) ? 4 : 2;
   static constexpr int kStagesV = (D == 64) ? 4 : 2;
@@ -111,7 +116,9 @@ struct FwdCfg {
 // walks [first, last], the union (the ranges of consecutive query tiles overlap or touch).
 struct FwdItem {
   int bh;
+  int n;        // the sequence's real length (N unless the batch is variable-length)
   int m[2];
+  bool has_a;   // query tile A lies within the real length (else the item has no work)
   bool has_b;
   int lo[2];
   int hi[2];
@@ -128,10 +135,13 @@ __device__ __forceinline__ FwdItem fwd_item(int k, const FwdArgs& a) {
     it.bh = k / a.n_pairs;
     pair = k % a.n_pairs;
   }
-  const Mask mk{a.N, a.left, a.right};
+  it.n = real_length(a.seq_len, it.bh, a.H, a.N);
+  const Mask mk{it.n, a.left, a.right};
+  const int n_qtiles = num_tiles(it.n);
   it.m[0] = 2 * pair;
   it.m[1] = 2 * pair + 1;
-  it.has_b = it.m[1] < a.n_qtiles;
+  it.has_a = it.m[0] < n_qtiles;
+  it.has_b = it.m[1] < n_qtiles;
   kv_tiles_for_q_tile(it.m[0], mk, it.lo[0], it.hi[0]);
   if (it.has_b) {
     kv_tiles_for_q_tile(it.m[1], mk, it.lo[1], it.hi[1]);
@@ -158,7 +168,7 @@ struct FwdRange {
 
 __device__ __forceinline__ FwdRange fwd_range(const FwdItem& it, int s) {
   FwdRange r;
-  r.has = s == 0 || it.has_b;
+  r.has = s == 0 ? it.has_a : it.has_b;
   r.m = s ? it.m[1] : it.m[0];
   r.lo = s ? it.lo[1] : it.lo[0];
   r.hi = s ? it.hi[1] : it.hi[0];
@@ -169,12 +179,15 @@ __device__ __forceinline__ FwdRange fwd_range(const FwdItem& it, int s) {
 // scaled score; kFeatKpad masks the keys a.kpad flags; kFeatResidual also writes
 // O - bf16(O) to a.o_low; kFeatDropout zeroes the weights whose Philox keep flag is
 // clear before the P V product (the row sum l keeps them: dropout follows the softmax)
-// and scales O by 1 / (1 - p').
+// and scales O by 1 / (1 - p'); kFeatFp8 takes e4m3 Q, K, V (S = Q K^T and P V as
+// kind::f8f6f4 products, P rounded to e4m3, four per tensor-memory column; the Q and K
+// descales are folded into scale_log2, the V descale into O).
 template <int D, int kFeat = 0>
-__global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
+__global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
-  using C = FwdCfg<D>;
+  constexpr bool kFp8 = (kFeat & kFeatFp8) != 0;
+  using C = FwdCfg<D, kFp8>;
   constexpr bool kAlibi = (kFeat & kFeatAlibi) != 0;
   constexpr bool kKpad = (kFeat & kFeatKpad) != 0;
   constexpr bool kResidual = (kFeat & kFeatResidual) != 0;
@@ -185,7 +198,6 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const Mask mk{a.N, a.left, a.right};
 
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
@@ -237,6 +249,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
       bool ok = true;
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         const FwdItem it = fwd_item(k, a);
+        if (!it.has_a) continue;  // past the real length: nothing to load
         for (int s = 0; s < 2; ++s) {
           if (s == 1 && !it.has_b) break;
           // Q_s of this item replaces the previous item's once its last S_s has been read
@@ -303,8 +316,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     // only passing where it does not; a ring slot is released by one arrival per stream.
     if (lane == 0) {
       const int s = warp - C::kWarpMma;
-      constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t idS = kFp8 ? idesc_e4m3_f32(128, 128, false, false)
+                                    : idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idO = kFp8 ? idesc_e4m3_f32(128, D, false, true)
+                                    : idesc_bf16_f32(128, D, false, true);
       int nq = 0;     // Q tiles consumed
       int nsi = 0;    // S products issued (all items)
       int npv = 0;    // P V products issued (all items)
@@ -328,13 +343,20 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
               !free_s)
             return false;
           tc_fence_after();
+          const uint32_t qbase = sb + C::kQ + (s * C::kQBufs + nq % C::kQBufs) * C::kTile;
+          if constexpr (kFp8) {
+            // K-steps of 32 e4m3 values: 32 bytes of the 128-byte rows
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-            mma_ss(tmem + C::tS + 128u * s,
-                   sdesc_sw128(sb + C::kQ + (s * C::kQBufs + nq % C::kQBufs) * C::kTile + off, 16,
-                               1024),
-                   sdesc_sw128(sb + C::kK + sk * C::kTile + off, 16, 1024), idS, kk > 0);
+            for (int kk = 0; kk < D / 32; ++kk)
+              mma_ss_f8(tmem + C::tS + 128u * s, sdesc_sw128(qbase + kk * 32, 16, 1024),
+                        sdesc_sw128(sb + C::kK + sk * C::kTile + kk * 32, 16, 1024), idS, kk > 0);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
+              mma_ss(tmem + C::tS + 128u * s, sdesc_sw128(qbase + off, 16, 1024),
+                     sdesc_sw128(sb + C::kK + sk * C::kTile + off, 16, 1024), idS, kk > 0);
+            }
           }
           tc_commit(bar(C::bSFull + s));
           ++nsi;
@@ -359,12 +381,21 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
               (first && nitem > 0 && !mbar_wait(bar(C::bOFree + s), (nitem - 1) & 1, abort_flag)))
             return false;
           tc_fence_after();
+          const uint32_t pcol = tmem + (C::kSepP ? C::tP + 64u * s : C::tS + 128u * s);
+          if constexpr (kFp8) {
+            // K-steps of 32 keys: 8 columns of P (four e4m3 per column), 32 rows of V
 #pragma unroll
-          for (int kk = 0; kk < kBlock / 16; ++kk)
-            mma_ts(tmem + C::tO + D * s,
-                   tmem + (C::kSepP ? C::tP + 64u * s : C::tS + 128u * s) + kk * 8,
-                   sdesc_sw128(sb + C::kV + sv * C::kTile + kk * 2048, C::kRegionBytes, 1024),
-                   idO, (!first || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kBlock / 32; ++kk)
+              mma_ts_f8(tmem + C::tO + D * s, pcol + kk * 8,
+                        sdesc_sw128(sb + C::kV + sv * C::kTile + kk * 4096, C::kRegionBytes, 1024),
+                        idO, (!first || kk > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < kBlock / 16; ++kk)
+              mma_ts(tmem + C::tO + D * s, pcol + kk * 8,
+                     sdesc_sw128(sb + C::kV + sv * C::kTile + kk * 2048, C::kRegionBytes, 1024),
+                     idO, (!first || kk > 0) ? 1u : 0u);
+          }
           tc_commit(bar(C::bODone + s));
           ++npv;
           if (j == rg.hi) ++nitem;
@@ -375,6 +406,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
 
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         const FwdItem it = fwd_item(k, a);
+        if (!it.has_a) continue;  // past the real length: no products
         const FwdRange rg = fwd_range(it, s);
         const int n = it.last - it.first + 1;
         if (C::kSepP) {
@@ -427,6 +459,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
       const FwdRange rg = fwd_range(it, s);
       if (!rg.has) continue;
       const bool turns = it.has_b;
+      const Mask mk{it.n, a.left, a.right};
       const int row = rg.m * kBlock + r;
       // with ALiBi the scores are scaled and biased as they are loaded (in log2 units), so
       // the later steps take them as they are
@@ -563,19 +596,33 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
-          uint32_t pk[16];
+          if constexpr (kFp8) {
+            // e4m3 P, four per column: keys 32h .. 32h+31 in columns 8h .. 8h+7
+            uint32_t pk[8];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            float p0 = ex2(fmaf(x[32 * h + 2 * c], xs, -mb));
-            float p1 = ex2(fmaf(x[32 * h + 2 * c + 1], xs, -mb));
-            ls[c & 3] += p0 + p1;
-            if (kDropout) {
-              p0 = ((keep[h] >> (2 * c)) & 1u) ? p0 : 0.f;
-              p1 = ((keep[h] >> (2 * c + 1)) & 1u) ? p1 : 0.f;
+            for (int c = 0; c < 8; ++c) {
+              float p4[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) p4[e] = ex2(fmaf(x[32 * h + 4 * c + e], xs, -mb));
+              ls[c & 3] += (p4[0] + p4[1]) + (p4[2] + p4[3]);
+              pk[c] = pack_e4m3x4(p4[0], p4[1], p4[2], p4[3]);
             }
-            pk[c] = pack_bf16x2(p0, p1);
+            tmem_st8(tP + 8 * h, pk);
+          } else {
+            uint32_t pk[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              float p0 = ex2(fmaf(x[32 * h + 2 * c], xs, -mb));
+              float p1 = ex2(fmaf(x[32 * h + 2 * c + 1], xs, -mb));
+              ls[c & 3] += p0 + p1;
+              if (kDropout) {
+                p0 = ((keep[h] >> (2 * c)) & 1u) ? p0 : 0.f;
+                p1 = ((keep[h] >> (2 * c + 1)) & 1u) ? p1 : 0.f;
+              }
+              pk[c] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(tP + 16 * h, pk);
           }
-          tmem_st16(tP + 16 * h, pk);
         }
         if (turns) pass_turn();
         l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
@@ -606,6 +653,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
       tc_fence_after();
       float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
       if (kDropout) inv_l *= a.drop.keep_scale;
+      if (kFp8) inv_l *= a.o_scale;
       __nv_bfloat16* orow = a.o + ((size_t)it.bh * a.N + (row < a.N ? row : 0)) * D;
 #pragma unroll
       for (int q = 0; q < D / 32; ++q) {

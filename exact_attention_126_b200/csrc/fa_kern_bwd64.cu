@@ -11,6 +11,8 @@ FA_INSTANTIATE_BWD(64, 10) FA_INSTANTIATE_BWD(64, 11)
 template fa_status_t launch_preprocess<64>(const void*, const void*, const void*, const float*,
                                            float*, float*, int, int, cudaStream_t);
 template fa_status_t launch_dq_convert<64>(const float*, void*, int, int, float, cudaStream_t);
+template fa_status_t launch_fill_past_length<64>(void*, void*, void*, float*, const int*, int,
+                                                 int, int, cudaStream_t);
 
 int take_status_bwd64() { return take_unit_status(); }
 

@@ -10,6 +10,8 @@ FA_INSTANTIATE_FWD(128, 6)  FA_INSTANTIATE_FWD(128, 7)  FA_INSTANTIATE_FWD(128, 
 FA_INSTANTIATE_FWD(128, 9)  FA_INSTANTIATE_FWD(128, 10) FA_INSTANTIATE_FWD(128, 11)
 FA_INSTANTIATE_FWD(128, 12) FA_INSTANTIATE_FWD(128, 13) FA_INSTANTIATE_FWD(128, 14)
 FA_INSTANTIATE_FWD(128, 15)
+// the e4m3 forward (no other option)
+FA_INSTANTIATE_FWD(128, 16)
 
 int take_status_fwd128() { return take_unit_status(); }
 

@@ -20,13 +20,18 @@ struct Extras {
   const uint8_t* kpad = nullptr;   // (B, N) key-padding flags: the kFeatKpad kernels
   void* o_low = nullptr;           // bf16 residual of O: written by the forward, read by delta
   bool dropout = false;            // the kFeatDropout kernels, with `drop`
-  bool deterministic = false;      // backward: separate dQ pass instead of the fused one
+  bool fused = false;              // backward: the fused pass (head_dim 64) instead of the
+                                   // dK/dV and dQ passes
+  const int* seq_len = nullptr;    // variable-length batch: B real lengths
+  bool fp8 = false;                // forward on e4m3 Q, K, V (the kFeatFp8 kernel)
+  float o_scale = 1.f;             // with fp8: the V descale, applied to O
   fa::DropoutArgs drop = {0, 0, 0, 0, 1.f};
 
   // The kernel variant these options select (the backward passes ignore kFeatResidual).
   int features() const {
     return (alibi ? fa::kFeatAlibi : 0) | (kpad ? fa::kFeatKpad : 0) |
-           (o_low ? fa::kFeatResidual : 0) | (dropout ? fa::kFeatDropout : 0);
+           (o_low ? fa::kFeatResidual : 0) | (dropout ? fa::kFeatDropout : 0) |
+           (fp8 ? fa::kFeatFp8 : 0);
   }
 };
 
@@ -69,6 +74,12 @@ template <int D, int kFeat>
 fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* dout,
                       const void* ws, void* dq, const Problem& pb, const Extras& x,
                       cudaStream_t st);
+
+// Variable-length batches: zero rows past each entry's real length of up to three bf16
+// tensors (null = absent) and set their LSE to -inf (lse null = absent).
+template <int D>
+fa_status_t launch_fill_past_length(void* t0, void* t1, void* t2, float* lse,
+                                    const int* seq_len, int BH, int H, int N, cudaStream_t st);
 
 // Reads and clears the device status word of each kernel unit (0 = nothing recorded);
 // returns -1 if reading it failed.

@@ -50,6 +50,20 @@ inline bool make_acc_map(CUtensorMap* map, float* base, int BH, int Np) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// (B*H, N, d) e4m3 tensor (one byte per value), box of 128 rows x 128 columns (128 bytes),
+// 128-byte swizzle.
+inline bool make_map_u8(CUtensorMap* map, const void* base, int BH, int N, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)d, (cuuint64_t)N * d};
+  const cuuint32_t box[3] = {128, (cuuint32_t)kBlock, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // (B*H, N, d) bf16 tensor, box of 128 rows x 64 columns (128 bytes), 128-byte swizzle.
 inline bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d) {
   EncodeTiledFn enc = encode_fn();
@@ -100,10 +114,17 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
                        const Problem& pb, const Extras& x, int fault, cudaStream_t st) {
   const int BH = pb.BH, H = pb.H, N = pb.N, left = pb.left, right = pb.right;
   const float scale = pb.scale;
+  constexpr bool kFp8 = (kFeat & fa::kFeatFp8) != 0;
   CUtensorMap mq, mkk, mv;
-  if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) || !make_map(&mv, v, BH, N, D))
+  if (kFp8) {
+    if (!make_map_u8(&mq, q, BH, N, D) || !make_map_u8(&mkk, k, BH, N, D) ||
+        !make_map_u8(&mv, v, BH, N, D))
+      return FA_ERR_CUDA;
+  } else if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
+             !make_map(&mv, v, BH, N, D)) {
     return FA_ERR_CUDA;
-  using C = fa::FwdCfg<D>;
+  }
+  using C = fa::FwdCfg<D, kFp8>;
   if (set_smem(fa::fa_fwd_kernel<D, kFeat>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
   fa::FwdArgs a;
   a.o = static_cast<__nv_bfloat16*>(o);
@@ -124,6 +145,8 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   a.kpad = x.kpad;
   a.o_low = static_cast<__nv_bfloat16*>(x.o_low);
   a.drop = x.drop;
+  a.seq_len = x.seq_len;
+  a.o_scale = x.o_scale;
   const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
   fa::fa_fwd_kernel<D, kFeat><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, a);
   return launched();
@@ -169,6 +192,7 @@ inline fa::BwdArgs bwd_args(const void* ws, const Problem& pb, const Extras& x) 
   a.H = H;
   a.kpad = x.kpad;
   a.drop = x.drop;
+  a.seq_len = x.seq_len;
   return a;
 }
 
@@ -244,6 +268,17 @@ fa_status_t launch_dq_convert(const float* dq_acc, void* dq, int BH, int N, floa
   const long long blocks = (threads + 255) / 256;
   fa::fa_bwd_dq_convert_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
       dq_acc, static_cast<__nv_bfloat16*>(dq), rows, N, padded_rows(N), scale);
+  return launched();
+}
+
+template <int D>
+fa_status_t launch_fill_past_length(void* t0, void* t1, void* t2, float* lse,
+                                    const int* seq_len, int BH, int H, int N, cudaStream_t st) {
+  const long long rows = (long long)BH * N;
+  const long long blocks = (rows * (D / 8) + 255) / 256;
+  fa::fa_fill_past_length_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
+      static_cast<__nv_bfloat16*>(t0), static_cast<__nv_bfloat16*>(t1),
+      static_cast<__nv_bfloat16*>(t2), lse, seq_len, rows, N, H);
   return launched();
 }
 

@@ -18,6 +18,7 @@ constexpr int kFeatAlibi = 1;     // linear bias -m_h |i - j| on the scaled scor
 constexpr int kFeatKpad = 2;      // (B, N) key-padding flags
 constexpr int kFeatResidual = 4;  // forward also writes O - bf16(O)
 constexpr int kFeatDropout = 8;   // attention weights dropped with Philox keep flags
+constexpr int kFeatFp8 = 16;      // forward on e4m3 Q, K, V (P in e4m3 for the P V product)
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Mask {
@@ -31,6 +32,16 @@ __host__ __device__ inline int resolve_right(int causal, int right) {
 }
 
 __host__ __device__ inline int num_tiles(int N) { return (N + kBlock - 1) / kBlock; }
+
+#ifdef __CUDACC__
+// The real length of (batch, head) bh's sequence in a variable-length batch: seq_len[bh / H]
+// clamped to [0, N], or N when the batch is not variable-length (seq_len == nullptr).
+__device__ __forceinline__ int real_length(const int* seq_len, int bh, int H, int N) {
+  if (seq_len == nullptr) return N;
+  const int L = __ldg(seq_len + bh / H);
+  return L < 0 ? 0 : (L > N ? N : L);
+}
+#endif
 
 // Key tiles [lo, hi] holding at least one key visible from some valid row of query tile m.
 __host__ __device__ inline void kv_tiles_for_q_tile(int m, const Mask& k, int& lo, int& hi) {

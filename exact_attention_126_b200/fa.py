@@ -23,13 +23,14 @@ STATUS_NAMES = {
 }
 
 #: every symbol include/fa.h declares
-EXPORTED = ("fa_fwd", "fa_fwd_ex", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_ex",
+EXPORTED = ("fa_fwd", "fa_fwd_ex", "fa_fwd_fp8", "fa_bwd_workspace_bytes",
+            "fa_bwd_workspace_bytes_ex", "fa_bwd", "fa_bwd_ex",
             "fa_fwd_alibi", "fa_bwd_alibi", "fa_bwd_preprocess", "fa_bwd_dkdv", "fa_bwd_dq",
             "fa_bwd_fused", "fa_bwd_dq_convert", "fa_bwd_noalloc", "fa_status_string",
             "fa_debug_status", "fa_debug_set_fault", "fa_version")
 
-#: fa_options_t.flags: the backward with a separate, deterministic dQ pass
-FA_BWD_DETERMINISTIC = 1
+#: fa_options_t.flags: the fused backward (head_dim 64; dQ by fp32 reductions)
+FA_BWD_FUSED = 1
 
 
 class FAError(RuntimeError):
@@ -48,16 +49,18 @@ class fa_options_t(ctypes.Structure):
     _fields_ = [("alibi_slopes", ctypes.c_void_p), ("key_padding", ctypes.c_void_p),
                 ("o_low", ctypes.c_void_p), ("dropout_p", ctypes.c_float),
                 ("flags", ctypes.c_uint), ("dropout_seed", ctypes.c_ulonglong),
-                ("dropout_offset", ctypes.c_ulonglong)]
+                ("dropout_offset", ctypes.c_ulonglong), ("seq_lengths", ctypes.c_void_p)]
 
 
 def options(alibi_slopes=None, key_padding=None, o_low=None, dropout_p=0.0, dropout_seed=0,
-            dropout_offset=0, deterministic=False):
+            dropout_offset=0, fused=False, seq_lengths=None):
     """An fa_options_t holding the device pointers of the given tensors (None = absent), the
-    dropout parameters (probability, 64-bit seed, 32-bit offset) and the backward's flags."""
+    dropout parameters (probability, 64-bit seed, 32-bit offset), the backward's flags and
+    the real lengths of a variable-length batch (B int32 on the device)."""
     return fa_options_t(_ptr(alibi_slopes), _ptr(key_padding), _ptr(o_low), float(dropout_p),
-                        FA_BWD_DETERMINISTIC if deterministic else 0,
-                        int(dropout_seed) & 0xFFFFFFFFFFFFFFFF, int(dropout_offset))
+                        FA_BWD_FUSED if fused else 0,
+                        int(dropout_seed) & 0xFFFFFFFFFFFFFFFF, int(dropout_offset),
+                        _ptr(seq_lengths))
 
 
 _LIB = None
@@ -76,10 +79,13 @@ def _lib() -> ctypes.CDLL:
         OP = ctypes.POINTER(fa_options_t)
         lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp]
         lib.fa_fwd_ex.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, W, OP, vp]
+        lib.fa_fwd_fp8.argtypes = [vp, vp, vp, F, F, F, vp, vp, I, I, I, I, F, I, W, vp]
         lib.fa_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, OP,
                                   vp, ctypes.c_size_t, vp]
         lib.fa_bwd_workspace_bytes.argtypes = [I, I, I, I]
         lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
+        lib.fa_bwd_workspace_bytes_ex.argtypes = [I, I, I, I, OP]
+        lib.fa_bwd_workspace_bytes_ex.restype = ctypes.c_size_t
         lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp,
                                ctypes.c_size_t, vp]
         lib.fa_fwd_alibi.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, W, vp, vp]
@@ -97,7 +103,7 @@ def _lib() -> ctypes.CDLL:
         lib.fa_debug_status.argtypes = [vp]
         lib.fa_debug_set_fault.argtypes = [I]
         lib.fa_version.argtypes = []
-        for name in ("fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_ex", "fa_fwd_alibi",
+        for name in ("fa_fwd", "fa_fwd_ex", "fa_fwd_fp8", "fa_bwd", "fa_bwd_ex", "fa_fwd_alibi",
                      "fa_bwd_alibi", "fa_bwd_preprocess", "fa_bwd_fused", "fa_bwd_dq_convert",
                      "fa_bwd_dkdv", "fa_bwd_dq", "fa_bwd_noalloc", "fa_debug_status",
                      "fa_debug_set_fault", "fa_version"):
@@ -152,8 +158,40 @@ def fa_fwd(q, k, v, o, lse, scale=None, causal=False, window=(-1, -1), stream=No
                          _stream(stream)), "fa_fwd")
 
 
+def fa_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, scale=None, causal=False,
+               window=(-1, -1), stream=None) -> None:
+    """The forward on e4m3 tensors (torch.float8_e4m3fn or uint8 bytes) with per-tensor
+    descales; o is bf16."""
+    B, H, N, d = _shape(q8)
+    c, w = _window(causal, window)
+    s = default_scale(d) if scale is None else float(scale)
+    _check(_lib().fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), float(q_scale), float(k_scale),
+                             float(v_scale), _ptr(o), _ptr(lse), B, H, N, d, s, c, w,
+                             _stream(stream)), "fa_fwd_fp8")
+
+
+def attention_forward_fp8(q8, k8, v8, q_scale=1.0, k_scale=1.0, v_scale=1.0, scale=None,
+                          causal=False, window=(-1, -1), stream=None):
+    """Returns (O, LSE) of the attention of q8*q_scale, k8*k_scale, v8*v_scale for e4m3 CUDA
+    tensors of shape (B, H, N, 128); O is bf16."""
+    for t in (q8, k8, v8):
+        if not t.is_cuda or t.dtype not in (torch.float8_e4m3fn, torch.uint8):
+            raise ValueError("q8, k8, v8 must be float8_e4m3fn (or uint8) CUDA tensors")
+        if not t.is_contiguous() or t.shape != q8.shape:
+            raise ValueError("q8, k8, v8 must be contiguous and share one shape")
+    B, H, N, d = _shape(q8)
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    fa_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, scale, causal, window, stream)
+    return o, lse
+
+
 def fa_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
     return int(_lib().fa_bwd_workspace_bytes(B, H, N, d))
+
+
+def fa_bwd_workspace_bytes_ex(B: int, H: int, N: int, d: int, opt=None) -> int:
+    return int(_lib().fa_bwd_workspace_bytes_ex(B, H, N, d, _opt_ref(opt)))
 
 
 def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale=None, causal=False,
@@ -315,8 +353,16 @@ def _check_padding(key_padding, q):
         raise ValueError("key_padding must be a contiguous (batch, seq_len) tensor")
 
 
+def _check_lengths(seq_lengths, q):
+    if not seq_lengths.is_cuda or seq_lengths.dtype != torch.int32:
+        raise ValueError("seq_lengths must be an int32 CUDA tensor")
+    if seq_lengths.numel() != q.shape[0] or not seq_lengths.is_contiguous():
+        raise ValueError("seq_lengths must hold one length per batch entry, contiguous")
+
+
 def attention_forward(q, k, v, scale=None, causal=False, window=(-1, -1), stream=None,
-                      alibi_slopes=None, key_padding=None, keep_residual=False, dropout=None):
+                      alibi_slopes=None, key_padding=None, keep_residual=False, dropout=None,
+                      seq_lengths=None):
     """Returns (O, LSE) for bf16 CUDA tensors q, k, v of shape (B, H, N, d), or
     (O, LSE, O_low) with keep_residual: O_low = O_fp32 - bf16(O) in bf16, which
     attention_backward uses to form rowsum(dO o O) from O to about 16 bits.
@@ -324,7 +370,9 @@ def attention_forward(q, k, v, scale=None, causal=False, window=(-1, -1), stream
     key_padding ((B, N) bool or uint8, True = padded key): padded keys are masked out
     for every head and query. dropout: (p, seed, offset) drops each attention weight with
     probability p (rounded to a multiple of 1/256) after the softmax and scales the kept
-    ones by 1 / (1 - p); the backward needs the same triple."""
+    ones by 1 / (1 - p); the backward needs the same triple. seq_lengths ((B,) int32):
+    entry b holds seq_lengths[b] real tokens; rows past it are zero (LSE -inf) and tiles
+    wholly past it are not computed."""
     _check_inputs(q, k, v)
     B, H, N, d = _shape(q)
     o = torch.empty_like(q)
@@ -334,39 +382,45 @@ def attention_forward(q, k, v, scale=None, causal=False, window=(-1, -1), stream
         _check_slopes(alibi_slopes, q)
     if key_padding is not None:
         _check_padding(key_padding, q)
-    if alibi_slopes is None and key_padding is None and o_low is None and dropout is None:
+    if seq_lengths is not None:
+        _check_lengths(seq_lengths, q)
+    if (alibi_slopes is None and key_padding is None and o_low is None and dropout is None
+            and seq_lengths is None):
         fa_fwd(q, k, v, o, lse, scale, causal, window, stream)
     else:
-        opt = options(alibi_slopes, key_padding, o_low, *(dropout or ()))
+        opt = options(alibi_slopes, key_padding, o_low, *(dropout or ()),
+                      seq_lengths=seq_lengths)
         fa_fwd_ex(q, k, v, o, lse, opt, scale, causal, window, stream)
     return (o, lse, o_low) if keep_residual else (o, lse)
 
 
 def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, window=(-1, -1),
                        stream=None, alibi_slopes=None, key_padding=None, o_low=None,
-                       dropout=None, deterministic=False):
+                       dropout=None, fused=False, seq_lengths=None):
     """Returns (dQ, dK, dV): the gradient of <O, dO>; lse (and o_low, if kept) come from
-    attention_forward with the same alibi_slopes, key_padding and dropout. deterministic:
-    the backward with a separate dQ pass (bit-identical results run to run); otherwise
-    head_dim 64 adds dQ up in fp32 in no fixed order."""
+    attention_forward with the same alibi_slopes, key_padding, dropout and seq_lengths.
+    fused: at head_dim 64, the backward in one pass over key tiles with dQ added up in fp32
+    in no fixed order (see FA_BWD_FUSED); otherwise the deterministic dK/dV and dQ passes."""
     _check_inputs(q, k, v, o, do)
     B, H, N, d = _shape(q)
     dq = torch.empty_like(q)
     dk = torch.empty_like(q)
     dv = torch.empty_like(q)
-    ws = torch.empty(max(1, fa_bwd_workspace_bytes(B, H, N, d)), dtype=torch.uint8,
-                     device=q.device)
+    ws = torch.empty(max(1, fa_bwd_workspace_bytes_ex(B, H, N, d, options(fused=fused))),
+                     dtype=torch.uint8, device=q.device)
     if alibi_slopes is not None:
         _check_slopes(alibi_slopes, q)
     if key_padding is not None:
         _check_padding(key_padding, q)
     if o_low is not None:
         _check_inputs(q, o_low)
+    if seq_lengths is not None:
+        _check_lengths(seq_lengths, q)
     if (alibi_slopes is None and key_padding is None and o_low is None and dropout is None
-            and not deterministic):
+            and not fused and seq_lengths is None):
         fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, scale, causal, window, stream)
     else:
         opt = options(alibi_slopes, key_padding, o_low, *(dropout or ()),
-                      **({"deterministic": True} if deterministic else {}))
+                      fused=fused, seq_lengths=seq_lengths)
         fa_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, ws, opt, scale, causal, window, stream)
     return dq, dk, dv

@@ -29,14 +29,23 @@ class Workload:
     seed_index: int
     scale: float | None = None  # None: 1/sqrt(d)
     alibi: bool = False         # linear bias -m_h |i - j| with the slopes of alibi_slopes()
+    varlen: bool = False        # variable-length batch with the lengths of seq_lengths()
 
     @property
     def softmax_scale(self) -> float:
         return self.scale if self.scale is not None else 1.0 / math.sqrt(self.d)
 
-    def visible_pairs(self) -> int:
-        """Exact number of visible (query, key) pairs of one (batch, head)."""
-        N = self.N
+    def seq_lengths(self) -> list:
+        """The real lengths of a variable-length batch: seeded, uniform in [N/4, N]."""
+        if not self.varlen:
+            return [self.N] * self.B
+        import numpy as np
+        rng = np.random.default_rng(0x5EED0000 + 16 * self.seed_index + 7)
+        return [int(x) for x in rng.integers(self.N // 4, self.N + 1, size=self.B)]
+
+    def visible_pairs(self, N: int | None = None) -> int:
+        """Exact number of visible (query, key) pairs of one (batch, head) of length N."""
+        N = self.N if N is None else N
         left, right = self.window
         if self.causal:
             right = 0
@@ -50,7 +59,10 @@ class Workload:
         return total
 
     def fwd_flops(self) -> float:
-        """Forward flops by the metric's convention."""
+        """Forward flops by the metric's convention (a variable-length batch counts the
+        pairs of its real lengths)."""
+        if self.varlen:
+            return 4.0 * self.H * self.d * sum(self.visible_pairs(L) for L in self.seq_lengths())
         base = 4.0 * self.B * self.H * self.N * self.N * self.d
         if self.window != (-1, -1) and self.window[0] >= 0:
             return 4.0 * self.B * self.H * self.d * self.visible_pairs()
@@ -82,6 +94,10 @@ WORKLOADS = {
     # C4 with the ALiBi bias of the `alibi_slopes` parameter (page "告别OOM和训练慢…" §4.2)
     "c4a": Workload("c4_causal_alibi_b32h16n2048d64", 32, 16, 2048, 64, True, (-1, -1), True, 3,
                     alibi=True),
+    # C4 as a variable-length batch: real lengths uniform in [512, 2048] (the `lengths` of
+    # the dynamic batching of page "告别OOM和训练慢…" §6); work counted on the real pairs
+    "c4v": Workload("c4_causal_varlen_b32h16n2048d64", 32, 16, 2048, 64, True, (-1, -1), True,
+                    3, varlen=True),
 }
 
 

@@ -109,8 +109,16 @@ typedef struct {
  *                 2^32 (else FA_ERR_INVALID_ARG); t = 0 is no dropout. The backward must get
  *                 the same three values; it regenerates the flags instead of storing them.
  *                 Use a new offset (or seed) per call to draw new flags.
- *   flags         FA_BWD_DETERMINISTIC or 0 (see below).
- * The layout is that of a C struct with natural alignment (48 bytes on LP64).
+ *   flags         FA_BWD_FUSED or 0 (see below).
+ *   seq_lengths   B int32 real lengths, device memory, 4-byte aligned, or NULL: a
+ *                 variable-length batch (the `lengths` of the dynamic batching of page
+ *                 "告别OOM和训练慢…" §6, each sample's real length). Batch entry b holds
+ *                 L_b real tokens at the start of its rows: query i and key j interact only
+ *                 if i < L_b and j < L_b. Rows past L_b get O = 0, LSE = -inf and zero
+ *                 gradients, and no tile that lies wholly past L_b is computed, so a batch
+ *                 costs what its real lengths cost. Values are clamped to [0, N]. The
+ *                 backward must get the same lengths.
+ * The layout is that of a C struct with natural alignment (56 bytes on LP64).
  */
 typedef struct {
     const float *alibi_slopes;
@@ -120,18 +128,21 @@ typedef struct {
     unsigned int flags;                 /* FA_BWD_* bits below; 0 = none */
     unsigned long long dropout_seed;
     unsigned long long dropout_offset;
+    const int *seq_lengths;
 } fa_options_t;
 
 /*
- * flags: FA_BWD_DETERMINISTIC selects the backward whose dQ comes from a separate pass per
- * query tile (fa_bwd_dkdv, then fa_bwd_dq): bit-identical results from run to run. Without
- * it, head_dim 64 uses the fused pass (fa_bwd_fused), which adds each (query tile, key
- * tile) share of dQ into an fp32 accumulator with L2 reductions in no fixed order, so dQ is
- * reproducible to fp32 rounding only (dK and dV are still bit-identical); it does about 2/7
- * less tensor work. head_dim 128 always uses the separate pass. Other bits give
+ * flags: FA_BWD_FUSED selects, at head_dim 64, the backward that computes dK, dV and dQ in
+ * one pass over key tiles (fa_bwd_fused): each (query tile, key tile) pair's share of dQ is
+ * added into an fp32 accumulator by TMA bulk reduce-adds at L2, in no fixed order, so dQ is
+ * reproducible to fp32 rounding only (dK, dV stay bit-identical), and the workspace must
+ * also hold the accumulator (fa_bwd_workspace_bytes_ex). It does 2/7 less tensor work than
+ * the default, but moves P and dS through shared memory and is not faster on B200 (see the
+ * design notes). Without it (and always at head_dim 128) the backward runs the dK/dV pass
+ * and a separate dQ pass: bit-identical results from run to run. Other bits give
  * FA_ERR_INVALID_ARG.
  */
-#define FA_BWD_DETERMINISTIC 1u
+#define FA_BWD_FUSED 1u
 
 /*
  * Forward pass.
@@ -156,13 +167,35 @@ fa_status_t fa_fwd_ex(const void *q, const void *k, const void *v, void *o, floa
                       fa_window_t window, const fa_options_t *options, void *stream);
 
 /*
+ * Forward pass on 8-bit inputs (page "告别OOM和训练慢…" §6 lists FP8 support among the next
+ * steps of the method). q, k, v are e4m3 (OCP FP8 E4M3, one byte per value) tensors of shape
+ * (B, H, N, d); the values they stand for are q * q_scale, k * k_scale, v * v_scale (per-tensor
+ * descales, finite and > 0, else FA_ERR_INVALID_ARG). S = Q K^T and P V run on the tensor core
+ * in FP8 (tcgen05 kind::f8f6f4) with fp32 accumulation; P is rounded to e4m3 for the second
+ * product, so O carries a relative error of a few percent (the 3-bit mantissa of each weight),
+ * while LSE, formed from the fp32 scores, is as exact as in fa_fwd.
+ *   out: o (B,H,N,d) bf16 (the attention of the descaled values); lse (B,H,N) fp32.
+ * d must be 128 (else FA_ERR_UNSUPPORTED). Masks, scale, errors and memory rules as fa_fwd; no
+ * options. There is no FP8 backward.
+ */
+fa_status_t fa_fwd_fp8(const void *q, const void *k, const void *v, float q_scale,
+                       float k_scale, float v_scale, void *o, float *lse, int B, int H, int N,
+                       int d, float scale, int causal, fa_window_t window, void *stream);
+
+/*
  * Bytes of device workspace fa_bwd() needs: two fp32 arrays of B*H*Np values, where
  * Np = N rounded up to a multiple of 128 (the row statistics of the backward, see
- * fa_bwd_preprocess), rounded up to 256 bytes; for head_dim 64, followed by the fused
- * pass's fp32 dQ accumulator of B*H*Np*64 values. (With FA_BWD_DETERMINISTIC the first
- * part alone is enough.) Returns 0 for an empty problem or invalid sizes.
+ * fa_bwd_preprocess), rounded up to 256 bytes. Returns 0 for an empty problem or invalid
+ * sizes.
  */
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * The same for fa_bwd_ex with `options` (may be NULL): with FA_BWD_FUSED at head_dim 64 the
+ * row statistics are followed by the fused pass's fp32 dQ accumulator of B*H*Np*64 values.
+ * Returns 0 for an empty problem, invalid sizes or invalid options.
+ */
+size_t fa_bwd_workspace_bytes_ex(int B, int H, int N, int d, const fa_options_t *options);
 
 /*
  * Backward pass: the gradient of the scalar <O, dO> with respect to q, k and v.
@@ -178,9 +211,8 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
  *   P = exp(scale Q K^T - LSE), dP = dO V^T, dS = P o (dP - delta),
  *   dV = P^T dO, dK = scale dS^T Q             (fa_bwd_dkdv, one pass per key tile)
  *   dQ = scale dS K                            (fa_bwd_dq, one pass per query tile)
- * The kernels run in that order on the stream. At head_dim 64 the two passes are fused
- * into one over key tiles that also adds dQ into an fp32 accumulator, converted to bf16 by
- * a last kernel (see FA_BWD_DETERMINISTIC for what that changes).
+ * The kernels run in that order on the stream; results are deterministic. (fa_bwd_ex with
+ * FA_BWD_FUSED replaces the two passes by one at head_dim 64, see FA_BWD_FUSED.)
  */
 fa_status_t fa_bwd(const void *q, const void *k, const void *v, const void *o,
                    const void *dout, const float *lse, void *dq, void *dk, void *dv,
@@ -226,8 +258,8 @@ fa_status_t fa_bwd_alibi(const void *q, const void *k, const void *v, const void
  *   workspace[B*H*Np .. 2*B*H*Np)   delta = rowsum(dout * o), summed in fp32
  *                                   (o + options->o_low when o_low is given)
  * The padding lets each 128-row tile of both arrays be fetched with one bulk copy.
- * At head_dim 64 without FA_BWD_DETERMINISTIC it also zeroes the fused pass's dQ
- * accumulator (the workspace must then hold fa_bwd_workspace_bytes()).
+ * With FA_BWD_FUSED at head_dim 64 it also zeroes the fused pass's dQ accumulator (the
+ * workspace must then hold fa_bwd_workspace_bytes_ex() bytes).
  * `options` may be NULL; its o_low and flags are used here.
  */
 fa_status_t fa_bwd_preprocess(const void *o, const void *dout, const float *lse,
@@ -251,8 +283,8 @@ fa_status_t fa_bwd_dq(const void *q, const void *k, const void *v, const void *d
 /*
  * Step 2 of the fused backward alone (head_dim 64, else FA_ERR_UNSUPPORTED): dk, dv, and
  * dQ / scale added into the accumulator part of `workspace` (which fa_bwd_preprocess,
- * called without FA_BWD_DETERMINISTIC, zeroed). `options`: alibi_slopes, key_padding and
- * dropout, or NULL.
+ * called with FA_BWD_FUSED, zeroed). `options`: alibi_slopes, key_padding, dropout and
+ * seq_lengths, or NULL.
  */
 fa_status_t fa_bwd_fused(const void *q, const void *k, const void *v, const void *dout,
                          void *workspace, void *dk, void *dv,
@@ -269,8 +301,8 @@ fa_status_t fa_bwd_dq_convert(void *workspace, void *dq, int B, int H, int N, in
  *
  * Some callers may not allocate: an engine that reserves all of its device memory up
  * front and may not grow it while serving, or a framework plugin whose enqueue step
- * is not allowed to call cudaMalloc. fa_bwd_noalloc computes exactly what fa_bwd with
- * FA_BWD_DETERMINISTIC computes, with the same arguments except the workspace: its row
+ * is not allowed to call cudaMalloc. fa_bwd_noalloc computes exactly what fa_bwd
+ * computes, with the same arguments except the workspace: its row
  * statistics go to a fixed 8 MiB array in device memory that the library holds on every
  * GPU that loads it, until the process exits. It calls no cudaMalloc, cudaFree or other
  * allocating routine.

@@ -32,20 +32,22 @@ def rel_frob(x: np.ndarray, ref: np.ndarray) -> float:
 
 def run_library(inp: dict, scale: float, causal: bool, window, backward: bool = True,
                 alibi=None, key_padding=None, residual: bool = True, dropout=None,
-                deterministic: bool = False) -> dict:
+                fused: bool = False, lengths=None) -> dict:
     """Runs the forward (and backward) on cuda:0 through the C ABI and returns host tensors.
     `alibi`: H slopes; `key_padding`: a (B, N) bool host tensor (True = padded key);
     `residual`: the forward keeps O - bf16(O) for the backward's delta (the training path
     the benchmark times); False runs plain fa_fwd / fa_bwd; `dropout`: (p, seed, offset);
-    `deterministic`: the backward with the separate dQ pass."""
+    `fused`: the fused backward (head_dim 64); `lengths`: B real lengths of a
+    variable-length batch."""
     ensure_built()
     dev = torch.device("cuda:0")
     q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
     slopes = None if alibi is None else torch.tensor(alibi, dtype=torch.float32, device=dev)
     kpad = None if key_padding is None else key_padding.to(dev)
+    lens = None if lengths is None else torch.tensor(lengths, dtype=torch.int32, device=dev)
     res = fa.attention_forward(q, k, v, scale, causal, window, alibi_slopes=slopes,
                                key_padding=kpad, keep_residual=residual and backward,
-                               dropout=dropout)
+                               dropout=dropout, seq_lengths=lens)
     o, lse = res[0], res[1]
     o_low = res[2] if len(res) > 2 else None
     out = {"o": o, "lse": lse}
@@ -53,7 +55,8 @@ def run_library(inp: dict, scale: float, causal: bool, window, backward: bool = 
         do = inp["do"].to(dev)
         dq, dk, dv = fa.attention_backward(q, k, v, o, lse, do, scale, causal, window,
                                            alibi_slopes=slopes, key_padding=kpad, o_low=o_low,
-                                           dropout=dropout, deterministic=deterministic)
+                                           dropout=dropout, fused=fused,
+                                           seq_lengths=lens)
         out.update(dq=dq, dk=dk, dv=dv)
     torch.cuda.synchronize()
     assert fa.fa_debug_status() == 0
@@ -61,7 +64,8 @@ def run_library(inp: dict, scale: float, causal: bool, window, backward: bool = 
 
 
 def compare(inp: dict, out: dict, scale: float, causal: bool, window, heads=None,
-            backward: bool = True, alibi=None, key_padding=None, dropout=None) -> dict:
+            backward: bool = True, alibi=None, key_padding=None, dropout=None,
+            lengths=None) -> dict:
     """Errors of the library's outputs against the oracle, on all heads or on the listed
     (b, h) pairs (each head is an independent problem, so a subset is exact); `alibi`: the
     H slopes the library ran with, if any; `key_padding`: its (B, N) flags, if any.
@@ -84,10 +88,10 @@ def compare(inp: dict, out: dict, scale: float, causal: bool, window, heads=None
             # one batch entry per sampled head, in the layout pick() gives: (1, n, N, d)
             # tensors need (1, N) flags per head, so compare head by head instead
             raise ValueError("sampled heads with key padding are not supported")
-    if dropout is not None and heads is not None:
+    if (dropout is not None or lengths is not None) and heads is not None:
         # the keep flags depend on the (batch, head) index, which sampling renumbers
         raise ValueError("sampled heads with dropout are not supported")
-    o_ref, lse_ref = oracle.fwd(q, k, v, scale, causal, window, slopes, kp, dropout)
+    o_ref, lse_ref = oracle.fwd(q, k, v, scale, causal, window, slopes, kp, dropout, lengths)
     lse = pick(out["lse"])
     dead = np.isneginf(lse_ref)
     assert np.array_equal(np.isneginf(lse), dead), "rows with no visible key differ"
@@ -98,7 +102,7 @@ def compare(inp: dict, out: dict, scale: float, causal: bool, window, heads=None
     if backward:
         do = pick(inp["do"])
         dq_ref, dk_ref, dv_ref = oracle.bwd(q, k, v, do, scale, causal, window, slopes, kp,
-                                            dropout)
+                                            dropout, lengths)
         errs["dq"] = rel_frob(pick(out["dq"]), dq_ref)
         errs["dk"] = rel_frob(pick(out["dk"]), dk_ref)
         errs["dv"] = rel_frob(pick(out["dv"]), dv_ref)

@@ -91,10 +91,9 @@ def test_empty_problem_is_a_no_op(lib):
 
 
 def test_workspace_size(lib):
-    # two fp32 arrays (LSE*log2e and delta) of B*H rows padded to whole 128-row tiles; at
-    # head_dim 64 followed by the fused pass's fp32 dQ accumulator (64 values per row)
-    assert lib.fa_bwd_workspace_bytes(2, 8, 4096, 64) == 2 * 2 * 8 * 4096 * 4 * (1 + 32)
-    assert lib.fa_bwd_workspace_bytes(1, 1, 3, 64) == 2 * 128 * 4 + 128 * 64 * 4
+    # two fp32 arrays (LSE*log2e and delta) of B*H rows padded to whole 128-row tiles
+    assert lib.fa_bwd_workspace_bytes(2, 8, 4096, 64) == 2 * 2 * 8 * 4096 * 4
+    assert lib.fa_bwd_workspace_bytes(1, 1, 3, 64) == 2 * 128 * 4
     assert lib.fa_bwd_workspace_bytes(1, 2, 129, 128) == 2 * 2 * 256 * 4
     assert lib.fa_bwd_workspace_bytes(1, 1, 3, 80) == 0
 
@@ -143,14 +142,20 @@ def test_options_are_checked(lib):
     assert fwd_ex(O(dropout_p=float("nan"))) == 1
     assert fwd_ex(O(dropout_p=0.1, dropout_offset=1 << 32)) == 1  # offset wider than 32 bits
     assert fwd_ex(O(flags=2)) == 1                  # unknown flag
+    assert fwd_ex(O(seq_lengths=A + 2)) == 3        # lengths not 4-byte aligned
     assert fwd_ex(O(key_padding=A + 1), q=None) == 1
     assert fwd_ex(None, d=96) == 2
     assert bwd_ex(O(o_low=A + 4)) == 3
     assert bwd_ex(O(dropout_p=1.5)) == 1
     assert bwd_ex(None, ws_bytes=8) == 4
-    # the fused backward (head_dim 64) needs the dQ accumulator; the deterministic one not
+    # the fused backward (head_dim 64) needs the dQ accumulator as well
     stats = 2 * 2 * 128 * 4
-    assert bwd_ex(None, ws_bytes=stats) == 4
+    assert bwd_ex(O(flags=1), ws_bytes=stats) == 4
+    assert lib.fa_bwd_workspace_bytes_ex(1, 2, 128, 64, ctypes.byref(O(flags=1))) == \
+        stats + 2 * 128 * 64 * 4
+    assert lib.fa_bwd_workspace_bytes_ex(1, 2, 128, 64, None) == stats
+    assert lib.fa_bwd_workspace_bytes_ex(1, 2, 128, 128, ctypes.byref(O(flags=1))) == stats
+    assert lib.fa_bwd_workspace_bytes_ex(1, 2, 128, 64, ctypes.byref(O(flags=4))) == 0
     assert lib.fa_bwd_fused(A, A, A, A, A, A, A, 1, 1, 128, 128, 0.1, 0, W(-1, -1), None,
                             None) == 2   # the fused pass is for head_dim 64
     assert lib.fa_bwd_dq_convert(A, None, 1, 1, 128, 64, 0.1, None) == 1
@@ -160,13 +165,28 @@ def test_options_are_checked(lib):
                          O(alibi_slopes=A + 2, dropout_p=0.5), None) == 0
 
 
+def test_fp8_forward_rejects_bad_arguments(lib):
+    def fwd8(q=A, d=128, qs=1.0, ks=1.0, vs=1.0, scale=0.09, o=A):
+        return lib.fa_fwd_fp8(q, A, A, qs, ks, vs, o, A, 1, 2, 128, d, scale, 1, W(-1, -1), None)
+
+    assert fwd8(d=64) == 2            # the e4m3 forward is for head_dim 128
+    assert fwd8(qs=0.0) == 1
+    assert fwd8(ks=float("nan")) == 1
+    assert fwd8(vs=-1.0) == 1
+    assert fwd8(scale=0.0) == 1
+    assert fwd8(q=None) == 1
+    assert fwd8(o=A + 2) == 3
+    assert lib.fa_fwd_fp8(None, None, None, 1.0, 1.0, 1.0, None, None, 0, 2, 128, 128, 0.1, 0,
+                          W(-1, -1), None) == 0
+
+
 def test_options_struct_layout():
     import ctypes
     O = fa.fa_options_t
-    assert ctypes.sizeof(O) == 48
+    assert ctypes.sizeof(O) == 56
     assert [O.alibi_slopes.offset, O.key_padding.offset, O.o_low.offset, O.dropout_p.offset,
-            O.flags.offset, O.dropout_seed.offset, O.dropout_offset.offset] == [
-                0, 8, 16, 24, 28, 32, 40]
+            O.flags.offset, O.dropout_seed.offset, O.dropout_offset.offset,
+            O.seq_lengths.offset] == [0, 8, 16, 24, 28, 32, 40, 48]
 
 
 def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):

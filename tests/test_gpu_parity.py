@@ -204,30 +204,30 @@ def test_zero_queries_closed_form():
 
 
 def test_deterministic():
-    """With FA_BWD_DETERMINISTIC, two runs give bit-identical O, LSE, dQ, dK and dV (no
-    atomics anywhere on that path)."""
+    """Two runs give bit-identical O, LSE, dQ, dK and dV (no atomics on the default path)."""
     w = WORKLOADS["c3"]
     inp = inputs(w.B, w.H, w.N, w.d, w.seed_index)
-    a = G.run_library(inp, w.softmax_scale, True, (-1, -1), deterministic=True)
-    b = G.run_library(inp, w.softmax_scale, True, (-1, -1), deterministic=True)
+    a = G.run_library(inp, w.softmax_scale, True, (-1, -1))
+    b = G.run_library(inp, w.softmax_scale, True, (-1, -1))
     for n in a:
         assert torch.equal(a[n], b[n]), n
 
 
 def test_fused_backward_run_to_run():
-    """The fused backward (head_dim 64): O, LSE, dK and dV are bit-identical from run to run;
-    dQ, added up in fp32 in no fixed order, differs by fp32 rounding only (far below bf16's
-    resolution), and both runs agree with the deterministic backward within the bounds."""
+    """The fused backward (FA_BWD_FUSED, head_dim 64): O, LSE, dK and dV are bit-identical
+    from run to run; dQ, added up in fp32 in no fixed order, differs by fp32 rounding only
+    (far below bf16's resolution), and both runs agree with the default backward within the
+    bounds."""
     w = WORKLOADS["c3"]
     inp = inputs(w.B, w.H, w.N, w.d, w.seed_index)
-    a = G.run_library(inp, w.softmax_scale, True, (-1, -1))
-    b = G.run_library(inp, w.softmax_scale, True, (-1, -1))
-    c = G.run_library(inp, w.softmax_scale, True, (-1, -1), deterministic=True)
+    a = G.run_library(inp, w.softmax_scale, True, (-1, -1), fused=True)
+    b = G.run_library(inp, w.softmax_scale, True, (-1, -1), fused=True)
+    c = G.run_library(inp, w.softmax_scale, True, (-1, -1))
     for n in ("o", "lse", "dk", "dv"):
         assert torch.equal(a[n], b[n]), n
     spread = G.rel_frob(synth.to_f64(a["dq"]), synth.to_f64(b["dq"]))
     to_det = G.rel_frob(synth.to_f64(a["dq"]), synth.to_f64(c["dq"]))
-    print("fused dQ run-to-run relative spread %.3g, vs deterministic %.3g" % (spread, to_det))
+    print("fused dQ run-to-run relative spread %.3g, vs the default path %.3g" % (spread, to_det))
     assert spread <= 1e-3 and to_det <= 2e-3
     errs = G.compare(inp, a, w.softmax_scale, True, (-1, -1))
     G.assert_within_bounds(errs, "fused")
@@ -235,16 +235,26 @@ def test_fused_backward_run_to_run():
 
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("mode", ["none", "causal", "win100_30"])
-def test_deterministic_path_small_and_ragged(d, mode):
-    """The three-kernel backward (separate dQ pass) against the oracle at head_dim 64, where
-    the default is the fused pass (and at 128, where both are the same path)."""
+def test_fused_path_small_and_ragged(d, mode):
+    """The fused backward against the oracle (at head_dim 128 the flag selects the same
+    separate passes)."""
     causal, window = MODES[mode]
     for N in (17, 300):
         inp = inputs(2, 2, N, d, 150 + N + d)
         scale = 1.0 / np.sqrt(d)
-        out = G.run_library(inp, scale, causal, window, deterministic=True)
+        out = G.run_library(inp, scale, causal, window, fused=True)
         errs = G.compare(inp, out, scale, causal, window)
         G.assert_within_bounds(errs, (N, d, mode))
+
+
+@pytest.mark.parametrize("name", ["c3", "c4"])
+def test_fused_path_full_size(name):
+    w = WORKLOADS[name]
+    inp = inputs(w.B, w.H, w.N, w.d, w.seed_index)
+    out = G.run_library(inp, w.softmax_scale, w.causal, w.window, fused=True)
+    heads = None if w.B * w.H * w.N <= 2 * 8 * 4096 else _sampled_heads(w)
+    errs = G.compare(inp, out, w.softmax_scale, w.causal, w.window, heads)
+    G.assert_within_bounds(errs, name)
 
 
 @pytest.mark.parametrize("d", [64, 128])

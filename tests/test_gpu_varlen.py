@@ -1,0 +1,107 @@
+"""Variable-length batches (fa_options_t.seq_lengths: each sample's real length, the
+`lengths` of the dynamic batching of page "告别OOM和训练慢…(含A100环境配置)" §6) against the
+fp64 oracle with the same lengths, forward and backward (separate and fused dQ), in every
+mask mode, both head sizes, with lengths that end inside a tile, on a tile boundary, at 1,
+at 0 and at N; with key padding, ALiBi and dropout on top; with many items per CTA. Rows
+past a length must be exactly zero (LSE -inf), and the tiles past it are not computed."""
+import numpy as np
+import pytest
+import torch
+
+import gpu_helpers as G
+from exact_attention_126_b200 import synth
+from exact_attention_126_b200.workloads import alibi_slopes
+
+pytestmark = pytest.mark.gpu
+
+MODES = {
+    "none": (False, (-1, -1)),
+    "causal": (True, (-1, -1)),
+    "win64_0": (False, (64, 0)),
+    "win100_30": (False, (100, 30)),
+}
+
+
+def _lengths(B, N, seed):
+    rng = np.random.default_rng(seed)
+    base = [N, 0, 1, 128 if N > 128 else N, N - 1]
+    return [base[b] if b < len(base) else int(rng.integers(1, N + 1)) for b in range(B)]
+
+
+def check_past_length(out, lengths):
+    for b, L in enumerate(lengths):
+        assert np.all(out["o"][b, :, L:].float().numpy() == 0.0)
+        assert np.all(np.isneginf(out["lse"][b, :, L:].numpy()))
+        for g in ("dq", "dk", "dv"):
+            if g in out:
+                assert np.all(out[g][b, :, L:].float().numpy() == 0.0), g
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [129, 300, 520])
+@pytest.mark.parametrize("mode", list(MODES))
+def test_varlen_small_and_ragged(N, d, mode):
+    causal, window = MODES[mode]
+    B, H = 6, 2
+    lens = _lengths(B, N, N + d)
+    inp = synth.attention_inputs(B, H, N, d, 2000 + N + d)
+    scale = 1.0 / np.sqrt(d)
+    out = G.run_library(inp, scale, causal, window, lengths=lens)
+    errs = G.compare(inp, out, scale, causal, window, lengths=lens)
+    G.assert_within_bounds(errs, (N, d, mode, lens))
+    check_past_length(out, lens)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_varlen_fused_backward(d):
+    B, H, N = 5, 3, 400
+    lens = _lengths(B, N, 7)
+    inp = synth.attention_inputs(B, H, N, d, 2100 + d)
+    scale = 1.0 / np.sqrt(d)
+    out = G.run_library(inp, scale, True, (-1, -1), lengths=lens, fused=True)
+    errs = G.compare(inp, out, scale, True, (-1, -1), lengths=lens)
+    G.assert_within_bounds(errs, d)
+    check_past_length(out, lens)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_varlen_with_padding_alibi_dropout(d):
+    B, H, N = 4, 2, 300
+    lens = [300, 170, 5, 129]
+    inp = synth.attention_inputs(B, H, N, d, 2200 + d)
+    flags = np.zeros((B, N), dtype=bool)
+    flags[0, 250:] = True
+    flags[1, ::4] = True
+    kp = torch.from_numpy(flags)
+    slopes = alibi_slopes(H)
+    scale = 1.0 / np.sqrt(d)
+    drop = (0.2, 99, 4)
+    out = G.run_library(inp, scale, True, (-1, -1), alibi=slopes, key_padding=kp, dropout=drop,
+                        lengths=lens)
+    errs = G.compare(inp, out, scale, True, (-1, -1), alibi=slopes, key_padding=kp,
+                     dropout=drop, lengths=lens)
+    G.assert_within_bounds(errs, d)
+    check_past_length(out, lens)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_varlen_many_items_per_cta(d):
+    """More items than SMs, most of them past their entry's length (skipped by every role)."""
+    B, H, N = 8, 16, 640
+    lens = [640, 1, 300, 0, 129, 512, 77, 640]
+    inp = synth.attention_inputs(B, H, N, d, 2300 + d)
+    scale = 1.0 / np.sqrt(d)
+    out = G.run_library(inp, scale, True, (-1, -1), lengths=lens)
+    errs = G.compare(inp, out, scale, True, (-1, -1), lengths=lens)
+    G.assert_within_bounds(errs, d)
+    check_past_length(out, lens)
+
+
+def test_full_lengths_are_no_restriction():
+    """seq_lengths = N everywhere: bit-identical to a call without lengths."""
+    B, H, N, d = 2, 2, 300, 64
+    inp = synth.attention_inputs(B, H, N, d, 2400)
+    a = G.run_library(inp, 0.125, True, (-1, -1), lengths=[N, N])
+    b = G.run_library(inp, 0.125, True, (-1, -1))
+    for n in a:
+        assert torch.equal(a[n], b[n]), n

@@ -2,8 +2,7 @@
 that reserved all of its memory up front, a plugin whose enqueue step may not call
 cudaMalloc). It must give what fa_bwd gives, call after call, using the library's own
 fixed device array instead of a caller workspace. The two run the same deterministic
-kernels on the same statistics (the backward with the separate dQ pass), so their outputs
-must be bit-identical.
+kernels on the same statistics, so their outputs must be bit-identical.
 
 This file is collected last on purpose: should it fail, a run that stops at the first
 failure has run every other test already. It passes alone in a fresh process as well.
@@ -28,8 +27,7 @@ def _problem(B, H, N, d, causal, window, seed):
     q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
     scale = 1.0 / np.sqrt(d)
     o, lse = fa.attention_forward(q, k, v, scale, causal, window)
-    # the deterministic backward: the one fa_bwd_noalloc runs
-    ref = fa.attention_backward(q, k, v, o, lse, do, scale, causal, window, deterministic=True)
+    ref = fa.attention_backward(q, k, v, o, lse, do, scale, causal, window)
     return (q, k, v, o, do, lse, scale), ref
 
 
