@@ -204,6 +204,10 @@ class Problem:
             self.q, self.k, self.v, self.do = (
                 torch.randn(shape, generator=g, device=dev, dtype=torch.float32)
                 .to(torch.bfloat16) for _ in range(4))
+        if w.fp8:
+            # e4m3 copies of the inputs, descales 1 (N(0, 1) values fit e4m3's range)
+            self.q8, self.k8, self.v8 = (t.to(torch.float8_e4m3fn) for t in
+                                         (self.q, self.k, self.v))
         self.o = torch.empty_like(self.q)
         self.o_low = torch.empty_like(self.q)
         self.lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
@@ -232,6 +236,12 @@ class Problem:
         stream = self.stream
         if evs is not None:
             evs[0].record(stream)
+        if w.fp8:
+            fa.fa_fwd_fp8(self.q8, self.k8, self.v8, 1.0, 1.0, 1.0, self.o, self.lse,
+                          w.softmax_scale, w.causal, w.window, sp)
+            if evs is not None:
+                evs[1].record(stream)
+            return
         fa.fa_fwd_ex(self.q, self.k, self.v, self.o, self.lse, self.opt, w.softmax_scale,
                      w.causal, w.window, sp)
         if evs is not None:
@@ -368,6 +378,10 @@ def run_ours(args, w, rank, world, local_rank):
                              ("dk", prob.dk), ("dv", prob.dv))}
     in_names = ("q", "k", "v", "do") if w.backward else ("q", "k", "v")
     out_names = ("o", "lse", "dq", "dk", "dv") if w.backward else ("o", "lse")
+    if w.fp8:
+        # the e4m3 forward's inputs are e4m3 on the host too
+        inp_host = {n: inp_host[n].to(torch.float8_e4m3fn).pin_memory() for n in in_names}
+        q, k, v = prob.q8, prob.k8, prob.v8
     h2d_bytes = sum(inp_host[n].numel() * inp_host[n].element_size() for n in in_names)
     d2h_bytes = sum(host_out[n].numel() * host_out[n].element_size() for n in out_names)
 
@@ -375,9 +389,13 @@ def run_ours(args, w, rank, world, local_rank):
         for n, t in zip(("q", "k", "v", "do"), (q, k, v, do)):
             if n in in_names:
                 t.copy_(inp_host[n], non_blocking=True)
-        res = fa.attention_forward(q, k, v, w.softmax_scale, w.causal, w.window, sp,
-                                   alibi_slopes=prob.slopes, keep_residual=w.backward,
-                                   seq_lengths=prob.lengths)
+        if w.fp8:
+            res = fa.attention_forward_fp8(q, k, v, scale=w.softmax_scale, causal=w.causal,
+                                           window=w.window, stream=sp)
+        else:
+            res = fa.attention_forward(q, k, v, w.softmax_scale, w.causal, w.window, sp,
+                                       alibi_slopes=prob.slopes, keep_residual=w.backward,
+                                       seq_lengths=prob.lengths)
         host_out["o"].copy_(res[0], non_blocking=True)
         host_out["lse"].copy_(res[1], non_blocking=True)
         if w.backward:
@@ -473,7 +491,7 @@ def run_ours(args, w, rank, world, local_rank):
         "data": "synthetic (seeded i.i.d. N(0,1) bf16, SplitMix64 + Box-Muller)",
         "config": {
             "workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
-            "window": list(w.window), "alibi": w.alibi, "varlen": w.varlen,
+            "window": list(w.window), "alibi": w.alibi, "varlen": w.varlen, "fp8": w.fp8,
             "pass": "fwd+bwd" if w.backward else "fwd",
             "path": ("plain: delta from the bf16 O" if args.plain else
                      "training path: forward keeps O - bf16(O) for the backward's delta")
@@ -601,12 +619,13 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="c4", help="c1, c2, c3, c4, c5c, c5w, c4a or c4v")
+    ap.add_argument("--workload", default="c4",
+                    help="c1, c2, c3, c4, c5c, c5w, c4a, c4v or c5f8")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--also", default="c2,c3,c4,c5c,c5w,c4v",
+    ap.add_argument("--also", default="c2,c3,c4,c5c,c5w,c4v,c5f8",
                     help="other workloads timed at full size in the same run (comma list)")
     ap.add_argument("--fused", action="store_true",
                     help="time the fused backward (dQ by fp32 bulk reductions) at head_dim 64")

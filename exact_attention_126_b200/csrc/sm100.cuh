@@ -21,7 +21,7 @@ static __device__ int g_fa_status;
 
 constexpr int kStatusTimeout = 6;                         // FA_ERR_TIMEOUT
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
-constexpr uint32_t kWaitLimitPolls = 1u << 28;              // backstop if the timer stalls
+constexpr uint32_t kWaitLimitPolls = 1u << 24;              // backstop if the timer stalls
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -73,6 +73,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
+// The same test, but a thread whose phase is not complete yet may be suspended by the
+// hardware until it completes or `hint_ns` nanoseconds have passed, instead of returning at
+// once: a waiting warp then takes no issue slots from the warps that do the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return done != 0;
+}
+
+constexpr uint32_t kSuspendHintNs = 1000000;  // 1 ms: a wait polls at most ~2000 times
+
 // Gives up a wait that ran out of time: raises the CTA's abort flag (so that its other
 // roles stop too) and records FA_ERR_TIMEOUT in the device status word.
 __device__ __forceinline__ void wait_timed_out(volatile int* abort_flag) {
@@ -90,13 +108,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 31u) == 0) {
-      if (abort_flag != nullptr && *abort_flag) return false;
-      if (global_ns() - t0 > kWaitLimitNs || n > kWaitLimitPolls) {
-        wait_timed_out(abort_flag);
-        return false;
-      }
+    // each test may suspend the thread until the phase completes (or the hint runs out), so
+    // the abort flag and the clock are looked at on every turn
+    if (mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) return true;
+    if (abort_flag != nullptr && *abort_flag) return false;
+    if (global_ns() - t0 > kWaitLimitNs || n > kWaitLimitPolls) {
+      wait_timed_out(abort_flag);
+      return false;
     }
   }
 }

@@ -30,6 +30,7 @@ class Workload:
     scale: float | None = None  # None: 1/sqrt(d)
     alibi: bool = False         # linear bias -m_h |i - j| with the slopes of alibi_slopes()
     varlen: bool = False        # variable-length batch with the lengths of seq_lengths()
+    fp8: bool = False           # e4m3 Q, K, V (forward only)
 
     @property
     def softmax_scale(self) -> float:
@@ -98,6 +99,9 @@ WORKLOADS = {
     # the dynamic batching of page "告别OOM和训练慢…" §6); work counted on the real pairs
     "c4v": Workload("c4_causal_varlen_b32h16n2048d64", 32, 16, 2048, 64, True, (-1, -1), True,
                     3, varlen=True),
+    # the long-sequence causal forward on e4m3 inputs (FP8 support, page "告别OOM和训练慢…" §6)
+    "c5f8": Workload("c5_causal_fp8_fwd_b2h32n8192d128", 2, 32, 8192, 128, True, (-1, -1), False,
+                     4, fp8=True),
 }
 
 
