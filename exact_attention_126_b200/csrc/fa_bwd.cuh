@@ -347,8 +347,12 @@ __device__ __forceinline__ void bwd_teardown(uint32_t tmem, int warp) {
 // stage Y0 = Q_i with the LSE (log2 units) and delta of its 128 rows, Y1 = dO_i.
 // TMEM: S^T in kSBufs buffers (two for head_dim 64, so that S^T of the next query tile
 // is computed while the softmax works on this one), dP^T, dK, dV. Warpgroup h writes its
-// bf16 part of P^T (dS^T) over the first 16 of its own 32 fp32 columns of S^T (dP^T), so
-// the A operand of dV (dK) takes K-step kk from column packed_col(kk).
+// bf16 part of P^T over the first 16 of its own 32 fp32 columns of S^T, so the A operand
+// of dV takes K-step kk from column packed_col(kk). With two S^T buffers, dS^T goes over
+// the other 16 of those columns (packed_col(kk) + 16), whose scores are in registers by
+// then: dP^T is free as soon as the softmax has loaded it, and dP^T of the next query
+// tile is computed while dS^T and dK of this one are. With one buffer, dS^T goes over
+// the first half of the group's dP^T columns and dP^T waits for dK.
 // Two MMA issuers: one computes S^T and dP^T of each query tile in order, the other
 // dV += P^T dO and dK += dS^T Q as soon as the softmax publishes P^T and dS^T. Tile
 // counters (for barrier parities) run over all items of the CTA.
@@ -371,15 +375,18 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
   constexpr bool kKpad = (kFeat & kFeatKpad) != 0;
   constexpr bool kDropout = (kFeat & kFeatDropout) != 0;
   constexpr int kSBufs = (D == 64) ? 2 : 1;
+  constexpr bool kDsInS = kSBufs == 2;               // dS^T over the second half of S^T
   constexpr uint32_t tS = 0;                         // + 128 * buffer
   constexpr uint32_t tDP = 128 * kSBufs, tDK = tDP + 128, tDV = tDK + D;
   static_assert(tDV + D <= C::kTmemCols, "tensor memory columns");
-  // per S^T buffer: S^T full, P^T full, dV done (dV read that buffer's P^T); dP^T full,
-  // dS^T full, dK done, dK/dV read by the epilogue, dK/dV of the item complete. Every
-  // barrier that one side may complete twice before the other has waited once is kept
-  // per buffer, so that no parity wait can mistake a later phase for the one it wants.
-  constexpr int bSFull = C::bA + 0, bPFull = C::bA + 2, bDVDone = C::bA + 4,
-                bDPFull = C::bA + 6, bDSFull = C::bA + 7, bDKDone = C::bA + 8,
+  // per S^T buffer: S^T full, P^T full, buffer free (the last product that reads it, dV
+  // or with kDsInS dK, has completed); dP^T full, dS^T full, dP^T free (loaded by the
+  // softmax with kDsInS, else read by dK), dK/dV read by the epilogue, dK/dV of the item
+  // complete. Every barrier that one side may complete twice before the other has waited
+  // once is kept per buffer, so that no parity wait can mistake a later phase for the one
+  // it wants.
+  constexpr int bSFull = C::bA + 0, bPFull = C::bA + 2, bSFree = C::bA + 4,
+                bDPFull = C::bA + 6, bDSFull = C::bA + 7, bDPFree = C::bA + 8,
                 bAccFree = C::bA + 9, bAccReady = C::bA + 10, bStaged = C::bA + 11;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -408,12 +415,12 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(bSFull + b), 1);
       mbar_init(bar(bPFull + b), C::kSoftmax / 32);
-      mbar_init(bar(bDVDone + b), 1);
+      mbar_init(bar(bSFree + b), 1);
       mbar_init(bar(C::bMmaFin + b), 1);
     }
     mbar_init(bar(bDPFull), 1);
     mbar_init(bar(bDSFull), C::kSoftmax / 32);
-    mbar_init(bar(bDKDone), 1);
+    mbar_init(bar(bDPFree), kDsInS ? C::kSoftmax / 32 : 1);
     mbar_init(bar(bAccFree), C::kSoftmax / 32);
     mbar_init(bar(bAccReady), 1);
     mbar_init(bar(bStaged), C::kSoftmax / 32);
@@ -496,10 +503,11 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
         if (!mbar_wait(bar(C::bXFull + xb), xu & 1, abort_flag)) break;
         for (int i = i_lo; i <= i_hi; ++i, ++t) {
           const int b = t % kSBufs, s0 = t % C::kStages0, s1 = t % C::kStages1;
-          // S^T = K_j Q_i^T, once dV has read the P^T its buffer held
+          // S^T = K_j Q_i^T, once the products that read its buffer's P^T (and dS^T) have
+          // completed
           if (!mbar_wait(bar(C::bY0Full + s0), (t / C::kStages0) & 1, abort_flag) ||
               (t >= kSBufs &&
-               !mbar_wait(bar(bDVDone + b), ((t / kSBufs) - 1) & 1, abort_flag))) {
+               !mbar_wait(bar(bSFree + b), ((t / kSBufs) - 1) & 1, abort_flag))) {
             ok = false;
             break;
           }
@@ -513,9 +521,9 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
           }
           tc_commit(bar(bSFull + b));
           tc_commit(bar(C::bY0Empty + s0));
-          // dP^T = V_j dO_i^T, once dK has read the dS^T of the previous tile
+          // dP^T = V_j dO_i^T, once the previous tile's dP^T is free
           if (!mbar_wait(bar(C::bY1Full + s1), (t / C::kStages1) & 1, abort_flag) ||
-              (t >= 1 && !mbar_wait(bar(bDKDone), (t - 1) & 1, abort_flag))) {
+              (t >= 1 && !mbar_wait(bar(bDPFree), (t - 1) & 1, abort_flag))) {
             ok = false;
             break;
           }
@@ -567,7 +575,7 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
                    sdesc_sw128(sb + C::kY1 + s1 * C::kTile + kk * 2048, C::kRegionBytes, 1024),
                    idA, (!first || kk > 0) ? 1u : 0u);
           tc_commit(bar(C::bY1Empty + s1));
-          tc_commit(bar(bDVDone + b));
+          if (!kDsInS) tc_commit(bar(bSFree + b));
           // dK += dS^T Q_i
           if (!mbar_wait(bar(C::bY0Full + s0), (t / C::kStages0) & 1, abort_flag) ||
               !mbar_wait(bar(bDSFull), t & 1, abort_flag)) {
@@ -577,11 +585,12 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kBlock / 16; ++kk)
-            mma_ts(tmem + tDK, tmem + tDP + packed_col(kk),
+            mma_ts(tmem + tDK,
+                   tmem + (kDsInS ? tS + 128u * b + 16u : tDP) + packed_col(kk),
                    sdesc_sw128(sb + C::kY0 + s0 * C::kTile + kk * 2048, C::kRegionBytes, 1024),
                    idA, (!first || kk > 0) ? 1u : 0u);
           tc_commit(bar(C::bY0Empty + s0));
-          tc_commit(bar(bDKDone));
+          tc_commit(bar(kDsInS ? bSFree + b : bDPFree));
           if (i == i_hi) tc_commit(bar(bAccReady));  // dK, dV of the item are complete
         }
         ++items;
@@ -715,6 +724,11 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
         tc_fence_after();
         float dp[NC];
         load_cols32(tmem + lane_base + tDP + NC * h, dp);
+        if (kDsInS) {
+          // dP^T is in registers: the next query tile's dP^T may overwrite it
+          tc_fence_before();
+          mbar_arrive_warp(bar(bDPFree));
+        }
         if (kDropout) {
           // dP o Z / (1 - p'): the gradient reaching the weights before dropout
           const float ks = a.drop.keep_scale;
@@ -729,8 +743,9 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
           w[e] = pack_bf16x2(p[r0] * (dp[r0] - d4.x), p[r0 + 1] * (dp[r0 + 1] - d4.y));
           w[e + 1] = pack_bf16x2(p[r0 + 2] * (dp[r0 + 2] - d4.z), p[r0 + 3] * (dp[r0 + 3] - d4.w));
         }
-        // bf16 dS^T goes over the first half of this warpgroup's own fp32 dP^T columns
-        tmem_st16(tmem + lane_base + tDP + NC * h, w);
+        // bf16 dS^T goes over the second half of this warpgroup's own fp32 S^T columns
+        // (kDsInS) or the first half of its dP^T columns
+        tmem_st16(kDsInS ? tSb + 16 : tmem + lane_base + tDP + NC * h, w);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive_warp(bar(bDSFull));
