@@ -218,7 +218,7 @@ struct BwdCfgT {
 template <int D>
 using DkdvCfg = BwdCfgT<D, (D == 64) ? 2 : 1, (D == 64) ? 4 : 2, (D == 64) ? 4 : 2, true>;
 template <int D>
-using DqCfg = BwdCfgT<D, (D == 64) ? 2 : 1, (D == 64) ? 5 : 3, (D == 64) ? 4 : 2, false>;
+using DqCfg = BwdCfgT<D, (D == 64) ? 2 : 1, (D == 64) ? 5 : 3, (D == 64) ? 5 : 2, false>;
 
 // Waits until every copy a ring's producer issued (n uses of stages 0..S-1) has landed.
 __device__ __forceinline__ void drain_ring(uint32_t full_bar0, int S, int n) {
@@ -371,6 +371,7 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
                        const __grid_constant__ CUtensorMap tmdK,
                        const __grid_constant__ CUtensorMap tmdV, const BwdArgs a) {
   using C = DkdvCfg<D>;
+  static_assert(C::kStages0 == C::kStages1, "one ring of (Q, dO) stages");
   constexpr bool kAlibi = (kFeat & kFeatAlibi) != 0;
   constexpr bool kKpad = (kFeat & kFeatKpad) != 0;
   constexpr bool kDropout = (kFeat & kFeatDropout) != 0;
@@ -402,15 +403,15 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
       mbar_init(bar(C::bXFull + b), 1);
       mbar_init(bar(C::bXEmpty + b), 1);
     }
-    // Q_i (with its statistics) is read by S^T and dK, dO_i by dP^T and dV: one release
-    // from each issuer
+    // One stage of the ring holds Q_i (with its statistics) and dO_i; it is released by
+    // one commit after dK(i), the last product of the query tile: by then S^T, dP^T and dV
+    // of the tile have completed too (the softmax consumed S^T and dP^T before it
+    // published dS^T, and dV was issued before dK by the same thread). Each commit holds
+    // its issuing thread for a few hundred clocks, so releases are not made separately.
     for (int s = 0; s < C::kStages0; ++s) {
       mbar_init(bar(C::bY0Full + s), 1);
-      mbar_init(bar(C::bY0Empty + s), 2);
-    }
-    for (int s = 0; s < C::kStages1; ++s) {
       mbar_init(bar(C::bY1Full + s), 1);
-      mbar_init(bar(C::bY1Empty + s), 2);
+      mbar_init(bar(C::bY0Empty + s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(bSFull + b), 1);
@@ -436,7 +437,7 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
       tma_prefetch_map(&tmK);
       tma_prefetch_map(&tmV);
       tma_prefetch_map(&tmdO);
-      int items = 0, n0 = 0, n1 = 0;  // items started; loads into ring 0 and ring 1
+      int items = 0, n = 0;  // items started; query tiles loaded into the ring
       bool ok = true;
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, j;
@@ -454,37 +455,31 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
                       bar(C::bXFull + xb), r * 64, j * kBlock, bh);
         }
         ++items;
-        for (int i = i_lo; i <= i_hi; ++i) {
-          const int s0 = n0 % C::kStages0, s1 = n1 % C::kStages1;
-          if (!mbar_wait(bar(C::bY0Empty + s0), ((n0 / C::kStages0) & 1) ^ 1, abort_flag)) {
+        for (int i = i_lo; i <= i_hi; ++i, ++n) {
+          const int s = n % C::kStages0;
+          if (!mbar_wait(bar(C::bY0Empty + s), ((n / C::kStages0) & 1) ^ 1, abort_flag)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(bar(C::bY0Full + s0), C::kTile + 2 * 512);
+          mbar_arrive_expect_tx(bar(C::bY0Full + s), C::kTile + 2 * 512);
           for (int r = 0; r < C::kRegions; ++r)
-            tma_load_3d(sb + C::kY0 + s0 * C::kTile + r * C::kRegionBytes, &tmQ,
-                        bar(C::bY0Full + s0), r * 64, i * kBlock, bh);
+            tma_load_3d(sb + C::kY0 + s * C::kTile + r * C::kRegionBytes, &tmQ,
+                        bar(C::bY0Full + s), r * 64, i * kBlock, bh);
           // LSE*log2e and delta of the 128 rows of query tile i (512 bytes each)
           const float* st = a.stats + (size_t)bh * a.Np + (size_t)i * kBlock;
-          bulk_load(sb + C::kLse + s0 * 512, st, 512, bar(C::bY0Full + s0));
-          bulk_load(sb + C::kDelta + s0 * 512, st + a.stat_rows, 512, bar(C::bY0Full + s0));
-          ++n0;
-          if (!mbar_wait(bar(C::bY1Empty + s1), ((n1 / C::kStages1) & 1) ^ 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(bar(C::bY1Full + s1), C::kTile);
+          bulk_load(sb + C::kLse + s * 512, st, 512, bar(C::bY0Full + s));
+          bulk_load(sb + C::kDelta + s * 512, st + a.stat_rows, 512, bar(C::bY0Full + s));
+          mbar_arrive_expect_tx(bar(C::bY1Full + s), C::kTile);
           for (int r = 0; r < C::kRegions; ++r)
-            tma_load_3d(sb + C::kY1 + s1 * C::kTile + r * C::kRegionBytes, &tmdO,
-                        bar(C::bY1Full + s1), r * 64, i * kBlock, bh);
-          ++n1;
+            tma_load_3d(sb + C::kY1 + s * C::kTile + r * C::kRegionBytes, &tmdO,
+                        bar(C::bY1Full + s), r * 64, i * kBlock, bh);
         }
       }
       // Drain: every copy issued must have landed before the CTA may exit.
-      for (int n = (items > C::kXBufs ? items - C::kXBufs : 0); n < items; ++n)
-        mbar_wait(bar(C::bXFull + n % C::kXBufs), (n / C::kXBufs) & 1, nullptr);
-      drain_ring(bar(C::bY0Full), C::kStages0, n0);
-      drain_ring(bar(C::bY1Full), C::kStages1, n1);
+      for (int x = (items > C::kXBufs ? items - C::kXBufs : 0); x < items; ++x)
+        mbar_wait(bar(C::bXFull + x % C::kXBufs), (x / C::kXBufs) & 1, nullptr);
+      drain_ring(bar(C::bY0Full), C::kStages0, n);
+      drain_ring(bar(C::bY1Full), C::kStages0, n);
     }
     __syncwarp();
   } else if (warp == C::kWarpMma) {
@@ -502,12 +497,16 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
         const int xb = items % C::kXBufs, xu = items / C::kXBufs;
         if (!mbar_wait(bar(C::bXFull + xb), xu & 1, abort_flag)) break;
         for (int i = i_lo; i <= i_hi; ++i, ++t) {
-          const int b = t % kSBufs, s0 = t % C::kStages0, s1 = t % C::kStages1;
+          const int b = t % kSBufs, s0 = t % C::kStages0, s1 = s0;
           // S^T = K_j Q_i^T, once the products that read its buffer's P^T (and dS^T) have
-          // completed
+          // completed: dV of the previous tile, or with kDsInS dK of tile t - 2, whose
+          // completion releases that tile's ring stage
+          const int tp = t - kSBufs;
           if (!mbar_wait(bar(C::bY0Full + s0), (t / C::kStages0) & 1, abort_flag) ||
-              (t >= kSBufs &&
-               !mbar_wait(bar(bSFree + b), ((t / kSBufs) - 1) & 1, abort_flag))) {
+              (tp >= 0 && !(kDsInS ? mbar_wait(bar(C::bY0Empty + tp % C::kStages0),
+                                               (tp / C::kStages0) & 1, abort_flag)
+                                   : mbar_wait(bar(bSFree + b), ((t / kSBufs) - 1) & 1,
+                                               abort_flag)))) {
             ok = false;
             break;
           }
@@ -520,7 +519,6 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
                    sdesc_sw128(sb + C::kY0 + s0 * C::kTile + off, 16, 1024), idS, kk > 0);
           }
           tc_commit(bar(bSFull + b));
-          tc_commit(bar(C::bY0Empty + s0));
           // dP^T = V_j dO_i^T, once the previous tile's dP^T is free
           if (!mbar_wait(bar(C::bY1Full + s1), (t / C::kStages1) & 1, abort_flag) ||
               (t >= 1 && !mbar_wait(bar(bDPFree), (t - 1) & 1, abort_flag))) {
@@ -535,7 +533,6 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
                    sdesc_sw128(sb + C::kY1 + s1 * C::kTile + off, 16, 1024), idS, kk > 0);
           }
           tc_commit(bar(bDPFull));
-          tc_commit(bar(C::bY1Empty + s1));
           // without staged outputs, K_j and V_j are free after their last product
           if (!C::kStageOut && i == i_hi) tc_commit(bar(C::bXEmpty + xb));
         }
@@ -558,7 +555,7 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
         int i_lo, i_hi;
         q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
         for (int i = i_lo; i <= i_hi; ++i, ++t) {
-          const int b = t % kSBufs, s0 = t % C::kStages0, s1 = t % C::kStages1;
+          const int b = t % kSBufs, s0 = t % C::kStages0, s1 = s0;
           const bool first = i == i_lo;
           // dV += P^T dO_i; the item's first product overwrites dV, which the previous
           // item's epilogue must have read
@@ -574,7 +571,6 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
             mma_ts(tmem + tDV, tmem + tS + 128u * b + packed_col(kk),
                    sdesc_sw128(sb + C::kY1 + s1 * C::kTile + kk * 2048, C::kRegionBytes, 1024),
                    idA, (!first || kk > 0) ? 1u : 0u);
-          tc_commit(bar(C::bY1Empty + s1));
           if (!kDsInS) tc_commit(bar(bSFree + b));
           // dK += dS^T Q_i
           if (!mbar_wait(bar(C::bY0Full + s0), (t / C::kStages0) & 1, abort_flag) ||
@@ -589,8 +585,9 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
                    tmem + (kDsInS ? tS + 128u * b + 16u : tDP) + packed_col(kk),
                    sdesc_sw128(sb + C::kY0 + s0 * C::kTile + kk * 2048, C::kRegionBytes, 1024),
                    idA, (!first || kk > 0) ? 1u : 0u);
+          // the tile's ring stage (and with kDsInS its S^T buffer) is free
           tc_commit(bar(C::bY0Empty + s0));
-          tc_commit(bar(kDsInS ? bSFree + b : bDPFree));
+          if (!kDsInS) tc_commit(bar(bDPFree));
           if (i == i_hi) tc_commit(bar(bAccReady));  // dK, dV of the item are complete
         }
         ++items;
@@ -801,6 +798,12 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
                      const __grid_constant__ CUtensorMap tmdO,
                      const __grid_constant__ CUtensorMap tmdQ, const BwdArgs a) {
   using C = DqCfg<D>;
+  // With equal rings, one stage holds K_j and V_j and is released by one commit after
+  // dQ(j), the last product of the key tile (S and dP of the tile have completed by then:
+  // the softmax consumed both before it published dS); the S buffer of tile t - 2 is free
+  // with that tile's stage. Otherwise K_j is released by S and dQ, V_j by dP, and the S
+  // buffer by its own barrier.
+  constexpr bool kOneRelease = C::kStages0 == C::kStages1;
   constexpr bool kAlibi = (kFeat & kFeatAlibi) != 0;
   constexpr bool kKpad = (kFeat & kFeatKpad) != 0;
   constexpr bool kDropout = (kFeat & kFeatDropout) != 0;
@@ -824,10 +827,9 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
       mbar_init(bar(C::bXFull + b), 1);
       mbar_init(bar(C::bXEmpty + b), 1);
     }
-    // K_j is read by S and dQ: one release from each issuer
     for (int s = 0; s < C::kStages0; ++s) {
       mbar_init(bar(C::bY0Full + s), 1);
-      mbar_init(bar(C::bY0Empty + s), 2);
+      mbar_init(bar(C::bY0Empty + s), kOneRelease ? 1 : 2);
     }
     for (int s = 0; s < C::kStages1; ++s) {
       mbar_init(bar(C::bY1Full + s), 1);
@@ -884,7 +886,8 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
             tma_load_3d(sb + C::kY0 + s0 * C::kTile + r * C::kRegionBytes, &tmK,
                         bar(C::bY0Full + s0), r * 64, jj * kBlock, bh);
           ++n0;
-          if (!mbar_wait(bar(C::bY1Empty + s1), ((n1 / C::kStages1) & 1) ^ 1, abort_flag)) {
+          if (!kOneRelease &&
+              !mbar_wait(bar(C::bY1Empty + s1), ((n1 / C::kStages1) & 1) ^ 1, abort_flag)) {
             ok = false;
             break;
           }
@@ -918,8 +921,12 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
         for (int jj = j_lo; jj <= j_hi; ++jj, ++t) {
           const int s0 = t % C::kStages0, s1 = t % C::kStages1;
           // S(t) = Q_i K_j^T into buffer t & 1, which held dS(t-2): dQ(t-2) must have read it
+          const int tp = t - 2;
           if (!mbar_wait(bar(C::bY0Full + s0), (t / C::kStages0) & 1, abort_flag) ||
-              (t >= 2 && !mbar_wait(bar(bDQDone + (t & 1)), ((t >> 1) - 1) & 1, abort_flag))) {
+              (tp >= 0 && !(kOneRelease ? mbar_wait(bar(C::bY0Empty + tp % C::kStages0),
+                                                    (tp / C::kStages0) & 1, abort_flag)
+                                        : mbar_wait(bar(bDQDone + (t & 1)), ((t >> 1) - 1) & 1,
+                                                    abort_flag)))) {
             ok = false;
             break;
           }
@@ -932,7 +939,7 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
                    sdesc_sw128(sb + C::kY0 + s0 * C::kTile + off, 16, 1024), idS, kk > 0);
           }
           tc_commit(bar(bSFull + (t & 1)));
-          tc_commit(bar(C::bY0Empty + s0));
+          if (!kOneRelease) tc_commit(bar(C::bY0Empty + s0));
           // dP(t) = dO_i V_j^T, once the softmax has loaded dP(t-1); V_j is then free
           if (!mbar_wait(bar(C::bY1Full + s1), (t / C::kStages1) & 1, abort_flag) ||
               (t >= 1 && !mbar_wait(bar(bDPFree), (t - 1) & 1, abort_flag))) {
@@ -947,7 +954,7 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
                    sdesc_sw128(sb + C::kY1 + s1 * C::kTile + off, 16, 1024), idS, kk > 0);
           }
           tc_commit(bar(bDPFull));
-          tc_commit(bar(C::bY1Empty + s1));
+          if (!kOneRelease) tc_commit(bar(C::bY1Empty + s1));
           // without a staged output, Q_i and dO_i are free after their last product
           if (!C::kStageOut && jj == j_hi) tc_commit(bar(C::bXEmpty + xb));
         }
@@ -987,7 +994,7 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
                    sdesc_sw128(sb + C::kY0 + s0 * C::kTile + kk * 2048, C::kRegionBytes, 1024),
                    idA, (!first || kk > 0) ? 1u : 0u);
           tc_commit(bar(C::bY0Empty + s0));
-          tc_commit(bar(bDQDone + (t & 1)));
+          if (!kOneRelease) tc_commit(bar(bDQDone + (t & 1)));
           if (jj == j_hi) tc_commit(bar(bAccReady));  // dQ of the item is complete
         }
         ++items;
