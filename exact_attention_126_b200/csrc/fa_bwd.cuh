@@ -386,9 +386,13 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
   // complete. Every barrier that one side may complete twice before the other has waited
   // once is kept per buffer, so that no parity wait can mistake a later phase for the one
   // it wants.
+  // With kDsInS, dS^T full is kept per buffer (a second tile's dS^T may be published before
+  // dK has waited for the first), in the slots of S^T free, which kDsInS does not use (the
+  // ring stage of tile t - 2 frees its S^T buffer).
   constexpr int bSFull = C::bA + 0, bPFull = C::bA + 2, bSFree = C::bA + 4,
-                bDPFull = C::bA + 6, bDSFull = C::bA + 7, bDPFree = C::bA + 8,
-                bAccFree = C::bA + 9, bAccReady = C::bA + 10, bStaged = C::bA + 11;
+                bDPFull = C::bA + 6, bDSFull = kDsInS ? C::bA + 4 : C::bA + 7,
+                bDPFree = C::bA + 8, bAccFree = C::bA + 9, bAccReady = C::bA + 10,
+                bStaged = C::bA + 11;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -416,11 +420,11 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(bSFull + b), 1);
       mbar_init(bar(bPFull + b), C::kSoftmax / 32);
-      mbar_init(bar(bSFree + b), 1);
+      mbar_init(bar(bSFree + b), kDsInS ? C::kSoftmax / 32 : 1);  // dS^T full with kDsInS
       mbar_init(bar(C::bMmaFin + b), 1);
     }
     mbar_init(bar(bDPFull), 1);
-    mbar_init(bar(bDSFull), C::kSoftmax / 32);
+    if (!kDsInS) mbar_init(bar(bDSFull), C::kSoftmax / 32);
     mbar_init(bar(bDPFree), kDsInS ? C::kSoftmax / 32 : 1);
     mbar_init(bar(bAccFree), C::kSoftmax / 32);
     mbar_init(bar(bAccReady), 1);
@@ -511,12 +515,14 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
             break;
           }
           tc_fence_after();
+          {
+            const uint64_t dx = sdesc_sw128(sb + C::kX0 + xb * 2 * C::kTile, 16, 1024);
+            const uint64_t dy = sdesc_sw128(sb + C::kY0 + s0 * C::kTile, 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-            mma_ss(tmem + tS + 128u * b,
-                   sdesc_sw128(sb + C::kX0 + xb * 2 * C::kTile + off, 16, 1024),
-                   sdesc_sw128(sb + C::kY0 + s0 * C::kTile + off, 16, 1024), idS, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
+              mma_ss(tmem + tS + 128u * b, sdesc_add(dx, off), sdesc_add(dy, off), idS, kk > 0);
+            }
           }
           tc_commit(bar(bSFull + b));
           // dP^T = V_j dO_i^T, once the previous tile's dP^T is free
@@ -526,11 +532,14 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
             break;
           }
           tc_fence_after();
+          {
+            const uint64_t dx = sdesc_sw128(sb + C::kX1 + xb * 2 * C::kTile, 16, 1024);
+            const uint64_t dy = sdesc_sw128(sb + C::kY1 + s1 * C::kTile, 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-            mma_ss(tmem + tDP, sdesc_sw128(sb + C::kX1 + xb * 2 * C::kTile + off, 16, 1024),
-                   sdesc_sw128(sb + C::kY1 + s1 * C::kTile + off, 16, 1024), idS, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
+              mma_ss(tmem + tDP, sdesc_add(dx, off), sdesc_add(dy, off), idS, kk > 0);
+            }
           }
           tc_commit(bar(bDPFull));
           // without staged outputs, K_j and V_j are free after their last product
@@ -566,25 +575,30 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
             break;
           }
           tc_fence_after();
+          {
+            const uint64_t dy = sdesc_sw128(sb + C::kY1 + s1 * C::kTile, C::kRegionBytes, 1024);
 #pragma unroll
-          for (int kk = 0; kk < kBlock / 16; ++kk)
-            mma_ts(tmem + tDV, tmem + tS + 128u * b + packed_col(kk),
-                   sdesc_sw128(sb + C::kY1 + s1 * C::kTile + kk * 2048, C::kRegionBytes, 1024),
-                   idA, (!first || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kBlock / 16; ++kk)
+              mma_ts(tmem + tDV, tmem + tS + 128u * b + packed_col(kk), sdesc_add(dy, kk * 2048),
+                     idA, (!first || kk > 0) ? 1u : 0u);
+          }
           if (!kDsInS) tc_commit(bar(bSFree + b));
           // dK += dS^T Q_i
           if (!mbar_wait(bar(C::bY0Full + s0), (t / C::kStages0) & 1, abort_flag) ||
-              !mbar_wait(bar(bDSFull), t & 1, abort_flag)) {
+              !mbar_wait(bar(bDSFull + (kDsInS ? b : 0)), (kDsInS ? t / 2 : t) & 1,
+                         abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
+          {
+            const uint64_t dy = sdesc_sw128(sb + C::kY0 + s0 * C::kTile, C::kRegionBytes, 1024);
+            const uint32_t ta = tmem + (kDsInS ? tS + 128u * b + 16u : tDP);
 #pragma unroll
-          for (int kk = 0; kk < kBlock / 16; ++kk)
-            mma_ts(tmem + tDK,
-                   tmem + (kDsInS ? tS + 128u * b + 16u : tDP) + packed_col(kk),
-                   sdesc_sw128(sb + C::kY0 + s0 * C::kTile + kk * 2048, C::kRegionBytes, 1024),
-                   idA, (!first || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kBlock / 16; ++kk)
+              mma_ts(tmem + tDK, ta + packed_col(kk), sdesc_add(dy, kk * 2048), idA,
+                     (!first || kk > 0) ? 1u : 0u);
+          }
           // the tile's ring stage (and with kDsInS its S^T buffer) is free
           tc_commit(bar(C::bY0Empty + s0));
           if (!kDsInS) tc_commit(bar(bDPFree));
@@ -745,7 +759,7 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
         tmem_st16(kDsInS ? tSb + 16 : tmem + lane_base + tDP + NC * h, w);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive_warp(bar(bDSFull));
+        mbar_arrive_warp(bar(bDSFull + (kDsInS ? t % kSBufs : 0)));
       }
       if (!ok) break;
       g += n_it;
@@ -931,12 +945,15 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
             break;
           }
           tc_fence_after();
+          {
+            const uint64_t dx = sdesc_sw128(sb + C::kX0 + xb * 2 * C::kTile, 16, 1024);
+            const uint64_t dy = sdesc_sw128(sb + C::kY0 + s0 * C::kTile, 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-            mma_ss(tmem + tS0 + 128u * (t & 1),
-                   sdesc_sw128(sb + C::kX0 + xb * 2 * C::kTile + off, 16, 1024),
-                   sdesc_sw128(sb + C::kY0 + s0 * C::kTile + off, 16, 1024), idS, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
+              mma_ss(tmem + tS0 + 128u * (t & 1), sdesc_add(dx, off), sdesc_add(dy, off), idS,
+                     kk > 0);
+            }
           }
           tc_commit(bar(bSFull + (t & 1)));
           if (!kOneRelease) tc_commit(bar(C::bY0Empty + s0));
@@ -947,11 +964,14 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
             break;
           }
           tc_fence_after();
+          {
+            const uint64_t dx = sdesc_sw128(sb + C::kX1 + xb * 2 * C::kTile, 16, 1024);
+            const uint64_t dy = sdesc_sw128(sb + C::kY1 + s1 * C::kTile, 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-            mma_ss(tmem + tDP, sdesc_sw128(sb + C::kX1 + xb * 2 * C::kTile + off, 16, 1024),
-                   sdesc_sw128(sb + C::kY1 + s1 * C::kTile + off, 16, 1024), idS, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
+              mma_ss(tmem + tDP, sdesc_add(dx, off), sdesc_add(dy, off), idS, kk > 0);
+            }
           }
           tc_commit(bar(bDPFull));
           if (!kOneRelease) tc_commit(bar(C::bY1Empty + s1));
@@ -988,11 +1008,14 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
             break;
           }
           tc_fence_after();
+          {
+            const uint64_t dy = sdesc_sw128(sb + C::kY0 + s0 * C::kTile, C::kRegionBytes, 1024);
+            const uint32_t ta = tmem + tS0 + 128u * (t & 1);
 #pragma unroll
-          for (int kk = 0; kk < kBlock / 16; ++kk)
-            mma_ts(tmem + tDQ, tmem + tS0 + 128u * (t & 1) + packed_col(kk),
-                   sdesc_sw128(sb + C::kY0 + s0 * C::kTile + kk * 2048, C::kRegionBytes, 1024),
-                   idA, (!first || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kBlock / 16; ++kk)
+              mma_ts(tmem + tDQ, ta + packed_col(kk), sdesc_add(dy, kk * 2048), idA,
+                     (!first || kk > 0) ? 1u : 0u);
+          }
           tc_commit(bar(C::bY0Empty + s0));
           if (!kOneRelease) tc_commit(bar(bDQDone + (t & 1)));
           if (jj == j_hi) tc_commit(bar(bAccReady));  // dQ of the item is complete

@@ -245,10 +245,13 @@ __global__ void __launch_bounds__(FusedCfg::kThreads, 1)
             break;
           }
           tc_fence_after();
+          {
+            const uint64_t dx = sdesc_sw128(xK, 16, 1024);
+            const uint64_t dy = sdesc_sw128(sb + C::kY0 + s0 * C::kTile, 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + C::tS, sdesc_sw128(xK + kk * 32, 16, 1024),
-                   sdesc_sw128(sb + C::kY0 + s0 * C::kTile + kk * 32, 16, 1024), idS, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tmem + C::tS, sdesc_add(dx, kk * 32), sdesc_add(dy, kk * 32), idS, kk > 0);
+          }
           tc_commit(bar(C::bSFull));
           tc_commit(bar(C::bY0Empty + s0));
           // dP^T = V_j dO_i^T, once the softmax has loaded the previous dP^T
@@ -258,10 +261,13 @@ __global__ void __launch_bounds__(FusedCfg::kThreads, 1)
             break;
           }
           tc_fence_after();
+          {
+            const uint64_t dx = sdesc_sw128(xV, 16, 1024);
+            const uint64_t dy = sdesc_sw128(sb + C::kY1 + s1 * C::kTile, 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + C::tDP, sdesc_sw128(xV + kk * 32, 16, 1024),
-                   sdesc_sw128(sb + C::kY1 + s1 * C::kTile + kk * 32, 16, 1024), idS, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tmem + C::tDP, sdesc_add(dx, kk * 32), sdesc_add(dy, kk * 32), idS, kk > 0);
+          }
           tc_commit(bar(C::bDPFull));
           tc_commit(bar(C::bY1Empty + s1));
         }
@@ -300,12 +306,14 @@ __global__ void __launch_bounds__(FusedCfg::kThreads, 1)
             break;
           }
           tc_fence_after();
+          {
+            const uint64_t dp = sdesc_sw128(sb + C::kP, 16, 1024);
+            const uint64_t dy = sdesc_sw128(sb + C::kY1 + s1 * C::kTile, C::kRegionBytes, 1024);
 #pragma unroll
-          for (int kk = 0; kk < kBlock / 16; ++kk)
-            mma_ss(tmem + C::tDV,
-                   sdesc_sw128(sb + C::kP + (kk >> 2) * C::kRegionBytes + (kk & 3) * 32, 16, 1024),
-                   sdesc_sw128(sb + C::kY1 + s1 * C::kTile + kk * 2048, C::kRegionBytes, 1024),
-                   idKV, (!first || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kBlock / 16; ++kk)
+              mma_ss(tmem + C::tDV, sdesc_add(dp, (kk >> 2) * C::kRegionBytes + (kk & 3) * 32),
+                     sdesc_add(dy, kk * 2048), idKV, (!first || kk > 0) ? 1u : 0u);
+          }
           tc_commit(bar(C::bPFree));
           tc_commit(bar(C::bY1Empty + s1));
           // dK += dS^T Q_i, then dQ_t = dS K_j into buffer t & 1 once tile t-2's is drained
@@ -316,17 +324,20 @@ __global__ void __launch_bounds__(FusedCfg::kThreads, 1)
             break;
           }
           tc_fence_after();
+          {
+            const uint64_t dsk = sdesc_sw128(sb + C::kDS, 16, 1024);
+            const uint64_t dy = sdesc_sw128(sb + C::kY0 + s0 * C::kTile, C::kRegionBytes, 1024);
 #pragma unroll
-          for (int kk = 0; kk < kBlock / 16; ++kk)
-            mma_ss(tmem + C::tDK,
-                   sdesc_sw128(sb + C::kDS + (kk >> 2) * C::kRegionBytes + (kk & 3) * 32, 16, 1024),
-                   sdesc_sw128(sb + C::kY0 + s0 * C::kTile + kk * 2048, C::kRegionBytes, 1024),
-                   idKV, (!first || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kBlock / 16; ++kk)
+              mma_ss(tmem + C::tDK, sdesc_add(dsk, (kk >> 2) * C::kRegionBytes + (kk & 3) * 32),
+                     sdesc_add(dy, kk * 2048), idKV, (!first || kk > 0) ? 1u : 0u);
+            const uint64_t dsm = sdesc_sw128(sb + C::kDS, C::kRegionBytes, 1024);
+            const uint64_t dk = sdesc_sw128(xK, C::kRegionBytes, 1024);
 #pragma unroll
-          for (int kk = 0; kk < kBlock / 16; ++kk)
-            mma_ss(tmem + C::tDQ + 64u * (t & 1),
-                   sdesc_sw128(sb + C::kDS + kk * 2048, C::kRegionBytes, 1024),
-                   sdesc_sw128(xK + kk * 2048, C::kRegionBytes, 1024), idQ, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < kBlock / 16; ++kk)
+              mma_ss(tmem + C::tDQ + 64u * (t & 1), sdesc_add(dsm, kk * 2048),
+                     sdesc_add(dk, kk * 2048), idQ, kk > 0 ? 1u : 0u);
+          }
           tc_commit(bar(C::bY0Empty + s0));
           tc_commit(bar(C::bDQFull + (t & 1)));
           if (i == i_hi) tc_commit(bar(C::bAccReady));  // dK, dV (and the last dQ) complete

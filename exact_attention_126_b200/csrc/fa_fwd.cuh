@@ -69,8 +69,9 @@ struct FwdCfg {
   static constexpr int kTile = kBlock * D * kElemBytes;  // bytes of a 128 x D tile
   static constexpr int kRegions = D * kElemBytes / 128;  // 128-byte-wide column regions per tile
   static constexpr int kRegionBytes = kBlock * 128;
+  // K_j and V_j share a ring stage, released by one commit per stream after its P V_j
   static constexpr int kStagesK = (D == 64) ? 4 : 2;
-  static constexpr int kStagesV = (D == 64) ? 4 : 2;
+  static constexpr int kStagesV = kStagesK;
   // shared memory map (offsets from a 1024-aligned base)
   // Q buffers per stream: with head_dim 64 two, so that the next item's Q_s loads while
   // the current one is in use
@@ -218,13 +219,14 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
       mbar_init(bar(C::bTurn + s), 4);
       mbar_init(bar(C::bSFree + s), 4);
     }
+    // a K/V stage is released by one commit per stream after its P V product of the
+    // stage's key tile (which the stream's S product of that tile precedes); each commit
+    // holds its issuing thread for a few hundred clocks, so K and V are not released
+    // separately
     for (int s = 0; s < C::kStagesK; ++s) {
       mbar_init(bar(C::bKFull + s), 1);
-      mbar_init(bar(C::bKEmpty + s), 2);  // one release per stream
-    }
-    for (int s = 0; s < C::kStagesV; ++s) {
       mbar_init(bar(C::bVFull + s), 1);
-      mbar_init(bar(C::bVEmpty + s), 2);
+      mbar_init(bar(C::bKEmpty + s), 2);
     }
     mbar_init(bar(C::bMmaFin), 1);
     mbar_init(bar(C::bMmaFin + 1), 1);
@@ -279,15 +281,10 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
                         bar(C::bKFull + sk), r * 64, j * kBlock, it.bh);
           ++kc;
           if (a.fault == 1) continue;
-          const int sv = vc % C::kStagesV;
-          if (!mbar_wait(bar(C::bVEmpty + sv), ((vc / C::kStagesV) & 1) ^ 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(bar(C::bVFull + sv), C::kTile);
+          mbar_arrive_expect_tx(bar(C::bVFull + sk), C::kTile);
           for (int r = 0; r < C::kRegions; ++r)
-            tma_load_3d(sb + C::kV + sv * C::kTile + r * C::kRegionBytes, &tmV,
-                        bar(C::bVFull + sv), r * 64, j * kBlock, it.bh);
+            tma_load_3d(sb + C::kV + sk * C::kTile + r * C::kRegionBytes, &tmV,
+                        bar(C::bVFull + sk), r * 64, j * kBlock, it.bh);
           ++vc;
         }
       }
@@ -327,7 +324,15 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
       int npv = 0;    // P V products issued (all items)
       int nitem = 0;  // items whose last P V has been issued
       int pos = 0;    // K/V ring position
+      int pend = -1;  // K/V stage whose release waits for the next S product, or -1
       bool ok = true;
+      // Commits the pending release of a K/V stage. Without separate P the next S product
+      // waits for the P V product to complete, so the release is committed after that S
+      // product, off the path from P V to S.
+      auto release = [&]() {
+        if (pend >= 0) tc_commit(bar(C::bKEmpty + pend));
+        pend = -1;
+      };
       // K step of key tile j (ring position p): S_s = Q_s K_j^T if the stream sees j
       auto k_step = [&](const FwdItem& it, const FwdRange& rg, int j, int p) -> bool {
         const bool sees = rg.has && rg.lo <= j && j <= rg.hi;
@@ -346,28 +351,30 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
             return false;
           tc_fence_after();
           const uint32_t qbase = sb + C::kQ + (s * C::kQBufs + nq % C::kQBufs) * C::kTile;
+          const uint64_t dq = sdesc_sw128(qbase, 16, 1024);
+          const uint64_t dk = sdesc_sw128(sb + C::kK + sk * C::kTile, 16, 1024);
           if constexpr (kFp8) {
             // K-steps of 32 e4m3 values: 32 bytes of the 128-byte rows
 #pragma unroll
             for (int kk = 0; kk < D / 32; ++kk)
-              mma_ss_f8(tmem + C::tS + 128u * s, sdesc_sw128(qbase + kk * 32, 16, 1024),
-                        sdesc_sw128(sb + C::kK + sk * C::kTile + kk * 32, 16, 1024), idS, kk > 0);
+              mma_ss_f8(tmem + C::tS + 128u * s, sdesc_add(dq, kk * 32), sdesc_add(dk, kk * 32),
+                        idS, kk > 0);
           } else {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
-              mma_ss(tmem + C::tS + 128u * s, sdesc_sw128(qbase + off, 16, 1024),
-                     sdesc_sw128(sb + C::kK + sk * C::kTile + off, 16, 1024), idS, kk > 0);
+              mma_ss(tmem + C::tS + 128u * s, sdesc_add(dq, off), sdesc_add(dk, off), idS,
+                     kk > 0);
             }
           }
           tc_commit(bar(C::bSFull + s));
           ++nsi;
+          release();
           if (j == rg.hi) {
             tc_commit(bar(C::bQEmpty + qb));  // last read of this Q_s buffer
             ++nq;
           }
         }
-        tc_commit(bar(C::bKEmpty + sk));
         return true;
       };
       // V step of key tile j (ring position p): O_s += P_s V_j if the stream sees j
@@ -384,25 +391,26 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
             return false;
           tc_fence_after();
           const uint32_t pcol = tmem + (C::kSepP ? C::tP + 64u * s : C::tS + 128u * s);
+          const uint64_t dv = sdesc_sw128(sb + C::kV + sv * C::kTile, C::kRegionBytes, 1024);
           if constexpr (kFp8) {
             // K-steps of 32 keys: 8 columns of P (four e4m3 per column), 32 rows of V
 #pragma unroll
             for (int kk = 0; kk < kBlock / 32; ++kk)
-              mma_ts_f8(tmem + C::tO + D * s, pcol + kk * 8,
-                        sdesc_sw128(sb + C::kV + sv * C::kTile + kk * 4096, C::kRegionBytes, 1024),
-                        idO, (!first || kk > 0) ? 1u : 0u);
+              mma_ts_f8(tmem + C::tO + D * s, pcol + kk * 8, sdesc_add(dv, kk * 4096), idO,
+                        (!first || kk > 0) ? 1u : 0u);
           } else {
 #pragma unroll
             for (int kk = 0; kk < kBlock / 16; ++kk)
-              mma_ts(tmem + C::tO + D * s, pcol + kk * 8,
-                     sdesc_sw128(sb + C::kV + sv * C::kTile + kk * 2048, C::kRegionBytes, 1024),
-                     idO, (!first || kk > 0) ? 1u : 0u);
+              mma_ts(tmem + C::tO + D * s, pcol + kk * 8, sdesc_add(dv, kk * 2048), idO,
+                     (!first || kk > 0) ? 1u : 0u);
           }
           tc_commit(bar(C::bODone + s));
           ++npv;
           if (j == rg.hi) ++nitem;
         }
-        tc_commit(bar(C::bVEmpty + sv));
+        release();  // a stage whose release is still pending goes now
+        pend = sv;
+        if (C::kSepP) release();
         return true;
       };
 
@@ -426,6 +434,7 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
         }
         pos += n;
       }
+      release();
       // Wait for every MMA this thread issued before the CTA may release tensor memory.
       tc_commit(bar(C::bMmaFin + s));
       mbar_wait(bar(C::bMmaFin + s), 0, nullptr);
