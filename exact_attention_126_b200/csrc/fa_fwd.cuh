@@ -8,25 +8,27 @@
 // tensor core computes the other's products, so neither the special-function unit nor
 // the tensor core waits for the other. Roles:
 //
-//   warp 10      TMA producer: Q_A, Q_B per item, then K_j and V_j through two rings of
+//   warp 10      TMA producer: Q_A, Q_B per item, then K_j and V_j through a ring of
 //                shared-memory stages (128-byte swizzle), guarded by full/empty mbarriers.
 //   warps 8, 9   MMA issuers (one thread each), for stream A and B: per key tile j,
-//                S_s = Q_s K_j^T, and O_s += P_s V_j once P_s is published. At head_dim 128
-//                P_s lies over S_s, so the next tile's S_s waits for that product; at
-//                head_dim 64 P_s has its own columns and the next S_s is issued one key tile
-//                ahead, as soon as the softmax has loaded S_s.
+//                S_s = Q_s K_j^T, and O_s += P_s V_j once P_s is published. At head_dim 64
+//                P_s has its own columns and the next S_s is issued one key tile ahead, as
+//                soon as the softmax has loaded S_s. At head_dim 128 P_s must lie over
+//                S_s, so each key tile is processed as two 64-key halves: S of half h of
+//                the next tile waits only for the P V product of half h, which runs while
+//                the softmax works on the other half.
 //   warps 0..3   softmax of stream A, warps 4..7 of stream B: thread r owns query row r
-//                of its tile (TMEM lane r) and all 128 scores of it. Per key tile it
-//                updates the running max m and sum l (page "告别OOM和训练慢…" §2.2),
-//                rescales its row of O when m grew by more than 2^8 (exact: O and l carry
-//                the same stale m), and writes P = exp2(s*scale*log2e - m) in bf16 to
-//                TMEM, where the P V product reads it (with ALiBi, the linear bias
-//                -m_h |i - j| joins every scaled score first). The two streams take turns
-//                on the exponentials. At the end of an item it writes O / l and
-//                LSE = ln2 * (m + log2 l).
+//                of its tile (TMEM lane r) and the scores of it. Per key tile (head_dim
+//                64) or half tile (head_dim 128) it updates the running max m and sum l
+//                (page "告别OOM和训练慢…" §2.2), rescales its row of O when m grew by more
+//                than 2^8 (exact: O and l carry the same stale m), and writes
+//                P = exp2(s*scale*log2e - m) in bf16 to TMEM, where the P V product reads
+//                it (with ALiBi, the linear bias -m_h |i - j| joins every scaled score
+//                first). At the end of an item it writes O / l and LSE = ln2 * (m + log2 l).
 //
 // TMEM: S_A (128 columns), S_B (128), O_A (head_dim), O_B (head_dim), and for head_dim 64
-// P_A, P_B (64 each); for head_dim 128 P_s goes over the first half of S_s.
+// P_A, P_B (64 each); for head_dim 128 P of half h goes over the first 32 (e4m3: 16)
+// columns of half h of S_s.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -92,8 +94,12 @@ struct FwdCfg {
   static constexpr int bODone = bPFull + 2;          // + stream: a P_s V product completed
   static constexpr int bOFree = bODone + 2;          // + stream: O_s read by the epilogue
   static constexpr int bSFree = bOFree + 2;          // + stream: S_s loaded (separate P)
-  static constexpr int bTurn = bSFree + 2;           // + stream: its turn on the exps
-  static constexpr int bMmaFin = bTurn + 2;          // + stream
+  // head_dim 128 works in 64-key halves of each key tile: the barriers above serve half 0,
+  // these half 1
+  static constexpr int bSFull2 = bSFree + 2;         // + stream
+  static constexpr int bPFull2 = bSFull2 + 2;        // + stream
+  static constexpr int bODone2 = bPFull2 + 2;        // + stream
+  static constexpr int bMmaFin = bODone2 + 2;        // + stream
   static constexpr int kNumBars = bMmaFin + 2;
   static constexpr int kMisc = kBar + kNumBars * 8;  // TMEM base address (+0), abort flag (+4)
   static constexpr int kSmemBytes = kMisc + 16 + 1024;
@@ -106,6 +112,11 @@ struct FwdCfg {
   // then be computed as soon as the softmax has loaded S_s, instead of waiting for the
   // P V product that reads P from the columns of S_s.
   static constexpr bool kSepP = (D == 64);
+  // Without room for P (head_dim 128), each key tile is processed as two 64-key halves:
+  // P of half h goes over the first columns of half h of S_s, so S of half h of the next
+  // key tile waits only for the P V product of half h, which runs while the softmax works
+  // on the other half.
+  static constexpr bool kHalves = !kSepP;
   static constexpr uint32_t tP = 256 + 2 * D;  // + 64 * stream, when kSepP
   static constexpr int kThreads = 352;  // 8 softmax warps, 2 MMA warps, producer warp
   static constexpr int kWarpMma = 8;     // + stream
@@ -216,8 +227,10 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
       mbar_init(bar(C::bPFull + s), 4);
       mbar_init(bar(C::bODone + s), 1);
       mbar_init(bar(C::bOFree + s), 4);
-      mbar_init(bar(C::bTurn + s), 4);
       mbar_init(bar(C::bSFree + s), 4);
+      mbar_init(bar(C::bSFull2 + s), 1);
+      mbar_init(bar(C::bPFull2 + s), 4);
+      mbar_init(bar(C::bODone2 + s), 1);
     }
     // a K/V stage is released by one commit per stream after its P V product of the
     // stage's key tile (which the stream's S product of that tile precedes); each commit
@@ -414,6 +427,85 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
         return true;
       };
 
+      // head_dim 128, in 64-key halves: products issued per half, S_h overwrites P_h
+      int nsh[2] = {0, 0};  // S products issued per half
+      int nph[2] = {0, 0};  // P V products issued per half
+      constexpr uint32_t idS64 = kFp8 ? idesc_e4m3_f32(128, 64, false, false)
+                                      : idesc_bf16_f32(128, 64, false, false);
+      // S_h = Q_s K_j[64h .. 64h+63]^T of key tile j (ring position p), if the stream sees j
+      auto s_half = [&](const FwdRange& rg, int j, int p, int h) -> bool {
+        const int sk = p % C::kStagesK;
+        if (h == 0 && !mbar_wait(bar(C::bKFull + sk), (p / C::kStagesK) & 1, abort_flag))
+          return false;
+        if (!(rg.has && rg.lo <= j && j <= rg.hi)) return true;
+        const bool first = j == rg.lo;
+        const int qb = 2 * s + nq % C::kQBufs;
+        // S_h overwrites P_h of the previous key tile, whose P V must have completed
+        if ((nsh[h] > 0 &&
+             !mbar_wait(bar((h ? C::bODone2 : C::bODone) + s), (nph[h] - 1) & 1, abort_flag)) ||
+            (first && h == 0 && !mbar_wait(bar(C::bQFull + qb), (nq / C::kQBufs) & 1, abort_flag)))
+          return false;
+        tc_fence_after();
+        const uint32_t qbase = sb + C::kQ + (s * C::kQBufs + nq % C::kQBufs) * C::kTile;
+        const uint64_t dq = sdesc_sw128(qbase, 16, 1024);
+        // rows 64h .. of K_j: 64 rows of 128 bytes into each 128-byte-wide region
+        const uint64_t dk = sdesc_sw128(sb + C::kK + sk * C::kTile + 64 * 128 * h, 16, 1024);
+        const uint32_t td = tmem + C::tS + 128u * s + 64u * h;
+        if constexpr (kFp8) {
+#pragma unroll
+          for (int kk = 0; kk < D / 32; ++kk)
+            mma_ss_f8(td, sdesc_add(dq, kk * 32), sdesc_add(dk, kk * 32), idS64, kk > 0);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
+            mma_ss(td, sdesc_add(dq, off), sdesc_add(dk, off), idS64, kk > 0);
+          }
+        }
+        tc_commit(bar((h ? C::bSFull2 : C::bSFull) + s));
+        ++nsh[h];
+        if (h == 1 && j == rg.hi) {
+          tc_commit(bar(C::bQEmpty + qb));  // last read of this Q_s buffer
+          ++nq;
+        }
+        return true;
+      };
+      // O_s += P_h V_j[64h .. 64h+63] of key tile j, if the stream sees j; after half 1 the
+      // stream's share of the K/V stage is released
+      auto v_half = [&](const FwdRange& rg, int j, int p, int h) -> bool {
+        const int sv = p % C::kStagesV;
+        if (h == 0 && !mbar_wait(bar(C::bVFull + sv), (p / C::kStagesV) & 1, abort_flag))
+          return false;
+        if (rg.has && rg.lo <= j && j <= rg.hi) {
+          const bool first = j == rg.lo;
+          // the item's first product overwrites O_s: the previous epilogue must have read it
+          if (!mbar_wait(bar((h ? C::bPFull2 : C::bPFull) + s), nph[h] & 1, abort_flag) ||
+              (first && h == 0 && nitem > 0 &&
+               !mbar_wait(bar(C::bOFree + s), (nitem - 1) & 1, abort_flag)))
+            return false;
+          tc_fence_after();
+          const uint32_t pcol = tmem + C::tS + 128u * s + 64u * h;
+          const uint64_t dv = sdesc_sw128(sb + C::kV + sv * C::kTile, C::kRegionBytes, 1024);
+          if constexpr (kFp8) {
+            // K-steps of 32 keys: 8 columns of P (four e4m3 per column), 32 rows of V
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk)
+              mma_ts_f8(tmem + C::tO + D * s, pcol + kk * 8, sdesc_add(dv, (2 * h + kk) * 4096),
+                        idO, (!first || h > 0 || kk > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ts(tmem + C::tO + D * s, pcol + kk * 8, sdesc_add(dv, (4 * h + kk) * 2048),
+                     idO, (!first || h > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(bar((h ? C::bODone2 : C::bODone) + s));
+          ++nph[h];
+          if (h == 1 && j == rg.hi) ++nitem;
+        }
+        if (h == 1) tc_commit(bar(C::bKEmpty + sv));
+        return true;
+      };
+
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         const FwdItem it = fwd_item(k, a);
         if (!it.has_a) continue;  // past the real length: no products
@@ -427,9 +519,14 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
             if (ok) ok = v_step(it, rg, it.first + t, pos + t);
           }
         } else {
+          // halves: S_0, S_1 of the first key tile, then P V of half h of tile t followed
+          // by S of half h of tile t + 1
+          ok = s_half(rg, it.first, pos, 0) && s_half(rg, it.first, pos, 1);
           for (int t = 0; ok && t < n; ++t) {
-            ok = k_step(it, rg, it.first + t, pos + t);
-            if (ok) ok = v_step(it, rg, it.first + t, pos + t);
+            ok = v_half(rg, it.first + t, pos + t, 0);
+            if (ok && t + 1 < n) ok = s_half(rg, it.first + t + 1, pos + t + 1, 0);
+            if (ok) ok = v_half(rg, it.first + t, pos + t, 1);
+            if (ok && t + 1 < n) ok = s_half(rg, it.first + t + 1, pos + t + 1, 1);
           }
         }
         pos += n;
@@ -450,30 +547,15 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
     const uint32_t tO = tmem + lane_base + C::tO + D * s;
     const float sl2 = a.scale_log2;
     int ns = 0;  // S tiles of this stream consumed (all items)
+    int nsh[2] = {0, 0};   // kHalves: S halves consumed, per half
+    int npub[2] = {0, 0};  // kHalves: P halves published, per half
     bool ok = true;
 
-    // When an item has both query tiles, the streams take turns on the exponentials of
-    // each key tile of the item (A first), so that one stream's exponentials run while the
-    // other loads and reduces its scores and the tensor core serves it. A stream that does
-    // not see a key tile only passes the turn on.
-    // The turns pay off at head_dim 128, where the exponentials weigh as much as the
-    // products; at head_dim 64 the two streams' softmax warps interleave better without them
-    // (measured on C4: 0.687 against 0.712 ms; on C5 1.56 against 1.47 ms the other way).
-    constexpr bool kTurns = D == 128;
-    int nturn = 0;  // turns taken
-    if (kTurns && s == 1) mbar_arrive_warp(bar(C::bTurn + 0));  // stream A starts
-    auto take_turn = [&]() -> bool {
-      const bool got = mbar_wait_warp(bar(C::bTurn + s), nturn & 1, abort_flag);
-      ++nturn;
-      return got;
-    };
-    auto pass_turn = [&]() { mbar_arrive_warp(bar(C::bTurn + (s ^ 1))); };
 
     for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
       const FwdItem it = fwd_item(k, a);
       const FwdRange rg = fwd_range(it, s);
       if (!rg.has) continue;
-      const bool turns = kTurns && it.has_b;
       const Mask mk{it.n, a.left, a.right};
       const int row = rg.m * kBlock + r;
       // with ALiBi the scores are scaled and biased as they are loaded (in log2 units), so
@@ -482,13 +564,155 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
       const float xs = kAlibi ? 1.f : sl2;
       float m_run = -INFINITY;  // running max of scale*log2e*s (the m that P and O carry)
       float l_run = 0.f;        // running sum of P
-      for (int j = turns ? it.first : rg.lo; j <= (turns ? it.last : rg.hi); ++j) {
-        if (j < rg.lo || j > rg.hi) {
-          if (!take_turn()) {
-            ok = false;
-            break;
+      for (int j = rg.lo; j <= rg.hi; ++j) {
+        if constexpr (C::kHalves) {
+          // the key tile as two 64-key halves, each its own step of the online softmax
+          for (int h = 0; h < 2; ++h) {
+            // keep flags of this row's 64 weights: bit c of keep[g] for key 64h + 32g + c
+            uint32_t keep[2] = {~0u, ~0u};
+            if (kDropout) {
+#pragma unroll
+              for (int g = 0; g < 2; ++g) {
+                const uint32_t blk = (uint32_t)(8 * j + 4 * h + 2 * g);
+                keep[g] = keep_bits16(a.drop, blk, (uint32_t)row, (uint32_t)it.bh) |
+                          (keep_bits16(a.drop, blk + 1, (uint32_t)row, (uint32_t)it.bh) << 16);
+              }
+            }
+            if (!mbar_wait_warp(bar((h ? C::bSFull2 : C::bSFull) + s), nsh[h] & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t tSh = tS + 64u * h;
+            float x[64];
+            {
+              uint32_t u[64];
+              tmem_ld32(tSh, *reinterpret_cast<uint32_t(*)[32]>(u));
+              tmem_ld32(tSh + 32, *reinterpret_cast<uint32_t(*)[32]>(u + 32));
+              tmem_wait_ld();
+              reg_fence(u);
+#pragma unroll
+              for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(u[c]);
+            }
+            if (kAlibi) {
+              // key minus query index at column 0 of the half
+              const long long kq = (long long)j * kBlock + 64 * h - row;
+              const float base = (float)kq;
+              const bool below = __all_sync(0xffffffffu, kq + 63 <= 0);
+              const bool above = __all_sync(0xffffffffu, kq >= 0);
+              if (below || above) {
+                const float s2 = below ? slope2 : -slope2;
+                const float c0 = s2 * base;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) x[c] = fmaf(x[c], sl2, fmaf(s2, (float)c, c0));
+              } else {
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                  x[c] = fmaf(x[c], sl2, -slope2 * fabsf(base + (float)c));
+              }
+            }
+            if (!tile_all_visible(rg.m, j, mk)) {
+              int c_lo, c_hi;
+              visible_keys(row, (long long)j * kBlock + 64 * h, 64, mk, c_lo, c_hi);
+#pragma unroll
+              for (int c = 0; c < 64; ++c) x[c] = (c >= c_lo && c <= c_hi) ? x[c] : -INFINITY;
+            }
+            if (kKpad) {
+              uint32_t pm[2];
+              const uint8_t* fl = a.kpad + (size_t)(it.bh / a.H) * a.N;
+#pragma unroll
+              for (int g = 0; g < 2; ++g) {
+                const int col = j * kBlock + 64 * h + 32 * g + lane;
+                pm[g] = __ballot_sync(0xffffffffu, col < a.N && fl[col] != 0);
+              }
+              if ((pm[0] | pm[1]) != 0u) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                  x[c] = ((pm[c >> 5] >> (c & 31)) & 1u) ? -INFINITY : x[c];
+              }
+            }
+            float mx;
+            {
+              float t[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) t[e] = fmax3(x[e], x[e + 16], x[e + 32]);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) t[e] = fmaxf(t[e], x[48 + e]);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) t[e] = fmax3(t[e], t[e + 4], t[e + 8]);
+              mx = fmax3(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[12], t[13]),
+                         fmaxf(t[14], t[15]));
+            }
+            const float m_new = fmaxf(m_run, mx * xs);
+            const bool grow = m_new > m_run + 8.0f;
+            float alpha = 1.f;
+            if (grow) {
+              alpha = ex2(m_run - m_new);
+              m_run = m_new;
+              l_run *= alpha;
+            }
+            const float mb = (m_run == -INFINITY) ? 0.f : m_run;
+            // P over the first columns of this half of S_s, 32 keys at a time
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              if constexpr (kFp8) {
+                uint32_t pk[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                  float p4[4];
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) p4[e] = ex2(fmaf(x[32 * hh + 4 * c + e], xs, -mb));
+                  ls[c & 3] += (p4[0] + p4[1]) + (p4[2] + p4[3]);
+                  pk[c] = pack_e4m3x4(p4[0], p4[1], p4[2], p4[3]);
+                }
+                tmem_st8(tSh + 8 * hh, pk);
+              } else {
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                  float p0 = ex2(fmaf(x[32 * hh + 2 * c], xs, -mb));
+                  float p1 = ex2(fmaf(x[32 * hh + 2 * c + 1], xs, -mb));
+                  ls[c & 3] += p0 + p1;
+                  if (kDropout) {
+                    p0 = ((keep[hh] >> (2 * c)) & 1u) ? p0 : 0.f;
+                    p1 = ((keep[hh] >> (2 * c + 1)) & 1u) ? p1 : 0.f;
+                  }
+                  pk[c] = pack_bf16x2(p0, p1);
+                }
+                tmem_st16(tSh + 16 * hh, pk);
+              }
+            }
+            l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            // rescale this row of O before P_h V accumulates into it, once the previous
+            // half's P V (the last product into O) has completed
+            if (!(j == rg.lo && h == 0) && __any_sync(0xffffffffu, grow)) {
+              const int hp = h ^ 1;
+              if (!mbar_wait_warp(bar((hp ? C::bODone2 : C::bODone) + s), (npub[hp] - 1) & 1,
+                                  abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+#pragma unroll
+              for (int q = 0; q < D / 32; ++q) {
+                uint32_t o[32];
+                tmem_ld32(tO + 32 * q, o);
+                tmem_wait_ld();
+                reg_fence(o);
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                  o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                tmem_st32(tO + 32 * q, o);
+              }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive_warp(bar((h ? C::bPFull2 : C::bPFull) + s));
+            ++nsh[h];
+            ++npub[h];
           }
-          pass_turn();
+          if (!ok) break;
           continue;
         }
         // keep flags of this row's 128 weights (they depend on no score, so they are drawn
@@ -594,10 +818,6 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
           l_run *= alpha;
         }
         const float mb = (m_run == -INFINITY) ? 0.f : m_run;
-        if (turns && !take_turn()) {
-          ok = false;
-          break;
-        }
         // with separate P, P_s and O_s are free once the previous P V has completed
         if (C::kSepP && ns > 0) {
           if (!mbar_wait_warp(bar(C::bODone + s), (ns - 1) & 1, abort_flag)) {
@@ -639,7 +859,6 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
             tmem_st16(tP + 16 * h, pk);
           }
         }
-        if (turns) pass_turn();
         l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         // rescale this row of O before P_s V_j accumulates into it (that waits for p_full)
         if (j > rg.lo && __any_sync(0xffffffffu, grow)) {
@@ -661,7 +880,8 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
       }
       if (!ok) break;
       // epilogue of the item: O / l and LSE, once the last P V product has completed
-      if (!mbar_wait_warp(bar(C::bODone + s), (ns - 1) & 1, abort_flag)) {
+      if (!(C::kHalves ? mbar_wait_warp(bar(C::bODone2 + s), (npub[1] - 1) & 1, abort_flag)
+                       : mbar_wait_warp(bar(C::bODone + s), (ns - 1) & 1, abort_flag))) {
         ok = false;
         break;
       }
