@@ -35,42 +35,60 @@ L2_BYTES = 126 * 1024 * 1024
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a kernel on a
-# workload, from one ncu capture, keyed by the SHA-256 of the kernel sources the capture
-# ran (kernel_source_hash()); an entry whose hash no longer matches is reported as null.
+# workload, from one ncu capture, with the SHA-256 of the sources that kernel was built from
+# (kernel_source_hash(kernel)); an entry whose hash no longer matches is reported as null.
 MEASURED_TRAFFIC = {
-    ("c4_causal_b32h16n2048d64", "fwd"): (973623296, "5a5757760830",
+    ("c4_causal_b32h16n2048d64", "fwd"): (970862336, "2dd28ea17974",
                                           "ncu --set full, one launch"),
-    ("c4_causal_b32h16n2048d64", "bwd_preprocess"): (416424704, "5a5757760830",
+    ("c5_causal_b2h32n8192d128", "fwd"): (1051133952, "2dd28ea17974",
+                                          "ncu --set full, one launch"),
+    ("c4_causal_b32h16n2048d64", "bwd_preprocess"): (416424704, "3ca0efabb645",
                                                      "ncu --set full, one launch"),
-    ("c4_causal_b32h16n2048d64", "bwd_dkdv"): (791025408, "5a5757760830",
+    ("c4_causal_b32h16n2048d64", "bwd_dkdv"): (791025408, "3ca0efabb645",
                                                "ncu --set full, one launch"),
-    ("c4_causal_b32h16n2048d64", "bwd_dq"): (666822144, "5a5757760830",
+    ("c4_causal_b32h16n2048d64", "bwd_dq"): (666822144, "3ca0efabb645",
                                              "ncu --set full, one launch"),
-    ("c5_causal_b2h32n8192d128", "fwd"): (1098435584, "5a5757760830",
-                                          "ncu --set full, one launch"),
-    ("c5_causal_b2h32n8192d128", "bwd_dkdv"): (796998208, "5a5757760830",
+    ("c5_causal_b2h32n8192d128", "bwd_dkdv"): (796998208, "3ca0efabb645",
                                                "ncu --set full, one launch"),
-    ("c5_causal_b2h32n8192d128", "bwd_dq"): (665432832, "5a5757760830",
+    ("c5_causal_b2h32n8192d128", "bwd_dq"): (665432832, "3ca0efabb645",
                                              "ncu --set full, one launch"),
 }
 
 
-def kernel_source_hash() -> str:
-    """SHA-256 (first 12 hex digits) of the CUDA sources of the library."""
+# The sources each kernel is compiled from, besides the shared headers: a measured traffic
+# figure stays valid while these are unchanged.
+COMMON_SOURCES = ("sm100.cuh", "tiles.cuh", "rng.cuh", "launch_impl.cuh", "launch.h")
+KERNEL_SOURCES = {
+    "fwd": ("fa_fwd.cuh",),
+    "bwd_preprocess": ("fa_bwd.cuh",),
+    "bwd_dkdv": ("fa_bwd.cuh",),
+    "bwd_dq": ("fa_bwd.cuh",),
+    "bwd_fused": ("fa_bwd_fused.cuh", "fa_bwd.cuh"),
+    "bwd_dq_convert": ("fa_bwd_fused.cuh", "fa_bwd.cuh"),
+}
+
+
+def kernel_source_hash(kernel: str | None = None) -> str:
+    """SHA-256 (first 12 hex digits) of the CUDA sources of the library, or, for a kernel
+    named in KERNEL_SOURCES, of the shared headers and that kernel's own sources."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_attention_126_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    if kernel in KERNEL_SOURCES:
+        names = sorted(COMMON_SOURCES + KERNEL_SOURCES[kernel])
+    else:
+        names = sorted(n for n in os.listdir(csrc) if n.endswith((".cu", ".cuh", ".h")))
+    for name in names:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:12]
 
 
 def measured_traffic(workload: str, kernel: str):
-    """(bytes per launch, source) from MEASURED_TRAFFIC if it was taken on these sources."""
+    """(bytes per launch, source) from MEASURED_TRAFFIC if it was taken on the sources the
+    kernel is built from now."""
     entry = MEASURED_TRAFFIC.get((workload, kernel))
-    if entry is None or entry[1] != kernel_source_hash():
+    if entry is None or entry[1] != kernel_source_hash(kernel):
         return None, None
     return entry[0], entry[2]
 

@@ -86,9 +86,19 @@ def test_roofline_peak_follows_the_timed_region():
 def test_traffic_is_null_once_the_kernels_change(monkeypatch):
     sys.path.insert(0, ROOT)
     import bench
-    h = bench.kernel_source_hash()
+    h = bench.kernel_source_hash("k")
     monkeypatch.setattr(bench, "MEASURED_TRAFFIC", {
         ("w", "k"): (123, h, "ncu capture"), ("w", "old"): (456, "0" * 12, "old capture")})
     assert bench.measured_traffic("w", "k") == (123, "ncu capture")
     assert bench.measured_traffic("w", "old") == (None, None)
     assert bench.measured_traffic("w", "none") == (None, None)
+
+
+def test_traffic_hash_covers_only_the_kernels_sources():
+    """A kernel's traffic figure depends on the shared headers and its own sources only."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.kernel_source_hash("bwd_dkdv") == bench.kernel_source_hash("bwd_dq")
+    assert bench.kernel_source_hash("bwd_dkdv") != bench.kernel_source_hash("fwd")
+    assert bench.kernel_source_hash() not in (bench.kernel_source_hash("fwd"),
+                                              bench.kernel_source_hash("bwd_dkdv"))

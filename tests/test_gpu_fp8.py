@@ -15,7 +15,7 @@ from exact_attention_126_b200 import fa, synth
 
 pytestmark = pytest.mark.gpu
 
-TOL_O_FP8 = 5e-2
+TOL_O_FP8 = G.TOL_O_FP8
 
 MODES = {
     "none": (False, (-1, -1)),

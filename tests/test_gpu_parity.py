@@ -69,10 +69,39 @@ def test_workload_full_size(name):
     the first, the last and two seeded random (batch, head) pairs (c4, c5)."""
     w = WORKLOADS[name]
     inp = inputs(w.B, w.H, w.N, w.d, w.seed_index)
-    slopes = alibi_slopes(w.H) if w.alibi else None
-    out = G.run_library(inp, w.softmax_scale, w.causal, w.window, w.backward, slopes)
     heads = None if w.B * w.H * w.N <= 2 * 8 * 4096 else _sampled_heads(w)
-    errs = G.compare(inp, out, w.softmax_scale, w.causal, w.window, heads, w.backward, slopes)
+    if w.fp8:
+        # the e4m3 forward on the seeded inputs rounded to e4m3 (descales 1), against the
+        # oracle on exactly those values, at the FP8 bound on O
+        G.ensure_built()
+        dev = torch.device("cuda:0")
+        x8 = {n: inp[n].float().to(torch.float8_e4m3fn) for n in ("q", "k", "v")}
+        o, lse = fa.attention_forward_fp8(x8["q"].to(dev), x8["k"].to(dev), x8["v"].to(dev),
+                                          scale=w.softmax_scale, causal=w.causal,
+                                          window=w.window)
+        torch.cuda.synchronize()
+        assert fa.fa_debug_status() == 0
+        ref = {n: x8[n].to(torch.float64).numpy() for n in ("q", "k", "v")}
+        pick = lambda a: np.stack([a[b, h] for b, h in heads])[None]
+        o_ref, lse_ref = G.oracle.fwd(pick(ref["q"]), pick(ref["k"]), pick(ref["v"]),
+                                      w.softmax_scale, w.causal, w.window)
+        err_o = G.rel_frob(pick(synth.to_f64(o.cpu())), o_ref)
+        err_l = float(np.abs(pick(lse.cpu().double().numpy()) - lse_ref).max())
+        print(name, {"o": err_o, "lse": err_l})
+        assert err_o <= G.TOL_O_FP8 and err_l <= G.TOL_LSE, (err_o, err_l)
+        return
+    slopes = alibi_slopes(w.H) if w.alibi else None
+    lengths = w.seq_lengths() if w.varlen else None
+    out = G.run_library(inp, w.softmax_scale, w.causal, w.window, w.backward, slopes,
+                        lengths=lengths)
+    if lengths is not None and heads is not None:
+        # one sampled head at a time, each with its batch entry's real length
+        per = [G.compare(inp, out, w.softmax_scale, w.causal, w.window, [bh], w.backward,
+                         slopes, lengths=lengths) for bh in heads]
+        errs = {key: max(e[key] for e in per) for key in per[0]}
+    else:
+        errs = G.compare(inp, out, w.softmax_scale, w.causal, w.window, heads, w.backward,
+                         slopes)
     print(name, errs)
     G.assert_within_bounds(errs, name)
 
