@@ -157,6 +157,8 @@ struct BwdArgs {
   int n_items;          // BH * n_tiles: one item per (batch*head, stationary tile)
   int longest_first;    // masked problems: chunks of `group` heads, longest items first
   int group;
+  int paired;           // causal problems: complementary items paired per CTA (paired_item)
+  int n_double;         // ... over n_double pairs; n_items then counts the schedule's slots
   float scale;
   float scale_log2;
   int left;
@@ -308,7 +310,9 @@ __device__ __forceinline__ constexpr uint32_t packed_col(int kk) {
 // advancing its counters. `mk` is the item's mask, over the real length.
 __device__ __forceinline__ bool bwd_item(int k, const BwdArgs& a, bool rising, int& bh,
                                          int& tile, Mask& mk) {
-  if (a.longest_first) {
+  if (a.paired) {
+    if (!paired_item(k, (int)gridDim.x, a.n_double, a.n_tiles, rising, bh, tile)) return false;
+  } else if (a.longest_first) {
     chunked_item(k, a.BH, a.n_tiles, a.group, rising, bh, tile);
   } else {
     bh = k / a.n_tiles;

@@ -49,6 +49,8 @@ struct FwdArgs {
   int n_items;        // BH * n_pairs
   int longest_first;  // masked problems: chunks of `group` heads, longest items first
   int group;
+  int paired;         // causal problems: complementary items paired per CTA (paired_item)
+  int n_double;       // ... over n_double pairs; n_items then counts the schedule's slots
   float scale_log2;   // scale * log2(e)
   int left;
   int right;
@@ -141,7 +143,20 @@ struct FwdItem {
 __device__ __forceinline__ FwdItem fwd_item(int k, const FwdArgs& a) {
   FwdItem it;
   int pair;
-  if (a.longest_first) {
+  if (a.paired) {
+    if (!paired_item(k, (int)gridDim.x, a.n_double, a.n_pairs, false, it.bh, pair)) {
+      // a slot past the last pair: no work
+      it.bh = 0;
+      it.n = 0;
+      it.m[0] = it.m[1] = 0;
+      it.has_a = it.has_b = false;
+      it.lo[0] = it.lo[1] = 1;
+      it.hi[0] = it.hi[1] = 0;
+      it.first = 1;
+      it.last = 0;
+      return it;
+    }
+  } else if (a.longest_first) {
     chunked_item(k, a.BH, a.n_pairs, a.group, false, it.bh, pair);
   } else {
     it.bh = k / a.n_pairs;

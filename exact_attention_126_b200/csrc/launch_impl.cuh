@@ -104,6 +104,29 @@ inline int head_group(int BH, int tiles) {
   return g;
 }
 
+// The causal schedule of paired_item: for a causal mask (no window), an even number T of
+// tiles per head and one length for every batch entry, items go in complementary pairs
+// (with real lengths the pairs would not weigh the same). Sets paired, n_double and n_items
+// (the slots of whole round pairs over the grid that persistent_grid() returns).
+template <typename Args>
+inline void pair_schedule(Args& a, int BH, int T, int left, int right, bool varlen) {
+  a.paired = (left < 0 && right == 0 && T % 2 == 0 && !varlen) ? 1 : 0;
+  a.n_double = 0;
+  if (a.paired) {
+    a.n_double = BH * (T / 2);
+    const int P = a.n_double < sm_count() ? a.n_double : sm_count();
+    a.n_items = 2 * ((a.n_double + P - 1) / P) * P;
+  }
+}
+
+// Persistent CTAs: one per SM, or one per item (one per pair of items with the causal
+// schedule) when there are fewer.
+template <typename Args>
+inline int persistent_grid(const Args& a) {
+  const int units = a.paired ? a.n_double : a.n_items;
+  return units < sm_count() ? units : sm_count();
+}
+
 inline fa_status_t launched() {
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -136,6 +159,7 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   a.n_items = BH * a.n_pairs;
   a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
   a.group = head_group(BH, a.n_pairs);
+  pair_schedule(a, BH, a.n_pairs, left, right, x.seq_len != nullptr);
   a.scale_log2 = scale * fa::kLog2e;
   a.left = left;
   a.right = right;
@@ -147,7 +171,7 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   a.drop = x.drop;
   a.seq_len = x.seq_len;
   a.o_scale = x.o_scale;
-  const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
+  const int grid = persistent_grid(a);
   fa::fa_fwd_kernel<D, kFeat><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, a);
   return launched();
 }
@@ -188,6 +212,7 @@ inline fa::BwdArgs bwd_args(const void* ws, const Problem& pb, const Extras& x) 
   a.n_items = BH * a.n_tiles;
   a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
   a.group = head_group(BH, a.n_tiles);
+  pair_schedule(a, BH, a.n_tiles, left, right, x.seq_len != nullptr);
   a.alibi = x.alibi;
   a.H = H;
   a.kpad = x.kpad;
@@ -211,7 +236,7 @@ fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void*
   fa::BwdArgs a = bwd_args(ws, pb, x);
   a.out0 = static_cast<__nv_bfloat16*>(dk);
   a.out1 = static_cast<__nv_bfloat16*>(dv);
-  const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
+  const int grid = persistent_grid(a);
   fa::fa_bwd_dkdv_kernel<D, kFeat><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo,
                                                                                mdk, mdv, a);
   return launched();
@@ -231,7 +256,7 @@ fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* d
   if (set_smem(fa::fa_bwd_dq_kernel<D, kFeat>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
   fa::BwdArgs a = bwd_args(ws, pb, x);
   a.out0 = static_cast<__nv_bfloat16*>(dq);
-  const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
+  const int grid = persistent_grid(a);
   fa::fa_bwd_dq_kernel<D, kFeat><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, mdq,
                                                                              a);
   return launched();
@@ -254,7 +279,7 @@ fa_status_t launch_fused(const void* q, const void* k, const void* v, const void
   fa::BwdArgs a = bwd_args(ws, pb, x);
   a.out0 = static_cast<__nv_bfloat16*>(dk);
   a.out1 = static_cast<__nv_bfloat16*>(dv);
-  const int grid = a.n_items < sm_count() ? a.n_items : sm_count();
+  const int grid = persistent_grid(a);
   fa::fa_bwd_fused_kernel<kFeat><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, mdo, mdk,
                                                                            mdv, macc, a);
   return launched();

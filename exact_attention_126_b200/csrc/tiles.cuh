@@ -124,4 +124,26 @@ __host__ __device__ inline void chunked_item(int k, int BH, int T, int group, bo
   tile = rising ? step : T - 1 - step;
 }
 
+// Work item of slot k of a persistent schedule for causal problems, where tile t of a head
+// has work growing linearly with t (or with T - 1 - t): the items go in pairs of a tile and
+// its complement T - 1 - t of the same head, whose work adds up to the same for every pair.
+// CTA c (of P) takes pair q = (r / 2) P + c of its rounds r = 2m, 2m + 1: the longer item in
+// round 2m, the shorter in 2m + 1. Every CTA then gets nearly the same work, and the two
+// items of a pair read the same head's tiles one after the other (from L2 the second time).
+// Returns false for the slots past the last pair (n_double = BH T / 2 pairs, T even).
+// `rising`: tile 0 is the longest (dK/dV), else tile T - 1 (forward, dQ).
+__host__ __device__ inline bool paired_item(int k, int P, int n_double, int T, bool rising,
+                                            int& bh, int& tile) {
+  const int r = k / P;
+  const int c = k - r * P;
+  const int q = (r >> 1) * P + c;
+  if (q >= n_double) return false;
+  const int half = T / 2;
+  bh = q / half;
+  const int p = q - bh * half;
+  const int longer = rising ? p : T - 1 - p;
+  tile = (r & 1) ? T - 1 - longer : longer;
+  return true;
+}
+
 }  // namespace fa

@@ -83,6 +83,35 @@ int main() {
           for (int v : seen)
             if (v != 1) return fail("chunked_item cover", BH, T, group, rising);
         }
+  // paired_item: over the whole round pairs of P CTAs every (head, tile) appears exactly
+  // once, each CTA's two items of a round pair are a tile and its complement of one head
+  // (longer first), and with work t + 1 (or T - t) per tile every pair weighs T + 1.
+  for (int BH = 1; BH <= 9; ++BH)
+    for (int T = 2; T <= 12; T += 2)
+      for (int P = 1; P <= 13; ++P)
+        for (int rising = 0; rising < 2; ++rising) {
+          const int n_double = BH * (T / 2);
+          const int Pg = n_double < P ? n_double : P;
+          const int slots = 2 * ((n_double + Pg - 1) / Pg) * Pg;
+          std::vector<int> seen(BH * T, 0);
+          for (int k = 0; k < slots; ++k) {
+            int bh, tile;
+            if (!paired_item(k, Pg, n_double, T, rising != 0, bh, tile)) continue;
+            if (bh < 0 || bh >= BH || tile < 0 || tile >= T) return fail("paired_item range", BH, T, Pg, k);
+            ++seen[bh * T + tile];
+            const int r = k / Pg;
+            if (r % 2 == 1) {
+              int bh0, tile0;
+              if (!paired_item(k - Pg, Pg, n_double, T, rising != 0, bh0, tile0))
+                return fail("paired_item partner", BH, T, Pg, k);
+              const int w0 = rising ? T - tile0 : tile0 + 1, w1 = rising ? T - tile : tile + 1;
+              if (bh0 != bh || tile0 + tile != T - 1 || w0 < w1 || w0 + w1 != T + 1)
+                return fail("paired_item pair", BH, T, Pg, k);
+            }
+          }
+          for (int v : seen)
+            if (v != 1) return fail("paired_item cover", BH, T, Pg, rising);
+        }
   std::printf("OK\n");
   return 0;
 }
