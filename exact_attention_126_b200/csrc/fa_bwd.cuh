@@ -197,8 +197,8 @@ struct BwdCfgT {
   static constexpr int bY0Empty = bY0Full + S0;
   static constexpr int bY1Full = bY0Empty + S0;
   static constexpr int bY1Empty = bY1Full + S1;
-  static constexpr int bA = bY1Empty + S1;  // 12 kernel-specific barriers
-  static constexpr int bMmaFin = bA + 12;   // + issuer
+  static constexpr int bA = bY1Empty + S1;  // 16 kernel-specific barriers
+  static constexpr int bMmaFin = bA + 16;   // + issuer
   static constexpr int kNumBars = bMmaFin + 2;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kSmemBytes = kMisc + 16 + 1024;
@@ -381,6 +381,11 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
   constexpr bool kDropout = (kFeat & kFeatDropout) != 0;
   constexpr int kSBufs = (D == 64) ? 2 : 1;
   constexpr bool kDsInS = kSBufs == 2;               // dS^T over the second half of S^T
+  // With one S^T buffer (head_dim 128) the products go in two 64-query halves: S^T, dP^T,
+  // dV and dK of half h have barriers of their own, so S^T of half h of the next tile waits
+  // only for dV of half h (and dP^T for dK of half h), while the other half's products
+  // run. Softmax warpgroups 0, 1 own half 0 of the query columns, 2, 3 half 1.
+  constexpr bool kHalves = !kDsInS;
   constexpr uint32_t tS = 0;                         // + 128 * buffer
   constexpr uint32_t tDP = 128 * kSBufs, tDK = tDP + 128, tDV = tDK + D;
   static_assert(tDV + D <= C::kTmemCols, "tensor memory columns");
@@ -397,6 +402,10 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
                 bDPFull = C::bA + 6, bDSFull = kDsInS ? C::bA + 4 : C::bA + 7,
                 bDPFree = C::bA + 8, bAccFree = C::bA + 9, bAccReady = C::bA + 10,
                 bStaged = C::bA + 11;
+  // kHalves: dP^T full, dS^T full and dP^T free of half 1 (those above serve half 0; S^T
+  // full, P^T full and S^T free are kept per half in their two slots)
+  constexpr int bDPFull1 = C::bA + 12, bDSFull1 = C::bA + 13, bDPFree1 = C::bA + 14;
+  auto half_bar = [](int b0, int b1, int h) { return h ? b1 : b0; };
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -421,15 +430,22 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
       mbar_init(bar(C::bY1Full + s), 1);
       mbar_init(bar(C::bY0Empty + s), 1);
     }
+    // softmax warps that publish a P^T or dS^T: all of them, or with kHalves those of a half
+    constexpr int kPub = kHalves ? C::kSoftmax / 64 : C::kSoftmax / 32;
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(bSFull + b), 1);
-      mbar_init(bar(bPFull + b), C::kSoftmax / 32);
+      mbar_init(bar(bPFull + b), kPub);
       mbar_init(bar(bSFree + b), kDsInS ? C::kSoftmax / 32 : 1);  // dS^T full with kDsInS
       mbar_init(bar(C::bMmaFin + b), 1);
     }
     mbar_init(bar(bDPFull), 1);
-    if (!kDsInS) mbar_init(bar(bDSFull), C::kSoftmax / 32);
+    if (!kDsInS) mbar_init(bar(bDSFull), kPub);
     mbar_init(bar(bDPFree), kDsInS ? C::kSoftmax / 32 : 1);
+    if (kHalves) {
+      mbar_init(bar(bDPFull1), 1);
+      mbar_init(bar(bDSFull1), kPub);
+      mbar_init(bar(bDPFree1), 1);
+    }
     mbar_init(bar(bAccFree), C::kSoftmax / 32);
     mbar_init(bar(bAccReady), 1);
     mbar_init(bar(bStaged), C::kSoftmax / 32);
@@ -506,6 +522,56 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
         if (!mbar_wait(bar(C::bXFull + xb), xu & 1, abort_flag)) break;
         for (int i = i_lo; i <= i_hi; ++i, ++t) {
           const int b = t % kSBufs, s0 = t % C::kStages0, s1 = s0;
+          if constexpr (kHalves) {
+            // S^T_h = K_j Q_i[64h ..]^T, then dP^T_h = V_j dO_i[64h ..]^T, each once the
+            // previous tile's product that read its columns (dV_h, dK_h) has completed
+            constexpr uint32_t idS64 = idesc_bf16_f32(128, 64, false, false);
+            if (!mbar_wait(bar(C::bY0Full + s0), (t / C::kStages0) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            for (int h = 0; h < 2 && ok; ++h) {
+              if (t >= 1 && !mbar_wait(bar(bSFree + h), (t - 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint64_t dx = sdesc_sw128(sb + C::kX0 + xb * 2 * C::kTile, 16, 1024);
+              const uint64_t dy = sdesc_sw128(sb + C::kY0 + s0 * C::kTile + 64 * 128 * h, 16, 1024);
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
+                mma_ss(tmem + tS + 64u * h, sdesc_add(dx, off), sdesc_add(dy, off), idS64,
+                       kk > 0);
+              }
+              tc_commit(bar(bSFull + h));
+            }
+            if (!ok) break;
+            if (!mbar_wait(bar(C::bY1Full + s1), (t / C::kStages1) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            for (int h = 0; h < 2 && ok; ++h) {
+              if (t >= 1 &&
+                  !mbar_wait(bar(half_bar(bDPFree, bDPFree1, h)), (t - 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint64_t dx = sdesc_sw128(sb + C::kX1 + xb * 2 * C::kTile, 16, 1024);
+              const uint64_t dy = sdesc_sw128(sb + C::kY1 + s1 * C::kTile + 64 * 128 * h, 16, 1024);
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * C::kRegionBytes + (kk & 3) * 32;
+                mma_ss(tmem + tDP + 64u * h, sdesc_add(dx, off), sdesc_add(dy, off), idS64,
+                       kk > 0);
+              }
+              tc_commit(bar(half_bar(bDPFull, bDPFull1, h)));
+            }
+            if (!ok) break;
+            if (!C::kStageOut && i == i_hi) tc_commit(bar(C::bXEmpty + xb));
+            continue;
+          }
           // S^T = K_j Q_i^T, once the products that read its buffer's P^T (and dS^T) have
           // completed: dV of the previous tile, or with kDsInS dK of tile t - 2, whose
           // completion releases that tile's ring stage
@@ -570,6 +636,56 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
         for (int i = i_lo; i <= i_hi; ++i, ++t) {
           const int b = t % kSBufs, s0 = t % C::kStages0, s1 = s0;
           const bool first = i == i_lo;
+          if constexpr (kHalves) {
+            // dV += P^T_h dO_i[64h ..] (K-steps 4h .. 4h+3) as each half of P^T is
+            // published, then dK += dS^T_h Q_i[64h ..] likewise; the item's first product
+            // overwrites dV (dK), which the previous item's epilogue must have read
+            if (!mbar_wait(bar(C::bY1Full + s1), (t / C::kStages1) & 1, abort_flag) ||
+                (first && items > 0 && !mbar_wait(bar(bAccFree), (items - 1) & 1, abort_flag))) {
+              ok = false;
+              break;
+            }
+            const uint64_t dyo = sdesc_sw128(sb + C::kY1 + s1 * C::kTile, C::kRegionBytes, 1024);
+            for (int h = 0; h < 2 && ok; ++h) {
+              if (!mbar_wait(bar(bPFull + h), t & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+#pragma unroll
+              for (int kq = 0; kq < 4; ++kq) {
+                const int kk = 4 * h + kq;
+                mma_ts(tmem + tDV, tmem + tS + packed_col(kk), sdesc_add(dyo, kk * 2048), idA,
+                       (!first || kk > 0) ? 1u : 0u);
+              }
+              tc_commit(bar(bSFree + h));
+            }
+            if (!ok) break;
+            if (!mbar_wait(bar(C::bY0Full + s0), (t / C::kStages0) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            const uint64_t dyq = sdesc_sw128(sb + C::kY0 + s0 * C::kTile, C::kRegionBytes, 1024);
+            for (int h = 0; h < 2 && ok; ++h) {
+              if (!mbar_wait(bar(half_bar(bDSFull, bDSFull1, h)), t & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+#pragma unroll
+              for (int kq = 0; kq < 4; ++kq) {
+                const int kk = 4 * h + kq;
+                mma_ts(tmem + tDK, tmem + tDP + packed_col(kk), sdesc_add(dyq, kk * 2048), idA,
+                       (!first || kk > 0) ? 1u : 0u);
+              }
+              tc_commit(bar(half_bar(bDPFree, bDPFree1, h)));
+            }
+            if (!ok) break;
+            // the tile's ring stage is free
+            tc_commit(bar(C::bY0Empty + s0));
+            if (i == i_hi) tc_commit(bar(bAccReady));  // dK, dV of the item are complete
+            continue;
+          }
           // dV += P^T dO_i; the item's first product overwrites dV, which the previous
           // item's epilogue must have read
           if (!mbar_wait(bar(C::bY1Full + s1), (t / C::kStages1) & 1, abort_flag) ||
@@ -679,7 +795,8 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
           }
         }
         if (!mbar_wait_warp(bar(C::bY0Full + s), (t / C::kStages0) & 1, abort_flag) ||
-            !mbar_wait_warp(bar(bSFull + t % kSBufs), (t / kSBufs) & 1, abort_flag)) {
+            !mbar_wait_warp(bar(bSFull + (kHalves ? (h >> 1) : t % kSBufs)), (t / kSBufs) & 1,
+                            abort_flag)) {
           ok = false;
           break;
         }
@@ -731,8 +848,9 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive_warp(bar(bPFull + t % kSBufs));
-        if (!mbar_wait_warp(bar(bDPFull), t & 1, abort_flag)) {
+        mbar_arrive_warp(bar(bPFull + (kHalves ? (h >> 1) : t % kSBufs)));
+        if (!mbar_wait_warp(bar(kHalves ? half_bar(bDPFull, bDPFull1, h >> 1) : bDPFull), t & 1,
+                            abort_flag)) {
           ok = false;
           break;
         }
@@ -763,7 +881,8 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
         tmem_st16(kDsInS ? tSb + 16 : tmem + lane_base + tDP + NC * h, w);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive_warp(bar(bDSFull + (kDsInS ? t % kSBufs : 0)));
+        mbar_arrive_warp(bar(kHalves ? half_bar(bDSFull, bDSFull1, h >> 1)
+                                     : bDSFull + (kDsInS ? t % kSBufs : 0)));
       }
       if (!ok) break;
       g += n_it;
