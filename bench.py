@@ -418,37 +418,63 @@ def run_ours(args, w, rank, world, local_rank):
     h2d_bytes = sum(inp_host[n].numel() * inp_host[n].element_size() for n in in_names)
     d2h_bytes = sum(host_out[n].numel() * host_out[n].element_size() for n in out_names)
 
-    def e2e_step():
-        for n, t in zip(("q", "k", "v", "do"), (q, k, v, do)):
-            if n in in_names:
-                t.copy_(inp_host[n], non_blocking=True)
-        if w.fp8:
-            res = fa.attention_forward_fp8(q, k, v, scale=w.softmax_scale, causal=w.causal,
-                                           window=w.window, stream=sp)
-        else:
-            res = fa.attention_forward(q, k, v, w.softmax_scale, w.causal, w.window, sp,
-                                       alibi_slopes=prob.slopes, keep_residual=w.backward,
-                                       seq_lengths=prob.lengths)
-        host_out["o"].copy_(res[0], non_blocking=True)
-        host_out["lse"].copy_(res[1], non_blocking=True)
-        if w.backward:
-            grads = fa.attention_backward(q, k, v, res[0], res[1], do, w.softmax_scale, w.causal,
-                                          w.window, sp, alibi_slopes=prob.slopes, o_low=res[2],
-                                          fused=args.fused,
-                                          seq_lengths=prob.lengths)
-            for n, t in zip(("dq", "dk", "dv"), grads):
-                host_out[n].copy_(t, non_blocking=True)
+    # Steps are pipelined over three streams: the host-to-device copies of step k + 1 and
+    # the device-to-host copies of step k - 1 run on the two copy engines while step k
+    # computes. Inputs go through two device buffer sets, each reused once the step that
+    # read it has finished; outputs are fresh tensors from the public calls, kept alive for
+    # their copy stream.
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    dev_in = [{n: torch.empty_like(t) for n, t in zip(("q", "k", "v", "do"), (q, k, v, do))}
+              for _ in range(2)]
+    freed = [None, None]  # event: the compute that last read buffer set b has finished
 
-    e2e_step()
+    def e2e_step(step):
+        b = step % 2
+        bufs = dev_in[b]
+        with torch.cuda.stream(s_in):
+            if freed[b] is not None:
+                s_in.wait_event(freed[b])
+            for n in in_names:
+                bufs[n].copy_(inp_host[n], non_blocking=True)
+            loaded = torch.cuda.Event()
+            loaded.record(s_in)
+        stream.wait_event(loaded)
+        with torch.cuda.stream(stream):  # the outputs are allocated for the compute stream
+            if w.fp8:
+                res = fa.attention_forward_fp8(bufs["q"], bufs["k"], bufs["v"],
+                                               scale=w.softmax_scale, causal=w.causal,
+                                               window=w.window, stream=sp)
+            else:
+                res = fa.attention_forward(bufs["q"], bufs["k"], bufs["v"], w.softmax_scale,
+                                           w.causal, w.window, sp, alibi_slopes=prob.slopes,
+                                           keep_residual=w.backward, seq_lengths=prob.lengths)
+            outs = [("o", res[0]), ("lse", res[1])]
+            if w.backward:
+                grads = fa.attention_backward(bufs["q"], bufs["k"], bufs["v"], res[0], res[1],
+                                              bufs["do"], w.softmax_scale, w.causal, w.window,
+                                              sp, alibi_slopes=prob.slopes, o_low=res[2],
+                                              fused=args.fused, seq_lengths=prob.lengths)
+                outs += list(zip(("dq", "dk", "dv"), grads))
+            done = torch.cuda.Event()
+            done.record(stream)
+        freed[b] = done
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done)
+            for n, t in outs:
+                t.record_stream(s_out)
+                host_out[n].copy_(t, non_blocking=True)
+        return s_out
+
+    e2e_step(0)
     torch.cuda.synchronize(dev)
     if dist is not None:
         dist.barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_in)
+    for i in range(e2e_steps):
+        last = e2e_step(i + 1)
+    e1.record(last)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
     if dist is not None:
@@ -655,7 +681,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="c4",
                     help="c1, c2, c3, c4, c5c, c5w, c4a, c4v or c5f8")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--also", default="c2,c3,c4,c5c,c5w,c4v,c5f8",
