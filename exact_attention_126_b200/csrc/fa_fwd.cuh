@@ -45,7 +45,9 @@ struct FwdArgs {
   int N;
   int BH;
   int n_qtiles;
-  int n_pairs;        // items per (batch, head): query tiles taken two at a time
+  int n_pairs;        // items per (batch, head): query tiles taken per_item at a time
+  int per_item;       // query tiles per item: 2 (streams A and B), or 1 when pairs would
+                      // leave SMs idle (stream B then has no tile)
   int n_items;        // BH * n_pairs
   int longest_first;  // masked problems: chunks of `group` heads, longest items first
   int group;
@@ -165,10 +167,10 @@ __device__ __forceinline__ FwdItem fwd_item(int k, const FwdArgs& a) {
   it.n = real_length(a.seq_len, it.bh, a.H, a.N);
   const Mask mk{it.n, a.left, a.right};
   const int n_qtiles = num_tiles(it.n);
-  it.m[0] = 2 * pair;
-  it.m[1] = 2 * pair + 1;
+  it.m[0] = a.per_item * pair;
+  it.m[1] = it.m[0] + 1;
   it.has_a = it.m[0] < n_qtiles;
-  it.has_b = it.m[1] < n_qtiles;
+  it.has_b = a.per_item == 2 && it.m[1] < n_qtiles;
   kv_tiles_for_q_tile(it.m[0], mk, it.lo[0], it.hi[0]);
   if (it.has_b) {
     kv_tiles_for_q_tile(it.m[1], mk, it.lo[1], it.hi[1]);

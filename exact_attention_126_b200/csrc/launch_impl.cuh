@@ -155,7 +155,9 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   a.N = N;
   a.BH = BH;
   a.n_qtiles = fa::num_tiles(N);
-  a.n_pairs = (a.n_qtiles + 1) / 2;
+  // two query tiles per item, unless that leaves SMs without an item
+  a.per_item = (BH * ((a.n_qtiles + 1) / 2) < sm_count() && a.n_qtiles > 1) ? 1 : 2;
+  a.n_pairs = (a.n_qtiles + a.per_item - 1) / a.per_item;
   a.n_items = BH * a.n_pairs;
   a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
   a.group = head_group(BH, a.n_pairs);
