@@ -245,9 +245,6 @@ class Problem:
         self.o_low = torch.empty_like(self.q)
         self.lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
         self.dq, self.dk, self.dv = (torch.empty_like(self.q) for _ in range(3))
-        self.ws = torch.empty(max(1, fa.fa_bwd_workspace_bytes_ex(B, H, N, d,
-                                                                  fa.options(fused=fused))),
-                              dtype=torch.uint8, device=dev)
         self.slopes = None
         if w.alibi:
             self.slopes = torch.tensor(workloads.alibi_slopes(H), dtype=torch.float32,
@@ -258,6 +255,9 @@ class Problem:
             self.lengths = torch.tensor(w.seq_lengths(), dtype=torch.int32, device=dev)
         self.opt = fa.options(alibi_slopes=self.slopes, o_low=None if plain else self.o_low,
                               fused=fused, seq_lengths=self.lengths)
+        # the workspace holds the row statistics (and with real lengths, the schedule)
+        self.ws = torch.empty(max(1, fa.fa_bwd_workspace_bytes_ex(B, H, N, d, self.opt)),
+                              dtype=torch.uint8, device=dev)
         self.names = kernel_names(w, fused)
         self.fused = "bwd_fused" in self.names
         self.launches = len(self.names)

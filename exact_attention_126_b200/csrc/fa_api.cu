@@ -118,12 +118,35 @@ size_t dq_acc_bytes(int B, int H, int N, int d) {
   return (size_t)B * H * padded_rows(N) * (size_t)d * sizeof(float);
 }
 
+// A variable-length batch (up to kVarlenSchedMaxB entries) adds, last, the tables of its
+// schedule (varlen_item), which the preprocess step writes.
+size_t sched_bytes(int B, int N, const Extras& x) {
+  if (x.seq_len == nullptr || B > fa::kVarlenSchedMaxB) return 0;
+  const size_t raw = 4 * (size_t)fa::varlen_sched_ints(B, fa::num_tiles(N));
+  return (raw + 255) & ~size_t(255);
+}
+
 size_t workspace_bytes(int B, int H, int N, int d, const Extras& x) {
-  return stats_bytes(B, H, N) + (uses_fused(d, x) ? dq_acc_bytes(B, H, N, d) : 0);
+  return stats_bytes(B, H, N) + (uses_fused(d, x) ? dq_acc_bytes(B, H, N, d) : 0) +
+         sched_bytes(B, N, x);
 }
 
 float* dq_acc_of(void* workspace, int B, int H, int N) {
   return reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + stats_bytes(B, H, N));
+}
+
+// The schedule tables in `workspace`, or null without them.
+int* sched_of(const void* workspace, int B, int H, int N, int d, const Extras& x) {
+  if (sched_bytes(B, N, x) == 0) return nullptr;
+  const size_t off = stats_bytes(B, H, N) + (uses_fused(d, x) ? dq_acc_bytes(B, H, N, d) : 0);
+  return reinterpret_cast<int*>(static_cast<uint8_t*>(const_cast<void*>(workspace)) + off);
+}
+
+// x with the schedule tables of `workspace` (a variable-length batch).
+Extras with_sched(const Extras& x, const void* workspace, int B, int H, int N, int d) {
+  Extras xs = x;
+  xs.sched = sched_of(workspace, B, H, N, d, x);
+  return xs;
 }
 
 // Checks the optional arguments of an _ex call and resolves them; a null `opt` means none.
@@ -204,9 +227,13 @@ fa_status_t preprocess(const void* o, const void* dout, const float* lse, void* 
   float* stats = static_cast<float*>(workspace);
   // the fused pass accumulates dQ: its accumulator starts at zero
   float* acc = uses_fused(d, x) ? dq_acc_of(workspace, B, H, N) : nullptr;
-  return d == 64 ? fa_host::launch_preprocess<64>(o, x.o_low, dout, lse, stats, acc, B * H, N, st)
-                 : fa_host::launch_preprocess<128>(o, x.o_low, dout, lse, stats, acc, B * H, N,
-                                                   st);
+  // and with real lengths, the tables of the passes' schedule
+  const fa::SchedBuild sb{x.seq_len, sched_of(workspace, B, H, N, d, x), B, H, N,
+                          fa::num_tiles(N)};
+  return d == 64
+             ? fa_host::launch_preprocess<64>(o, x.o_low, dout, lse, stats, acc, sb, B * H, N, st)
+             : fa_host::launch_preprocess<128>(o, x.o_low, dout, lse, stats, acc, sb, B * H, N,
+                                               st);
 }
 
 // The fused pass (head_dim 64): dK, dV, and dQ added into the workspace's accumulator.
@@ -224,8 +251,9 @@ fa_status_t fused_pass(const void* q, const void* k, const void* v, const void* 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Problem pb{B * H, H, N, scale, window.left, right};
   const int feat = x.features() & ~fa::kFeatResidual;
+  const Extras xs = with_sched(x, workspace, B, H, N, d);
   s = dispatch_features<FusedLaunch>(BwdFeatures(), feat, q, k, v, dout, workspace,
-                                     dq_acc_of(workspace, B, H, N), dk, dv, pb, x, st);
+                                     dq_acc_of(workspace, B, H, N), dk, dv, pb, xs, st);
   // rows of dQ past the real length stay zero in the accumulator
   if (s != FA_OK || x.seq_len == nullptr) return s;
   return fill(dk, dv, nullptr, nullptr, d, B * H, H, N, x, st);
@@ -259,10 +287,11 @@ fa_status_t dkdv_pass(const void* q, const void* k, const void* v, const void* d
   const int l = window.left, BH = B * H;
   const int feat = x.features() & ~fa::kFeatResidual;
   const Problem pb{BH, H, N, scale, l, right};
+  const Extras xs = with_sched(x, workspace, B, H, N, d);
   s = d == 64 ? dispatch_features<DkdvLaunch<64>>(BwdFeatures(), feat, q, k, v, dout, workspace,
-                                                  dk, dv, pb, x, st)
+                                                  dk, dv, pb, xs, st)
               : dispatch_features<DkdvLaunch<128>>(BwdFeatures(), feat, q, k, v, dout, workspace,
-                                                   dk, dv, pb, x, st);
+                                                   dk, dv, pb, xs, st);
   if (s != FA_OK || x.seq_len == nullptr) return s;
   return fill(dk, dv, nullptr, nullptr, d, BH, H, N, x, st);
 }
@@ -281,10 +310,11 @@ fa_status_t dq_pass(const void* q, const void* k, const void* v, const void* dou
   const int l = window.left, BH = B * H;
   const int feat = x.features() & ~fa::kFeatResidual;
   const Problem pb{BH, H, N, scale, l, right};
+  const Extras xs = with_sched(x, workspace, B, H, N, d);
   s = d == 64 ? dispatch_features<DqLaunch<64>>(BwdFeatures(), feat, q, k, v, dout, workspace,
-                                                dq, pb, x, st)
+                                                dq, pb, xs, st)
               : dispatch_features<DqLaunch<128>>(BwdFeatures(), feat, q, k, v, dout, workspace,
-                                                 dq, pb, x, st);
+                                                 dq, pb, xs, st);
   if (s != FA_OK || x.seq_len == nullptr) return s;
   return fill(dq, nullptr, nullptr, nullptr, d, BH, H, N, x, st);
 }

@@ -59,12 +59,16 @@ __global__ void __launch_bounds__(256)
     fa_bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o,
                              const __nv_bfloat16* __restrict__ o_low,
                              const __nv_bfloat16* __restrict__ dout, const float* __restrict__ lse,
-                             float* __restrict__ stats, float* __restrict__ dq_acc, int BH, int N,
-                             int Np) {
+                             float* __restrict__ stats, float* __restrict__ dq_acc, SchedBuild sb,
+                             int BH, int N, int Np) {
   constexpr int G = D / 8;                      // lanes per row
   constexpr int kRowsPerPass = 32 / G;          // rows a warp covers per load
   constexpr int kPasses = 8 / kRowsPerPass;     // 8 rows per warp
   const int blocks_per_head = Np / 64;
+  if ((int)blockIdx.x >= BH * blocks_per_head) {
+    if (threadIdx.x < 32) build_varlen_sched(sb.seq_len, sb.B, sb.H, sb.N, 1, sb.U, sb.tables);
+    return;
+  }
   const int bh = blockIdx.x / blocks_per_head;
   const int xb = blockIdx.x - bh * blocks_per_head;
   const int lane = threadIdx.x & 31;
@@ -168,6 +172,8 @@ struct BwdArgs {
   const uint8_t* kpad;  // (B, N) key-padding flags (nonzero = padded key), or null
   DropoutArgs drop;     // kFeatDropout kernels
   const int* seq_len;   // variable-length batch: B real lengths, or null
+  int sorted;           // variable-length batch: the schedule of varlen_item, with ...
+  const int* sched;     // ... its tables, written by fa_bwd_preprocess_kernel
 };
 
 // Shared layout of both backward kernels: the stationary tiles X0, X1 of an item (in XB
@@ -312,6 +318,14 @@ __device__ __forceinline__ bool bwd_item(int k, const BwdArgs& a, bool rising, i
                                          int& tile, Mask& mk) {
   if (a.paired) {
     if (!paired_item(k, (int)gridDim.x, a.n_double, a.n_tiles, rising, bh, tile)) return false;
+  } else if (a.sorted) {
+    int u;
+    if (!varlen_item(k, (int)gridDim.x, a.sched, a.n_tiles, a.H, bh, u)) return false;
+    const int n = real_length(a.seq_len, bh, a.H, a.N);
+    mk = Mask{n, a.left, a.right};
+    // key tiles count from the end of the sequence, query tiles from its start
+    tile = rising ? num_tiles(n) - 1 - u : u;
+    return true;
   } else if (a.longest_first) {
     chunked_item(k, a.BH, a.n_tiles, a.group, rising, bh, tile);
   } else {

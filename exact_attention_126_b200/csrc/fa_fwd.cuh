@@ -63,6 +63,8 @@ struct FwdArgs {
   __nv_bfloat16* o_low;      // (B, H, N, d) bf16 residual O - bf16(O), or null
   DropoutArgs drop;          // kFeatDropout kernels
   const int* seq_len;        // variable-length batch: B real lengths, or null
+  int sorted;                // variable-length batch: the schedule of varlen_item, whose
+                             // tables each CTA builds in shared memory after kMisc
   float o_scale;             // kFeatFp8: the V descale, applied to O in the epilogue
 };
 
@@ -142,22 +144,29 @@ struct FwdItem {
   int last;
 };
 
-__device__ __forceinline__ FwdItem fwd_item(int k, const FwdArgs& a) {
+__device__ __forceinline__ FwdItem no_fwd_item() {
+  FwdItem it;
+  it.bh = 0;
+  it.n = 0;
+  it.m[0] = it.m[1] = 0;
+  it.has_a = it.has_b = false;
+  it.lo[0] = it.lo[1] = 1;
+  it.hi[0] = it.hi[1] = 0;
+  it.first = 1;
+  it.last = 0;
+  return it;
+}
+
+// `sched`: the varlen_item tables (shared memory) when a.sorted.
+__device__ __forceinline__ FwdItem fwd_item(int k, const FwdArgs& a, const int* sched) {
   FwdItem it;
   int pair;
   if (a.paired) {
-    if (!paired_item(k, (int)gridDim.x, a.n_double, a.n_pairs, false, it.bh, pair)) {
-      // a slot past the last pair: no work
-      it.bh = 0;
-      it.n = 0;
-      it.m[0] = it.m[1] = 0;
-      it.has_a = it.has_b = false;
-      it.lo[0] = it.lo[1] = 1;
-      it.hi[0] = it.hi[1] = 0;
-      it.first = 1;
-      it.last = 0;
-      return it;
-    }
+    // a slot past the last pair: no work
+    if (!paired_item(k, (int)gridDim.x, a.n_double, a.n_pairs, false, it.bh, pair))
+      return no_fwd_item();
+  } else if (a.sorted) {
+    if (!varlen_item(k, (int)gridDim.x, sched, a.n_pairs, a.H, it.bh, pair)) return no_fwd_item();
   } else if (a.longest_first) {
     chunked_item(k, a.BH, a.n_pairs, a.group, false, it.bh, pair);
   } else {
@@ -267,6 +276,9 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
     tmem_relinquish();
   }
+  int* sched = reinterpret_cast<int*>(smem + C::kMisc + 16);
+  if (a.sorted && warp == 1) build_varlen_sched(a.seq_len, a.BH / a.H, a.H, a.N, a.per_item,
+                                                a.n_pairs, sched);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -282,7 +294,7 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
       int kc = 0, vc = 0;  // K and V loads issued (ring positions)
       bool ok = true;
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
-        const FwdItem it = fwd_item(k, a);
+        const FwdItem it = fwd_item(k, a, sched);
         if (!it.has_a) continue;  // past the real length: nothing to load
         for (int s = 0; s < 2; ++s) {
           if (s == 1 && !it.has_b) break;
@@ -524,7 +536,7 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
       };
 
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
-        const FwdItem it = fwd_item(k, a);
+        const FwdItem it = fwd_item(k, a, sched);
         if (!it.has_a) continue;  // past the real length: no products
         const FwdRange rg = fwd_range(it, s);
         const int n = it.last - it.first + 1;
@@ -570,7 +582,7 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
 
 
     for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
-      const FwdItem it = fwd_item(k, a);
+      const FwdItem it = fwd_item(k, a, sched);
       const FwdRange rg = fwd_range(it, s);
       if (!rg.has) continue;
       const Mask mk{it.n, a.left, a.right};

@@ -23,6 +23,7 @@ struct Extras {
   bool fused = false;              // backward: the fused pass (head_dim 64) instead of the
                                    // dK/dV and dQ passes
   const int* seq_len = nullptr;    // variable-length batch: B real lengths
+  const int* sched = nullptr;      // ... and the backward's schedule tables in its workspace
   bool fp8 = false;                // forward on e4m3 Q, K, V (the kFeatFp8 kernel)
   float o_scale = 1.f;             // with fp8: the V descale, applied to O
   fa::DropoutArgs drop = {0, 0, 0, 0, 1.f};
@@ -52,8 +53,8 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
 
 template <int D>
 fa_status_t launch_preprocess(const void* o, const void* o_low, const void* dout,
-                              const float* lse, float* stats, float* dq_acc, int BH, int N,
-                              cudaStream_t st);
+                              const float* lse, float* stats, float* dq_acc,
+                              const fa::SchedBuild& sb, int BH, int N, cudaStream_t st);
 
 // The fused backward pass (head_dim 64): dK, dV, and dQ added into `dq_acc`.
 template <int kFeat>

@@ -77,6 +77,8 @@ inline bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+constexpr int kMaxSmemPerBlock = 232448;  // the opt-in limit of sm_100
+
 template <typename Kernel>
 fa_status_t set_smem(Kernel k, int bytes) {
   // Per device and kernel; cheap enough to repeat, but only needed once per device.
@@ -119,6 +121,16 @@ inline void pair_schedule(Args& a, int BH, int T, int left, int right, bool varl
   }
 }
 
+// The schedule of a variable-length batch (varlen_item) over U units per head: the slots of
+// whole rounds of the persistent grid, so that both directions of the last round are
+// visited. Sets sorted and n_items.
+template <typename Args>
+inline void varlen_schedule(Args& a, int BH, int U) {
+  a.sorted = 1;
+  const int P = BH * U < sm_count() ? BH * U : sm_count();
+  a.n_items = (BH * U + P - 1) / P * P;
+}
+
 // Persistent CTAs: one per SM, or one per item (one per pair of items with the causal
 // schedule) when there are fewer.
 template <typename Args>
@@ -148,7 +160,6 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     return FA_ERR_CUDA;
   }
   using C = fa::FwdCfg<D, kFp8>;
-  if (set_smem(fa::fa_fwd_kernel<D, kFeat>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
   fa::FwdArgs a;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
@@ -162,6 +173,16 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
   a.group = head_group(BH, a.n_pairs);
   pair_schedule(a, BH, a.n_pairs, left, right, x.seq_len != nullptr);
+  // a variable-length batch: the varlen_item schedule, its tables in shared memory
+  a.sorted = 0;
+  int smem = C::kSmemBytes;
+  const int sched_bytes = 4 * fa::varlen_sched_ints(BH / H, a.n_pairs);
+  if (x.seq_len != nullptr && BH / H <= fa::kVarlenSchedMaxB &&
+      C::kSmemBytes + sched_bytes <= kMaxSmemPerBlock) {
+    varlen_schedule(a, BH, a.n_pairs);
+    smem += sched_bytes;
+  }
+  if (set_smem(fa::fa_fwd_kernel<D, kFeat>, smem) != FA_OK) return FA_ERR_CUDA;
   a.scale_log2 = scale * fa::kLog2e;
   a.left = left;
   a.right = right;
@@ -174,7 +195,7 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   a.seq_len = x.seq_len;
   a.o_scale = x.o_scale;
   const int grid = persistent_grid(a);
-  fa::fa_fwd_kernel<D, kFeat><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mkk, mv, a);
+  fa::fa_fwd_kernel<D, kFeat><<<grid, C::kThreads, smem, st>>>(mq, mkk, mv, a);
   return launched();
 }
 
@@ -182,15 +203,15 @@ inline int padded_rows(int N) { return fa::num_tiles(N) * kBlock; }
 
 template <int D>
 fa_status_t launch_preprocess(const void* o, const void* o_low, const void* dout,
-                              const float* lse, float* stats, float* dq_acc, int BH, int N,
-                              cudaStream_t st) {
+                              const float* lse, float* stats, float* dq_acc,
+                              const fa::SchedBuild& sb, int BH, int N, cudaStream_t st) {
   const int Np = padded_rows(N);
   // 64 rows per block, blocks of one head consecutive; BH * Np / 64 < 2^31 because every
-  // tensor has fewer than 2^31 elements (d >= 64)
-  const long long blocks = (long long)BH * (Np / 64);
+  // tensor has fewer than 2^31 elements (d >= 64); one more block builds the tables of sb
+  const long long blocks = (long long)BH * (Np / 64) + (sb.tables != nullptr ? 1 : 0);
   fa::fa_bwd_preprocess_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(o_low),
-      static_cast<const __nv_bfloat16*>(dout), lse, stats, dq_acc, BH, N, Np);
+      static_cast<const __nv_bfloat16*>(dout), lse, stats, dq_acc, sb, BH, N, Np);
   return launched();
 }
 
@@ -215,6 +236,9 @@ inline fa::BwdArgs bwd_args(const void* ws, const Problem& pb, const Extras& x) 
   a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
   a.group = head_group(BH, a.n_tiles);
   pair_schedule(a, BH, a.n_tiles, left, right, x.seq_len != nullptr);
+  a.sorted = 0;
+  a.sched = x.sched;
+  if (x.sched != nullptr) varlen_schedule(a, BH, a.n_tiles);
   a.alibi = x.alibi;
   a.H = H;
   a.kpad = x.kpad;

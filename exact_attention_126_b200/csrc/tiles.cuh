@@ -146,4 +146,134 @@ __host__ __device__ inline bool paired_item(int k, int P, int n_double, int T, b
   return true;
 }
 
+// ---- The schedule of a variable-length batch ----
+// With real lengths L_b the work of an item is set by the distance u of its tile from the
+// start of the sequence (query tiles: a causal query tile i sees i + 1 key tiles) or from
+// its end (key tiles: causal key tile j is seen by T_b - j query tiles, T_b the tiles of
+// L_b); u counts units, a unit being a tile or, in the forward, the per_item query tiles
+// of an item. Items go in order of u, largest first. Bucket u holds the H heads of every
+// batch entry with more than u units, and those entries are the first M_u of the batch
+// entries ordered by units, most first (ties by index), so that an item's position is
+// resolved by one search over the buckets. Slot k of a grid of P persistent CTAs takes
+// position p of that order, the rounds of P positions alternating in direction (CTA c
+// takes positions c, 2P - 1 - c, 2P + c, ...), which evens out what the CTAs add up along
+// a decreasing sequence. Entries past a sequence's last unit are never scheduled.
+//
+// Tables, in ints: start[0 .. U] (start[q] = position of the first item of bucket
+// u = U - 1 - q; start[U] = the number of items), sigma[0 .. B) (the ordered batch
+// entries), then U + 1 ints of scratch for building them.
+__host__ __device__ inline int varlen_sched_ints(int B, int U) { return 2 * (U + 1) + B; }
+
+// What the backward's preprocess kernel needs to build the tables of the schedule above
+// (one unit per tile) in one block past its row blocks; `tables` null = none.
+struct SchedBuild {
+  const int* seq_len;
+  int* tables;
+  int B;
+  int H;
+  int N;
+  int U;  // tiles per head
+};
+
+// Largest batch for which the schedule above is built (the build is one warp's pass over
+// the batch); larger batches keep the chunked schedule.
+constexpr int kVarlenSchedMaxB = 8192;
+
+#ifdef __CUDACC__
+__device__ __forceinline__ int varlen_units(const int* seq_len, int b, int N, int per_item) {
+  int L = seq_len[b];
+  L = L < 0 ? 0 : (L > N ? N : L);
+  return (num_tiles(L) + per_item - 1) / per_item;
+}
+
+// Builds the tables of the schedule above; called by all 32 lanes of one warp.
+__device__ __forceinline__ void build_varlen_sched(const int* seq_len, int B, int H, int N,
+                                                   int per_item, int U, int* tables) {
+  int* start = tables;
+  int* sigma = tables + U + 1;
+  int* cnt = sigma + B;  // cnt[v], v in [0, U]: entries with v units, then a running count
+  const int lane = threadIdx.x & 31;
+  for (int v = lane; v <= U; v += 32) cnt[v] = 0;
+  __syncwarp();
+  // counted without atomics (the tables may be in global memory): the lowest lane of each
+  // group of lanes with equal units adds the group's size
+  for (int b0 = 0; b0 < B; b0 += 32) {
+    const int b = b0 + lane;
+    const int u = b < B ? varlen_units(seq_len, b, N, per_item) : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, u);
+    if (b < B && (peers & ((1u << lane) - 1u)) == 0) cnt[u] += __popc(peers);
+    __syncwarp();
+  }
+  // M(q) = entries with more than u = U - 1 - q units = sum of cnt[v] over v >= U - q;
+  // bucket q has H M(q) items: start is the exclusive prefix sum of H M
+  int carry_m = 0, carry_s = 0;
+  if (lane == 0) start[0] = 0;
+  for (int q0 = 0; q0 < U; q0 += 32) {
+    const int q = q0 + lane;
+    int m = q < U ? cnt[U - q] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, m, off);
+      if (lane >= off) m += t;
+    }
+    m += carry_m;
+    int s = q < U ? H * m : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, s, off);
+      if (lane >= off) s += t;
+    }
+    s += carry_s;
+    if (q < U) start[q + 1] = s;
+    carry_m = __shfl_sync(0xffffffffu, m, 31);
+    carry_s = __shfl_sync(0xffffffffu, s, 31);
+  }
+  __syncwarp();
+  for (int v = lane; v <= U; v += 32) cnt[v] = 0;
+  __syncwarp();
+  // rank of entry b = (entries with more units) + (earlier entries with as many units)
+  for (int b0 = 0; b0 < B; b0 += 32) {
+    const int b = b0 + lane;
+    const int u = b < B ? varlen_units(seq_len, b, N, per_item) : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, u);
+    const int before = __popc(peers & ((1u << lane) - 1u));
+    const int seen = b < B ? cnt[u] : 0;
+    __syncwarp();
+    if (b < B) {
+      const int more = u >= U ? 0 : (start[U - u] - start[U - 1 - u]) / H;
+      sigma[more + seen + before] = b;
+      if (before == 0) cnt[u] = seen + __popc(peers);
+    }
+    __syncwarp();
+  }
+}
+
+#endif
+
+// Slot k of the schedule above over a grid of P CTAs: the item's (batch*head) and its unit
+// distance u, or false past the last item.
+__host__ __device__ inline bool varlen_item(int k, int P, const int* tables, int U, int H,
+                                            int& bh, int& u) {
+  const int* start = tables;
+  const int* sigma = tables + U + 1;
+  const int r = k / P;
+  const int c = k - r * P;
+  const int p = r * P + ((r & 1) ? P - 1 - c : c);
+  if (p >= start[U]) return false;
+  int lo = 0, hi = U - 1;  // the last bucket q with start[q] <= p (it is not empty)
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (start[mid] <= p) {
+      lo = mid;
+    } else {
+      hi = mid - 1;
+    }
+  }
+  const int idx = p - start[lo];
+  const int e = idx / H;
+  u = U - 1 - lo;
+  bh = sigma[e] * H + (idx - e * H);
+  return true;
+}
+
 }  // namespace fa

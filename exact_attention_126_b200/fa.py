@@ -406,7 +406,8 @@ def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, window=(-1
     dq = torch.empty_like(q)
     dk = torch.empty_like(q)
     dv = torch.empty_like(q)
-    ws = torch.empty(max(1, fa_bwd_workspace_bytes_ex(B, H, N, d, options(fused=fused))),
+    ws = torch.empty(max(1, fa_bwd_workspace_bytes_ex(
+        B, H, N, d, options(fused=fused, seq_lengths=seq_lengths))),
                      dtype=torch.uint8, device=q.device)
     if alibi_slopes is not None:
         _check_slopes(alibi_slopes, q)

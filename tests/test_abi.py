@@ -156,6 +156,16 @@ def test_options_are_checked(lib):
     assert lib.fa_bwd_workspace_bytes_ex(1, 2, 128, 64, None) == stats
     assert lib.fa_bwd_workspace_bytes_ex(1, 2, 128, 128, ctypes.byref(O(flags=1))) == stats
     assert lib.fa_bwd_workspace_bytes_ex(1, 2, 128, 64, ctypes.byref(O(flags=4))) == 0
+    # a variable-length batch adds, last, the tables of its schedule: start (T + 1 ints),
+    # the batch entries by length (B ints) and T + 1 ints of scratch, rounded to 256 bytes
+    def sched(B, T):
+        return (4 * (2 * (T + 1) + B) + 255) // 256 * 256
+    for B, H, N, d, flags in ((1, 2, 128, 64, 0), (3, 2, 1000, 128, 0), (70, 1, 4096, 64, 1)):
+        base = lib.fa_bwd_workspace_bytes_ex(B, H, N, d, ctypes.byref(O(flags=flags)))
+        got = lib.fa_bwd_workspace_bytes_ex(B, H, N, d,
+                                            ctypes.byref(O(flags=flags, seq_lengths=A)))
+        assert got == base + sched(B, (N + 127) // 128)
+    assert bwd_ex(O(seq_lengths=A), ws_bytes=stats) == 4
     assert lib.fa_bwd_fused(A, A, A, A, A, A, A, 1, 1, 128, 128, 0.1, 0, W(-1, -1), None,
                             None) == 2   # the fused pass is for head_dim 64
     assert lib.fa_bwd_dq_convert(A, None, 1, 1, 128, 64, 0.1, None) == 1

@@ -6,6 +6,7 @@
 // mismatch and exits non-zero.
 #define __host__
 #define __device__
+#include <algorithm>
 #include <cstdio>
 #include <vector>
 #include "tiles.cuh"
@@ -112,6 +113,50 @@ int main() {
           for (int v : seen)
             if (v != 1) return fail("paired_item cover", BH, T, Pg, rising);
         }
+  // varlen_item: with the tables built here by a plain sort (the kernels build them with a
+  // warp; the GPU parity tests cover that), the slots of whole rounds of P CTAs visit every
+  // (head, unit) of every sequence exactly once, units in decreasing order of position.
+  const int lens_sets[4][6] = {{0, 1, 128, 129, 640, 300},
+                               {640, 640, 640, 640, 640, 640},
+                               {5, 0, 0, 700, 256, 1},
+                               {0, 0, 0, 0, 0, 0}};
+  for (auto& lens : lens_sets)
+    for (int B = 1; B <= 6; ++B)
+      for (int H = 1; H <= 3; ++H)
+        for (int per_item = 1; per_item <= 2; ++per_item)
+          for (int P = 1; P <= 11; ++P) {
+            const int N = 700, U = (num_tiles(N) + per_item - 1) / per_item;
+            std::vector<int> units(B), sigma(B), start(U + 1, 0);
+            for (int b = 0; b < B; ++b)
+              units[b] = (num_tiles(lens[b] < N ? lens[b] : N) + per_item - 1) / per_item;
+            for (int b = 0; b < B; ++b) sigma[b] = b;
+            std::stable_sort(sigma.begin(), sigma.end(),
+                             [&](int x, int y) { return units[x] > units[y]; });
+            for (int q = 0; q < U; ++q) {
+              int m = 0;
+              for (int b = 0; b < B; ++b) m += units[b] > U - 1 - q;
+              start[q + 1] = start[q] + H * m;
+            }
+            std::vector<int> tables(start);
+            tables.insert(tables.end(), sigma.begin(), sigma.end());
+            const int slots = (B * H * U + P - 1) / P * P;
+            std::vector<int> seen(B * H * U, 0), by_pos(slots, -1);
+            for (int k = 0; k < slots; ++k) {
+              int bh, u;
+              if (!varlen_item(k, P, tables.data(), U, H, bh, u)) continue;
+              if (bh < 0 || bh >= B * H || u < 0 || u >= units[bh / H])
+                return fail("varlen_item range", B, H, P, k);
+              ++seen[bh * U + u];
+              const int r = k / P, c = k % P;
+              by_pos[r * P + ((r & 1) ? P - 1 - c : c)] = u;
+            }
+            for (int bh = 0; bh < B * H; ++bh)
+              for (int u = 0; u < U; ++u)
+                if (seen[bh * U + u] != (u < units[bh / H] ? 1 : 0))
+                  return fail("varlen_item cover", B, H, P, bh * U + u);
+            for (int p = 1; p < slots; ++p)
+              if (by_pos[p] > by_pos[p - 1]) return fail("varlen_item order", B, H, P, p);
+          }
   std::printf("OK\n");
   return 0;
 }
