@@ -127,26 +127,34 @@ __global__ void __launch_bounds__(256)
 // Variable-length batches: rows r >= L_b (the real length of the row's batch entry) of up to
 // three bf16 (B*H, N, D) tensors become zero and, with `lse`, their LSE becomes -inf. The
 // attention kernels skip every tile that lies wholly past the real length; this fills what
-// they leave. 8 values (16 bytes) per thread; threads of rows below L_b do nothing.
+// they leave. Block b covers rows 128x .. 128x+127 of head bh, (bh, x) = divmod(b, tiles):
+// a block whose rows are all below L_b returns at once, the others write 16 bytes per
+// thread and step, the 256 threads of a step covering 256 / (D / 8) consecutive rows.
 // ------------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256)
     fa_fill_past_length_kernel(__nv_bfloat16* __restrict__ t0, __nv_bfloat16* __restrict__ t1,
                                __nv_bfloat16* __restrict__ t2, float* __restrict__ lse,
-                               const int* __restrict__ seq_len, long long rows, int N, int H) {
+                               const int* __restrict__ seq_len, int N, int H) {
   constexpr int kPerRow = D / 8;
-  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long long row = idx / kPerRow;  // over the B*H*N rows
-  if (row >= rows) return;
-  const int part = (int)(idx - row * kPerRow);
-  const long long bh = row / N;
-  const int r = (int)(row - bh * N);
-  if (r < real_length(seq_len, (int)bh, H, N)) return;
-  const size_t off = (size_t)row * D + part * 8;
-  if (t0 != nullptr) st_global_v4(t0 + off, 0u, 0u, 0u, 0u);
-  if (t1 != nullptr) st_global_v4(t1 + off, 0u, 0u, 0u, 0u);
-  if (t2 != nullptr) st_global_v4(t2 + off, 0u, 0u, 0u, 0u);
-  if (lse != nullptr && part == 0) lse[row] = -INFINITY;
+  const int tiles = num_tiles(N);
+  const int bh = blockIdx.x / tiles;
+  const int r0 = (blockIdx.x - bh * tiles) * kBlock;
+  const int L = real_length(seq_len, bh, H, N);
+  const int r_end = r0 + kBlock < N ? r0 + kBlock : N;
+  const int r_begin = r0 > L ? r0 : L;
+  if (r_begin >= r_end) return;
+  const size_t base = (size_t)bh * N;
+  for (int e = r_begin * kPerRow - r0 * kPerRow + threadIdx.x;
+       e < (r_end - r0) * kPerRow; e += blockDim.x) {
+    const int r = r0 + e / kPerRow;
+    const int part = e % kPerRow;
+    const size_t off = (base + r) * D + part * 8;
+    if (t0 != nullptr) st_global_v4(t0 + off, 0u, 0u, 0u, 0u);
+    if (t1 != nullptr) st_global_v4(t1 + off, 0u, 0u, 0u, 0u);
+    if (t2 != nullptr) st_global_v4(t2 + off, 0u, 0u, 0u, 0u);
+    if (lse != nullptr && part == 0) lse[base + r] = -INFINITY;
+  }
 }
 
 struct BwdArgs {

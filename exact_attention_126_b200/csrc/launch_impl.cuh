@@ -325,11 +325,11 @@ fa_status_t launch_dq_convert(const float* dq_acc, void* dq, int BH, int N, floa
 template <int D>
 fa_status_t launch_fill_past_length(void* t0, void* t1, void* t2, float* lse,
                                     const int* seq_len, int BH, int H, int N, cudaStream_t st) {
-  const long long rows = (long long)BH * N;
-  const long long blocks = (rows * (D / 8) + 255) / 256;
+  // one block per 128-row tile: BH * tiles < 2^31 (every tensor has < 2^31 elements)
+  const long long blocks = (long long)BH * fa::num_tiles(N);
   fa::fa_fill_past_length_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
       static_cast<__nv_bfloat16*>(t0), static_cast<__nv_bfloat16*>(t1),
-      static_cast<__nv_bfloat16*>(t2), lse, seq_len, rows, N, H);
+      static_cast<__nv_bfloat16*>(t2), lse, seq_len, N, H);
   return launched();
 }
 

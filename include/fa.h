@@ -192,7 +192,11 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 
 /*
  * The same for fa_bwd_ex with `options` (may be NULL): with FA_BWD_FUSED at head_dim 64 the
- * row statistics are followed by the fused pass's fp32 dQ accumulator of B*H*Np*64 values.
+ * row statistics are followed by the fused pass's fp32 dQ accumulator of B*H*Np*64 values;
+ * with seq_lengths (and B <= 8192) the last part holds the tables of the variable-length
+ * work schedule, 2*(Np/128 + 1) + B ints rounded up to 256 bytes, which fa_bwd_preprocess
+ * writes and the passes read (items ordered by their tile's distance from the start or end
+ * of its sequence, so that the persistent CTAs get even shares of uneven sequences).
  * Returns 0 for an empty problem, invalid sizes or invalid options.
  */
 size_t fa_bwd_workspace_bytes_ex(int B, int H, int N, int d, const fa_options_t *options);
@@ -251,30 +255,35 @@ fa_status_t fa_bwd_alibi(const void *q, const void *k, const void *v, const void
                          size_t workspace_bytes, void *stream);
 
 /*
- * Step 1 of fa_bwd alone: fills `workspace` (at least fa_bwd_workspace_bytes()) with
+ * Step 1 of fa_bwd alone: fills `workspace` (at least fa_bwd_workspace_bytes(), or
+ * fa_bwd_workspace_bytes_ex() with the same options when they carry FA_BWD_FUSED or
+ * seq_lengths: the workspace is not bounds-checked here) with
  * the per-row statistics the two passes read, each as B*H rows of Np = N rounded up to
  * 128 fp32 values (padding rows: +inf and 0):
  *   workspace[0 .. B*H*Np)          LSE * log2(e)      (from `lse`)
  *   workspace[B*H*Np .. 2*B*H*Np)   delta = rowsum(dout * o), summed in fp32
  *                                   (o + options->o_low when o_low is given)
  * The padding lets each 128-row tile of both arrays be fetched with one bulk copy.
- * With FA_BWD_FUSED at head_dim 64 it also zeroes the fused pass's dQ accumulator (the
- * workspace must then hold fa_bwd_workspace_bytes_ex() bytes).
- * `options` may be NULL; its o_low and flags are used here.
+ * With FA_BWD_FUSED at head_dim 64 it also zeroes the fused pass's dQ accumulator, and
+ * with seq_lengths it writes the tables of the variable-length schedule (both after the
+ * statistics, as fa_bwd_workspace_bytes_ex() lays them out).
+ * `options` may be NULL; its o_low, flags and seq_lengths are used here.
  */
 fa_status_t fa_bwd_preprocess(const void *o, const void *dout, const float *lse,
                               void *workspace, int B, int H, int N, int d,
                               const fa_options_t *options, void *stream);
 
 /* Step 2 of fa_bwd alone: dk, dv from q, k, v, dout and the workspace of step 1
- * (`options`: alibi_slopes, key_padding and dropout, or NULL). */
+ * (`options`: alibi_slopes, key_padding, dropout and seq_lengths as given to step 1, or
+ * NULL). */
 fa_status_t fa_bwd_dkdv(const void *q, const void *k, const void *v, const void *dout,
                         const void *workspace, void *dk, void *dv,
                         int B, int H, int N, int d, float scale, int causal,
                         fa_window_t window, const fa_options_t *options, void *stream);
 
 /* Step 3 of fa_bwd alone: dq from q, k, v, dout and the workspace of step 1
- * (`options`: alibi_slopes, key_padding and dropout, or NULL). */
+ * (`options`: alibi_slopes, key_padding, dropout and seq_lengths as given to step 1, or
+ * NULL). */
 fa_status_t fa_bwd_dq(const void *q, const void *k, const void *v, const void *dout,
                       const void *workspace, void *dq,
                       int B, int H, int N, int d, float scale, int causal,
