@@ -895,8 +895,16 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
         for (int e = 0; e < NC / 2; e += 2) {
           const int r0 = 2 * e;
           const float4 d4 = *reinterpret_cast<const float4*>(del_s + r0);
-          w[e] = pack_bf16x2(p[r0] * (dp[r0] - d4.x), p[r0 + 1] * (dp[r0 + 1] - d4.y));
-          w[e + 1] = pack_bf16x2(p[r0 + 2] * (dp[r0 + 2] - d4.z), p[r0 + 3] * (dp[r0 + 3] - d4.w));
+          // two columns per instruction (packed fp32 add and multiply of sm_100): the same
+          // roundings as the scalar form, half the issue slots
+          const float2 v0 = __fmul2_rn(make_float2(p[r0], p[r0 + 1]),
+                                       __fadd2_rn(make_float2(dp[r0], dp[r0 + 1]),
+                                                  make_float2(-d4.x, -d4.y)));
+          const float2 v1 = __fmul2_rn(make_float2(p[r0 + 2], p[r0 + 3]),
+                                       __fadd2_rn(make_float2(dp[r0 + 2], dp[r0 + 3]),
+                                                  make_float2(-d4.z, -d4.w)));
+          w[e] = pack_bf16x2(v0.x, v0.y);
+          w[e + 1] = pack_bf16x2(v1.x, v1.y);
         }
         // bf16 dS^T goes over the second half of this warpgroup's own fp32 S^T columns
         // (kDsInS) or the first half of its dP^T columns
@@ -1233,10 +1241,21 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
         {
           // with ALiBi, -m |key - query| in log2 units joins the exponent
           const float base = (float)((long long)jj * kBlock + NC * h - r);
+          if constexpr (kAlibi) {
 #pragma unroll
-          for (int c = 0; c < NC; ++c) {
-            const float arg = kAlibi ? -slope2 * fabsf(base + (float)c) - lse2 : -lse2;
-            p[c] = ex2(fmaf(p[c], sl2, arg));
+            for (int c = 0; c < NC; ++c) {
+              const float arg = -slope2 * fabsf(base + (float)c) - lse2;
+              p[c] = ex2(fmaf(p[c], sl2, arg));
+            }
+          } else {
+            // exponent arguments two at a time (packed fp32 FMA), rounded as fmaf rounds
+            const float2 s2 = make_float2(sl2, sl2), a2 = make_float2(-lse2, -lse2);
+#pragma unroll
+            for (int c = 0; c < NC; c += 2) {
+              const float2 x = __ffma2_rn(make_float2(p[c], p[c + 1]), s2, a2);
+              p[c] = ex2(x.x);
+              p[c + 1] = ex2(x.y);
+            }
           }
         }
         if (!tile_all_visible(i, jj, mk)) {
@@ -1271,9 +1290,15 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
           for (int c = 0; c < NC; ++c) dp[c] = ((keep >> c) & 1u) ? dp[c] * ks : 0.f;
         }
         uint32_t w[NC / 2];
+        {
+          const float2 ndl = make_float2(-dl, -dl);
 #pragma unroll
-        for (int e = 0; e < NC / 2; ++e)
-          w[e] = pack_bf16x2(p[2 * e] * (dp[2 * e] - dl), p[2 * e + 1] * (dp[2 * e + 1] - dl));
+          for (int e = 0; e < NC / 2; ++e) {
+            const float2 v = __fmul2_rn(make_float2(p[2 * e], p[2 * e + 1]),
+                                        __fadd2_rn(make_float2(dp[2 * e], dp[2 * e + 1]), ndl));
+            w[e] = pack_bf16x2(v.x, v.y);
+          }
+        }
         // bf16 dS goes over the first half of this warpgroup's own fp32 S columns
         tmem_st16(tmem + lane_base + tS0 + 128u * b + NC * h, w);
         tmem_wait_st();
