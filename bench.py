@@ -44,15 +44,15 @@ MEASURED_TRAFFIC = {
                                           "ncu --set full, one launch"),
     ("c4_causal_varlen_b32h16n2048d64", "fwd"): (791061760, "730a9286a82c",
                                                  "ncu --set full, one launch"),
-    ("c4_causal_b32h16n2048d64", "bwd_preprocess"): (417330176, "25eef99ccbb6",
+    ("c4_causal_b32h16n2048d64", "bwd_preprocess"): (417137152, "5594d3d7498f",
                                                      "ncu --set full, one launch"),
-    ("c4_causal_b32h16n2048d64", "bwd_dkdv"): (785554688, "25eef99ccbb6",
+    ("c4_causal_b32h16n2048d64", "bwd_dkdv"): (785500416, "5594d3d7498f",
                                                "ncu --set full, one launch"),
-    ("c4_causal_b32h16n2048d64", "bwd_dq"): (666776832, "25eef99ccbb6",
+    ("c4_causal_b32h16n2048d64", "bwd_dq"): (665004288, "5594d3d7498f",
                                              "ncu --set full, one launch"),
-    ("c5_causal_b2h32n8192d128", "bwd_dkdv"): (781176320, "25eef99ccbb6",
+    ("c5_causal_b2h32n8192d128", "bwd_dkdv"): (784435456, "5594d3d7498f",
                                                "ncu --set full, one launch"),
-    ("c5_causal_b2h32n8192d128", "bwd_dq"): (661154816, "25eef99ccbb6",
+    ("c5_causal_b2h32n8192d128", "bwd_dq"): (664123392, "5594d3d7498f",
                                              "ncu --set full, one launch"),
 }
 
