@@ -105,3 +105,29 @@ def test_full_lengths_are_no_restriction():
     b = G.run_library(inp, 0.125, True, (-1, -1))
     for n in a:
         assert torch.equal(a[n], b[n]), n
+
+
+@pytest.mark.parametrize("d", [64])
+def test_varlen_schedules_agree(d):
+    """Items are scheduled by their tile's distance from the start or end of the sequence
+    for batches of up to 8192 entries (tables built on the GPU), by the chunked order
+    beyond. Every item's result is independent of the CTA that computes it, so the first
+    entries of an 8200-entry batch (chunked order) must equal, bit for bit, the same entries
+    run as a batch of their own (the sorted order); sampled entries are also checked against
+    the oracle, and every row past a length must be zero."""
+    B, H, N = 8200, 1, 130
+    rng = np.random.default_rng(2500)
+    lens = [int(x) for x in rng.integers(0, N + 1, size=B)]
+    lens[:6] = [N, 0, 1, 128, 129, 64]
+    inp = synth.attention_inputs(B, H, N, d, 2500)
+    scale = 1.0 / np.sqrt(d)
+    big = G.run_library(inp, scale, True, (-1, -1), lengths=lens)
+    small_inp = {n: t[:16].clone() for n, t in inp.items()}
+    small = G.run_library(small_inp, scale, True, (-1, -1), lengths=lens[:16])
+    for n in small:
+        assert torch.equal(big[n][:16], small[n]), n
+    for b in (0, 2, 3, 4, 5, 4097, B - 1):
+        errs = G.compare(inp, big, scale, True, (-1, -1), heads=[(b, 0)], lengths=lens)
+        G.assert_within_bounds(errs, (b, lens[b]))
+    check_past_length(big, lens)
+
