@@ -39,6 +39,16 @@ fa_status_t check_problem(int B, int H, int N, int d, bool* empty) {
   return FA_OK;
 }
 
+// check_problem, and for a packed batch (cumulative lengths) its token count: a (total, H, d)
+// tensor must also have fewer than 2^31 elements; no tokens is an empty problem.
+fa_status_t check_problem_x(int B, int H, int N, int d, const Extras& x, bool* empty) {
+  const fa_status_t s = check_problem(B, H, N, d, empty);
+  if (s != FA_OK || *empty || x.cu == nullptr) return s;
+  if ((long long)x.total * H * d >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  if (x.total == 0) *empty = true;
+  return FA_OK;
+}
+
 fa_status_t check_mask(float scale, fa_window_t w) {
   if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
   if (w.left < -1 || w.right < -1) return FA_ERR_INVALID_ARG;
@@ -63,14 +73,19 @@ fa_status_t dispatch_features(std::integer_sequence<int, Fs...>, int feat, Args&
   return found ? s : FA_ERR_UNSUPPORTED;
 }
 
-// forward: every combination of ALiBi, key padding, residual and dropout; at head_dim 128
-// also the e4m3 forward
+// forward: every combination of ALiBi, key padding, residual and dropout, in the (B, H, N, d)
+// layout and packed (kFeatPacked = 32); at head_dim 128 also the e4m3 forward
 using FwdFeatures64 = std::integer_sequence<int, 0, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14,
-                                            15>;
+                                            15, 32, 33, 34, 35, 36, 37, 38, 39, 40, 41, 42, 43,
+                                            44, 45, 46, 47>;
 using FwdFeatures128 = std::integer_sequence<int, 0, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13,
-                                             14, 15, 16>;
-// backward passes: ALiBi, key padding and dropout (the residual only changes delta)
-using BwdFeatures = std::integer_sequence<int, 0, 1, 2, 3, 8, 9, 10, 11>;
+                                             14, 15, 16, 32, 33, 34, 35, 36, 37, 38, 39, 40, 41,
+                                             42, 43, 44, 45, 46, 47>;
+// backward passes: ALiBi, key padding and dropout (the residual only changes delta), in both
+// layouts; the fused pass only in the (B, H, N, d) layout
+using BwdFeatures = std::integer_sequence<int, 0, 1, 2, 3, 8, 9, 10, 11, 32, 33, 34, 35, 40, 41,
+                                          42, 43>;
+using FusedFeatures = std::integer_sequence<int, 0, 1, 2, 3, 8, 9, 10, 11>;
 
 // The launchers as class templates over the feature flags, for dispatch_features.
 template <int D>
@@ -121,7 +136,7 @@ size_t dq_acc_bytes(int B, int H, int N, int d) {
 // A variable-length batch (up to kVarlenSchedMaxB entries) adds, last, the tables of its
 // schedule (varlen_item), which the preprocess step writes.
 size_t sched_bytes(int B, int N, const Extras& x) {
-  if (x.seq_len == nullptr || B > fa::kVarlenSchedMaxB) return 0;
+  if (!x.varlen() || B > fa::kVarlenSchedMaxB) return 0;
   const size_t raw = 4 * (size_t)fa::varlen_sched_ints(B, fa::num_tiles(N));
   return (raw + 255) & ~size_t(255);
 }
@@ -170,6 +185,15 @@ fa_status_t resolve_options(const fa_options_t* opt, Extras* x) {
   if (opt->seq_lengths != nullptr && (reinterpret_cast<uintptr_t>(opt->seq_lengths) & 3u) != 0)
     return FA_ERR_MISALIGNED;
   x->seq_len = opt->seq_lengths;
+  // a packed batch: exclusive with seq_lengths, a token count >= 0, not the fused backward
+  // (its dQ conversion takes no options)
+  if (opt->cu_seqlens != nullptr) {
+    if ((reinterpret_cast<uintptr_t>(opt->cu_seqlens) & 3u) != 0) return FA_ERR_MISALIGNED;
+    if (opt->seq_lengths != nullptr || opt->total_tokens < 0) return FA_ERR_INVALID_ARG;
+    if (x->fused) return FA_ERR_UNSUPPORTED;
+    x->cu = opt->cu_seqlens;
+    x->total = opt->total_tokens;
+  }
   if (t > 0) {
     x->dropout = true;
     x->drop.seed_lo = (uint32_t)(opt->dropout_seed & 0xFFFFFFFFull);
@@ -199,7 +223,7 @@ fa_status_t forward(const void* q, const void* k, const void* v, void* o, float*
                     int N, int d, float scale, int causal, fa_window_t window, const Extras& x,
                     void* stream) {
   bool empty;
-  fa_status_t s = check_problem(B, H, N, d, &empty);
+  fa_status_t s = check_problem_x(B, H, N, d, x, &empty);
   if (s != FA_OK || empty) return s;
   if ((s = check_mask(scale, window)) != FA_OK) return s;
   if ((s = check_ptrs({q, k, v, o, lse})) != FA_OK) return s;
@@ -220,7 +244,7 @@ fa_status_t forward(const void* q, const void* k, const void* v, void* o, float*
 fa_status_t preprocess(const void* o, const void* dout, const float* lse, void* workspace, int B,
                        int H, int N, int d, const Extras& x, void* stream) {
   bool empty;
-  fa_status_t s = check_problem(B, H, N, d, &empty);
+  fa_status_t s = check_problem_x(B, H, N, d, x, &empty);
   if (s != FA_OK || empty) return s;
   if ((s = check_ptrs({o, dout, lse, workspace})) != FA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -228,12 +252,13 @@ fa_status_t preprocess(const void* o, const void* dout, const float* lse, void* 
   // the fused pass accumulates dQ: its accumulator starts at zero
   float* acc = uses_fused(d, x) ? dq_acc_of(workspace, B, H, N) : nullptr;
   // and with real lengths, the tables of the passes' schedule
-  const fa::SchedBuild sb{x.seq_len, sched_of(workspace, B, H, N, d, x), B, H, N,
+  const fa::SchedBuild sb{x.seq_len, x.cu, sched_of(workspace, B, H, N, d, x), B, H, N,
                           fa::num_tiles(N)};
   return d == 64
-             ? fa_host::launch_preprocess<64>(o, x.o_low, dout, lse, stats, acc, sb, B * H, N, st)
-             : fa_host::launch_preprocess<128>(o, x.o_low, dout, lse, stats, acc, sb, B * H, N,
-                                               st);
+             ? fa_host::launch_preprocess<64>(o, x.o_low, dout, lse, stats, acc, sb, x.cu,
+                                              x.total, H, B * H, N, st)
+             : fa_host::launch_preprocess<128>(o, x.o_low, dout, lse, stats, acc, sb, x.cu,
+                                               x.total, H, B * H, N, st);
 }
 
 // The fused pass (head_dim 64): dK, dV, and dQ added into the workspace's accumulator.
@@ -242,7 +267,7 @@ fa_status_t fused_pass(const void* q, const void* k, const void* v, const void* 
                        float scale, int causal, fa_window_t window, const Extras& x,
                        void* stream) {
   bool empty;
-  fa_status_t s = check_problem(B, H, N, d, &empty);
+  fa_status_t s = check_problem_x(B, H, N, d, x, &empty);
   if (s != FA_OK || empty) return s;
   if (d != 64) return FA_ERR_UNSUPPORTED;
   if ((s = check_mask(scale, window)) != FA_OK) return s;
@@ -252,7 +277,7 @@ fa_status_t fused_pass(const void* q, const void* k, const void* v, const void* 
   const Problem pb{B * H, H, N, scale, window.left, right};
   const int feat = x.features() & ~fa::kFeatResidual;
   const Extras xs = with_sched(x, workspace, B, H, N, d);
-  s = dispatch_features<FusedLaunch>(BwdFeatures(), feat, q, k, v, dout, workspace,
+  s = dispatch_features<FusedLaunch>(FusedFeatures(), feat, q, k, v, dout, workspace,
                                      dq_acc_of(workspace, B, H, N), dk, dv, pb, xs, st);
   // rows of dQ past the real length stay zero in the accumulator
   if (s != FA_OK || x.seq_len == nullptr) return s;
@@ -278,7 +303,7 @@ fa_status_t dkdv_pass(const void* q, const void* k, const void* v, const void* d
                       float scale, int causal, fa_window_t window, const Extras& x,
                       void* stream) {
   bool empty;
-  fa_status_t s = check_problem(B, H, N, d, &empty);
+  fa_status_t s = check_problem_x(B, H, N, d, x, &empty);
   if (s != FA_OK || empty) return s;
   if ((s = check_mask(scale, window)) != FA_OK) return s;
   if ((s = check_ptrs({q, k, v, dout, workspace, dk, dv})) != FA_OK) return s;
@@ -301,7 +326,7 @@ fa_status_t dq_pass(const void* q, const void* k, const void* v, const void* dou
                     const void* workspace, void* dq, int B, int H, int N, int d, float scale,
                     int causal, fa_window_t window, const Extras& x, void* stream) {
   bool empty;
-  fa_status_t s = check_problem(B, H, N, d, &empty);
+  fa_status_t s = check_problem_x(B, H, N, d, x, &empty);
   if (s != FA_OK || empty) return s;
   if ((s = check_mask(scale, window)) != FA_OK) return s;
   if ((s = check_ptrs({q, k, v, dout, workspace, dq})) != FA_OK) return s;
@@ -612,9 +637,11 @@ const char* fa_status_string(fa_status_t status) {
 fa_status_t fa_debug_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
   // every kernel unit has its own copy of the status word: read and clear them all
-  const int words[5] = {fa_host::take_status_fwd64(), fa_host::take_status_fwd128(),
-                        fa_host::take_status_bwd64(), fa_host::take_status_bwd128(),
-                        fa_host::take_status_fused64()};
+  const int words[9] = {fa_host::take_status_fwd64(),  fa_host::take_status_fwd128(),
+                        fa_host::take_status_bwd64(),  fa_host::take_status_bwd128(),
+                        fa_host::take_status_fused64(), fa_host::take_status_fwdp64(),
+                        fa_host::take_status_fwdp128(), fa_host::take_status_bwdp64(),
+                        fa_host::take_status_bwdp128()};
   bool timeout = false;
   for (int w : words) {
     if (w < 0) return FA_ERR_CUDA;

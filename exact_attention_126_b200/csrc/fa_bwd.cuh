@@ -52,21 +52,26 @@ namespace fa {
 // zeroes the accumulator rows it covers.
 // Block b covers rows 64x .. 64x+63 of head bh, with (bh, x) = divmod(b, Np/64), 8 rows
 // per warp; G = D/8 lanes share a row, 16 bytes of O and dO per lane, and a warp's loads
-// for its 8 rows are all issued before any is used.
+// for its 8 rows are all issued before any is used. In a packed batch (cu: B + 1 cumulative
+// lengths; O, dO (total, H, D), LSE (H, total)) the rows are those of the sequence, and
+// rows at or past its real length count as padding (+inf and 0).
 // ------------------------------------------------------------------------------------
-template <int D>
+template <int D, bool kPacked>
 __global__ void __launch_bounds__(256)
     fa_bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o,
                              const __nv_bfloat16* __restrict__ o_low,
                              const __nv_bfloat16* __restrict__ dout, const float* __restrict__ lse,
                              float* __restrict__ stats, float* __restrict__ dq_acc, SchedBuild sb,
-                             int BH, int N, int Np) {
+                             const int* __restrict__ cu_in, int total, int H, int BH, int N,
+                             int Np) {
+  const int* const cu = kPacked ? cu_in : nullptr;
   constexpr int G = D / 8;                      // lanes per row
   constexpr int kRowsPerPass = 32 / G;          // rows a warp covers per load
   constexpr int kPasses = 8 / kRowsPerPass;     // 8 rows per warp
   const int blocks_per_head = Np / 64;
   if ((int)blockIdx.x >= BH * blocks_per_head) {
-    if (threadIdx.x < 32) build_varlen_sched(sb.seq_len, sb.B, sb.H, sb.N, 1, sb.U, sb.tables);
+    if (threadIdx.x < 32)
+      build_varlen_sched(sb.seq_len, sb.cu, sb.B, sb.H, sb.N, 1, sb.U, sb.tables);
     return;
   }
   const int bh = blockIdx.x / blocks_per_head;
@@ -82,6 +87,15 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int e = threadIdx.x; e < kVec; e += 256) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  // rows this head holds: N, or in a packed batch its real length (and no row past the
+  // tensor's end)
+  const int base = seq_base(cu, bh, H);
+  int n_rows = N;
+  if (cu != nullptr) {
+    n_rows = real_length(nullptr, cu, bh, H, N);
+    if (base < 0) n_rows = 0;  // offsets outside [0, total] read nothing
+    if (total - base < n_rows) n_rows = total - base < 0 ? 0 : total - base;
+  }
   uint4 a[kPasses], b[kPasses], c[kPasses];
 #pragma unroll
   for (int p = 0; p < kPasses; ++p) {
@@ -89,8 +103,8 @@ __global__ void __launch_bounds__(256)
     a[p] = make_uint4(0, 0, 0, 0);
     b[p] = make_uint4(0, 0, 0, 0);
     c[p] = make_uint4(0, 0, 0, 0);
-    if (r < N) {
-      const size_t src = ((size_t)bh * N + r) * D + part * 8;
+    if (r < n_rows) {
+      const size_t src = row_at(cu, bh, H, N, base, r, D) + part * 8;
       a[p] = *reinterpret_cast<const uint4*>(o + src);
       b[p] = *reinterpret_cast<const uint4*>(dout + src);
       if (o_low != nullptr) c[p] = *reinterpret_cast<const uint4*>(o_low + src);
@@ -117,7 +131,7 @@ __global__ void __launch_bounds__(256)
     const int r = row0 + p * kRowsPerPass + sub;
     if (part == 0 && r < Np) {
       const size_t rp = (size_t)bh * Np + r;
-      stats[rp] = r < N ? lse[(size_t)bh * N + r] * kLog2e : INFINITY;
+      stats[rp] = r < n_rows ? lse[lse_at(cu, total, bh, H, N, base, r)] * kLog2e : INFINITY;
       stats[rows + rp] = acc;
     }
   }
@@ -140,7 +154,7 @@ __global__ void __launch_bounds__(256)
   const int tiles = num_tiles(N);
   const int bh = blockIdx.x / tiles;
   const int r0 = (blockIdx.x - bh * tiles) * kBlock;
-  const int L = real_length(seq_len, bh, H, N);
+  const int L = real_length(seq_len, nullptr, bh, H, N);
   const int r_end = r0 + kBlock < N ? r0 + kBlock : N;
   const int r_begin = r0 > L ? r0 : L;
   if (r_begin >= r_end) return;
@@ -155,6 +169,16 @@ __global__ void __launch_bounds__(256)
     if (t2 != nullptr) st_global_v4(t2 + off, 0u, 0u, 0u, 0u);
     if (lse != nullptr && part == 0) lse[base + r] = -INFINITY;
   }
+}
+
+// Whether the output tile of rows r0 .. r0+127 of a sequence of real length L (first token
+// `base`) leaves through a bulk store of the whole tile: always, except in a packed batch
+// (cu) the last, partial tile of a sequence, whose rows past L are the next sequence's, and
+// a tile not wholly inside the tensor's `total` tokens; those are written row by row
+// (row_written).
+__device__ __forceinline__ bool whole_tile_store(const int* cu, int total, int L, int base,
+                                                 int r0) {
+  return cu == nullptr || (r0 + kBlock <= L && base >= 0 && base + r0 + kBlock <= total);
 }
 
 struct BwdArgs {
@@ -180,6 +204,8 @@ struct BwdArgs {
   const uint8_t* kpad;  // (B, N) key-padding flags (nonzero = padded key), or null
   DropoutArgs drop;     // kFeatDropout kernels
   const int* seq_len;   // variable-length batch: B real lengths, or null
+  const int* cu;        // packed batch: B + 1 cumulative lengths (tensors (total, H, D),
+  int total;            // LSE (H, total)), or null
   int sorted;           // variable-length batch: the schedule of varlen_item, with ...
   const int* sched;     // ... its tables, written by fa_bwd_preprocess_kernel
 };
@@ -322,14 +348,16 @@ __device__ __forceinline__ constexpr uint32_t packed_col(int kk) {
 // Returns false when the stationary tile lies past the sequence's real length (a
 // variable-length batch): such an item has no work, and every role skips it without
 // advancing its counters. `mk` is the item's mask, over the real length.
+template <bool kPacked = false>
 __device__ __forceinline__ bool bwd_item(int k, const BwdArgs& a, bool rising, int& bh,
                                          int& tile, Mask& mk) {
+  const int* const cu = kPacked ? a.cu : nullptr;
   if (a.paired) {
     if (!paired_item(k, (int)gridDim.x, a.n_double, a.n_tiles, rising, bh, tile)) return false;
   } else if (a.sorted) {
     int u;
     if (!varlen_item(k, (int)gridDim.x, a.sched, a.n_tiles, a.H, bh, u)) return false;
-    const int n = real_length(a.seq_len, bh, a.H, a.N);
+    const int n = real_length(a.seq_len, cu, bh, a.H, a.N);
     mk = Mask{n, a.left, a.right};
     // key tiles count from the end of the sequence, query tiles from its start
     tile = rising ? num_tiles(n) - 1 - u : u;
@@ -340,7 +368,7 @@ __device__ __forceinline__ bool bwd_item(int k, const BwdArgs& a, bool rising, i
     bh = k / a.n_tiles;
     tile = k % a.n_tiles;
   }
-  const int n = real_length(a.seq_len, bh, a.H, a.N);
+  const int n = real_length(a.seq_len, cu, bh, a.H, a.N);
   mk = Mask{n, a.left, a.right};
   return tile < num_tiles(n);
 }
@@ -401,6 +429,8 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
   constexpr bool kAlibi = (kFeat & kFeatAlibi) != 0;
   constexpr bool kKpad = (kFeat & kFeatKpad) != 0;
   constexpr bool kDropout = (kFeat & kFeatDropout) != 0;
+  constexpr bool kPacked = (kFeat & kFeatPacked) != 0;
+  const int* const cu = kPacked ? a.cu : nullptr;  // a packed batch's cumulative lengths
   constexpr int kSBufs = (D == 64) ? 2 : 1;
   constexpr bool kDsInS = kSBufs == 2;               // dS^T over the second half of S^T
   // With one S^T buffer (head_dim 128) the products go in two 64-query halves: S^T, dP^T,
@@ -488,17 +518,18 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, j;
         Mask mk;
-        if (!bwd_item(k, a, true, bh, j, mk)) continue;
+        if (!bwd_item<kPacked>(k, a, true, bh, j, mk)) continue;
         int i_lo, i_hi;
         q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
         const int xb = items % C::kXBufs, xu = items / C::kXBufs;
+        const int base = seq_base(cu, bh, a.H), ty = tma_y(cu, bh, a.H, j * kBlock);
         if (!mbar_wait(bar(C::bXEmpty + xb), (xu & 1) ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar(C::bXFull + xb), 2 * C::kTile);
         for (int r = 0; r < C::kRegions; ++r) {
           tma_load_3d(sb + C::kX0 + xb * 2 * C::kTile + r * C::kRegionBytes, &tmK,
-                      bar(C::bXFull + xb), r * 64, j * kBlock, bh);
+                      bar(C::bXFull + xb), r * 64, ty, tma_z(cu, bh, base, j * kBlock));
           tma_load_3d(sb + C::kX1 + xb * 2 * C::kTile + r * C::kRegionBytes, &tmV,
-                      bar(C::bXFull + xb), r * 64, j * kBlock, bh);
+                      bar(C::bXFull + xb), r * 64, ty, tma_z(cu, bh, base, j * kBlock));
         }
         ++items;
         for (int i = i_lo; i <= i_hi; ++i, ++n) {
@@ -508,9 +539,10 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(bar(C::bY0Full + s), C::kTile + 2 * 512);
+          const int yi = tma_y(cu, bh, a.H, i * kBlock), zi = tma_z(cu, bh, base, i * kBlock);
           for (int r = 0; r < C::kRegions; ++r)
             tma_load_3d(sb + C::kY0 + s * C::kTile + r * C::kRegionBytes, &tmQ,
-                        bar(C::bY0Full + s), r * 64, i * kBlock, bh);
+                        bar(C::bY0Full + s), r * 64, yi, zi);
           // LSE*log2e and delta of the 128 rows of query tile i (512 bytes each)
           const float* st = a.stats + (size_t)bh * a.Np + (size_t)i * kBlock;
           bulk_load(sb + C::kLse + s * 512, st, 512, bar(C::bY0Full + s));
@@ -518,7 +550,7 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
           mbar_arrive_expect_tx(bar(C::bY1Full + s), C::kTile);
           for (int r = 0; r < C::kRegions; ++r)
             tma_load_3d(sb + C::kY1 + s * C::kTile + r * C::kRegionBytes, &tmdO,
-                        bar(C::bY1Full + s), r * 64, i * kBlock, bh);
+                        bar(C::bY1Full + s), r * 64, yi, zi);
         }
       }
       // Drain: every copy issued must have landed before the CTA may exit.
@@ -537,7 +569,7 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, j;
         Mask mk;
-        if (!bwd_item(k, a, true, bh, j, mk)) continue;
+        if (!bwd_item<kPacked>(k, a, true, bh, j, mk)) continue;
         int i_lo, i_hi;
         q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
         const int xb = items % C::kXBufs, xu = items / C::kXBufs;
@@ -652,7 +684,7 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, j;
         Mask mk;
-        if (!bwd_item(k, a, true, bh, j, mk)) continue;
+        if (!bwd_item<kPacked>(k, a, true, bh, j, mk)) continue;
         int i_lo, i_hi;
         q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
         for (int i = i_lo; i <= i_hi; ++i, ++t) {
@@ -761,15 +793,20 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
       for (int k = blockIdx.x; k < a.n_items; k += gridDim.x) {
         int bh, j;
         Mask mk;
-        if (!bwd_item(k, a, true, bh, j, mk)) continue;
+        if (!bwd_item<kPacked>(k, a, true, bh, j, mk)) continue;
         const int xb = items % C::kXBufs;
         if (!mbar_wait(bar(bStaged), items & 1, abort_flag)) break;
         ++items;
-        for (int r = 0; r < C::kRegions; ++r) {
-          tma_store_3d(&tmdK, sb + C::kX0 + xb * 2 * C::kTile + r * C::kRegionBytes, r * 64,
-                       j * kBlock, bh);
-          tma_store_3d(&tmdV, sb + C::kX1 + xb * 2 * C::kTile + r * C::kRegionBytes, r * 64,
-                       j * kBlock, bh);
+        // (a partial tile of a packed batch was written row by row)
+        if (whole_tile_store(cu, a.total, mk.N, seq_base(cu, bh, a.H), j * kBlock)) {
+          const int base = seq_base(cu, bh, a.H);
+          const int ty = tma_y(cu, bh, a.H, j * kBlock), tz = tma_z(cu, bh, base, j * kBlock);
+          for (int r = 0; r < C::kRegions; ++r) {
+            tma_store_3d(&tmdK, sb + C::kX0 + xb * 2 * C::kTile + r * C::kRegionBytes, r * 64,
+                         ty, tz);
+            tma_store_3d(&tmdV, sb + C::kX1 + xb * 2 * C::kTile + r * C::kRegionBytes, r * 64,
+                         ty, tz);
+          }
         }
         bulk_commit();
         bulk_wait_read();
@@ -790,7 +827,7 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
     for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
       int bh, j;
       Mask mk;
-      if (!bwd_item(k, a, true, bh, j, mk)) continue;
+      if (!bwd_item<kPacked>(k, a, true, bh, j, mk)) continue;
       int i_lo, i_hi;
       q_tiles_for_kv_tile(j, mk, i_lo, i_hi);
       const int n_it = i_hi - i_lo + 1;
@@ -929,13 +966,14 @@ __global__ void __launch_bounds__(DkdvCfg<D>::kThreads, 1)
       ++items;
       tc_fence_after();
       constexpr int NO = D / C::kGroups;
-      if (C::kStageOut) {
+      if (C::kStageOut && whole_tile_store(cu, a.total, mk.N, seq_base(cu, bh, a.H), j * kBlock)) {
         stage_acc_cols<NO>(tmem + lane_base + tDV + NO * h, 1.f, tV, t_row, NO * h);
         stage_acc_cols<NO>(tmem + lane_base + tDK + NO * h, a.scale, tK, t_row, NO * h);
         fence_async_smem();
       } else {
-        const bool valid = c < a.N;
-        const size_t off = ((size_t)bh * a.N + (valid ? c : 0)) * D + NO * h;
+        const int base = seq_base(cu, bh, a.H);
+        const bool valid = row_written(cu, a.total, a.N, mk.N, base, c);
+        const size_t off = row_at(cu, bh, a.H, a.N, base, valid ? c : 0, D) + NO * h;
         store_acc_cols<NO>(tmem + lane_base + tDV + NO * h, 1.f, a.out1 + off, valid);
         store_acc_cols<NO>(tmem + lane_base + tDK + NO * h, a.scale, a.out0 + off, valid);
       }
@@ -974,6 +1012,8 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
   constexpr bool kAlibi = (kFeat & kFeatAlibi) != 0;
   constexpr bool kKpad = (kFeat & kFeatKpad) != 0;
   constexpr bool kDropout = (kFeat & kFeatDropout) != 0;
+  constexpr bool kPacked = (kFeat & kFeatPacked) != 0;
+  const int* const cu = kPacked ? a.cu : nullptr;  // a packed batch's cumulative lengths
   constexpr uint32_t tS0 = 0, tDP = 256, tDQ = 384;
   // per S buffer: S full, dS full, dQ done (dQ read that buffer's dS); dP full, dP free;
   // dQ read by the epilogue, dQ of the item complete
@@ -1029,17 +1069,19 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, i;
         Mask mk;
-        if (!bwd_item(k, a, false, bh, i, mk)) continue;
+        if (!bwd_item<kPacked>(k, a, false, bh, i, mk)) continue;
         int j_lo, j_hi;
         kv_tiles_for_q_tile(i, mk, j_lo, j_hi);
         const int xb = items % C::kXBufs, xu = items / C::kXBufs;
+        const int base = seq_base(cu, bh, a.H);
         if (!mbar_wait(bar(C::bXEmpty + xb), (xu & 1) ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar(C::bXFull + xb), 2 * C::kTile);
+        const int yi = tma_y(cu, bh, a.H, i * kBlock), zi = tma_z(cu, bh, base, i * kBlock);
         for (int r = 0; r < C::kRegions; ++r) {
           tma_load_3d(sb + C::kX0 + xb * 2 * C::kTile + r * C::kRegionBytes, &tmQ,
-                      bar(C::bXFull + xb), r * 64, i * kBlock, bh);
+                      bar(C::bXFull + xb), r * 64, yi, zi);
           tma_load_3d(sb + C::kX1 + xb * 2 * C::kTile + r * C::kRegionBytes, &tmdO,
-                      bar(C::bXFull + xb), r * 64, i * kBlock, bh);
+                      bar(C::bXFull + xb), r * 64, yi, zi);
         }
         ++items;
         for (int jj = j_lo; jj <= j_hi; ++jj) {
@@ -1051,7 +1093,8 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
           mbar_arrive_expect_tx(bar(C::bY0Full + s0), C::kTile);
           for (int r = 0; r < C::kRegions; ++r)
             tma_load_3d(sb + C::kY0 + s0 * C::kTile + r * C::kRegionBytes, &tmK,
-                        bar(C::bY0Full + s0), r * 64, jj * kBlock, bh);
+                        bar(C::bY0Full + s0), r * 64, tma_y(cu, bh, a.H, jj * kBlock),
+                        tma_z(cu, bh, base, jj * kBlock));
           ++n0;
           if (!kOneRelease &&
               !mbar_wait(bar(C::bY1Empty + s1), ((n1 / C::kStages1) & 1) ^ 1, abort_flag)) {
@@ -1061,7 +1104,8 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
           mbar_arrive_expect_tx(bar(C::bY1Full + s1), C::kTile);
           for (int r = 0; r < C::kRegions; ++r)
             tma_load_3d(sb + C::kY1 + s1 * C::kTile + r * C::kRegionBytes, &tmV,
-                        bar(C::bY1Full + s1), r * 64, jj * kBlock, bh);
+                        bar(C::bY1Full + s1), r * 64, tma_y(cu, bh, a.H, jj * kBlock),
+                        tma_z(cu, bh, base, jj * kBlock));
           ++n1;
         }
       }
@@ -1080,7 +1124,7 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, i;
         Mask mk;
-        if (!bwd_item(k, a, false, bh, i, mk)) continue;
+        if (!bwd_item<kPacked>(k, a, false, bh, i, mk)) continue;
         int j_lo, j_hi;
         kv_tiles_for_q_tile(i, mk, j_lo, j_hi);
         const int xb = items % C::kXBufs, xu = items / C::kXBufs;
@@ -1146,7 +1190,7 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
         int bh, i;
         Mask mk;
-        if (!bwd_item(k, a, false, bh, i, mk)) continue;
+        if (!bwd_item<kPacked>(k, a, false, bh, i, mk)) continue;
         int j_lo, j_hi;
         kv_tiles_for_q_tile(i, mk, j_lo, j_hi);
         for (int jj = j_lo; jj <= j_hi; ++jj, ++t) {
@@ -1186,13 +1230,18 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
       for (int k = blockIdx.x; k < a.n_items; k += gridDim.x) {
         int bh, i;
         Mask mk;
-        if (!bwd_item(k, a, false, bh, i, mk)) continue;
+        if (!bwd_item<kPacked>(k, a, false, bh, i, mk)) continue;
         const int xb = items % C::kXBufs;
         if (!mbar_wait(bar(bStaged), items & 1, abort_flag)) break;
         ++items;
-        for (int rg = 0; rg < C::kRegions; ++rg)
-          tma_store_3d(&tmdQ, sb + C::kX0 + xb * 2 * C::kTile + rg * C::kRegionBytes, rg * 64,
-                       i * kBlock, bh);
+        // (a partial tile of a packed batch was written row by row)
+        if (whole_tile_store(cu, a.total, mk.N, seq_base(cu, bh, a.H), i * kBlock)) {
+          const int base = seq_base(cu, bh, a.H);
+          for (int rg = 0; rg < C::kRegions; ++rg)
+            tma_store_3d(&tmdQ, sb + C::kX0 + xb * 2 * C::kTile + rg * C::kRegionBytes,
+                         rg * 64, tma_y(cu, bh, a.H, i * kBlock),
+                         tma_z(cu, bh, base, i * kBlock));
+        }
         bulk_commit();
         bulk_wait_read();
         mbar_arrive(bar(C::bXEmpty + xb));
@@ -1211,7 +1260,7 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
     for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
       int bh, i;
       Mask mk;
-      if (!bwd_item(k, a, false, bh, i, mk)) continue;
+      if (!bwd_item<kPacked>(k, a, false, bh, i, mk)) continue;
       int j_lo, j_hi;
       kv_tiles_for_q_tile(i, mk, j_lo, j_hi);
       const int n_it = j_hi - j_lo + 1;
@@ -1320,12 +1369,13 @@ __global__ void __launch_bounds__(DqCfg<D>::kThreads, 1)
       ++items;
       tc_fence_after();
       constexpr int NO = D / C::kGroups;
-      if (C::kStageOut) {
+      if (C::kStageOut && whole_tile_store(cu, a.total, mk.N, seq_base(cu, bh, a.H), i * kBlock)) {
         stage_acc_cols<NO>(tmem + lane_base + tDQ + NO * h, a.scale, tQ, t_row, NO * h);
         fence_async_smem();
       } else {
-        const bool valid = r < a.N;
-        const size_t off = ((size_t)bh * a.N + (valid ? r : 0)) * D + NO * h;
+        const int base = seq_base(cu, bh, a.H);
+        const bool valid = row_written(cu, a.total, a.N, mk.N, base, r);
+        const size_t off = row_at(cu, bh, a.H, a.N, base, valid ? r : 0, D) + NO * h;
         store_acc_cols<NO>(tmem + lane_base + tDQ + NO * h, a.scale, a.out0 + off, valid);
       }
       // dQ has been read: the next item's first product may overwrite it

@@ -63,6 +63,8 @@ struct FwdArgs {
   __nv_bfloat16* o_low;      // (B, H, N, d) bf16 residual O - bf16(O), or null
   DropoutArgs drop;          // kFeatDropout kernels
   const int* seq_len;        // variable-length batch: B real lengths, or null
+  const int* cu;             // packed batch: B + 1 cumulative lengths (tensors (total, H, D),
+  int total;                 // LSE (H, total)), or null
   int sorted;                // variable-length batch: the schedule of varlen_item, whose
                              // tables each CTA builds in shared memory after kMisc
   float o_scale;             // kFeatFp8: the V descale, applied to O in the epilogue
@@ -157,8 +159,11 @@ __device__ __forceinline__ FwdItem no_fwd_item() {
   return it;
 }
 
-// `sched`: the varlen_item tables (shared memory) when a.sorted.
+// `sched`: the varlen_item tables (shared memory) when a.sorted; kPacked: a packed batch
+// (a.cu), else a.cu is not looked at.
+template <bool kPacked>
 __device__ __forceinline__ FwdItem fwd_item(int k, const FwdArgs& a, const int* sched) {
+  const int* const cu = kPacked ? a.cu : nullptr;
   FwdItem it;
   int pair;
   if (a.paired) {
@@ -173,7 +178,7 @@ __device__ __forceinline__ FwdItem fwd_item(int k, const FwdArgs& a, const int* 
     it.bh = k / a.n_pairs;
     pair = k % a.n_pairs;
   }
-  it.n = real_length(a.seq_len, it.bh, a.H, a.N);
+  it.n = real_length(a.seq_len, cu, it.bh, a.H, a.N);
   const Mask mk{it.n, a.left, a.right};
   const int n_qtiles = num_tiles(it.n);
   it.m[0] = a.per_item * pair;
@@ -232,6 +237,8 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
   constexpr bool kKpad = (kFeat & kFeatKpad) != 0;
   constexpr bool kResidual = (kFeat & kFeatResidual) != 0;
   constexpr bool kDropout = (kFeat & kFeatDropout) != 0;
+  constexpr bool kPacked = (kFeat & kFeatPacked) != 0;
+  const int* const cu = kPacked ? a.cu : nullptr;  // a packed batch's cumulative lengths
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -277,8 +284,8 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
     tmem_relinquish();
   }
   int* sched = reinterpret_cast<int*>(smem + C::kMisc + 16);
-  if (a.sorted && warp == 1) build_varlen_sched(a.seq_len, a.BH / a.H, a.H, a.N, a.per_item,
-                                                a.n_pairs, sched);
+  if (a.sorted && warp == 1)
+    build_varlen_sched(a.seq_len, cu, a.BH / a.H, a.H, a.N, a.per_item, a.n_pairs, sched);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -294,8 +301,9 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
       int kc = 0, vc = 0;  // K and V loads issued (ring positions)
       bool ok = true;
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
-        const FwdItem it = fwd_item(k, a, sched);
+        const FwdItem it = fwd_item<kPacked>(k, a, sched);
         if (!it.has_a) continue;  // past the real length: nothing to load
+        const int base = seq_base(cu, it.bh, a.H);
         for (int s = 0; s < 2; ++s) {
           if (s == 1 && !it.has_b) break;
           // Q_s of this item replaces the previous item's once its last S_s has been read
@@ -308,7 +316,8 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
           const int qslot = s * C::kQBufs + nq[s] % C::kQBufs;
           for (int r = 0; r < C::kRegions; ++r)
             tma_load_3d(sb + C::kQ + qslot * C::kTile + r * C::kRegionBytes, &tmQ, bar(C::bQFull + qb),
-                        r * 64, it.m[s] * kBlock, it.bh);
+                        r * 64, tma_y(cu, it.bh, a.H, it.m[s] * kBlock),
+                        tma_z(cu, it.bh, base, it.m[s] * kBlock));
           ++nq[s];
         }
         for (int j = it.first; ok && j <= it.last; ++j) {
@@ -320,13 +329,15 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
           mbar_arrive_expect_tx(bar(C::bKFull + sk), C::kTile);
           for (int r = 0; r < C::kRegions; ++r)
             tma_load_3d(sb + C::kK + sk * C::kTile + r * C::kRegionBytes, &tmK,
-                        bar(C::bKFull + sk), r * 64, j * kBlock, it.bh);
+                        bar(C::bKFull + sk), r * 64, tma_y(cu, it.bh, a.H, j * kBlock),
+                        tma_z(cu, it.bh, base, j * kBlock));
           ++kc;
           if (a.fault == 1) continue;
           mbar_arrive_expect_tx(bar(C::bVFull + sk), C::kTile);
           for (int r = 0; r < C::kRegions; ++r)
             tma_load_3d(sb + C::kV + sk * C::kTile + r * C::kRegionBytes, &tmV,
-                        bar(C::bVFull + sk), r * 64, j * kBlock, it.bh);
+                        bar(C::bVFull + sk), r * 64, tma_y(cu, it.bh, a.H, j * kBlock),
+                        tma_z(cu, it.bh, base, j * kBlock));
           ++vc;
         }
       }
@@ -536,7 +547,7 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
       };
 
       for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
-        const FwdItem it = fwd_item(k, a, sched);
+        const FwdItem it = fwd_item<kPacked>(k, a, sched);
         if (!it.has_a) continue;  // past the real length: no products
         const FwdRange rg = fwd_range(it, s);
         const int n = it.last - it.first + 1;
@@ -582,7 +593,7 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
 
 
     for (int k = blockIdx.x; ok && k < a.n_items; k += gridDim.x) {
-      const FwdItem it = fwd_item(k, a, sched);
+      const FwdItem it = fwd_item<kPacked>(k, a, sched);
       const FwdRange rg = fwd_range(it, s);
       if (!rg.has) continue;
       const Mask mk{it.n, a.left, a.right};
@@ -918,7 +929,13 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
       float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
       if (kDropout) inv_l *= a.drop.keep_scale;
       if (kFp8) inv_l *= a.o_scale;
-      __nv_bfloat16* orow = a.o + ((size_t)it.bh * a.N + (row < a.N ? row : 0)) * D;
+      // (the (B*H, N, d) layout forms its row pointer directly: through the packed helpers
+      // the same expression compiled to a measurably slower d = 64 kernel)
+      const int base = kPacked ? seq_base(cu, it.bh, a.H) : 0;
+      const bool written = kPacked ? row_written(cu, a.total, a.N, it.n, base, row) : row < a.N;
+      __nv_bfloat16* orow =
+          kPacked ? a.o + row_at(cu, it.bh, a.H, a.N, base, written ? row : 0, D)
+                  : a.o + ((size_t)it.bh * a.N + (row < a.N ? row : 0)) * D;
 #pragma unroll
       for (int q = 0; q < D / 32; ++q) {
         uint32_t o[32];
@@ -929,7 +946,7 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
 #pragma unroll
         for (int c = 0; c < 16; ++c)
           w[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
-        if (row < a.N) {
+        if (written) {
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
             st_global_v4(orow + 32 * q + 8 * v4, w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2],
@@ -945,8 +962,8 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
                 __uint_as_float(o[2 * c + 1]) * inv_l - __uint_as_float(w[c] & 0xFFFF0000u);
             w[c] = pack_bf16x2(r0, r1);
           }
-          if (row < a.N) {
-            __nv_bfloat16* lrow = a.o_low + ((size_t)it.bh * a.N + row) * D;
+          if (written) {
+            __nv_bfloat16* lrow = a.o_low + row_at(cu, it.bh, a.H, a.N, base, row, D);
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4)
               st_global_v4(lrow + 32 * q + 8 * v4, w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2],
@@ -957,8 +974,8 @@ __global__ void __launch_bounds__(FwdCfg<D, (kFeat & kFeatFp8) != 0>::kThreads, 
       // O_s has been read: the next item's first P V may overwrite it
       tc_fence_before();
       mbar_arrive_warp(bar(C::bOFree + s));
-      if (row < a.N)
-        a.lse[(size_t)it.bh * a.N + row] =
+      if (written)
+        a.lse[lse_at(cu, a.total, it.bh, a.H, a.N, base, row)] =
             (l_run > 0.f) ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
     }
   }

@@ -9,7 +9,8 @@ FA_INSTANTIATE_BWD(64, 0) FA_INSTANTIATE_BWD(64, 1) FA_INSTANTIATE_BWD(64, 2)
 FA_INSTANTIATE_BWD(64, 3) FA_INSTANTIATE_BWD(64, 8) FA_INSTANTIATE_BWD(64, 9)
 FA_INSTANTIATE_BWD(64, 10) FA_INSTANTIATE_BWD(64, 11)
 template fa_status_t launch_preprocess<64>(const void*, const void*, const void*, const float*,
-                                           float*, float*, const fa::SchedBuild&, int, int,
+                                           float*, float*, const fa::SchedBuild&, const int*, int,
+                                           int, int, int,
                                            cudaStream_t);
 template fa_status_t launch_dq_convert<64>(const float*, void*, int, int, float, cudaStream_t);
 template fa_status_t launch_fill_past_length<64>(void*, void*, void*, float*, const int*, int,

@@ -24,15 +24,20 @@ struct Extras {
                                    // dK/dV and dQ passes
   const int* seq_len = nullptr;    // variable-length batch: B real lengths
   const int* sched = nullptr;      // ... and the backward's schedule tables in its workspace
+  const int* cu = nullptr;         // packed batch: B + 1 cumulative lengths, and ...
+  int total = 0;                   // ... the tokens of its (total, H, d) tensors
   bool fp8 = false;                // forward on e4m3 Q, K, V (the kFeatFp8 kernel)
   float o_scale = 1.f;             // with fp8: the V descale, applied to O
   fa::DropoutArgs drop = {0, 0, 0, 0, 1.f};
+
+  // A batch of sequences of their own lengths (padded or packed).
+  bool varlen() const { return seq_len != nullptr || cu != nullptr; }
 
   // The kernel variant these options select (the backward passes ignore kFeatResidual).
   int features() const {
     return (alibi ? fa::kFeatAlibi : 0) | (kpad ? fa::kFeatKpad : 0) |
            (o_low ? fa::kFeatResidual : 0) | (dropout ? fa::kFeatDropout : 0) |
-           (fp8 ? fa::kFeatFp8 : 0);
+           (fp8 ? fa::kFeatFp8 : 0) | (cu ? fa::kFeatPacked : 0);
   }
 };
 
@@ -54,7 +59,8 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
 template <int D>
 fa_status_t launch_preprocess(const void* o, const void* o_low, const void* dout,
                               const float* lse, float* stats, float* dq_acc,
-                              const fa::SchedBuild& sb, int BH, int N, cudaStream_t st);
+                              const fa::SchedBuild& sb, const int* cu, int total, int H,
+                              int BH, int N, cudaStream_t st);
 
 // The fused backward pass (head_dim 64): dK, dV, and dQ added into `dq_acc`.
 template <int kFeat>
@@ -86,6 +92,10 @@ fa_status_t launch_fill_past_length(void* t0, void* t1, void* t2, float* lse,
 // returns -1 if reading it failed.
 int take_status_fwd64();
 int take_status_fwd128();
+int take_status_fwdp64();
+int take_status_fwdp128();
+int take_status_bwdp64();
+int take_status_bwdp128();
 int take_status_bwd64();
 int take_status_bwd128();
 int take_status_fused64();

@@ -77,6 +77,28 @@ inline bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A packed (total, H, d) bf16 tensor viewed as (d, H, total): a box of 1 head x 128 tokens x
+// 64 columns lands in shared memory as the (B*H, N, d) view's 128 x 64 box does.
+inline bool make_map_packed(CUtensorMap* map, const void* base, int total, int H, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)total};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
+  const cuuint32_t box[3] = {64, 1, (cuuint32_t)kBlock};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The map of a bf16 attention tensor of the problem: (B*H, N, d), or packed (total, H, d)
+// when the options carry cumulative lengths.
+inline bool map_rows(CUtensorMap* map, const void* base, const Problem& pb, const Extras& x,
+                     int d) {
+  return x.cu != nullptr ? make_map_packed(map, base, x.total, pb.H, d)
+                         : make_map(map, base, pb.BH, pb.N, d);
+}
+
 constexpr int kMaxSmemPerBlock = 232448;  // the opt-in limit of sm_100
 
 template <typename Kernel>
@@ -155,8 +177,8 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     if (!make_map_u8(&mq, q, BH, N, D) || !make_map_u8(&mkk, k, BH, N, D) ||
         !make_map_u8(&mv, v, BH, N, D))
       return FA_ERR_CUDA;
-  } else if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
-             !make_map(&mv, v, BH, N, D)) {
+  } else if (!map_rows(&mq, q, pb, x, D) || !map_rows(&mkk, k, pb, x, D) ||
+             !map_rows(&mv, v, pb, x, D)) {
     return FA_ERR_CUDA;
   }
   using C = fa::FwdCfg<D, kFp8>;
@@ -172,12 +194,12 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   a.n_items = BH * a.n_pairs;
   a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
   a.group = head_group(BH, a.n_pairs);
-  pair_schedule(a, BH, a.n_pairs, left, right, x.seq_len != nullptr);
+  pair_schedule(a, BH, a.n_pairs, left, right, x.varlen());
   // a variable-length batch: the varlen_item schedule, its tables in shared memory
   a.sorted = 0;
   int smem = C::kSmemBytes;
   const int sched_bytes = 4 * fa::varlen_sched_ints(BH / H, a.n_pairs);
-  if (x.seq_len != nullptr && BH / H <= fa::kVarlenSchedMaxB &&
+  if (x.varlen() && BH / H <= fa::kVarlenSchedMaxB &&
       C::kSmemBytes + sched_bytes <= kMaxSmemPerBlock) {
     varlen_schedule(a, BH, a.n_pairs);
     smem += sched_bytes;
@@ -193,6 +215,8 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   a.o_low = static_cast<__nv_bfloat16*>(x.o_low);
   a.drop = x.drop;
   a.seq_len = x.seq_len;
+  a.cu = x.cu;
+  a.total = x.total;
   a.o_scale = x.o_scale;
   const int grid = persistent_grid(a);
   fa::fa_fwd_kernel<D, kFeat><<<grid, C::kThreads, smem, st>>>(mq, mkk, mv, a);
@@ -204,14 +228,17 @@ inline int padded_rows(int N) { return fa::num_tiles(N) * kBlock; }
 template <int D>
 fa_status_t launch_preprocess(const void* o, const void* o_low, const void* dout,
                               const float* lse, float* stats, float* dq_acc,
-                              const fa::SchedBuild& sb, int BH, int N, cudaStream_t st) {
+                              const fa::SchedBuild& sb, const int* cu, int total, int H,
+                              int BH, int N, cudaStream_t st) {
   const int Np = padded_rows(N);
   // 64 rows per block, blocks of one head consecutive; BH * Np / 64 < 2^31 because every
   // tensor has fewer than 2^31 elements (d >= 64); one more block builds the tables of sb
   const long long blocks = (long long)BH * (Np / 64) + (sb.tables != nullptr ? 1 : 0);
-  fa::fa_bwd_preprocess_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
+  auto kernel = cu != nullptr ? fa::fa_bwd_preprocess_kernel<D, true>
+                              : fa::fa_bwd_preprocess_kernel<D, false>;
+  kernel<<<(unsigned)blocks, 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(o_low),
-      static_cast<const __nv_bfloat16*>(dout), lse, stats, dq_acc, sb, BH, N, Np);
+      static_cast<const __nv_bfloat16*>(dout), lse, stats, dq_acc, sb, cu, total, H, BH, N, Np);
   return launched();
 }
 
@@ -235,7 +262,7 @@ inline fa::BwdArgs bwd_args(const void* ws, const Problem& pb, const Extras& x) 
   a.n_items = BH * a.n_tiles;
   a.longest_first = (left >= 0 || right >= 0) ? 1 : 0;
   a.group = head_group(BH, a.n_tiles);
-  pair_schedule(a, BH, a.n_tiles, left, right, x.seq_len != nullptr);
+  pair_schedule(a, BH, a.n_tiles, left, right, x.varlen());
   a.sorted = 0;
   a.sched = x.sched;
   if (x.sched != nullptr) varlen_schedule(a, BH, a.n_tiles);
@@ -244,6 +271,8 @@ inline fa::BwdArgs bwd_args(const void* ws, const Problem& pb, const Extras& x) 
   a.kpad = x.kpad;
   a.drop = x.drop;
   a.seq_len = x.seq_len;
+  a.cu = x.cu;
+  a.total = x.total;
   return a;
 }
 
@@ -251,11 +280,10 @@ template <int D, int kFeat>
 fa_status_t launch_dkdv(const void* q, const void* k, const void* v, const void* dout,
                         const void* ws, void* dk, void* dv, const Problem& pb, const Extras& x,
                         cudaStream_t st) {
-  const int BH = pb.BH, N = pb.N;
   CUtensorMap mq, mkk, mv, mdo, mdk, mdv;
-  if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
-      !make_map(&mv, v, BH, N, D) || !make_map(&mdo, dout, BH, N, D) ||
-      !make_map(&mdk, dk, BH, N, D) || !make_map(&mdv, dv, BH, N, D))
+  if (!map_rows(&mq, q, pb, x, D) || !map_rows(&mkk, k, pb, x, D) ||
+      !map_rows(&mv, v, pb, x, D) || !map_rows(&mdo, dout, pb, x, D) ||
+      !map_rows(&mdk, dk, pb, x, D) || !map_rows(&mdv, dv, pb, x, D))
     return FA_ERR_CUDA;
   using C = fa::DkdvCfg<D>;
   if (set_smem(fa::fa_bwd_dkdv_kernel<D, kFeat>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;
@@ -272,11 +300,10 @@ template <int D, int kFeat>
 fa_status_t launch_dq(const void* q, const void* k, const void* v, const void* dout,
                       const void* ws, void* dq, const Problem& pb, const Extras& x,
                       cudaStream_t st) {
-  const int BH = pb.BH, N = pb.N;
   CUtensorMap mq, mkk, mv, mdo, mdq;
-  if (!make_map(&mq, q, BH, N, D) || !make_map(&mkk, k, BH, N, D) ||
-      !make_map(&mv, v, BH, N, D) || !make_map(&mdo, dout, BH, N, D) ||
-      !make_map(&mdq, dq, BH, N, D))
+  if (!map_rows(&mq, q, pb, x, D) || !map_rows(&mkk, k, pb, x, D) ||
+      !map_rows(&mv, v, pb, x, D) || !map_rows(&mdo, dout, pb, x, D) ||
+      !map_rows(&mdq, dq, pb, x, D))
     return FA_ERR_CUDA;
   using C = fa::DqCfg<D>;
   if (set_smem(fa::fa_bwd_dq_kernel<D, kFeat>, C::kSmemBytes) != FA_OK) return FA_ERR_CUDA;

@@ -19,6 +19,7 @@ constexpr int kFeatKpad = 2;      // (B, N) key-padding flags
 constexpr int kFeatResidual = 4;  // forward also writes O - bf16(O)
 constexpr int kFeatDropout = 8;   // attention weights dropped with Philox keep flags
 constexpr int kFeatFp8 = 16;      // forward on e4m3 Q, K, V (P in e4m3 for the P V product)
+constexpr int kFeatPacked = 32;   // a packed batch: (total, H, D) tensors, cumulative lengths
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Mask {
@@ -34,12 +35,55 @@ __host__ __device__ inline int resolve_right(int causal, int right) {
 __host__ __device__ inline int num_tiles(int N) { return (N + kBlock - 1) / kBlock; }
 
 #ifdef __CUDACC__
-// The real length of (batch, head) bh's sequence in a variable-length batch: seq_len[bh / H]
-// clamped to [0, N], or N when the batch is not variable-length (seq_len == nullptr).
-__device__ __forceinline__ int real_length(const int* seq_len, int bh, int H, int N) {
-  if (seq_len == nullptr) return N;
-  const int L = __ldg(seq_len + bh / H);
+// The real length of (batch, head) bh's sequence in a variable-length batch: seq_len[bh / H],
+// or in a packed batch (cumulative lengths cu) cu[b + 1] - cu[b], clamped to [0, N]; N when
+// the batch is not variable-length (both null).
+__device__ __forceinline__ int real_length(const int* seq_len, const int* cu, int bh, int H,
+                                           int N) {
+  int L;
+  if (cu != nullptr) {
+    const int b = bh / H;
+    L = __ldg(cu + b + 1) - __ldg(cu + b);
+  } else if (seq_len != nullptr) {
+    L = __ldg(seq_len + bh / H);
+  } else {
+    return N;
+  }
   return L < 0 ? 0 : (L > N ? N : L);
+}
+
+// Where the rows of (batch, head) bh lie. Without cumulative lengths the tensors are
+// (B*H, N, D) and the LSE (B*H, N). A packed batch (cu = B + 1 cumulative lengths, `total`
+// tokens) stores the tensors as (total, H, D) and the LSE as (H, total): row r of sequence
+// b is token cu[b] + r. `base` is seq_base() of the head.
+__device__ __forceinline__ int seq_base(const int* cu, int bh, int H) {
+  return cu != nullptr ? __ldg(cu + bh / H) : 0;
+}
+// element offset of row r in a D-wide tensor
+__device__ __forceinline__ size_t row_at(const int* cu, int bh, int H, int N, int base, int r,
+                                         int D) {
+  return cu != nullptr ? ((size_t)(base + r) * H + (size_t)(bh % H)) * D
+                       : ((size_t)bh * N + r) * D;
+}
+// index of row r in the LSE
+__device__ __forceinline__ size_t lse_at(const int* cu, int total, int bh, int H, int N,
+                                         int base, int r) {
+  return cu != nullptr ? (size_t)(bh % H) * total + base + r : (size_t)bh * N + r;
+}
+// whether the kernels write row r: below N, or in a packed batch below the real length L
+// and inside the tensor (a row past L is the next sequence's; offsets outside [0, total]
+// write nothing)
+__device__ __forceinline__ bool row_written(const int* cu, int total, int N, int L, int base,
+                                            int r) {
+  return cu != nullptr ? (r < L && base + r >= 0 && base + r < total) : r < N;
+}
+// the (y, z) coordinates of row r for a TMA copy: (r, bh) in the (D, N, B*H) view of a
+// (B*H, N, D) tensor, (h, cu[b] + r) in the (D, H, total) view of a packed one
+__device__ __forceinline__ int tma_y(const int* cu, int bh, int H, int r) {
+  return cu != nullptr ? bh % H : r;
+}
+__device__ __forceinline__ int tma_z(const int* cu, int bh, int base, int r) {
+  return cu != nullptr ? base + r : bh;
 }
 #endif
 
@@ -168,6 +212,7 @@ __host__ __device__ inline int varlen_sched_ints(int B, int U) { return 2 * (U +
 // (one unit per tile) in one block past its row blocks; `tables` null = none.
 struct SchedBuild {
   const int* seq_len;
+  const int* cu;  // or cumulative lengths (a packed batch)
   int* tables;
   int B;
   int H;
@@ -180,15 +225,18 @@ struct SchedBuild {
 constexpr int kVarlenSchedMaxB = 8192;
 
 #ifdef __CUDACC__
-__device__ __forceinline__ int varlen_units(const int* seq_len, int b, int N, int per_item) {
-  int L = seq_len[b];
+__device__ __forceinline__ int varlen_units(const int* seq_len, const int* cu, int b, int N,
+                                            int per_item) {
+  int L = cu != nullptr ? cu[b + 1] - cu[b] : seq_len[b];
   L = L < 0 ? 0 : (L > N ? N : L);
   return (num_tiles(L) + per_item - 1) / per_item;
 }
 
-// Builds the tables of the schedule above; called by all 32 lanes of one warp.
-__device__ __forceinline__ void build_varlen_sched(const int* seq_len, int B, int H, int N,
-                                                   int per_item, int U, int* tables) {
+// Builds the tables of the schedule above from the lengths seq_len (or the cumulative
+// lengths cu); called by all 32 lanes of one warp.
+__device__ __forceinline__ void build_varlen_sched(const int* seq_len, const int* cu, int B,
+                                                   int H, int N, int per_item, int U,
+                                                   int* tables) {
   int* start = tables;
   int* sigma = tables + U + 1;
   int* cnt = sigma + B;  // cnt[v], v in [0, U]: entries with v units, then a running count
@@ -199,7 +247,7 @@ __device__ __forceinline__ void build_varlen_sched(const int* seq_len, int B, in
   // group of lanes with equal units adds the group's size
   for (int b0 = 0; b0 < B; b0 += 32) {
     const int b = b0 + lane;
-    const int u = b < B ? varlen_units(seq_len, b, N, per_item) : -1;
+    const int u = b < B ? varlen_units(seq_len, cu, b, N, per_item) : -1;
     const unsigned peers = __match_any_sync(0xffffffffu, u);
     if (b < B && (peers & ((1u << lane) - 1u)) == 0) cnt[u] += __popc(peers);
     __syncwarp();
@@ -234,7 +282,7 @@ __device__ __forceinline__ void build_varlen_sched(const int* seq_len, int B, in
   // rank of entry b = (entries with more units) + (earlier entries with as many units)
   for (int b0 = 0; b0 < B; b0 += 32) {
     const int b = b0 + lane;
-    const int u = b < B ? varlen_units(seq_len, b, N, per_item) : -1;
+    const int u = b < B ? varlen_units(seq_len, cu, b, N, per_item) : -1;
     const unsigned peers = __match_any_sync(0xffffffffu, u);
     const int before = __popc(peers & ((1u << lane) - 1u));
     const int seen = b < B ? cnt[u] : 0;

@@ -49,18 +49,20 @@ class fa_options_t(ctypes.Structure):
     _fields_ = [("alibi_slopes", ctypes.c_void_p), ("key_padding", ctypes.c_void_p),
                 ("o_low", ctypes.c_void_p), ("dropout_p", ctypes.c_float),
                 ("flags", ctypes.c_uint), ("dropout_seed", ctypes.c_ulonglong),
-                ("dropout_offset", ctypes.c_ulonglong), ("seq_lengths", ctypes.c_void_p)]
+                ("dropout_offset", ctypes.c_ulonglong), ("seq_lengths", ctypes.c_void_p),
+                ("cu_seqlens", ctypes.c_void_p), ("total_tokens", ctypes.c_int)]
 
 
 def options(alibi_slopes=None, key_padding=None, o_low=None, dropout_p=0.0, dropout_seed=0,
-            dropout_offset=0, fused=False, seq_lengths=None):
+            dropout_offset=0, fused=False, seq_lengths=None, cu_seqlens=None, total_tokens=0):
     """An fa_options_t holding the device pointers of the given tensors (None = absent), the
-    dropout parameters (probability, 64-bit seed, 32-bit offset), the backward's flags and
-    the real lengths of a variable-length batch (B int32 on the device)."""
+    dropout parameters (probability, 64-bit seed, 32-bit offset), the backward's flags, the
+    real lengths of a variable-length batch (B int32 on the device), or the cumulative
+    lengths (B + 1 int32 on the device) and token count of a packed batch."""
     return fa_options_t(_ptr(alibi_slopes), _ptr(key_padding), _ptr(o_low), float(dropout_p),
                         FA_BWD_FUSED if fused else 0,
                         int(dropout_seed) & 0xFFFFFFFFFFFFFFFF, int(dropout_offset),
-                        _ptr(seq_lengths))
+                        _ptr(seq_lengths), _ptr(cu_seqlens), int(total_tokens))
 
 
 _LIB = None
@@ -133,7 +135,11 @@ def _stream(stream) -> int | None:
     return int(stream)
 
 
-def _shape(q: torch.Tensor):
+def _shape(q: torch.Tensor, dims=None):
+    """(B, H, N, d) of a (batch, heads, seq_len, head_dim) tensor, or `dims` as given (a
+    packed batch's (total, heads, head_dim) tensors do not carry B and N)."""
+    if dims is not None:
+        return tuple(int(x) for x in dims)
     if q.dim() != 4:
         raise ValueError("expected a (batch, heads, seq_len, head_dim) tensor")
     return tuple(int(x) for x in q.shape)
@@ -233,9 +239,9 @@ def _opt_ref(opt):
 
 
 def fa_fwd_ex(q, k, v, o, lse, opt=None, scale=None, causal=False, window=(-1, -1),
-              stream=None) -> None:
-    """fa_fwd with an fa_options_t (see options())."""
-    B, H, N, d = _shape(q)
+              stream=None, dims=None) -> None:
+    """fa_fwd with an fa_options_t (see options()); `dims` = (B, H, N, d) for a packed batch."""
+    B, H, N, d = _shape(q, dims)
     c, w = _window(causal, window)
     s = default_scale(d) if scale is None else float(scale)
     _check(_lib().fa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, s, c, w,
@@ -243,9 +249,9 @@ def fa_fwd_ex(q, k, v, o, lse, opt=None, scale=None, causal=False, window=(-1, -
 
 
 def fa_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, workspace, opt=None, scale=None, causal=False,
-              window=(-1, -1), stream=None) -> None:
-    """fa_bwd with an fa_options_t (see options())."""
-    B, H, N, d = _shape(q)
+              window=(-1, -1), stream=None, dims=None) -> None:
+    """fa_bwd with an fa_options_t (see options()); `dims` = (B, H, N, d) for a packed batch."""
+    B, H, N, d = _shape(q, dims)
     c, w = _window(causal, window)
     s = default_scale(d) if scale is None else float(scale)
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -254,15 +260,15 @@ def fa_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, workspace, opt=None, scale=None, 
                             _ptr(workspace), nbytes, _stream(stream)), "fa_bwd_ex")
 
 
-def fa_bwd_preprocess(o, do, lse, workspace, opt=None, stream=None) -> None:
-    B, H, N, d = _shape(o)
+def fa_bwd_preprocess(o, do, lse, workspace, opt=None, stream=None, dims=None) -> None:
+    B, H, N, d = _shape(o, dims)
     _check(_lib().fa_bwd_preprocess(_ptr(o), _ptr(do), _ptr(lse), _ptr(workspace), B, H, N, d,
                                     _opt_ref(opt), _stream(stream)), "fa_bwd_preprocess")
 
 
 def fa_bwd_dkdv(q, k, v, do, workspace, dk, dv, scale=None, causal=False, window=(-1, -1),
-                stream=None, opt=None) -> None:
-    B, H, N, d = _shape(q)
+                stream=None, opt=None, dims=None) -> None:
+    B, H, N, d = _shape(q, dims)
     c, w = _window(causal, window)
     s = default_scale(d) if scale is None else float(scale)
     _check(_lib().fa_bwd_dkdv(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(workspace), _ptr(dk),
@@ -288,8 +294,8 @@ def fa_bwd_dq_convert(workspace, dq, scale=None, stream=None) -> None:
 
 
 def fa_bwd_dq(q, k, v, do, workspace, dq, scale=None, causal=False, window=(-1, -1),
-              stream=None, opt=None) -> None:
-    B, H, N, d = _shape(q)
+              stream=None, opt=None, dims=None) -> None:
+    B, H, N, d = _shape(q, dims)
     c, w = _window(causal, window)
     s = default_scale(d) if scale is None else float(scale)
     _check(_lib().fa_bwd_dq(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(workspace), _ptr(dq),
@@ -346,10 +352,10 @@ def _check_slopes(alibi_slopes, q):
         raise ValueError("alibi_slopes must hold one slope per head, contiguous")
 
 
-def _check_padding(key_padding, q):
+def _check_padding(key_padding, B, N):
     if not key_padding.is_cuda or key_padding.dtype not in (torch.bool, torch.uint8):
         raise ValueError("key_padding must be a bool or uint8 CUDA tensor")
-    if tuple(key_padding.shape) != (q.shape[0], q.shape[2]) or not key_padding.is_contiguous():
+    if tuple(key_padding.shape) != (B, N) or not key_padding.is_contiguous():
         raise ValueError("key_padding must be a contiguous (batch, seq_len) tensor")
 
 
@@ -360,9 +366,24 @@ def _check_lengths(seq_lengths, q):
         raise ValueError("seq_lengths must hold one length per batch entry, contiguous")
 
 
+def _packed_dims(q, cu_seqlens, max_seqlen, seq_lengths):
+    """(B, H, N, d) of a packed batch: q is (total, H, d), cu_seqlens B + 1 int32 offsets."""
+    if seq_lengths is not None:
+        raise ValueError("seq_lengths and cu_seqlens exclude each other")
+    if not cu_seqlens.is_cuda or cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1:
+        raise ValueError("cu_seqlens must be a 1-D int32 CUDA tensor")
+    if cu_seqlens.numel() < 2 or not cu_seqlens.is_contiguous():
+        raise ValueError("cu_seqlens must hold B + 1 >= 2 offsets, contiguous")
+    if q.dim() != 3:
+        raise ValueError("a packed batch takes (total_tokens, heads, head_dim) tensors")
+    if max_seqlen is None or int(max_seqlen) < 1:
+        raise ValueError("a packed batch needs max_seqlen >= 1 (the longest sequence)")
+    return cu_seqlens.numel() - 1, int(q.shape[1]), int(max_seqlen), int(q.shape[2])
+
+
 def attention_forward(q, k, v, scale=None, causal=False, window=(-1, -1), stream=None,
                       alibi_slopes=None, key_padding=None, keep_residual=False, dropout=None,
-                      seq_lengths=None):
+                      seq_lengths=None, cu_seqlens=None, max_seqlen=None):
     """Returns (O, LSE) for bf16 CUDA tensors q, k, v of shape (B, H, N, d), or
     (O, LSE, O_low) with keep_residual: O_low = O_fp32 - bf16(O) in bf16, which
     attention_backward uses to form rowsum(dO o O) from O to about 16 bits.
@@ -372,56 +393,71 @@ def attention_forward(q, k, v, scale=None, causal=False, window=(-1, -1), stream
     probability p (rounded to a multiple of 1/256) after the softmax and scales the kept
     ones by 1 / (1 - p); the backward needs the same triple. seq_lengths ((B,) int32):
     entry b holds seq_lengths[b] real tokens; rows past it are zero (LSE -inf) and tiles
-    wholly past it are not computed."""
+    wholly past it are not computed. cu_seqlens ((B + 1,) int32) with max_seqlen: a packed
+    batch, q, k, v of shape (total, H, d) holding sequence b at tokens cu_seqlens[b] ..
+    cu_seqlens[b+1]-1; O is (total, H, d) and LSE (H, total)."""
     _check_inputs(q, k, v)
-    B, H, N, d = _shape(q)
+    if cu_seqlens is not None:
+        B, H, N, d = _packed_dims(q, cu_seqlens, max_seqlen, seq_lengths)
+        lse = torch.empty((H, q.shape[0]), dtype=torch.float32, device=q.device)
+    else:
+        B, H, N, d = _shape(q)
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     o = torch.empty_like(q)
-    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     o_low = torch.empty_like(q) if keep_residual else None
     if alibi_slopes is not None:
         _check_slopes(alibi_slopes, q)
     if key_padding is not None:
-        _check_padding(key_padding, q)
+        _check_padding(key_padding, B, N)
     if seq_lengths is not None:
         _check_lengths(seq_lengths, q)
     if (alibi_slopes is None and key_padding is None and o_low is None and dropout is None
-            and seq_lengths is None):
+            and seq_lengths is None and cu_seqlens is None):
         fa_fwd(q, k, v, o, lse, scale, causal, window, stream)
     else:
         opt = options(alibi_slopes, key_padding, o_low, *(dropout or ()),
-                      seq_lengths=seq_lengths)
-        fa_fwd_ex(q, k, v, o, lse, opt, scale, causal, window, stream)
+                      seq_lengths=seq_lengths, cu_seqlens=cu_seqlens,
+                      total_tokens=q.shape[0] if cu_seqlens is not None else 0)
+        fa_fwd_ex(q, k, v, o, lse, opt, scale, causal, window, stream, dims=(B, H, N, d))
     return (o, lse, o_low) if keep_residual else (o, lse)
 
 
 def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, window=(-1, -1),
                        stream=None, alibi_slopes=None, key_padding=None, o_low=None,
-                       dropout=None, fused=False, seq_lengths=None):
+                       dropout=None, fused=False, seq_lengths=None, cu_seqlens=None,
+                       max_seqlen=None):
     """Returns (dQ, dK, dV): the gradient of <O, dO>; lse (and o_low, if kept) come from
     attention_forward with the same alibi_slopes, key_padding, dropout and seq_lengths.
     fused: at head_dim 64, the backward in one pass over key tiles with dQ added up in fp32
     in no fixed order (see FA_BWD_FUSED); otherwise the deterministic dK/dV and dQ passes."""
     _check_inputs(q, k, v, o, do)
-    B, H, N, d = _shape(q)
+    if cu_seqlens is not None:
+        B, H, N, d = _packed_dims(q, cu_seqlens, max_seqlen, seq_lengths)
+    else:
+        B, H, N, d = _shape(q)
+    total = q.shape[0] if cu_seqlens is not None else 0
     dq = torch.empty_like(q)
     dk = torch.empty_like(q)
     dv = torch.empty_like(q)
     ws = torch.empty(max(1, fa_bwd_workspace_bytes_ex(
-        B, H, N, d, options(fused=fused, seq_lengths=seq_lengths))),
+        B, H, N, d, options(fused=fused, seq_lengths=seq_lengths, cu_seqlens=cu_seqlens,
+                            total_tokens=total))),
                      dtype=torch.uint8, device=q.device)
     if alibi_slopes is not None:
         _check_slopes(alibi_slopes, q)
     if key_padding is not None:
-        _check_padding(key_padding, q)
+        _check_padding(key_padding, B, N)
     if o_low is not None:
         _check_inputs(q, o_low)
     if seq_lengths is not None:
         _check_lengths(seq_lengths, q)
     if (alibi_slopes is None and key_padding is None and o_low is None and dropout is None
-            and not fused and seq_lengths is None):
+            and not fused and seq_lengths is None and cu_seqlens is None):
         fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, scale, causal, window, stream)
     else:
         opt = options(alibi_slopes, key_padding, o_low, *(dropout or ()),
-                      fused=fused, seq_lengths=seq_lengths)
-        fa_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, ws, opt, scale, causal, window, stream)
+                      fused=fused, seq_lengths=seq_lengths, cu_seqlens=cu_seqlens,
+                      total_tokens=total)
+        fa_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, ws, opt, scale, causal, window, stream,
+                  dims=(B, H, N, d))
     return dq, dk, dv

@@ -118,7 +118,27 @@ typedef struct {
  *                 gradients, and no tile that lies wholly past L_b is computed, so a batch
  *                 costs what its real lengths cost. Values are clamped to [0, N]. The
  *                 backward must get the same lengths.
- * The layout is that of a C struct with natural alignment (56 bytes on LP64).
+ *   cu_seqlens, total_tokens
+ *                 a packed batch, or NULL / 0: the B sequences stored back to back with no
+ *                 padding (the page's dynamic batching groups sequences to avoid padding
+ *                 waste, page "告别OOM和训练慢…" §6). cu_seqlens holds B + 1 int32 cumulative
+ *                 lengths in device memory, 4-byte aligned: sequence b is tokens
+ *                 cu_seqlens[b] .. cu_seqlens[b+1]-1 of q, k, v, o, dout, dq, dk, dv (and
+ *                 o_low), which are then (total_tokens, H, d) bf16 instead of (B, H, N, d);
+ *                 lse is (H, total_tokens) fp32. N is the longest length the call handles:
+ *                 a sequence is cut at N (its tokens past N are not written) and empty or
+ *                 decreasing entries count as length 0. The offsets must lie in
+ *                 [0, total_tokens]; the kernels write no token at or past total_tokens.
+ *                 Masks, scale, ALiBi, key padding ((B, N) flags by position in the
+ *                 sequence) and dropout apply per sequence as in the padded layout; the
+ *                 results of each sequence are bit-identical to those of the same sequence
+ *                 in a (B, H, N, d) batch with seq_lengths (and finite padding). Exclusive
+ *                 with seq_lengths
+ *                 (FA_ERR_INVALID_ARG); not with FA_BWD_FUSED (FA_ERR_UNSUPPORTED); the
+ *                 backward must get the same two values, and its workspace
+ *                 (fa_bwd_workspace_bytes_ex) then holds the schedule tables as with
+ *                 seq_lengths. total_tokens < 0 gives FA_ERR_INVALID_ARG; 0 is an empty call.
+ * The layout is that of a C struct with natural alignment (72 bytes on LP64).
  */
 typedef struct {
     const float *alibi_slopes;
@@ -129,6 +149,8 @@ typedef struct {
     unsigned long long dropout_seed;
     unsigned long long dropout_offset;
     const int *seq_lengths;
+    const int *cu_seqlens;
+    int total_tokens;
 } fa_options_t;
 
 /*

@@ -166,6 +166,19 @@ def test_options_are_checked(lib):
                                             ctypes.byref(O(flags=flags, seq_lengths=A)))
         assert got == base + sched(B, (N + 127) // 128)
     assert bwd_ex(O(seq_lengths=A), ws_bytes=stats) == 4
+    # a packed batch: cumulative lengths 4-byte aligned, exclusive with seq_lengths, a token
+    # count >= 0, not with the fused backward; no tokens is an empty call
+    assert fwd_ex(O(cu_seqlens=A + 2, total_tokens=5)) == 3
+    assert fwd_ex(O(cu_seqlens=A, seq_lengths=A, total_tokens=5)) == 1
+    assert fwd_ex(O(cu_seqlens=A, total_tokens=-1)) == 1
+    assert bwd_ex(O(cu_seqlens=A, total_tokens=5, flags=1)) == 2
+    assert lib.fa_fwd_ex(None, None, None, None, None, 1, 2, 128, 64, 0.125, 0, W(-1, -1),
+                         O(cu_seqlens=A, total_tokens=0), None) == 0
+    assert lib.fa_fwd_ex(A, A, A, A, A, 1, 2, 128, 64, 0.125, 0, W(-1, -1),
+                         O(cu_seqlens=A, total_tokens=1 << 24), None) == 2  # >= 2^31 elements
+    assert lib.fa_bwd_workspace_bytes_ex(3, 2, 1000, 128,
+                                         ctypes.byref(O(cu_seqlens=A, total_tokens=9))) == \
+        lib.fa_bwd_workspace_bytes_ex(3, 2, 1000, 128, None) + sched(3, 8)
     assert lib.fa_bwd_fused(A, A, A, A, A, A, A, 1, 1, 128, 128, 0.1, 0, W(-1, -1), None,
                             None) == 2   # the fused pass is for head_dim 64
     assert lib.fa_bwd_dq_convert(A, None, 1, 1, 128, 64, 0.1, None) == 1
@@ -190,13 +203,31 @@ def test_fp8_forward_rejects_bad_arguments(lib):
                           W(-1, -1), None) == 0
 
 
-def test_options_struct_layout():
+def test_options_struct_layout(tmp_path):
+    """The binding's fa_options_t has the C header's layout (checked against the header
+    compiled by the host C compiler)."""
     import ctypes
+    import shutil
+    import subprocess
     O = fa.fa_options_t
-    assert ctypes.sizeof(O) == 56
-    assert [O.alibi_slopes.offset, O.key_padding.offset, O.o_low.offset, O.dropout_p.offset,
-            O.flags.offset, O.dropout_seed.offset, O.dropout_offset.offset,
-            O.seq_lengths.offset] == [0, 8, 16, 24, 28, 32, 40, 48]
+    names = ["alibi_slopes", "key_padding", "o_low", "dropout_p", "flags", "dropout_seed",
+             "dropout_offset", "seq_lengths", "cu_seqlens", "total_tokens"]
+    py = [ctypes.sizeof(O)] + [getattr(O, n).offset for n in names]
+    assert py == [72, 0, 8, 16, 24, 28, 32, 40, 48, 56, 64]
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stddef.h>\n#include <stdio.h>\n#include "fa.h"\nint main(void) {\n'
+                   '  printf("%zu", sizeof(fa_options_t));\n' +
+                   "".join('  printf(" %%zu", offsetof(fa_options_t, %s));\n' % n for n in names) +
+                   "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", build.INCLUDE, str(src), "-o", str(exe)],
+                   check=True)
+    c = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True,
+                                        check=True).stdout.split()]
+    assert c == py
 
 
 def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -131,3 +131,85 @@ def test_varlen_schedules_agree(d):
         G.assert_within_bounds(errs, (b, lens[b]))
     check_past_length(big, lens)
 
+
+def _pack(t, lens):
+    """(B, H, N, d) -> (total, H, d): the first lens[b] rows of entry b, back to back."""
+    return torch.cat([t[b, :, :L].transpose(0, 1) for b, L in enumerate(lens)], 0).contiguous()
+
+
+def _cu(lens):
+    return [0] + list(np.cumsum(lens).astype(int))
+
+
+def _run_packed(inp, lens, scale, causal, window, d, **kw):
+    """The same problem as a packed batch (fa_options_t.cu_seqlens) through the public calls;
+    returns the outputs in the padded layout's shape for the rows < length (the rest 0 and
+    LSE -inf, as the padded path writes them)."""
+    G.ensure_built()
+    from exact_attention_126_b200 import fa
+    dev = torch.device("cuda:0")
+    B, H, N, _ = inp["q"].shape
+    q, k, v, do = (_pack(inp[n], lens).to(dev) for n in ("q", "k", "v", "do"))
+    cu = torch.tensor(_cu(lens), dtype=torch.int32, device=dev)
+    o, lse, o_low = fa.attention_forward(q, k, v, scale, causal, window, keep_residual=True,
+                                         cu_seqlens=cu, max_seqlen=N, **kw)
+    dq, dk, dv = fa.attention_backward(q, k, v, o, lse, do, scale, causal, window, o_low=o_low,
+                                       cu_seqlens=cu, max_seqlen=N, **kw)
+    torch.cuda.synchronize()
+    assert fa.fa_debug_status() == 0
+    out = {}
+    c = _cu(lens)
+    for n, t in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv)):
+        full = torch.zeros((B, H, N, d), dtype=torch.bfloat16)
+        t = t.cpu()
+        for b, L in enumerate(lens):
+            full[b, :, :L] = t[c[b]:c[b] + L].transpose(0, 1)
+        out[n] = full
+    full = torch.full((B, H, N), float("-inf"), dtype=torch.float32)
+    lse = lse.cpu()
+    for b, L in enumerate(lens):
+        full[b, :, :L] = lse[:, c[b]:c[b] + L]
+    out["lse"] = full
+    return out
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("mode", list(MODES))
+def test_packed_batch_matches_padded(d, mode):
+    """cu_seqlens: the sequences stored back to back with no padding (the page's dynamic
+    batching avoids padding waste). Every real row of every output is bit-identical to the
+    padded layout with seq_lengths (the same arithmetic per tile; a tile that runs into the
+    next sequence only sees masked keys and unwritten rows there), and matches the oracle."""
+    causal, window = MODES[mode]
+    B, H, N = 7, 2, 300
+    lens = _lengths(B, N, 31 + d)
+    lens[5] = 200
+    inp = synth.attention_inputs(B, H, N, d, 2600 + d)
+    scale = 1.0 / np.sqrt(d)
+    padded = G.run_library(inp, scale, causal, window, lengths=lens)
+    packed = _run_packed(inp, lens, scale, causal, window, d)
+    for n in padded:
+        assert torch.equal(packed[n], padded[n]), (n, mode, d)
+    errs = G.compare(inp, packed, scale, causal, window, lengths=lens)
+    G.assert_within_bounds(errs, (d, mode, lens))
+
+
+def test_packed_batch_with_alibi_padding_dropout():
+    """The options that act per sequence (ALiBi, key padding by position, dropout by
+    (batch, head, position)) give the packed batch the padded batch's results."""
+    B, H, N, d = 5, 3, 260, 64
+    lens = [260, 0, 129, 1, 200]
+    inp = synth.attention_inputs(B, H, N, d, 2700)
+    scale = 1.0 / np.sqrt(d)
+    dev = torch.device("cuda:0")
+    rng = np.random.default_rng(2700)
+    kpad = torch.tensor(rng.random((B, N)) < 0.2)
+    slopes = alibi_slopes(H)
+    kw = dict(alibi_slopes=torch.tensor(slopes, dtype=torch.float32, device=dev),
+              key_padding=kpad.to(dev), dropout=(0.1, 1234, 5))
+    padded = G.run_library(inp, scale, True, (-1, -1), lengths=lens, alibi=slopes,
+                           key_padding=kpad, dropout=(0.1, 1234, 5))
+    packed = _run_packed(inp, lens, scale, True, (-1, -1), d, **kw)
+    for n in padded:
+        assert torch.equal(packed[n], padded[n]), n
+
