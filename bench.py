@@ -215,6 +215,15 @@ def kernel_names(w, fused=False):
     return ["fwd", "bwd_preprocess", "bwd_dkdv", "bwd_dq"]
 
 
+def pack_rows(host, lengths, pin=False):
+    """A (B, H, N, d) batch as a packed one: the first lengths[b] rows of entry b, back to
+    back, (total, H, d)."""
+    import torch
+    out = torch.cat([host[b, :, :L].transpose(0, 1) for b, L in enumerate(lengths)], 0)
+    out = out.contiguous()
+    return out.pin_memory() if pin else out
+
+
 class Problem:
     """Device buffers of one workload and the library calls of one step.
 
@@ -228,7 +237,13 @@ class Problem:
         self.w, self.dev, self.fa = w, dev, fa
         B, H, N, d = w.B, w.H, w.N, w.d
         shape = (B, H, N, d)
+        # a packed batch: the sequences back to back as (total, H, d), with cumulative lengths
+        self.dims, self.cu, total = None, None, 0
+        if w.packed:
+            total = sum(w.seq_lengths())
+            shape, self.dims = (total, H, d), (B, H, N, d)
         if host is not None:
+            # (a packed workload's host inputs are packed already)
             self.q, self.k, self.v, self.do = (host[n].to(dev, non_blocking=True)
                                                for n in ("q", "k", "v", "do"))
         else:
@@ -245,7 +260,8 @@ class Problem:
                                          (self.q, self.k, self.v))
         self.o = torch.empty_like(self.q)
         self.o_low = torch.empty_like(self.q)
-        self.lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        self.lse = torch.empty((H, total) if w.packed else (B, H, N), dtype=torch.float32,
+                               device=dev)
         self.dq, self.dk, self.dv = (torch.empty_like(self.q) for _ in range(3))
         self.slopes = None
         if w.alibi:
@@ -253,10 +269,16 @@ class Problem:
                                        device=dev)
         # plain: the forward keeps no residual and delta is formed from the bf16 O
         self.lengths = None
-        if w.varlen:
+        if w.packed:
+            cum = [0]
+            for L in w.seq_lengths():
+                cum.append(cum[-1] + L)
+            self.cu = torch.tensor(cum, dtype=torch.int32, device=dev)
+        elif w.varlen:
             self.lengths = torch.tensor(w.seq_lengths(), dtype=torch.int32, device=dev)
         self.opt = fa.options(alibi_slopes=self.slopes, o_low=None if plain else self.o_low,
-                              fused=fused, seq_lengths=self.lengths)
+                              fused=fused, seq_lengths=self.lengths, cu_seqlens=self.cu,
+                              total_tokens=total)
         # the workspace holds the row statistics (and with real lengths, the schedule)
         self.ws = torch.empty(max(1, fa.fa_bwd_workspace_bytes_ex(B, H, N, d, self.opt)),
                               dtype=torch.uint8, device=dev)
@@ -278,12 +300,12 @@ class Problem:
                 evs[1].record(stream)
             return
         fa.fa_fwd_ex(self.q, self.k, self.v, self.o, self.lse, self.opt, w.softmax_scale,
-                     w.causal, w.window, sp)
+                     w.causal, w.window, sp, dims=self.dims)
         if evs is not None:
             evs[1].record(stream)
         if not w.backward:
             return
-        fa.fa_bwd_preprocess(self.o, self.do, self.lse, self.ws, self.opt, sp)
+        fa.fa_bwd_preprocess(self.o, self.do, self.lse, self.ws, self.opt, sp, dims=self.dims)
         if evs is not None:
             evs[2].record(stream)
         if self.fused:
@@ -294,11 +316,11 @@ class Problem:
             fa.fa_bwd_dq_convert(self.ws, self.dq, w.softmax_scale, sp)
         else:
             fa.fa_bwd_dkdv(self.q, self.k, self.v, self.do, self.ws, self.dk, self.dv,
-                           w.softmax_scale, w.causal, w.window, sp, self.opt)
+                           w.softmax_scale, w.causal, w.window, sp, self.opt, dims=self.dims)
             if evs is not None:
                 evs[3].record(stream)
             fa.fa_bwd_dq(self.q, self.k, self.v, self.do, self.ws, self.dq, w.softmax_scale,
-                         w.causal, w.window, sp, self.opt)
+                         w.causal, w.window, sp, self.opt, dims=self.dims)
         if evs is not None:
             evs[4].record(stream)
 
@@ -388,7 +410,10 @@ def run_ours(args, w, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    inp_host = synth.attention_inputs(w.B, w.H, w.N, w.d, w.seed_index, with_grad=True, pin=True)
+    inp_host = synth.attention_inputs(w.B, w.H, w.N, w.d, w.seed_index, with_grad=True,
+                                      pin=not w.packed)
+    if w.packed:
+        inp_host = {n: pack_rows(t, w.seq_lengths(), pin=True) for n, t in inp_host.items()}
     prob = Problem(w, dev, host=inp_host, plain=args.plain, fused=args.fused)
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
@@ -449,13 +474,17 @@ def run_ours(args, w, rank, world, local_rank):
             else:
                 res = fa.attention_forward(bufs["q"], bufs["k"], bufs["v"], w.softmax_scale,
                                            w.causal, w.window, sp, alibi_slopes=prob.slopes,
-                                           keep_residual=w.backward, seq_lengths=prob.lengths)
+                                           keep_residual=w.backward, seq_lengths=prob.lengths,
+                                           cu_seqlens=prob.cu,
+                                           max_seqlen=w.N if w.packed else None)
             outs = [("o", res[0]), ("lse", res[1])]
             if w.backward:
                 grads = fa.attention_backward(bufs["q"], bufs["k"], bufs["v"], res[0], res[1],
                                               bufs["do"], w.softmax_scale, w.causal, w.window,
                                               sp, alibi_slopes=prob.slopes, o_low=res[2],
-                                              fused=args.fused, seq_lengths=prob.lengths)
+                                              fused=args.fused, seq_lengths=prob.lengths,
+                                              cu_seqlens=prob.cu,
+                                              max_seqlen=w.N if w.packed else None)
                 outs += list(zip(("dq", "dk", "dv"), grads))
             done = torch.cuda.Event()
             done.record(stream)
@@ -681,12 +710,12 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="c4",
-                    help="c1, c2, c3, c4, c5c, c5w, c4a, c4v or c5f8")
+                    help="c1, c2, c3, c4, c5c, c5w, c4a, c4v, c4p or c5f8")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--also", default="c2,c3,c4,c5c,c5w,c4v,c5f8",
+    ap.add_argument("--also", default="c2,c3,c4,c5c,c5w,c4v,c4p,c5f8",
                     help="other workloads timed at full size in the same run (comma list)")
     ap.add_argument("--fused", action="store_true",
                     help="time the fused backward (dQ by fp32 bulk reductions) at head_dim 64")

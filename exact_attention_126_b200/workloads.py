@@ -31,6 +31,7 @@ class Workload:
     alibi: bool = False         # linear bias -m_h |i - j| with the slopes of alibi_slopes()
     varlen: bool = False        # variable-length batch with the lengths of seq_lengths()
     fp8: bool = False           # e4m3 Q, K, V (forward only)
+    packed: bool = False        # with varlen: the sequences back to back, (total, H, d)
 
     @property
     def softmax_scale(self) -> float:
@@ -99,6 +100,10 @@ WORKLOADS = {
     # the dynamic batching of page "告别OOM和训练慢…" §6); work counted on the real pairs
     "c4v": Workload("c4_causal_varlen_b32h16n2048d64", 32, 16, 2048, 64, True, (-1, -1), True,
                     3, varlen=True),
+    # the same batch packed back to back with no padding (cumulative lengths): the page's
+    # dynamic batching groups sequences to avoid padding waste
+    "c4p": Workload("c4_causal_packed_b32h16n2048d64", 32, 16, 2048, 64, True, (-1, -1), True,
+                    3, varlen=True, packed=True),
     # the long-sequence causal forward on e4m3 inputs (FP8 support, page "告别OOM和训练慢…" §6)
     "c5f8": Workload("c5_causal_fp8_fwd_b2h32n8192d128", 2, 32, 8192, 128, True, (-1, -1), False,
                      4, fp8=True),

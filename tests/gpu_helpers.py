@@ -68,6 +68,46 @@ def run_library(inp: dict, scale: float, causal: bool, window, backward: bool = 
     return {n: t.cpu() for n, t in out.items()}
 
 
+def pack_rows(t, lens):
+    """(B, H, N, d) -> (total, H, d): the first lens[b] rows of entry b, back to back."""
+    return torch.cat([t[b, :, :L].transpose(0, 1) for b, L in enumerate(lens)], 0).contiguous()
+
+
+def cumulative(lens):
+    return [0] + list(np.cumsum(lens).astype(int))
+
+
+def run_library_packed(inp, lens, scale, causal, window, **kw):
+    """The same problem as a packed batch (fa_options_t.cu_seqlens) through the public calls;
+    returns the outputs in the padded layout's shape for the rows < length (the rest 0 and
+    LSE -inf, as the padded path writes them)."""
+    ensure_built()
+    dev = torch.device("cuda:0")
+    B, H, N, d = inp["q"].shape
+    q, k, v, do = (pack_rows(inp[n], lens).to(dev) for n in ("q", "k", "v", "do"))
+    cu = torch.tensor(cumulative(lens), dtype=torch.int32, device=dev)
+    o, lse, o_low = fa.attention_forward(q, k, v, scale, causal, window, keep_residual=True,
+                                         cu_seqlens=cu, max_seqlen=N, **kw)
+    dq, dk, dv = fa.attention_backward(q, k, v, o, lse, do, scale, causal, window, o_low=o_low,
+                                       cu_seqlens=cu, max_seqlen=N, **kw)
+    torch.cuda.synchronize()
+    assert fa.fa_debug_status() == 0
+    out = {}
+    c = cumulative(lens)
+    for n, t in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv)):
+        full = torch.zeros((B, H, N, d), dtype=torch.bfloat16)
+        t = t.cpu()
+        for b, L in enumerate(lens):
+            full[b, :, :L] = t[c[b]:c[b] + L].transpose(0, 1)
+        out[n] = full
+    full = torch.full((B, H, N), float("-inf"), dtype=torch.float32)
+    lse = lse.cpu()
+    for b, L in enumerate(lens):
+        full[b, :, :L] = lse[:, c[b]:c[b] + L]
+    out["lse"] = full
+    return out
+
+
 def compare(inp: dict, out: dict, scale: float, causal: bool, window, heads=None,
             backward: bool = True, alibi=None, key_padding=None, dropout=None,
             lengths=None) -> dict:

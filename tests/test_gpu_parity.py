@@ -94,6 +94,13 @@ def test_workload_full_size(name):
     lengths = w.seq_lengths() if w.varlen else None
     out = G.run_library(inp, w.softmax_scale, w.causal, w.window, w.backward, slopes,
                         lengths=lengths)
+    if w.packed:
+        # the packed batch: bit-identical to the padded one on every real row (checked
+        # against the oracle below)
+        packed = G.run_library_packed(inp, lengths, w.softmax_scale, w.causal, w.window)
+        for n in out:
+            assert torch.equal(packed[n], out[n]), n
+        out = packed
     if lengths is not None and heads is not None:
         # one sampled head at a time, each with its batch entry's real length
         per = [G.compare(inp, out, w.softmax_scale, w.causal, w.window, [bh], w.backward,

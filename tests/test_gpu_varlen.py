@@ -132,47 +132,6 @@ def test_varlen_schedules_agree(d):
     check_past_length(big, lens)
 
 
-def _pack(t, lens):
-    """(B, H, N, d) -> (total, H, d): the first lens[b] rows of entry b, back to back."""
-    return torch.cat([t[b, :, :L].transpose(0, 1) for b, L in enumerate(lens)], 0).contiguous()
-
-
-def _cu(lens):
-    return [0] + list(np.cumsum(lens).astype(int))
-
-
-def _run_packed(inp, lens, scale, causal, window, d, **kw):
-    """The same problem as a packed batch (fa_options_t.cu_seqlens) through the public calls;
-    returns the outputs in the padded layout's shape for the rows < length (the rest 0 and
-    LSE -inf, as the padded path writes them)."""
-    G.ensure_built()
-    from exact_attention_126_b200 import fa
-    dev = torch.device("cuda:0")
-    B, H, N, _ = inp["q"].shape
-    q, k, v, do = (_pack(inp[n], lens).to(dev) for n in ("q", "k", "v", "do"))
-    cu = torch.tensor(_cu(lens), dtype=torch.int32, device=dev)
-    o, lse, o_low = fa.attention_forward(q, k, v, scale, causal, window, keep_residual=True,
-                                         cu_seqlens=cu, max_seqlen=N, **kw)
-    dq, dk, dv = fa.attention_backward(q, k, v, o, lse, do, scale, causal, window, o_low=o_low,
-                                       cu_seqlens=cu, max_seqlen=N, **kw)
-    torch.cuda.synchronize()
-    assert fa.fa_debug_status() == 0
-    out = {}
-    c = _cu(lens)
-    for n, t in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv)):
-        full = torch.zeros((B, H, N, d), dtype=torch.bfloat16)
-        t = t.cpu()
-        for b, L in enumerate(lens):
-            full[b, :, :L] = t[c[b]:c[b] + L].transpose(0, 1)
-        out[n] = full
-    full = torch.full((B, H, N), float("-inf"), dtype=torch.float32)
-    lse = lse.cpu()
-    for b, L in enumerate(lens):
-        full[b, :, :L] = lse[:, c[b]:c[b] + L]
-    out["lse"] = full
-    return out
-
-
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("mode", list(MODES))
 def test_packed_batch_matches_padded(d, mode):
@@ -187,7 +146,7 @@ def test_packed_batch_matches_padded(d, mode):
     inp = synth.attention_inputs(B, H, N, d, 2600 + d)
     scale = 1.0 / np.sqrt(d)
     padded = G.run_library(inp, scale, causal, window, lengths=lens)
-    packed = _run_packed(inp, lens, scale, causal, window, d)
+    packed = G.run_library_packed(inp, lens, scale, causal, window)
     for n in padded:
         assert torch.equal(packed[n], padded[n]), (n, mode, d)
     errs = G.compare(inp, packed, scale, causal, window, lengths=lens)
@@ -209,7 +168,54 @@ def test_packed_batch_with_alibi_padding_dropout():
               key_padding=kpad.to(dev), dropout=(0.1, 1234, 5))
     padded = G.run_library(inp, scale, True, (-1, -1), lengths=lens, alibi=slopes,
                            key_padding=kpad, dropout=(0.1, 1234, 5))
-    packed = _run_packed(inp, lens, scale, True, (-1, -1), d, **kw)
+    packed = G.run_library_packed(inp, lens, scale, True, (-1, -1), **kw)
     for n in padded:
         assert torch.equal(packed[n], padded[n]), n
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_packed_outputs_stay_in_bounds(d):
+    """A packed batch writes only its sequences' tokens: sentinels in guard bands around
+    every output and workspace, and in the tokens past the last sequence (which no
+    sequence covers), survive the forward and the backward."""
+    from exact_attention_126_b200 import fa
+    G.ensure_built()
+    dev = torch.device("cuda:0")
+    B, H, N = 3, 2, 300
+    lens = [300, 5, 129]
+    extra = 40
+    total = sum(lens) + extra
+    g = torch.Generator(device=dev).manual_seed(2800 + d)
+    q, k, v, do = (torch.randn((total, H, d), generator=g, device=dev).to(torch.bfloat16)
+                   for _ in range(4))
+    pad = 4096
+
+    def guarded(count, dtype):
+        buf = torch.full((count + 2 * pad,), 7.0, dtype=dtype, device=dev)
+        return buf, buf[pad:pad + count]
+
+    n = total * H * d
+    ob, o = guarded(n, torch.bfloat16)
+    olb, o_low = guarded(n, torch.bfloat16)
+    lb, lse = guarded(H * total, torch.float32)
+    cu = torch.tensor(G.cumulative(lens), dtype=torch.int32, device=dev)
+    dims = (B, H, N, d)
+    opt = fa.options(o_low=o_low, cu_seqlens=cu, total_tokens=total)
+    fa.fa_fwd_ex(q, k, v, o.view(total, H, d), lse.view(H, total), opt, None, True, (-1, -1),
+                 dims=dims)
+    gb = [guarded(n, torch.bfloat16) for _ in range(3)]
+    wb, ws = guarded(fa.fa_bwd_workspace_bytes_ex(B, H, N, d, opt) // 4, torch.float32)
+    fa.fa_bwd_ex(q, k, v, o.view(total, H, d), do, lse.view(H, total),
+                 *(x[1].view(total, H, d) for x in gb), ws, opt, None, True, (-1, -1),
+                 dims=dims)
+    torch.cuda.synchronize()
+    assert fa.fa_debug_status() == 0
+    for buf, _ in [(ob, o), (olb, o_low), (lb, lse), (wb, ws)] + gb:
+        assert torch.all(buf[:pad] == 7.0) and torch.all(buf[-pad:] == 7.0)
+    covered = sum(lens)
+    for t in [o, o_low] + [x[1] for x in gb]:
+        rows = t.view(total, H, d)
+        assert torch.all(rows[covered:] == 7.0)          # nobody's tokens: untouched
+        assert torch.isfinite(rows[:covered].float()).all()
+    assert torch.all(lse.view(H, total)[:, covered:] == 7.0)
 
