@@ -296,16 +296,16 @@ fa_status_t fa_bwd_preprocess(const void *o, const void *dout, const float *lse,
                               const fa_options_t *options, void *stream);
 
 /* Step 2 of fa_bwd alone: dk, dv from q, k, v, dout and the workspace of step 1
- * (`options`: alibi_slopes, key_padding, dropout and seq_lengths as given to step 1, or
- * NULL). */
+ * (`options`: alibi_slopes, key_padding, dropout, and seq_lengths or cu_seqlens with
+ * total_tokens, as given to step 1; or NULL). */
 fa_status_t fa_bwd_dkdv(const void *q, const void *k, const void *v, const void *dout,
                         const void *workspace, void *dk, void *dv,
                         int B, int H, int N, int d, float scale, int causal,
                         fa_window_t window, const fa_options_t *options, void *stream);
 
 /* Step 3 of fa_bwd alone: dq from q, k, v, dout and the workspace of step 1
- * (`options`: alibi_slopes, key_padding, dropout and seq_lengths as given to step 1, or
- * NULL). */
+ * (`options`: alibi_slopes, key_padding, dropout, and seq_lengths or cu_seqlens with
+ * total_tokens, as given to step 1; or NULL). */
 fa_status_t fa_bwd_dq(const void *q, const void *k, const void *v, const void *dout,
                       const void *workspace, void *dq,
                       int B, int H, int N, int d, float scale, int causal,
