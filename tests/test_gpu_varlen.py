@@ -176,15 +176,15 @@ def test_packed_batch_with_alibi_padding_dropout():
 @pytest.mark.parametrize("d", [64, 128])
 def test_packed_outputs_stay_in_bounds(d):
     """A packed batch writes only its sequences' tokens: sentinels in guard bands around
-    every output and workspace, and in the tokens past the last sequence (which no
-    sequence covers), survive the forward and the backward."""
+    every output and workspace, and in the tokens before the first and after the last
+    sequence (which no sequence covers), survive the forward and the backward."""
     from exact_attention_126_b200 import fa
     G.ensure_built()
     dev = torch.device("cuda:0")
     B, H, N = 3, 2, 300
     lens = [300, 5, 129]
-    extra = 40
-    total = sum(lens) + extra
+    lead, extra = 7, 40  # tokens before the first sequence and after the last
+    total = lead + sum(lens) + extra
     g = torch.Generator(device=dev).manual_seed(2800 + d)
     q, k, v, do = (torch.randn((total, H, d), generator=g, device=dev).to(torch.bfloat16)
                    for _ in range(4))
@@ -198,7 +198,7 @@ def test_packed_outputs_stay_in_bounds(d):
     ob, o = guarded(n, torch.bfloat16)
     olb, o_low = guarded(n, torch.bfloat16)
     lb, lse = guarded(H * total, torch.float32)
-    cu = torch.tensor(G.cumulative(lens), dtype=torch.int32, device=dev)
+    cu = torch.tensor([lead + c for c in G.cumulative(lens)], dtype=torch.int32, device=dev)
     dims = (B, H, N, d)
     opt = fa.options(o_low=o_low, cu_seqlens=cu, total_tokens=total)
     fa.fa_fwd_ex(q, k, v, o.view(total, H, d), lse.view(H, total), opt, None, True, (-1, -1),
@@ -212,10 +212,12 @@ def test_packed_outputs_stay_in_bounds(d):
     assert fa.fa_debug_status() == 0
     for buf, _ in [(ob, o), (olb, o_low), (lb, lse), (wb, ws)] + gb:
         assert torch.all(buf[:pad] == 7.0) and torch.all(buf[-pad:] == 7.0)
-    covered = sum(lens)
+    end = lead + sum(lens)
     for t in [o, o_low] + [x[1] for x in gb]:
         rows = t.view(total, H, d)
-        assert torch.all(rows[covered:] == 7.0)          # nobody's tokens: untouched
-        assert torch.isfinite(rows[:covered].float()).all()
-    assert torch.all(lse.view(H, total)[:, covered:] == 7.0)
+        # nobody's tokens, before the first sequence and after the last: untouched
+        assert torch.all(rows[:lead] == 7.0) and torch.all(rows[end:] == 7.0)
+        assert torch.isfinite(rows[lead:end].float()).all()
+    lse_rows = lse.view(H, total)
+    assert torch.all(lse_rows[:, :lead] == 7.0) and torch.all(lse_rows[:, end:] == 7.0)
 
