@@ -221,3 +221,35 @@ def test_packed_outputs_stay_in_bounds(d):
     lse_rows = lse.view(H, total)
     assert torch.all(lse_rows[:, :lead] == 7.0) and torch.all(lse_rows[:, end:] == 7.0)
 
+
+def test_packed_sequence_longer_than_n_is_cut():
+    """A sequence longer than N (the longest length the call handles) is cut at N: its
+    first N tokens get the results of an N-token sequence and the tokens past N are not
+    written (their sentinels survive)."""
+    from exact_attention_126_b200 import fa
+    G.ensure_built()
+    dev = torch.device("cuda:0")
+    H, d, N = 2, 64, 256
+    lens = [300, 129]
+    total = sum(lens)
+    g = torch.Generator(device=dev).manual_seed(2900)
+    q, k, v, do = (torch.randn((total, H, d), generator=g, device=dev).to(torch.bfloat16)
+                   for _ in range(4))
+    cu = torch.tensor(G.cumulative(lens), dtype=torch.int32, device=dev)
+    o = torch.full((total, H, d), 7.0, dtype=torch.bfloat16, device=dev)
+    lse = torch.full((H, total), 7.0, dtype=torch.float32, device=dev)
+    opt = fa.options(cu_seqlens=cu, total_tokens=total)
+    fa.fa_fwd_ex(q, k, v, o, lse, opt, None, True, (-1, -1), dims=(2, H, N, d))
+    # the same first sequence cut to N tokens, as a batch of its own
+    cu1 = torch.tensor([0, N], dtype=torch.int32, device=dev)
+    o1 = torch.empty((N, H, d), dtype=torch.bfloat16, device=dev)
+    lse1 = torch.empty((H, N), dtype=torch.float32, device=dev)
+    fa.fa_fwd_ex(q[:N].contiguous(), k[:N].contiguous(), v[:N].contiguous(), o1, lse1,
+                 fa.options(cu_seqlens=cu1, total_tokens=N), None, True, (-1, -1),
+                 dims=(1, H, N, d))
+    torch.cuda.synchronize()
+    assert fa.fa_debug_status() == 0
+    assert torch.equal(o[:N], o1) and torch.equal(lse[:, :N], lse1)
+    assert torch.all(o[N:300] == 7.0) and torch.all(lse[:, N:300] == 7.0)
+    assert torch.isfinite(o[300:].float()).all()
+
