@@ -389,11 +389,23 @@ def workload_line(w, ms, per_kernel, flushed):
     for n, t in per_kernel.items():
         kernels[n] = {"ms": round(t, 5), "share": round(t / sum(per_kernel.values()), 4),
                       "algorithmic_tflops": round(kf[n] / (t * 1e-3) / 1e12, 2) if kf[n] else None}
-    return {"workload": w.name, "pass": "fwd+bwd" if w.backward else "fwd",
+    line = {"workload": w.name, "pass": "fwd+bwd" if w.backward else "fwd",
             "ms_per_step": round(ms, 5), "tflops": round(value, 2),
             "pct_of_dense_peak": round(100 * value / DATASHEET_BF16_TFLOPS, 2),
             "step_gflop": round(w.step_flops() / 1e9, 3), "kernels": kernels,
             "l2": "L2 flushed before every timed step" if flushed else "inputs larger than L2"}
+    if w.window != (-1, -1) and w.window[0] >= 0 and not w.varlen:
+        # a sliding window's work is its visible pairs; the causal-halved count that a
+        # plain causal problem of this shape would be credited with, for comparison only
+        halved = 4.0 * w.B * w.H * w.N * w.N * w.d / 2 * (3.5 if w.backward else 1.0)
+        line["tflops_if_counted_causal_halved"] = round(halved / (ms * 1e-3) / 1e12, 2)
+        line["causal_halved_overcount"] = round(halved / w.step_flops(), 2)
+    if not w.backward:
+        # forward-only (launch-bound small) workloads: also microseconds and the compulsory
+        # HBM bytes per second
+        line["us_per_step"] = round(ms * 1e3, 2)
+        line["hbm_gbs_compulsory"] = round(w.fwd_bytes() / (ms * 1e-3) / 1e9, 1)
+    return line
 
 
 def run_ours(args, w, rank, world, local_rank):
@@ -528,6 +540,11 @@ def run_ours(args, w, rank, world, local_rank):
             with ClockSampler(local_rank) as oc:
                 oms, oker, _ = op.time(max(20, args.steps), args.warmup, stream)
             line = workload_line(ow, oms, oker, op.flushed)
+            # the same rate against the measured (else fallback) burst bf16 peak
+            pk, pk_src = load_peaks()
+            line["pct_of_measured_peak"] = round(
+                100 * line["tflops"] / float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])), 2)
+            line["peak_source"] = pk_src
             line["clocks"] = oc.summary()
             line["data"] = "synthetic (seeded torch.randn on the device, bf16)"
             others[name] = line
