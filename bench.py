@@ -217,6 +217,29 @@ def kernel_names(w, fused=False):
     return ["fwd", "bwd_preprocess", "bwd_dkdv", "bwd_dq"]
 
 
+def bind_near_gpu(dev_index):
+    """Restricts this process to the CPUs next to the GPU (its PCI device's local_cpulist),
+    so that pinned host buffers allocated meanwhile live on the GPU's NUMA node; returns the
+    previous CPU set to restore, or None when the system does not say (nothing changed)."""
+    import torch
+    try:
+        p = torch.cuda.get_device_properties(dev_index)
+        path = "/sys/bus/pci/devices/%04x:%02x:%02x.0/local_cpulist" % (
+            p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+        cpus = set()
+        for part in open(path).read().strip().split(","):
+            lo, _, hi = part.partition("-")
+            cpus.update(range(int(lo), int(hi or lo) + 1))
+        before = os.sched_getaffinity(0)
+        near = before & cpus
+        if not near or near == before:
+            return None
+        os.sched_setaffinity(0, near)
+        return before
+    except (OSError, ValueError, AttributeError):
+        return None
+
+
 def pack_rows(host, lengths, pin=False):
     """A (B, H, N, d) batch as a packed one: the first lengths[b] rows of entry b, back to
     back, (total, H, d)."""
@@ -424,6 +447,9 @@ def run_ours(args, w, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
+    # the pinned host buffers of the end-to-end run go on the GPU's NUMA node (the process
+    # runs on the CPUs next to the GPU while they are allocated)
+    cpus_before = bind_near_gpu(local_rank)
     inp_host = synth.attention_inputs(w.B, w.H, w.N, w.d, w.seed_index, with_grad=True,
                                       pin=not w.packed)
     if w.packed:
@@ -464,6 +490,8 @@ def run_ours(args, w, rank, world, local_rank):
     # computes. Inputs go through two device buffer sets, each reused once the step that
     # read it has finished; outputs are fresh tensors from the public calls, kept alive for
     # their copy stream.
+    if cpus_before is not None:
+        os.sched_setaffinity(0, cpus_before)
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     dev_in = [{n: torch.empty_like(t) for n, t in zip(("q", "k", "v", "do"), (q, k, v, do))}
               for _ in range(2)]
@@ -615,7 +643,9 @@ def run_ours(args, w, rank, world, local_rank):
         "clocks": clocks.summary(),
         "e2e": {"value": round(job_tflops(flops, world, e2e_ms), 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "steps": e2e_steps,
-                "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes},
+                "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
+                "host_buffers": "pinned, on the GPU's NUMA node" if cpus_before is not None
+                else "pinned (the CPU affinity was left as it was)"},
         "gpu_launches": len(per_kernel) * args.steps,
         "kernels": kernels,
         "roofline": roofline,
